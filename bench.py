@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the SSA hot path (one JSON line on stdout, rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa_16k|mha_8k|long_64k|sweep_32k|tiny_f32] [--topk k]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+block scores -> top-k selection -> fused dual-stream forward -> backward with
+the alignment loss (next-stage dummy loss sum(h_sparse), alpha = 10) ->
+standalone dropped-mass probe.  Work is counted in attended FLOPs over the
+P = B*Hq*N(N+1)/2 causal pairs: forward 4dP, backward 10dP, dropped-mass
+probe 2dP (QK^T only); pooling, top-k and exponentials are not counted.
+
+`value` is whole-job attended TFLOP/s (N GPUs each run the full workload:
+weak scaling, no collective on the data path).  Inputs are resident in HBM
+when the timed region starts and are larger than L2 (Q alone is 268 MB at the
+default workload), so no explicit L2 flush is needed.  `e2e` repeats the
+step through the same C ABI with Q, K, V in pinned host memory: the
+host-to-device copies and the read-back of the alignment loss are inside its
+timed region.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PAGES_DROPPED_MASS = 0.47  # share of attention mass dropped by sparse attention in full-attention models
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gqa_16k")
+    ap.add_argument("--topk", type=int, default=None, help="override the workload's budget")
+    ap.add_argument("--alpha", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload(args):
+    from block_sparse_attention_ssa_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.topk is not None:
+        w = w.with_topk(args.topk)
+    return w
+
+
+def flops(w):
+    P = w.causal_pairs()
+    return {"fwd": 4 * w.d * P, "bwd": 10 * w.d * P, "dropped": 2 * w.d * P}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid: str | None):
+        self.uuid = device_uuid
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def oracle_sample(w, host, budget_s: float, alpha: float):
+    """Time the fp64 oracle (forward, backward, dropped mass) on sampled
+    (batch, head, query block) units of the workload until `budget_s` of CPU
+    time is used.  Returns (attended FLOPs done, seconds, description)."""
+    import numpy as np
+    from oracle import ssa_oracle as O
+
+    s, n, d = w.block, w.n_blocks, w.d
+    scale = w.scale
+    M = w.B * w.Hq * w.N * d
+    rng = np.random.Generator(np.random.PCG64(12345))
+    # selection for the sampled heads is part of the work: it needs every block
+    units, done, secs = [], 0, 0.0
+    t_start = time.perf_counter()
+    while secs < budget_s:
+        b = int(rng.integers(w.B))
+        h = int(rng.integers(w.Hq))
+        i = int(rng.integers(n))
+        kv = h // w.group
+        N1 = (i + 1) * s
+        t0 = time.perf_counter()
+        Q = host["Q"][b:b + 1, h:h + 1, :N1].astype(np.float64)
+        K = host["K"][b:b + 1, kv:kv + 1, :N1].astype(np.float64)
+        V = host["V"][b:b + 1, kv:kv + 1, :N1].astype(np.float64)
+        idx = O.select_blocks(O.block_scores(Q, K, s, scale), w.topk)
+        g = np.ones((1, 1, N1, d))
+        O.ssa_backward(Q, K, V, idx, s, scale, None, g, alpha, qblocks=[i], M=M)
+        O.dropped_mass(Q[:, :, : N1], K, idx, s, scale)
+        secs += time.perf_counter() - t0
+        pairs = sum(t + 1 for t in range(i * s, (i + 1) * s))
+        done += (4 + 10 + 2) * d * pairs
+        units.append((b, h, i))
+        if time.perf_counter() - t_start > 4 * budget_s:
+            break
+    desc = (f"{len(units)} random (batch, head, query block) units of {w.name}: block scores + top-k "
+            f"over the unit's prefix, dual forward, backward (alpha={alpha}, sum(h_sparse)) and "
+            f"dropped mass, fp64 numpy")
+    return done, secs, desc
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, rank: int):
+    if rank != 0:
+        return 0
+    from block_sparse_attention_ssa_b200.inputs import make_workload_inputs
+    w = workload(args)
+    host = make_workload_inputs(w)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, host, per_step / 4, args.alpha)
+    tot_f, tot_s, desc = 0, 0.0, ""
+    for _ in range(args.steps):
+        f, s_, desc = oracle_sample(w, host, per_step, args.alpha)
+        tot_f += f
+        tot_s += s_
+    value = tot_f / tot_s / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": "attended TFLOP/s (fwd+bwd+dropped-mass step)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded planted-direction Q/K/V)",
+        "config": config_dict(w, args),
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, args):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "block": w.block,
+            "topk": w.topk, "dtype": w.dtype, "alpha": args.alpha, "primary": "sparse",
+            "step": "block_scores+select_topk+fwd_dual+bwd_dual+dropped_mass",
+            "l2": "no flush: inputs larger than L2 (Q alone exceeds 126 MB)" if w.N * w.Hq * w.B * w.d * 2 > 126e6
+            else "inputs smaller than L2", "parallelism": f"dp{args.gpus} (independent replicas of the workload)"}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank: int, world: int, dist_on: bool):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_attention_ssa_b200 import api
+    from block_sparse_attention_ssa_b200.inputs import make_workload_inputs
+
+    api.load_library()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    w = workload(args)
+    host = make_workload_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def to_pinned(name):
+        if w.dtype == "bf16":
+            t = torch.from_numpy(host[name + "_bits"].view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(host[name])
+        return t.pin_memory()
+
+    pinned = {k: to_pinned(k) for k in ("Q", "K", "V")}
+    D = {k: v.to(dev, non_blocking=False) for k, v in pinned.items()}
+    dims = api.make_dims(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, w.topk, w.dtype)
+    ws = api.alloc_workspace(dims, dev)
+    out = api.alloc_forward(dims, dev)
+    grads = api.alloc_backward(dims, dev)
+    g_sparse = torch.ones((w.B, w.Hq, w.N, w.d), dtype=tdt, device=dev)
+    delta2 = torch.empty_like(out["delta"])
+    loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    rows = ["block_scores", "select_topk", "fwd_dual", "bwd_dual", "dropped_mass"]
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        api.ssa_block_scores(dims, D["Q"], D["K"], out["scores"], ws, stream)
+        if evs is not None:
+            evs[1].record(stream)
+        api.ssa_select_topk(dims, out["scores"], out["idx"], stream)
+        if evs is not None:
+            evs[2].record(stream)
+        api.ssa_fwd_dual(dims, D["Q"], D["K"], D["V"], out["idx"], out["h_full"], out["h_sparse"],
+                         out["lse_full"], out["lse_sel"], out["delta"], stream)
+        if evs is not None:
+            evs[3].record(stream)
+        api.ssa_bwd_dual(dims, D["Q"], D["K"], D["V"], out["idx"], out["h_full"], out["h_sparse"],
+                         out["lse_full"], out["lse_sel"], None, g_sparse, args.alpha, grads["align_loss"],
+                         grads["dQ"], grads["dK"], grads["dV"], ws, stream)
+        if evs is not None:
+            evs[4].record(stream)
+        api.ssa_dropped_mass(dims, D["Q"], D["K"], out["idx"], out["lse_full"], delta2, ws, stream)
+        if evs is not None:
+            evs[5].record(stream)
+
+    def barrier():
+        if dist_on:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if not dist_on:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = api.ssa_device_status(clear=True, stream=stream)
+    if status != api.SSA_OK:
+        raise RuntimeError(f"device status after warm-up: {api.status_string(status)}")
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = None if args.no_clocks else ClockSampler(uuid)
+    step_events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    n_launch0 = api.ssa_launch_count()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(step_events[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    n_launch = api.ssa_launch_count() - n_launch0
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = t_start.elapsed_time(t_end) / args.steps
+    ms_max = max_over_ranks(ms)
+    row_ms = {r: statistics.mean(step_events[k][i].elapsed_time(step_events[k][i + 1]) for k in range(args.steps))
+              for i, r in enumerate(rows)}
+    status = api.ssa_device_status(clear=True, stream=stream)
+    if status != api.SSA_OK:
+        raise RuntimeError(f"device status after timing: {api.status_string(status)}")
+
+    F = flops(w)
+    step_flops = F["fwd"] + F["bwd"] + F["dropped"]
+    value = world * step_flops / (ms_max * 1e-3) / 1e12
+
+    # ---------------- e2e: host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+
+        def e2e_step():
+            for k_ in ("Q", "K", "V"):
+                D[k_].copy_(pinned[k_], non_blocking=True)
+            step()
+            loss_host.copy_(grads["align_loss"], non_blocking=True)
+            stream.synchronize()
+            return float(loss_host.item())
+
+        e2e_step()
+        barrier()
+        torch.cuda.synchronize()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b_) / args.steps)
+        e2e = {"value": world * step_flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4, "ms_per_step": e_ms}
+
+    # ---------------- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    row_flops = {"fwd_dual": F["fwd"], "bwd_dual": F["bwd"], "dropped_mass": F["dropped"]}
+    dom = max(row_flops, key=lambda r: row_ms[r])
+    achieved = row_flops[dom] / (row_ms[dom] * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"}
+    per_row = {r: {"ms": row_ms[r]} for r in rows}
+    for r, f in row_flops.items():
+        per_row[r]["attended_tflops"] = f / (row_ms[r] * 1e-3) / 1e12
+        per_row[r]["frac_of_sustained_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops_sustained"]
+        per_row[r]["frac_of_burst_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops"]
+    fwd_ms = row_ms["block_scores"] + row_ms["select_topk"] + row_ms["fwd_dual"]
+    extra = {
+        "fwd_tflops": F["fwd"] / (fwd_ms * 1e-3) / 1e12,
+        "fwd_bwd_tflops": (F["fwd"] + F["bwd"]) / ((fwd_ms + row_ms["bwd_dual"]) * 1e-3) / 1e12,
+        "rows": per_row,
+        "mean_delta": float(out["delta"].mean().item()),
+        "pages_dropped_mass_context": PAGES_DROPPED_MASS,
+        "align_loss": float(grads["align_loss"].item()),
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, secs, desc = oracle_sample(w, host, args.cpu_seconds, args.alpha)
+        cpu = {"value": f / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc, "seconds": secs}
+
+    if rank == 0:
+        line = {
+            "metric": "attended TFLOP/s (fwd+bwd+dropped-mass step)", "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded planted-direction Q/K/V)", "config": config_dict(w, args),
+            "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+            "gpu_launches": int(n_launch), **extra,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        return run_ours(args, rank, world, dist_on)
+    finally:
+        if dist_on:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

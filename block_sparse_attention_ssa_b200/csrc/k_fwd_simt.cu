@@ -1,0 +1,267 @@
+// CUDA-core dual-stream forward and dropped-mass kernels (fp32 arithmetic).
+//
+// This is the path for fp32 inputs (tensor cores have no fp32-input kind
+// accurate enough for a 1e-4 tolerance) and for shapes outside the tensor-core
+// kernel's envelope.
+//
+// What it computes ("SSA: Achieving Sparser Attention ...", "Practical
+// Implementation of SSA"; "Technische Samenvatting: SSA", sections
+// "1. Probleemstelling" and "Bidirectionele Uitlijning"): for each query t,
+// two softmaxes over disjoint key sets, A_t (keys in selected blocks) and D_t
+// (the other causal keys), are kept online side by side, each with its own
+// running max, sum and output accumulator.  A key tile lies in one key block,
+// and a 64-row query tile in one query block, so every tile belongs wholly to
+// A or to D for the whole CTA.  At the end:
+//   h_sparse = o_A / l_A,
+//   h_full   = (e^{m_A-M} o_A + e^{m_D-M} o_D) / (e^{m_A-M} l_A + e^{m_D-M} l_D),
+//   delta    = e^{lse_D - lse_full},  lse_full = logaddexp(lse_A, lse_D).
+#include "ssa_internal.cuh"
+
+namespace ssa {
+namespace {
+
+constexpr int BM = 64;   // query rows per CTA
+constexpr int BN = 64;   // keys per tile
+constexpr int NT = 256;  // threads
+
+struct SimtShape {
+  int Hq, g, N, s, n, k;
+  float scale;
+};
+
+template <int D>
+struct FwdSmem {
+  float q[BM][D];
+  float kt[D][BN];      // K tile, transposed
+  float v[BN][D];
+  float p[BM][BN + 1];  // logits, then probabilities
+  float m[2][BM], l[2][BM], corr[BM];
+  uint32_t sel[64];     // selected-block bit set of this query block
+};
+
+// o = corr * o + P V for the 4 x CW patch this thread owns.
+template <int D, int CW>
+__device__ __forceinline__ void pv_update(float (&o)[4][CW], const float (&cr)[4],
+                                          const float (*p)[BN + 1], const float (*v)[D], int pr,
+                                          int pc) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < CW; ++c) o[r][c] *= cr[r];
+#pragma unroll 4
+  for (int kk = 0; kk < BN; ++kk) {
+    float pv[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) pv[r] = p[pr * 4 + r][kk];
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+      const float vv = v[kk][pc * CW + c];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) o[r][c] = fmaf(pv[r], vv, o[r][c]);
+    }
+  }
+}
+
+template <typename T, int D, bool WITH_V>
+__global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  FwdSmem<D>& S = *reinterpret_cast<FwdSmem<D>*>(smem_raw);
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / sh.g;
+  const int t0 = qt * BM;
+  const int iblk = t0 / sh.s;
+  const int tid = threadIdx.x;
+
+  // Selected-block bits of query block iblk.
+  const int words = (sh.n + 31) / 32;
+  for (int w = tid; w < words; w += NT) S.sel[w] = 0u;
+  __syncthreads();
+  const int32_t* irow = a.idx + (((int64_t)b * sh.Hq + h) * sh.n + iblk) * sh.k;
+  for (int e = tid; e < sh.k; e += NT) {
+    const int j = irow[e];
+    if (j >= 0 && j <= iblk) atomicOr(&S.sel[j >> 5], 1u << (j & 31));
+  }
+  // Q tile -> fp32 smem.
+  constexpr int VEC = Vec16<T>::kN;
+  for (int e = tid; e < BM * D / VEC; e += NT) {
+    const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
+    Vec16<T>::load(row_ptr<T>(a.q, b, h, t0 + r) + c, &S.q[r][c]);
+  }
+  if (tid < BM) {
+    S.m[0][tid] = S.m[1][tid] = kNegInf;
+    S.l[0][tid] = S.l[1][tid] = 0.f;
+  }
+
+  // PV ownership: rows pr*4..+3, columns pc*CW..+CW-1.
+  constexpr int CW = D / 16;
+  const int pr = tid / 16, pc = tid % 16;
+  float oA[4][CW], oD[4][CW];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < CW; ++c) oA[r][c] = oD[r][c] = 0.f;
+
+  // Score ownership: rows ty*4..+3, keys tx*4..+3.
+  const int ty = tid / 16, tx = tid % 16;
+  // Softmax ownership: row sr, 16 keys starting at sq*16.
+  const int sr = tid / 4, sq = tid % 4;
+
+  for (int kt = 0; kt <= qt; ++kt) {
+    const int u0 = kt * BN;
+    const int jblk = u0 / sh.s;
+    __syncthreads();  // previous tile fully consumed; sel bits visible
+    const bool sel = (S.sel[jblk >> 5] >> (jblk & 31)) & 1u;
+    for (int e = tid; e < BN * D / VEC; e += NT) {
+      const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
+      float tmp[VEC];
+      Vec16<T>::load(row_ptr<T>(a.k, b, kvh, u0 + r) + c, tmp);
+#pragma unroll
+      for (int x = 0; x < VEC; ++x) S.kt[c + x][r] = tmp[x];
+      if (WITH_V) Vec16<T>::load(row_ptr<T>(a.v, b, kvh, u0 + r) + c, &S.v[r][c]);
+    }
+    __syncthreads();
+
+    // x = scale * Q K^T for a 4x4 patch.
+    float acc[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < D; ++c) {
+      const float4 kv = *reinterpret_cast<const float4*>(&S.kt[c][tx * 4]);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float qv = S.q[ty * 4 + r][c];
+        acc[r][0] = fmaf(qv, kv.x, acc[r][0]);
+        acc[r][1] = fmaf(qv, kv.y, acc[r][1]);
+        acc[r][2] = fmaf(qv, kv.z, acc[r][2]);
+        acc[r][3] = fmaf(qv, kv.w, acc[r][3]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int row = ty * 4 + r, col = tx * 4 + c;
+        const bool ok = (u0 + col) <= (t0 + row);
+        S.p[row][col] = ok ? sh.scale * acc[r][c] : kNegInf;
+      }
+    __syncthreads();
+
+    // Online softmax update of the set this tile belongs to.
+    {
+      const int set = sel ? 0 : 1;
+      float mt = kNegInf;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) mt = fmaxf(mt, S.p[sr][sq * 16 + c]);
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+      const float m_old = S.m[set][sr];
+      const float m_new = fmaxf(m_old, mt);
+      float sum = 0.f;
+      if (m_new != kNegInf) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float x = S.p[sr][sq * 16 + c];
+          const float p = (x == kNegInf) ? 0.f : expf(x - m_new);
+          S.p[sr][sq * 16 + c] = p;
+          sum += p;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) S.p[sr][sq * 16 + c] = 0.f;
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      if (sq == 0) {
+        const float corr = (m_old == kNegInf) ? 0.f : expf(m_old - m_new);
+        S.corr[sr] = corr;
+        S.l[set][sr] = S.l[set][sr] * corr + sum;
+        S.m[set][sr] = m_new;
+      }
+    }
+    __syncthreads();
+
+    if (WITH_V) {
+      float cr[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) cr[r] = S.corr[pr * 4 + r];
+      if (sel) pv_update<D, CW>(oA, cr, S.p, S.v, pr, pc);
+      else pv_update<D, CW>(oD, cr, S.p, S.v, pr, pc);
+    }
+  }
+  __syncthreads();
+
+  // Epilogue.
+  if (WITH_V) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int row = pr * 4 + r;
+      const float mA = S.m[0][row], lA = S.l[0][row], mD = S.m[1][row], lD = S.l[1][row];
+      const float M = fmaxf(mA, mD);
+      const float wa = (lA > 0.f) ? expf(mA - M) : 0.f;
+      const float wd = (lD > 0.f) ? expf(mD - M) : 0.f;
+      const float inv_full = 1.0f / (wa * lA + wd * lD);
+      const float inv_sel = (lA > 0.f) ? 1.0f / lA : 0.f;
+      T* hf = row_ptr_w<T>(a.hf, b, h, t0 + row) + pc * CW;
+      T* hs = row_ptr_w<T>(a.hs, b, h, t0 + row) + pc * CW;
+#pragma unroll
+      for (int c = 0; c < CW; ++c) {
+        hs[c] = from_f32<T>(oA[r][c] * inv_sel);
+        hf[c] = from_f32<T>((wa * oA[r][c] + wd * oD[r][c]) * inv_full);
+      }
+    }
+  }
+  if (tid < BM) {
+    const int row = tid;
+    const int64_t o = ((int64_t)b * sh.Hq + h) * sh.N + t0 + row;
+    const float mA = S.m[0][row], lA = S.l[0][row], mD = S.m[1][row], lD = S.l[1][row];
+    const float lse_a = (lA > 0.f) ? mA + logf(lA) : kNegInf;
+    const float lse_d = (lD > 0.f) ? mD + logf(lD) : kNegInf;
+    const float hi = fmaxf(lse_a, lse_d), lo = fminf(lse_a, lse_d);
+    const float lse_f = (lo == kNegInf) ? hi : hi + log1pf(expf(lo - hi));
+    if (WITH_V) {
+      a.lse_full[o] = lse_f;
+      a.lse_sel[o] = lse_a;
+      a.delta[o] = (lD > 0.f) ? expf(lse_d - lse_f) : 0.f;
+    } else if (a.lse_in != nullptr) {
+      a.delta[o] = (lD > 0.f) ? lD * expf(mD - a.lse_in[o]) : 0.f;
+    } else {
+      a.delta[o] = (lD > 0.f) ? expf(lse_d - lse_f) : 0.f;
+    }
+  }
+}
+
+template <typename T, int D, bool WITH_V>
+cudaError_t launch_t(const Dims& Dm, const FwdArgs& a, cudaStream_t st) {
+  auto kern = fwd_simt_kernel<T, D, WITH_V>;
+  const size_t smem = sizeof(FwdSmem<D>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  SimtShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale};
+  dim3 grid(Dm.N / BM, Dm.Hq, Dm.B);
+  kern<<<grid, NT, smem, st>>>(a, sh);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <bool WITH_V>
+cudaError_t dispatch(const Dims& D, const FwdArgs& a, cudaStream_t st) {
+  if (D.dtype == SSA_BF16)
+    return D.d == 128 ? launch_t<__nv_bfloat16, 128, WITH_V>(D, a, st)
+                      : launch_t<__nv_bfloat16, 64, WITH_V>(D, a, st);
+  return D.d == 128 ? launch_t<float, 128, WITH_V>(D, a, st) : launch_t<float, 64, WITH_V>(D, a, st);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_simt(const Dims& D, const FwdArgs& a, cudaStream_t st) {
+  return dispatch<true>(D, a, st);
+}
+
+cudaError_t launch_dropped_simt(const Dims& D, const FwdArgs& a, cudaStream_t st) {
+  return dispatch<false>(D, a, st);
+}
+
+}  // namespace ssa

@@ -1,0 +1,224 @@
+// Block pooling, block scoring and top-k block selection.
+//
+// "SSA: Achieving Sparser Attention by Aligning Full and Sparse Attention
+// Outputs in Feature Space", section "Practical Implementation of SSA": the
+// sequence is cut into blocks, each block is represented by the mean of its
+// keys, the query is scored against every earlier block representation and
+// the top-k blocks are kept.  Selection is per query block (the query side is
+// the mean of the block's queries) and per query head; the diagonal block is
+// always kept and counts toward k.
+//
+// All three kernels are HBM- or latency-bound and run on CUDA cores.
+#include <climits>
+
+#include "ssa_internal.cuh"
+
+namespace ssa {
+namespace {
+
+// ------------------------------------------------------------------ pooling
+// grid (n, H, B), 128 threads.  Each thread owns 16 bytes of a row; RPI rows
+// are summed in parallel and folded through shared memory.  Reads are 16-byte
+// vectors, a warp covers 2 (bf16, d=128) to 8 rows of 256 / 512 bytes.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) pool_kernel(TensorRef X, int H, int s, int n, float* out) {
+  constexpr int VEC = Vec16<T>::kN;
+  constexpr int TPR = D / VEC;     // threads per row
+  constexpr int RPI = 128 / TPR;   // rows per iteration
+  __shared__ float part[RPI][D];
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int r = threadIdx.x / TPR, c0 = (threadIdx.x % TPR) * VEC;
+  float acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  for (int rr = r; rr < s; rr += RPI) {
+    float v[VEC];
+    Vec16<T>::load(row_ptr<T>(X, b, h, (int64_t)blk * s + rr) + c0, v);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] += v[e];
+  }
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) part[r][c0 + e] = acc[e];
+  __syncthreads();
+  const float inv = 1.0f / (float)s;
+  for (int c = threadIdx.x; c < D; c += 128) {
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < RPI; ++q) sum += part[q][c];
+    out[(((int64_t)b * H + h) * n + blk) * D + c] = sum * inv;
+  }
+}
+
+// ------------------------------------------------------------------ scores
+// grid (ceil(n/32) j-tiles, ceil(n/32) i-tiles, B*Hq), 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qbar,
+                                                    const float* __restrict__ kbar,
+                                                    float* __restrict__ scores, int Hq, int g,
+                                                    int n, float scale) {
+  __shared__ float qs[32][D + 1];
+  __shared__ float ks[32][D + 1];
+  const int j0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
+  const int bh = blockIdx.z, b = bh / Hq, h = bh % Hq, kvh = h / g;
+  const int Hkv = Hq / g;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  float* out = scores + (int64_t)bh * n * n;
+  if (j0 >= i0 + 31) {  // every (i, j) of the tile has j >= i
+    for (int r = ty; r < 32; r += 8) {
+      int i = i0 + r, j = j0 + tx;
+      if (i < n && j < n) out[(int64_t)i * n + j] = kNegInf;
+    }
+    return;
+  }
+  const float* qsrc = qbar + (int64_t)bh * n * D;
+  const float* ksrc = kbar + ((int64_t)b * Hkv + kvh) * n * D;
+  for (int e = threadIdx.x; e < 32 * D; e += 256) {
+    int r = e / D, c = e % D;
+    qs[r][c] = (i0 + r < n) ? qsrc[(int64_t)(i0 + r) * D + c] : 0.f;
+    ks[r][c] = (j0 + r < n) ? ksrc[(int64_t)(j0 + r) * D + c] : 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int r = ty + 8 * q, i = i0 + r, j = j0 + tx;
+    float acc = 0.f;
+#pragma unroll 16
+    for (int c = 0; c < D; ++c) acc = fmaf(qs[r][c], ks[tx][c], acc);
+    if (i < n && j < n) out[(int64_t)i * n + j] = (j < i) ? scale * acc : kNegInf;
+  }
+}
+
+// ------------------------------------------------------------------ top-k
+// One warp per (b, h, i) row.  Candidate j lives in lane j % 32, slot j / 32.
+// k-1 rounds of a warp arg-max with the order (score desc, index asc) pick the
+// blocks; the chosen set is then written in ascending order by a ballot scan.
+__device__ __forceinline__ bool better(float a, int ja, float b, int jb) {
+  return a > b || (a == b && ja < jb);
+}
+
+template <int CPL>
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ scores,
+                                                     int32_t* __restrict__ idx, int64_t rows,
+                                                     int n, int k) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int i = (int)(row % n);
+  const float* srow = scores + row * n;
+  int32_t* orow = idx + row * k;
+  uint64_t taken = 0;
+  if (i + 1 <= k) {
+#pragma unroll
+    for (int m = 0; m < CPL; ++m)
+      if (lane + 32 * m <= i) taken |= 1ull << m;
+  } else {
+    float v[CPL];
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) {
+      const int j = lane + 32 * m;
+      float x = (j < i) ? srow[j] : kNegInf;
+      v[m] = (x != x) ? kNegInf : x;  // NaN ranks as -inf
+    }
+    for (int round = 0; round < k - 1; ++round) {
+      float bv = kNegInf;
+      int bj = INT_MAX;
+#pragma unroll
+      for (int m = 0; m < CPL; ++m) {
+        const int j = lane + 32 * m;
+        if (j < i && !((taken >> m) & 1ull) && better(v[m], j, bv, bj)) {
+          bv = v[m];
+          bj = j;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+        if (better(ov, oj, bv, bj)) {
+          bv = ov;
+          bj = oj;
+        }
+      }
+      if (bj != INT_MAX && (bj & 31) == lane) taken |= 1ull << (bj >> 5);
+    }
+    if ((i & 31) == lane) taken |= 1ull << (i >> 5);
+  }
+  int base = 0;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int m = 0; m < CPL; ++m) {
+    if (32 * m >= n) break;
+    const bool mine = (taken >> m) & 1ull;
+    const unsigned bal = __ballot_sync(0xffffffffu, mine);
+    if (mine) orow[base + __popc(bal & lt)] = lane + 32 * m;
+    base += __popc(bal);
+  }
+  for (int p = base + lane; p < k; p += 32) orow[p] = -1;
+}
+
+// ------------------------------------------------------------------ mask
+// grid = rows, 32 threads: words of the selected-block bit set of one row.
+__global__ void mask_kernel(const int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int n,
+                            int k, int words) {
+  __shared__ uint32_t w[64];
+  const int64_t row = blockIdx.x;
+  const int i = (int)(row % n);
+  for (int q = threadIdx.x; q < words; q += 32) w[q] = 0u;
+  __syncwarp();
+  for (int e = threadIdx.x; e < k; e += 32) {
+    const int j = idx[row * k + e];
+    if (j >= 0 && j <= i) atomicOr(&w[j >> 5], 1u << (j & 31));
+  }
+  __syncwarp();
+  for (int q = threadIdx.x; q < words; q += 32) mask[row * words + q] = w[q];
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Dims& D, const TensorRef& X, int H, float* out, cudaStream_t st) {
+  dim3 grid(D.n, H, D.B);
+  if (D.dtype == SSA_BF16) {
+    if (D.d == 128) pool_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(X, H, D.s, D.n, out);
+    else pool_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(X, H, D.s, D.n, out);
+  } else {
+    if (D.d == 128) pool_kernel<float, 128><<<grid, 128, 0, st>>>(X, H, D.s, D.n, out);
+    else pool_kernel<float, 64><<<grid, 128, 0, st>>>(X, H, D.s, D.n, out);
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scores(const Dims& D, const float* qbar, const float* kbar, float* scores,
+                          cudaStream_t st) {
+  const int t = (D.n + 31) / 32;
+  dim3 grid(t, t, D.B * D.Hq);
+  if (D.d == 128) score_kernel<128><<<grid, 256, 0, st>>>(qbar, kbar, scores, D.Hq, D.g, D.n, D.scale);
+  else score_kernel<64><<<grid, 256, 0, st>>>(qbar, kbar, scores, D.Hq, D.g, D.n, D.scale);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Dims& D, const float* scores, int32_t* idx, cudaStream_t st) {
+  const int64_t rows = (int64_t)D.B * D.Hq * D.n;
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  const int cpl = (D.n + 31) / 32;
+  if (cpl <= 1) select_kernel<1><<<blocks, 256, 0, st>>>(scores, idx, rows, D.n, D.k);
+  else if (cpl <= 2) select_kernel<2><<<blocks, 256, 0, st>>>(scores, idx, rows, D.n, D.k);
+  else if (cpl <= 4) select_kernel<4><<<blocks, 256, 0, st>>>(scores, idx, rows, D.n, D.k);
+  else if (cpl <= 8) select_kernel<8><<<blocks, 256, 0, st>>>(scores, idx, rows, D.n, D.k);
+  else if (cpl <= 16) select_kernel<16><<<blocks, 256, 0, st>>>(scores, idx, rows, D.n, D.k);
+  else if (cpl <= 32) select_kernel<32><<<blocks, 256, 0, st>>>(scores, idx, rows, D.n, D.k);
+  else select_kernel<64><<<blocks, 256, 0, st>>>(scores, idx, rows, D.n, D.k);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_mask(const Dims& D, const int32_t* idx, uint32_t* mask, int words,
+                              cudaStream_t st) {
+  const int64_t rows = (int64_t)D.B * D.Hq * D.n;
+  mask_kernel<<<(unsigned)rows, 32, 0, st>>>(idx, mask, D.n, D.k, words);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace ssa

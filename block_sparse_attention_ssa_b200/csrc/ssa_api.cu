@@ -1,0 +1,336 @@
+// libssa C ABI: argument checks, workspace layout, kernel dispatch.
+// Every check runs on the host before anything is enqueued; see include/ssa.h.
+#include <atomic>
+#include <cstring>
+
+#include "ssa_internal.cuh"
+
+namespace ssa {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+namespace {
+
+// Status word that kernels with bounded waits write when a wait runs out.
+__device__ int32_t g_device_status = 0;
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+ssa_status_t check_dims(const ssa_dims_t* in, Dims* out, bool* empty) {
+  if (in == nullptr) return SSA_ERR_INVALID_ARG;
+  Dims D{};
+  D.B = in->B; D.Hq = in->Hq; D.Hkv = in->Hkv; D.N = in->N; D.d = in->d;
+  D.s = in->block; D.topk = in->topk; D.scale = in->scale; D.dtype = in->dtype;
+  if (D.B < 0 || D.Hq < 0 || D.N < 0 || D.Hkv < 1 || D.topk < 1) return SSA_ERR_INVALID_ARG;
+  if (D.dtype != SSA_F32 && D.dtype != SSA_BF16) return SSA_ERR_INVALID_ARG;
+  if (!(D.scale == D.scale) || D.scale == __builtin_huge_valf() || D.scale == -__builtin_huge_valf())
+    return SSA_ERR_INVALID_ARG;
+  if (D.Hq % D.Hkv != 0) return SSA_ERR_INVALID_ARG;
+  if (D.s != 64 && D.s != 128) return SSA_ERR_UNSUPPORTED;
+  if (D.d != 64 && D.d != 128) return SSA_ERR_UNSUPPORTED;
+  if (D.N % D.s != 0) return SSA_ERR_UNSUPPORTED;
+  D.n = D.N / D.s;
+  if (D.n > 2048) return SSA_ERR_UNSUPPORTED;
+  D.k = D.topk < D.n ? D.topk : D.n;
+  D.g = D.Hkv > 0 ? D.Hq / D.Hkv : 0;
+  *empty = ((int64_t)D.B * D.Hq * D.N == 0);
+  if (*empty) D.k = D.topk;
+  *out = D;
+  return SSA_OK;
+}
+
+size_t elem_size(const Dims& D) { return D.dtype == SSA_BF16 ? 2 : 4; }
+
+ssa_status_t check_tensor(const Dims& D, const ssa_tensor_t* t, bool nullable, TensorRef* out) {
+  if (t == nullptr) {
+    if (!nullable) return SSA_ERR_INVALID_ARG;
+    *out = TensorRef{nullptr, 0, 0, 0};
+    return SSA_OK;
+  }
+  if (t->ptr == nullptr) return SSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(t->ptr) % 16 != 0) return SSA_ERR_INVALID_ARG;
+  const int64_t es = (int64_t)elem_size(D);
+  if (t->stride_b < 0 || t->stride_h < 0 || t->stride_n < 0) return SSA_ERR_INVALID_ARG;
+  if ((t->stride_b * es) % 16 || (t->stride_h * es) % 16 || (t->stride_n * es) % 16)
+    return SSA_ERR_INVALID_ARG;
+  if (t->stride_n < D.d) return SSA_ERR_INVALID_ARG;  // rows may not overlap
+  *out = TensorRef{t->ptr, t->stride_b, t->stride_h, t->stride_n};
+  return SSA_OK;
+}
+
+ssa_status_t check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SSA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  if (major != 10 || minor != 0) return SSA_ERR_UNSUPPORTED;
+  return SSA_OK;
+}
+
+ssa_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA; }
+
+// ---------------------------------------------------------------- workspace
+struct Layout {
+  size_t qbar, kbar;          // block scores
+  size_t dhf, doc, Df, Dc, mask, partials;  // backward
+  size_t lse;                 // dropped mass
+  size_t bytes_scores, bytes_bwd, bytes_dropped, bytes_align;
+  int words, n_partials;
+};
+
+Layout layout(const Dims& D) {
+  Layout L{};
+  const size_t rows = (size_t)D.B * D.Hq * D.N;
+  L.words = (D.n + 31) / 32;
+  L.n_partials = sqdiff_partial_count(D);
+  size_t o = 0;
+  L.qbar = o; o = align_up(o + (size_t)D.B * D.Hq * D.n * D.d * 4);
+  L.kbar = o; o = align_up(o + (size_t)D.B * D.Hkv * D.n * D.d * 4);
+  L.bytes_scores = o;
+  o = 0;
+  L.dhf = o; o = align_up(o + rows * D.d * 4);
+  L.doc = o; o = align_up(o + rows * D.d * 4);
+  L.Df = o; o = align_up(o + rows * 4);
+  L.Dc = o; o = align_up(o + rows * 4);
+  L.mask = o; o = align_up(o + (size_t)D.B * D.Hq * D.n * L.words * 4);
+  L.partials = o; o = align_up(o + (size_t)L.n_partials * 4);
+  L.bytes_bwd = o;
+  L.lse = 0;
+  L.bytes_dropped = align_up(rows * 4);
+  L.bytes_align = align_up((size_t)L.n_partials * 4);
+  return L;
+}
+
+size_t total_bytes(const Layout& L) {
+  size_t m = L.bytes_scores;
+  if (L.bytes_bwd > m) m = L.bytes_bwd;
+  if (L.bytes_dropped > m) m = L.bytes_dropped;
+  if (L.bytes_align > m) m = L.bytes_align;
+  return m;
+}
+
+ssa_status_t check_ws(const Dims& D, const void* ws, size_t ws_bytes) {
+  const size_t need = total_bytes(layout(D));
+  if (ws == nullptr || ws_bytes < need) return SSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign != 0) return SSA_ERR_INVALID_ARG;
+  return SSA_OK;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(ws) + off); }
+
+int32_t* device_status_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+  return static_cast<int32_t*>(p);
+}
+
+}  // namespace
+}  // namespace ssa
+
+using namespace ssa;
+
+extern "C" {
+
+int ssa_version(void) { return 100; }
+
+uint64_t ssa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* ssa_status_string(ssa_status_t s) {
+  switch (s) {
+    case SSA_OK: return "SSA_OK";
+    case SSA_ERR_INVALID_ARG: return "SSA_ERR_INVALID_ARG";
+    case SSA_ERR_UNSUPPORTED: return "SSA_ERR_UNSUPPORTED";
+    case SSA_ERR_CUDA: return "SSA_ERR_CUDA";
+    case SSA_ERR_TIMEOUT: return "SSA_ERR_TIMEOUT";
+    case SSA_ERR_WORKSPACE: return "SSA_ERR_WORKSPACE";
+  }
+  return "SSA_ERR_UNKNOWN";
+}
+
+size_t ssa_workspace_bytes(const ssa_dims_t* dims) {
+  Dims D;
+  bool empty = false;
+  if (check_dims(dims, &D, &empty) != SSA_OK || empty) return 0;
+  return total_bytes(layout(D));
+}
+
+ssa_status_t ssa_block_scores(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
+                              float* scores, void* ws, size_t ws_bytes, ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  TensorRef q, k;
+  if ((s = check_tensor(D, Q, false, &q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &k)) != SSA_OK) return s;
+  if (scores == nullptr || reinterpret_cast<uintptr_t>(scores) % 4) return SSA_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
+  if ((s = check_device()) != SSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(D);
+  float* qbar = at<float>(ws, L.qbar);
+  float* kbar = at<float>(ws, L.kbar);
+  cudaError_t e = launch_pool(D, q, D.Hq, qbar, st);
+  if (e == cudaSuccess) e = launch_pool(D, k, D.Hkv, kbar, st);
+  if (e == cudaSuccess) e = launch_scores(D, qbar, kbar, scores, st);
+  return from_cuda(e);
+}
+
+ssa_status_t ssa_select_topk(const ssa_dims_t* dims, const float* scores, int32_t* idx,
+                             ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  if (scores == nullptr || idx == nullptr) return SSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(scores) % 4 || reinterpret_cast<uintptr_t>(idx) % 4)
+    return SSA_ERR_INVALID_ARG;
+  if ((s = check_device()) != SSA_OK) return s;
+  return from_cuda(launch_select(D, scores, idx, static_cast<cudaStream_t>(stream)));
+}
+
+ssa_status_t ssa_fwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
+                          const ssa_tensor_t* V, const int32_t* idx, const ssa_tensor_t* h_full,
+                          const ssa_tensor_t* h_sparse, float* lse_full, float* lse_sel,
+                          float* delta, ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  FwdArgs a{};
+  if ((s = check_tensor(D, Q, false, &a.q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &a.k)) != SSA_OK) return s;
+  if ((s = check_tensor(D, V, false, &a.v)) != SSA_OK) return s;
+  if ((s = check_tensor(D, h_full, false, &a.hf)) != SSA_OK) return s;
+  if ((s = check_tensor(D, h_sparse, false, &a.hs)) != SSA_OK) return s;
+  if (!idx || !lse_full || !lse_sel || !delta) return SSA_ERR_INVALID_ARG;
+  if ((s = check_device()) != SSA_OK) return s;
+  a.idx = idx;
+  a.lse_full = lse_full;
+  a.lse_sel = lse_sel;
+  a.delta = delta;
+  a.lse_in = nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fwd_tc_supported(D)) {
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_fwd_tc(D, a, status, st));
+  }
+  return from_cuda(launch_fwd_simt(D, a, st));
+}
+
+ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
+                          const ssa_tensor_t* V, const int32_t* idx, const ssa_tensor_t* h_full,
+                          const ssa_tensor_t* h_sparse, const float* lse_full,
+                          const float* lse_sel, const ssa_tensor_t* g_full,
+                          const ssa_tensor_t* g_sparse, float alpha, float* align_loss,
+                          const ssa_tensor_t* dQ, const ssa_tensor_t* dK, const ssa_tensor_t* dV,
+                          void* ws, size_t ws_bytes, ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  BwdArgs a{};
+  if ((s = check_tensor(D, Q, false, &a.q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &a.k)) != SSA_OK) return s;
+  if ((s = check_tensor(D, V, false, &a.v)) != SSA_OK) return s;
+  if ((s = check_tensor(D, h_full, false, &a.hf)) != SSA_OK) return s;
+  if ((s = check_tensor(D, h_sparse, false, &a.hs)) != SSA_OK) return s;
+  if ((s = check_tensor(D, g_full, true, &a.gf)) != SSA_OK) return s;
+  if ((s = check_tensor(D, g_sparse, true, &a.gs)) != SSA_OK) return s;
+  if ((s = check_tensor(D, dQ, false, &a.dq)) != SSA_OK) return s;
+  if ((s = check_tensor(D, dK, false, &a.dk)) != SSA_OK) return s;
+  if ((s = check_tensor(D, dV, false, &a.dv)) != SSA_OK) return s;
+  if (!(alpha == alpha)) return SSA_ERR_INVALID_ARG;
+  if (!idx || !lse_full || !lse_sel) return SSA_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
+  if ((s = check_device()) != SSA_OK) return s;
+  const Layout L = layout(D);
+  a.idx = idx;
+  a.lse_full = lse_full;
+  a.lse_sel = lse_sel;
+  a.alpha = alpha;
+  a.align_loss = align_loss;
+  a.dhf = at<float>(ws, L.dhf);
+  a.doc = at<float>(ws, L.doc);
+  a.Df = at<float>(ws, L.Df);
+  a.Dc = at<float>(ws, L.Dc);
+  a.mask = at<uint32_t>(ws, L.mask);
+  a.words = L.words;
+  a.partials = at<float>(ws, L.partials);
+  a.n_partials = L.n_partials;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_build_mask(D, idx, a.mask, L.words, st);
+  if (e == cudaSuccess) e = launch_bwd_pre(D, a, st);
+  if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
+  return from_cuda(e);
+}
+
+ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
+                              const int32_t* idx, const float* lse_full, float* delta, void* ws,
+                              size_t ws_bytes, ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  FwdArgs a{};
+  if ((s = check_tensor(D, Q, false, &a.q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &a.k)) != SSA_OK) return s;
+  if (!idx || !delta) return SSA_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
+  if ((s = check_device()) != SSA_OK) return s;
+  a.v = a.k;  // unused
+  a.idx = idx;
+  a.delta = delta;
+  a.lse_in = lse_full;
+  return from_cuda(launch_dropped_simt(D, a, static_cast<cudaStream_t>(stream)));
+}
+
+ssa_status_t ssa_align_mse(const ssa_dims_t* dims, const ssa_tensor_t* h_full,
+                           const ssa_tensor_t* h_sparse, float* loss, void* ws, size_t ws_bytes,
+                           ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  TensorRef hf, hs;
+  if ((s = check_tensor(D, h_full, false, &hf)) != SSA_OK) return s;
+  if ((s = check_tensor(D, h_sparse, false, &hs)) != SSA_OK) return s;
+  if (loss == nullptr) return SSA_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
+  if ((s = check_device()) != SSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(D);
+  float* partials = static_cast<float*>(ws);
+  const double M = (double)D.B * D.Hq * D.N * D.d;
+  cudaError_t e = launch_sqdiff_partials(D, hf, hs, partials, L.n_partials, st);
+  if (e == cudaSuccess) e = launch_finish_mean(partials, L.n_partials, M, 1.0f, loss, 2, st);
+  return from_cuda(e);
+}
+
+ssa_status_t ssa_device_status(int32_t* status, int clear, ssa_stream_t stream) {
+  if (status == nullptr) return SSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SSA_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return SSA_ERR_CUDA;
+  *status = v;
+  if (clear) {
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return SSA_ERR_CUDA;
+  }
+  return SSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,138 @@
+// Internal declarations shared by the libssa translation units.
+// Nothing here is part of the C ABI (see include/ssa.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssa.h"
+
+namespace ssa {
+
+// Validated problem shape.
+struct Dims {
+  int B, Hq, Hkv, N, d, s, topk, k, n, g;  // k = min(topk, n), g = Hq / Hkv
+  float scale;
+  int dtype;
+};
+
+// A [B, H, N, d] tensor with a contiguous d dimension; strides in elements.
+struct TensorRef {
+  const void* p;
+  int64_t sb, sh, sn;
+};
+
+template <typename T>
+__device__ __forceinline__ const T* row_ptr(const TensorRef& t, int b, int h, int64_t r) {
+  return static_cast<const T*>(t.p) + b * t.sb + h * t.sh + r * t.sn;
+}
+template <typename T>
+__device__ __forceinline__ T* row_ptr_w(const TensorRef& t, int b, int h, int64_t r) {
+  return const_cast<T*>(static_cast<const T*>(t.p)) + b * t.sb + h * t.sh + r * t.sn;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Loads 16 bytes of T (4 floats or 8 bf16) starting at a 16-byte aligned
+// address and widens them to float.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+  static constexpr int kN = 4;
+  __device__ __forceinline__ static void load(const float* p, float* out) {
+    float4 v = *reinterpret_cast<const float4*>(p);
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+  }
+};
+template <> struct Vec16<__nv_bfloat16> {
+  static constexpr int kN = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out) {
+    uint4 v = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      out[2 * i] = f.x;
+      out[2 * i + 1] = f.y;
+    }
+  }
+};
+
+constexpr float kNegInf = -__builtin_huge_valf();
+
+// Host-side count of kernels enqueued by this library (ssa_launch_count).
+void count_launches(int n);
+
+// ---------------------------------------------------------------- launchers
+// Each returns the launch status; none synchronises.
+
+// Mean of each block of s rows: X [B,H,N,d] -> out [B,H,n,d] fp32 (dense).
+cudaError_t launch_pool(const Dims& D, const TensorRef& X, int H, float* out, cudaStream_t st);
+
+// scores[b,h,i,j] = scale * qbar[b,h,i] . kbar[b,h/g,j] for j < i, else -inf.
+cudaError_t launch_scores(const Dims& D, const float* qbar, const float* kbar, float* scores,
+                          cudaStream_t st);
+
+// Top-k block selection with the forced diagonal.
+cudaError_t launch_select(const Dims& D, const float* scores, int32_t* idx, cudaStream_t st);
+
+// Bit mask [B, Hq, n, words] of Sel(i) built from idx (entries outside [0,i] ignored).
+cudaError_t launch_build_mask(const Dims& D, const int32_t* idx, uint32_t* mask, int words,
+                              cudaStream_t st);
+
+struct FwdArgs {
+  TensorRef q, k, v, hf, hs;
+  const int32_t* idx;
+  float* lse_full;
+  float* lse_sel;
+  float* delta;
+  const float* lse_in;  // dropped-mass mode only: given lse_full, or nullptr
+};
+
+// CUDA-core dual-stream forward (fp32 math; any supported dtype / d).
+cudaError_t launch_fwd_simt(const Dims& D, const FwdArgs& a, cudaStream_t st);
+// CUDA-core dropped mass (no V).
+cudaError_t launch_dropped_simt(const Dims& D, const FwdArgs& a, cudaStream_t st);
+
+// Tensor-core (tcgen05 / TMEM / TMA) dual-stream forward, bf16, d = 128.
+// Returns cudaErrorNotSupported when the shape is outside its envelope.
+cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
+bool fwd_tc_supported(const Dims& D);
+
+struct BwdArgs {
+  TensorRef q, k, v, hf, hs, gf, gs, dq, dk, dv;  // gf / gs .p may be null
+  const int32_t* idx;
+  const float* lse_full;
+  const float* lse_sel;
+  float alpha;
+  float* align_loss;  // may be null
+  // workspace pieces
+  float* dhf;          // [B,Hq,N,d] fp32: dL/dh_full
+  float* doc;          // [B,Hq,N,d] fp32: dh_full + r * dh_sparse
+  float* Df;           // [B,Hq,N]
+  float* Dc;           // [B,Hq,N]
+  uint32_t* mask;      // [B,Hq,n,words]
+  int words;
+  float* partials;     // per-block partial sums of (h_full - h_sparse)^2
+  int n_partials;
+};
+
+cudaError_t launch_bwd_pre(const Dims& D, const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_simt(const Dims& D, const BwdArgs& a, cudaStream_t st);
+
+// Sum of squared differences of two [B,Hq,N,d] tensors into per-block
+// partials, then a fixed-order final reduction: out[0..n_out) = sum / count.
+cudaError_t launch_sqdiff_partials(const Dims& D, const TensorRef& a, const TensorRef& b,
+                                   float* partials, int n_partials, cudaStream_t st);
+cudaError_t launch_finish_mean(const float* partials, int n_partials, double count, float mult,
+                               float* out, int n_out, cudaStream_t st);
+int sqdiff_partial_count(const Dims& D);
+
+}  // namespace ssa

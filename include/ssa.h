@@ -1,0 +1,223 @@
+/*
+ * ssa.h -- C ABI of libssa, the B200 (sm_100a) hot path of SSA, Sparse Sparse
+ * Attention: causal block-sparse attention with per-query-block top-k block
+ * selection, computed in one pass together with the full causal attention,
+ * the dropped attention mass delta(t), and the backward of both streams with
+ * the bidirectional alignment loss folded in.
+ *
+ * Sources (page title, then section):
+ *   [digest]  "SSA: Achieving Sparser Attention by Aligning Full and Sparse
+ *             Attention Outputs in Feature Space" (blog digest of the paper).
+ *   [summary] "Technische Samenvatting: SSA (Sparse Sparse Attention)".
+ *   [record]  "SSA: Sparse Sparse Attention by Aligning Full and Sparse
+ *             Attention Outputs in Feature Space" (arXiv 2511.20102 record).
+ *
+ * Notation: B batch, Hq query heads, Hkv key/value heads (g = Hq/Hkv query
+ * heads share one kv head; query head h reads kv head h/g), N tokens, d head
+ * dim, s = block, n = N/s blocks, k = topk budget in blocks counting the
+ * diagonal block, scale = attention scale (1/sqrt(d) in the paper's models).
+ * Query token t lies in block i = t/s.  Sel(i) is the selected block set of
+ * query block i; A_t = {u <= t : u/s in Sel(i)} is attended by both streams,
+ * D_t = {u <= t : u/s not in Sel(i)} only by the full stream.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.  Every pointer is a DEVICE pointer the caller allocated on the
+ *   current CUDA device; the caller keeps ownership.  libssa never allocates,
+ *   frees or synchronises (except ssa_device_status).  All work is enqueued
+ *   on `stream` (a cudaStream_t; NULL means the legacy default stream) in
+ *   stream order; calls are stateless and may be issued from several host
+ *   threads on different streams.
+ * Tensors.  ssa_tensor_t describes a 4-D tensor [B, H, N, d] of dims->dtype
+ *   elements whose last (d) dimension is contiguous; stride_b / stride_h /
+ *   stride_n are in ELEMENTS.  Q, h_full, h_sparse, dQ, g_full, g_sparse use
+ *   H = Hq; K, V, dK, dV use H = Hkv.  Base pointers must be 16-byte aligned
+ *   and every stride times the element size a multiple of 16 bytes.
+ *   Plain arrays (scores, idx, lse_*, delta) are dense row-major as stated.
+ * Shapes.  B, Hq, N >= 0 and Hkv >= 1 with Hq % Hkv == 0; block in {64, 128};
+ *   N % block == 0; d in {64, 128}; topk >= 1 (a budget above n is clamped:
+ *   k_eff = min(topk, n)); n <= 2048.  When B*Hq*N == 0 the call is a no-op
+ *   and returns SSA_OK.
+ * Errors.  Arguments are checked on the host before anything is enqueued;
+ *   a failed check returns SSA_ERR_INVALID_ARG (bad pointer, stride,
+ *   alignment or value), SSA_ERR_UNSUPPORTED (a shape outside the list above,
+ *   or a device that is not sm_100) or SSA_ERR_WORKSPACE (ws_bytes below
+ *   ssa_workspace_bytes) and enqueues nothing.  A failed launch returns
+ *   SSA_ERR_CUDA.  Kernels that wait on hardware barriers bound every wait;
+ *   a wait that runs out records SSA_ERR_TIMEOUT in a device status word
+ *   (read it with ssa_device_status) and the kernel returns.  No kernel traps.
+ * Precision.  dtype SSA_BF16: inputs/outputs bf16, products on tensor cores
+ *   with fp32 accumulation and fp32 softmax statistics.  SSA_F32: fp32 inputs
+ *   and outputs, fp32 arithmetic throughout (CUDA cores).
+ */
+#ifndef SSA_H_
+#define SSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSA_API __attribute__((visibility("default")))
+#else
+#define SSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSA_OK = 0,
+  SSA_ERR_INVALID_ARG = 1,
+  SSA_ERR_UNSUPPORTED = 2,
+  SSA_ERR_CUDA = 3,
+  SSA_ERR_TIMEOUT = 4,
+  SSA_ERR_WORKSPACE = 5
+} ssa_status_t;
+
+typedef enum { SSA_F32 = 0, SSA_BF16 = 1 } ssa_dtype_t;
+
+typedef struct {
+  int32_t B, Hq, Hkv, N, d, block, topk;
+  float scale;
+  int32_t dtype; /* ssa_dtype_t */
+} ssa_dims_t;
+
+typedef struct {
+  void* ptr;
+  int64_t stride_b, stride_h, stride_n; /* elements; the d stride is 1 */
+} ssa_tensor_t;
+
+typedef void* ssa_stream_t; /* cudaStream_t */
+
+/* ABI version of this header (major * 100 + minor). */
+SSA_API int ssa_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+SSA_API const char* ssa_status_string(ssa_status_t status);
+
+/* Bytes of device workspace that ssa_block_scores, ssa_bwd_dual,
+ * ssa_dropped_mass and ssa_align_mse need for these dims (one size serves
+ * all of them).  Returns 0 for an invalid or empty shape.  The workspace is
+ * caller-owned scratch: its contents on entry are ignored and on return
+ * undefined; two calls in flight at once must not share one workspace. */
+SSA_API size_t ssa_workspace_bytes(const ssa_dims_t* dims);
+
+/* Step 1: block pooling and block scores.
+ * [digest] "Practical Implementation of SSA": split the sequence into blocks,
+ * represent each block by the mean of its keys, and score the query against
+ * every earlier block representation; pooling keeps the ranking because the
+ * mean of q K^T over a block equals q times the mean of the block's keys.
+ * The query side is the mean of the query block (selection is per query
+ * block and per query head).
+ *   scores [B, Hq, n, n] fp32 (out): scores[b,h,i,j] = scale * qbar_i . kbar_j
+ *     for j < i, with qbar / kbar the fp32 means of query block i (head h) and
+ *     key block j (kv head h/g); -INFINITY for j >= i (the diagonal is kept
+ *     unconditionally by ssa_select_topk and is not scored).
+ *   ws: workspace of at least ssa_workspace_bytes(dims) bytes (holds qbar, kbar). */
+SSA_API ssa_status_t ssa_block_scores(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                              const ssa_tensor_t* K, float* scores, void* ws,
+                              size_t ws_bytes, ssa_stream_t stream);
+
+/* Step 2: top-k block selection.
+ * [digest] "Practical Implementation of SSA": keep the top-k most relevant
+ * blocks.  Sel(i) = {i} plus the k_eff-1 largest scores[b,h,i,j], j < i;
+ * equal scores go to the smaller j; if i + 1 <= k_eff, Sel(i) = {0..i}.
+ *   scores [B, Hq, n, n] fp32 (in): only the strictly lower triangle is read.
+ *     NaN scores give an unspecified (but in-range) selection.
+ *   idx [B, Hq, n, k_eff] int32 (out): Sel(i) in ascending order, padded
+ *     with -1 when i + 1 < k_eff.  Deterministic. */
+SSA_API ssa_status_t ssa_select_topk(const ssa_dims_t* dims, const float* scores,
+                             int32_t* idx, ssa_stream_t stream);
+
+/* Step 3: fused dual-stream forward.
+ * One pass over every causal K/V tile keeps two disjoint online softmaxes,
+ * over A_t and over D_t, and merges them at the end:
+ *   h_sparse = softmax over A_t of x_tu applied to V   ([digest] "Practical
+ *     Implementation of SSA"; [summary] "1. Probleemstelling": the sparse
+ *     stream normalises over the selected subset only);
+ *   h_full   = causal softmax over all u <= t applied to V, the counterpart
+ *     output kept for alignment ([summary] "Bidirectionele Uitlijning");
+ *   delta[t] = full-softmax weight on D_t, the dropped attention mass
+ *     ([summary] "1. Probleemstelling"; [record] abstract); 0 when D_t is empty;
+ *   lse_full[t], lse_sel[t] = natural-log normalisers of the two softmaxes.
+ * x_tu = scale * q_t . k_u.
+ *   idx [B, Hq, n, k_eff] int32 (in): as written by ssa_select_topk.  Any
+ *     other selection may be passed: entries outside [0, i] are ignored and
+ *     duplicates are harmless.  A row that omits its diagonal block attends
+ *     only the listed blocks; a query whose A_t is empty gets h_sparse = 0,
+ *     lse_sel = -INFINITY and delta = 1.
+ *   h_full, h_sparse (out): [B, Hq, N, d] strided, dims->dtype.
+ *   lse_full, lse_sel, delta [B, Hq, N] fp32 (out). */
+SSA_API ssa_status_t ssa_fwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                          const ssa_tensor_t* K, const ssa_tensor_t* V,
+                          const int32_t* idx, const ssa_tensor_t* h_full,
+                          const ssa_tensor_t* h_sparse, float* lse_full,
+                          float* lse_sel, float* delta, ssa_stream_t stream);
+
+/* Step 4: backward of both streams with the alignment loss folded in.
+ * Gradients of L = <g_full, h_full> + <g_sparse, h_sparse> + alpha * L_align
+ * with L_align = L_sparsity + L_commitment, L_sparsity = MSE(h_full, sg h_sparse),
+ * L_commitment = MSE(h_sparse, sg h_full), MSE = mean over all B*Hq*N*d
+ * elements ([digest] "Bidirectional Attention Alignment"; [summary]
+ * "Bidirectionele Uitlijning": total objective E_mode[L_ce] + alpha L_align,
+ * alpha = 10 in the paper, [digest] "Alignment Weight").  g_full / g_sparse
+ * carry the next stage's gradient of whichever stream is forwarded (for a
+ * next-stage loss sum(h_primary) pass all-ones on the primary stream and NULL
+ * on the other).  The selection is held fixed: no gradient flows through idx
+ * or delta.  dK and dV are summed over the g query heads of each kv head.
+ *   Q, K, V, idx, h_full, h_sparse, lse_full, lse_sel: as passed to / written
+ *     by ssa_fwd_dual for the same inputs.
+ *   g_full, g_sparse: [B, Hq, N, d] dims->dtype, or NULL for zero.
+ *   align_loss: device fp32 scalar (out) = L_align, or NULL.
+ *   dQ [B,Hq,N,d], dK, dV [B,Hkv,N,d] (out): strided, dims->dtype; fully
+ *     overwritten.
+ *   ws: workspace of at least ssa_workspace_bytes(dims) bytes. */
+SSA_API ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                          const ssa_tensor_t* K, const ssa_tensor_t* V,
+                          const int32_t* idx, const ssa_tensor_t* h_full,
+                          const ssa_tensor_t* h_sparse, const float* lse_full,
+                          const float* lse_sel, const ssa_tensor_t* g_full,
+                          const ssa_tensor_t* g_sparse, float alpha,
+                          float* align_loss, const ssa_tensor_t* dQ,
+                          const ssa_tensor_t* dK, const ssa_tensor_t* dV,
+                          void* ws, size_t ws_bytes, ssa_stream_t stream);
+
+/* Standalone dropped attention mass, without V.
+ * delta[t] = sum over u in D_t of exp(x_tu - lse_full[t]) ([summary]
+ * "1. Probleemstelling"; [digest] "Phenomenon 3" reports this quantity for
+ * full-attention models).  The sum runs over D_t directly (not 1 - sum over
+ * A_t) so small masses keep their relative precision.
+ *   lse_full [B, Hq, N] fp32 (in) or NULL: when NULL the causal log-sum-exp is
+ *     computed in the same pass.
+ *   delta [B, Hq, N] fp32 (out).
+ *   ws: workspace of at least ssa_workspace_bytes(dims) bytes. */
+SSA_API ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                              const ssa_tensor_t* K, const int32_t* idx,
+                              const float* lse_full, float* delta, void* ws,
+                              size_t ws_bytes, ssa_stream_t stream);
+
+/* Forward value of the alignment loss on its own.
+ * loss (out): device fp32[2] = {L_sparsity, L_commitment}, each the mean of
+ * (h_full - h_sparse)^2 over all B*Hq*N*d elements ([digest] "Bidirectional
+ * Attention Alignment").  Deterministic (fixed-order reduction).
+ *   ws: workspace of at least ssa_workspace_bytes(dims) bytes. */
+SSA_API ssa_status_t ssa_align_mse(const ssa_dims_t* dims, const ssa_tensor_t* h_full,
+                           const ssa_tensor_t* h_sparse, float* loss, void* ws,
+                           size_t ws_bytes, ssa_stream_t stream);
+
+/* Number of kernels this library has enqueued in this process so far (all
+ * devices, all threads).  Lets a caller count the launches of a region. */
+SSA_API uint64_t ssa_launch_count(void);
+
+/* Synchronises `stream`, copies the device status word of the current device
+ * to *status (SSA_OK, or the first SSA_ERR_TIMEOUT a kernel recorded) and,
+ * if clear != 0, resets it.  Returns SSA_ERR_CUDA if the synchronisation or
+ * the copy fails. */
+SSA_API ssa_status_t ssa_device_status(int32_t* status, int clear, ssa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H_ */

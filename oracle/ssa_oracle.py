@@ -192,7 +192,7 @@ def _block_masks(idx_row: np.ndarray, i: int, s: int):
     return causal, causal & sel
 
 
-def forward_dual(Q, K, V, idx, s: int, scale: float) -> dict[str, np.ndarray]:
+def forward_dual(Q, K, V, idx, s: int, scale: float, qblocks=None) -> dict[str, np.ndarray]:
     """Both attention streams, the dropped mass and the log-sum-exps.
 
     Returns float64 arrays:
@@ -205,6 +205,8 @@ def forward_dual(Q, K, V, idx, s: int, scale: float) -> dict[str, np.ndarray]:
                dropped attention mass ([summary] "1. Probleemstelling" and
                "Bidirectionele Uitlijning"; [record] abstract);
       lse_full, lse_sel [B,Hq,N]  natural-log normalisers of the two softmaxes.
+    qblocks: optional iterable of query-block indices to compute (rows of other
+    blocks are left at zero); used to sample large problems.
     """
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     B, Hq, N, d = Q.shape
@@ -215,10 +217,11 @@ def forward_dual(Q, K, V, idx, s: int, scale: float) -> dict[str, np.ndarray]:
     delta = np.zeros((B, Hq, N))
     lse_full = np.zeros((B, Hq, N))
     lse_sel = np.zeros((B, Hq, N))
+    blocks = range(n) if qblocks is None else sorted(set(int(i) for i in qblocks))
     for b in range(B):
         for h in range(Hq):
             kv = h // g
-            for i in range(n):
+            for i in blocks:
                 rows = slice(i * s, (i + 1) * s)
                 cols = (i + 1) * s
                 X = _row_logits(Q[b, h, rows], K[b, kv, :cols], scale)
@@ -248,22 +251,24 @@ def align_losses(h_full, h_sparse) -> tuple[float, float]:
     return mse, mse
 
 
-def align_grads(h_full, h_sparse) -> dict[str, np.ndarray]:
+def align_grads(h_full, h_sparse, M: int | None = None) -> dict[str, np.ndarray]:
     """Gradients of each alignment term w.r.t. each stream, stop-gradient applied.
 
     d L_sparsity / d h_full  = 2 (h_full - h_sparse) / M,  d L_sparsity / d h_sparse = 0;
     d L_commitment / d h_sparse = 2 (h_sparse - h_full) / M, d L_commitment / d h_full = 0;
     M = number of elements ([digest] "Bidirectional Attention Alignment":
-    sg[.] blocks the gradient through the auxiliary operand).
+    sg[.] blocks the gradient through the auxiliary operand).  M defaults to
+    the size of the arrays given; pass the full problem's count when the arrays
+    are a sample of it.
     """
     hf, hs = _f64(h_full), _f64(h_sparse)
-    M = hf.size
+    M = hf.size if M is None else int(M)
     zero = np.zeros_like(hf)
     return {"sp_full": 2.0 * (hf - hs) / M, "sp_sparse": zero,
             "cm_full": zero, "cm_sparse": 2.0 * (hs - hf) / M}
 
 
-def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse):
+def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse, qblocks=None):
     """Backpropagate upstream gradients of h_full and h_sparse to Q, K, V.
 
     The two streams are differentiated separately, each through its own
@@ -276,6 +281,8 @@ def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse):
     selection is held fixed ([digest] "The Root Cause Behind the Paradox" and
     "SSA's Dual-Stream Training Mechanism": dropped pairs get gradient only
     through the full stream).  dh_full / dh_sparse may be None (zero).
+    qblocks: optional query blocks whose contributions are summed (all if None);
+    dQ is then exact on those blocks, dK / dV hold only their contributions.
     """
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     B, Hq, N, d = Q.shape
@@ -287,10 +294,11 @@ def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse):
     dQ = np.zeros_like(Q)
     dK = np.zeros_like(K)
     dV = np.zeros_like(V)
+    blocks = range(n) if qblocks is None else sorted(set(int(i) for i in qblocks))
     for b in range(B):
         for h in range(Hq):
             kv = h // g
-            for i in range(n):
+            for i in blocks:
                 rows = slice(i * s, (i + 1) * s)
                 cols = (i + 1) * s
                 Kc, Vc = K[b, kv, :cols], V[b, kv, :cols]
@@ -310,25 +318,27 @@ def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse):
 
 
 def ssa_backward(Q, K, V, idx, s: int, scale: float, g_full, g_sparse, alpha: float,
-                 fwd: dict | None = None):
+                 fwd: dict | None = None, qblocks=None, M: int | None = None):
     """Gradients of L = <g_full, h_full> + <g_sparse, h_sparse> + alpha * L_align.
 
     [summary] "Bidirectionele Uitlijning": the objective adds alpha times the
     alignment loss to the stream losses; the stream losses reach this layer
     as the upstream gradients g_full / g_sparse (either may be None).
+    qblocks / M sample a large problem: only those query blocks are computed,
+    M is the full problem's element count (L_align is then that sample's share).
     Returns (dQ, dK, dV, L_align, fwd).
     """
     if fwd is None:
-        fwd = forward_dual(Q, K, V, idx, s, scale)
+        fwd = forward_dual(Q, K, V, idx, s, scale, qblocks=qblocks)
     hf, hs = fwd["h_full"], fwd["h_sparse"]
-    gr = align_grads(hf, hs)
+    gr = align_grads(hf, hs, M)
     dh_full = alpha * (gr["sp_full"] + gr["cm_full"])
     dh_sparse = alpha * (gr["sp_sparse"] + gr["cm_sparse"])
     if g_full is not None:
         dh_full = dh_full + _f64(g_full)
     if g_sparse is not None:
         dh_sparse = dh_sparse + _f64(g_sparse)
-    dQ, dK, dV = backward_streams(Q, K, V, idx, s, scale, dh_full, dh_sparse)
+    dQ, dK, dV = backward_streams(Q, K, V, idx, s, scale, dh_full, dh_sparse, qblocks=qblocks)
     l_sp, l_cm = align_losses(hf, hs)
     return dQ, dK, dV, l_sp + l_cm, fwd
 
