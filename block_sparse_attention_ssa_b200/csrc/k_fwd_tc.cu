@@ -1,12 +1,519 @@
-// Tensor-core (tcgen05 / TMEM / TMA) dual-stream forward: not built yet.
+// Tensor-core dual-stream forward for sm_100a (bf16 in, fp32 accumulate, d = 128).
+//
+// What it computes is the same as the CUDA-core kernel ("SSA: Achieving
+// Sparser Attention ...", "Practical Implementation of SSA"; "Technische
+// Samenvatting: SSA", "1. Probleemstelling" and "Bidirectionele Uitlijning"):
+// per query t two disjoint online softmaxes, over A_t (keys in selected
+// blocks) and D_t (the other causal keys), merged at the end into h_sparse,
+// h_full, lse_sel, lse_full and the dropped mass delta.  Every causal K/V tile
+// is read once and multiplied once: each tile's P goes into exactly one of the
+// two output accumulators per row, so the dual stream costs the MMAs of one
+// causal attention.
+//
+// CTA = one 128-row query tile of one (batch, query head), 192 threads:
+//   warps 0-3  softmax / rescale / epilogue; warp w owns TMEM lanes 32w..32w+31,
+//              i.e. query rows 32w..32w+31 of the tile (one row per thread);
+//   warp 4     TMA producer (Q once, then K and V tiles through an NS-stage ring);
+//   warp 5     TMEM allocator and single-thread tcgen05.mma issuer.
+// Key tiles are one key block (BN = block size, 64 or 128 keys).
+// TMEM (512 columns): O_A [0,128), O_D [128,256), S ping-pong [256,256+2BN).
+// P (bf16, two per column) overwrites the first BN/2 columns of its S buffer
+// and feeds the PV MMA from TMEM.
+//
+// With block 64 a 128-row query tile covers two query blocks whose selections
+// differ.  A key tile can then be selected for one half and dropped for the
+// other ("mixed"): that half's rows write P into a second P region (the next
+// BN/2 columns of the S buffer), the other half writes zeros there and into
+// the first region as needed, and the MMA warp issues one PV per accumulator.
+//
+// Softmax in base 2 with the scale folded in: p = 2^(S*c - m), c = scale*log2(e).
+// A row's running max m is raised only when a tile's max exceeds it by more
+// than 8 (p stays below 2^8); O and l are then rescaled in place after the
+// previous PV into that accumulator has completed.
 #include "ssa_internal.cuh"
+#include "sm100_ptx.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace ssa {
+namespace {
 
-bool fwd_tc_supported(const Dims&) { return false; }
+using namespace sm100;
 
-cudaError_t launch_fwd_tc(const Dims&, const FwdArgs&, int32_t*, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int BM = 128;
+constexpr int HD = 128;
+constexpr int NTHREADS = 192;
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int BN>
+struct Cfg {
+  static constexpr int NS = (BN == 64) ? 4 : 2;
+  static constexpr int Q_BYTES = BM * HD * 2;
+  static constexpr int KV_BYTES = BN * HD * 2;  // one K or V tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr int OFF_MISC = OFF_V + NS * KV_BYTES;
+  static constexpr int MISC_BYTES = 2048;
+  static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+  static constexpr uint32_t COL_OA = 0, COL_OD = 128, COL_S = 256;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
+};
+
+struct Misc {
+  uint64_t q_full;
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_done, o_final, drain;
+  uint32_t tmem_base;
+  int abort;
+  uint32_t sel[2][64];  // selected-block bits of the tile's two query blocks
+};
+
+struct TcParams {
+  TensorRef hf, hs;
+  const int32_t* idx;
+  float* lse_full;
+  float* lse_sel;
+  float* delta;
+  int32_t* status;
+  int Hq, g, N, n, k;
+  float c;  // scale * log2(e)
+};
+
+// Tile state of one half of the query tile: 0 none (no causal key), 1 selected, 2 dropped.
+__device__ __forceinline__ int tile_state(int j, int ib, bool valid, const uint32_t* selw) {
+  if (!valid || j > ib) return 0;
+  return ((selw[j >> 5] >> (j & 31)) & 1u) ? 1 : 2;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, TcParams p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Misc& M = *reinterpret_cast<Misc*>(smem + C::OFF_MISC);
+  volatile int* abort = &M.abort;
+
+  // A kernel of this library already gave up on a wait: skip the work so a
+  // broken launch fails fast; the caller sees the status word.
+  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = (int)(gridDim.x - 1 - blockIdx.x);  // heaviest tiles first
+  const int h = blockIdx.y, b = blockIdx.z, kvh = h / p.g;
+  const int q0 = qt * BM;
+  const int ib0 = (BN == 64) ? 2 * qt : qt;
+  const int ib1 = (BN == 64) ? 2 * qt + 1 : qt;
+  const bool valid1 = (BN == 64) ? (ib1 < p.n) : true;
+  const int q_end = min(q0 + BM, p.N);
+  const int T = (q_end + BN - 1) / BN;  // causal key tiles
+
+  // ---- set-up
+  if (threadIdx.x == 0) {
+    mbar_init(&M.q_full, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&M.k_full[s], 1);
+      mbar_init(&M.k_empty[s], 1);
+      mbar_init(&M.v_full[s], 1);
+      mbar_init(&M.v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&M.s_full[s], 1);
+      mbar_init(&M.p_full[s], 4);
+    }
+    mbar_init(&M.o_done, 1);
+    mbar_init(&M.o_final, 1);
+    mbar_init(&M.drain, 1);
+    M.abort = 0;
+    fence_mbar_init();
+  }
+  for (int w = threadIdx.x; w < 2 * 64; w += NTHREADS) (&M.sel[0][0])[w] = 0u;
+  if (warp == 5) {
+    tmem_alloc(&M.tmem_base, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  {
+    const int32_t* r0 = p.idx + (((int64_t)b * p.Hq + h) * p.n + ib0) * p.k;
+    for (int e = threadIdx.x; e < p.k; e += NTHREADS) {
+      const int j = r0[e];
+      if (j >= 0 && j <= ib0) atomicOr(&M.sel[0][j >> 5], 1u << (j & 31));
+    }
+    if (BN == 64 && valid1) {
+      const int32_t* r1 = p.idx + (((int64_t)b * p.Hq + h) * p.n + ib1) * p.k;
+      for (int e = threadIdx.x; e < p.k; e += NTHREADS) {
+        const int j = r1[e];
+        if (j >= 0 && j <= ib1) atomicOr(&M.sel[1][j >> 5], 1u << (j & 31));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = M.tmem_base;
+  const uint32_t* sel0 = M.sel[0];
+  const uint32_t* sel1 = (BN == 64) ? M.sel[1] : M.sel[0];
+
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+
+  if (warp == 4) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      mbar_expect_tx(&M.q_full, C::Q_BYTES);
+      tma_load_4d(sQ, &tmQ, &M.q_full, 0, q0, h, b);
+      tma_load_4d(sQ + C::Q_BYTES / 2, &tmQ, &M.q_full, 64, q0, h, b);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < T; ++j) {
+        const int st = j % C::NS;
+        const uint32_t use = (uint32_t)(j / C::NS);
+        if (j >= C::NS && !mbar_wait(&M.k_empty[st], (use - 1) & 1u, abort)) break;
+        mbar_expect_tx(&M.k_full[st], C::KV_BYTES);
+        tma_load_4d(sK + st * C::KV_BYTES, &tmK, &M.k_full[st], 0, j * BN, kvh, b);
+        tma_load_4d(sK + st * C::KV_BYTES + C::KV_BYTES / 2, &tmK, &M.k_full[st], 64, j * BN, kvh, b);
+        k_issued = j + 1;
+        if (j >= C::NS && !mbar_wait(&M.v_empty[st], (use - 1) & 1u, abort)) break;
+        mbar_expect_tx(&M.v_full[st], C::KV_BYTES);
+        tma_load_4d(sV + st * C::KV_BYTES, &tmV, &M.v_full[st], 0, j * BN, kvh, b);
+        tma_load_4d(sV + st * C::KV_BYTES + C::KV_BYTES / 2, &tmV, &M.v_full[st], 64, j * BN, kvh, b);
+        v_issued = j + 1;
+      }
+      // Drain: every copy this thread issued must have landed before the CTA exits.
+      int dummy = 0;
+      mbar_wait(&M.q_full, 0, &dummy);
+      for (int j = (k_issued > C::NS ? k_issued - C::NS : 0); j < k_issued; ++j) {
+        dummy = 0;
+        mbar_wait(&M.k_full[j % C::NS], (uint32_t)(j / C::NS) & 1u, &dummy);
+      }
+      for (int j = (v_issued > C::NS ? v_issued - C::NS : 0); j < v_issued; ++j) {
+        dummy = 0;
+        mbar_wait(&M.v_full[j % C::NS], (uint32_t)(j / C::NS) & 1u, &dummy);
+      }
+    }
+  } else if (warp == 5) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(sQ);
+      bool started_a = false, started_d = false;
+      bool ok = mbar_wait(&M.q_full, 0, abort);
+      auto issue_pv = [&](int jj) -> bool {
+        const int sb = jj & 1;
+        if (!mbar_wait(&M.p_full[sb], (uint32_t)(jj >> 1) & 1u, abort)) return false;
+        const int st = jj % C::NS;
+        if (!mbar_wait(&M.v_full[st], (uint32_t)(jj / C::NS) & 1u, abort)) return false;
+        tc_fence_after();
+        const int s0 = tile_state(jj, ib0, true, sel0);
+        const int s1 = tile_state(jj, ib1, valid1, sel1);
+        const bool mixed = (s0 != 0 && s1 != 0 && s0 != s1);
+        const int target = s0 != 0 ? s0 : s1;
+        const uint32_t v_addr = smem_u32(sV + st * C::KV_BYTES);
+        const uint32_t p_col = C::COL_S + (uint32_t)sb * BN;
+        auto pv = [&](uint32_t o_col, uint32_t pcol, bool& started) {
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
+            mma_ts(tmem + o_col, tmem + pcol + kk * 8, bdesc, C::IDESC_PV, (started || kk > 0) ? 1u : 0u);
+          }
+          started = true;
+        };
+        if (mixed) {
+          pv(C::COL_OA, p_col, started_a);
+          pv(C::COL_OD, p_col + BN / 2, started_d);
+        } else if (target == 1) {
+          pv(C::COL_OA, p_col, started_a);
+        } else {
+          pv(C::COL_OD, p_col, started_d);
+        }
+        tc_commit(&M.v_empty[st]);
+        tc_commit(&M.o_done);
+        return true;
+      };
+      for (int j = 0; ok && j < T; ++j) {
+        const int st = j % C::NS;
+        if (!mbar_wait(&M.k_full[st], (uint32_t)(j / C::NS) & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sK + st * C::KV_BYTES);
+        const uint32_t s_col = C::COL_S + (uint32_t)(j & 1) * BN;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off_q = (kk >> 2) * (C::Q_BYTES / 2) + (kk & 3) * 32;
+          const uint32_t off_k = (kk >> 2) * (C::KV_BYTES / 2) + (kk & 3) * 32;
+          const uint64_t adesc = smem_desc_sw128(q_addr + off_q, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(k_addr + off_k, 16, 1024);
+          mma_ss(tmem + s_col, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&M.s_full[j & 1]);
+        tc_commit(&M.k_empty[st]);
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && T >= 1) ok = issue_pv(T - 1);
+      tc_commit(&M.o_final);
+      tc_commit(&M.drain);
+      int dummy = 0;
+      mbar_wait(&M.drain, 0, &dummy);
+    }
+  } else {
+    // ================================================================ softmax
+    const int half = (BN == 64) ? (warp >> 1) : 0;
+    const int row = warp * 32 + lane;  // row within the tile == TMEM lane
+    const int t = q0 + row;            // query token
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float m2[2] = {kNegInf, kNegInf};  // running max (scaled, base 2), [0]=A [1]=D
+    float l[2] = {0.f, 0.f};
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int sb = j & 1;
+      if (!mbar_wait(&M.s_full[sb], (uint32_t)(j >> 1) & 1u, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int s0 = tile_state(j, ib0, true, sel0);
+      const int s1 = tile_state(j, ib1, valid1, sel1);
+      const bool mixed = (s0 != 0 && s1 != 0 && s0 != s1);
+      const int mine = half ? s1 : s0;
+      const uint32_t s_addr = lane_base + C::COL_S + (uint32_t)sb * BN;
+      uint32_t pk[BN / 2];
+      if (mine == 0) {
+#pragma unroll
+        for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
+      } else {
+        float x[BN];
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(s_addr + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(r[c]) * p.c;
+        }
+        // causal mask inside the diagonal tile
+        const int u0 = j * BN;
+        if (u0 + BN - 1 > t) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (u0 + c > t) x[c] = kNegInf;
+        }
+        float mx = kNegInf;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, x[c]);
+        const int X = mine - 1;  // 0 = A, 1 = D
+        const float m_old = m2[X];
+        const bool need = (m_old != kNegInf) && (mx > m_old + kRescaleThreshold);
+        if (__any_sync(0xffffffffu, need)) {
+          // O_X must hold every earlier PV before it is rescaled.
+          if (!mbar_wait(&M.o_done, (uint32_t)(j - 1) & 1u, abort)) {
+            ok = false;
+          }
+          if (__any_sync(0xffffffffu, !ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = need ? ex2(m_old - mx) : 1.0f;
+          const uint32_t o_addr = lane_base + (X == 0 ? C::COL_OA : C::COL_OD);
+#pragma unroll 1
+          for (int c0 = 0; c0 < HD; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(o_addr + c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
+            tmem_st32(o_addr + c0, r);
+          }
+          tmem_wait_st();
+          if (need) {
+            l[X] *= f;
+            m2[X] = mx;
+          }
+        }
+        if (m2[X] == kNegInf) m2[X] = mx;
+        const float m = m2[X];
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float e0 = ex2(x[c] - m);
+          const float e1 = ex2(x[c + 1] - m);
+          sum += e0 + e1;
+          pk[c / 2] = pack_bf16(e0, e1);
+        }
+        l[X] += sum;
+      }
+      // Write P where the MMA warp will read it.
+      const uint32_t p0 = s_addr, p1 = s_addr + BN / 2;
+      if (mixed && mine == 2) {
+        uint32_t z[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) z[c] = 0u;
+#pragma unroll
+        for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+          tmem_st32(p0 + c0, z);
+          tmem_st32(p1 + c0, *reinterpret_cast<uint32_t(*)[32]>(&pk[c0]));
+        }
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < BN / 2; c0 += 32) tmem_st32(p0 + c0, *reinterpret_cast<uint32_t(*)[32]>(&pk[c0]));
+        if (mixed) {
+          uint32_t z[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) z[c] = 0u;
+#pragma unroll
+          for (int c0 = 0; c0 < BN / 2; c0 += 32) tmem_st32(p1 + c0, z);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.p_full[sb]);
+    }
+
+    // ================================================================ epilogue
+    if (ok && mbar_wait(&M.o_final, 0, abort)) {
+      tc_fence_after();
+      const bool store = t < p.N;
+      const float mA = m2[0], mD = m2[1], lA = l[0], lD = l[1];
+      const float Mx = fmaxf(mA, mD);
+      const float wa = (lA > 0.f) ? ex2(mA - Mx) : 0.f;
+      const float wd = (lD > 0.f) ? ex2(mD - Mx) : 0.f;
+      const float inv_full = 1.0f / (wa * lA + wd * lD);
+      const float inv_sel = (lA > 0.f) ? 1.0f / lA : 0.f;
+      __nv_bfloat16* hf = store ? row_ptr_w<__nv_bfloat16>(p.hf, b, h, t) : nullptr;
+      __nv_bfloat16* hs = store ? row_ptr_w<__nv_bfloat16>(p.hs, b, h, t) : nullptr;
+#pragma unroll 1
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        uint32_t ra[32], rd[32];
+        tmem_ld32(lane_base + C::COL_OA + c0, ra);
+        tmem_ld32(lane_base + C::COL_OD + c0, rd);
+        tmem_wait_ld();
+        if (store) {
+          uint32_t of[16], os[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float a0 = (lA > 0.f) ? __uint_as_float(ra[c]) : 0.f;
+            const float a1 = (lA > 0.f) ? __uint_as_float(ra[c + 1]) : 0.f;
+            const float d0 = (lD > 0.f) ? __uint_as_float(rd[c]) : 0.f;
+            const float d1 = (lD > 0.f) ? __uint_as_float(rd[c + 1]) : 0.f;
+            os[c / 2] = pack_bf16(a0 * inv_sel, a1 * inv_sel);
+            of[c / 2] = pack_bf16((wa * a0 + wd * d0) * inv_full, (wa * a1 + wd * d1) * inv_full);
+          }
+          uint4* dst_s = reinterpret_cast<uint4*>(hs + c0);
+          uint4* dst_f = reinterpret_cast<uint4*>(hf + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            dst_s[q] = make_uint4(os[4 * q], os[4 * q + 1], os[4 * q + 2], os[4 * q + 3]);
+            dst_f[q] = make_uint4(of[4 * q], of[4 * q + 1], of[4 * q + 2], of[4 * q + 3]);
+          }
+        }
+      }
+      if (store) {
+        constexpr float kLn2 = 0.6931471805599453f;
+        const float lse2_a = (lA > 0.f) ? mA + log2f(lA) : kNegInf;
+        const float lse2_d = (lD > 0.f) ? mD + log2f(lD) : kNegInf;
+        const float hi = fmaxf(lse2_a, lse2_d), lo = fminf(lse2_a, lse2_d);
+        const float lse2_f = (lo == kNegInf) ? hi : hi + log2f(1.0f + ex2(lo - hi));
+        const int64_t o = ((int64_t)b * p.Hq + h) * p.N + t;
+        p.lse_full[o] = lse2_f * kLn2;
+        p.lse_sel[o] = (lA > 0.f) ? lse2_a * kLn2 : kNegInf;
+        p.delta[o] = (lD > 0.f) ? ex2(lse2_d - lse2_f) : 0.f;
+      }
+    }
+  }
+
+  // ---- tear-down
+  tc_fence_before();
+  __syncthreads();
+  if (M.abort && threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_TIMEOUT);
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 4-D map over a [B, H, N, d] bf16 tensor: dims (d, N, H, B), box (64, rows, 1, 1).
+bool make_map(CUtensorMap* map, const TensorRef& t, int B, int H, int N, int rows) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)t.sn * 2, (cuuint64_t)t.sh * 2, (cuuint64_t)t.sb * 2};
+  // A zero stride (a broadcast dimension of size 1) is not accepted; any
+  // positive multiple of 16 describes the same single slice.
+  for (int i = 0; i < 3; ++i)
+    if (strides[i] == 0) strides[i] = 16;
+  cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(t.p), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_bn(const Dims& D, const FwdArgs& a, int32_t* status, cudaStream_t st) {
+  using C = Cfg<BN>;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, D.B, D.Hq, D.N, BM) || !make_map(&mk, a.k, D.B, D.Hkv, D.N, BN) ||
+      !make_map(&mv, a.v, D.B, D.Hkv, D.N, BN))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.hf = a.hf;
+  p.hs = a.hs;
+  p.idx = a.idx;
+  p.lse_full = a.lse_full;
+  p.lse_sel = a.lse_sel;
+  p.delta = a.delta;
+  p.status = status;
+  p.Hq = D.Hq;
+  p.g = D.g;
+  p.N = D.N;
+  p.n = D.n;
+  p.k = D.k;
+  p.c = D.scale * 1.4426950408889634f;
+  auto kern = fwd_tc_kernel<BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid((D.N + BM - 1) / BM, D.Hq, D.B);
+  kern<<<grid, NTHREADS, C::SMEM, st>>>(mq, mk, mv, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool fwd_tc_supported(const Dims& D) {
+  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048;
+}
+
+cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st) {
+  if (!fwd_tc_supported(D)) return cudaErrorNotSupported;
+  return D.s == 64 ? launch_bn<64>(D, a, dev_status, st) : launch_bn<128>(D, a, dev_status, st);
 }
 
 }  // namespace ssa

@@ -45,7 +45,9 @@
  *   ssa_workspace_bytes) and enqueues nothing.  A failed launch returns
  *   SSA_ERR_CUDA.  Kernels that wait on hardware barriers bound every wait;
  *   a wait that runs out records SSA_ERR_TIMEOUT in a device status word
- *   (read it with ssa_device_status) and the kernel returns.  No kernel traps.
+ *   (read it with ssa_device_status) and the kernel returns.  While that word
+ *   holds an error, the tensor-core kernels skip their work (their outputs
+ *   are then undefined) until ssa_device_status clears it.  No kernel traps.
  * Precision.  dtype SSA_BF16: inputs/outputs bf16, products on tensor cores
  *   with fp32 accumulation and fp32 softmax statistics.  SSA_F32: fp32 inputs
  *   and outputs, fp32 arithmetic throughout (CUDA cores).

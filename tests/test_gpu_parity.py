@@ -27,7 +27,7 @@ CASES = {
     "f32_mha_d64": (1, 2, 2, 512, 64, 64, 4, "f32"),
     "f32_gqa_d128": (1, 4, 2, 384, 128, 64, 3, "f32"),
     "f32_many_blocks": (1, 1, 1, 2112, 64, 64, 5, "f32"),
-    "bf16_gqa_odd_blocks": (1, 4, 1, 640, 128, 64, 4, "bf16"),
+    "bf16_gqa_odd_blocks": (1, 4, 1, 576, 128, 64, 4, "bf16"),
     "bf16_s128": (1, 2, 1, 768, 128, 128, 3, "bf16"),
     "bf16_d64_b2": (2, 2, 2, 448, 64, 64, 3, "bf16"),
     "bf16_full_budget": (1, 2, 1, 512, 128, 64, 16, "bf16"),
@@ -239,3 +239,83 @@ def test_unsupported_shape_raises():
         api.ssa_fwd_dual(dims, x, x, x, torch.zeros(1, dtype=torch.int32, device="cuda"), x, x,
                          o["lse_full"], o["lse_sel"], o["delta"])
     assert ei.value.code == api.SSA_ERR_UNSUPPORTED
+
+
+def _custom_idx(B, H, n, k, seed, drop_diag_frac=0.0, pad_frac=0.0):
+    """Random selections: the diagonal plus k-1 random earlier blocks, with an
+    optional share of rows that omit the diagonal, pad with -1 or repeat an
+    entry.  Adjacent query blocks disagree often, which at block 64 makes many
+    key tiles selected for one half of a 128-row query tile and dropped for
+    the other."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    idx = np.full((B, H, n, k), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(n):
+                if i + 1 <= k:
+                    row = list(range(i + 1))
+                else:
+                    row = sorted(rng.choice(i, size=k - 1, replace=False).tolist() + [i])
+                if rng.random() < drop_diag_frac and len(row) > 1:
+                    row = row[:-1]
+                if rng.random() < pad_frac and len(row) > 1:
+                    row = row[:-1] + [row[0]]
+                idx[b, h, i, :len(row)] = row
+    return idx
+
+
+@pytest.mark.parametrize("cfg", [(1, 4, 2, 1024, 128, 64, 5), (1, 2, 1, 1152, 128, 64, 4),
+                                 (1, 2, 2, 1024, 128, 128, 3)])
+@pytest.mark.parametrize("extra", ["plain", "no_diag"])
+def test_forward_custom_selection(cfg, extra):
+    """Given selections (not computed by the path): mixed tiles, rows without
+    their diagonal block, duplicated entries and -1 padding."""
+    B, Hq, Hkv, N, d, s, k = cfg
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 303, "bf16")
+    n = N // s
+    idx = _custom_idx(B, Hq, n, k, seed=N + k, drop_diag_frac=0.3 if extra == "no_diag" else 0.0,
+                      pad_frac=0.2 if extra == "no_diag" else 0.0)
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
+    out = api.alloc_forward(dims)
+    api.ssa_fwd_dual(dims, dev["Q"], dev["K"], dev["V"], torch.from_numpy(idx).cuda(), out["h_full"],
+                     out["h_sparse"], out["lse_full"], out["lse_sel"], out["delta"])
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    ora = O.forward_dual(host["Q"], host["K"], host["V"], idx, s, 1 / math.sqrt(d))
+    for key in ("h_full", "h_sparse", "delta"):
+        err = np.abs(f64(out[key]) - ora[key]).max()
+        assert err <= TOL["bf16"]["out"], (key, err)
+    fin = np.isfinite(ora["lse_sel"])
+    assert np.array_equal(np.isfinite(f64(out["lse_sel"])), fin)
+    assert np.abs(f64(out["lse_sel"])[fin] - ora["lse_sel"][fin]).max() <= TOL["bf16"]["lse"]
+    assert np.abs(f64(out["lse_full"]) - ora["lse_full"]).max() <= TOL["bf16"]["lse"]
+
+
+@pytest.mark.parametrize("s", [64, 128])
+def test_forward_large_logits(s):
+    """Logits with a wide range (keys scaled up, one late block boosted) make
+    the running max jump by far more than the rescale threshold mid-row."""
+    B, Hq, Hkv, N, d, k = 1, 2, 1, 1024, 128, 4
+    from block_sparse_attention_ssa_b200.inputs import make_qkv
+    t = make_qkv(B, Hq, Hkv, N, d, s, 404)
+    t["K"] *= 3.0
+    t["K"][:, :, 5 * s:6 * s] *= 2.5
+    host = {x: oracle_view(t[x], "bf16") for x in ("Q", "K", "V")}
+    dev = {x: upload(t[x], "bf16") for x in ("Q", "K", "V")}
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
+    ws = api.alloc_workspace(dims)
+    out = api.alloc_forward(dims)
+    api.forward(dims, dev["Q"], dev["K"], dev["V"], out, ws)
+    torch.cuda.synchronize()
+    ora_scores = O.block_scores(host["Q"], host["K"], s, 1 / math.sqrt(d))
+    ora_idx = O.select_blocks(ora_scores, k)
+    if compare_selection(out["idx"].cpu().numpy(), ora_idx, ora_scores):
+        out["idx"].copy_(torch.from_numpy(ora_idx))
+        api.ssa_fwd_dual(dims, dev["Q"], dev["K"], dev["V"], out["idx"], out["h_full"], out["h_sparse"],
+                         out["lse_full"], out["lse_sel"], out["delta"])
+        torch.cuda.synchronize()
+    ora = O.forward_dual(host["Q"], host["K"], host["V"], ora_idx, s, 1 / math.sqrt(d))
+    for key in ("h_full", "h_sparse", "delta"):
+        err = np.abs(f64(out[key]) - ora[key]).max()
+        assert err <= TOL["bf16"]["out"], (key, err)
+    assert np.abs(f64(out["lse_full"]) - ora["lse_full"]).max() <= 2e-2
