@@ -81,6 +81,8 @@ _SIGS = {
                                       ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "ssa_device_status": (ctypes.c_int, [_P(ctypes.c_int32), ctypes.c_int, ctypes.c_void_p]),
     "ssa_launch_count": (ctypes.c_uint64, []),
+    "ssa_block_scores_noalloc": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
+                                                 ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 _lib = None
@@ -154,6 +156,13 @@ def ssa_workspace_bytes(dims: ssa_dims_t) -> int:
 def ssa_block_scores(dims, Q, K, scores, ws, stream=None) -> None:
     _check("ssa_block_scores", load_library().ssa_block_scores(
         ctypes.byref(dims), _t(Q), _t(K), _p(scores), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def ssa_block_scores_noalloc(dims, Q, K, scores, stream=None) -> None:
+    """ssa_block_scores with the library's fixed device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    _check("ssa_block_scores_noalloc", load_library().ssa_block_scores_noalloc(
+        ctypes.byref(dims), _t(Q), _t(K), _p(scores), _stream(stream)))
 
 
 def ssa_select_topk(dims, scores, idx, stream=None) -> None:

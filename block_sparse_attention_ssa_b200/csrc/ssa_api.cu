@@ -2,6 +2,7 @@
 // Every check runs on the host before anything is enqueued; see include/ssa.h.
 #include <atomic>
 #include <cstring>
+#include <mutex>
 
 #include "ssa_internal.cuh"
 
@@ -334,3 +335,63 @@ ssa_status_t ssa_device_status(int32_t* status, int clear, ssa_stream_t stream) 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc variant
+// Fixed device scratch for ssa_block_scores_noalloc (see include/ssa.h).  In
+// host code this name is only a stand-in for the symbol, never a device
+// address: the address is looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) float g_noalloc_scratch[SSA_NOALLOC_SCRATCH_FLOATS];
+
+namespace ssa {
+namespace {
+
+constexpr int kMaxDevices = 128;
+float* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device, looked up once.
+ssa_status_t noalloc_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return SSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return SSA_OK;
+}
+
+}  // namespace
+}  // namespace ssa
+
+extern "C" ssa_status_t ssa_block_scores_noalloc(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                                                 const ssa_tensor_t* K, float* scores,
+                                                 ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  TensorRef q, k;
+  if ((s = check_tensor(D, Q, false, &q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &k)) != SSA_OK) return s;
+  if (scores == nullptr || reinterpret_cast<uintptr_t>(scores) % 4) return SSA_ERR_INVALID_ARG;
+  const uint64_t q_floats = (uint64_t)D.B * D.Hq * D.n * D.d;
+  const uint64_t k_floats = (uint64_t)D.B * D.Hkv * D.n * D.d;
+  if (q_floats + k_floats > (uint64_t)SSA_NOALLOC_SCRATCH_FLOATS) return SSA_ERR_WORKSPACE;
+  if ((s = check_device()) != SSA_OK) return s;
+  float* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != SSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // q-bar at the start, k-bar after it (256-byte aligned, like the workspace layout).
+  float* qbar = scratch;
+  float* kbar = scratch + (q_floats + 63) / 64 * 64;
+  if ((uint64_t)(kbar - scratch) + k_floats > (uint64_t)SSA_NOALLOC_SCRATCH_FLOATS) return SSA_ERR_WORKSPACE;
+  cudaError_t e = launch_pool(D, q, D.Hq, qbar, st);
+  if (e == cudaSuccess) e = launch_pool(D, k, D.Hkv, kbar, st);
+  if (e == cudaSuccess) e = launch_scores(D, qbar, kbar, scores, st);
+  return from_cuda(e);
+}

@@ -208,6 +208,37 @@ SSA_API ssa_status_t ssa_align_mse(const ssa_dims_t* dims, const ssa_tensor_t* h
                            const ssa_tensor_t* h_sparse, float* loss, void* ws,
                            size_t ws_bytes, ssa_stream_t stream);
 
+/* Capacity, in floats, of the fixed device scratch array used by
+ * ssa_block_scores_noalloc: B * (Hq + Hkv) * n * d must not exceed it
+ * (4 Mi floats = 16 MiB; the gqa_16k, long_64k and sweep_32k shapes fit). */
+#define SSA_NOALLOC_SCRATCH_FLOATS (4u << 20)
+
+/* ssa_block_scores without a caller-supplied workspace.
+ * The paper has no counterpart: this exists for callers that cannot call
+ * cudaMalloc -- for example code running inside a host framework that owns
+ * all device memory and only hands out the tensors it allocated itself, or a
+ * latency-critical loop where an allocation (and the device synchronisation
+ * a cudaFree implies) is not acceptable.  It computes exactly what
+ * ssa_block_scores computes, from the same kernels, but keeps the pooled
+ * block means in a fixed array of SSA_NOALLOC_SCRATCH_FLOATS floats that the
+ * library declares in device memory; every GPU that loads the library holds
+ * those 16 MiB until the process exits.  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   Q, K, scores: as for ssa_block_scores (the caller still owns inputs and
+ *     outputs).
+ *   Returns SSA_ERR_WORKSPACE, enqueuing nothing, when
+ *     B * (Hq + Hkv) * n * d > SSA_NOALLOC_SCRATCH_FLOATS.
+ * The first call on a device looks up the array's device address once (with
+ * that device current) and caches it; make that first call before any
+ * stream capture.  All calls share the one array and it keeps the last
+ * call's contents; nothing in it needs to start at zero, because every value
+ * the scoring kernel reads was written by the same call.  Calls whose work
+ * overlaps on the GPU (different streams, or different host threads without
+ * ordering) race on the array: order them on one stream. */
+SSA_API ssa_status_t ssa_block_scores_noalloc(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                                              const ssa_tensor_t* K, float* scores,
+                                              ssa_stream_t stream);
+
 /* Number of kernels this library has enqueued in this process so far (all
  * devices, all threads).  Lets a caller count the launches of a region. */
 SSA_API uint64_t ssa_launch_count(void);
