@@ -444,43 +444,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// 4-D map over a [B, H, N, d] bf16 tensor: dims (d, N, H, B), box (64, rows, 1, 1).
-bool make_map(CUtensorMap* map, const TensorRef& t, int B, int H, int N, int rows) {
-  auto enc = get_encode();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)t.sn * 2, (cuuint64_t)t.sh * 2, (cuuint64_t)t.sb * 2};
-  // A zero stride (a broadcast dimension of size 1) is not accepted; any
-  // positive multiple of 16 describes the same single slice.
-  for (int i = 0; i < 3; ++i)
-    if (strides[i] == 0) strides[i] = 16;
-  cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(t.p), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int BN>
 cudaError_t launch_bn(const Dims& D, const FwdArgs& a, int32_t* status, cudaStream_t st) {
   using C = Cfg<BN>;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.q, D.B, D.Hq, D.N, BM) || !make_map(&mk, a.k, D.B, D.Hkv, D.N, BN) ||
-      !make_map(&mv, a.v, D.B, D.Hkv, D.N, BN))
+  if (!make_tma_map_bf16(&mq, a.q, D.B, D.Hq, D.N, BM) || !make_tma_map_bf16(&mk, a.k, D.B, D.Hkv, D.N, BN) ||
+      !make_tma_map_bf16(&mv, a.v, D.B, D.Hkv, D.N, BN))
     return cudaErrorInvalidValue;
   TcParams p;
   p.hf = a.hf;
@@ -506,6 +475,37 @@ cudaError_t launch_bn(const Dims& D, const FwdArgs& a, int32_t* status, cudaStre
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 4-D map over a [B, H, N, d] bf16 tensor: dims (d, N, H, B), box (64, rows, 1, 1).
+bool make_tma_map_bf16(CUtensorMap* map, const TensorRef& t, int B, int H, int N, int rows) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)t.sn * 2, (cuuint64_t)t.sh * 2, (cuuint64_t)t.sb * 2};
+  // A zero stride (a broadcast dimension of size 1) is not accepted; any
+  // positive multiple of 16 describes the same single slice.
+  for (int i = 0; i < 3; ++i)
+    if (strides[i] == 0) strides[i] = 16;
+  cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(t.p), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 bool fwd_tc_supported(const Dims& D) {
   return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048;

@@ -253,6 +253,8 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
   if ((s = check_tensor(D, dV, false, &a.dv)) != SSA_OK) return s;
   if (!(alpha == alpha)) return SSA_ERR_INVALID_ARG;
   if (!idx || !lse_full || !lse_sel) return SSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(lse_full) % 16 || reinterpret_cast<uintptr_t>(lse_sel) % 16)
+    return SSA_ERR_INVALID_ARG;
   if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
   if ((s = check_device()) != SSA_OK) return s;
   const Layout L = layout(D);
@@ -271,7 +273,13 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
   a.n_partials = L.n_partials;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_build_mask(D, idx, a.mask, L.words, st);
-  if (e == cudaSuccess) e = launch_bwd_pre(D, a, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (bwd_tc_supported(D)) {
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_bwd_tc(D, a, status, st));
+  }
+  e = launch_bwd_pre(D, a, st);
   if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
   return from_cuda(e);
 }
@@ -294,6 +302,11 @@ ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, con
   a.idx = idx;
   a.delta = delta;
   a.lse_in = lse_full;
+  if (fwd_tc_supported(D)) {
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_dropped_tc(D, a, status, static_cast<cudaStream_t>(stream)));
+  }
   return from_cuda(launch_dropped_simt(D, a, static_cast<cudaStream_t>(stream)));
 }
 

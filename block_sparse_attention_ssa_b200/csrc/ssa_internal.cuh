@@ -2,6 +2,7 @@
 // Nothing here is part of the C ABI (see include/ssa.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -100,11 +101,17 @@ struct FwdArgs {
 cudaError_t launch_fwd_simt(const Dims& D, const FwdArgs& a, cudaStream_t st);
 // CUDA-core dropped mass (no V).
 cudaError_t launch_dropped_simt(const Dims& D, const FwdArgs& a, cudaStream_t st);
+// Tensor-core dropped mass (bf16, d = 128; same envelope as the forward).
+cudaError_t launch_dropped_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
 
 // Tensor-core (tcgen05 / TMEM / TMA) dual-stream forward, bf16, d = 128.
 // Returns cudaErrorNotSupported when the shape is outside its envelope.
 cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
 bool fwd_tc_supported(const Dims& D);
+
+// 4-D TMA map over a [B, H, N, 128] bf16 tensor: dims (d, N, H, B), box
+// (64 columns, `rows` rows), 128-byte swizzle, zero fill out of bounds.
+bool make_tma_map_bf16(CUtensorMap* map, const TensorRef& t, int B, int H, int N, int rows);
 
 struct BwdArgs {
   TensorRef q, k, v, hf, hs, gf, gs, dq, dk, dv;  // gf / gs .p may be null
@@ -125,6 +132,9 @@ struct BwdArgs {
 };
 
 cudaError_t launch_bwd_pre(const Dims& D, const BwdArgs& a, cudaStream_t st);
+// Tensor-core backward (bf16, d = 128): preprocess + dK/dV + dQ launches.
+bool bwd_tc_supported(const Dims& D);
+cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* dev_status, cudaStream_t st);
 cudaError_t launch_bwd_simt(const Dims& D, const BwdArgs& a, cudaStream_t st);
 
 // Sum of squared differences of two [B,Hq,N,d] tensors into per-block

@@ -169,7 +169,8 @@ SSA_API ssa_status_t ssa_fwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q,
  * on the other).  The selection is held fixed: no gradient flows through idx
  * or delta.  dK and dV are summed over the g query heads of each kv head.
  *   Q, K, V, idx, h_full, h_sparse, lse_full, lse_sel: as passed to / written
- *     by ssa_fwd_dual for the same inputs.
+ *     by ssa_fwd_dual for the same inputs; lse_full and lse_sel must be
+ *     16-byte aligned.
  *   g_full, g_sparse: [B, Hq, N, d] dims->dtype, or NULL for zero.
  *   align_loss: device fp32 scalar (out) = L_align, or NULL.
  *   dQ [B,Hq,N,d], dK, dV [B,Hkv,N,d] (out): strided, dims->dtype; fully

@@ -319,3 +319,51 @@ def test_forward_large_logits(s):
         err = np.abs(f64(out[key]) - ora[key]).max()
         assert err <= TOL["bf16"]["out"], (key, err)
     assert np.abs(f64(out["lse_full"]) - ora["lse_full"]).max() <= 2e-2
+
+
+@pytest.mark.parametrize("cfg", [(1, 4, 2, 1024, 128, 64, 5), (1, 2, 1, 1152, 128, 64, 4),
+                                 (1, 4, 1, 1024, 128, 128, 3)])
+@pytest.mark.parametrize("extra", ["plain", "no_diag"])
+def test_backward_custom_selection(cfg, extra):
+    """Backward under given selections (tiles selected for one query block and
+    dropped for its neighbour, rows without their diagonal block), with
+    upstream gradients on both streams and the alignment term."""
+    B, Hq, Hkv, N, d, s, k = cfg
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 505, "bf16")
+    n = N // s
+    idx = _custom_idx(B, Hq, n, k, seed=N * 3 + k, drop_diag_frac=0.3 if extra == "no_diag" else 0.0,
+                      pad_frac=0.2 if extra == "no_diag" else 0.0)
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
+    ws = api.alloc_workspace(dims)
+    out = api.alloc_forward(dims)
+    out["idx"] = torch.from_numpy(idx).cuda()
+    api.ssa_fwd_dual(dims, dev["Q"], dev["K"], dev["V"], out["idx"], out["h_full"], out["h_sparse"],
+                     out["lse_full"], out["lse_sel"], out["delta"])
+    gf = make_upstream((B, Hq, N, d), 61)
+    gs = make_upstream((B, Hq, N, d), 62)
+    grads = api.alloc_backward(dims)
+    api.backward(dims, dev["Q"], dev["K"], dev["V"], out, upload(gf, "bf16"), upload(gs, "bf16"), 10.0, grads, ws)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    dQ, dK, dV, l_align, _ = O.ssa_backward(host["Q"], host["K"], host["V"], idx, s, 1 / math.sqrt(d),
+                                            oracle_view(gf, "bf16").astype(np.float64),
+                                            oracle_view(gs, "bf16").astype(np.float64), 10.0)
+    for name_, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        err = rel_l2(f64(got), ref)
+        assert err < TOL["bf16"]["grad"], (name_, err)
+
+
+def test_backward_alignment_only_bf16():
+    """bf16 path with no upstream gradient: every gradient comes from the
+    alignment terms, whose h_full - h_sparse is formed from bf16 outputs."""
+    r = run_case("bf16_gqa_odd_blocks")
+    B, Hq, Hkv, N, d, s, k, dt = r["cfg"]
+    grads = api.alloc_backward(r["dims"])
+    alpha = 1000.0
+    api.backward(r["dims"], r["dev"]["Q"], r["dev"]["K"], r["dev"]["V"], r["out"], None, None, alpha, grads, r["ws"])
+    torch.cuda.synchronize()
+    dQ, dK, dV, l_align, _ = O.ssa_backward(r["host"]["Q"], r["host"]["K"], r["host"]["V"], r["ora_idx"], s,
+                                            r["scale"], None, None, alpha, fwd=r["ora"])
+    for name_, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        err = rel_l2(f64(got), ref)
+        assert err < TOL["bf16"]["grad"], (name_, err)
