@@ -6,30 +6,30 @@
 // per query t two disjoint online softmaxes, over A_t (keys in selected
 // blocks) and D_t (the other causal keys), merged at the end into h_sparse,
 // h_full, lse_sel, lse_full and the dropped mass delta.  Every causal K/V tile
-// is read once and multiplied once: each tile's P goes into exactly one of the
+// is read once and multiplied once: each key's P goes into exactly one of the
 // two output accumulators per row, so the dual stream costs the MMAs of one
 // causal attention.
 //
 // CTA = one 128-row query tile of one (batch, query head), 192 threads:
 //   warps 0-3  softmax / rescale / epilogue; warp w owns TMEM lanes 32w..32w+31,
 //              i.e. query rows 32w..32w+31 of the tile (one row per thread);
-//   warp 4     TMA producer (Q once, then K and V tiles through an NS-stage ring);
+//   warp 4     TMA producer (Q once, then 128-key K and V tiles, 2-stage ring);
 //   warp 5     TMEM allocator and single-thread tcgen05.mma issuer.
-// Key tiles are one key block (BN = block size, 64 or 128 keys).
-// TMEM (512 columns): O_A [0,128), O_D [128,256), S ping-pong [256,256+2BN).
-// P (bf16, two per column) overwrites the first BN/2 columns of its S buffer
-// and feeds the PV MMA from TMEM.
+// TMEM (512 columns): O_A [0,128), O_D [128,256), S ping-pong [256,384), [384,512).
+// P (bf16, two per column) overwrites its S buffer and feeds the PV MMA from TMEM.
 //
-// With block 64 a 128-row query tile covers two query blocks whose selections
-// differ.  A key tile can then be selected for one half and dropped for the
-// other ("mixed"): that half's rows write P into a second P region (the next
-// BN/2 columns of the S buffer), the other half writes zeros there and into
-// the first region as needed, and the MMA warp issues one PV per accumulator.
+// A 128-key tile is two 64-key sub-blocks.  With block 64 each sub-block is a
+// key block of its own, and each 64-row half of the query tile is a query
+// block of its own, so a sub-block can be selected for one half and dropped
+// for the other ("mixed"): that sub-block then gets a second P region in which
+// only the dropped half's rows are non-zero, and the MMA warp issues one PV
+// per accumulator for it.  Every (half, sub-block) pair is in one of three
+// states: no causal key, selected (A) or dropped (D).
 //
 // Softmax in base 2 with the scale folded in: p = 2^(S*c - m), c = scale*log2(e).
-// A row's running max m is raised only when a tile's max exceeds it by more
-// than 8 (p stays below 2^8); O and l are then rescaled in place after the
-// previous PV into that accumulator has completed.
+// A row's running max m of each set is raised only when a tile's max for that
+// set exceeds it by more than 8 (p stays below 2^8); O and l are then rescaled
+// in place after the previous PV has completed.
 #include "ssa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -40,30 +40,28 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;
+constexpr int BM = 128;    // query rows per CTA
+constexpr int BN = 128;    // keys per tile
+constexpr int SUB = 64;    // keys per sub-block
 constexpr int HD = 128;
 constexpr int NTHREADS = 192;
+constexpr int NS = 2;      // K/V stages
 constexpr float kRescaleThreshold = 8.0f;
 
-template <int BN>
-struct Cfg {
-  static constexpr int NS = (BN == 64) ? 4 : 2;
-  static constexpr int Q_BYTES = BM * HD * 2;
-  static constexpr int KV_BYTES = BN * HD * 2;  // one K or V tile
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_MISC = OFF_V + NS * KV_BYTES;
-  static constexpr int MISC_BYTES = 2048;
-  static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-  static constexpr uint32_t COL_OA = 0, COL_OD = 128, COL_S = 256;
-  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
-  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-};
+constexpr int Q_BYTES = BM * HD * 2;
+constexpr int KV_BYTES = BN * HD * 2;  // one K or V tile
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = Q_BYTES;
+constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+constexpr int OFF_MISC = OFF_V + NS * KV_BYTES;
+constexpr int SMEM_BYTES = OFF_MISC + 2048 + 1024;  // + alignment slack
+constexpr uint32_t COL_OA = 0, COL_OD = 128, COL_S = 256;
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
 
 struct Misc {
   uint64_t q_full;
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t s_full[2], p_full[2];
   uint64_t o_done, o_final, drain;
   uint32_t tmem_base;
@@ -82,40 +80,38 @@ struct TcParams {
   float c;  // scale * log2(e)
 };
 
-// Tile state of one half of the query tile: 0 none (no causal key), 1 selected, 2 dropped.
-__device__ __forceinline__ int tile_state(int j, int ib, bool valid, const uint32_t* selw) {
-  if (!valid || j > ib) return 0;
-  return ((selw[j >> 5] >> (j & 31)) & 1u) ? 1 : 2;
+// State of (query block ib, key block kb): 0 no causal key, 1 selected, 2 dropped.
+__device__ __forceinline__ int pair_state(int kb, int ib, bool valid, const uint32_t* selw) {
+  if (!valid || kb > ib) return 0;
+  return ((selw[kb >> 5] >> (kb & 31)) & 1u) ? 1 : 2;
 }
 
-template <int BN>
+template <int S_BLK>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, TcParams p) {
-  using C = Cfg<BN>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Misc& M = *reinterpret_cast<Misc*>(smem + C::OFF_MISC);
-  volatile int* abort = &M.abort;
-
   // A kernel of this library already gave up on a wait: skip the work so a
   // broken launch fails fast; the caller sees the status word.
   if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Misc& M = *reinterpret_cast<Misc*>(smem + OFF_MISC);
+  volatile int* abort = &M.abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = (int)(gridDim.x - 1 - blockIdx.x);  // heaviest tiles first
   const int h = blockIdx.y, b = blockIdx.z, kvh = h / p.g;
   const int q0 = qt * BM;
-  const int ib0 = (BN == 64) ? 2 * qt : qt;
-  const int ib1 = (BN == 64) ? 2 * qt + 1 : qt;
-  const bool valid1 = (BN == 64) ? (ib1 < p.n) : true;
-  const int q_end = min(q0 + BM, p.N);
-  const int T = (q_end + BN - 1) / BN;  // causal key tiles
+  const int ib0 = q0 / S_BLK, ib1 = (q0 + SUB) / S_BLK;  // query blocks of the two halves
+  const bool valid1 = q0 + SUB < p.N;
+  const int T = (min(q0 + BM, p.N) + BN - 1) / BN;  // causal key tiles
+  // key block of sub-block q of tile j
+  auto kblk = [](int j, int q) { return (j * BN + q * SUB) / S_BLK; };
 
   // ---- set-up
   if (threadIdx.x == 0) {
     mbar_init(&M.q_full, 1);
-    for (int s = 0; s < C::NS; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&M.k_full[s], 1);
       mbar_init(&M.k_empty[s], 1);
       mbar_init(&M.v_full[s], 1);
@@ -143,7 +139,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int j = r0[e];
       if (j >= 0 && j <= ib0) atomicOr(&M.sel[0][j >> 5], 1u << (j & 31));
     }
-    if (BN == 64 && valid1) {
+    if (ib1 != ib0 && valid1) {
       const int32_t* r1 = p.idx + (((int64_t)b * p.Hq + h) * p.n + ib1) * p.k;
       for (int e = threadIdx.x; e < p.k; e += NTHREADS) {
         const int j = r1[e];
@@ -156,11 +152,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = M.tmem_base;
   const uint32_t* sel0 = M.sel[0];
-  const uint32_t* sel1 = (BN == 64) ? M.sel[1] : M.sel[0];
+  const uint32_t* sel1 = (ib1 != ib0) ? M.sel[1] : M.sel[0];
 
-  uint8_t* sQ = smem + C::OFF_Q;
-  uint8_t* sK = smem + C::OFF_K;
-  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sQ = smem + OFF_Q;
+  uint8_t* sK = smem + OFF_K;
+  uint8_t* sV = smem + OFF_V;
 
   if (warp == 4) {
     // ================================================================ producer
@@ -168,34 +164,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      mbar_expect_tx(&M.q_full, C::Q_BYTES);
+      mbar_expect_tx(&M.q_full, Q_BYTES);
       tma_load_4d(sQ, &tmQ, &M.q_full, 0, q0, h, b);
-      tma_load_4d(sQ + C::Q_BYTES / 2, &tmQ, &M.q_full, 64, q0, h, b);
+      tma_load_4d(sQ + Q_BYTES / 2, &tmQ, &M.q_full, 64, q0, h, b);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < T; ++j) {
-        const int st = j % C::NS;
-        const uint32_t use = (uint32_t)(j / C::NS);
-        if (j >= C::NS && !mbar_wait(&M.k_empty[st], (use - 1) & 1u, abort)) break;
-        mbar_expect_tx(&M.k_full[st], C::KV_BYTES);
-        tma_load_4d(sK + st * C::KV_BYTES, &tmK, &M.k_full[st], 0, j * BN, kvh, b);
-        tma_load_4d(sK + st * C::KV_BYTES + C::KV_BYTES / 2, &tmK, &M.k_full[st], 64, j * BN, kvh, b);
+        const int st = j % NS;
+        const uint32_t use = (uint32_t)(j / NS);
+        if (j >= NS && !mbar_wait(&M.k_empty[st], (use - 1) & 1u, abort)) break;
+        mbar_expect_tx(&M.k_full[st], KV_BYTES);
+        tma_load_4d(sK + st * KV_BYTES, &tmK, &M.k_full[st], 0, j * BN, kvh, b);
+        tma_load_4d(sK + st * KV_BYTES + KV_BYTES / 2, &tmK, &M.k_full[st], 64, j * BN, kvh, b);
         k_issued = j + 1;
-        if (j >= C::NS && !mbar_wait(&M.v_empty[st], (use - 1) & 1u, abort)) break;
-        mbar_expect_tx(&M.v_full[st], C::KV_BYTES);
-        tma_load_4d(sV + st * C::KV_BYTES, &tmV, &M.v_full[st], 0, j * BN, kvh, b);
-        tma_load_4d(sV + st * C::KV_BYTES + C::KV_BYTES / 2, &tmV, &M.v_full[st], 64, j * BN, kvh, b);
+        if (j >= NS && !mbar_wait(&M.v_empty[st], (use - 1) & 1u, abort)) break;
+        mbar_expect_tx(&M.v_full[st], KV_BYTES);
+        tma_load_4d(sV + st * KV_BYTES, &tmV, &M.v_full[st], 0, j * BN, kvh, b);
+        tma_load_4d(sV + st * KV_BYTES + KV_BYTES / 2, &tmV, &M.v_full[st], 64, j * BN, kvh, b);
         v_issued = j + 1;
       }
       // Drain: every copy this thread issued must have landed before the CTA exits.
       int dummy = 0;
       mbar_wait(&M.q_full, 0, &dummy);
-      for (int j = (k_issued > C::NS ? k_issued - C::NS : 0); j < k_issued; ++j) {
+      for (int j = (k_issued > NS ? k_issued - NS : 0); j < k_issued; ++j) {
         dummy = 0;
-        mbar_wait(&M.k_full[j % C::NS], (uint32_t)(j / C::NS) & 1u, &dummy);
+        mbar_wait(&M.k_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
       }
-      for (int j = (v_issued > C::NS ? v_issued - C::NS : 0); j < v_issued; ++j) {
+      for (int j = (v_issued > NS ? v_issued - NS : 0); j < v_issued; ++j) {
         dummy = 0;
-        mbar_wait(&M.v_full[j % C::NS], (uint32_t)(j / C::NS) & 1u, &dummy);
+        mbar_wait(&M.v_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
       }
     }
   } else if (warp == 5) {
@@ -207,51 +203,56 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       auto issue_pv = [&](int jj) -> bool {
         const int sb = jj & 1;
         if (!mbar_wait(&M.p_full[sb], (uint32_t)(jj >> 1) & 1u, abort)) return false;
-        const int st = jj % C::NS;
-        if (!mbar_wait(&M.v_full[st], (uint32_t)(jj / C::NS) & 1u, abort)) return false;
+        const int st = jj % NS;
+        if (!mbar_wait(&M.v_full[st], (uint32_t)(jj / NS) & 1u, abort)) return false;
         tc_fence_after();
-        const int s0 = tile_state(jj, ib0, true, sel0);
-        const int s1 = tile_state(jj, ib1, valid1, sel1);
-        const bool mixed = (s0 != 0 && s1 != 0 && s0 != s1);
-        const int target = s0 != 0 ? s0 : s1;
-        const uint32_t v_addr = smem_u32(sV + st * C::KV_BYTES);
-        const uint32_t p_col = C::COL_S + (uint32_t)sb * BN;
-        auto pv = [&](uint32_t o_col, uint32_t pcol, bool& started) {
+        const uint32_t v_addr = smem_u32(sV + st * KV_BYTES);
+        const uint32_t s_col = COL_S + (uint32_t)sb * BN;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, BN * 128, 1024);
-            mma_ts(tmem + o_col, tmem + pcol + kk * 8, bdesc, C::IDESC_PV, (started || kk > 0) ? 1u : 0u);
+        for (int q = 0; q < 2; ++q) {
+          const int kb = kblk(jj, q);
+          const int s0 = pair_state(kb, ib0, true, sel0);
+          const int s1 = pair_state(kb, ib1, valid1, sel1);
+          if (s0 == 0 && s1 == 0) continue;
+          const bool mixed = (s0 != 0 && s1 != 0 && s0 != s1);
+          const int target = s0 != 0 ? s0 : s1;
+          auto pv = [&](uint32_t o_col, uint32_t pcol, bool& started) {
+#pragma unroll
+            for (int kk = 0; kk < SUB / 16; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128(v_addr + (q * SUB + kk * 16) * 128, KV_BYTES / 2, 1024);
+              mma_ts(tmem + o_col, tmem + pcol + kk * 8, bdesc, IDESC_PV, (started || kk > 0) ? 1u : 0u);
+            }
+            started = true;
+          };
+          const uint32_t p0 = s_col + 32 * q, p1 = s_col + 64 + 32 * q;
+          if (mixed) {
+            pv(COL_OA, p0, started_a);
+            pv(COL_OD, p1, started_d);
+          } else if (target == 1) {
+            pv(COL_OA, p0, started_a);
+          } else {
+            pv(COL_OD, p0, started_d);
           }
-          started = true;
-        };
-        if (mixed) {
-          pv(C::COL_OA, p_col, started_a);
-          pv(C::COL_OD, p_col + BN / 2, started_d);
-        } else if (target == 1) {
-          pv(C::COL_OA, p_col, started_a);
-        } else {
-          pv(C::COL_OD, p_col, started_d);
         }
         tc_commit(&M.v_empty[st]);
         tc_commit(&M.o_done);
         return true;
       };
       for (int j = 0; ok && j < T; ++j) {
-        const int st = j % C::NS;
-        if (!mbar_wait(&M.k_full[st], (uint32_t)(j / C::NS) & 1u, abort)) {
+        const int st = j % NS;
+        if (!mbar_wait(&M.k_full[st], (uint32_t)(j / NS) & 1u, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + st * C::KV_BYTES);
-        const uint32_t s_col = C::COL_S + (uint32_t)(j & 1) * BN;
+        const uint32_t k_addr = smem_u32(sK + st * KV_BYTES);
+        const uint32_t s_col = COL_S + (uint32_t)(j & 1) * BN;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off_q = (kk >> 2) * (C::Q_BYTES / 2) + (kk & 3) * 32;
-          const uint32_t off_k = (kk >> 2) * (C::KV_BYTES / 2) + (kk & 3) * 32;
-          const uint64_t adesc = smem_desc_sw128(q_addr + off_q, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(k_addr + off_k, 16, 1024);
-          mma_ss(tmem + s_col, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off_q = (kk >> 2) * (Q_BYTES / 2) + (kk & 3) * 32;
+          const uint32_t off_k = (kk >> 2) * (KV_BYTES / 2) + (kk & 3) * 32;
+          mma_ss(tmem + s_col, smem_desc_sw128(q_addr + off_q, 16, 1024), smem_desc_sw128(k_addr + off_k, 16, 1024),
+                 IDESC_QK, kk > 0 ? 1u : 0u);
         }
         tc_commit(&M.s_full[j & 1]);
         tc_commit(&M.k_empty[st]);
@@ -268,7 +269,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else {
     // ================================================================ softmax
-    const int half = (BN == 64) ? (warp >> 1) : 0;
+    const int half = warp >> 1;
+    const int ib = half ? ib1 : ib0;
+    const bool hvalid = half ? valid1 : true;
+    const uint32_t* selw = half ? sel1 : sel0;
     const int row = warp * 32 + lane;  // row within the tile == TMEM lane
     const int t = q0 + row;            // query token
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
@@ -282,97 +286,128 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
-      const int s0 = tile_state(j, ib0, true, sel0);
-      const int s1 = tile_state(j, ib1, valid1, sel1);
-      const bool mixed = (s0 != 0 && s1 != 0 && s0 != s1);
-      const int mine = half ? s1 : s0;
-      const uint32_t s_addr = lane_base + C::COL_S + (uint32_t)sb * BN;
+      int mine[2];
+      bool mixed[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int kb = kblk(j, q);
+        mine[q] = pair_state(kb, ib, hvalid, selw);
+        const int o0 = pair_state(kb, ib0, true, sel0);
+        const int o1 = pair_state(kb, ib1, valid1, sel1);
+        mixed[q] = (o0 != 0 && o1 != 0 && o0 != o1);
+      }
+      const uint32_t s_addr = lane_base + COL_S + (uint32_t)sb * BN;
       uint32_t pk[BN / 2];
-      if (mine == 0) {
+      if (mine[0] == 0 && mine[1] == 0) {
 #pragma unroll
         for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
       } else {
-        float x[BN];
+        float x[BN];  // raw S = q.k; the scale is folded into the exponent
 #pragma unroll
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(s_addr + c0, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(r[c]) * p.c;
+          for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(r[c]);
         }
-        // causal mask inside the diagonal tile
         const int u0 = j * BN;
-        if (u0 + BN - 1 > t) {
+        if (u0 + BN - 1 > t) {  // causal mask inside the diagonal tile
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (u0 + c > t) x[c] = kNegInf;
         }
-        float mx = kNegInf;
+        float mxq[2];
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, x[c]);
-        const int X = mine - 1;  // 0 = A, 1 = D
-        const float m_old = m2[X];
-        const bool need = (m_old != kNegInf) && (mx > m_old + kRescaleThreshold);
-        if (__any_sync(0xffffffffu, need)) {
-          // O_X must hold every earlier PV before it is rescaled.
-          if (!mbar_wait(&M.o_done, (uint32_t)(j - 1) & 1u, abort)) {
-            ok = false;
+        for (int q = 0; q < 2; ++q) {
+          float a0 = kNegInf, a1 = kNegInf, a2 = kNegInf, a3 = kNegInf;
+#pragma unroll
+          for (int c = q * SUB; c < (q + 1) * SUB; c += 4) {
+            a0 = fmaxf(a0, x[c]);
+            a1 = fmaxf(a1, x[c + 1]);
+            a2 = fmaxf(a2, x[c + 2]);
+            a3 = fmaxf(a3, x[c + 3]);
           }
-          if (__any_sync(0xffffffffu, !ok)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const float f = need ? ex2(m_old - mx) : 1.0f;
-          const uint32_t o_addr = lane_base + (X == 0 ? C::COL_OA : C::COL_OD);
+          mxq[q] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * p.c;  // scale > 0
+        }
+        // per-set tile max, rescale when it jumps past the threshold
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          float mx = kNegInf;
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+            if (mine[q] == X + 1) mx = fmaxf(mx, mxq[q]);
+          const float m_old = m2[X];
+          const bool need = (m_old != kNegInf) && (mx > m_old + kRescaleThreshold);
+          if (__any_sync(0xffffffffu, need)) {
+            // O_X must hold every earlier PV before it is rescaled.
+            if (j >= 1 && !mbar_wait(&M.o_done, (uint32_t)(j - 1) & 1u, abort)) ok = false;
+            if (__any_sync(0xffffffffu, !ok)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const float f = need ? ex2(m_old - mx) : 1.0f;
+            const uint32_t o_addr = lane_base + (X == 0 ? COL_OA : COL_OD);
 #pragma unroll 1
-          for (int c0 = 0; c0 < HD; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(o_addr + c0, r);
-            tmem_wait_ld();
+            for (int c0 = 0; c0 < HD; c0 += 32) {
+              uint32_t r[32];
+              tmem_ld32(o_addr + c0, r);
+              tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
-            tmem_st32(o_addr + c0, r);
+              for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
+              tmem_st32(o_addr + c0, r);
+            }
+            tmem_wait_st();
+            if (need) {
+              l[X] *= f;
+              m2[X] = mx;
+            }
           }
-          tmem_wait_st();
-          if (need) {
-            l[X] *= f;
-            m2[X] = mx;
-          }
+          if (m2[X] == kNegInf) m2[X] = mx;
         }
-        if (m2[X] == kNegInf) m2[X] = mx;
-        const float m = m2[X];
-        float sum = 0.f;
+        if (!ok) break;
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float e0 = ex2(x[c] - m);
-          const float e1 = ex2(x[c + 1] - m);
-          sum += e0 + e1;
-          pk[c / 2] = pack_bf16(e0, e1);
+        for (int q = 0; q < 2; ++q) {
+          if (mine[q] == 0) {
+#pragma unroll
+            for (int c = 0; c < SUB / 2; ++c) pk[q * SUB / 2 + c] = 0u;
+            continue;
+          }
+          const int X = mine[q] - 1;
+          const float nm = -m2[X];
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int c = q * SUB; c < (q + 1) * SUB; c += 2) {
+            const float e0 = ex2(fmaf(x[c], p.c, nm));
+            const float e1 = ex2(fmaf(x[c + 1], p.c, nm));
+            s0 += e0;
+            s1 += e1;
+            pk[c / 2] = pack_bf16(e0, e1);
+          }
+          l[X] += s0 + s1;
         }
-        l[X] += sum;
       }
-      // Write P where the MMA warp will read it.
-      const uint32_t p0 = s_addr, p1 = s_addr + BN / 2;
-      if (mixed && mine == 2) {
-        uint32_t z[32];
+      // Write P where the MMA warp will read it: sub-block q's P at columns
+      // [32q, 32q+32) of the S buffer; for a mixed sub-block the dropped
+      // half's rows use [64+32q, 64+32q+32) instead and write zeros to the first.
+      uint32_t z[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) z[c] = 0u;
+      for (int c = 0; c < 32; ++c) z[c] = 0u;
 #pragma unroll
-        for (int c0 = 0; c0 < BN / 2; c0 += 32) {
-          tmem_st32(p0 + c0, z);
-          tmem_st32(p1 + c0, *reinterpret_cast<uint32_t(*)[32]>(&pk[c0]));
-        }
-      } else {
-#pragma unroll
-        for (int c0 = 0; c0 < BN / 2; c0 += 32) tmem_st32(p0 + c0, *reinterpret_cast<uint32_t(*)[32]>(&pk[c0]));
-        if (mixed) {
-          uint32_t z[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) z[c] = 0u;
-#pragma unroll
-          for (int c0 = 0; c0 < BN / 2; c0 += 32) tmem_st32(p1 + c0, z);
+      for (int q = 0; q < 2; ++q) {
+        const uint32_t p0 = s_addr + 32 * q, p1 = s_addr + 64 + 32 * q;
+        const uint32_t(&blk)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * q]);
+        if (mixed[q]) {
+          if (mine[q] == 1) {
+            tmem_st32(p0, blk);
+            tmem_st32(p1, z);
+          } else {
+            tmem_st32(p0, z);
+            tmem_st32(p1, blk);
+          }
+        } else {
+          tmem_st32(p0, blk);
         }
       }
       tmem_wait_st();
@@ -396,8 +431,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < HD; c0 += 32) {
         uint32_t ra[32], rd[32];
-        tmem_ld32(lane_base + C::COL_OA + c0, ra);
-        tmem_ld32(lane_base + C::COL_OD + c0, rd);
+        tmem_ld32(lane_base + COL_OA + c0, ra);
+        tmem_ld32(lane_base + COL_OD + c0, rd);
         tmem_wait_ld();
         if (store) {
           uint32_t of[16], os[16];
@@ -444,9 +479,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <int BN>
-cudaError_t launch_bn(const Dims& D, const FwdArgs& a, int32_t* status, cudaStream_t st) {
-  using C = Cfg<BN>;
+template <int S_BLK>
+cudaError_t launch_blk(const Dims& D, const FwdArgs& a, int32_t* status, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_tma_map_bf16(&mq, a.q, D.B, D.Hq, D.N, BM) || !make_tma_map_bf16(&mk, a.k, D.B, D.Hkv, D.N, BN) ||
       !make_tma_map_bf16(&mv, a.v, D.B, D.Hkv, D.N, BN))
@@ -465,18 +499,17 @@ cudaError_t launch_bn(const Dims& D, const FwdArgs& a, int32_t* status, cudaStre
   p.n = D.n;
   p.k = D.k;
   p.c = D.scale * 1.4426950408889634f;
-  auto kern = fwd_tc_kernel<BN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  auto kern = fwd_tc_kernel<S_BLK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((D.N + BM - 1) / BM, D.Hq, D.B);
-  kern<<<grid, NTHREADS, C::SMEM, st>>>(mq, mk, mv, p);
+  kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(mq, mk, mv, p);
   count_launches(1);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-// ---------------------------------------------------------------- host side
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -513,7 +546,7 @@ bool fwd_tc_supported(const Dims& D) {
 
 cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st) {
   if (!fwd_tc_supported(D)) return cudaErrorNotSupported;
-  return D.s == 64 ? launch_bn<64>(D, a, dev_status, st) : launch_bn<128>(D, a, dev_status, st);
+  return D.s == 64 ? launch_blk<64>(D, a, dev_status, st) : launch_blk<128>(D, a, dev_status, st);
 }
 
 }  // namespace ssa

@@ -26,8 +26,7 @@ ssa_status_t check_dims(const ssa_dims_t* in, Dims* out, bool* empty) {
   D.s = in->block; D.topk = in->topk; D.scale = in->scale; D.dtype = in->dtype;
   if (D.B < 0 || D.Hq < 0 || D.N < 0 || D.Hkv < 1 || D.topk < 1) return SSA_ERR_INVALID_ARG;
   if (D.dtype != SSA_F32 && D.dtype != SSA_BF16) return SSA_ERR_INVALID_ARG;
-  if (!(D.scale == D.scale) || D.scale == __builtin_huge_valf() || D.scale == -__builtin_huge_valf())
-    return SSA_ERR_INVALID_ARG;
+  if (!(D.scale > 0.f) || D.scale == __builtin_huge_valf()) return SSA_ERR_INVALID_ARG;
   if (D.Hq % D.Hkv != 0) return SSA_ERR_INVALID_ARG;
   if (D.s != 64 && D.s != 128) return SSA_ERR_UNSUPPORTED;
   if (D.d != 64 && D.d != 128) return SSA_ERR_UNSUPPORTED;

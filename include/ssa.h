@@ -15,7 +15,8 @@
  * Notation: B batch, Hq query heads, Hkv key/value heads (g = Hq/Hkv query
  * heads share one kv head; query head h reads kv head h/g), N tokens, d head
  * dim, s = block, n = N/s blocks, k = topk budget in blocks counting the
- * diagonal block, scale = attention scale (1/sqrt(d) in the paper's models).
+ * diagonal block, scale = attention scale (1/sqrt(d) in the paper's models;
+ * any finite positive value is accepted).
  * Query token t lies in block i = t/s.  Sel(i) is the selected block set of
  * query block i; A_t = {u <= t : u/s in Sel(i)} is attended by both streams,
  * D_t = {u <= t : u/s not in Sel(i)} only by the full stream.

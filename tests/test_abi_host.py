@@ -58,6 +58,9 @@ def _tensor(ptr=16, sb=4096 * 128, sh=4096 * 128, sn=128):
     ("B", -1, api.SSA_ERR_INVALID_ARG),
     ("dtype", 7, api.SSA_ERR_INVALID_ARG),
     ("scale", float("nan"), api.SSA_ERR_INVALID_ARG),
+    ("scale", 0.0, api.SSA_ERR_INVALID_ARG),
+    ("scale", -0.125, api.SSA_ERR_INVALID_ARG),
+    ("scale", float("inf"), api.SSA_ERR_INVALID_ARG),
 ])
 def test_bad_dims_rejected_on_host(lib, field, value, code):
     d = api.make_dims(1, 4, 2, 1024, 128, 64, 4)
