@@ -44,7 +44,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) bwd_pre_tc_kernel(TensorRef hf_t, TensorRef hs_t, TensorRef gf_t,
                                                         TensorRef gs_t, int Hq, int N, float c2,
                                                         __nv_bfloat16* dhf, __nv_bfloat16* dhs, float* Df,
-                                                        float* Ds, float* partials) {
+                                                        float* Ds, float* partials, const float* lse_full,
+                                                        const float* lse_sel, float4* scal) {
   constexpr int PER = HD / 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t row = (int64_t)blockIdx.x * 8 + w;
@@ -80,6 +81,10 @@ __global__ void __launch_bounds__(256) bwd_pre_tc_kernel(TensorRef hf_t, TensorR
     Df[row] = df;
     Ds[row] = ds;
     part[w] = sq;
+    // {lse_full, lse_sel} in base 2 (an empty selected set maps to +inf, so
+    // 2^(x - lse) is 0 there), then D_f, D_s: one 16-byte load per query.
+    const float ls = lse_sel[row];
+    scal[row] = make_float4(lse_full[row] * kLog2e, ls == kNegInf ? __builtin_huge_valf() : ls * kLog2e, df, ds);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -97,6 +102,7 @@ struct BwdTcParams {
   const float* Df;          // [B,Hq,N]
   const float* Ds;
   const uint32_t* mask;     // [B,Hq,n,words]
+  const float4* scal;       // [B,Hq,N]: {lse2_full, lse2_sel, D_f, D_s}
   int words;
   int32_t* status;
   int Hq, g, N, n, s;
@@ -126,11 +132,12 @@ constexpr int OFF_Q = 0, OFF_DHF = TILE_A, OFF_DHS = 2 * TILE_A;
 constexpr int OFF_K = 3 * TILE_A;
 constexpr int OFF_V = OFF_K + NS * TILE_K;
 constexpr int OFF_MISC = OFF_V + NS * TILE_K;
-constexpr int SMEM = OFF_MISC + 1024 + 1024;
+constexpr int SMEM = OFF_MISC + 1024 + 4096 + 1024;
 constexpr uint32_t COL_DQ = 0, COL_S = 128, COL_DPF = 256, COL_DPS = 384;
 constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BK, false, false);
 constexpr uint32_t IDESC_DQ = idesc_bf16_f32(BM, HD, false, true);
 
+constexpr int MAX_TILES = 4096;  // N / 64 for n <= 2048 and block <= 128
 struct Misc {
   uint64_t a_full;
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
@@ -138,6 +145,7 @@ struct Misc {
   uint64_t done, drain;
   uint32_t tmem_base;
   int abort;
+  uint8_t state[MAX_TILES];  // per key tile: half-0 state | half-1 state << 2
 };
 }  // namespace dq
 
@@ -182,6 +190,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_alloc(&M.tmem_base, 512);
     tmem_relinquish();
   }
+  // (half, key block) states of every key tile, read once from the mask
+  for (int j = threadIdx.x; j < T; j += NTHREADS) {
+    const int jb = (j * BK) / p.s;
+    M.state[j] = (uint8_t)(pair_state(p, b, h, ib0, true, jb) | (pair_state(p, b, h, ib1, valid1, jb) << 2));
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -191,8 +204,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sDhs = smem + OFF_DHS;
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
-  // key tile j covers keys [64j, 64j+64), key block j*64/s
-  auto kblock = [&](int j) { return (j * BK) / p.s; };
 
   if (warp == 4) {
     if (lane == 0) {
@@ -259,8 +270,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           break;
         }
         tc_fence_after();
-        const int jb = kblock(j);
-        const bool any_sel = pair_state(p, b, h, ib0, true, jb) == 1 || pair_state(p, b, h, ib1, valid1, jb) == 1;
+        const int stj = M.state[j];
+        const bool any_sel = (stj & 3) == 1 || (stj >> 2) == 1;
         const uint32_t k_addr = smem_u32(sK + st * TILE_K), v_addr = smem_u32(sV + st * TILE_K);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
@@ -289,15 +300,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int row = warp * 32 + lane;
     const int t = q0 + row;
     const int half = warp >> 1;
-    const int ib = half ? ib1 : ib0;
-    const bool qvalid = half ? valid1 : true;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const bool in_range = t < p.N;
     const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + (in_range ? t : 0);
-    const float l2f = p.lse_full[ro] * kLog2e;
-    const float l2s_raw = p.lse_sel[ro];
-    const float l2s = (l2s_raw == kNegInf) ? __builtin_huge_valf() : l2s_raw * kLog2e;
-    const float Dfv = p.Df[ro], Dsv = p.Ds[ro];
+    const float4 sc = p.scal[ro];
+    const float l2f = sc.x, l2s = sc.y, Dfv = sc.z, Dsv = sc.w;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1;
@@ -306,8 +313,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
-      const int jb = kblock(j);
-      const int mine = pair_state(p, b, h, ib, qvalid, jb);
+      const int mine = half ? (M.state[j] >> 2) : (M.state[j] & 3);
       uint32_t pk[32];
       if (mine == 0) {
 #pragma unroll
@@ -387,22 +393,27 @@ constexpr int BQ = 64;     // queries per step
 constexpr int NS = 3;
 constexpr int TILE_KV = BKEY * HD * 2;  // 32 KB: K or V
 constexpr int TILE_Q = BQ * HD * 2;     // 16 KB: Q, dh_f or dh_s step tile
-constexpr int SCAL = 4 * BQ * 4;        // lse_f, lse_s, D_f, D_s of one step (1 KB)
+constexpr int SCAL = BQ * 16;           // {lse2_f, lse2_s, D_f, D_s} of one step (1 KB)
+constexpr int MAX_STEPS = 8192;         // g * N / 64
 constexpr int STAGE = 3 * TILE_Q + SCAL;
 constexpr int OFF_K = 0, OFF_V = TILE_KV;
 constexpr int OFF_STAGE = 2 * TILE_KV;
 constexpr int OFF_MISC = OFF_STAGE + NS * STAGE;
-constexpr int SMEM = OFF_MISC + 1024 + 1024;
-constexpr uint32_t COL_DK = 0, COL_DV = 128, COL_S = 256, COL_DPF = 320, COL_DPS = 384;
+constexpr int SMEM = OFF_MISC + 1024 + MAX_STEPS + 1024;
+// TMEM: dK, dV, then two step buffers of [S^T 64 | dP_f^T 64] columns.  A step
+// with a selected pair puts dP_s^T in the other buffer's dP_f^T columns.
+constexpr uint32_t COL_DK = 0, COL_DV = 128, COL_BUF = 256, BUF_COLS = 128, OFF_DP = 64;
 constexpr uint32_t IDESC_S = idesc_bf16_f32(BKEY, BQ, false, false);
 constexpr uint32_t IDESC_ACC = idesc_bf16_f32(BKEY, HD, false, true);
 
 struct Misc {
   uint64_t kv_full;
   uint64_t full[NS], empty[NS];
-  uint64_t s_full, p_full, done, drain;
+  uint64_t s_full[2], p_full[2], done, drain;
   uint32_t tmem_base;
   int abort;
+  // per step: key-half-0 state | key-half-1 state << 2 | any selected << 4
+  uint8_t state[MAX_STEPS];
 };
 }  // namespace dkv
 
@@ -434,8 +445,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&M.full[s], 1);
       mbar_init(&M.empty[s], 1);
     }
-    mbar_init(&M.s_full, 1);
-    mbar_init(&M.p_full, 4);
+    for (int s2 = 0; s2 < 2; ++s2) {
+      mbar_init(&M.s_full[s2], 1);
+      mbar_init(&M.p_full[s2], 4);
+    }
     mbar_init(&M.done, 1);
     mbar_init(&M.drain, 1);
     M.abort = 0;
@@ -445,6 +458,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_alloc(&M.tmem_base, 512);
     tmem_relinquish();
   }
+  // Steps walk (head hh, query tile qt) with qt fastest.  Their states are
+  // read once from the mask into shared memory.
+  for (int it = threadIdx.x; it < steps; it += NTHREADS) {
+    const int h = kvh * p.g + it / steps_per_head;
+    const int i = ((qt0 + it % steps_per_head) * BQ) / p.s;
+    const int s0 = pair_state(p, b, h, i, true, kb0);
+    const int s1 = kvalid1 ? pair_state(p, b, h, i, true, kb1) : 0;
+    M.state[it] = (uint8_t)(s0 | (s1 << 2) | ((s0 == 1 || s1 == 1) ? 16 : 0));
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -452,15 +474,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
   auto stage_ptr = [&](int st) { return smem + OFF_STAGE + st * STAGE; };
-
-  // step -> (head, query tile, query block)
-  auto step_head = [&](int it) { return kvh * p.g + it / steps_per_head; };
-  auto step_qt = [&](int it) { return qt0 + it % steps_per_head; };
-  auto step_anysel = [&](int it) {
-    const int h = step_head(it), qt = step_qt(it);
-    const int i = (qt * BQ) / p.s;
-    return pair_state(p, b, h, i, true, kb0) == 1 || (kvalid1 && pair_state(p, b, h, i, true, kb1) == 1);
-  };
 
   if (warp == 4) {
     if (lane == 0) {
@@ -473,12 +486,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tma_load_4d(sV, &tmV, &M.kv_full, 0, u0, kvh, b);
       tma_load_4d(sV + TILE_KV / 2, &tmV, &M.kv_full, 64, u0, kvh, b);
       int issued = 0;
+      int h = kvh * p.g, qt = qt0;
       for (int it = 0; it < steps; ++it) {
         const int st = it % NS;
         const uint32_t use = (uint32_t)(it / NS);
         if (it >= NS && !mbar_wait(&M.empty[st], (use - 1) & 1u, abort)) break;
-        const int h = step_head(it), qt = step_qt(it), t0 = qt * BQ;
-        const bool any = step_anysel(it);
+        const int t0 = qt * BQ;
+        const bool any = (M.state[it] & 16) != 0;
         uint8_t* sp = stage_ptr(st);
         mbar_expect_tx(&M.full[st], (any ? 3 : 2) * TILE_Q + SCAL);
         tma_load_4d(sp, &tmQ, &M.full[st], 0, t0, h, b);
@@ -490,12 +504,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_4d(sp + 2 * TILE_Q + TILE_Q / 2, &tmDhs, &M.full[st], 64, t0, h, b);
         }
         const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + t0;
-        float* sc = reinterpret_cast<float*>(sp + 3 * TILE_Q);
-        bulk_load(sc, p.lse_full + ro, BQ * 4, &M.full[st]);
-        bulk_load(sc + BQ, p.lse_sel + ro, BQ * 4, &M.full[st]);
-        bulk_load(sc + 2 * BQ, p.Df + ro, BQ * 4, &M.full[st]);
-        bulk_load(sc + 3 * BQ, p.Ds + ro, BQ * 4, &M.full[st]);
+        bulk_load(sp + 3 * TILE_Q, p.scal + ro, SCAL, &M.full[st]);
         issued = it + 1;
+        if (++qt == qt0 + steps_per_head) {
+          qt = qt0;
+          ++h;
+        }
       }
       int dummy = 0;
       mbar_wait(&M.kv_full, 0, &dummy);
@@ -509,48 +523,78 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t ak = smem_u32(sK), av = smem_u32(sV);
       bool ok = mbar_wait(&M.kv_full, 0, abort);
       bool started = false;
-      for (int it = 0; ok && it < steps; ++it) {
-        const int st = it % NS;
-        if (!mbar_wait(&M.full[st], (uint32_t)(it / NS) & 1u, abort)) {
-          ok = false;
-          break;
-        }
+      // dV += P^T dh_f (+ P_s^T dh_s), dK += dS^T Q for step jt (buffer jt & 1).
+      auto accumulate = [&](int jt) -> bool {
+        if (!mbar_wait(&M.p_full[jt & 1], (uint32_t)(jt >> 1) & 1u, abort)) return false;
         tc_fence_after();
-        const bool any = step_anysel(it);
+        const int st = jt % NS;
         const uint32_t sq = smem_u32(stage_ptr(st));
         const uint32_t sf = sq + TILE_Q, ss = sq + 2 * TILE_Q;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * (TILE_KV / 2) + (kk & 3) * 32;
-          const uint32_t offb = (kk >> 2) * (TILE_Q / 2) + (kk & 3) * 32;
-          const uint64_t kdesc = smem_desc_sw128(ak + offa, 16, 1024);
-          const uint64_t vdesc = smem_desc_sw128(av + offa, 16, 1024);
-          mma_ss(tmem + COL_S, kdesc, smem_desc_sw128(sq + offb, 16, 1024), IDESC_S, kk > 0);
-          mma_ss(tmem + COL_DPF, vdesc, smem_desc_sw128(sf + offb, 16, 1024), IDESC_S, kk > 0);
-          if (any) mma_ss(tmem + COL_DPS, vdesc, smem_desc_sw128(ss + offb, 16, 1024), IDESC_S, kk > 0);
-        }
-        tc_commit(&M.s_full);
-        if (!mbar_wait(&M.p_full, (uint32_t)it & 1u, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        const uint32_t buf = COL_BUF + (uint32_t)(jt & 1) * BUF_COLS;
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint32_t off = kk * 16 * 128;
           const uint32_t acc = (started || kk > 0) ? 1u : 0u;
-          mma_ts(tmem + COL_DV, tmem + COL_S + kk * 8, smem_desc_sw128(sf + off, TILE_Q / 2, 1024), IDESC_ACC, acc);
-          mma_ts(tmem + COL_DK, tmem + COL_DPF + kk * 8, smem_desc_sw128(sq + off, TILE_Q / 2, 1024), IDESC_ACC, acc);
+          mma_ts(tmem + COL_DV, tmem + buf + kk * 8, smem_desc_sw128(sf + off, TILE_Q / 2, 1024), IDESC_ACC, acc);
+          mma_ts(tmem + COL_DK, tmem + buf + OFF_DP + kk * 8, smem_desc_sw128(sq + off, TILE_Q / 2, 1024), IDESC_ACC,
+                 acc);
         }
         started = true;
-        if (any) {
+        if (M.state[jt] & 16) {
 #pragma unroll
           for (int kk = 0; kk < BQ / 16; ++kk)
-            mma_ts(tmem + COL_DV, tmem + COL_S + 32 + kk * 8, smem_desc_sw128(ss + kk * 16 * 128, TILE_Q / 2, 1024),
+            mma_ts(tmem + COL_DV, tmem + buf + 32 + kk * 8, smem_desc_sw128(ss + kk * 16 * 128, TILE_Q / 2, 1024),
                    IDESC_ACC, 1u);
         }
         tc_commit(&M.empty[st]);
+        return true;
+      };
+      for (int it = 0; ok && it < steps; ++it) {
+        const int st = it % NS, b2 = it & 1;
+        if (!mbar_wait(&M.full[st], (uint32_t)(it / NS) & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        // A selected previous step left its dP_s^T in this step's buffer:
+        // its softmax must be done with it first.
+        if (it >= 1 && (M.state[it - 1] & 16) &&
+            !mbar_wait(&M.p_full[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool sel = (M.state[it] & 16) != 0;
+        const uint32_t sq = smem_u32(stage_ptr(st));
+        const uint32_t sf = sq + TILE_Q, ss = sq + 2 * TILE_Q;
+        const uint32_t buf = COL_BUF + (uint32_t)b2 * BUF_COLS;
+        const uint32_t other = COL_BUF + (uint32_t)(b2 ^ 1) * BUF_COLS;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t offa = (kk >> 2) * (TILE_KV / 2) + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * (TILE_Q / 2) + (kk & 3) * 32;
+          mma_ss(tmem + buf, smem_desc_sw128(ak + offa, 16, 1024), smem_desc_sw128(sq + offb, 16, 1024), IDESC_S,
+                 kk > 0);
+          mma_ss(tmem + buf + OFF_DP, smem_desc_sw128(av + offa, 16, 1024), smem_desc_sw128(sf + offb, 16, 1024),
+                 IDESC_S, kk > 0);
+        }
+        if (!sel) tc_commit(&M.s_full[b2]);
+        if (it >= 1 && !accumulate(it - 1)) {
+          ok = false;
+          break;
+        }
+        if (sel) {
+          // after dK of the previous step has read its dS^T from `other`
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t offa = (kk >> 2) * (TILE_KV / 2) + (kk & 3) * 32;
+            const uint32_t offb = (kk >> 2) * (TILE_Q / 2) + (kk & 3) * 32;
+            mma_ss(tmem + other + OFF_DP, smem_desc_sw128(av + offa, 16, 1024), smem_desc_sw128(ss + offb, 16, 1024),
+                   IDESC_S, kk > 0);
+          }
+          tc_commit(&M.s_full[b2]);
+        }
       }
+      if (ok && steps >= 1) accumulate(steps - 1);
       tc_commit(&M.done);
       tc_commit(&M.drain);
       int dummy = 0;
@@ -559,27 +603,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     const int row = warp * 32 + lane;  // key within the tile
     const int u = u0 + row;
-    const int kb = (warp >> 1) ? kb1 : kb0;
-    const bool kvalid = (warp >> 1) ? kvalid1 : true;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    int qt = qt0;
     bool ok = true;
     for (int it = 0; it < steps; ++it) {
-      if (!mbar_wait(&M.s_full, (uint32_t)it & 1u, abort)) {
+      const int b2 = it & 1;
+      if (!mbar_wait(&M.s_full[b2], (uint32_t)(it >> 1) & 1u, abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int st = it % NS;
+      const uint32_t COL_S = COL_BUF + (uint32_t)b2 * BUF_COLS;
+      const uint32_t COL_DPF = COL_S + OFF_DP;
+      const uint32_t COL_DPS = COL_BUF + (uint32_t)(b2 ^ 1) * BUF_COLS + OFF_DP;
       // the per-query scalars of this stage arrived with the stage's copies
       if (!mbar_wait(&M.full[st], (uint32_t)(it / NS) & 1u, abort)) {
         ok = false;
         break;
       }
-      const int h = step_head(it), qt = step_qt(it), t0 = qt * BQ;
-      const int i = t0 / p.s;
-      const int mine = kvalid ? pair_state(p, b, h, i, true, kb) : 0;
-      const bool any = step_anysel(it);
-      const float* sc = reinterpret_cast<const float*>(stage_ptr(st) + 3 * TILE_Q);
+      const int t0 = qt * BQ;
+      const int stt = M.state[it];
+      const int mine = (warp >> 1) ? ((stt >> 2) & 3) : (stt & 3);
+      const bool any = (stt & 16) != 0;
+      if (++qt == qt0 + steps_per_head) qt = qt0;
+      const float4* sc = reinterpret_cast<const float4*>(stage_ptr(st) + 3 * TILE_Q);
       // P^T -> S cols [0,32); P_s^T -> S cols [32,64); dS^T -> dP_f cols [0,32).
       if (mine == 0) {
         uint32_t z[32];
@@ -606,15 +654,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int q = c0 + c + e;
-              const float x = __uint_as_float(rs[q]) * p.c;
+              const float4 v4 = sc[q];  // lse2_f, lse2_s, D_f, D_s of query t0 + q
+              const float x = __uint_as_float(rs[q]);
               const bool causal = u <= t0 + q;
-              pf[e] = causal ? ex2(x - sc[q] * kLog2e) : 0.f;
-              dsv[e] = pf[e] * (__uint_as_float(rf[c + e]) - sc[2 * BQ + q]);
+              pf[e] = causal ? ex2(fmaf(x, p.c, -v4.x)) : 0.f;
+              dsv[e] = pf[e] * (__uint_as_float(rf[c + e]) - v4.z);
               ps[e] = 0.f;
               if (mine == 1) {
-                const float ls = sc[BQ + q];
-                ps[e] = (causal && ls != kNegInf) ? ex2(x - ls * kLog2e) : 0.f;
-                dsv[e] = fmaf(ps[e], __uint_as_float(rp[c + e]) - sc[3 * BQ + q], dsv[e]);
+                ps[e] = causal ? ex2(fmaf(x, p.c, -v4.y)) : 0.f;
+                dsv[e] = fmaf(ps[e], __uint_as_float(rp[c + e]) - v4.w, dsv[e]);
               }
             }
             pf_pk[c / 2] = pack_bf16(pf[0], pf[1]);
@@ -629,7 +677,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&M.p_full);
+      if (lane == 0) mbar_arrive(&M.p_full[b2]);
     }
     if (ok && mbar_wait(&M.done, 0, abort)) {
       tc_fence_after();
@@ -673,7 +721,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace
 
 bool bwd_tc_supported(const Dims& D) {
-  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048;
+  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048 &&
+         (int64_t)D.g * (D.N / dkv::BQ) <= dkv::MAX_STEPS && D.N / dq::BK <= dq::MAX_TILES;
 }
 
 cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cudaStream_t st) {
@@ -685,8 +734,12 @@ cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cuda
   const double Mtot = (double)D.B * D.Hq * D.N * D.d;
   const float c2 = (float)(2.0 * (double)a.alpha / Mtot);
   const unsigned pre_blocks = (unsigned)sqdiff_partial_count(D);
+  // The packed per-query scalars go in the upper half of the fp32 dh_f
+  // region (the bf16 dh_f uses only the lower half).
+  const int64_t rows = (int64_t)D.B * D.Hq * D.N;
+  float4* scal = reinterpret_cast<float4*>(reinterpret_cast<char*>(a.dhf) + rows * D.d * 2);
   bwd_pre_tc_kernel<__nv_bfloat16><<<pre_blocks, 256, 0, st>>>(a.hf, a.hs, a.gf, a.gs, D.Hq, D.N, c2, dhf, dhs,
-                                                                a.Df, a.Dc, a.partials);
+                                                                a.Df, a.Dc, a.partials, a.lse_full, a.lse_sel, scal);
   count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -713,6 +766,7 @@ cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cuda
   p.Df = a.Df;
   p.Ds = a.Dc;
   p.mask = a.mask;
+  p.scal = scal;
   p.words = a.words;
   p.status = status;
   p.Hq = D.Hq;

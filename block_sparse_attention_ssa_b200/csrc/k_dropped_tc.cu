@@ -13,8 +13,10 @@
 // keep their relative precision.
 //
 // CTA = one 128-row query tile, 192 threads: warps 0-3 read S rows from TMEM
-// (one row per thread), warp 4 streams K tiles by TMA, warp 5 issues the
-// QK^T MMAs into a TMEM double buffer (256 columns).
+// (one row per thread), warp 4 streams 128-key K tiles by TMA, warp 5 issues
+// the QK^T MMAs into a TMEM double buffer (256 columns).  A tile is two 64-key
+// sub-blocks; each (64-row query half, sub-block) pair is "none", selected or
+// dropped, as in the fused forward.
 #include "ssa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -24,12 +26,13 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int SUB = 64;
 constexpr int HD = 128;
 constexpr int NTHREADS = 192;
 
-template <int BN>
 struct DCfg {
-  static constexpr int NS = (BN == 64) ? 4 : 2;
+  static constexpr int NS = 2;
   static constexpr int Q_BYTES = BM * HD * 2;
   static constexpr int K_BYTES = BN * HD * 2;
   static constexpr int OFF_K = Q_BYTES;
@@ -57,15 +60,15 @@ struct DParams {
   float c;  // scale * log2(e)
 };
 
-__device__ __forceinline__ int dstate(int j, int ib, bool valid, const uint32_t* selw) {
-  if (!valid || j > ib) return 0;
-  return ((selw[j >> 5] >> (j & 31)) & 1u) ? 1 : 2;
+__device__ __forceinline__ int dstate(int kb, int ib, bool valid, const uint32_t* selw) {
+  if (!valid || kb > ib) return 0;
+  return ((selw[kb >> 5] >> (kb & 31)) & 1u) ? 1 : 2;
 }
 
-template <int BN, bool GIVEN>
+template <int S_BLK, bool GIVEN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     dropped_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, DParams p) {
-  using C = DCfg<BN>;
+  using C = DCfg;
   if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -75,10 +78,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int qt = (int)(gridDim.x - 1 - blockIdx.x);
   const int h = blockIdx.y, b = blockIdx.z, kvh = h / p.g;
   const int q0 = qt * BM;
-  const int ib0 = (BN == 64) ? 2 * qt : qt;
-  const int ib1 = (BN == 64) ? 2 * qt + 1 : qt;
-  const bool valid1 = (BN == 64) ? (ib1 < p.n) : true;
+  const int ib0 = q0 / S_BLK, ib1 = (q0 + SUB) / S_BLK;
+  const bool valid1 = q0 + SUB < p.N;
   const int T = (min(q0 + BM, p.N) + BN - 1) / BN;
+  auto kblk = [](int j, int q) { return (j * BN + q * SUB) / S_BLK; };
 
   if (threadIdx.x == 0) {
     mbar_init(&M.q_full, 1);
@@ -106,7 +109,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int j = r0[e];
       if (j >= 0 && j <= ib0) atomicOr(&M.sel[0][j >> 5], 1u << (j & 31));
     }
-    if (BN == 64 && valid1) {
+    if (ib1 != ib0 && valid1) {
       const int32_t* r1 = p.idx + (((int64_t)b * p.Hq + h) * p.n + ib1) * p.k;
       for (int e = threadIdx.x; e < p.k; e += NTHREADS) {
         const int j = r1[e];
@@ -119,11 +122,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = M.tmem_base;
   const uint32_t* sel0 = M.sel[0];
-  const uint32_t* sel1 = (BN == 64) ? M.sel[1] : M.sel[0];
+  const uint32_t* sel1 = (ib1 != ib0) ? M.sel[1] : M.sel[0];
   // With lse_full given only tiles holding a dropped pair do any work.
   auto useful = [&](int j) {
     if (!GIVEN) return true;
-    return dstate(j, ib0, true, sel0) == 2 || dstate(j, ib1, valid1, sel1) == 2;
+    bool any = false;
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      any |= dstate(kblk(j, q), ib0, true, sel0) == 2 || dstate(kblk(j, q), ib1, valid1, sel1) == 2;
+    return any;
   };
   uint8_t* sQ = smem;
   uint8_t* sK = smem + C::OFF_K;
@@ -179,7 +186,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_wait(&M.drain, 0, &dummy);
     }
   } else {
-    const int half = (BN == 64) ? (warp >> 1) : 0;
+    const int half = warp >> 1;
+    const int ib = half ? ib1 : ib0;
+    const bool hvalid = half ? valid1 : true;
+    const uint32_t* selw = half ? sel1 : sel0;
     const int t = q0 + warp * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const int64_t o = ((int64_t)b * p.Hq + h) * p.N + (t < p.N ? t : 0);
@@ -196,62 +206,50 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
-      const int s0 = dstate(j, ib0, true, sel0);
-      const int s1 = dstate(j, ib1, valid1, sel1);
-      const int mine = half ? s1 : s0;
-      const uint32_t sa = lane_base + (uint32_t)sb * BN;
-      const int u0 = j * BN;
-      const bool diag = u0 + BN - 1 > t;
-      if (GIVEN) {
-        if (mine == 2) {
 #pragma unroll
-          for (int c0 = 0; c0 < BN; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(sa + c0, r);
-            tmem_wait_ld();
-            float acc0 = 0.f, acc1 = 0.f;
+      for (int q = 0; q < 2; ++q) {
+        const int mine = dstate(kblk(j, q), ib, hvalid, selw);
+        if (mine == 0 || (GIVEN && mine != 2)) continue;
+        const uint32_t sa = lane_base + (uint32_t)sb * BN + q * SUB;
+        const int u0 = j * BN + q * SUB;
+        const bool diag = u0 + SUB - 1 > t;
+        uint32_t r[64];
+        tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+        if (diag) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const float e0 = (!diag || u0 + c0 + c <= t) ? ex2(fmaf(__uint_as_float(r[c]), p.c, -lse2_in)) : 0.f;
-              const float e1 =
-                  (!diag || u0 + c0 + c + 1 <= t) ? ex2(fmaf(__uint_as_float(r[c + 1]), p.c, -lse2_in)) : 0.f;
-              acc0 += e0;
-              acc1 += e1;
-            }
-            dsum += acc0 + acc1;
-          }
+          for (int c = 0; c < SUB; ++c)
+            if (u0 + c > t) r[c] = __float_as_uint(kNegInf);
         }
-      } else if (mine != 0) {
-        const int X = mine - 1;
-        float mx = kNegInf;
+        if (GIVEN) {
+          float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(sa + c0, r);
-          tmem_wait_ld();
-          float a0 = kNegInf, a1 = kNegInf;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            if (!diag || u0 + c0 + c <= t) a0 = fmaxf(a0, __uint_as_float(r[c]));
-            if (!diag || u0 + c0 + c + 1 <= t) a1 = fmaxf(a1, __uint_as_float(r[c + 1]));
+          for (int c = 0; c < SUB; c += 2) {
+            acc0 += ex2(fmaf(__uint_as_float(r[c]), p.c, -lse2_in));
+            acc1 += ex2(fmaf(__uint_as_float(r[c + 1]), p.c, -lse2_in));
           }
-          mx = fmaxf(mx, fmaxf(a0, a1));
-        }
-        const float mnew = fmaxf(m2[X], mx * p.c);
-        float acc0 = 0.f, acc1 = 0.f;
+          dsum += acc0 + acc1;
+        } else {
+          const int X = mine - 1;
+          float a0 = kNegInf, a1 = kNegInf, a2 = kNegInf, a3 = kNegInf;
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(sa + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            acc0 += (!diag || u0 + c0 + c <= t) ? ex2(fmaf(__uint_as_float(r[c]), p.c, -mnew)) : 0.f;
-            acc1 += (!diag || u0 + c0 + c + 1 <= t) ? ex2(fmaf(__uint_as_float(r[c + 1]), p.c, -mnew)) : 0.f;
+          for (int c = 0; c < SUB; c += 4) {
+            a0 = fmaxf(a0, __uint_as_float(r[c]));
+            a1 = fmaxf(a1, __uint_as_float(r[c + 1]));
+            a2 = fmaxf(a2, __uint_as_float(r[c + 2]));
+            a3 = fmaxf(a3, __uint_as_float(r[c + 3]));
           }
+          const float mnew = fmaxf(m2[X], fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * p.c);
+          float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+          for (int c = 0; c < SUB; c += 2) {
+            acc0 += ex2(fmaf(__uint_as_float(r[c]), p.c, -mnew));
+            acc1 += ex2(fmaf(__uint_as_float(r[c + 1]), p.c, -mnew));
+          }
+          l[X] = (m2[X] == kNegInf ? 0.f : l[X] * ex2(m2[X] - mnew)) + acc0 + acc1;
+          m2[X] = mnew;
         }
-        l[X] = (m2[X] == kNegInf ? 0.f : l[X] * ex2(m2[X] - mnew)) + acc0 + acc1;
-        m2[X] = mnew;
       }
       tc_fence_before();
       __syncwarp();
@@ -280,9 +278,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <int BN, bool GIVEN>
+template <int S_BLK, bool GIVEN>
 cudaError_t launch_d(const Dims& D, const FwdArgs& a, int32_t* status, cudaStream_t st) {
-  using C = DCfg<BN>;
+  using C = DCfg;
   CUtensorMap mq, mk;
   if (!make_tma_map_bf16(&mq, a.q, D.B, D.Hq, D.N, BM) || !make_tma_map_bf16(&mk, a.k, D.B, D.Hkv, D.N, BN))
     return cudaErrorInvalidValue;
@@ -297,7 +295,7 @@ cudaError_t launch_d(const Dims& D, const FwdArgs& a, int32_t* status, cudaStrea
   p.n = D.n;
   p.k = D.k;
   p.c = D.scale * 1.4426950408889634f;
-  auto kern = dropped_tc_kernel<BN, GIVEN>;
+  auto kern = dropped_tc_kernel<S_BLK, GIVEN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<dim3((D.N + BM - 1) / BM, D.Hq, D.B), NTHREADS, C::SMEM, st>>>(mq, mk, p);
