@@ -36,7 +36,11 @@ namespace {
 using namespace sm100;
 
 constexpr int HD = 128;
-constexpr int NTHREADS = 192;
+// Gradient kernels: warps 0-7 compute P / dS (warps w and w+4 share TMEM lanes
+// 32(w%4).. and split a tile's columns), warp 8 loads by TMA, warp 9 owns
+// TMEM and issues the MMAs.
+constexpr int NTHREADS = 320;
+constexpr int WARP_TMA = 8, WARP_MMA = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ================================================================ preprocess
@@ -95,6 +99,19 @@ __global__ void __launch_bounds__(256) bwd_pre_tc_kernel(TensorRef hf_t, TensorR
   }
 }
 
+// Both warps of a lane quarter (w, w+4) reach this point before either
+// continues; bounded like every other wait.  `uses` counts this warp's
+// passes, which the partner matches one for one.
+__device__ __forceinline__ bool pair_sync(uint64_t* bar, uint32_t& uses, int lane, volatile int* abort) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, uses & 1u, abort);
+  ++uses;
+  tc_fence_after();
+  return ok;
+}
+
 struct BwdTcParams {
   TensorRef dq, dk, dv;     // outputs (bf16, strided)
   const float* lse_full;    // [B,Hq,N]
@@ -142,11 +159,13 @@ struct Misc {
   uint64_t a_full;
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t s_full[2], ds_full[2];
+  uint64_t pair[4];  // warps w and w+4: both hold their inputs before either writes
   uint64_t done, drain;
   uint32_t tmem_base;
   int abort;
   uint8_t state[MAX_TILES];  // per key tile: half-0 state | half-1 state << 2
 };
+static_assert(sizeof(Misc) <= SMEM - OFF_MISC - 1024, "dq shared-memory budget");
 }  // namespace dq
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -179,14 +198,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&M.s_full[s], 1);
-      mbar_init(&M.ds_full[s], 4);
+      mbar_init(&M.ds_full[s], 8);
     }
+    for (int q = 0; q < 4; ++q) mbar_init(&M.pair[q], 2);
     mbar_init(&M.done, 1);
     mbar_init(&M.drain, 1);
     M.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == WARP_MMA) {
     tmem_alloc(&M.tmem_base, 512);
     tmem_relinquish();
   }
@@ -205,7 +225,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
 
-  if (warp == 4) {
+  if (warp == WARP_TMA) {
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
@@ -243,7 +263,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_wait(&M.v_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == WARP_MMA) {
     if (lane == 0) {
       const uint32_t aq = smem_u32(sQ), af = smem_u32(sDhf), as = smem_u32(sDhs);
       bool ok = mbar_wait(&M.a_full, 0, abort);
@@ -297,14 +317,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_wait(&M.drain, 0, &dummy);
     }
   } else {
-    const int row = warp * 32 + lane;
+    const int quarter = warp & 3, ch = warp >> 2;  // lanes 32*quarter.., key columns 32*ch..
+    const int row = quarter * 32 + lane;
     const int t = q0 + row;
-    const int half = warp >> 1;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int half = quarter >> 1;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const bool in_range = t < p.N;
     const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + (in_range ? t : 0);
     const float4 sc = p.scal[ro];
     const float l2f = sc.x, l2s = sc.y, Dfv = sc.z, Dsv = sc.w;
+    uint32_t pair_uses = 0;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1;
@@ -314,43 +336,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_after();
       const int mine = half ? (M.state[j] >> 2) : (M.state[j] & 3);
-      uint32_t pk[32];
+      const uint32_t c0 = 32 * ch;
+      uint32_t pk[16];
       if (mine == 0) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        for (int c = 0; c < 16; ++c) pk[c] = 0u;
       } else {
-        uint32_t rs[32], rf[32];
-        float ds[64];
-        const uint32_t sa = lane_base + COL_S + sb * 64;
-        const uint32_t fa = lane_base + COL_DPF + sb * 64;
-        const int u0 = j * BK;
+        uint32_t rs[32], rf[32], rp[32];
+        tmem_ld32(lane_base + COL_S + sb * 64 + c0, rs);
+        tmem_ld32(lane_base + COL_DPF + sb * 64 + c0, rf);
+        if (mine == 1) tmem_ld32(lane_base + COL_DPS + sb * 64 + c0, rp);
+        tmem_wait_ld();
+        // dS overwrites the S columns this pair reads: both warps must hold
+        // their inputs before either writes.
+        if (!pair_sync(&M.pair[quarter], pair_uses, lane, abort)) {
+          ok = false;
+          break;
+        }
+        const int u0 = j * BK + (int)c0;
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          tmem_ld32(sa + c0, rs);
-          tmem_ld32(fa + c0, rf);
-          tmem_wait_ld();
+        for (int c = 0; c < 32; c += 2) {
+          float ds[2];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float x = __uint_as_float(rs[c]) * p.c;
-            const float pf = (u0 + c0 + c <= t) ? ex2(x - l2f) : 0.f;
-            ds[c0 + c] = pf * (__uint_as_float(rf[c]) - Dfv);
-          }
-          if (mine == 1) {
-            uint32_t rps[32];
-            tmem_ld32(lane_base + COL_DPS + sb * 64 + c0, rps);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float x = __uint_as_float(rs[c]) * p.c;
-              const float ps = (u0 + c0 + c <= t) ? ex2(x - l2s) : 0.f;
-              ds[c0 + c] = fmaf(ps, __uint_as_float(rps[c]) - Dsv, ds[c0 + c]);
+          for (int e = 0; e < 2; ++e) {
+            const float x = __uint_as_float(rs[c + e]);
+            const bool causal = u0 + c + e <= t;
+            const float pf = causal ? ex2(fmaf(x, p.c, -l2f)) : 0.f;
+            ds[e] = pf * (__uint_as_float(rf[c + e]) - Dfv);
+            if (mine == 1) {
+              const float ps = causal ? ex2(fmaf(x, p.c, -l2s)) : 0.f;
+              ds[e] = fmaf(ps, __uint_as_float(rp[c + e]) - Dsv, ds[e]);
             }
           }
+          pk[c / 2] = pack_bf16(ds[0], ds[1]);
         }
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(ds[2 * c], ds[2 * c + 1]);
       }
-      tmem_st32(lane_base + COL_S + sb * 64, pk);
+      tmem_st16(lane_base + COL_S + sb * 64 + 16 * ch, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -360,7 +381,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       __nv_bfloat16* out = in_range ? row_ptr_w<__nv_bfloat16>(p.dq, b, h, t) : nullptr;
 #pragma unroll 1
-      for (int c0 = 0; c0 < HD; c0 += 32) {
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(lane_base + COL_DQ + c0, r);
         tmem_wait_ld();
@@ -379,7 +400,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (M.abort && threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_TIMEOUT);
-  if (warp == 5) {
+  if (warp == WARP_MMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -410,11 +431,13 @@ struct Misc {
   uint64_t kv_full;
   uint64_t full[NS], empty[NS];
   uint64_t s_full[2], p_full[2], done, drain;
+  uint64_t pair[4];  // warps w and w+4: both hold their inputs before either writes
   uint32_t tmem_base;
   int abort;
   // per step: key-half-0 state | key-half-1 state << 2 | any selected << 4
   uint8_t state[MAX_STEPS];
 };
+static_assert(sizeof(Misc) <= SMEM - OFF_MISC - 1024, "dkv shared-memory budget");
 }  // namespace dkv
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -447,14 +470,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s2 = 0; s2 < 2; ++s2) {
       mbar_init(&M.s_full[s2], 1);
-      mbar_init(&M.p_full[s2], 4);
+      mbar_init(&M.p_full[s2], 8);
     }
+    for (int q = 0; q < 4; ++q) mbar_init(&M.pair[q], 2);
     mbar_init(&M.done, 1);
     mbar_init(&M.drain, 1);
     M.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == WARP_MMA) {
     tmem_alloc(&M.tmem_base, 512);
     tmem_relinquish();
   }
@@ -475,7 +499,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sV = smem + OFF_V;
   auto stage_ptr = [&](int st) { return smem + OFF_STAGE + st * STAGE; };
 
-  if (warp == 4) {
+  if (warp == WARP_TMA) {
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmDhf);
@@ -518,7 +542,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_wait(&M.full[it % NS], (uint32_t)(it / NS) & 1u, &dummy);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == WARP_MMA) {
     if (lane == 0) {
       const uint32_t ak = smem_u32(sK), av = smem_u32(sV);
       bool ok = mbar_wait(&M.kv_full, 0, abort);
@@ -601,10 +625,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_wait(&M.drain, 0, &dummy);
     }
   } else {
-    const int row = warp * 32 + lane;  // key within the tile
+    const int quarter = warp & 3, ch = warp >> 2;  // lanes 32*quarter.., query columns 32*ch..
+    const int row = quarter * 32 + lane;           // key within the tile
     const int u = u0 + row;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     int qt = qt0;
+    uint32_t pair_uses = 0;
     bool ok = true;
     for (int it = 0; it < steps; ++it) {
       const int b2 = it & 1;
@@ -624,56 +650,52 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       const int t0 = qt * BQ;
       const int stt = M.state[it];
-      const int mine = (warp >> 1) ? ((stt >> 2) & 3) : (stt & 3);
+      const int mine = (quarter >> 1) ? ((stt >> 2) & 3) : (stt & 3);
       const bool any = (stt & 16) != 0;
       if (++qt == qt0 + steps_per_head) qt = qt0;
       const float4* sc = reinterpret_cast<const float4*>(stage_ptr(st) + 3 * TILE_Q);
-      // P^T -> S cols [0,32); P_s^T -> S cols [32,64); dS^T -> dP_f cols [0,32).
+      const uint32_t c0 = 32 * ch;
+      // P^T -> S cols [16ch, 16ch+16); P_s^T -> S cols [32+16ch, ...); dS^T -> dP_f cols [16ch, ...).
+      uint32_t pf_pk[16], ps_pk[16], ds_pk[16];
       if (mine == 0) {
-        uint32_t z[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) z[c] = 0u;
-        tmem_st32(lane_base + COL_S, z);
-        if (any) tmem_st32(lane_base + COL_S + 32, z);
-        tmem_st32(lane_base + COL_DPF, z);
+        for (int c = 0; c < 16; ++c) pf_pk[c] = ps_pk[c] = ds_pk[c] = 0u;
       } else {
-        uint32_t rs[64];  // the whole S^T row, so P_s^T may overwrite its upper half
-        tmem_ld32(lane_base + COL_S, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
-        tmem_ld32(lane_base + COL_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
+        uint32_t rs[32], rf[32], rp[32];
+        tmem_ld32(lane_base + COL_S + c0, rs);
+        tmem_ld32(lane_base + COL_DPF + c0, rf);
+        if (mine == 1) tmem_ld32(lane_base + COL_DPS + c0, rp);
         tmem_wait_ld();
+        // the outputs overwrite columns the partner warp reads
+        if (!pair_sync(&M.pair[quarter], pair_uses, lane, abort)) {
+          ok = false;
+          break;
+        }
 #pragma unroll
-        for (int c0 = 0; c0 < BQ; c0 += 32) {
-          uint32_t rf[32], rp[32];
-          tmem_ld32(lane_base + COL_DPF + c0, rf);
-          if (mine == 1) tmem_ld32(lane_base + COL_DPS + c0, rp);
-          tmem_wait_ld();
-          uint32_t pf_pk[16], ps_pk[16], ds_pk[16];
+        for (int c = 0; c < 32; c += 2) {
+          float pf[2], ps[2], dsv[2];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float pf[2], ps[2], dsv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int q = c0 + c + e;
-              const float4 v4 = sc[q];  // lse2_f, lse2_s, D_f, D_s of query t0 + q
-              const float x = __uint_as_float(rs[q]);
-              const bool causal = u <= t0 + q;
-              pf[e] = causal ? ex2(fmaf(x, p.c, -v4.x)) : 0.f;
-              dsv[e] = pf[e] * (__uint_as_float(rf[c + e]) - v4.z);
-              ps[e] = 0.f;
-              if (mine == 1) {
-                ps[e] = causal ? ex2(fmaf(x, p.c, -v4.y)) : 0.f;
-                dsv[e] = fmaf(ps[e], __uint_as_float(rp[c + e]) - v4.w, dsv[e]);
-              }
+          for (int e = 0; e < 2; ++e) {
+            const int q = (int)c0 + c + e;
+            const float4 v4 = sc[q];  // lse2_f, lse2_s, D_f, D_s of query t0 + q
+            const float x = __uint_as_float(rs[c + e]);
+            const bool causal = u <= t0 + q;
+            pf[e] = causal ? ex2(fmaf(x, p.c, -v4.x)) : 0.f;
+            dsv[e] = pf[e] * (__uint_as_float(rf[c + e]) - v4.z);
+            ps[e] = 0.f;
+            if (mine == 1) {
+              ps[e] = causal ? ex2(fmaf(x, p.c, -v4.y)) : 0.f;
+              dsv[e] = fmaf(ps[e], __uint_as_float(rp[c + e]) - v4.w, dsv[e]);
             }
-            pf_pk[c / 2] = pack_bf16(pf[0], pf[1]);
-            ps_pk[c / 2] = pack_bf16(ps[0], ps[1]);
-            ds_pk[c / 2] = pack_bf16(dsv[0], dsv[1]);
           }
-          tmem_st16(lane_base + COL_S + c0 / 2, pf_pk);
-          if (any) tmem_st16(lane_base + COL_S + 32 + c0 / 2, ps_pk);
-          tmem_st16(lane_base + COL_DPF + c0 / 2, ds_pk);
+          pf_pk[c / 2] = pack_bf16(pf[0], pf[1]);
+          ps_pk[c / 2] = pack_bf16(ps[0], ps[1]);
+          ds_pk[c / 2] = pack_bf16(dsv[0], dsv[1]);
         }
       }
+      tmem_st16(lane_base + COL_S + 16 * ch, pf_pk);
+      if (any) tmem_st16(lane_base + COL_S + 32 + 16 * ch, ps_pk);
+      tmem_st16(lane_base + COL_DPF + 16 * ch, ds_pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -685,7 +707,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __nv_bfloat16* ok_ = store ? row_ptr_w<__nv_bfloat16>(p.dk, b, kvh, u) : nullptr;
       __nv_bfloat16* ov_ = store ? row_ptr_w<__nv_bfloat16>(p.dv, b, kvh, u) : nullptr;
 #pragma unroll 1
-      for (int c0 = 0; c0 < HD; c0 += 32) {
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 32) {
         uint32_t rk[32], rv[32];
         tmem_ld32(lane_base + COL_DK + c0, rk);
         tmem_ld32(lane_base + COL_DV + c0, rv);
@@ -711,7 +733,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (M.abort && threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_TIMEOUT);
-  if (warp == 5) {
+  if (warp == WARP_MMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -50,6 +50,7 @@ struct DMisc {
   int abort;
   uint32_t sel[2][64];
 };
+static_assert(sizeof(DMisc) <= DCfg::SMEM - DCfg::OFF_MISC - 1024, "dropped shared-memory budget");
 
 struct DParams {
   const int32_t* idx;
