@@ -10,11 +10,12 @@
 // two output accumulators per row, so the dual stream costs the MMAs of one
 // causal attention.
 //
-// CTA = one 128-row query tile of one (batch, query head), 192 threads:
-//   warps 0-3  softmax / rescale / epilogue; warp w owns TMEM lanes 32w..32w+31,
-//              i.e. query rows 32w..32w+31 of the tile (one row per thread);
-//   warp 4     TMA producer (Q once, then 128-key K and V tiles, 2-stage ring);
-//   warp 5     TMEM allocator and single-thread tcgen05.mma issuer.
+// CTA = one 128-row query tile of one (batch, query head), 320 threads:
+//   warps 0-7  softmax / rescale / epilogue; warps w and w+4 share TMEM lanes
+//              32(w%4)..+31, i.e. query rows 32(w%4).. of the tile, one row per
+//              thread; warp w takes the tile's 64-key sub-block w/4;
+//   warp 8     TMA producer (Q once, then 128-key K and V tiles, 2-stage ring);
+//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer.
 // TMEM (512 columns): O_A [0,128), O_D [128,256), S ping-pong [256,384), [384,512).
 // P (bf16, two per column) overwrites its S buffer and feeds the PV MMA from TMEM.
 //
@@ -27,9 +28,12 @@
 // states: no causal key, selected (A) or dropped (D).
 //
 // Softmax in base 2 with the scale folded in: p = 2^(S*c - m), c = scale*log2(e).
-// A row's running max m of each set is raised only when a tile's max for that
-// set exceeds it by more than 8 (p stays below 2^8); O and l are then rescaled
-// in place after the previous PV has completed.
+// The two warps of a row trade their sub-block maxima through shared memory,
+// so both hold the same running max per set; each keeps its own partial row
+// sum, and the partials are added at the end.  A row's running max m of each
+// set is raised only when a tile's max for that set exceeds it by more than 8
+// (p stays below 2^8); O and l are then rescaled in place (each warp of the
+// pair rescales half of the columns) after the previous PV has completed.
 #include "ssa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -44,7 +48,8 @@ constexpr int BM = 128;    // query rows per CTA
 constexpr int BN = 128;    // keys per tile
 constexpr int SUB = 64;    // keys per sub-block
 constexpr int HD = 128;
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 320;
+constexpr int WARP_TMA = 8, WARP_MMA = 9;
 constexpr int NS = 2;      // K/V stages
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -54,7 +59,6 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = Q_BYTES;
 constexpr int OFF_V = OFF_K + NS * KV_BYTES;
 constexpr int OFF_MISC = OFF_V + NS * KV_BYTES;
-constexpr int SMEM_BYTES = OFF_MISC + 2048 + 1024;  // + alignment slack
 constexpr uint32_t COL_OA = 0, COL_OD = 128, COL_S = 256;
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
@@ -64,10 +68,14 @@ struct Misc {
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t s_full[2], p_full[2];
   uint64_t o_done, o_final, drain;
+  uint64_t pair[4];     // warps w and w+4 (one per lane quarter)
   uint32_t tmem_base;
   int abort;
   uint32_t sel[2][64];  // selected-block bits of the tile's two query blocks
+  float xmax[2][2][128];  // [tile parity][sub-block][row]: scaled tile max of its set
+  float lsum[2][2][128];  // epilogue: per sub-block warp, per set, per row
 };
+constexpr int SMEM_BYTES = OFF_MISC + (int)sizeof(Misc) + 1024;  // + alignment slack
 
 struct TcParams {
   TensorRef hf, hs;
@@ -84,6 +92,19 @@ struct TcParams {
 __device__ __forceinline__ int pair_state(int kb, int ib, bool valid, const uint32_t* selw) {
   if (!valid || kb > ib) return 0;
   return ((selw[kb >> 5] >> (kb & 31)) & 1u) ? 1 : 2;
+}
+
+// Both warps of a lane quarter (w, w+4) reach this point before either
+// continues; bounded like every other wait.  `uses` counts this warp's
+// passes, which the partner matches one for one.
+__device__ __forceinline__ bool pair_sync(uint64_t* bar, uint32_t& uses, int lane, volatile int* abort) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, uses & 1u, abort);
+  ++uses;
+  tc_fence_after();
+  return ok;
 }
 
 template <int S_BLK>
@@ -119,16 +140,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&M.s_full[s], 1);
-      mbar_init(&M.p_full[s], 4);
+      mbar_init(&M.p_full[s], 8);
     }
     mbar_init(&M.o_done, 1);
     mbar_init(&M.o_final, 1);
     mbar_init(&M.drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&M.pair[q], 2);
     M.abort = 0;
     fence_mbar_init();
   }
   for (int w = threadIdx.x; w < 2 * 64; w += NTHREADS) (&M.sel[0][0])[w] = 0u;
-  if (warp == 5) {
+  if (warp == WARP_MMA) {
     tmem_alloc(&M.tmem_base, 512);
     tmem_relinquish();
   }
@@ -158,7 +180,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
 
-  if (warp == 4) {
+  if (warp == WARP_TMA) {
     // ================================================================ producer
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
@@ -194,7 +216,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_wait(&M.v_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == WARP_MMA) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       const uint32_t q_addr = smem_u32(sQ);
@@ -269,15 +291,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else {
     // ================================================================ softmax
-    const int half = warp >> 1;
+    const int quarter = warp & 3, q = warp >> 2;  // lane quarter, key sub-block
+    const int half = quarter >> 1;
     const int ib = half ? ib1 : ib0;
     const bool hvalid = half ? valid1 : true;
     const uint32_t* selw = half ? sel1 : sel0;
-    const int row = warp * 32 + lane;  // row within the tile == TMEM lane
-    const int t = q0 + row;            // query token
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int row = quarter * 32 + lane;  // row within the tile == TMEM lane
+    const int t = q0 + row;               // query token
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     float m2[2] = {kNegInf, kNegInf};  // running max (scaled, base 2), [0]=A [1]=D
-    float l[2] = {0.f, 0.f};
+    float l[2] = {0.f, 0.f};           // this warp's partial sums
+    uint32_t pair_uses = 0;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1;
@@ -286,129 +310,125 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
-      int mine[2];
-      bool mixed[2];
+      int st[2];  // this row's state of sub-blocks 0 and 1
+      bool mixed_q;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int qq = 0; qq < 2; ++qq) st[qq] = pair_state(kblk(j, qq), ib, hvalid, selw);
+      {
         const int kb = kblk(j, q);
-        mine[q] = pair_state(kb, ib, hvalid, selw);
         const int o0 = pair_state(kb, ib0, true, sel0);
         const int o1 = pair_state(kb, ib1, valid1, sel1);
-        mixed[q] = (o0 != 0 && o1 != 0 && o0 != o1);
+        mixed_q = (o0 != 0 && o1 != 0 && o0 != o1);
       }
+      const int mine = st[q];
       const uint32_t s_addr = lane_base + COL_S + (uint32_t)sb * BN;
-      uint32_t pk[BN / 2];
-      if (mine[0] == 0 && mine[1] == 0) {
+      float x[SUB];  // raw S of this warp's sub-block; the scale is folded into the exponent
+      float mx = kNegInf;
+      if (mine != 0) {
 #pragma unroll
-        for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
-      } else {
-        float x[BN];  // raw S = q.k; the scale is folded into the exponent
-#pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 32) {
+        for (int c0 = 0; c0 < SUB; c0 += 32) {
           uint32_t r[32];
-          tmem_ld32(s_addr + c0, r);
+          tmem_ld32(s_addr + q * SUB + c0, r);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(r[c]);
         }
-        const int u0 = j * BN;
-        if (u0 + BN - 1 > t) {  // causal mask inside the diagonal tile
+        const int u0 = j * BN + q * SUB;
+        if (u0 + SUB - 1 > t) {  // causal mask inside the diagonal sub-block
 #pragma unroll
-          for (int c = 0; c < BN; ++c)
+          for (int c = 0; c < SUB; ++c)
             if (u0 + c > t) x[c] = kNegInf;
         }
-        float mxq[2];
+        float a0 = kNegInf, a1 = kNegInf, a2 = kNegInf, a3 = kNegInf;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float a0 = kNegInf, a1 = kNegInf, a2 = kNegInf, a3 = kNegInf;
-#pragma unroll
-          for (int c = q * SUB; c < (q + 1) * SUB; c += 4) {
-            a0 = fmaxf(a0, x[c]);
-            a1 = fmaxf(a1, x[c + 1]);
-            a2 = fmaxf(a2, x[c + 2]);
-            a3 = fmaxf(a3, x[c + 3]);
-          }
-          mxq[q] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * p.c;  // scale > 0
+        for (int c = 0; c < SUB; c += 4) {
+          a0 = fmaxf(a0, x[c]);
+          a1 = fmaxf(a1, x[c + 1]);
+          a2 = fmaxf(a2, x[c + 2]);
+          a3 = fmaxf(a3, x[c + 3]);
         }
-        // per-set tile max, rescale when it jumps past the threshold
-#pragma unroll
-        for (int X = 0; X < 2; ++X) {
-          float mx = kNegInf;
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-            if (mine[q] == X + 1) mx = fmaxf(mx, mxq[q]);
-          const float m_old = m2[X];
-          const bool need = (m_old != kNegInf) && (mx > m_old + kRescaleThreshold);
-          if (__any_sync(0xffffffffu, need)) {
-            // O_X must hold every earlier PV before it is rescaled.
-            if (j >= 1 && !mbar_wait(&M.o_done, (uint32_t)(j - 1) & 1u, abort)) ok = false;
-            if (__any_sync(0xffffffffu, !ok)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const float f = need ? ex2(m_old - mx) : 1.0f;
-            const uint32_t o_addr = lane_base + (X == 0 ? COL_OA : COL_OD);
-#pragma unroll 1
-            for (int c0 = 0; c0 < HD; c0 += 32) {
-              uint32_t r[32];
-              tmem_ld32(o_addr + c0, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
-              tmem_st32(o_addr + c0, r);
-            }
-            tmem_wait_st();
-            if (need) {
-              l[X] *= f;
-              m2[X] = mx;
-            }
-          }
-          if (m2[X] == kNegInf) m2[X] = mx;
-        }
-        if (!ok) break;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          if (mine[q] == 0) {
-#pragma unroll
-            for (int c = 0; c < SUB / 2; ++c) pk[q * SUB / 2 + c] = 0u;
-            continue;
-          }
-          const int X = mine[q] - 1;
-          const float nm = -m2[X];
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int c = q * SUB; c < (q + 1) * SUB; c += 2) {
-            const float e0 = ex2(fmaf(x[c], p.c, nm));
-            const float e1 = ex2(fmaf(x[c + 1], p.c, nm));
-            s0 += e0;
-            s1 += e1;
-            pk[c / 2] = pack_bf16(e0, e1);
-          }
-          l[X] += s0 + s1;
-        }
+        mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * p.c;  // scale > 0
       }
-      // Write P where the MMA warp will read it: sub-block q's P at columns
-      // [32q, 32q+32) of the S buffer; for a mixed sub-block the dropped
-      // half's rows use [64+32q, 64+32q+32) instead and write zeros to the first.
-      uint32_t z[32];
+      // Trade sub-block maxima with the partner warp; after this point both
+      // warps have read their S columns, so P may overwrite them.
+      M.xmax[sb][q][row] = mx;
+      if (!pair_sync(&M.pair[quarter], pair_uses, lane, abort)) {
+        ok = false;
+        break;
+      }
+      const float mx_other = M.xmax[sb][q ^ 1][row];
+      const int st_other = st[q ^ 1];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) z[c] = 0u;
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const uint32_t p0 = s_addr + 32 * q, p1 = s_addr + 64 + 32 * q;
-        const uint32_t(&blk)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * q]);
-        if (mixed[q]) {
-          if (mine[q] == 1) {
-            tmem_st32(p0, blk);
-            tmem_st32(p1, z);
-          } else {
-            tmem_st32(p0, z);
-            tmem_st32(p1, blk);
+      for (int X = 0; X < 2; ++X) {
+        float mxs = kNegInf;
+        if (mine == X + 1) mxs = mx;
+        if (st_other == X + 1) mxs = fmaxf(mxs, mx_other);
+        const float m_old = m2[X];
+        const bool need = (m_old != kNegInf) && (mxs > m_old + kRescaleThreshold);
+        if (__any_sync(0xffffffffu, need)) {
+          // O_X must hold every earlier PV before it is rescaled; this warp
+          // rescales its half of the columns.
+          if (j >= 1 && !mbar_wait(&M.o_done, (uint32_t)(j - 1) & 1u, abort)) ok = false;
+          if (__any_sync(0xffffffffu, !ok)) {
+            ok = false;
+            break;
           }
-        } else {
-          tmem_st32(p0, blk);
+          tc_fence_after();
+          const float f = need ? ex2(m_old - mxs) : 1.0f;
+          const uint32_t o_addr = lane_base + (X == 0 ? COL_OA : COL_OD) + q * (HD / 2);
+#pragma unroll 1
+          for (int c0 = 0; c0 < HD / 2; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(o_addr + c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
+            tmem_st32(o_addr + c0, r);
+          }
+          tmem_wait_st();
+          if (need) {
+            l[X] *= f;
+            m2[X] = mxs;
+          }
         }
+        if (m2[X] == kNegInf) m2[X] = mxs;
+      }
+      if (!ok) break;
+      uint32_t pk[SUB / 2];
+      if (mine == 0) {
+#pragma unroll
+        for (int c = 0; c < SUB / 2; ++c) pk[c] = 0u;
+      } else {
+        const float nm = -m2[mine - 1];
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < SUB; c += 2) {
+          const float e0 = ex2(fmaf(x[c], p.c, nm));
+          const float e1 = ex2(fmaf(x[c + 1], p.c, nm));
+          s0 += e0;
+          s1 += e1;
+          pk[c / 2] = pack_bf16(e0, e1);
+        }
+        l[mine - 1] += s0 + s1;
+      }
+      // Sub-block q's P at columns [32q, 32q+32) of the S buffer; for a mixed
+      // sub-block the dropped half's rows use [64+32q, 64+32q+32) instead and
+      // write zeros to the first.
+      const uint32_t p0 = s_addr + 32 * q, p1 = s_addr + 64 + 32 * q;
+      const uint32_t(&blk)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]);
+      if (mixed_q) {
+        uint32_t z[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) z[c] = 0u;
+        if (mine == 1) {
+          tmem_st32(p0, blk);
+          tmem_st32(p1, z);
+        } else {
+          tmem_st32(p0, z);
+          tmem_st32(p1, blk);
+        }
+      } else {
+        tmem_st32(p0, blk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -417,10 +437,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 
     // ================================================================ epilogue
+    // Add the partner's partial sums (same running maxima in both warps).
+    M.lsum[q][0][row] = l[0];
+    M.lsum[q][1][row] = l[1];
+    if (ok && !pair_sync(&M.pair[quarter], pair_uses, lane, abort)) ok = false;
     if (ok && mbar_wait(&M.o_final, 0, abort)) {
       tc_fence_after();
+      const float lA = l[0] + M.lsum[q ^ 1][0][row], lD = l[1] + M.lsum[q ^ 1][1][row];
       const bool store = t < p.N;
-      const float mA = m2[0], mD = m2[1], lA = l[0], lD = l[1];
+      const float mA = m2[0], mD = m2[1];
       const float Mx = fmaxf(mA, mD);
       const float wa = (lA > 0.f) ? ex2(mA - Mx) : 0.f;
       const float wd = (lD > 0.f) ? ex2(mD - Mx) : 0.f;
@@ -429,7 +454,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __nv_bfloat16* hf = store ? row_ptr_w<__nv_bfloat16>(p.hf, b, h, t) : nullptr;
       __nv_bfloat16* hs = store ? row_ptr_w<__nv_bfloat16>(p.hs, b, h, t) : nullptr;
 #pragma unroll 1
-      for (int c0 = 0; c0 < HD; c0 += 32) {
+      for (int c0 = q * (HD / 2); c0 < (q + 1) * (HD / 2); c0 += 32) {
         uint32_t ra[32], rd[32];
         tmem_ld32(lane_base + COL_OA + c0, ra);
         tmem_ld32(lane_base + COL_OD + c0, rd);
@@ -448,13 +473,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint4* dst_s = reinterpret_cast<uint4*>(hs + c0);
           uint4* dst_f = reinterpret_cast<uint4*>(hf + c0);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            dst_s[q] = make_uint4(os[4 * q], os[4 * q + 1], os[4 * q + 2], os[4 * q + 3]);
-            dst_f[q] = make_uint4(of[4 * q], of[4 * q + 1], of[4 * q + 2], of[4 * q + 3]);
+          for (int v = 0; v < 4; ++v) {
+            dst_s[v] = make_uint4(os[4 * v], os[4 * v + 1], os[4 * v + 2], os[4 * v + 3]);
+            dst_f[v] = make_uint4(of[4 * v], of[4 * v + 1], of[4 * v + 2], of[4 * v + 3]);
           }
         }
       }
-      if (store) {
+      if (store && q == 0) {
         constexpr float kLn2 = 0.6931471805599453f;
         const float lse2_a = (lA > 0.f) ? mA + log2f(lA) : kNegInf;
         const float lse2_d = (lD > 0.f) ? mD + log2f(lD) : kNegInf;
@@ -472,7 +497,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (M.abort && threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_TIMEOUT);
-  if (warp == 5) {
+  if (warp == WARP_MMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
