@@ -138,6 +138,60 @@ __device__ __forceinline__ int pair_state(const BwdTcParams& p, int b, int h, in
   return sel_bit(p, b, h, i, j) ? 1 : 2;
 }
 
+// P / dS of one 32-column slice of a dK/dV step (keys in lanes, queries in
+// columns).  SEL: the slice's key block is selected for the query block, so
+// the sparse stream contributes; DIAG: the slice touches the causal diagonal.
+template <bool SEL, bool DIAG>
+__device__ __forceinline__ void dkv_slice(const uint32_t (&rs)[32], const uint32_t (&rf)[32],
+                                          const uint32_t (&rp)[32], const float4* sc, int u, int tq0, float c,
+                                          uint32_t (&pf_pk)[16], uint32_t (&ps_pk)[16], uint32_t (&ds_pk)[16]) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    float pf[2], ps[2], dsv[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float4 v4 = sc[k + e];  // lse2_f, lse2_s, D_f, D_s of query tq0 + k + e
+      const float x = __uint_as_float(rs[k + e]);
+      pf[e] = ex2(fmaf(x, c, -v4.x));
+      if (DIAG && u > tq0 + k + e) pf[e] = 0.f;
+      dsv[e] = pf[e] * (__uint_as_float(rf[k + e]) - v4.z);
+      ps[e] = 0.f;
+      if (SEL) {
+        ps[e] = ex2(fmaf(x, c, -v4.y));
+        if (DIAG && u > tq0 + k + e) ps[e] = 0.f;
+        dsv[e] = fmaf(ps[e], __uint_as_float(rp[k + e]) - v4.w, dsv[e]);
+      }
+    }
+    pf_pk[k / 2] = pack_bf16(pf[0], pf[1]);
+    if (SEL) ps_pk[k / 2] = pack_bf16(ps[0], ps[1]);
+    ds_pk[k / 2] = pack_bf16(dsv[0], dsv[1]);
+  }
+}
+
+// dS of one 32-key slice of a dQ tile (queries in lanes, keys in columns).
+template <bool SEL, bool DIAG>
+__device__ __forceinline__ void dq_slice(const uint32_t (&rs)[32], const uint32_t (&rf)[32],
+                                         const uint32_t (&rp)[32], float l2f, float l2s, float Dfv, float Dsv,
+                                         int u0, int t, float c, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    float ds[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float x = __uint_as_float(rs[k + e]);
+      float pf = ex2(fmaf(x, c, -l2f));
+      if (DIAG && u0 + k + e > t) pf = 0.f;
+      ds[e] = pf * (__uint_as_float(rf[k + e]) - Dfv);
+      if (SEL) {
+        float ps = ex2(fmaf(x, c, -l2s));
+        if (DIAG && u0 + k + e > t) ps = 0.f;
+        ds[e] = fmaf(ps, __uint_as_float(rp[k + e]) - Dsv, ds[e]);
+      }
+    }
+    pk[k / 2] = pack_bf16(ds[0], ds[1]);
+  }
+}
+
 // ================================================================ dQ kernel
 namespace dq {
 constexpr int BM = 128;  // query rows
@@ -354,21 +408,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           break;
         }
         const int u0 = j * BK + (int)c0;
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float x = __uint_as_float(rs[c + e]);
-            const bool causal = u0 + c + e <= t;
-            const float pf = causal ? ex2(fmaf(x, p.c, -l2f)) : 0.f;
-            ds[e] = pf * (__uint_as_float(rf[c + e]) - Dfv);
-            if (mine == 1) {
-              const float ps = causal ? ex2(fmaf(x, p.c, -l2s)) : 0.f;
-              ds[e] = fmaf(ps, __uint_as_float(rp[c + e]) - Dsv, ds[e]);
-            }
-          }
-          pk[c / 2] = pack_bf16(ds[0], ds[1]);
+        const bool diag = u0 + 31 > q0 + quarter * 32;  // some key of the slice is after some row
+        if (mine == 1) {
+          if (diag) dq_slice<true, true>(rs, rf, rp, l2f, l2s, Dfv, Dsv, u0, t, p.c, pk);
+          else dq_slice<true, false>(rs, rf, rp, l2f, l2s, Dfv, Dsv, u0, t, p.c, pk);
+        } else {
+          if (diag) dq_slice<false, true>(rs, rf, rp, l2f, l2s, Dfv, Dsv, u0, t, p.c, pk);
+          else dq_slice<false, false>(rs, rf, rp, l2f, l2s, Dfv, Dsv, u0, t, p.c, pk);
         }
       }
       tmem_st16(lane_base + COL_S + sb * 64 + 16 * ch, pk);
@@ -671,26 +717,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
+        const int tq0 = t0 + (int)c0;                   // first query of the slice
+        const bool diag = u0 + quarter * 32 + 31 > tq0;  // some key of the warp after some query
+        if (mine == 1) {
+          if (diag) dkv_slice<true, true>(rs, rf, rp, sc + c0, u, tq0, p.c, pf_pk, ps_pk, ds_pk);
+          else dkv_slice<true, false>(rs, rf, rp, sc + c0, u, tq0, p.c, pf_pk, ps_pk, ds_pk);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pf[2], ps[2], dsv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int q = (int)c0 + c + e;
-            const float4 v4 = sc[q];  // lse2_f, lse2_s, D_f, D_s of query t0 + q
-            const float x = __uint_as_float(rs[c + e]);
-            const bool causal = u <= t0 + q;
-            pf[e] = causal ? ex2(fmaf(x, p.c, -v4.x)) : 0.f;
-            dsv[e] = pf[e] * (__uint_as_float(rf[c + e]) - v4.z);
-            ps[e] = 0.f;
-            if (mine == 1) {
-              ps[e] = causal ? ex2(fmaf(x, p.c, -v4.y)) : 0.f;
-              dsv[e] = fmaf(ps[e], __uint_as_float(rp[c + e]) - v4.w, dsv[e]);
-            }
-          }
-          pf_pk[c / 2] = pack_bf16(pf[0], pf[1]);
-          ps_pk[c / 2] = pack_bf16(ps[0], ps[1]);
-          ds_pk[c / 2] = pack_bf16(dsv[0], dsv[1]);
+          for (int c = 0; c < 16; ++c) ps_pk[c] = 0u;
+          if (diag) dkv_slice<false, true>(rs, rf, rp, sc + c0, u, tq0, p.c, pf_pk, ps_pk, ds_pk);
+          else dkv_slice<false, false>(rs, rf, rp, sc + c0, u, tq0, p.c, pf_pk, ps_pk, ds_pk);
         }
       }
       tmem_st16(lane_base + COL_S + 16 * ch, pf_pk);
