@@ -228,8 +228,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                      const __grid_constant__ CUtensorMap tmDhs, BwdTcParams p) {
   using namespace dq;
   if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Used directly (no pointer arithmetic on the address) so that accesses
+  // through it stay shared-memory loads; TMA tiles with 128-byte swizzle need
+  // the 1024-byte alignment, which is checked rather than assumed.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_UNSUPPORTED);
+    return;
+  }
   dq::Misc& M = *reinterpret_cast<dq::Misc*>(smem + OFF_MISC);
   volatile int* abort = &M.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -492,8 +499,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                       const __grid_constant__ CUtensorMap tmDhs, BwdTcParams p) {
   using namespace dkv;
   if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Used directly (no pointer arithmetic on the address) so that accesses
+  // through it stay shared-memory loads; TMA tiles with 128-byte swizzle need
+  // the 1024-byte alignment, which is checked rather than assumed.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_UNSUPPORTED);
+    return;
+  }
   dkv::Misc& M = *reinterpret_cast<dkv::Misc*>(smem + OFF_MISC);
   volatile int* abort = &M.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
