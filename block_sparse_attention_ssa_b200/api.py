@@ -81,6 +81,7 @@ _SIGS = {
                                       ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "ssa_device_status": (ctypes.c_int, [_P(ctypes.c_int32), ctypes.c_int, ctypes.c_void_p]),
     "ssa_launch_count": (ctypes.c_uint64, []),
+    "ssa_selftest_timeout": (ctypes.c_int, [ctypes.c_void_p]),
     "ssa_block_scores_noalloc": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
                                                  ctypes.c_void_p, ctypes.c_void_p]),
 }
@@ -198,6 +199,10 @@ def ssa_align_mse(dims, h_full, h_sparse, loss, ws, stream=None) -> None:
 
 def ssa_launch_count() -> int:
     return int(load_library().ssa_launch_count())
+
+
+def ssa_selftest_timeout(stream=None) -> None:
+    _check("ssa_selftest_timeout", load_library().ssa_selftest_timeout(_stream(stream)))
 
 
 def ssa_device_status(clear: bool = True, stream=None) -> int:

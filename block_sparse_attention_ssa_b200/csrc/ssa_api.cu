@@ -332,6 +332,15 @@ ssa_status_t ssa_align_mse(const ssa_dims_t* dims, const ssa_tensor_t* h_full,
   return from_cuda(e);
 }
 
+ssa_status_t ssa_selftest_timeout(ssa_stream_t stream) {
+  ssa_status_t s = check_device();
+  if (s != SSA_OK) return s;
+  int32_t* status = device_status_ptr();
+  if (status == nullptr) return SSA_ERR_CUDA;
+  // ~10 ms at the B200's clock: long enough to be a real wait, short for a test
+  return from_cuda(launch_selftest_timeout(status, 20000000LL, static_cast<cudaStream_t>(stream)));
+}
+
 ssa_status_t ssa_device_status(int32_t* status, int clear, ssa_stream_t stream) {
   if (status == nullptr) return SSA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -137,6 +137,9 @@ bool bwd_tc_supported(const Dims& D);
 cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* dev_status, cudaStream_t st);
 cudaError_t launch_bwd_simt(const Dims& D, const BwdArgs& a, cudaStream_t st);
 
+// One-CTA kernel whose bounded barrier wait runs out: records SSA_ERR_TIMEOUT.
+cudaError_t launch_selftest_timeout(int32_t* status, long long limit_cycles, cudaStream_t st);
+
 // Sum of squared differences of two [B,Hq,N,d] tensors into per-block
 // partials, then a fixed-order final reduction: out[0..n_out) = sum / count.
 cudaError_t launch_sqdiff_partials(const Dims& D, const TensorRef& a, const TensorRef& b,

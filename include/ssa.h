@@ -245,6 +245,14 @@ SSA_API ssa_status_t ssa_block_scores_noalloc(const ssa_dims_t* dims, const ssa_
  * devices, all threads).  Lets a caller count the launches of a region. */
 SSA_API uint64_t ssa_launch_count(void);
 
+/* Failure-detection self-test.  Enqueues a one-CTA kernel that waits on a
+ * barrier nothing will ever complete, using the same bounded wait as every
+ * tensor-core kernel; after about 10 ms the wait gives up, the kernel records
+ * SSA_ERR_TIMEOUT in the device status word and returns.  Nothing faults or
+ * hangs; the status word then behaves as after a real timeout (read and clear
+ * it with ssa_device_status).  Returns SSA_ERR_UNSUPPORTED off sm_100. */
+SSA_API ssa_status_t ssa_selftest_timeout(ssa_stream_t stream);
+
 /* Synchronises `stream`, copies the device status word of the current device
  * to *status (SSA_OK, or the first SSA_ERR_TIMEOUT a kernel recorded) and,
  * if clear != 0, resets it.  Returns SSA_ERR_CUDA if the synchronisation or
