@@ -5,28 +5,29 @@
 // Alignment"): L = <g_f, h_full> + <g_s, h_sparse> + alpha (L_sp + L_cm), with
 // dh_f = g_f + 2 alpha (h_f - h_s)/M and dh_s = g_s + 2 alpha (h_s - h_f)/M.
 //
-// The two streams are kept apart.  For a causal pair (t, u):
-//   P_f = exp(x - lse_full)                      (every causal pair)
-//   P_s = exp(x - lse_sel)  if u is in A_t, else 0
-//   dX  = P_f (dh_f . v_u - D_f) + P_s (dh_s . v_u - D_s),
-//   D_f = dh_f . h_f,  D_s = dh_s . h_s,
-//   dQ_t = scale sum_u dX K_u,  dK_u = scale sum_t dX Q_t,
-//   dV_u = sum_t P_f dh_f,t + sum_t P_s dh_s,t.
-// The sparse-stream products run only for tiles that contain a selected pair,
-// and a tile never needs a per-row choice of operand.
+// The two streams are independent softmax attentions over the same Q, K, V
+// and their gradients add.  Each is differentiated on its own:
+//   stream f (full):   every causal pair,        P = exp(x - lse_full), dh_f, D_f = dh_f . h_f
+//   stream s (sparse): pairs with u in A_t only, P = exp(x - lse_sel),  dh_s, D_s = dh_s . h_s
+//   dS = P (dh . v_u - D),  dQ_t += scale sum_u dS K_u,  dK_u += scale sum_t dS Q_t,
+//   dV_u += sum_t P dh_t.
+// A kernel walks 128 x 128 (key, query) tiles: first every causal tile of
+// stream f, then the tiles of stream s that hold at least one selected
+// (query block, key block) pair; inside such a tile the unselected blocks are
+// masked like the causal triangle.  Every tile is therefore the same uniform
+// step, and all tensor-core products are 128 x 128 x 16.
 //
 // Three launches:
-//   pre  (CUDA cores, HBM-bound): dh_f, dh_s in bf16, D_f, D_s, and the
-//        partial sums of (h_f - h_s)^2 for the alignment loss;
-//   dq   one 128-row query tile per CTA, walking 64-key tiles:
-//        S = Q K^T, dP_f = dh_f V^T, dP_s = dh_s V^T (SS MMAs into TMEM),
-//        dS -> TMEM (bf16), dQ += dS K (TS MMA);
-//   dkv  one 128-key tile per CTA, walking the g query heads of its kv head and
-//        every causal 64-row query tile:
-//        S^T = K Q^T, dP_f^T = V dh_f^T, dP_s^T = V dh_s^T (SS MMAs),
-//        P^T, P_s^T, dS^T -> TMEM (bf16), dV += P^T dh_f + P_s^T dh_s,
-//        dK += dS^T Q (TS MMAs).
-// No atomics: every output element is written by exactly one CTA.
+//   pre  (CUDA cores, HBM-bound): dh_f, dh_s in bf16, D_f, D_s, lse in base 2,
+//        and the partial sums of (h_f - h_s)^2 for the alignment loss;
+//   dkv  one 128-key tile per CTA, walking the g query heads of its kv head:
+//        S^T = K Q^T, dP^T = V dh^T (SS MMAs into TMEM); P^T and dS^T go back
+//        to TMEM as bf16; dV += P^T dh, dK += dS^T Q (TS MMAs);
+//   dq   one 128-row query tile per CTA, with Q and dh held in TMEM as the A
+//        operands: S = Q K^T, dP = dh V^T (TS MMAs), dS -> TMEM over dP
+//        (bf16), dQ += dS K (TS MMA); K and V stream through a 3-deep ring.
+// No atomics: every output element is written by exactly one CTA, in a fixed
+// order of steps, so results are bit-reproducible.
 #include "ssa_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -36,44 +37,65 @@ namespace {
 using namespace sm100;
 
 constexpr int HD = 128;
-// Gradient kernels: warps 0-7 compute P / dS (warps w and w+4 share TMEM lanes
-// 32(w%4).. and split a tile's columns), warp 8 loads by TMA, warp 9 owns
-// TMEM and issues the MMAs.
+// Gradient kernels: warps 0-7 compute P / dS (warp w reads TMEM lanes
+// 32(w%4).. and columns 64(w/4)..; no two warps touch the same columns),
+// warp 8 loads by TMA, warp 9 owns TMEM and issues the MMAs.
 constexpr int NTHREADS = 320;
 constexpr int WARP_TMA = 8, WARP_MMA = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
+constexpr int TILE = 128;                // keys and queries per step
+constexpr int HALF = TILE * 128;         // 16 KB: 128 rows x 64 bf16 (one 128-byte swizzle span)
+constexpr int TILE_B = 2 * HALF;         // 32 KB: one 128 x 128 bf16 tile
+constexpr int kMaxSmem = 232448;         // 227 KB per CTA
+constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, TILE, false, false);  // both operands K-major
+constexpr uint32_t IDESC_ACC = idesc_bf16_f32(TILE, HD, false, true);   // B (rows = reduction) MN-major
+
 // ================================================================ preprocess
-template <typename T>
+// One warp per row (b, h, t); lane l holds columns 4l .. 4l+3.
 __global__ void __launch_bounds__(256) bwd_pre_tc_kernel(TensorRef hf_t, TensorRef hs_t, TensorRef gf_t,
                                                         TensorRef gs_t, int Hq, int N, float c2,
                                                         __nv_bfloat16* dhf, __nv_bfloat16* dhs, float* Df,
                                                         float* Ds, float* partials, const float* lse_full,
-                                                        const float* lse_sel, float4* scal) {
-  constexpr int PER = HD / 32;
+                                                        const float* lse_sel, float* lse2f, float* lse2s) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t row = (int64_t)blockIdx.x * 8 + w;
   const int t = (int)(row % N), bh = (int)(row / N), b = bh / Hq, h = bh % Hq;
-  const T* hf = row_ptr<T>(hf_t, b, h, t);
-  const T* hs = row_ptr<T>(hs_t, b, h, t);
-  const T* gf = gf_t.p ? row_ptr<T>(gf_t, b, h, t) : nullptr;
-  const T* gs = gs_t.p ? row_ptr<T>(gs_t, b, h, t) : nullptr;
+  const int c = 4 * lane;
+  auto load4 = [](const __nv_bfloat16* p, float (&x)[4]) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    x[0] = __uint_as_float(v.x << 16);
+    x[1] = __uint_as_float(v.x & 0xffff0000u);
+    x[2] = __uint_as_float(v.y << 16);
+    x[3] = __uint_as_float(v.y & 0xffff0000u);
+  };
+  float xf[4], xs[4], gf[4] = {0.f, 0.f, 0.f, 0.f}, gs[4] = {0.f, 0.f, 0.f, 0.f};
+  load4(row_ptr<__nv_bfloat16>(hf_t, b, h, t) + c, xf);
+  load4(row_ptr<__nv_bfloat16>(hs_t, b, h, t) + c, xs);
+  if (gf_t.p) load4(row_ptr<__nv_bfloat16>(gf_t, b, h, t) + c, gf);
+  if (gs_t.p) load4(row_ptr<__nv_bfloat16>(gs_t, b, h, t) + c, gs);
   float sq = 0.f, df = 0.f, ds = 0.f;
+  uint32_t of[2], os[2];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) {
-    const int c = lane + 32 * e;
-    const float xf = to_f32(hf[c]), xs = to_f32(hs[c]);
-    const float diff = xf - xs;
-    sq = fmaf(diff, diff, sq);
-    const float vf = (gf ? to_f32(gf[c]) : 0.f) + c2 * diff;
-    const float vs = (gs ? to_f32(gs[c]) : 0.f) - c2 * diff;
-    const __nv_bfloat16 bf = __float2bfloat16_rn(vf), bs = __float2bfloat16_rn(vs);
+  for (int e = 0; e < 4; e += 2) {
+    float bf[2], bs[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float diff = xf[e + k] - xs[e + k];
+      sq = fmaf(diff, diff, sq);
+      bf[k] = gf[e + k] + c2 * diff;
+      bs[k] = gs[e + k] - c2 * diff;
+    }
+    of[e / 2] = pack_bf16(bf[0], bf[1]);
+    os[e / 2] = pack_bf16(bs[0], bs[1]);
     // D is formed from the rounded values the MMAs will see.
-    df = fmaf(__bfloat162float(bf), xf, df);
-    ds = fmaf(__bfloat162float(bs), xs, ds);
-    dhf[row * HD + c] = bf;
-    dhs[row * HD + c] = bs;
+    df = fmaf(__uint_as_float(of[e / 2] << 16), xf[e], df);
+    df = fmaf(__uint_as_float(of[e / 2] & 0xffff0000u), xf[e + 1], df);
+    ds = fmaf(__uint_as_float(os[e / 2] << 16), xs[e], ds);
+    ds = fmaf(__uint_as_float(os[e / 2] & 0xffff0000u), xs[e + 1], ds);
   }
+  *reinterpret_cast<uint2*>(dhf + row * HD + c) = make_uint2(of[0], of[1]);
+  *reinterpret_cast<uint2*>(dhs + row * HD + c) = make_uint2(os[0], os[1]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     sq += __shfl_xor_sync(0xffffffffu, sq, off);
@@ -85,10 +107,10 @@ __global__ void __launch_bounds__(256) bwd_pre_tc_kernel(TensorRef hf_t, TensorR
     Df[row] = df;
     Ds[row] = ds;
     part[w] = sq;
-    // {lse_full, lse_sel} in base 2 (an empty selected set maps to +inf, so
-    // 2^(x - lse) is 0 there), then D_f, D_s: one 16-byte load per query.
+    // lse in base 2; an empty selected set maps to +inf, so 2^(x - lse) is 0.
     const float ls = lse_sel[row];
-    scal[row] = make_float4(lse_full[row] * kLog2e, ls == kNegInf ? __builtin_huge_valf() : ls * kLog2e, df, ds);
+    lse2f[row] = lse_full[row] * kLog2e;
+    lse2s[row] = ls == kNegInf ? __builtin_huge_valf() : ls * kLog2e;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -99,398 +121,199 @@ __global__ void __launch_bounds__(256) bwd_pre_tc_kernel(TensorRef hf_t, TensorR
   }
 }
 
-// Both warps of a lane quarter (w, w+4) reach this point before either
-// continues; bounded like every other wait.  `uses` counts this warp's
-// passes, which the partner matches one for one.
-__device__ __forceinline__ bool pair_sync(uint64_t* bar, uint32_t& uses, int lane, volatile int* abort) {
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, uses & 1u, abort);
-  ++uses;
-  tc_fence_after();
-  return ok;
-}
-
 struct BwdTcParams {
   TensorRef dq, dk, dv;     // outputs (bf16, strided)
-  const float* lse_full;    // [B,Hq,N]
-  const float* lse_sel;
-  const float* Df;          // [B,Hq,N]
-  const float* Ds;
+  const float* lse2[2];     // [B,Hq,N] per stream (0 = full, 1 = sparse), base 2
+  const float* D[2];        // [B,Hq,N] per stream
   const uint32_t* mask;     // [B,Hq,n,words]
-  const float4* scal;       // [B,Hq,N]: {lse2_full, lse2_sel, D_f, D_s}
   int words;
   int32_t* status;
-  int Hq, g, N, n, s;
+  int Hq, g, N, n, s, NT;   // NT = number of 128-row tiles
   float c;                  // scale * log2(e)
   float scale;
 };
 
-__device__ __forceinline__ bool sel_bit(const BwdTcParams& p, int b, int h, int i, int j) {
-  const uint32_t w = __ldg(p.mask + (((int64_t)b * p.Hq + h) * p.n + i) * p.words + (j >> 5));
-  return (w >> (j & 31)) & 1u;
+__device__ __forceinline__ uint32_t mask_word(const BwdTcParams& p, int b, int h, int i, int j) {
+  return __ldg(p.mask + (((int64_t)b * p.Hq + h) * p.n + i) * p.words + (j >> 5));
 }
 
-// State of a (query block i, key block j) pair: 0 no causal key, 1 selected, 2 dropped.
-__device__ __forceinline__ int pair_state(const BwdTcParams& p, int b, int h, int i, bool qvalid, int j) {
-  if (!qvalid || j > i) return 0;
-  return sel_bit(p, b, h, i, j) ? 1 : 2;
-}
-
-// P / dS of one 32-column slice of a dK/dV step (keys in lanes, queries in
-// columns).  SEL: the slice's key block is selected for the query block, so
-// the sparse stream contributes; DIAG: the slice touches the causal diagonal.
-template <bool SEL, bool DIAG>
-__device__ __forceinline__ void dkv_slice(const uint32_t (&rs)[32], const uint32_t (&rf)[32],
-                                          const uint32_t (&rp)[32], const float4* sc, int u, int tq0, float c,
-                                          uint32_t (&pf_pk)[16], uint32_t (&ps_pk)[16], uint32_t (&ds_pk)[16]) {
+// Which (query block, key block) pairs of the 128 x 128 tile (qt, kt) of query
+// head h the sparse stream holds: bit 2*qh + kh for the 64-row halves (block
+// 64), all four bits for block 128.  Blocks past the end and key blocks after
+// the query block are never set.
+__device__ __forceinline__ uint32_t tile_bits(const BwdTcParams& p, int b, int h, int qt, int kt) {
+  if (p.s == 128) {
+    if (kt > qt || qt >= p.n) return 0u;
+    return ((mask_word(p, b, h, qt, kt) >> (kt & 31)) & 1u) ? 0xFu : 0u;
+  }
+  uint32_t bits = 0;
 #pragma unroll
-  for (int k = 0; k < 32; k += 2) {
-    float pf[2], ps[2], dsv[2];
+  for (int qh = 0; qh < 2; ++qh) {
+    const int i = 2 * qt + qh;
+    if (i >= p.n) continue;
+    const uint32_t wd = mask_word(p, b, h, i, 2 * kt);
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float4 v4 = sc[k + e];  // lse2_f, lse2_s, D_f, D_s of query tq0 + k + e
-      const float x = __uint_as_float(rs[k + e]);
-      pf[e] = ex2(fmaf(x, c, -v4.x));
-      if (DIAG && u > tq0 + k + e) pf[e] = 0.f;
-      dsv[e] = pf[e] * (__uint_as_float(rf[k + e]) - v4.z);
-      ps[e] = 0.f;
-      if (SEL) {
-        ps[e] = ex2(fmaf(x, c, -v4.y));
-        if (DIAG && u > tq0 + k + e) ps[e] = 0.f;
-        dsv[e] = fmaf(ps[e], __uint_as_float(rp[k + e]) - v4.w, dsv[e]);
-      }
+    for (int kh = 0; kh < 2; ++kh) {
+      const int j = 2 * kt + kh;
+      if (j <= i && ((wd >> (j & 31)) & 1u)) bits |= 1u << (2 * qh + kh);
     }
-    pf_pk[k / 2] = pack_bf16(pf[0], pf[1]);
-    if (SEL) ps_pk[k / 2] = pack_bf16(ps[0], ps[1]);
-    ds_pk[k / 2] = pack_bf16(dsv[0], dsv[1]);
   }
+  return bits;
 }
 
-// dS of one 32-key slice of a dQ tile (queries in lanes, keys in columns).
-template <bool SEL, bool DIAG>
-__device__ __forceinline__ void dq_slice(const uint32_t (&rs)[32], const uint32_t (&rf)[32],
-                                         const uint32_t (&rp)[32], float l2f, float l2s, float Dfv, float Dsv,
-                                         int u0, int t, float c, uint32_t (&pk)[16]) {
-#pragma unroll
-  for (int k = 0; k < 32; k += 2) {
-    float ds[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float x = __uint_as_float(rs[k + e]);
-      float pf = ex2(fmaf(x, c, -l2f));
-      if (DIAG && u0 + k + e > t) pf = 0.f;
-      ds[e] = pf * (__uint_as_float(rf[k + e]) - Dfv);
-      if (SEL) {
-        float ps = ex2(fmaf(x, c, -l2s));
-        if (DIAG && u0 + k + e > t) ps = 0.f;
-        ds[e] = fmaf(ps, __uint_as_float(rp[k + e]) - Dsv, ds[e]);
-      }
-    }
-    pk[k / 2] = pack_bf16(ds[0], ds[1]);
-  }
-}
-
-// ================================================================ dQ kernel
-namespace dq {
-constexpr int BM = 128;  // query rows
-constexpr int BK = 64;   // keys per tile
-constexpr int NS = 3;
-constexpr int TILE_A = BM * HD * 2;  // 32 KB: Q, dh_f, dh_s tiles
-constexpr int TILE_K = BK * HD * 2;  // 16 KB: K or V tile
-constexpr int OFF_Q = 0, OFF_DHF = TILE_A, OFF_DHS = 2 * TILE_A;
-constexpr int OFF_K = 3 * TILE_A;
-constexpr int OFF_V = OFF_K + NS * TILE_K;
-constexpr int OFF_MISC = OFF_V + NS * TILE_K;
-constexpr int SMEM = OFF_MISC + 1024 + 4096 + 1024;
-constexpr uint32_t COL_DQ = 0, COL_S = 128, COL_DPF = 256, COL_DPS = 384;
-constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BK, false, false);
-constexpr uint32_t IDESC_DQ = idesc_bf16_f32(BM, HD, false, true);
-
-constexpr int MAX_TILES = 4096;  // N / 64 for n <= 2048 and block <= 128
-struct Misc {
-  uint64_t a_full;
-  uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
-  uint64_t s_full[2], ds_full[2];
-  uint64_t pair[4];  // warps w and w+4: both hold their inputs before either writes
-  uint64_t done, drain;
-  uint32_t tmem_base;
-  int abort;
-  uint8_t state[MAX_TILES];  // per key tile: half-0 state | half-1 state << 2
-};
-static_assert(sizeof(Misc) <= SMEM - OFF_MISC - 1024, "dq shared-memory budget");
-}  // namespace dq
-
-__global__ void __launch_bounds__(NTHREADS, 1)
-    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDhf,
-                     const __grid_constant__ CUtensorMap tmDhs, BwdTcParams p) {
-  using namespace dq;
-  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
-  // Used directly (no pointer arithmetic on the address) so that accesses
-  // through it stay shared-memory loads; TMA tiles with 128-byte swizzle need
-  // the 1024-byte alignment, which is checked rather than assumed.
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = smem_raw;
-  if (smem_u32(smem) & 1023u) {
-    if (threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_UNSUPPORTED);
-    return;
-  }
-  dq::Misc& M = *reinterpret_cast<dq::Misc*>(smem + OFF_MISC);
-  volatile int* abort = &M.abort;
+// Block-wide compaction: every thread offers one candidate (`keep`, `entry`);
+// kept entries are appended to list[] in candidate order.  `total` is the
+// running count (same value in every thread); wsum is 10 ints of scratch.
+template <typename E>
+__device__ __forceinline__ void compact_append(bool keep, uint32_t entry, E* list, int cap, int* wsum,
+                                               int& total) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = (int)(gridDim.x - 1 - blockIdx.x);
-  const int h = blockIdx.y, b = blockIdx.z, kvh = h / p.g;
-  const int q0 = qt * BM;
-  const int q_end = min(q0 + BM, p.N);
-  const int T = (q_end + BK - 1) / BK;
-  // query blocks of the two 64-row halves
-  const int ib0 = q0 / p.s, ib1 = (q0 + 64) / p.s;
-  const bool valid1 = q0 + 64 < p.N;
-
-  if (threadIdx.x == 0) {
-    mbar_init(&M.a_full, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&M.k_full[s], 1);
-      mbar_init(&M.k_empty[s], 1);
-      mbar_init(&M.v_full[s], 1);
-      mbar_init(&M.v_empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&M.s_full[s], 1);
-      mbar_init(&M.ds_full[s], 8);
-    }
-    for (int q = 0; q < 4; ++q) mbar_init(&M.pair[q], 2);
-    mbar_init(&M.done, 1);
-    mbar_init(&M.drain, 1);
-    M.abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == WARP_MMA) {
-    tmem_alloc(&M.tmem_base, 512);
-    tmem_relinquish();
-  }
-  // (half, key block) states of every key tile, read once from the mask
-  for (int j = threadIdx.x; j < T; j += NTHREADS) {
-    const int jb = (j * BK) / p.s;
-    M.state[j] = (uint8_t)(pair_state(p, b, h, ib0, true, jb) | (pair_state(p, b, h, ib1, valid1, jb) << 2));
-  }
-  tc_fence_before();
+  const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+  if (lane == 0) wsum[warp] = __popc(bal);
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = M.tmem_base;
-  uint8_t* sQ = smem + OFF_Q;
-  uint8_t* sDhf = smem + OFF_DHF;
-  uint8_t* sDhs = smem + OFF_DHS;
-  uint8_t* sK = smem + OFF_K;
-  uint8_t* sV = smem + OFF_V;
-
-  if (warp == WARP_TMA) {
-    if (lane == 0) {
-      prefetch_tensormap(&tmQ);
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      mbar_expect_tx(&M.a_full, 3 * TILE_A);
-      tma_load_4d(sQ, &tmQ, &M.a_full, 0, q0, h, b);
-      tma_load_4d(sQ + TILE_A / 2, &tmQ, &M.a_full, 64, q0, h, b);
-      tma_load_4d(sDhf, &tmDhf, &M.a_full, 0, q0, h, b);
-      tma_load_4d(sDhf + TILE_A / 2, &tmDhf, &M.a_full, 64, q0, h, b);
-      tma_load_4d(sDhs, &tmDhs, &M.a_full, 0, q0, h, b);
-      tma_load_4d(sDhs + TILE_A / 2, &tmDhs, &M.a_full, 64, q0, h, b);
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < T; ++j) {
-        const int st = j % NS;
-        const uint32_t use = (uint32_t)(j / NS);
-        if (j >= NS && !mbar_wait(&M.k_empty[st], (use - 1) & 1u, abort)) break;
-        mbar_expect_tx(&M.k_full[st], TILE_K);
-        tma_load_4d(sK + st * TILE_K, &tmK, &M.k_full[st], 0, j * BK, kvh, b);
-        tma_load_4d(sK + st * TILE_K + TILE_K / 2, &tmK, &M.k_full[st], 64, j * BK, kvh, b);
-        k_issued = j + 1;
-        if (j >= NS && !mbar_wait(&M.v_empty[st], (use - 1) & 1u, abort)) break;
-        mbar_expect_tx(&M.v_full[st], TILE_K);
-        tma_load_4d(sV + st * TILE_K, &tmV, &M.v_full[st], 0, j * BK, kvh, b);
-        tma_load_4d(sV + st * TILE_K + TILE_K / 2, &tmV, &M.v_full[st], 64, j * BK, kvh, b);
-        v_issued = j + 1;
-      }
-      int dummy = 0;
-      mbar_wait(&M.a_full, 0, &dummy);
-      for (int j = (k_issued > NS ? k_issued - NS : 0); j < k_issued; ++j) {
-        dummy = 0;
-        mbar_wait(&M.k_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
-      }
-      for (int j = (v_issued > NS ? v_issued - NS : 0); j < v_issued; ++j) {
-        dummy = 0;
-        mbar_wait(&M.v_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
-      }
-    }
-  } else if (warp == WARP_MMA) {
-    if (lane == 0) {
-      const uint32_t aq = smem_u32(sQ), af = smem_u32(sDhf), as = smem_u32(sDhs);
-      bool ok = mbar_wait(&M.a_full, 0, abort);
-      bool started = false;
-      auto issue_dq = [&](int jj) -> bool {
-        const int sb = jj & 1;
-        if (!mbar_wait(&M.ds_full[sb], (uint32_t)(jj >> 1) & 1u, abort)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + (jj % NS) * TILE_K);
+  int before = 0, all = 0;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(k_addr + kk * 16 * 128, TILE_K / 2, 1024);
-          mma_ts(tmem + COL_DQ, tmem + COL_S + sb * 64 + kk * 8, bdesc, IDESC_DQ, (started || kk > 0) ? 1u : 0u);
-        }
-        started = true;
-        tc_commit(&M.k_empty[jj % NS]);
-        return true;
-      };
-      for (int j = 0; ok && j < T; ++j) {
-        const int st = j % NS, sb = j & 1;
-        const uint32_t ph = (uint32_t)(j / NS) & 1u;
-        if (!mbar_wait(&M.k_full[st], ph, abort) || !mbar_wait(&M.v_full[st], ph, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int stj = M.state[j];
-        const bool any_sel = (stj & 3) == 1 || (stj >> 2) == 1;
-        const uint32_t k_addr = smem_u32(sK + st * TILE_K), v_addr = smem_u32(sV + st * TILE_K);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * (TILE_A / 2) + (kk & 3) * 32;
-          const uint32_t offb = (kk >> 2) * (TILE_K / 2) + (kk & 3) * 32;
-          const uint64_t kdesc = smem_desc_sw128(k_addr + offb, 16, 1024);
-          const uint64_t vdesc = smem_desc_sw128(v_addr + offb, 16, 1024);
-          mma_ss(tmem + COL_S + sb * 64, smem_desc_sw128(aq + offa, 16, 1024), kdesc, IDESC_S, kk > 0);
-          mma_ss(tmem + COL_DPF + sb * 64, smem_desc_sw128(af + offa, 16, 1024), vdesc, IDESC_S, kk > 0);
-          if (any_sel) mma_ss(tmem + COL_DPS + sb * 64, smem_desc_sw128(as + offa, 16, 1024), vdesc, IDESC_S, kk > 0);
-        }
-        tc_commit(&M.s_full[sb]);
-        tc_commit(&M.v_empty[st]);
-        if (j >= 1 && !issue_dq(j - 1)) {
-          ok = false;
-          break;
-        }
-      }
-      if (ok && T >= 1) issue_dq(T - 1);
-      tc_commit(&M.done);
-      tc_commit(&M.drain);
-      int dummy = 0;
-      mbar_wait(&M.drain, 0, &dummy);
-    }
-  } else {
-    const int quarter = warp & 3, ch = warp >> 2;  // lanes 32*quarter.., key columns 32*ch..
-    const int row = quarter * 32 + lane;
-    const int t = q0 + row;
-    const int half = quarter >> 1;
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const bool in_range = t < p.N;
-    const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + (in_range ? t : 0);
-    const float4 sc = p.scal[ro];
-    const float l2f = sc.x, l2s = sc.y, Dfv = sc.z, Dsv = sc.w;
-    uint32_t pair_uses = 0;
-    bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&M.s_full[sb], (uint32_t)(j >> 1) & 1u, abort)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int mine = half ? (M.state[j] >> 2) : (M.state[j] & 3);
-      const uint32_t c0 = 32 * ch;
-      uint32_t pk[16];
-      if (mine == 0) {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = 0u;
-      } else {
-        uint32_t rs[32], rf[32], rp[32];
-        tmem_ld32(lane_base + COL_S + sb * 64 + c0, rs);
-        tmem_ld32(lane_base + COL_DPF + sb * 64 + c0, rf);
-        if (mine == 1) tmem_ld32(lane_base + COL_DPS + sb * 64 + c0, rp);
-        tmem_wait_ld();
-        // dS overwrites the S columns this pair reads: both warps must hold
-        // their inputs before either writes.
-        if (!pair_sync(&M.pair[quarter], pair_uses, lane, abort)) {
-          ok = false;
-          break;
-        }
-        const int u0 = j * BK + (int)c0;
-        const bool diag = u0 + 31 > q0 + quarter * 32;  // some key of the slice is after some row
-        if (mine == 1) {
-          if (diag) dq_slice<true, true>(rs, rf, rp, l2f, l2s, Dfv, Dsv, u0, t, p.c, pk);
-          else dq_slice<true, false>(rs, rf, rp, l2f, l2s, Dfv, Dsv, u0, t, p.c, pk);
-        } else {
-          if (diag) dq_slice<false, true>(rs, rf, rp, l2f, l2s, Dfv, Dsv, u0, t, p.c, pk);
-          else dq_slice<false, false>(rs, rf, rp, l2f, l2s, Dfv, Dsv, u0, t, p.c, pk);
-        }
-      }
-      tmem_st16(lane_base + COL_S + sb * 64 + 16 * ch, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&M.ds_full[sb]);
-    }
-    if (ok && mbar_wait(&M.done, 0, abort)) {
-      tc_fence_after();
-      __nv_bfloat16* out = in_range ? row_ptr_w<__nv_bfloat16>(p.dq, b, h, t) : nullptr;
-#pragma unroll 1
-      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + COL_DQ + c0, r);
-        tmem_wait_ld();
-        if (in_range) {
-          uint32_t o[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            o[c] = pack_bf16(__uint_as_float(r[2 * c]) * p.scale, __uint_as_float(r[2 * c + 1]) * p.scale);
-          uint4* dst = reinterpret_cast<uint4*>(out + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        }
-      }
-    }
+  for (int w = 0; w < NTHREADS / 32; ++w) {
+    const int c = wsum[w];
+    before += (w < warp) ? c : 0;
+    all += c;
   }
-  tc_fence_before();
+  const int pos = total + before + __popc(bal & ((1u << lane) - 1u));
+  if (keep && pos < cap) list[pos] = (E)entry;
   __syncthreads();
-  if (M.abort && threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_TIMEOUT);
-  if (warp == WARP_MMA) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+  total += all;
+}
+
+// P = 2^(x c - lse2[col]) for 32 columns of one row, packed to bf16 pairs.
+// MASKED: columns with keep(col) false are 0.
+template <bool MASKED, typename Keep>
+__device__ __forceinline__ void p_block(const uint32_t (&x)[32], const float* lse2, float c, Keep keep,
+                                        uint32_t* pk) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 4) {
+    const float4 l = *reinterpret_cast<const float4*>(lse2 + k);
+    float v[4];
+    v[0] = ex2(fmaf(__uint_as_float(x[k]), c, -l.x));
+    v[1] = ex2(fmaf(__uint_as_float(x[k + 1]), c, -l.y));
+    v[2] = ex2(fmaf(__uint_as_float(x[k + 2]), c, -l.z));
+    v[3] = ex2(fmaf(__uint_as_float(x[k + 3]), c, -l.w));
+    if (MASKED) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (!keep(k + e)) v[e] = 0.f;
+    }
+    pk[k / 2] = pack_bf16(v[0], v[1]);
+    pk[k / 2 + 1] = pack_bf16(v[2], v[3]);
   }
+}
+
+// dS = P (dP - D[col]) for 32 columns, P given as packed bf16 pairs.
+__device__ __forceinline__ void ds_block(const uint32_t (&y)[32], const float* D, const uint32_t* pk,
+                                         uint32_t* out) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 4) {
+    const float4 dd = *reinterpret_cast<const float4*>(D + k);
+    const float p0 = __uint_as_float(pk[k / 2] << 16), p1 = __uint_as_float(pk[k / 2] & 0xffff0000u);
+    const float p2 = __uint_as_float(pk[k / 2 + 1] << 16), p3 = __uint_as_float(pk[k / 2 + 1] & 0xffff0000u);
+    out[k / 2] = pack_bf16(p0 * (__uint_as_float(y[k]) - dd.x), p1 * (__uint_as_float(y[k + 1]) - dd.y));
+    out[k / 2 + 1] = pack_bf16(p2 * (__uint_as_float(y[k + 2]) - dd.z), p3 * (__uint_as_float(y[k + 3]) - dd.w));
+  }
+}
+
+// Same with one D for the whole row (dQ kernel).
+__device__ __forceinline__ void ds_block_row(const uint32_t (&y)[32], float D, const uint32_t* pk,
+                                             uint32_t* out) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    const float p0 = __uint_as_float(pk[k / 2] << 16), p1 = __uint_as_float(pk[k / 2] & 0xffff0000u);
+    out[k / 2] = pack_bf16(p0 * (__uint_as_float(y[k]) - D), p1 * (__uint_as_float(y[k + 1]) - D));
+  }
+}
+
+// P for 32 columns of one row with one lse for the row (dQ kernel).
+template <bool MASKED, typename Keep>
+__device__ __forceinline__ void p_block_row(const uint32_t (&x)[32], float l2, float c, Keep keep,
+                                            uint32_t* pk) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    float v0 = ex2(fmaf(__uint_as_float(x[k]), c, -l2));
+    float v1 = ex2(fmaf(__uint_as_float(x[k + 1]), c, -l2));
+    if (MASKED) {
+      if (!keep(k)) v0 = 0.f;
+      if (!keep(k + 1)) v1 = 0.f;
+    }
+    pk[k / 2] = pack_bf16(v0, v1);
+  }
+}
+
+// SS product of two 128 x 128 K-major tiles (reduction over d = 128).
+__device__ __forceinline__ void mma_tile_ss(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+    mma_ss(d_tmem, smem_desc_sw128(a_smem + off, 16, 1024), smem_desc_sw128(b_smem + off, 16, 1024), IDESC_S,
+           kk > 0 ? 1u : 0u);
+  }
+}
+
+// TS product over d = 128: A = 128 rows x 128 bf16 in TMEM (d columns 16kk..
+// packed at column 8kk), B = a 128 x 128 K-major smem tile.
+__device__ __forceinline__ void mma_tile_ts_k(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem) {
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+    mma_ts(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_smem + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+  }
+}
+
+// TS product: D (+)= A[TMEM, 128 x 128 bf16 as written by the P / dS warps]
+// x B[smem tile, rows = reduction index, MN-major].  The warp with column
+// range 64h.. leaves its 64 packed values in columns 64h .. 64h+31.
+__device__ __forceinline__ void mma_tile_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < TILE / 16; ++kk) {
+    const uint32_t a = a_tmem + 64 * (kk >> 2) + 8 * (kk & 3);
+    mma_ts(d_tmem, a, smem_desc_sw128(b_smem + kk * 2048, HALF, 1024), IDESC_ACC,
+           (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&r)[32], float mult) {
+  uint32_t o[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) o[c] = pack_bf16(__uint_as_float(r[2 * c]) * mult, __uint_as_float(r[2 * c + 1]) * mult);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) d4[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
 }
 
 // ================================================================ dK / dV kernel
 namespace dkv {
-constexpr int BKEY = 128;  // keys per CTA
-constexpr int BQ = 64;     // queries per step
-constexpr int NS = 3;
-constexpr int TILE_KV = BKEY * HD * 2;  // 32 KB: K or V
-constexpr int TILE_Q = BQ * HD * 2;     // 16 KB: Q, dh_f or dh_s step tile
-constexpr int SCAL = BQ * 16;           // {lse2_f, lse2_s, D_f, D_s} of one step (1 KB)
-constexpr int MAX_STEPS = 8192;         // g * N / 64
-constexpr int STAGE = 3 * TILE_Q + SCAL;
-constexpr int OFF_K = 0, OFF_V = TILE_KV;
-constexpr int OFF_STAGE = 2 * TILE_KV;
+constexpr int NS = 2;
+constexpr int OFF_K = 0, OFF_V = TILE_B;
+constexpr int SCAL = TILE * 4;                 // 128 floats
+// A stage holds one step's Q tile with its lse2 and D (released after dK) and
+// its dh tile (released after dV, earlier), each with its own barriers.
+constexpr int STAGE = 2 * TILE_B + 2 * SCAL;
+constexpr int OFF_STAGE = 2 * TILE_B;
 constexpr int OFF_MISC = OFF_STAGE + NS * STAGE;
-constexpr int SMEM = OFF_MISC + 1024 + MAX_STEPS + 1024;
-// TMEM: dK, dV, then two step buffers of [S^T 64 | dP_f^T 64] columns.  A step
-// with a selected pair puts dP_s^T in the other buffer's dP_f^T columns.
-constexpr uint32_t COL_DK = 0, COL_DV = 128, COL_BUF = 256, BUF_COLS = 128, OFF_DP = 64;
-constexpr uint32_t IDESC_S = idesc_bf16_f32(BKEY, BQ, false, false);
-constexpr uint32_t IDESC_ACC = idesc_bf16_f32(BKEY, HD, false, true);
+constexpr int MAX_SPARSE = 4096;               // g * NT
+// TMEM columns: dK, dV accumulators, S^T (P^T over it), dP^T (dS^T over it).
+constexpr uint32_t COL_DK = 0, COL_DV = 128, COL_S = 256, COL_DP = 384;
 
 struct Misc {
   uint64_t kv_full;
-  uint64_t full[NS], empty[NS];
-  uint64_t s_full[2], p_full[2], done, drain;
-  uint64_t pair[4];  // warps w and w+4: both hold their inputs before either writes
+  uint64_t q_full[NS], q_empty[NS], dh_full[NS], dh_empty[NS];
+  uint64_t s_full, dp_full, p_full, ds_full, done, drain;
   uint32_t tmem_base;
   int abort;
-  // per step: key-half-0 state | key-half-1 state << 2 | any selected << 4
-  uint8_t state[MAX_STEPS];
+  int wsum[NTHREADS / 32];
+  // sparse steps: (head * query tiles + query tile offset) << 4 | pair bits
+  uint16_t list[MAX_SPARSE];
 };
-static_assert(sizeof(Misc) <= SMEM - OFF_MISC - 1024, "dkv shared-memory budget");
+constexpr int SMEM = OFF_MISC + (int)sizeof(Misc);
+static_assert(SMEM <= kMaxSmem, "dkv shared-memory budget");
+static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
 }  // namespace dkv
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -511,28 +334,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   dkv::Misc& M = *reinterpret_cast<dkv::Misc*>(smem + OFF_MISC);
   volatile int* abort = &M.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = (int)blockIdx.x;  // lightest-last order: low key tiles have the most query tiles
+  const int kt = (int)blockIdx.x;  // low key tiles have the most query tiles and launch first
   const int kvh = blockIdx.y, b = blockIdx.z;
-  const int u0 = kt * BKEY;
-  // key blocks of the two 64-key halves
-  const int kb0 = u0 / p.s, kb1 = (u0 + 64) / p.s;
-  const bool kvalid1 = u0 + 64 < p.N;
-  const int nq = p.N / BQ;
-  const int qt0 = u0 / BQ;               // first query tile with a causal pair
-  const int steps_per_head = nq - qt0;
-  const int steps = p.g * steps_per_head;
+  const int u0 = kt * TILE;
+  const int nqt = p.NT - kt;       // causal query tiles per head
+  const int n_full = p.g * nqt;
+  auto stage_ptr = [&](int st) { return smem + OFF_STAGE + st * STAGE; };
 
   if (threadIdx.x == 0) {
     mbar_init(&M.kv_full, 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&M.full[s], 1);
-      mbar_init(&M.empty[s], 1);
+      mbar_init(&M.q_full[s], 1);
+      mbar_init(&M.q_empty[s], 1);
+      mbar_init(&M.dh_full[s], 1);
+      mbar_init(&M.dh_empty[s], 1);
     }
-    for (int s2 = 0; s2 < 2; ++s2) {
-      mbar_init(&M.s_full[s2], 1);
-      mbar_init(&M.p_full[s2], 8);
-    }
-    for (int q = 0; q < 4; ++q) mbar_init(&M.pair[q], 2);
+    mbar_init(&M.s_full, 1);
+    mbar_init(&M.dp_full, 1);
+    mbar_init(&M.p_full, 8);
+    mbar_init(&M.ds_full, 8);
     mbar_init(&M.done, 1);
     mbar_init(&M.drain, 1);
     M.abort = 0;
@@ -542,220 +362,235 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_alloc(&M.tmem_base, 512);
     tmem_relinquish();
   }
-  // Steps walk (head hh, query tile qt) with qt fastest.  Their states are
-  // read once from the mask into shared memory.
-  for (int it = threadIdx.x; it < steps; it += NTHREADS) {
-    const int h = kvh * p.g + it / steps_per_head;
-    const int i = ((qt0 + it % steps_per_head) * BQ) / p.s;
-    const int s0 = pair_state(p, b, h, i, true, kb0);
-    const int s1 = kvalid1 ? pair_state(p, b, h, i, true, kb1) : 0;
-    M.state[it] = (uint8_t)(s0 | (s1 << 2) | ((s0 == 1 || s1 == 1) ? 16 : 0));
+  // A ragged last query tile copies only its valid scalars; the rest of the
+  // scalar slots must hold finite values (their columns are masked).
+  for (int i = threadIdx.x; i < NS * 2 * TILE; i += NTHREADS)
+    reinterpret_cast<float*>(stage_ptr(i / (2 * TILE)) + 2 * TILE_B)[i % (2 * TILE)] = 0.f;
+  // Sparse-stream steps: (head, query tile) pairs holding a selected pair.
+  int n_sparse = 0;
+  for (int base = 0; base < n_full; base += NTHREADS) {
+    const int it = base + (int)threadIdx.x;
+    uint32_t bits = 0;
+    if (it < n_full) bits = tile_bits(p, b, kvh * p.g + it / nqt, kt + it % nqt, kt);
+    compact_append(bits != 0, ((uint32_t)it << 4) | bits, M.list, MAX_SPARSE, M.wsum, n_sparse);
   }
+  n_sparse = min(n_sparse, MAX_SPARSE);
+  const int T = n_full + n_sparse;
+  // The scalar slots are also written by the async proxy (bulk copies).
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = M.tmem_base;
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
-  auto stage_ptr = [&](int st) { return smem + OFF_STAGE + st * STAGE; };
+  // step j -> (head within the group, query tile, stream, pair bits)
+  auto decode = [&](int j, int& hh, int& qt, int& sp, uint32_t& bits) {
+    int it;
+    if (j < n_full) {
+      it = j;
+      sp = 0;
+      bits = 0xFu;
+    } else {
+      const uint32_t e = M.list[j - n_full];
+      it = (int)(e >> 4);
+      sp = 1;
+      bits = e & 0xFu;
+    }
+    hh = it / nqt;
+    qt = kt + it % nqt;
+  };
 
   if (warp == WARP_TMA) {
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmDhf);
       prefetch_tensormap(&tmDhs);
-      mbar_expect_tx(&M.kv_full, 2 * TILE_KV);
+      mbar_expect_tx(&M.kv_full, 2 * TILE_B);
       tma_load_4d(sK, &tmK, &M.kv_full, 0, u0, kvh, b);
-      tma_load_4d(sK + TILE_KV / 2, &tmK, &M.kv_full, 64, u0, kvh, b);
+      tma_load_4d(sK + HALF, &tmK, &M.kv_full, 64, u0, kvh, b);
       tma_load_4d(sV, &tmV, &M.kv_full, 0, u0, kvh, b);
-      tma_load_4d(sV + TILE_KV / 2, &tmV, &M.kv_full, 64, u0, kvh, b);
+      tma_load_4d(sV + HALF, &tmV, &M.kv_full, 64, u0, kvh, b);
       int issued = 0;
-      int h = kvh * p.g, qt = qt0;
-      for (int it = 0; it < steps; ++it) {
-        const int st = it % NS;
-        const uint32_t use = (uint32_t)(it / NS);
-        if (it >= NS && !mbar_wait(&M.empty[st], (use - 1) & 1u, abort)) break;
-        const int t0 = qt * BQ;
-        const bool any = (M.state[it] & 16) != 0;
-        uint8_t* sp = stage_ptr(st);
-        mbar_expect_tx(&M.full[st], (any ? 3 : 2) * TILE_Q + SCAL);
-        tma_load_4d(sp, &tmQ, &M.full[st], 0, t0, h, b);
-        tma_load_4d(sp + TILE_Q / 2, &tmQ, &M.full[st], 64, t0, h, b);
-        tma_load_4d(sp + TILE_Q, &tmDhf, &M.full[st], 0, t0, h, b);
-        tma_load_4d(sp + TILE_Q + TILE_Q / 2, &tmDhf, &M.full[st], 64, t0, h, b);
-        if (any) {
-          tma_load_4d(sp + 2 * TILE_Q, &tmDhs, &M.full[st], 0, t0, h, b);
-          tma_load_4d(sp + 2 * TILE_Q + TILE_Q / 2, &tmDhs, &M.full[st], 64, t0, h, b);
+      for (int j = 0; j < T; ++j) {
+        const int st = j % NS;
+        const uint32_t ph = (uint32_t)(j / NS - 1) & 1u;
+        int hh, qt, sp;
+        uint32_t bits;
+        decode(j, hh, qt, sp, bits);
+        const int h = kvh * p.g + hh, t0 = qt * TILE;
+        uint8_t* sp_ = stage_ptr(st);
+        // dh first: its slot frees after dV, before the Q slot frees after dK
+        if (j >= NS && !mbar_wait(&M.dh_empty[st], ph, abort)) break;
+        const CUtensorMap* md = sp ? &tmDhs : &tmDhf;
+        mbar_expect_tx(&M.dh_full[st], TILE_B);
+        tma_load_4d(sp_ + TILE_B, md, &M.dh_full[st], 0, t0, h, b);
+        tma_load_4d(sp_ + TILE_B + HALF, md, &M.dh_full[st], 64, t0, h, b);
+        if (j >= NS && !mbar_wait(&M.q_empty[st], ph, abort)) {
+          issued = -(j + 1);  // dh of step j issued, Q not
+          break;
         }
+        const int valid = min(TILE, p.N - t0);  // a multiple of 64
+        mbar_expect_tx(&M.q_full[st], TILE_B + 2 * valid * 4);
+        tma_load_4d(sp_, &tmQ, &M.q_full[st], 0, t0, h, b);
+        tma_load_4d(sp_ + HALF, &tmQ, &M.q_full[st], 64, t0, h, b);
         const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + t0;
-        bulk_load(sp + 3 * TILE_Q, p.scal + ro, SCAL, &M.full[st]);
-        issued = it + 1;
-        if (++qt == qt0 + steps_per_head) {
-          qt = qt0;
-          ++h;
-        }
+        bulk_load(sp_ + 2 * TILE_B, p.lse2[sp] + ro, (uint32_t)valid * 4, &M.q_full[st]);
+        bulk_load(sp_ + 2 * TILE_B + SCAL, p.D[sp] + ro, (uint32_t)valid * 4, &M.q_full[st]);
+        issued = j + 1;
       }
+      // no copy may still be in flight when the CTA exits
       int dummy = 0;
       mbar_wait(&M.kv_full, 0, &dummy);
-      for (int it = (issued > NS ? issued - NS : 0); it < issued; ++it) {
+      const int nq = issued < 0 ? -issued - 1 : issued, nd = issued < 0 ? -issued : issued;
+      for (int j = (nq > NS ? nq - NS : 0); j < nq; ++j) {
         dummy = 0;
-        mbar_wait(&M.full[it % NS], (uint32_t)(it / NS) & 1u, &dummy);
+        mbar_wait(&M.q_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
+      }
+      for (int j = (nd > NS ? nd - NS : 0); j < nd; ++j) {
+        dummy = 0;
+        mbar_wait(&M.dh_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
       }
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
       const uint32_t ak = smem_u32(sK), av = smem_u32(sV);
-      bool ok = mbar_wait(&M.kv_full, 0, abort);
-      bool started = false;
-      // dV += P^T dh_f (+ P_s^T dh_s), dK += dS^T Q for step jt (buffer jt & 1).
-      auto accumulate = [&](int jt) -> bool {
-        if (!mbar_wait(&M.p_full[jt & 1], (uint32_t)(jt >> 1) & 1u, abort)) return false;
+      bool ok = mbar_wait(&M.kv_full, 0, abort) && mbar_wait(&M.q_full[0], 0, abort) &&
+                mbar_wait(&M.dh_full[0], 0, abort);
+      if (ok) {
         tc_fence_after();
-        const int st = jt % NS;
-        const uint32_t sq = smem_u32(stage_ptr(st));
-        const uint32_t sf = sq + TILE_Q, ss = sq + 2 * TILE_Q;
-        const uint32_t buf = COL_BUF + (uint32_t)(jt & 1) * BUF_COLS;
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint32_t off = kk * 16 * 128;
-          const uint32_t acc = (started || kk > 0) ? 1u : 0u;
-          mma_ts(tmem + COL_DV, tmem + buf + kk * 8, smem_desc_sw128(sf + off, TILE_Q / 2, 1024), IDESC_ACC, acc);
-          mma_ts(tmem + COL_DK, tmem + buf + OFF_DP + kk * 8, smem_desc_sw128(sq + off, TILE_Q / 2, 1024), IDESC_ACC,
-                 acc);
-        }
-        started = true;
-        if (M.state[jt] & 16) {
-#pragma unroll
-          for (int kk = 0; kk < BQ / 16; ++kk)
-            mma_ts(tmem + COL_DV, tmem + buf + 32 + kk * 8, smem_desc_sw128(ss + kk * 16 * 128, TILE_Q / 2, 1024),
-                   IDESC_ACC, 1u);
-        }
-        tc_commit(&M.empty[st]);
-        return true;
-      };
-      for (int it = 0; ok && it < steps; ++it) {
-        const int st = it % NS, b2 = it & 1;
-        if (!mbar_wait(&M.full[st], (uint32_t)(it / NS) & 1u, abort)) {
-          ok = false;
-          break;
-        }
-        // A selected previous step left its dP_s^T in this step's buffer:
-        // its softmax must be done with it first.
-        if (it >= 1 && (M.state[it - 1] & 16) &&
-            !mbar_wait(&M.p_full[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u, abort)) {
+        const uint32_t s0 = smem_u32(stage_ptr(0));
+        mma_tile_ss(tmem + COL_S, ak, s0);
+        tc_commit(&M.s_full);
+        mma_tile_ss(tmem + COL_DP, av, s0 + TILE_B);
+        tc_commit(&M.dp_full);
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        const int st = j % NS, st1 = (j + 1) % NS;
+        const uint32_t ph1 = (uint32_t)((j + 1) / NS) & 1u;
+        const uint32_t sq = smem_u32(stage_ptr(st)), sq1 = smem_u32(stage_ptr(st1));
+        const bool more = j + 1 < T;
+        // dV += P^T dh once the P warps have written P^T over S^T.
+        if (!mbar_wait(&M.p_full, (uint32_t)j & 1u, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const bool sel = (M.state[it] & 16) != 0;
-        const uint32_t sq = smem_u32(stage_ptr(st));
-        const uint32_t sf = sq + TILE_Q, ss = sq + 2 * TILE_Q;
-        const uint32_t buf = COL_BUF + (uint32_t)b2 * BUF_COLS;
-        const uint32_t other = COL_BUF + (uint32_t)(b2 ^ 1) * BUF_COLS;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * (TILE_KV / 2) + (kk & 3) * 32;
-          const uint32_t offb = (kk >> 2) * (TILE_Q / 2) + (kk & 3) * 32;
-          mma_ss(tmem + buf, smem_desc_sw128(ak + offa, 16, 1024), smem_desc_sw128(sq + offb, 16, 1024), IDESC_S,
-                 kk > 0);
-          mma_ss(tmem + buf + OFF_DP, smem_desc_sw128(av + offa, 16, 1024), smem_desc_sw128(sf + offb, 16, 1024),
-                 IDESC_S, kk > 0);
-        }
-        if (!sel) tc_commit(&M.s_full[b2]);
-        if (it >= 1 && !accumulate(it - 1)) {
-          ok = false;
-          break;
-        }
-        if (sel) {
-          // after dK of the previous step has read its dS^T from `other`
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t offa = (kk >> 2) * (TILE_KV / 2) + (kk & 3) * 32;
-            const uint32_t offb = (kk >> 2) * (TILE_Q / 2) + (kk & 3) * 32;
-            mma_ss(tmem + other + OFF_DP, smem_desc_sw128(av + offa, 16, 1024), smem_desc_sw128(ss + offb, 16, 1024),
-                   IDESC_S, kk > 0);
+        mma_tile_ts(tmem + COL_DV, tmem + COL_S, sq + TILE_B, j > 0);
+        tc_commit(&M.dh_empty[st]);
+        // S^T of the next step reuses the S columns (ordered after dV).
+        if (more) {
+          if (!mbar_wait(&M.q_full[st1], ph1, abort)) {
+            ok = false;
+            break;
           }
-          tc_commit(&M.s_full[b2]);
+          tc_fence_after();
+          mma_tile_ss(tmem + COL_S, ak, sq1);
+          tc_commit(&M.s_full);
+        }
+        // dK += dS^T Q once dS^T is over dP^T.
+        if (!mbar_wait(&M.ds_full, (uint32_t)j & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_tile_ts(tmem + COL_DK, tmem + COL_DP, sq, j > 0);
+        tc_commit(&M.q_empty[st]);
+        if (more) {
+          if (!mbar_wait(&M.dh_full[st1], ph1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_ss(tmem + COL_DP, av, sq1 + TILE_B);
+          tc_commit(&M.dp_full);
         }
       }
-      if (ok && steps >= 1) accumulate(steps - 1);
       tc_commit(&M.done);
       tc_commit(&M.drain);
       int dummy = 0;
       mbar_wait(&M.drain, 0, &dummy);
     }
   } else {
-    const int quarter = warp & 3, ch = warp >> 2;  // lanes 32*quarter.., query columns 32*ch..
-    const int row = quarter * 32 + lane;           // key within the tile
-    const int u = u0 + row;
+    const int quarter = warp & 3, ch = warp >> 2;  // lanes 32*quarter.., query columns 64*ch..
+    const int r = quarter * 32 + lane;             // key row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    int qt = qt0;
-    uint32_t pair_uses = 0;
+    const uint32_t cS = lane_base + COL_S + 64 * ch, cP = lane_base + COL_DP + 64 * ch;
     bool ok = true;
-    for (int it = 0; it < steps; ++it) {
-      const int b2 = it & 1;
-      if (!mbar_wait(&M.s_full[b2], (uint32_t)(it >> 1) & 1u, abort)) {
+    for (int j = 0; j < T; ++j) {
+      const int st = j % NS;
+      int hh, qt, sp;
+      uint32_t bits;
+      decode(j, hh, qt, sp, bits);
+      // the per-query scalars arrived with the Q copy of the stage
+      if (!mbar_wait(&M.q_full[st], (uint32_t)(j / NS) & 1u, abort) ||
+          !mbar_wait(&M.s_full, (uint32_t)j & 1u, abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int st = it % NS;
-      const uint32_t COL_S = COL_BUF + (uint32_t)b2 * BUF_COLS;
-      const uint32_t COL_DPF = COL_S + OFF_DP;
-      const uint32_t COL_DPS = COL_BUF + (uint32_t)(b2 ^ 1) * BUF_COLS + OFF_DP;
-      // the per-query scalars of this stage arrived with the stage's copies
-      if (!mbar_wait(&M.full[st], (uint32_t)(it / NS) & 1u, abort)) {
-        ok = false;
-        break;
-      }
-      const int t0 = qt * BQ;
-      const int stt = M.state[it];
-      const int mine = (quarter >> 1) ? ((stt >> 2) & 3) : (stt & 3);
-      const bool any = (stt & 16) != 0;
-      if (++qt == qt0 + steps_per_head) qt = qt0;
-      const float4* sc = reinterpret_cast<const float4*>(stage_ptr(st) + 3 * TILE_Q);
-      const uint32_t c0 = 32 * ch;
-      // P^T -> S cols [16ch, 16ch+16); P_s^T -> S cols [32+16ch, ...); dS^T -> dP_f cols [16ch, ...).
-      uint32_t pf_pk[16], ps_pk[16], ds_pk[16];
-      if (mine == 0) {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pf_pk[c] = ps_pk[c] = ds_pk[c] = 0u;
-      } else {
-        uint32_t rs[32], rf[32], rp[32];
-        tmem_ld32(lane_base + COL_S + c0, rs);
-        tmem_ld32(lane_base + COL_DPF + c0, rf);
-        if (mine == 1) tmem_ld32(lane_base + COL_DPS + c0, rp);
+      const float* L2 = reinterpret_cast<const float*>(stage_ptr(st) + 2 * TILE_B) + 64 * ch;
+      const float* Dq = reinterpret_cast<const float*>(stage_ptr(st) + 2 * TILE_B + SCAL) + 64 * ch;
+      const bool sel = (bits >> (2 * ch + (r >> 6))) & 1u;
+      const int tq = qt * TILE + 64 * ch;  // first query of this warp's columns
+      const bool diag = qt == kt;
+      const bool ragged = tq + 64 > p.N;
+      uint32_t pk[32];
+      if (sel) {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(cS, x0);
+        tmem_ld32(cS + 32, x1);
         tmem_wait_ld();
-        // the outputs overwrite columns the partner warp reads
-        if (!pair_sync(&M.pair[quarter], pair_uses, lane, abort)) {
-          ok = false;
-          break;
-        }
-        const int tq0 = t0 + (int)c0;                   // first query of the slice
-        const bool diag = u0 + quarter * 32 + 31 > tq0;  // some key of the warp after some query
-        if (mine == 1) {
-          if (diag) dkv_slice<true, true>(rs, rf, rp, sc + c0, u, tq0, p.c, pf_pk, ps_pk, ds_pk);
-          else dkv_slice<true, false>(rs, rf, rp, sc + c0, u, tq0, p.c, pf_pk, ps_pk, ds_pk);
+        if (diag || ragged) {
+          // key u0 + r may attend query tq + col only if r <= 64 ch + col, and the query must exist
+          const int lim = p.N - tq;
+          auto keep0 = [&](int col) { return (!diag || r <= 64 * ch + col) && col < lim; };
+          auto keep1 = [&](int col) { return (!diag || r <= 64 * ch + 32 + col) && 32 + col < lim; };
+          p_block<true>(x0, L2, p.c, keep0, pk);
+          p_block<true>(x1, L2 + 32, p.c, keep1, pk + 16);
         } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) ps_pk[c] = 0u;
-          if (diag) dkv_slice<false, true>(rs, rf, rp, sc + c0, u, tq0, p.c, pf_pk, ps_pk, ds_pk);
-          else dkv_slice<false, false>(rs, rf, rp, sc + c0, u, tq0, p.c, pf_pk, ps_pk, ds_pk);
+          auto all = [](int) { return true; };
+          p_block<false>(x0, L2, p.c, all, pk);
+          p_block<false>(x1, L2 + 32, p.c, all, pk + 16);
         }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      tmem_st16(lane_base + COL_S + 16 * ch, pf_pk);
-      if (any) tmem_st16(lane_base + COL_S + 32 + 16 * ch, ps_pk);
-      tmem_st16(lane_base + COL_DPF + 16 * ch, ds_pk);
+      tmem_st32(cS, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&M.p_full[b2]);
+      if (lane == 0) mbar_arrive(&M.p_full);
+      if (!mbar_wait(&M.dp_full, (uint32_t)j & 1u, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t dk[32];
+      if (sel) {
+        uint32_t y0[32], y1[32];
+        tmem_ld32(cP, y0);
+        tmem_ld32(cP + 32, y1);
+        tmem_wait_ld();
+        ds_block(y0, Dq, pk, dk);
+        ds_block(y1, Dq + 32, pk + 16, dk + 16);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) dk[c] = 0u;
+      }
+      tmem_st32(cP, dk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.ds_full);
     }
     if (ok && mbar_wait(&M.done, 0, abort)) {
       tc_fence_after();
+      const int u = u0 + r;
       const bool store = u < p.N;
-      __nv_bfloat16* ok_ = store ? row_ptr_w<__nv_bfloat16>(p.dk, b, kvh, u) : nullptr;
-      __nv_bfloat16* ov_ = store ? row_ptr_w<__nv_bfloat16>(p.dv, b, kvh, u) : nullptr;
+      __nv_bfloat16* okp = store ? row_ptr_w<__nv_bfloat16>(p.dk, b, kvh, u) : nullptr;
+      __nv_bfloat16* ovp = store ? row_ptr_w<__nv_bfloat16>(p.dv, b, kvh, u) : nullptr;
 #pragma unroll 1
       for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 32) {
         uint32_t rk[32], rv[32];
@@ -763,20 +598,309 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld32(lane_base + COL_DV + c0, rv);
         tmem_wait_ld();
         if (store) {
-          uint32_t okp[16], ovp[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            okp[c] = pack_bf16(__uint_as_float(rk[2 * c]) * p.scale, __uint_as_float(rk[2 * c + 1]) * p.scale);
-            ovp[c] = pack_bf16(__uint_as_float(rv[2 * c]), __uint_as_float(rv[2 * c + 1]));
-          }
-          uint4* dk4 = reinterpret_cast<uint4*>(ok_ + c0);
-          uint4* dv4 = reinterpret_cast<uint4*>(ov_ + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            dk4[q] = make_uint4(okp[4 * q], okp[4 * q + 1], okp[4 * q + 2], okp[4 * q + 3]);
-            dv4[q] = make_uint4(ovp[4 * q], ovp[4 * q + 1], ovp[4 * q + 2], ovp[4 * q + 3]);
-          }
+          store_row_bf16(okp + c0, rk, p.scale);
+          store_row_bf16(ovp + c0, rv, 1.f);
         }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (M.abort && threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_TIMEOUT);
+  if (warp == WARP_MMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ================================================================ dQ kernel
+namespace dq {
+constexpr int NS = 3;
+constexpr int OFF_K = 0, OFF_V = NS * TILE_B;  // rings of K and V tiles
+constexpr int OFF_MISC = 2 * NS * TILE_B;
+constexpr int MAX_KT = 1024;                   // NT
+// TMEM columns: dQ accumulator, S, dP (dS over it), then the A operands of
+// S = Q K^T and dP = dh V^T as packed bf16 (64 columns each).
+constexpr uint32_t COL_DQ = 0, COL_S = 128, COL_DP = 256, COL_Q = 384, COL_DH = 448;
+
+struct Misc {
+  uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
+  uint64_t a_ready, s_full, s_read, dp_full, ds_full, done, drain;
+  uint32_t tmem_base;
+  int abort;
+  int wsum[NTHREADS / 32];
+  uint32_t list[MAX_KT];  // sparse steps: key tile << 4 | pair bits
+};
+constexpr int SMEM = OFF_MISC + (int)sizeof(Misc);
+static_assert(SMEM <= kMaxSmem, "dq shared-memory budget");
+}  // namespace dq
+
+// Row t (64 columns from c0) of a [B,H,N,128] bf16 tensor into this thread's
+// TMEM lane as 32 packed columns; zeros past the end.
+__device__ __forceinline__ void row_to_tmem(const TensorRef& X, int b, int h, int t, bool valid, int c0,
+                                            uint32_t taddr) {
+  uint32_t v[32];
+  if (valid) {
+    const uint4* src = reinterpret_cast<const uint4*>(row_ptr<__nv_bfloat16>(X, b, h, t) + c0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 x = src[q];
+      v[4 * q] = x.x;
+      v[4 * q + 1] = x.y;
+      v[4 * q + 2] = x.z;
+      v[4 * q + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = 0u;
+  }
+  tmem_st32(taddr, v);
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     TensorRef Qr, TensorRef dhf_r, TensorRef dhs_r, BwdTcParams p) {
+  using namespace dq;
+  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_UNSUPPORTED);
+    return;
+  }
+  dq::Misc& M = *reinterpret_cast<dq::Misc*>(smem + OFF_MISC);
+  volatile int* abort = &M.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = (int)(gridDim.x - 1 - blockIdx.x);  // heaviest query tiles launch first
+  const int h = blockIdx.y, b = blockIdx.z, kvh = h / p.g;
+  const int q0 = qt * TILE;
+  const int n_full = qt + 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&M.k_full[s], 1);
+      mbar_init(&M.k_empty[s], 1);
+      mbar_init(&M.v_full[s], 1);
+      mbar_init(&M.v_empty[s], 1);
+    }
+    mbar_init(&M.a_ready, 8);
+    mbar_init(&M.s_full, 1);
+    mbar_init(&M.s_read, 8);
+    mbar_init(&M.dp_full, 1);
+    mbar_init(&M.ds_full, 8);
+    mbar_init(&M.done, 1);
+    mbar_init(&M.drain, 1);
+    M.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(&M.tmem_base, 512);
+    tmem_relinquish();
+  }
+  // Sparse-stream steps: key tiles holding a selected pair of this query tile.
+  int n_sparse = 0;
+  for (int base = 0; base < n_full; base += NTHREADS) {
+    const int kt = base + (int)threadIdx.x;
+    const uint32_t bits = kt < n_full ? tile_bits(p, b, h, qt, kt) : 0u;
+    compact_append(bits != 0, ((uint32_t)kt << 4) | bits, M.list, MAX_KT, M.wsum, n_sparse);
+  }
+  n_sparse = min(n_sparse, MAX_KT);
+  const int T = n_full + n_sparse;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = M.tmem_base;
+  auto decode = [&](int j, int& kt, int& sp, uint32_t& bits) {
+    if (j < n_full) {
+      kt = j;
+      sp = 0;
+      bits = 0xFu;
+    } else {
+      const uint32_t e = M.list[j - n_full];
+      kt = (int)(e >> 4);
+      sp = 1;
+      bits = e & 0xFu;
+    }
+  };
+
+  if (warp == WARP_TMA) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      int kiss = 0, viss = 0;
+      for (int j = 0; j < T; ++j) {
+        const int st = j % NS;
+        const uint32_t ph = (uint32_t)(j / NS - 1) & 1u;
+        int kt, sp;
+        uint32_t bits;
+        decode(j, kt, sp, bits);
+        if (j >= NS && !mbar_wait(&M.k_empty[st], ph, abort)) break;
+        mbar_expect_tx(&M.k_full[st], TILE_B);
+        tma_load_4d(smem + OFF_K + st * TILE_B, &tmK, &M.k_full[st], 0, kt * TILE, kvh, b);
+        tma_load_4d(smem + OFF_K + st * TILE_B + HALF, &tmK, &M.k_full[st], 64, kt * TILE, kvh, b);
+        kiss = j + 1;
+        if (j >= NS && !mbar_wait(&M.v_empty[st], ph, abort)) break;
+        mbar_expect_tx(&M.v_full[st], TILE_B);
+        tma_load_4d(smem + OFF_V + st * TILE_B, &tmV, &M.v_full[st], 0, kt * TILE, kvh, b);
+        tma_load_4d(smem + OFF_V + st * TILE_B + HALF, &tmV, &M.v_full[st], 64, kt * TILE, kvh, b);
+        viss = j + 1;
+      }
+      int dummy = 0;
+      for (int j = (kiss > NS ? kiss - NS : 0); j < kiss; ++j) {
+        dummy = 0;
+        mbar_wait(&M.k_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
+      }
+      for (int j = (viss > NS ? viss - NS : 0); j < viss; ++j) {
+        dummy = 0;
+        mbar_wait(&M.v_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      const uint32_t sk0 = smem_u32(smem + OFF_K), sv0 = smem_u32(smem + OFF_V);
+      bool ok = mbar_wait(&M.a_ready, 0, abort) && mbar_wait(&M.k_full[0], 0, abort) &&
+                mbar_wait(&M.v_full[0], 0, abort);
+      if (ok) {
+        tc_fence_after();
+        mma_tile_ts_k(tmem + COL_S, tmem + COL_Q, sk0);
+        tc_commit(&M.s_full);
+        mma_tile_ts_k(tmem + COL_DP, tmem + COL_DH, sv0);
+        tc_commit(&M.dp_full);
+        tc_commit(&M.v_empty[0]);
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        const int st = j % NS, st1 = (j + 1) % NS;
+        const uint32_t ph1 = (uint32_t)((j + 1) / NS) & 1u;
+        const bool more = j + 1 < T;
+        // S of the next step as soon as the dS warps hold S(j) in registers.
+        if (!mbar_wait(&M.s_read, (uint32_t)j & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        if (more) {
+          if (!mbar_wait(&M.k_full[st1], ph1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_ts_k(tmem + COL_S, tmem + COL_Q, sk0 + st1 * TILE_B);
+          tc_commit(&M.s_full);
+        }
+        // dQ += dS K once dS is over dP (for the first sparse step the dS
+        // warps have also put dh_s in place of dh_f by then).
+        if (!mbar_wait(&M.ds_full, (uint32_t)j & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_tile_ts(tmem + COL_DQ, tmem + COL_DP, sk0 + st * TILE_B, j > 0);
+        tc_commit(&M.k_empty[st]);
+        if (more) {
+          if (!mbar_wait(&M.v_full[st1], ph1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_ts_k(tmem + COL_DP, tmem + COL_DH, sv0 + st1 * TILE_B);
+          tc_commit(&M.dp_full);
+          tc_commit(&M.v_empty[st1]);
+        }
+      }
+      tc_commit(&M.done);
+      tc_commit(&M.drain);
+      int dummy = 0;
+      mbar_wait(&M.drain, 0, &dummy);
+    }
+  } else {
+    const int quarter = warp & 3, ch = warp >> 2;  // lanes 32*quarter.., key columns 64*ch..
+    const int r = quarter * 32 + lane;             // query row within the tile
+    const int t = q0 + r;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const bool in_range = t < p.N;
+    const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + (in_range ? t : 0);
+    const float l2[2] = {in_range ? p.lse2[0][ro] : 0.f, in_range ? p.lse2[1][ro] : 0.f};
+    const float Dv[2] = {in_range ? p.D[0][ro] : 0.f, in_range ? p.D[1][ro] : 0.f};
+    // A operands: Q and dh_f rows, d columns 64 ch .. 64 ch + 63.
+    row_to_tmem(Qr, b, h, t, in_range, 64 * ch, lane_base + COL_Q + 32 * ch);
+    row_to_tmem(dhf_r, b, h, t, in_range, 64 * ch, lane_base + COL_DH + 32 * ch);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&M.a_ready);
+    const uint32_t cS = lane_base + COL_S + 64 * ch, cP = lane_base + COL_DP + 64 * ch;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      int kt, sp;
+      uint32_t bits;
+      decode(j, kt, sp, bits);
+      if (!mbar_wait(&M.s_full, (uint32_t)j & 1u, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool sel = (bits >> (2 * (r >> 6) + ch)) & 1u;
+      uint32_t x0[32], x1[32];
+      if (sel) {
+        tmem_ld32(cS, x0);
+        tmem_ld32(cS + 32, x1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.s_read);
+      uint32_t pk[32];
+      if (sel) {
+        const float lv = sp ? l2[1] : l2[0];
+        if (kt == qt) {
+          // query q0 + r attends key 128 kt + 64 ch + col only if 64 ch + col <= r
+          auto keep0 = [&](int col) { return 64 * ch + col <= r; };
+          auto keep1 = [&](int col) { return 64 * ch + 32 + col <= r; };
+          p_block_row<true>(x0, lv, p.c, keep0, pk);
+          p_block_row<true>(x1, lv, p.c, keep1, pk + 16);
+        } else {
+          auto all = [](int) { return true; };
+          p_block_row<false>(x0, lv, p.c, all, pk);
+          p_block_row<false>(x1, lv, p.c, all, pk + 16);
+        }
+      }
+      if (!mbar_wait(&M.dp_full, (uint32_t)j & 1u, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t dsk[32];
+      if (sel) {
+        uint32_t y0[32], y1[32];
+        tmem_ld32(cP, y0);
+        tmem_ld32(cP + 32, y1);
+        tmem_wait_ld();
+        const float dv = sp ? Dv[1] : Dv[0];
+        ds_block_row(y0, dv, pk, dsk);
+        ds_block_row(y1, dv, pk + 16, dsk + 16);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) dsk[c] = 0u;
+      }
+      tmem_st32(cP, dsk);
+      // dP of this step was the last product to read dh_f: the sparse steps
+      // that follow use dh_s in the same columns.
+      if (j + 1 == n_full && n_sparse > 0)
+        row_to_tmem(dhs_r, b, h, t, in_range, 64 * ch, lane_base + COL_DH + 32 * ch);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.ds_full);
+    }
+    if (ok && mbar_wait(&M.done, 0, abort)) {
+      tc_fence_after();
+      __nv_bfloat16* out = in_range ? row_ptr_w<__nv_bfloat16>(p.dq, b, h, t) : nullptr;
+#pragma unroll 1
+      for (int c0 = 64 * ch; c0 < 64 * ch + 64; c0 += 32) {
+        uint32_t rq[32];
+        tmem_ld32(lane_base + COL_DQ + c0, rq);
+        tmem_wait_ld();
+        if (in_range) store_row_bf16(out + c0, rq, p.scale);
       }
     }
   }
@@ -793,25 +917,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace
 
 bool bwd_tc_supported(const Dims& D) {
+  const int NT = (D.N + TILE - 1) / TILE;
   return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048 &&
-         (int64_t)D.g * (D.N / dkv::BQ) <= dkv::MAX_STEPS && D.N / dq::BK <= dq::MAX_TILES;
+         (int64_t)D.g * NT <= dkv::MAX_SPARSE && NT <= dq::MAX_KT && D.g <= 255;
 }
 
 cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cudaStream_t st) {
   if (!bwd_tc_supported(D)) return cudaErrorNotSupported;
-  // Workspace reuse: the fp32 dh_f / dO_c regions hold bf16 dh_f / dh_s here,
-  // Df / Dc hold D_f / D_s.
+  // Workspace reuse: the fp32 dh_f / dO_c regions hold bf16 dh_f / dh_s in
+  // their lower halves, Df / Dc hold D_f / D_s, and the upper half of the dh_f
+  // region holds lse_full and lse_sel in base 2.
   __nv_bfloat16* dhf = reinterpret_cast<__nv_bfloat16*>(a.dhf);
   __nv_bfloat16* dhs = reinterpret_cast<__nv_bfloat16*>(a.doc);
   const double Mtot = (double)D.B * D.Hq * D.N * D.d;
   const float c2 = (float)(2.0 * (double)a.alpha / Mtot);
   const unsigned pre_blocks = (unsigned)sqdiff_partial_count(D);
-  // The packed per-query scalars go in the upper half of the fp32 dh_f
-  // region (the bf16 dh_f uses only the lower half).
   const int64_t rows = (int64_t)D.B * D.Hq * D.N;
-  float4* scal = reinterpret_cast<float4*>(reinterpret_cast<char*>(a.dhf) + rows * D.d * 2);
-  bwd_pre_tc_kernel<__nv_bfloat16><<<pre_blocks, 256, 0, st>>>(a.hf, a.hs, a.gf, a.gs, D.Hq, D.N, c2, dhf, dhs,
-                                                                a.Df, a.Dc, a.partials, a.lse_full, a.lse_sel, scal);
+  float* lse2f = reinterpret_cast<float*>(reinterpret_cast<char*>(a.dhf) + rows * D.d * 2);
+  float* lse2s = lse2f + rows;
+  bwd_pre_tc_kernel<<<pre_blocks, 256, 0, st>>>(a.hf, a.hs, a.gf, a.gs, D.Hq, D.N, c2, dhf, dhs, a.Df, a.Dc,
+                                                a.partials, a.lse_full, a.lse_sel, lse2f, lse2s);
   count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -822,23 +947,20 @@ cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cuda
   const int64_t rowstride = (int64_t)D.N * D.d;
   TensorRef rdhf{dhf, (int64_t)D.Hq * rowstride, rowstride, D.d};
   TensorRef rdhs{dhs, (int64_t)D.Hq * rowstride, rowstride, D.d};
-  CUtensorMap mq128, mk64, mv64, mf128, ms128, mq64, mk128, mv128, mf64, ms64;
-  if (!make_tma_map_bf16(&mq128, a.q, D.B, D.Hq, D.N, 128) || !make_tma_map_bf16(&mk64, a.k, D.B, D.Hkv, D.N, 64) ||
-      !make_tma_map_bf16(&mv64, a.v, D.B, D.Hkv, D.N, 64) || !make_tma_map_bf16(&mf128, rdhf, D.B, D.Hq, D.N, 128) ||
-      !make_tma_map_bf16(&ms128, rdhs, D.B, D.Hq, D.N, 128) || !make_tma_map_bf16(&mq64, a.q, D.B, D.Hq, D.N, 64) ||
-      !make_tma_map_bf16(&mk128, a.k, D.B, D.Hkv, D.N, 128) || !make_tma_map_bf16(&mv128, a.v, D.B, D.Hkv, D.N, 128) ||
-      !make_tma_map_bf16(&mf64, rdhf, D.B, D.Hq, D.N, 64) || !make_tma_map_bf16(&ms64, rdhs, D.B, D.Hq, D.N, 64))
+  CUtensorMap mq, mk, mv, mf, ms;
+  if (!make_tma_map_bf16(&mq, a.q, D.B, D.Hq, D.N, TILE) || !make_tma_map_bf16(&mk, a.k, D.B, D.Hkv, D.N, TILE) ||
+      !make_tma_map_bf16(&mv, a.v, D.B, D.Hkv, D.N, TILE) || !make_tma_map_bf16(&mf, rdhf, D.B, D.Hq, D.N, TILE) ||
+      !make_tma_map_bf16(&ms, rdhs, D.B, D.Hq, D.N, TILE))
     return cudaErrorInvalidValue;
   BwdTcParams p;
   p.dq = a.dq;
   p.dk = a.dk;
   p.dv = a.dv;
-  p.lse_full = a.lse_full;
-  p.lse_sel = a.lse_sel;
-  p.Df = a.Df;
-  p.Ds = a.Dc;
+  p.lse2[0] = lse2f;
+  p.lse2[1] = lse2s;
+  p.D[0] = a.Df;
+  p.D[1] = a.Dc;
   p.mask = a.mask;
-  p.scal = scal;
   p.words = a.words;
   p.status = status;
   p.Hq = D.Hq;
@@ -846,19 +968,18 @@ cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cuda
   p.N = D.N;
   p.n = D.n;
   p.s = D.s;
+  p.NT = (D.N + TILE - 1) / TILE;
   p.c = D.scale * kLog2e;
   p.scale = D.scale;
   e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM);
   if (e != cudaSuccess) return e;
-  bwd_dkv_tc_kernel<<<dim3((D.N + dkv::BKEY - 1) / dkv::BKEY, D.Hkv, D.B), NTHREADS, dkv::SMEM, st>>>(
-      mq64, mk128, mv128, mf64, ms64, p);
+  bwd_dkv_tc_kernel<<<dim3(p.NT, D.Hkv, D.B), NTHREADS, dkv::SMEM, st>>>(mq, mk, mv, mf, ms, p);
   count_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq_tc_kernel<<<dim3((D.N + dq::BM - 1) / dq::BM, D.Hq, D.B), NTHREADS, dq::SMEM, st>>>(mq128, mk64, mv64,
-                                                                                            mf128, ms128, p);
+  bwd_dq_tc_kernel<<<dim3(p.NT, D.Hq, D.B), NTHREADS, dq::SMEM, st>>>(mk, mv, a.q, rdhf, rdhs, p);
   count_launches(1);
   return cudaGetLastError();
 }
