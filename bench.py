@@ -55,6 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-sparse", action="store_true", help="skip the sparse-stream-alone rows")
     return ap.parse_args(argv)
 
 
@@ -426,6 +427,55 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
         "pages_dropped_mass_context": PAGES_DROPPED_MASS,
         "align_loss": float(grads["align_loss"].item()),
     }
+
+    # ---------------- sparse stream alone (inference mode), timed on its own
+    # after the step; not part of `value`.  Attended FLOPs count the selected
+    # causal pairs only: forward 4 d sum|A_t|, backward 10 d sum|A_t|.
+    if not args.no_sparse:
+        idx_np = out["idx"].cpu().numpy()
+        n_ = w.n_blocks
+        i_ax = np.arange(n_).reshape(1, 1, n_, 1)
+        sel = np.zeros(idx_np.shape[:3] + (n_,), dtype=bool)
+        valid = (idx_np >= 0) & (idx_np <= i_ax)
+        bb, hh, ii, kk = np.nonzero(valid)
+        sel[bb, hh, ii, idx_np[bb, hh, ii, kk]] = True
+        diag = np.eye(n_, dtype=bool)[None, None]
+        pairs_sel = int((sel & ~diag).sum()) * w.block * w.block + int((sel & diag).sum()) * w.block * (w.block + 1) // 2
+        hs2 = torch.empty_like(out["h_sparse"])
+        lse2 = torch.empty_like(out["lse_sel"])
+
+        def sparse_fwd():
+            api.ssa_fwd_sparse(dims, D["Q"], D["K"], D["V"], out["idx"], hs2, lse2, stream)
+
+        def sparse_bwd():
+            api.ssa_bwd_sparse(dims, D["Q"], D["K"], D["V"], out["idx"], hs2, lse2, g_sparse, grads["dQ"],
+                               grads["dK"], grads["dV"], ws, stream)
+
+        for _ in range(args.warmup):
+            sparse_fwd()
+            sparse_bwd()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            ev[k][0].record(stream)
+            sparse_fwd()
+            ev[k][1].record(stream)
+            sparse_bwd()
+            ev[k][2].record(stream)
+        torch.cuda.synchronize()
+        status = api.ssa_device_status(clear=True, stream=stream)
+        if status != api.SSA_OK:
+            raise RuntimeError(f"device status after the sparse rows: {api.status_string(status)}")
+        f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+        extra["sparse_only"] = {
+            "entry_points": "ssa_fwd_sparse, ssa_bwd_sparse (timed separately, not in value)",
+            "sparse_pairs": pairs_sel, "share_of_causal_pairs": pairs_sel / w.causal_pairs(),
+            "fwd_ms": f_ms, "bwd_ms": b_ms,
+            "fwd_attended_tflops": 4 * w.d * pairs_sel / (f_ms * 1e-3) / 1e12,
+            "bwd_attended_tflops": 10 * w.d * pairs_sel / (b_ms * 1e-3) / 1e12,
+            "fwd_speedup_vs_fwd_dual": row_ms["fwd_dual"] / f_ms,
+        }
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

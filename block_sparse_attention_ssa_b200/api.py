@@ -74,6 +74,12 @@ _SIGS = {
                                      ctypes.c_void_p, _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_float,
                                      ctypes.c_void_p, _P(ssa_tensor_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
                                      ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "ssa_fwd_sparse": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
+                                       ctypes.c_void_p, _P(ssa_tensor_t), ctypes.c_void_p, ctypes.c_void_p]),
+    "ssa_bwd_sparse": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
+                                       ctypes.c_void_p, _P(ssa_tensor_t), ctypes.c_void_p, _P(ssa_tensor_t),
+                                       _P(ssa_tensor_t), _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_void_p,
+                                       ctypes.c_size_t, ctypes.c_void_p]),
     "ssa_dropped_mass": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                          ctypes.c_void_p]),
@@ -183,6 +189,17 @@ def ssa_bwd_dual(dims, Q, K, V, idx, h_full, h_sparse, lse_full, lse_sel, g_full
         ctypes.byref(dims), _t(Q), _t(K), _t(V), _p(idx), _t(h_full), _t(h_sparse), _p(lse_full),
         _p(lse_sel), _t(g_full), _t(g_sparse), float(alpha), _p(align_loss), _t(dQ), _t(dK), _t(dV),
         _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def ssa_fwd_sparse(dims, Q, K, V, idx, h_sparse, lse_sel, stream=None) -> None:
+    _check("ssa_fwd_sparse", load_library().ssa_fwd_sparse(
+        ctypes.byref(dims), _t(Q), _t(K), _t(V), _p(idx), _t(h_sparse), _p(lse_sel), _stream(stream)))
+
+
+def ssa_bwd_sparse(dims, Q, K, V, idx, h_sparse, lse_sel, g_sparse, dQ, dK, dV, ws, stream=None) -> None:
+    _check("ssa_bwd_sparse", load_library().ssa_bwd_sparse(
+        ctypes.byref(dims), _t(Q), _t(K), _t(V), _p(idx), _t(h_sparse), _p(lse_sel), _t(g_sparse),
+        _t(dQ), _t(dK), _t(dV), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def ssa_dropped_mass(dims, Q, K, idx, lse_full, delta, ws, stream=None) -> None:

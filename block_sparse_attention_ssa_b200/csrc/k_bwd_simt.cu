@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(NT) bwd_dq_kernel(BwdArgs a, int Hq, int g, in
     const int u0 = kt * BT, jblk = u0 / s;
     __syncthreads();
     const bool sel = (S.sel[jblk >> 5] >> (jblk & 31)) & 1u;
+    if (a.sparse_only && !sel) continue;  // uniform over the CTA
     for (int e = tid; e < BT * D / VEC; e += NT) {
       const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
       float tk[VEC], tv[VEC];
@@ -257,6 +258,7 @@ __global__ void __launch_bounds__(NT) bwd_dkv_kernel(BwdArgs a, int Hq, int g, i
       const int64_t rbase = ((int64_t)b * Hq + h) * N + t0;
       const uint32_t word = a.mask[(((int64_t)b * Hq + h) * n + iblk) * a.words + (jblk >> 5)];
       const bool sel = (word >> (jblk & 31)) & 1u;
+      if (a.sparse_only && !sel) continue;  // uniform over the CTA
       const float* src = sel ? a.doc : a.dhf;
       const float* Dsrc = sel ? a.Dc : a.Df;
       __syncthreads();

@@ -129,6 +129,7 @@ struct BwdTcParams {
   int words;
   int32_t* status;
   int Hq, g, N, n, s, NT;   // NT = number of 128-row tiles
+  int full;                 // 0: sparse stream alone (no stream-f steps)
   float c;                  // scale * log2(e)
   float scale;
 };
@@ -338,7 +339,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int kvh = blockIdx.y, b = blockIdx.z;
   const int u0 = kt * TILE;
   const int nqt = p.NT - kt;       // causal query tiles per head
-  const int n_full = p.g * nqt;
+  const int n_cand = p.g * nqt;    // (head, query tile) pairs of the causal range
+  const int n_full = p.full ? n_cand : 0;
   auto stage_ptr = [&](int st) { return smem + OFF_STAGE + st * STAGE; };
 
   if (threadIdx.x == 0) {
@@ -368,10 +370,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     reinterpret_cast<float*>(stage_ptr(i / (2 * TILE)) + 2 * TILE_B)[i % (2 * TILE)] = 0.f;
   // Sparse-stream steps: (head, query tile) pairs holding a selected pair.
   int n_sparse = 0;
-  for (int base = 0; base < n_full; base += NTHREADS) {
+  for (int base = 0; base < n_cand; base += NTHREADS) {
     const int it = base + (int)threadIdx.x;
     uint32_t bits = 0;
-    if (it < n_full) bits = tile_bits(p, b, kvh * p.g + it / nqt, kt + it % nqt, kt);
+    if (it < n_cand) bits = tile_bits(p, b, kvh * p.g + it / nqt, kt + it % nqt, kt);
     compact_append(bits != 0, ((uint32_t)it << 4) | bits, M.list, MAX_SPARSE, M.wsum, n_sparse);
   }
   n_sparse = min(n_sparse, MAX_SPARSE);
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
       const uint32_t ak = smem_u32(sK), av = smem_u32(sV);
-      bool ok = mbar_wait(&M.kv_full, 0, abort) && mbar_wait(&M.q_full[0], 0, abort) &&
+      bool ok = T > 0 && mbar_wait(&M.kv_full, 0, abort) && mbar_wait(&M.q_full[0], 0, abort) &&
                 mbar_wait(&M.dh_full[0], 0, abort);
       if (ok) {
         tc_fence_after();
@@ -597,6 +599,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld32(lane_base + COL_DK + c0, rk);
         tmem_ld32(lane_base + COL_DV + c0, rv);
         tmem_wait_ld();
+        if (T == 0) {  // no step touched these keys (a selection without them)
+#pragma unroll
+          for (int c = 0; c < 32; ++c) rk[c] = rv[c] = 0u;
+        }
         if (store) {
           store_row_bf16(okp + c0, rk, p.scale);
           store_row_bf16(ovp + c0, rv, 1.f);
@@ -675,7 +681,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int qt = (int)(gridDim.x - 1 - blockIdx.x);  // heaviest query tiles launch first
   const int h = blockIdx.y, b = blockIdx.z, kvh = h / p.g;
   const int q0 = qt * TILE;
-  const int n_full = qt + 1;
+  const int n_cand = qt + 1;  // causal key tiles
+  const int n_full = p.full ? n_cand : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -700,9 +707,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   // Sparse-stream steps: key tiles holding a selected pair of this query tile.
   int n_sparse = 0;
-  for (int base = 0; base < n_full; base += NTHREADS) {
+  for (int base = 0; base < n_cand; base += NTHREADS) {
     const int kt = base + (int)threadIdx.x;
-    const uint32_t bits = kt < n_full ? tile_bits(p, b, h, qt, kt) : 0u;
+    const uint32_t bits = kt < n_cand ? tile_bits(p, b, h, qt, kt) : 0u;
     compact_append(bits != 0, ((uint32_t)kt << 4) | bits, M.list, MAX_KT, M.wsum, n_sparse);
   }
   n_sparse = min(n_sparse, MAX_KT);
@@ -759,7 +766,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
       const uint32_t sk0 = smem_u32(smem + OFF_K), sv0 = smem_u32(smem + OFF_V);
-      bool ok = mbar_wait(&M.a_ready, 0, abort) && mbar_wait(&M.k_full[0], 0, abort) &&
+      bool ok = T > 0 && mbar_wait(&M.a_ready, 0, abort) && mbar_wait(&M.k_full[0], 0, abort) &&
                 mbar_wait(&M.v_full[0], 0, abort);
       if (ok) {
         tc_fence_after();
@@ -821,9 +828,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + (in_range ? t : 0);
     const float l2[2] = {in_range ? p.lse2[0][ro] : 0.f, in_range ? p.lse2[1][ro] : 0.f};
     const float Dv[2] = {in_range ? p.D[0][ro] : 0.f, in_range ? p.D[1][ro] : 0.f};
-    // A operands: Q and dh_f rows, d columns 64 ch .. 64 ch + 63.
+    // A operands: Q and dh_f rows (dh_s when there are no stream-f steps),
+    // d columns 64 ch .. 64 ch + 63.
     row_to_tmem(Qr, b, h, t, in_range, 64 * ch, lane_base + COL_Q + 32 * ch);
-    row_to_tmem(dhf_r, b, h, t, in_range, 64 * ch, lane_base + COL_DH + 32 * ch);
+    row_to_tmem(n_full > 0 ? dhf_r : dhs_r, b, h, t, in_range, 64 * ch, lane_base + COL_DH + 32 * ch);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
@@ -900,6 +908,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint32_t rq[32];
         tmem_ld32(lane_base + COL_DQ + c0, rq);
         tmem_wait_ld();
+        if (T == 0) {  // this query tile attends no listed block
+#pragma unroll
+          for (int c = 0; c < 32; ++c) rq[c] = 0u;
+        }
         if (in_range) store_row_bf16(out + c0, rq, p.scale);
       }
     }
@@ -971,6 +983,7 @@ cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cuda
   p.NT = (D.N + TILE - 1) / TILE;
   p.c = D.scale * kLog2e;
   p.scale = D.scale;
+  p.full = a.sparse_only ? 0 : 1;
   e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM);

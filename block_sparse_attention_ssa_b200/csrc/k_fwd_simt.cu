@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
     const int jblk = u0 / sh.s;
     __syncthreads();  // previous tile fully consumed; sel bits visible
     const bool sel = (S.sel[jblk >> 5] >> (jblk & 31)) & 1u;
+    if (a.sparse_only && !sel) continue;  // the sparse stream reads selected tiles only
     for (int e = tid; e < BN * D / VEC; e += NT) {
       const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
       float tmp[VEC];
@@ -204,12 +205,13 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
       const float wd = (lD > 0.f) ? expf(mD - M) : 0.f;
       const float inv_full = 1.0f / (wa * lA + wd * lD);
       const float inv_sel = (lA > 0.f) ? 1.0f / lA : 0.f;
-      T* hf = row_ptr_w<T>(a.hf, b, h, t0 + row) + pc * CW;
       T* hs = row_ptr_w<T>(a.hs, b, h, t0 + row) + pc * CW;
 #pragma unroll
-      for (int c = 0; c < CW; ++c) {
-        hs[c] = from_f32<T>(oA[r][c] * inv_sel);
-        hf[c] = from_f32<T>((wa * oA[r][c] + wd * oD[r][c]) * inv_full);
+      for (int c = 0; c < CW; ++c) hs[c] = from_f32<T>(oA[r][c] * inv_sel);
+      if (!a.sparse_only) {
+        T* hf = row_ptr_w<T>(a.hf, b, h, t0 + row) + pc * CW;
+#pragma unroll
+        for (int c = 0; c < CW; ++c) hf[c] = from_f32<T>((wa * oA[r][c] + wd * oD[r][c]) * inv_full);
       }
     }
   }
@@ -222,9 +224,11 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
     const float hi = fmaxf(lse_a, lse_d), lo = fminf(lse_a, lse_d);
     const float lse_f = (lo == kNegInf) ? hi : hi + log1pf(expf(lo - hi));
     if (WITH_V) {
-      a.lse_full[o] = lse_f;
       a.lse_sel[o] = lse_a;
-      a.delta[o] = (lD > 0.f) ? expf(lse_d - lse_f) : 0.f;
+      if (!a.sparse_only) {
+        a.lse_full[o] = lse_f;
+        a.delta[o] = (lD > 0.f) ? expf(lse_d - lse_f) : 0.f;
+      }
     } else if (a.lse_in != nullptr) {
       a.delta[o] = (lD > 0.f) ? lD * expf(mD - a.lse_in[o]) : 0.f;
     } else {

@@ -72,6 +72,8 @@ struct Misc {
   uint32_t tmem_base;
   int abort;
   uint32_t sel[2][64];  // selected-block bits of the tile's two query blocks
+  int nlist;            // sparse-only mode: selected key blocks of either half,
+  uint16_t list[2048];  // ascending
   float xmax[2][2][128];  // [tile parity][sub-block][row]: scaled tile max of its set
   float lsum[2][2][128];  // epilogue: per sub-block warp, per set, per row
 };
@@ -107,7 +109,13 @@ __device__ __forceinline__ bool pair_sync(uint64_t* bar, uint32_t& uses, int lan
   return ok;
 }
 
-template <int S_BLK>
+// SPARSE: the sparse stream alone (inference mode).  Only the key blocks
+// that one of the tile's query blocks selected are loaded, by 64-row TMA
+// boxes: with block 64 a step pairs two selected blocks (in ascending order,
+// not necessarily adjacent) as its two sub-blocks, with block 128 a step is
+// one selected block.  Dropped pairs count as "no key"; only O_A is used and
+// only h_sparse and lse_sel are written.
+template <int S_BLK, bool SPARSE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, TcParams p) {
@@ -125,9 +133,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int q0 = qt * BM;
   const int ib0 = q0 / S_BLK, ib1 = (q0 + SUB) / S_BLK;  // query blocks of the two halves
   const bool valid1 = q0 + SUB < p.N;
-  const int T = (min(q0 + BM, p.N) + BN - 1) / BN;  // causal key tiles
-  // key block of sub-block q of tile j
-  auto kblk = [](int j, int q) { return (j * BN + q * SUB) / S_BLK; };
+  // First key of sub-block q of step j, or -1 when that sub-block is empty.
+  auto sub_start = [&](int j, int q) -> int {
+    if (!SPARSE) return j * BN + q * SUB;
+    if (S_BLK == 128) return (int)M.list[j] * 128 + q * SUB;
+    const int e = 2 * j + q;
+    return e < M.nlist ? (int)M.list[e] * 64 : -1;
+  };
+  // State of the (query block ib, sub-block starting at u) pair.
+  auto state_of = [&](int u, int ib, bool valid, const uint32_t* selw) -> int {
+    if (u < 0) return 0;
+    const int s = pair_state(u / S_BLK, ib, valid, selw);
+    return (SPARSE && s == 2) ? 0 : s;
+  };
 
   // ---- set-up
   if (threadIdx.x == 0) {
@@ -172,6 +190,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (SPARSE) {
+    // Ascending list of the blocks either half selected (bit sets of the
+    // halves: M.sel[1] is zero when both halves are one query block).
+    if (warp == 0) {
+      const uint32_t w0 = M.sel[0][2 * lane] | M.sel[1][2 * lane];
+      const uint32_t w1 = M.sel[0][2 * lane + 1] | M.sel[1][2 * lane + 1];
+      const int c = __popc(w0) + __popc(w1);
+      int incl = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int pos = incl - c;
+      for (uint32_t x = w0; x; x &= x - 1) M.list[pos++] = (uint16_t)(64 * lane + __ffs(x) - 1);
+      for (uint32_t x = w1; x; x &= x - 1) M.list[pos++] = (uint16_t)(64 * lane + 32 + __ffs(x) - 1);
+      if (lane == 31) M.nlist = incl;
+    }
+    __syncthreads();
+  }
+  const int T = !SPARSE ? (min(q0 + BM, p.N) + BN - 1) / BN                 // causal key tiles
+                        : (S_BLK == 128 ? M.nlist : (M.nlist + 1) / 2);  // selected blocks
   const uint32_t tmem = M.tmem_base;
   const uint32_t* sel0 = M.sel[0];
   const uint32_t* sel1 = (ib1 != ib0) ? M.sel[1] : M.sel[0];
@@ -193,15 +233,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int j = 0; j < T; ++j) {
         const int st = j % NS;
         const uint32_t use = (uint32_t)(j / NS);
+        // Dual mode: one 128-row box per column half.  Sparse mode: one
+        // 64-row box per non-empty sub-block and column half, placed at the
+        // sub-block's rows (the 128-byte swizzle repeats every 8 rows, so
+        // the layout equals that of a 128-row box).
+        const int ua = sub_start(j, 0), ub = SPARSE ? sub_start(j, 1) : -1;
+        const uint32_t bytes = !SPARSE ? KV_BYTES : (ub >= 0 ? KV_BYTES : KV_BYTES / 2);
+        auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar) {
+          mbar_expect_tx(bar, bytes);
+          tma_load_4d(dst, map, bar, 0, ua, kvh, b);
+          tma_load_4d(dst + KV_BYTES / 2, map, bar, 64, ua, kvh, b);
+          if (ub >= 0) {
+            tma_load_4d(dst + SUB * 128, map, bar, 0, ub, kvh, b);
+            tma_load_4d(dst + KV_BYTES / 2 + SUB * 128, map, bar, 64, ub, kvh, b);
+          }
+        };
         if (j >= NS && !mbar_wait(&M.k_empty[st], (use - 1) & 1u, abort)) break;
-        mbar_expect_tx(&M.k_full[st], KV_BYTES);
-        tma_load_4d(sK + st * KV_BYTES, &tmK, &M.k_full[st], 0, j * BN, kvh, b);
-        tma_load_4d(sK + st * KV_BYTES + KV_BYTES / 2, &tmK, &M.k_full[st], 64, j * BN, kvh, b);
+        load_tile(sK + st * KV_BYTES, &tmK, &M.k_full[st]);
         k_issued = j + 1;
         if (j >= NS && !mbar_wait(&M.v_empty[st], (use - 1) & 1u, abort)) break;
-        mbar_expect_tx(&M.v_full[st], KV_BYTES);
-        tma_load_4d(sV + st * KV_BYTES, &tmV, &M.v_full[st], 0, j * BN, kvh, b);
-        tma_load_4d(sV + st * KV_BYTES + KV_BYTES / 2, &tmV, &M.v_full[st], 64, j * BN, kvh, b);
+        load_tile(sV + st * KV_BYTES, &tmV, &M.v_full[st]);
         v_issued = j + 1;
       }
       // Drain: every copy this thread issued must have landed before the CTA exits.
@@ -232,9 +283,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t s_col = COL_S + (uint32_t)sb * BN;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          const int kb = kblk(jj, q);
-          const int s0 = pair_state(kb, ib0, true, sel0);
-          const int s1 = pair_state(kb, ib1, valid1, sel1);
+          const int u = sub_start(jj, q);
+          const int s0 = state_of(u, ib0, true, sel0);
+          const int s1 = state_of(u, ib1, valid1, sel1);
           if (s0 == 0 && s1 == 0) continue;
           const bool mixed = (s0 != 0 && s1 != 0 && s0 != s1);
           const int target = s0 != 0 ? s0 : s1;
@@ -313,11 +364,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int st[2];  // this row's state of sub-blocks 0 and 1
       bool mixed_q;
 #pragma unroll
-      for (int qq = 0; qq < 2; ++qq) st[qq] = pair_state(kblk(j, qq), ib, hvalid, selw);
+      for (int qq = 0; qq < 2; ++qq) st[qq] = state_of(sub_start(j, qq), ib, hvalid, selw);
+      const int u0 = sub_start(j, q);  // first key of this warp's sub-block
       {
-        const int kb = kblk(j, q);
-        const int o0 = pair_state(kb, ib0, true, sel0);
-        const int o1 = pair_state(kb, ib1, valid1, sel1);
+        const int o0 = state_of(u0, ib0, true, sel0);
+        const int o1 = state_of(u0, ib1, valid1, sel1);
         mixed_q = (o0 != 0 && o1 != 0 && o0 != o1);
       }
       const int mine = st[q];
@@ -333,7 +384,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(r[c]);
         }
-        const int u0 = j * BN + q * SUB;
         if (u0 + SUB - 1 > t) {  // causal mask inside the diagonal sub-block
 #pragma unroll
           for (int c = 0; c < SUB; ++c)
@@ -451,13 +501,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float wd = (lD > 0.f) ? ex2(mD - Mx) : 0.f;
       const float inv_full = 1.0f / (wa * lA + wd * lD);
       const float inv_sel = (lA > 0.f) ? 1.0f / lA : 0.f;
-      __nv_bfloat16* hf = store ? row_ptr_w<__nv_bfloat16>(p.hf, b, h, t) : nullptr;
+      __nv_bfloat16* hf = (store && !SPARSE) ? row_ptr_w<__nv_bfloat16>(p.hf, b, h, t) : nullptr;
       __nv_bfloat16* hs = store ? row_ptr_w<__nv_bfloat16>(p.hs, b, h, t) : nullptr;
 #pragma unroll 1
       for (int c0 = q * (HD / 2); c0 < (q + 1) * (HD / 2); c0 += 32) {
         uint32_t ra[32], rd[32];
         tmem_ld32(lane_base + COL_OA + c0, ra);
-        tmem_ld32(lane_base + COL_OD + c0, rd);
+        if (!SPARSE) tmem_ld32(lane_base + COL_OD + c0, rd);
         tmem_wait_ld();
         if (store) {
           uint32_t of[16], os[16];
@@ -465,17 +515,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int c = 0; c < 32; c += 2) {
             const float a0 = (lA > 0.f) ? __uint_as_float(ra[c]) : 0.f;
             const float a1 = (lA > 0.f) ? __uint_as_float(ra[c + 1]) : 0.f;
-            const float d0 = (lD > 0.f) ? __uint_as_float(rd[c]) : 0.f;
-            const float d1 = (lD > 0.f) ? __uint_as_float(rd[c + 1]) : 0.f;
             os[c / 2] = pack_bf16(a0 * inv_sel, a1 * inv_sel);
-            of[c / 2] = pack_bf16((wa * a0 + wd * d0) * inv_full, (wa * a1 + wd * d1) * inv_full);
+            if (!SPARSE) {
+              const float d0 = (lD > 0.f) ? __uint_as_float(rd[c]) : 0.f;
+              const float d1 = (lD > 0.f) ? __uint_as_float(rd[c + 1]) : 0.f;
+              of[c / 2] = pack_bf16((wa * a0 + wd * d0) * inv_full, (wa * a1 + wd * d1) * inv_full);
+            }
           }
           uint4* dst_s = reinterpret_cast<uint4*>(hs + c0);
-          uint4* dst_f = reinterpret_cast<uint4*>(hf + c0);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            dst_s[v] = make_uint4(os[4 * v], os[4 * v + 1], os[4 * v + 2], os[4 * v + 3]);
-            dst_f[v] = make_uint4(of[4 * v], of[4 * v + 1], of[4 * v + 2], of[4 * v + 3]);
+          for (int v = 0; v < 4; ++v) dst_s[v] = make_uint4(os[4 * v], os[4 * v + 1], os[4 * v + 2], os[4 * v + 3]);
+          if (!SPARSE) {
+            uint4* dst_f = reinterpret_cast<uint4*>(hf + c0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst_f[v] = make_uint4(of[4 * v], of[4 * v + 1], of[4 * v + 2], of[4 * v + 3]);
           }
         }
       }
@@ -486,9 +539,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float hi = fmaxf(lse2_a, lse2_d), lo = fminf(lse2_a, lse2_d);
         const float lse2_f = (lo == kNegInf) ? hi : hi + log2f(1.0f + ex2(lo - hi));
         const int64_t o = ((int64_t)b * p.Hq + h) * p.N + t;
-        p.lse_full[o] = lse2_f * kLn2;
         p.lse_sel[o] = (lA > 0.f) ? lse2_a * kLn2 : kNegInf;
-        p.delta[o] = (lD > 0.f) ? ex2(lse2_d - lse2_f) : 0.f;
+        if (!SPARSE) {
+          p.lse_full[o] = lse2_f * kLn2;
+          p.delta[o] = (lD > 0.f) ? ex2(lse2_d - lse2_f) : 0.f;
+        }
       }
     }
   }
@@ -504,11 +559,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <int S_BLK>
+template <int S_BLK, bool SPARSE>
 cudaError_t launch_blk(const Dims& D, const FwdArgs& a, int32_t* status, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_tma_map_bf16(&mq, a.q, D.B, D.Hq, D.N, BM) || !make_tma_map_bf16(&mk, a.k, D.B, D.Hkv, D.N, BN) ||
-      !make_tma_map_bf16(&mv, a.v, D.B, D.Hkv, D.N, BN))
+  const int kv_rows = SPARSE ? SUB : BN;  // sparse mode loads 64-key sub-blocks
+  if (!make_tma_map_bf16(&mq, a.q, D.B, D.Hq, D.N, BM) || !make_tma_map_bf16(&mk, a.k, D.B, D.Hkv, D.N, kv_rows) ||
+      !make_tma_map_bf16(&mv, a.v, D.B, D.Hkv, D.N, kv_rows))
     return cudaErrorInvalidValue;
   TcParams p;
   p.hf = a.hf;
@@ -524,7 +580,7 @@ cudaError_t launch_blk(const Dims& D, const FwdArgs& a, int32_t* status, cudaStr
   p.n = D.n;
   p.k = D.k;
   p.c = D.scale * 1.4426950408889634f;
-  auto kern = fwd_tc_kernel<S_BLK>;
+  auto kern = fwd_tc_kernel<S_BLK, SPARSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((D.N + BM - 1) / BM, D.Hq, D.B);
@@ -571,7 +627,9 @@ bool fwd_tc_supported(const Dims& D) {
 
 cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st) {
   if (!fwd_tc_supported(D)) return cudaErrorNotSupported;
-  return D.s == 64 ? launch_blk<64>(D, a, dev_status, st) : launch_blk<128>(D, a, dev_status, st);
+  if (a.sparse_only)
+    return D.s == 64 ? launch_blk<64, true>(D, a, dev_status, st) : launch_blk<128, true>(D, a, dev_status, st);
+  return D.s == 64 ? launch_blk<64, false>(D, a, dev_status, st) : launch_blk<128, false>(D, a, dev_status, st);
 }
 
 }  // namespace ssa

@@ -283,6 +283,90 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
   return from_cuda(e);
 }
 
+ssa_status_t ssa_fwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
+                            const ssa_tensor_t* V, const int32_t* idx, const ssa_tensor_t* h_sparse,
+                            float* lse_sel, ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  FwdArgs a{};
+  if ((s = check_tensor(D, Q, false, &a.q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &a.k)) != SSA_OK) return s;
+  if ((s = check_tensor(D, V, false, &a.v)) != SSA_OK) return s;
+  if ((s = check_tensor(D, h_sparse, false, &a.hs)) != SSA_OK) return s;
+  if (!idx || !lse_sel) return SSA_ERR_INVALID_ARG;
+  if ((s = check_device()) != SSA_OK) return s;
+  a.hf = TensorRef{nullptr, 0, 0, 0};
+  a.idx = idx;
+  a.lse_sel = lse_sel;
+  a.sparse_only = true;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fwd_tc_supported(D)) {
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_fwd_tc(D, a, status, st));
+  }
+  return from_cuda(launch_fwd_simt(D, a, st));
+}
+
+ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
+                            const ssa_tensor_t* V, const int32_t* idx, const ssa_tensor_t* h_sparse,
+                            const float* lse_sel, const ssa_tensor_t* g_sparse, const ssa_tensor_t* dQ,
+                            const ssa_tensor_t* dK, const ssa_tensor_t* dV, void* ws, size_t ws_bytes,
+                            ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  BwdArgs a{};
+  if ((s = check_tensor(D, Q, false, &a.q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &a.k)) != SSA_OK) return s;
+  if ((s = check_tensor(D, V, false, &a.v)) != SSA_OK) return s;
+  if ((s = check_tensor(D, h_sparse, false, &a.hs)) != SSA_OK) return s;
+  if ((s = check_tensor(D, g_sparse, false, &a.gs)) != SSA_OK) return s;
+  if ((s = check_tensor(D, dQ, false, &a.dq)) != SSA_OK) return s;
+  if ((s = check_tensor(D, dK, false, &a.dk)) != SSA_OK) return s;
+  if ((s = check_tensor(D, dV, false, &a.dv)) != SSA_OK) return s;
+  if (!idx || !lse_sel) return SSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(lse_sel) % 16) return SSA_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
+  if ((s = check_device()) != SSA_OK) return s;
+  const Layout L = layout(D);
+  // The sparse stream alone is the dual backward with h_full := h_sparse,
+  // lse_full := lse_sel, no full-stream gradient and no alignment term
+  // (dh_f = 0, r = 1), restricted to the selected pairs.
+  a.hf = a.hs;
+  a.gf = TensorRef{nullptr, 0, 0, 0};
+  a.idx = idx;
+  a.lse_full = lse_sel;
+  a.lse_sel = lse_sel;
+  a.alpha = 0.f;
+  a.align_loss = nullptr;
+  a.dhf = at<float>(ws, L.dhf);
+  a.doc = at<float>(ws, L.doc);
+  a.Df = at<float>(ws, L.Df);
+  a.Dc = at<float>(ws, L.Dc);
+  a.mask = at<uint32_t>(ws, L.mask);
+  a.words = L.words;
+  a.partials = at<float>(ws, L.partials);
+  a.n_partials = L.n_partials;
+  a.sparse_only = true;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_build_mask(D, idx, a.mask, L.words, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (bwd_tc_supported(D)) {
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_bwd_tc(D, a, status, st));
+  }
+  e = launch_bwd_pre(D, a, st);
+  if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
+  return from_cuda(e);
+}
+
 ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
                               const int32_t* idx, const float* lse_full, float* delta, void* ws,
                               size_t ws_bytes, ssa_stream_t stream) {

@@ -95,6 +95,8 @@ struct FwdArgs {
   float* lse_sel;
   float* delta;
   const float* lse_in;  // dropped-mass mode only: given lse_full, or nullptr
+  bool sparse_only;     // sparse stream alone: only selected blocks are read;
+                        // hf, lse_full and delta are not written (may be null)
 };
 
 // CUDA-core dual-stream forward (fp32 math; any supported dtype / d).
@@ -129,6 +131,10 @@ struct BwdArgs {
   int words;
   float* partials;     // per-block partial sums of (h_full - h_sparse)^2
   int n_partials;
+  // Sparse stream alone: the caller passes hf = hs, lse_full = lse_sel,
+  // gf = null and alpha = 0, so dh_f = 0 and r = 1; the kernels then skip
+  // every (query block, key block) pair that is not selected.
+  bool sparse_only;
 };
 
 cudaError_t launch_bwd_pre(const Dims& D, const BwdArgs& a, cudaStream_t st);

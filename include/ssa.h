@@ -100,7 +100,7 @@ SSA_API int ssa_version(void);
 SSA_API const char* ssa_status_string(ssa_status_t status);
 
 /* Bytes of device workspace that ssa_block_scores, ssa_bwd_dual,
- * ssa_dropped_mass and ssa_align_mse need for these dims (one size serves
+ * ssa_bwd_sparse, ssa_dropped_mass and ssa_align_mse need for these dims (one size serves
  * all of them).  Returns 0 for an invalid or empty shape.  The workspace is
  * caller-owned scratch: its contents on entry are ignored and on return
  * undefined; two calls in flight at once must not share one workspace. */
@@ -186,6 +186,42 @@ SSA_API ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q,
                           float* align_loss, const ssa_tensor_t* dQ,
                           const ssa_tensor_t* dK, const ssa_tensor_t* dV,
                           void* ws, size_t ws_bytes, ssa_stream_t stream);
+
+/* Sparse stream alone, forward (inference mode).
+ * [digest] "Training Efficiency Considerations": in sparse inference SSA
+ * runs the same block-sparse attention operation as MoBA; [summary]
+ * "4. Experimentele Resultaten" (efficiency item) reports the speed-up of
+ * this mode over full attention at long context.  Computes h_sparse and lse_sel
+ * exactly as ssa_fwd_dual does, but reads only the K/V blocks that a query
+ * block selected; the full stream and delta are not computed.
+ *   idx: as for ssa_fwd_dual (a query whose A_t is empty gets h_sparse = 0
+ *     and lse_sel = -INFINITY).
+ *   h_sparse [B, Hq, N, d] strided, dims->dtype (out); lse_sel [B, Hq, N] fp32
+ *     (out).  Needs no workspace. */
+SSA_API ssa_status_t ssa_fwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                            const ssa_tensor_t* K, const ssa_tensor_t* V,
+                            const int32_t* idx, const ssa_tensor_t* h_sparse,
+                            float* lse_sel, ssa_stream_t stream);
+
+/* Sparse stream alone, backward.
+ * Gradients of L = <g_sparse, h_sparse> for the sparse stream on its own
+ * (softmax over A_t; dropped pairs get no gradient, [digest] "The Root Cause
+ * Behind the Paradox"), with the selection held fixed.  dK and dV are summed
+ * over the g query heads of each kv head.  Only selected (query block, key
+ * block) pairs are visited.
+ *   Q, K, V, idx, h_sparse, lse_sel: as passed to / written by ssa_fwd_sparse
+ *     (or ssa_fwd_dual) for the same inputs; lse_sel must be 16-byte aligned.
+ *   g_sparse [B, Hq, N, d] dims->dtype (in, required).
+ *   dQ [B,Hq,N,d], dK, dV [B,Hkv,N,d] (out): fully overwritten; keys that no
+ *     query attends get zero.
+ *   ws: workspace of at least ssa_workspace_bytes(dims) bytes. */
+SSA_API ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                            const ssa_tensor_t* K, const ssa_tensor_t* V,
+                            const int32_t* idx, const ssa_tensor_t* h_sparse,
+                            const float* lse_sel, const ssa_tensor_t* g_sparse,
+                            const ssa_tensor_t* dQ, const ssa_tensor_t* dK,
+                            const ssa_tensor_t* dV, void* ws, size_t ws_bytes,
+                            ssa_stream_t stream);
 
 /* Standalone dropped attention mass, without V.
  * delta[t] = sum over u in D_t of exp(x_tu - lse_full[t]) ([summary]

@@ -365,3 +365,55 @@ def dropped_mass(Q, K, idx, s: int, scale: float) -> np.ndarray:
                 P_full = _masked_softmax(X, causal)
                 delta[b, h, rows] = np.where(causal & ~A, P_full, 0.0).sum(-1)
     return delta
+
+
+def forward_sparse(Q, K, V, idx, s: int, scale: float, qblocks=None) -> dict[str, np.ndarray]:
+    """The sparse stream alone: h_sparse and lse_sel, reading only selected blocks.
+
+    [digest] "Practical Implementation of SSA": the selected blocks are
+    concatenated into a reduced key/value set and the query attends over it;
+    [digest] "Training Efficiency Considerations": in sparse inference this
+    is the whole of SSA's attention (the same operation as MoBA's).  Written
+    the way the passage describes it -- gather the K/V rows of Sel(i) in
+    ascending block order, then one softmax per row with the causal mask on
+    the query's own block -- so that it checks forward_dual's masked
+    formulation independently.  Returns float64 {"h_sparse", "lse_sel"};
+    a row whose A_t is empty gets h_sparse = 0 and lse_sel = -inf.
+    """
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    B, Hq, N, d = Q.shape
+    g = Hq // K.shape[1]
+    n = N // s
+    h_sparse = np.zeros((B, Hq, N, d))
+    lse_sel = np.zeros((B, Hq, N))
+    blocks = range(n) if qblocks is None else sorted(set(int(i) for i in qblocks))
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // g
+            for i in blocks:
+                sel = sorted(set(int(j) for j in idx[b, h, i] if 0 <= j <= i))
+                keys = np.concatenate([np.arange(j * s, (j + 1) * s) for j in sel]) if sel else np.zeros(0, int)
+                for r in range(s):
+                    t = i * s + r
+                    cols = keys[keys <= t]
+                    if cols.size == 0:
+                        lse_sel[b, h, t] = -np.inf
+                        continue
+                    x = scale * (K[b, kv, cols] @ Q[b, h, t])
+                    m = x.max()
+                    w = np.exp(x - m)
+                    z = w.sum()
+                    h_sparse[b, h, t] = (w / z) @ V[b, kv, cols]
+                    lse_sel[b, h, t] = m + np.log(z)
+    return {"h_sparse": h_sparse, "lse_sel": lse_sel}
+
+
+def backward_sparse(Q, K, V, idx, s: int, scale: float, g_sparse, qblocks=None):
+    """Gradients (dQ, dK, dV) of <g_sparse, h_sparse> for the sparse stream alone.
+
+    The sparse stream's own softmax Jacobian over A_t, the selection held
+    fixed; dropped pairs get no gradient ([digest] "The Root Cause Behind the
+    Paradox": a purely sparse stream gives no gradient to the tokens it does
+    not select).  It is backward_streams with no full-stream gradient.
+    """
+    return backward_streams(Q, K, V, idx, s, scale, None, g_sparse, qblocks=qblocks)

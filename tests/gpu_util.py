@@ -70,3 +70,26 @@ def compare_selection(gpu_idx: np.ndarray, ora_idx: np.ndarray, ora_scores: np.n
             gap = abs(a - thr)
             assert gap <= NEAR_TIE_REL * max(abs(a), abs(thr)), (b, h, i, j, a, thr)
     return rows
+
+
+def custom_idx(B, H, n, k, seed, drop_diag_frac=0.0, pad_frac=0.0):
+    """Random selections: the diagonal plus k-1 random earlier blocks, with an
+    optional share of rows that omit the diagonal, pad with -1 or repeat an
+    entry.  Adjacent query blocks disagree often, which at block 64 makes many
+    key tiles selected for one half of a 128-row query tile and dropped for
+    the other."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    idx = np.full((B, H, n, k), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(n):
+                if i + 1 <= k:
+                    row = list(range(i + 1))
+                else:
+                    row = sorted(rng.choice(i, size=k - 1, replace=False).tolist() + [i])
+                if rng.random() < drop_diag_frac and len(row) > 1:
+                    row = row[:-1]
+                if rng.random() < pad_frac and len(row) > 1:
+                    row = row[:-1] + [row[0]]
+                idx[b, h, i, :len(row)] = row
+    return idx

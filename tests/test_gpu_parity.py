@@ -17,8 +17,8 @@ import torch
 from block_sparse_attention_ssa_b200 import api
 from block_sparse_attention_ssa_b200.inputs import make_scores, make_upstream
 from oracle import ssa_oracle as O
-from tests.gpu_util import (TOL, case_inputs, compare_selection, ensure_library, f64, oracle_view,
-                            rel_l2, upload)
+from tests.gpu_util import (TOL, case_inputs, compare_selection, custom_idx, ensure_library, f64,
+                            oracle_view, rel_l2, upload)
 
 pytestmark = pytest.mark.gpu
 
@@ -241,29 +241,6 @@ def test_unsupported_shape_raises():
     assert ei.value.code == api.SSA_ERR_UNSUPPORTED
 
 
-def _custom_idx(B, H, n, k, seed, drop_diag_frac=0.0, pad_frac=0.0):
-    """Random selections: the diagonal plus k-1 random earlier blocks, with an
-    optional share of rows that omit the diagonal, pad with -1 or repeat an
-    entry.  Adjacent query blocks disagree often, which at block 64 makes many
-    key tiles selected for one half of a 128-row query tile and dropped for
-    the other."""
-    rng = np.random.Generator(np.random.PCG64(seed))
-    idx = np.full((B, H, n, k), -1, dtype=np.int32)
-    for b in range(B):
-        for h in range(H):
-            for i in range(n):
-                if i + 1 <= k:
-                    row = list(range(i + 1))
-                else:
-                    row = sorted(rng.choice(i, size=k - 1, replace=False).tolist() + [i])
-                if rng.random() < drop_diag_frac and len(row) > 1:
-                    row = row[:-1]
-                if rng.random() < pad_frac and len(row) > 1:
-                    row = row[:-1] + [row[0]]
-                idx[b, h, i, :len(row)] = row
-    return idx
-
-
 @pytest.mark.parametrize("cfg", [(1, 4, 2, 1024, 128, 64, 5), (1, 2, 1, 1152, 128, 64, 4),
                                  (1, 2, 2, 1024, 128, 128, 3)])
 @pytest.mark.parametrize("extra", ["plain", "no_diag"])
@@ -273,7 +250,7 @@ def test_forward_custom_selection(cfg, extra):
     B, Hq, Hkv, N, d, s, k = cfg
     host, dev = case_inputs(B, Hq, Hkv, N, d, s, 303, "bf16")
     n = N // s
-    idx = _custom_idx(B, Hq, n, k, seed=N + k, drop_diag_frac=0.3 if extra == "no_diag" else 0.0,
+    idx = custom_idx(B, Hq, n, k, seed=N + k, drop_diag_frac=0.3 if extra == "no_diag" else 0.0,
                       pad_frac=0.2 if extra == "no_diag" else 0.0)
     dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
     out = api.alloc_forward(dims)
@@ -331,7 +308,7 @@ def test_backward_custom_selection(cfg, extra):
     B, Hq, Hkv, N, d, s, k = cfg
     host, dev = case_inputs(B, Hq, Hkv, N, d, s, 505, "bf16")
     n = N // s
-    idx = _custom_idx(B, Hq, n, k, seed=N * 3 + k, drop_diag_frac=0.3 if extra == "no_diag" else 0.0,
+    idx = custom_idx(B, Hq, n, k, seed=N * 3 + k, drop_diag_frac=0.3 if extra == "no_diag" else 0.0,
                       pad_frac=0.2 if extra == "no_diag" else 0.0)
     dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
     ws = api.alloc_workspace(dims)

@@ -356,6 +356,89 @@ def test_dropped_pairs_get_no_sparse_gradient():
         assert np.abs(dVf[0, 0, j * s:(j + 1) * s]).sum() > 0
 
 
+# ---------------------------------------------------------------- sparse stream alone
+
+def _random_selection(B, H, n, k, seed):
+    """Diagonal plus k-1 random earlier blocks per row; some rows drop their
+    diagonal, repeat an entry or pad with -1."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    idx = np.full((B, H, n, k), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(n):
+                row = list(range(i + 1)) if i + 1 <= k else sorted(
+                    rng.choice(i, size=k - 1, replace=False).tolist() + [i])
+                u = rng.random()
+                if u < 0.25 and len(row) > 1:
+                    row = row[:-1]
+                elif u < 0.4 and len(row) > 1:
+                    row = row[:-1] + [row[0]]
+                idx[b, h, i, :len(row)] = row
+    return idx
+
+
+def test_sparse_alone_equals_masked_sparse_stream():
+    """Gathering the selected blocks into a reduced K/V set ("Practical
+    Implementation of SSA") gives the same h_sparse and lse_sel as masking the
+    unselected blocks out of the whole causal row (forward_dual), for any
+    selection, including rows without their diagonal block."""
+    Q, K, V = tiny(Hq=4, Hkv=2, N=48, d=5, s=8, seed=21)
+    s, scale = 8, 0.45
+    idx = _random_selection(1, 4, 6, 3, seed=5)
+    idx[0, 1, 3] = -1  # a query block that attends nothing
+    a = O.forward_sparse(Q, K, V, idx, s, scale)
+    f = O.forward_dual(Q, K, V, idx, s, scale)
+    np.testing.assert_allclose(a["h_sparse"], f["h_sparse"], rtol=0, atol=1e-13)
+    fin = np.isfinite(f["lse_sel"])
+    assert np.array_equal(np.isfinite(a["lse_sel"]), fin) and not fin.all()
+    np.testing.assert_allclose(a["lse_sel"][fin], f["lse_sel"][fin], rtol=0, atol=1e-13)
+
+
+def test_sparse_alone_full_budget_is_causal_attention():
+    """With every causal block selected the sparse stream is textbook causal
+    attention (torch fp64 SDPA)."""
+    Q, K, V = tiny(Hq=2, Hkv=1, N=40, d=6, s=8, seed=22)
+    s, scale = 8, 1 / math.sqrt(6)
+    idx = O.select_blocks(O.block_scores(Q, K, s, scale), 5)
+    a = O.forward_sparse(Q, K, V, idx, s, scale)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q), torch.from_numpy(np.repeat(K, 2, axis=1)), torch.from_numpy(np.repeat(V, 2, axis=1)),
+        is_causal=True, scale=scale)
+    np.testing.assert_allclose(a["h_sparse"], ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_sparse_alone_reads_only_selected_blocks():
+    """K and V rows of a block that no query block selects may hold anything
+    (NaN here): the sparse stream never reads them."""
+    Q, K, V = tiny(Hq=2, Hkv=1, N=48, d=4, s=8, seed=23)
+    s, scale = 8, 0.5
+    idx = _random_selection(1, 2, 6, 2, seed=9)
+    idx[idx == 2] = -1  # nobody selects block 2, not even query block 2
+    ref = O.forward_sparse(Q, K, V, idx, s, scale)
+    K2, V2 = K.copy(), V.copy()
+    K2[:, :, 16:24] = np.nan
+    V2[:, :, 16:24] = np.nan
+    got = O.forward_sparse(Q, K2, V2, idx, s, scale)
+    np.testing.assert_array_equal(got["h_sparse"], ref["h_sparse"])
+    np.testing.assert_array_equal(got["lse_sel"], ref["lse_sel"])
+
+
+def test_sparse_backward_matches_finite_differences():
+    """Central differences of <g, h_sparse> for the sparse stream alone, the
+    selection held fixed."""
+    Q, K, V = tiny(**FD_CFG, seed=24)
+    s, scale = 8, 0.5
+    idx = _random_selection(1, FD_CFG["Hq"], FD_CFG["N"] // s, 2, seed=13)
+    g = make_upstream(Q.shape, 25).astype(np.float64)
+
+    def loss():
+        return float((g * O.forward_sparse(Q, K, V, idx, s, scale)["h_sparse"]).sum())
+
+    dQ, dK, dV = O.backward_sparse(Q, K, V, idx, s, scale, g)
+    fQ, fK, fV = _fd_grad(loss, [Q, K, V])
+    assert _rel(dQ, fQ) < 1e-6 and _rel(dK, fK) < 1e-6 and _rel(dV, fV) < 1e-6
+
+
 # ---------------------------------------------------------------- frozen regression fixture
 
 def test_golden_fixture_is_reproduced():
