@@ -17,7 +17,7 @@ when the timed region starts and are larger than L2 (Q alone is 268 MB at the
 default workload), so no explicit L2 flush is needed.  `e2e` repeats the
 step through the same C ABI with Q, K, V in pinned host memory: the
 host-to-device copies and the read-back of the alignment loss are inside its
-timed region.
+timed region (the next step's upload overlaps the current step's kernels).
 
 --impl reference times the fp64 CPU oracle (the only reference this method
 has) on a bounded sample of the same workload on the host cores.
@@ -45,7 +45,7 @@ PAGES_DROPPED_MASS = 0.47  # share of attention mass dropped by sparse attention
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gqa_16k")
@@ -121,7 +121,7 @@ class ClockSampler:
         self.thread = None
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if self.uuid:
             cmd += ["-i", self.uuid]
         try:
@@ -291,10 +291,9 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     grads = api.alloc_backward(dims, dev)
     g_sparse = torch.ones((w.B, w.Hq, w.N, w.d), dtype=tdt, device=dev)
     delta2 = torch.empty_like(out["delta"])
-    loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
     rows = ["block_scores", "select_topk", "fwd_dual", "bwd_dual", "dropped_mass"]
 
-    def step(evs=None):
+    def step(evs=None, D=D):
         if evs is not None:
             evs[0].record(stream)
         api.ssa_block_scores(dims, D["Q"], D["K"], out["scores"], ws, stream)
@@ -370,30 +369,56 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     value = world * step_flops / (ms_max * 1e-3) / 1e12
 
     # ---------------- e2e: host buffers, copies inside the timed region
+    # Every step uploads its Q, K, V from pinned host memory and reads its
+    # alignment loss back.  The upload of step k+1 runs on a copy stream into
+    # a second set of device buffers while step k computes (the two sets
+    # alternate), so the copies overlap the kernels; the timed region spans
+    # all uploads, all steps and all read-backs.
     e2e = None
     if not args.no_e2e:
         h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+        bufs = [D, {k_: torch.empty_like(v_) for k_, v_ in D.items()}]
+        copy_stream = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        consumed = [torch.cuda.Event() for _ in range(2)]
+        loss_slots = torch.empty(max(args.steps, 1), dtype=torch.float32).pin_memory()
 
-        def e2e_step():
-            for k_ in ("Q", "K", "V"):
-                D[k_].copy_(pinned[k_], non_blocking=True)
-            step()
-            loss_host.copy_(grads["align_loss"], non_blocking=True)
+        def upload(slot):
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(consumed[slot])  # the step that read this set has finished
+                for k_ in ("Q", "K", "V"):
+                    bufs[slot][k_].copy_(pinned[k_], non_blocking=True)
+                copied[slot].record(copy_stream)
+
+        def e2e_run(n_steps):
+            for e in consumed:
+                e.record(stream)
+            upload(0)
+            for k_ in range(n_steps):
+                cur = k_ % 2
+                if k_ + 1 < n_steps:
+                    upload(1 - cur)
+                stream.wait_event(copied[cur])
+                step(D=bufs[cur])
+                consumed[cur].record(stream)
+                loss_slots[k_].copy_(grads["align_loss"][0], non_blocking=True)
             stream.synchronize()
-            return float(loss_host.item())
+            return loss_slots[:n_steps].tolist()
 
-        e2e_step()
+        e2e_run(2)
         barrier()
         torch.cuda.synchronize()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        losses = e2e_run(args.steps)
         b_.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b_) / args.steps)
         e2e = {"value": world * step_flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4, "ms_per_step": e_ms}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4, "ms_per_step": e_ms,
+               "overlap": "upload of step k+1 on a copy stream during step k (two input buffer sets)",
+               "align_loss_read_back": losses[-1]}
+        del bufs[1]
 
     # ---------------- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
