@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-sparse", action="store_true", help="skip the sparse-stream-alone rows")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode row")
+    ap.add_argument("--decode-tokens", type=int, default=64, help="tokens decoded in the decode row")
     return ap.parse_args(argv)
 
 
@@ -500,6 +502,57 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
             "fwd_attended_tflops": 4 * w.d * pairs_sel / (f_ms * 1e-3) / 1e12,
             "bwd_attended_tflops": 10 * w.d * pairs_sel / (b_ms * 1e-3) / 1e12,
             "fwd_speedup_vs_fwd_dual": row_ms["fwd_dual"] / f_ms,
+        }
+
+    # ---------------- decode (sparse stream, one token per step), timed on its own:
+    # prefill the state from the first N - R tokens, then decode tokens
+    # N - R .. N - 1 of the same cache.  Memory-bound: the bytes counted are the
+    # K/V rows of the union of the selected blocks per (batch, kv head), the
+    # pooled keys scored, and q, h, qsum; not part of `value`.
+    if not args.no_decode:
+        R = max(1, min(args.decode_tokens, w.N))
+        t0 = w.N - R
+        dst = api.alloc_decode(dims, dev)
+        esz = 2 if w.dtype == "bf16" else 4
+
+        def decode_run(collect=False):
+            api.ssa_decode_prefill(dims, D["Q"], D["K"], t0, dst["qsum"], dst["kbar"], stream)
+            per_step = []
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            evs[0].record(stream)
+            for t in range(t0, w.N):
+                api.ssa_decode_step(dims, D["Q"][:, :, t:t + 1], D["K"], D["V"], t, dst["qsum"], dst["kbar"],
+                                    dst["h"], dst["lse"], dst["idx"], stream)
+                if collect:
+                    idx_t = dst["idx"].cpu().numpy()
+                    blocks = 0
+                    for b_ in range(w.B):
+                        for kv in range(w.Hkv):
+                            sel = idx_t[b_, kv * w.group:(kv + 1) * w.group].ravel()
+                            blocks += len(set(int(j) for j in sel if j >= 0))
+                    i_ = t // w.block
+                    kv_bytes = blocks * w.block * w.d * esz * 2
+                    pooled = w.B * w.Hkv * i_ * w.d * 4
+                    per_step.append(kv_bytes + pooled + w.B * w.Hq * w.d * (2 * esz + 8))
+            evs[1].record(stream)
+            torch.cuda.synchronize()
+            return evs[0].elapsed_time(evs[1]), per_step
+
+        _, bytes_steps = decode_run(collect=True)
+        decode_run()
+        ms_tot, _ = decode_run()
+        status = api.ssa_device_status(clear=True, stream=stream)
+        if status != api.SSA_OK:
+            raise RuntimeError(f"device status after the decode row: {api.status_string(status)}")
+        us = 1e3 * ms_tot / R
+        mean_bytes = sum(bytes_steps) / len(bytes_steps)
+        extra["decode"] = {
+            "entry_points": "ssa_decode_prefill (untimed) + ssa_decode_step per token (timed separately, not in value)",
+            "tokens": R, "positions": [t0, w.N - 1], "us_per_token": us,
+            "tokens_per_s": 1e6 / us * w.B, "bytes_per_token": mean_bytes,
+            "achieved_gbs": mean_bytes / (us * 1e-6) / 1e9,
+            "frac_of_hbm_peak": mean_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+            "bound": "hbm (a few MB per token: launch- and latency-bound at this size)",
         }
 
     cpu = None

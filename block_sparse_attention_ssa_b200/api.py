@@ -80,6 +80,11 @@ _SIGS = {
                                        ctypes.c_void_p, _P(ssa_tensor_t), ctypes.c_void_p, _P(ssa_tensor_t),
                                        _P(ssa_tensor_t), _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_void_p,
                                        ctypes.c_size_t, ctypes.c_void_p]),
+    "ssa_decode_prefill": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_int32,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "ssa_decode_step": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
+                                        ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, _P(ssa_tensor_t),
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "ssa_dropped_mass": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                          ctypes.c_void_p]),
@@ -202,6 +207,17 @@ def ssa_bwd_sparse(dims, Q, K, V, idx, h_sparse, lse_sel, g_sparse, dQ, dK, dV, 
         _t(dQ), _t(dK), _t(dV), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def ssa_decode_prefill(dims, Q, K, t0, qsum, kbar, stream=None) -> None:
+    _check("ssa_decode_prefill", load_library().ssa_decode_prefill(
+        ctypes.byref(dims), _t(Q), _t(K), int(t0), _p(qsum), _p(kbar), _stream(stream)))
+
+
+def ssa_decode_step(dims, q, K, V, t, qsum, kbar, h, lse, idx, stream=None) -> None:
+    _check("ssa_decode_step", load_library().ssa_decode_step(
+        ctypes.byref(dims), _t(q), _t(K), _t(V), int(t), _p(qsum), _p(kbar), _t(h), _p(lse), _p(idx),
+        _stream(stream)))
+
+
 def ssa_dropped_mass(dims, Q, K, idx, lse_full, delta, ws, stream=None) -> None:
     _check("ssa_dropped_mass", load_library().ssa_dropped_mass(
         ctypes.byref(dims), _t(Q), _t(K), _p(idx), _p(lse_full), _p(delta), _p(ws),
@@ -258,6 +274,18 @@ def alloc_backward(dims: ssa_dims_t, device="cuda") -> dict[str, torch.Tensor]:
         "dK": torch.empty((dims.B, dims.Hkv, dims.N, dims.d), dtype=dt, device=device),
         "dV": torch.empty((dims.B, dims.Hkv, dims.N, dims.d), dtype=dt, device=device),
         "align_loss": torch.empty((1,), dtype=torch.float32, device=device),
+    }
+
+
+def alloc_decode(dims: ssa_dims_t, device="cuda") -> dict[str, torch.Tensor]:
+    """Decode state (qsum, kbar) and per-step outputs (h, lse, idx)."""
+    B, Hq, Hkv, d, n, k = dims.B, dims.Hq, dims.Hkv, dims.d, dims.n_blocks, dims.k_eff
+    return {
+        "qsum": torch.zeros((B, Hq, d), dtype=torch.float32, device=device),
+        "kbar": torch.zeros((B, Hkv, n, d), dtype=torch.float32, device=device),
+        "h": torch.empty((B, Hq, 1, d), dtype=dims.torch_dtype, device=device),
+        "lse": torch.empty((B, Hq), dtype=torch.float32, device=device),
+        "idx": torch.empty((B, Hq, k), dtype=torch.int32, device=device),
     }
 
 

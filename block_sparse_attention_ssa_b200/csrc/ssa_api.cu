@@ -367,6 +367,54 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
   return from_cuda(e);
 }
 
+ssa_status_t ssa_decode_prefill(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
+                                int32_t t0, float* qsum, float* kbar, ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  DecodeArgs a{};
+  if ((s = check_tensor(D, Q, false, &a.q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &a.k)) != SSA_OK) return s;
+  if (t0 < 0 || t0 > D.N) return SSA_ERR_INVALID_ARG;
+  if (!qsum || !kbar || reinterpret_cast<uintptr_t>(qsum) % 4 || reinterpret_cast<uintptr_t>(kbar) % 4)
+    return SSA_ERR_INVALID_ARG;
+  if ((s = check_device()) != SSA_OK) return s;
+  a.qsum = qsum;
+  a.kbar = kbar;
+  a.t = t0;
+  return from_cuda(launch_decode_prefill(D, a, static_cast<cudaStream_t>(stream)));
+}
+
+ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q, const ssa_tensor_t* K,
+                             const ssa_tensor_t* V, int32_t t, float* qsum, float* kbar,
+                             const ssa_tensor_t* h, float* lse, int32_t* idx, ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (empty) return SSA_OK;
+  DecodeArgs a{};
+  if ((s = check_tensor(D, q, false, &a.q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &a.k)) != SSA_OK) return s;
+  if ((s = check_tensor(D, V, false, &a.v)) != SSA_OK) return s;
+  if ((s = check_tensor(D, h, false, &a.h)) != SSA_OK) return s;
+  if (t < 0 || t >= D.N) return SSA_ERR_INVALID_ARG;
+  if (!qsum || !kbar || !lse || !idx) return SSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(qsum) % 4 || reinterpret_cast<uintptr_t>(kbar) % 4 ||
+      reinterpret_cast<uintptr_t>(lse) % 4 || reinterpret_cast<uintptr_t>(idx) % 4)
+    return SSA_ERR_INVALID_ARG;
+  if (decode_smem_bytes(D) > 232448) return SSA_ERR_UNSUPPORTED;
+  if ((s = check_device()) != SSA_OK) return s;
+  a.lse = lse;
+  a.idx = idx;
+  a.qsum = qsum;
+  a.kbar = kbar;
+  a.t = t;
+  return from_cuda(launch_decode(D, a, static_cast<cudaStream_t>(stream)));
+}
+
 ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
                               const int32_t* idx, const float* lse_full, float* delta, void* ws,
                               size_t ws_bytes, ssa_stream_t stream) {

@@ -143,6 +143,22 @@ bool bwd_tc_supported(const Dims& D);
 cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* dev_status, cudaStream_t st);
 cudaError_t launch_bwd_simt(const Dims& D, const BwdArgs& a, cudaStream_t st);
 
+struct DecodeArgs {
+  TensorRef q, k, v, h;  // q, h: [B,Hq,1,d] (prefill: q = the prompt's Q [B,Hq,N,d]); k, v: caches [B,Hkv,N,d]
+  float* lse;            // [B,Hq]
+  int32_t* idx;          // [B,Hq,k_eff]
+  float* qsum;           // [B,Hq,d] running sum of the current block's queries
+  float* kbar;           // [B,Hkv,n,d] means of the complete key blocks
+  int t;                 // position of the new token (prefill: prompt length)
+};
+
+// Sparse-stream decode of the token at position a.t (CUDA cores).
+cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, cudaStream_t st);
+// Decode state from a prompt of a.t tokens: kbar of its complete blocks, qsum of the partial block.
+cudaError_t launch_decode_prefill(const Dims& D, const DecodeArgs& a, cudaStream_t st);
+// Dynamic shared memory the decode kernel needs for these dims.
+size_t decode_smem_bytes(const Dims& D);
+
 // One-CTA kernel whose bounded barrier wait runs out: records SSA_ERR_TIMEOUT.
 cudaError_t launch_selftest_timeout(int32_t* status, long long limit_cycles, cudaStream_t st);
 

@@ -223,6 +223,48 @@ SSA_API ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* 
                             const ssa_tensor_t* dV, void* ws, size_t ws_bytes,
                             ssa_stream_t stream);
 
+/* Decode (one generated token at a time), sparse stream.
+ * [digest] "Training Efficiency Considerations": at inference SSA runs its
+ * sparse attention alone; [skill] "6. Inference with Sparse or Full Mode":
+ * generation appends one token per step.  The token at position t (block
+ * i = t/s) selects blocks by the forward's rule, with the query side read as
+ * the mean of the queries of block i seen so far (positions i*s..t; at the
+ * last token of a block this is exactly the forward's block mean):
+ *   score_j = scale * qbar . kbar_j (j < i, kbar_j the mean of key block j),
+ *   Sel = {i} + the k_eff-1 best scores (ties to the smaller j), or {0..i}
+ *   when i + 1 <= k_eff;  h = softmax over A_t of scale q_t . k_u, times V.
+ * Two state buffers carry the pooling between calls:
+ *   qsum [B, Hq, d] fp32: sum of the queries of the current block so far;
+ *   kbar [B, Hkv, n, d] fp32: means of the complete key blocks.
+ * dims->N is the capacity of the K/V caches [B, Hkv, N, d] (a multiple of
+ * block); Hq/Hkv * n * 4 bytes of scores must fit the decode kernel's shared
+ * memory (SSA_ERR_UNSUPPORTED otherwise; every workload here fits). */
+
+/* Builds the decode state from a prompt of t0 tokens (0 <= t0 <= N): kbar of
+ * the complete blocks 0 .. t0/s - 1 and qsum of the queries of the partial
+ * block (rows (t0/s)*s .. t0-1; zero when t0 is a multiple of s).
+ *   Q [B, Hq, N, d], K [B, Hkv, N, d] (in): the prompt's rows 0 .. t0-1. */
+SSA_API ssa_status_t ssa_decode_prefill(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                                const ssa_tensor_t* K, int32_t t0, float* qsum,
+                                float* kbar, ssa_stream_t stream);
+
+/* One decode step for the token at position t (0 <= t < N).
+ *   q [B, Hq, 1, d] (in): the token's queries.
+ *   K, V [B, Hkv, N, d] (in): caches whose rows 0 .. t hold the keys and
+ *     values so far (the caller has written row t).
+ *   qsum, kbar (in/out): state as left by ssa_decode_prefill(t0 = t) or by
+ *     the call for t-1; q_t is added to qsum (which restarts at a block's
+ *     first token) and, when t is the last token of block i, kbar[i] is set
+ *     to the mean of that block's keys.
+ *   h [B, Hq, 1, d] (out), lse [B, Hq] fp32 (out, natural log of the
+ *     softmax normaliser), idx [B, Hq, k_eff] int32 (out, Sel ascending,
+ *     -1 padded).
+ * Calls for consecutive tokens must be ordered (same stream). */
+SSA_API ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q,
+                             const ssa_tensor_t* K, const ssa_tensor_t* V, int32_t t,
+                             float* qsum, float* kbar, const ssa_tensor_t* h, float* lse,
+                             int32_t* idx, ssa_stream_t stream);
+
 /* Standalone dropped attention mass, without V.
  * delta[t] = sum over u in D_t of exp(x_tu - lse_full[t]) ([summary]
  * "1. Probleemstelling"; [digest] "Phenomenon 3" reports this quantity for

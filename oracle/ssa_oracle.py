@@ -34,7 +34,8 @@ notes):
   * no gradient flows through the selection or through delta.
 Parity status: every function here is pinned by the CPU tests in
 tests/test_oracle_pins.py (closed forms, brute force, torch's fp64 causal
-attention, finite differences).
+attention, finite differences, and the decode functions against the
+forward's rule at the end of each block).
 """
 from __future__ import annotations
 
@@ -417,3 +418,61 @@ def backward_sparse(Q, K, V, idx, s: int, scale: float, g_sparse, qblocks=None):
     not select).  It is backward_streams with no full-stream gradient.
     """
     return backward_streams(Q, K, V, idx, s, scale, None, g_sparse, qblocks=qblocks)
+
+
+def decode_select(q_prefix, K, t: int, s: int, k: int, scale: float, n_cache: int | None = None) -> np.ndarray:
+    """Blocks kept for the generated token at position t: [B, Hq, k_eff] int32.
+
+    The forward's rule ([digest] "Practical Implementation of SSA": score the
+    query against every earlier block representation, keep the top-k; the
+    current block always kept) applied to the tokens that exist at decode
+    time: the query side is the mean of the current block's queries seen so
+    far (q_prefix holds rows i*s .. t of block i = t // s), the key side the
+    means of the complete blocks j < i.  k_eff = min(k, n_cache), n_cache the
+    number of blocks of the cache (default (t+1) rounded up to blocks).
+    """
+    Qp, K = _f64(q_prefix), _f64(K)
+    B, Hq, _, d = Qp.shape
+    g = Hq // K.shape[1]
+    i = t // s
+    n = n_cache if n_cache is not None else i + 1
+    kk = min(int(k), n)
+    qbar = Qp.mean(axis=2)                                   # [B,Hq,d]
+    idx = np.full((B, Hq, kk), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            if i + 1 <= kk:
+                chosen = np.arange(i + 1)
+            else:
+                kbar = K[b, h // g, : i * s].reshape(i, s, d).mean(axis=1)   # complete blocks
+                sc = scale * (kbar @ qbar[b, h])
+                order = np.lexsort((np.arange(i), -sc))
+                chosen = np.sort(np.append(order[: kk - 1], i))
+            idx[b, h, : chosen.size] = chosen
+    return idx
+
+
+def decode_attend(q_t, K, V, t: int, s: int, idx, scale: float):
+    """(h [B,Hq,d], lse [B,Hq]) of the token at position t over its kept blocks.
+
+    Softmax of scale * q_t . k_u over A_t = {u <= t : u // s in Sel}, applied
+    to V; Sel is idx[b, h] (entries outside [0, t // s] ignored).
+    """
+    q, K, V = _f64(q_t), _f64(K), _f64(V)
+    B, Hq, d = q.shape
+    g = Hq // K.shape[1]
+    i = t // s
+    h_out = np.zeros((B, Hq, d))
+    lse = np.full((B, Hq), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            sel = sorted(set(int(j) for j in idx[b, h] if 0 <= j <= i))
+            cols = np.array([u for j in sel for u in range(j * s, j * s + s) if u <= t], dtype=int)
+            if cols.size == 0:
+                continue
+            x = scale * (K[b, h // g, cols] @ q[b, h])
+            m = x.max()
+            w = np.exp(x - m)
+            h_out[b, h] = (w / w.sum()) @ V[b, h // g, cols]
+            lse[b, h] = m + np.log(w.sum())
+    return h_out, lse

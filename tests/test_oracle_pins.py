@@ -439,6 +439,76 @@ def test_sparse_backward_matches_finite_differences():
     assert _rel(dQ, fQ) < 1e-6 and _rel(dK, fK) < 1e-6 and _rel(dV, fV) < 1e-6
 
 
+# ---------------------------------------------------------------- decode
+
+def test_decode_at_block_end_equals_forward_rule():
+    """At the last token of a block the prefix of the block is the whole block,
+    so the decode selection is the forward's selection of that query block and
+    the decode output is the forward's sparse-stream row."""
+    Q, K, V = tiny(Hq=4, Hkv=2, N=48, d=5, s=8, seed=31)
+    s, k, scale = 8, 3, 0.4
+    n = 6
+    ref_idx = O.select_blocks(O.block_scores(Q, K, s, scale), k)
+    ref = O.forward_sparse(Q, K, V, ref_idx, s, scale)
+    for i in range(n):
+        t = i * s + s - 1
+        idx = O.decode_select(Q[:, :, i * s:t + 1], K, t, s, k, scale, n_cache=n)
+        np.testing.assert_array_equal(idx, ref_idx[:, :, i])
+        h, lse = O.decode_attend(Q[:, :, t], K, V, t, s, idx, scale)
+        np.testing.assert_allclose(h, ref["h_sparse"][:, :, t], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse, ref["lse_sel"][:, :, t], rtol=0, atol=1e-13)
+
+
+def test_decode_partial_block_uses_prefix_mean():
+    """Mid-block, the query side is the mean of the block's queries so far;
+    the kept set is the best-scoring (k-1)-subset of earlier blocks, found by
+    enumeration from scores summed by explicit loops."""
+    Q, K, _ = tiny(Hq=2, Hkv=1, N=48, d=3, s=8, seed=32)
+    s, k, scale = 8, 3, 0.7
+    for t in (19, 27, 41, 44):
+        i = t // s
+        idx = O.decode_select(Q[:, :, i * s:t + 1], K, t, s, k, scale, n_cache=6)
+        for h in range(2):
+            qbar = [sum(Q[0, h, u, c] for u in range(i * s, t + 1)) / (t - i * s + 1) for c in range(3)]
+            sc = []
+            for j in range(i):
+                kbar = [sum(K[0, 0, u, c] for u in range(j * s, j * s + s)) / s for c in range(3)]
+                sc.append(scale * sum(qbar[c] * kbar[c] for c in range(3)))
+            best = max(itertools.combinations(range(i), k - 1), key=lambda c: sum(sc[j] for j in c))
+            assert sorted(best) + [i] == [int(j) for j in idx[0, h] if j >= 0]
+
+
+def test_decode_uniform_scores_tie_rule():
+    """Q = 0: every score ties, so the smallest indices win: Sel = {0..k-2, i};
+    the weights are uniform, so h is the mean of V over the kept keys <= t."""
+    _, K, V = tiny(Hq=1, N=64, d=3, s=8, seed=33)
+    s, k = 8, 3
+    q = np.zeros((1, 1, 3))
+    for t in (20, 35, 63):
+        i = t // s
+        idx = O.decode_select(np.zeros((1, 1, t - i * s + 1, 3)), K, t, s, k, 0.5, n_cache=8)
+        assert [int(j) for j in idx[0, 0]] == [0, 1, i]
+        h, lse = O.decode_attend(q, K, V, t, s, idx, 0.5)
+        A = [u for u in range(t + 1) if u // s in (0, 1, i)]
+        np.testing.assert_allclose(h[0, 0], V[0, 0, A].mean(0), atol=1e-14)
+        assert lse[0, 0] == pytest.approx(math.log(len(A)), abs=1e-14)
+
+
+def test_decode_full_budget_is_causal_attention():
+    """With every block kept the decode output is the last row of textbook
+    causal attention over the prefix (torch fp64 SDPA)."""
+    Q, K, V = tiny(Hq=4, Hkv=2, N=40, d=6, s=8, seed=34)
+    s, scale = 8, 1 / math.sqrt(6)
+    for t in (0, 9, 23, 39):
+        i = t // s
+        idx = O.decode_select(Q[:, :, i * s:t + 1], K, t, s, 5, scale, n_cache=5)
+        h, _ = O.decode_attend(Q[:, :, t], K, V, t, s, idx, scale)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q[:, :, :t + 1]), torch.from_numpy(np.repeat(K[:, :, :t + 1], 2, axis=1)),
+            torch.from_numpy(np.repeat(V[:, :, :t + 1], 2, axis=1)), is_causal=True, scale=scale)
+        np.testing.assert_allclose(h, ref.numpy()[:, :, t], rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- frozen regression fixture
 
 def test_golden_fixture_is_reproduced():
