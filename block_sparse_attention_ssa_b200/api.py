@@ -84,7 +84,8 @@ _SIGS = {
                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "ssa_decode_step": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
                                         ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, _P(ssa_tensor_t),
-                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                        ctypes.c_void_p]),
     "ssa_dropped_mass": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                          ctypes.c_void_p]),
@@ -212,10 +213,10 @@ def ssa_decode_prefill(dims, Q, K, t0, qsum, kbar, stream=None) -> None:
         ctypes.byref(dims), _t(Q), _t(K), int(t0), _p(qsum), _p(kbar), _stream(stream)))
 
 
-def ssa_decode_step(dims, q, K, V, t, qsum, kbar, h, lse, idx, stream=None) -> None:
+def ssa_decode_step(dims, q, K, V, t, qsum, kbar, h, lse, idx, ws, stream=None) -> None:
     _check("ssa_decode_step", load_library().ssa_decode_step(
         ctypes.byref(dims), _t(q), _t(K), _t(V), int(t), _p(qsum), _p(kbar), _t(h), _p(lse), _p(idx),
-        _stream(stream)))
+        _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def ssa_dropped_mass(dims, Q, K, idx, lse_full, delta, ws, stream=None) -> None:

@@ -78,7 +78,7 @@ struct Layout {
   size_t qbar, kbar;          // block scores
   size_t dhf, doc, Df, Dc, mask, partials;  // backward
   size_t lse;                 // dropped mass
-  size_t bytes_scores, bytes_bwd, bytes_dropped, bytes_align;
+  size_t bytes_scores, bytes_bwd, bytes_dropped, bytes_align, bytes_decode;
   int words, n_partials;
 };
 
@@ -102,6 +102,7 @@ Layout layout(const Dims& D) {
   L.lse = 0;
   L.bytes_dropped = align_up(rows * 4);
   L.bytes_align = align_up((size_t)L.n_partials * 4);
+  L.bytes_decode = align_up(decode_ws_bytes(D));
   return L;
 }
 
@@ -110,6 +111,7 @@ size_t total_bytes(const Layout& L) {
   if (L.bytes_bwd > m) m = L.bytes_bwd;
   if (L.bytes_dropped > m) m = L.bytes_dropped;
   if (L.bytes_align > m) m = L.bytes_align;
+  if (L.bytes_decode > m) m = L.bytes_decode;
   return m;
 }
 
@@ -389,7 +391,8 @@ ssa_status_t ssa_decode_prefill(const ssa_dims_t* dims, const ssa_tensor_t* Q, c
 
 ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q, const ssa_tensor_t* K,
                              const ssa_tensor_t* V, int32_t t, float* qsum, float* kbar,
-                             const ssa_tensor_t* h, float* lse, int32_t* idx, ssa_stream_t stream) {
+                             const ssa_tensor_t* h, float* lse, int32_t* idx, void* ws, size_t ws_bytes,
+                             ssa_stream_t stream) {
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -406,7 +409,9 @@ ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q, cons
       reinterpret_cast<uintptr_t>(lse) % 4 || reinterpret_cast<uintptr_t>(idx) % 4)
     return SSA_ERR_INVALID_ARG;
   if (decode_smem_bytes(D) > 232448) return SSA_ERR_UNSUPPORTED;
+  if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
   if ((s = check_device()) != SSA_OK) return s;
+  a.ws = ws;
   a.lse = lse;
   a.idx = idx;
   a.qsum = qsum;

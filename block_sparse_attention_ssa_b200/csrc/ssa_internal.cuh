@@ -150,14 +150,17 @@ struct DecodeArgs {
   float* qsum;           // [B,Hq,d] running sum of the current block's queries
   float* kbar;           // [B,Hkv,n,d] means of the complete key blocks
   int t;                 // position of the new token (prefill: prompt length)
+  void* ws;              // decode step: caller workspace (decode_ws_bytes)
 };
 
 // Sparse-stream decode of the token at position a.t (CUDA cores).
 cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, cudaStream_t st);
 // Decode state from a prompt of a.t tokens: kbar of its complete blocks, qsum of the partial block.
 cudaError_t launch_decode_prefill(const Dims& D, const DecodeArgs& a, cudaStream_t st);
-// Dynamic shared memory the decode kernel needs for these dims.
+// Dynamic shared memory the decode kernels need for these dims.
 size_t decode_smem_bytes(const Dims& D);
+// Workspace bytes of one decode step.
+size_t decode_ws_bytes(const Dims& D);
 
 // One-CTA kernel whose bounded barrier wait runs out: records SSA_ERR_TIMEOUT.
 cudaError_t launch_selftest_timeout(int32_t* status, long long limit_cycles, cudaStream_t st);

@@ -100,7 +100,7 @@ SSA_API int ssa_version(void);
 SSA_API const char* ssa_status_string(ssa_status_t status);
 
 /* Bytes of device workspace that ssa_block_scores, ssa_bwd_dual,
- * ssa_bwd_sparse, ssa_dropped_mass and ssa_align_mse need for these dims (one size serves
+ * ssa_bwd_sparse, ssa_decode_step, ssa_dropped_mass and ssa_align_mse need for these dims (one size serves
  * all of them).  Returns 0 for an invalid or empty shape.  The workspace is
  * caller-owned scratch: its contents on entry are ignored and on return
  * undefined; two calls in flight at once must not share one workspace. */
@@ -259,11 +259,14 @@ SSA_API ssa_status_t ssa_decode_prefill(const ssa_dims_t* dims, const ssa_tensor
  *   h [B, Hq, 1, d] (out), lse [B, Hq] fp32 (out, natural log of the
  *     softmax normaliser), idx [B, Hq, k_eff] int32 (out, Sel ascending,
  *     -1 padded).
+ *   ws: workspace of at least ssa_workspace_bytes(dims) bytes (holds the
+ *     union of the kept blocks and the partial softmax states of the split
+ *     attention).
  * Calls for consecutive tokens must be ordered (same stream). */
 SSA_API ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q,
                              const ssa_tensor_t* K, const ssa_tensor_t* V, int32_t t,
                              float* qsum, float* kbar, const ssa_tensor_t* h, float* lse,
-                             int32_t* idx, ssa_stream_t stream);
+                             int32_t* idx, void* ws, size_t ws_bytes, ssa_stream_t stream);
 
 /* Standalone dropped attention mass, without V.
  * delta[t] = sum over u in D_t of exp(x_tu - lse_full[t]) ([summary]

@@ -56,6 +56,7 @@ def test_decode_sequence(name):
     dims = api.make_dims(B, Hq, Hkv, N, d, s, k, dt)
     scale = 1 / math.sqrt(d)
     st = api.alloc_decode(dims)
+    ws = api.alloc_workspace(dims)
     st["qsum"].fill_(float("nan"))  # prefill must define every entry it owns
     api.ssa_decode_prefill(dims, dev["Q"], dev["K"], t0, st["qsum"], st["kbar"])
     g = Hq // Hkv
@@ -64,7 +65,7 @@ def test_decode_sequence(name):
     for t in range(t0, t0 + L):
         i = t // s
         api.ssa_decode_step(dims, dev["Q"][:, :, t:t + 1], dev["K"], dev["V"], t, st["qsum"], st["kbar"],
-                            st["h"], st["lse"], st["idx"])
+                            st["h"], st["lse"], st["idx"], ws)
         torch.cuda.synchronize()
         gidx = st["idx"].cpu().numpy()
         qp = host["Q"][:, :, i * s:t + 1].astype(np.float64)
@@ -103,10 +104,11 @@ def test_decode_rejects_bad_positions():
     host, dev = case_inputs(B, Hq, Hkv, N, d, s, 3, "f32")
     dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "f32")
     st = api.alloc_decode(dims)
+    ws = api.alloc_workspace(dims)
     for t in (-1, N):
         with pytest.raises(api.SsaError) as ei:
             api.ssa_decode_step(dims, dev["Q"][:, :, 0:1], dev["K"], dev["V"], t, st["qsum"], st["kbar"],
-                                st["h"], st["lse"], st["idx"])
+                                st["h"], st["lse"], st["idx"], ws)
         assert ei.value.code == api.SSA_ERR_INVALID_ARG
     with pytest.raises(api.SsaError):
         api.ssa_decode_prefill(dims, dev["Q"], dev["K"], N + 1, st["qsum"], st["kbar"])
@@ -121,10 +123,11 @@ def test_decode_last_token_full_size(wname):
     dev = {x: torch.from_numpy(host[x + "_bits"].view(np.int16)).view(torch.bfloat16).cuda() for x in "QKV"}
     dims = api.make_dims(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, w.topk, w.dtype)
     st = api.alloc_decode(dims)
+    ws = api.alloc_workspace(dims)
     t = w.N - 1
     api.ssa_decode_prefill(dims, dev["Q"], dev["K"], t, st["qsum"], st["kbar"])
     api.ssa_decode_step(dims, dev["Q"][:, :, t:t + 1], dev["K"], dev["V"], t, st["qsum"], st["kbar"], st["h"],
-                        st["lse"], st["idx"])
+                        st["lse"], st["idx"], ws)
     torch.cuda.synchronize()
     assert api.ssa_device_status() == api.SSA_OK
     s, scale = w.block, w.scale
