@@ -425,12 +425,26 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     # ---------------- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     row_flops = {"fwd_dual": F["fwd"], "bwd_dual": F["bwd"], "dropped_mass": F["dropped"]}
-    scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_tc_kernel)",
-              "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_tc + finish + bwd_dkv_tc + bwd_dq_tc kernels",
-              "dropped_mass": "entry point ssa_dropped_mass = one kernel (dropped_tc_kernel)"}
+    # bf16 with d = 128 and blocks of 64 / 128 runs on the tensor-core kernels;
+    # every other shape on the CUDA-core kernels (fp32 FMA bound)
+    tc_path = w.dtype == "bf16" and w.d == 128 and w.block in (64, 128)
+    if tc_path:
+        scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_tc_kernel)",
+                  "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_tc + finish + bwd_dkv_tc + bwd_dq_tc kernels",
+                  "dropped_mass": "entry point ssa_dropped_mass = one kernel (dropped_tc_kernel)"}
+    else:
+        scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_simt_kernel, CUDA cores)",
+                  "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre + finish + bwd_dq + bwd_dkv kernels (CUDA cores)",
+                  "dropped_mass": "entry point ssa_dropped_mass = one kernel (fwd_simt_kernel without V, CUDA cores)"}
+    # fp32 FMA peak: 148 SMs x 128 FP32 lanes x 2 FLOP x the max SM clock
+    alu_peak = 148 * 128 * 2 * 1965e6 / 1e12
 
     def roof(r):
         achieved = row_flops[r] / (row_ms[r] * 1e-3) / 1e12
+        if not tc_path:
+            return {"bound": "alu", "kernel": r, "scope": scopes[r], "achieved": achieved, "peak": alu_peak,
+                    "unit": "TFLOP/s", "frac": achieved / alu_peak, "traffic": None,
+                    "peak_source": "fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz (attended FLOPs counted)"}
         return {"bound": "tensor", "kernel": r, "scope": scopes[r], "achieved": achieved,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops_sustained"],
@@ -443,8 +457,11 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     per_row = {r: {"ms": row_ms[r]} for r in rows}
     for r, f in row_flops.items():
         per_row[r]["attended_tflops"] = f / (row_ms[r] * 1e-3) / 1e12
-        per_row[r]["frac_of_sustained_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops_sustained"]
-        per_row[r]["frac_of_burst_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops"]
+        if tc_path:
+            per_row[r]["frac_of_sustained_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops_sustained"]
+            per_row[r]["frac_of_burst_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops"]
+        else:
+            per_row[r]["frac_of_fp32_fma_peak"] = per_row[r]["attended_tflops"] / alu_peak
     fwd_ms = row_ms["block_scores"] + row_ms["select_topk"] + row_ms["fwd_dual"]
     extra = {
         "fwd_tflops": F["fwd"] / (fwd_ms * 1e-3) / 1e12,

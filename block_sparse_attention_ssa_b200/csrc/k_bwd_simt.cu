@@ -79,7 +79,12 @@ __global__ void __launch_bounds__(NT) bwd_pre_kernel(BwdArgs a, int Hq, int N, f
 
 // ------------------------------------------------------------------ dQ
 // grid (N/64, Hq, B).  For its 64 query rows the CTA walks every causal key
-// tile; a tile belongs to A or to D for all 64 rows (one query block).
+// tile.  With blocks of 64 or more keys a tile belongs to A or to D for all
+// 64 rows; with smaller blocks each row's 64-bit mask of selected keys picks,
+// element by element, the combined (dO_c, D_c) or the full-stream
+// (dh_f, D_f) gradient.
+constexpr int QBMAX = 4;  // query blocks in a 64-row tile (block >= 16)
+
 template <int D>
 struct DqSmem {
   float q[BT][D];
@@ -89,8 +94,37 @@ struct DqSmem {
   float v[BT][D + 1];
   float p[BT][BT + 1];
   float lse[BT], dc[BT], df[BT];
-  uint32_t sel[64];
+  unsigned long long cm[BT];  // per query row: keys of the tile in selected blocks
+  uint32_t sel[QBMAX][64];
 };
+
+// xs = Q K^T, dpc = dO_c V^T, dpf = dh_f V^T for a 4 x 4 patch (only the
+// products a tile needs).
+template <int D, bool NC, bool NF>
+__device__ __forceinline__ void dq_dots(const DqSmem<D>& S, int ty, int tx, float (&xs)[4][4], float (&dpc)[4][4],
+                                        float (&dpf)[4][4]) {
+#pragma unroll 4
+  for (int c = 0; c < D; ++c) {
+    float kv[4], vv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      kv[j] = S.k[tx * 4 + j][c];
+      vv[j] = S.v[tx * 4 + j][c];
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float qv = S.q[ty * 4 + r][c];
+      const float oc = NC ? S.doc[ty * 4 + r][c] : 0.f;
+      const float of = NF ? S.dhf[ty * 4 + r][c] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xs[r][j] = fmaf(qv, kv[j], xs[r][j]);
+        if (NC) dpc[r][j] = fmaf(oc, vv[j], dpc[r][j]);
+        if (NF) dpf[r][j] = fmaf(of, vv[j], dpf[r][j]);
+      }
+    }
+  }
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(NT) bwd_dq_kernel(BwdArgs a, int Hq, int g, int N, int s, int n,
@@ -98,13 +132,16 @@ __global__ void __launch_bounds__(NT) bwd_dq_kernel(BwdArgs a, int Hq, int g, in
   extern __shared__ __align__(16) unsigned char smem_raw[];
   DqSmem<D>& S = *reinterpret_cast<DqSmem<D>*>(smem_raw);
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z, kvh = h / g;
-  const int t0 = qt * BT, iblk = t0 / s, tid = threadIdx.x;
+  const int t0 = qt * BT, ib0 = t0 / s, tid = threadIdx.x;
+  const int nqb = s >= BT ? 1 : BT / s;
   const int64_t rbase = ((int64_t)b * Hq + h) * N + t0;
   constexpr int VEC = Vec16<T>::kN;
 
   const int words = (n + 31) / 32;
-  for (int w = tid; w < words; w += NT)
-    S.sel[w] = a.mask[(((int64_t)b * Hq + h) * n + iblk) * a.words + w];
+  for (int w = tid; w < QBMAX * 64; w += NT) {
+    const int qb = w / 64, ww = w % 64;
+    S.sel[qb][ww] = (qb < nqb && ww < words) ? a.mask[(((int64_t)b * Hq + h) * n + ib0 + qb) * a.words + ww] : 0u;
+  }
   for (int e = tid; e < BT * D / VEC; e += NT) {
     const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
     Vec16<T>::load(row_ptr<T>(a.q, b, h, t0 + r) + c, &S.q[r][c]);
@@ -130,10 +167,19 @@ __global__ void __launch_bounds__(NT) bwd_dq_kernel(BwdArgs a, int Hq, int g, in
     for (int c = 0; c < CW; ++c) dq[r][c] = 0.f;
 
   for (int kt = 0; kt <= qt; ++kt) {
-    const int u0 = kt * BT, jblk = u0 / s;
+    const int u0 = kt * BT;
     __syncthreads();
-    const bool sel = (S.sel[jblk >> 5] >> (jblk & 31)) & 1u;
-    if (a.sparse_only && !sel) continue;  // uniform over the CTA
+    bool myA = false, myD = false;
+    if (tid < BT) {
+      const unsigned long long causal = causal_mask(t0 + tid, u0);
+      const unsigned long long cm = tile_keep_mask(S.sel[(t0 + tid) / s - ib0], u0, s) & causal;
+      S.cm[tid] = cm;
+      myA = cm != 0ull;
+      myD = (causal & ~cm) != 0ull;
+    }
+    const bool anyA = __syncthreads_or(myA);
+    const bool anyD = __syncthreads_or(myD) && !a.sparse_only;  // dropped pairs: no sparse-stream gradient
+    if (!anyA && !anyD) continue;  // uniform over the CTA
     for (int e = tid; e < BT * D / VEC; e += NT) {
       const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
       float tk[VEC], tv[VEC];
@@ -146,44 +192,32 @@ __global__ void __launch_bounds__(NT) bwd_dq_kernel(BwdArgs a, int Hq, int g, in
       }
     }
     __syncthreads();
-    const float (*dO)[D] = sel ? S.doc : S.dhf;
-    const float* Drow = sel ? S.dc : S.df;
-    float xs[4][4], dp[4][4];
+    float xs[4][4], dpc[4][4], dpf[4][4];
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) xs[r][c] = dp[r][c] = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < D; ++c) {
-      float kv[4], vv[4];
+      for (int c = 0; c < 4; ++c) xs[r][c] = dpc[r][c] = dpf[r][c] = 0.f;
+    if (anyA && anyD) dq_dots<D, true, true>(S, ty, tx, xs, dpc, dpf);
+    else if (anyA) dq_dots<D, true, false>(S, ty, tx, xs, dpc, dpf);
+    else dq_dots<D, false, true>(S, ty, tx, xs, dpc, dpf);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int row = ty * 4 + r;
+      const unsigned long long cm = S.cm[row];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        kv[j] = S.k[tx * 4 + j][c];
-        vv[j] = S.v[tx * 4 + j][c];
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float qv = S.q[ty * 4 + r][c];
-        const float ov = dO[ty * 4 + r][c];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          xs[r][j] = fmaf(qv, kv[j], xs[r][j]);
-          dp[r][j] = fmaf(ov, vv[j], dp[r][j]);
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int row = ty * 4 + r, col = tx * 4 + j;
+        const int col = tx * 4 + j;
         float ds = 0.f;
         if (u0 + col <= t0 + row) {
-          const float p = expf(scale * xs[r][j] - S.lse[row]);
-          ds = p * (dp[r][j] - Drow[row]);
+          const bool in_a = (cm >> col) & 1ull;
+          if (in_a || anyD) {
+            const float p = expf(scale * xs[r][j] - S.lse[row]);
+            ds = in_a ? p * (dpc[r][j] - S.dc[row]) : p * (dpf[r][j] - S.df[row]);
+          }
         }
         S.p[row][col] = ds;
       }
+    }
     __syncthreads();
 #pragma unroll 4
     for (int kk = 0; kk < BT; ++kk) {
@@ -207,20 +241,50 @@ __global__ void __launch_bounds__(NT) bwd_dq_kernel(BwdArgs a, int Hq, int g, in
 }
 
 // ------------------------------------------------------------------ dK, dV
-// grid (N/64, Hkv, B).  For its 64 keys (one key block j) the CTA walks the g
-// query heads of the group and every causal query tile; whether the keys are
-// selected for a query tile is read from the selected-block bit set of that
-// head's query block.
+// grid (N/64, Hkv, B).  For its 64 keys the CTA walks the g query heads of the
+// group and every causal query tile.  Each query row's 64-bit mask of
+// selected keys (from its query block's bit set) decides, element by
+// element, whether the pair is selected (combined gradient dO_c, D_c) or
+// dropped (dh_f, D_f); dV takes P_A^T dO_c + P_D^T dh_f.
 template <int D>
 struct DkvSmem {
   float k[BT][D + 1];
   float v[BT][D + 1];
   float q[BT][D + 1];
-  float dO[BT][D + 1];
-  float p[BT][BT + 1];   // P^T: [key][query]
+  float doc[BT][D + 1];
+  float dhf[BT][D + 1];
+  float p[BT][BT + 1];   // P^T on selected pairs: [key][query]
+  float pd[BT][BT + 1];  // P^T on dropped pairs
   float ds[BT][BT + 1];  // dS^T
-  float lse[BT], dd[BT];
+  float lse[BT], dc[BT], df[BT];
+  unsigned long long cm[BT];  // per query row: keys of this tile in selected blocks (causal ones)
 };
+
+template <int D, bool NC, bool NF>
+__device__ __forceinline__ void dkv_dots(const DkvSmem<D>& S, int ty, int tx, float (&xs)[4][4],
+                                         float (&dpc)[4][4], float (&dpf)[4][4]) {
+#pragma unroll 4
+  for (int c = 0; c < D; ++c) {
+    float qv[4], oc[4], of[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      qv[j] = S.q[tx * 4 + j][c];
+      oc[j] = NC ? S.doc[tx * 4 + j][c] : 0.f;
+      of[j] = NF ? S.dhf[tx * 4 + j][c] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float kv = S.k[ty * 4 + r][c];
+      const float vv = S.v[ty * 4 + r][c];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xs[r][j] = fmaf(kv, qv[j], xs[r][j]);
+        if (NC) dpc[r][j] = fmaf(vv, oc[j], dpc[r][j]);
+        if (NF) dpf[r][j] = fmaf(vv, of[j], dpf[r][j]);
+      }
+    }
+  }
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(NT) bwd_dkv_kernel(BwdArgs a, int Hq, int g, int N, int s, int n,
@@ -228,7 +292,7 @@ __global__ void __launch_bounds__(NT) bwd_dkv_kernel(BwdArgs a, int Hq, int g, i
   extern __shared__ __align__(16) unsigned char smem_raw[];
   DkvSmem<D>& S = *reinterpret_cast<DkvSmem<D>*>(smem_raw);
   const int kt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int u0 = kt * BT, jblk = u0 / s, tid = threadIdx.x;
+  const int u0 = kt * BT, tid = threadIdx.x;
   const int nqt = N / BT;
   constexpr int VEC = Vec16<T>::kN;
   for (int e = tid; e < BT * D / VEC; e += NT) {
@@ -254,14 +318,22 @@ __global__ void __launch_bounds__(NT) bwd_dkv_kernel(BwdArgs a, int Hq, int g, i
   for (int hh = 0; hh < g; ++hh) {
     const int h = kvh * g + hh;
     for (int qt = kt; qt < nqt; ++qt) {
-      const int t0 = qt * BT, iblk = t0 / s;
+      const int t0 = qt * BT;
       const int64_t rbase = ((int64_t)b * Hq + h) * N + t0;
-      const uint32_t word = a.mask[(((int64_t)b * Hq + h) * n + iblk) * a.words + (jblk >> 5)];
-      const bool sel = (word >> (jblk & 31)) & 1u;
-      if (a.sparse_only && !sel) continue;  // uniform over the CTA
-      const float* src = sel ? a.doc : a.dhf;
-      const float* Dsrc = sel ? a.Dc : a.Df;
       __syncthreads();
+      bool myA = false, myD = false;
+      if (tid < BT) {
+        const int t = t0 + tid;
+        const uint32_t* blocks = a.mask + (((int64_t)b * Hq + h) * n + t / s) * a.words;
+        const unsigned long long causal = causal_mask(t, u0);
+        const unsigned long long cm = tile_keep_mask(blocks, u0, s) & causal;
+        S.cm[tid] = cm;
+        myA = cm != 0ull;
+        myD = (causal & ~cm) != 0ull;
+      }
+      const bool anyA = __syncthreads_or(myA);
+      const bool anyD = __syncthreads_or(myD) && !a.sparse_only;  // dropped pairs: no sparse-stream gradient
+      if (!anyA && !anyD) continue;  // uniform over the CTA
       for (int e = tid; e < BT * D / VEC; e += NT) {
         const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
         float tq[VEC];
@@ -271,66 +343,64 @@ __global__ void __launch_bounds__(NT) bwd_dkv_kernel(BwdArgs a, int Hq, int g, i
       }
       for (int e = tid; e < BT * D; e += NT) {
         const int r = e / D, c = e % D;
-        S.dO[r][c] = src[(rbase + r) * D + c];
+        if (anyA) S.doc[r][c] = a.doc[(rbase + r) * D + c];
+        if (anyD) S.dhf[r][c] = a.dhf[(rbase + r) * D + c];
       }
       if (tid < BT) {
         S.lse[tid] = a.lse_full[rbase + tid];
-        S.dd[tid] = Dsrc[rbase + tid];
+        S.dc[tid] = a.Dc[rbase + tid];
+        S.df[tid] = a.Df[rbase + tid];
       }
       __syncthreads();
-      float xs[4][4], dp[4][4];
+      float xs[4][4], dpc[4][4], dpf[4][4];
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) xs[r][c] = dp[r][c] = 0.f;
-#pragma unroll 4
-      for (int c = 0; c < D; ++c) {
-        float qv[4], ov[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          qv[j] = S.q[tx * 4 + j][c];
-          ov[j] = S.dO[tx * 4 + j][c];
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const float kv = S.k[ty * 4 + r][c];
-          const float vv = S.v[ty * 4 + r][c];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            xs[r][j] = fmaf(kv, qv[j], xs[r][j]);
-            dp[r][j] = fmaf(vv, ov[j], dp[r][j]);
-          }
-        }
-      }
+        for (int c = 0; c < 4; ++c) xs[r][c] = dpc[r][c] = dpf[r][c] = 0.f;
+      if (anyA && anyD) dkv_dots<D, true, true>(S, ty, tx, xs, dpc, dpf);
+      else if (anyA) dkv_dots<D, true, false>(S, ty, tx, xs, dpc, dpf);
+      else dkv_dots<D, false, true>(S, ty, tx, xs, dpc, dpf);
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int key = ty * 4 + r, qr = tx * 4 + j;
-          float p = 0.f, ds = 0.f;
+          float pa = 0.f, pdv = 0.f, ds = 0.f;
           if (u0 + key <= t0 + qr) {
-            p = expf(scale * xs[r][j] - S.lse[qr]);
-            ds = p * (dp[r][j] - S.dd[qr]);
+            const bool in_a = (S.cm[qr] >> key) & 1ull;
+            if (in_a || anyD) {
+              const float p = expf(scale * xs[r][j] - S.lse[qr]);
+              if (in_a) {
+                pa = p;
+                ds = p * (dpc[r][j] - S.dc[qr]);
+              } else {
+                pdv = p;
+                ds = p * (dpf[r][j] - S.df[qr]);
+              }
+            }
           }
-          S.p[key][qr] = p;
+          S.p[key][qr] = pa;
+          S.pd[key][qr] = pdv;
           S.ds[key][qr] = ds;
         }
       __syncthreads();
 #pragma unroll 4
       for (int qq = 0; qq < BT; ++qq) {
-        float pv[4], dsv[4];
+        float pv[4], pdv[4], dsv[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           pv[r] = S.p[pr * 4 + r][qq];
+          pdv[r] = S.pd[pr * 4 + r][qq];
           dsv[r] = S.ds[pr * 4 + r][qq];
         }
 #pragma unroll
         for (int c = 0; c < CW; ++c) {
-          const float ov = S.dO[qq][pc * CW + c];
+          const float oc = anyA ? S.doc[qq][pc * CW + c] : 0.f;
+          const float of = anyD ? S.dhf[qq][pc * CW + c] : 0.f;
           const float qv = S.q[qq][pc * CW + c];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            dv[r][c] = fmaf(pv[r], ov, dv[r][c]);
+            dv[r][c] = fmaf(pv[r], oc, fmaf(pdv[r], of, dv[r][c]));
             dk[r][c] = fmaf(dsv[r], qv, dk[r][c]);
           }
         }

@@ -9,9 +9,11 @@
 // "1. Probleemstelling" and "Bidirectionele Uitlijning"): for each query t,
 // two softmaxes over disjoint key sets, A_t (keys in selected blocks) and D_t
 // (the other causal keys), are kept online side by side, each with its own
-// running max, sum and output accumulator.  A key tile lies in one key block,
-// and a 64-row query tile in one query block, so every tile belongs wholly to
-// A or to D for the whole CTA.  At the end:
+// running max, sum and output accumulator.  Tiles are 64 x 64; with blocks of
+// 64 or more keys a tile lies in one query block and one key block and
+// belongs wholly to A or to D, with smaller blocks (16, 32) every row carries
+// a 64-bit mask of its selected keys in the tile and each weight goes to the
+// accumulator of its own set.  At the end:
 //   h_sparse = o_A / l_A,
 //   h_full   = (e^{m_A-M} o_A + e^{m_D-M} o_D) / (e^{m_A-M} l_A + e^{m_D-M} l_D),
 //   delta    = e^{lse_D - lse_full},  lse_full = logaddexp(lse_A, lse_D).
@@ -23,6 +25,7 @@ namespace {
 constexpr int BM = 64;   // query rows per CTA
 constexpr int BN = 64;   // keys per tile
 constexpr int NT = 256;  // threads
+constexpr int QBMAX = 4; // query blocks in a 64-row tile (block >= 16)
 
 struct SimtShape {
   int Hq, g, N, s, n, k;
@@ -32,11 +35,13 @@ struct SimtShape {
 template <int D>
 struct FwdSmem {
   float q[BM][D];
-  float kt[D][BN];      // K tile, transposed
+  float kt[D][BN];       // K tile, transposed
   float v[BN][D];
-  float p[BM][BN + 1];  // logits, then probabilities
-  float m[2][BM], l[2][BM], corr[BM];
-  uint32_t sel[64];     // selected-block bit set of this query block
+  float p[BM][BN + 1];   // logits, then the weights of set A
+  float pd[BM][BN + 1];  // weights of set D
+  float m[2][BM], l[2][BM], corr[2][BM];
+  unsigned long long cm[BM];  // per row: keys of the tile in selected blocks (causal ones only)
+  uint32_t sel[QBMAX][64];    // selected-block bit sets of the tile's query blocks
 };
 
 // o = corr * o + P V for the 4 x CW patch this thread owns.
@@ -69,17 +74,20 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / sh.g;
   const int t0 = qt * BM;
-  const int iblk = t0 / sh.s;
+  const int ib0 = t0 / sh.s;                       // first query block of the tile
+  const int nqb = sh.s >= BM ? 1 : BM / sh.s;      // query blocks in the tile
   const int tid = threadIdx.x;
 
-  // Selected-block bits of query block iblk.
-  const int words = (sh.n + 31) / 32;
-  for (int w = tid; w < words; w += NT) S.sel[w] = 0u;
+  // Selected-block bits of the tile's query blocks.
+  for (int w = tid; w < QBMAX * 64; w += NT) (&S.sel[0][0])[w] = 0u;
   __syncthreads();
-  const int32_t* irow = a.idx + (((int64_t)b * sh.Hq + h) * sh.n + iblk) * sh.k;
-  for (int e = tid; e < sh.k; e += NT) {
-    const int j = irow[e];
-    if (j >= 0 && j <= iblk) atomicOr(&S.sel[j >> 5], 1u << (j & 31));
+  for (int qb = 0; qb < nqb; ++qb) {
+    const int iblk = ib0 + qb;
+    const int32_t* irow = a.idx + (((int64_t)b * sh.Hq + h) * sh.n + iblk) * sh.k;
+    for (int e = tid; e < sh.k; e += NT) {
+      const int j = irow[e];
+      if (j >= 0 && j <= iblk) atomicOr(&S.sel[qb][j >> 5], 1u << (j & 31));
+    }
   }
   // Q tile -> fp32 smem.
   constexpr int VEC = Vec16<T>::kN;
@@ -108,10 +116,17 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
 
   for (int kt = 0; kt <= qt; ++kt) {
     const int u0 = kt * BN;
-    const int jblk = u0 / sh.s;
     __syncthreads();  // previous tile fully consumed; sel bits visible
-    const bool sel = (S.sel[jblk >> 5] >> (jblk & 31)) & 1u;
-    if (a.sparse_only && !sel) continue;  // the sparse stream reads selected tiles only
+    bool myA = false, myD = false;
+    if (tid < BM) {
+      const unsigned long long causal = causal_mask(t0 + tid, u0);
+      const unsigned long long cm = tile_keep_mask(S.sel[(t0 + tid) / sh.s - ib0], u0, sh.s) & causal;
+      S.cm[tid] = cm;
+      myA = cm != 0ull;
+      myD = (causal & ~cm) != 0ull;
+    }
+    const bool anyA = __syncthreads_or(myA), anyD = __syncthreads_or(myD);
+    if (a.sparse_only && !anyA) continue;  // the sparse stream reads selected keys only
     for (int e = tid; e < BN * D / VEC; e += NT) {
       const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
       float tmp[VEC];
@@ -150,46 +165,67 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
       }
     __syncthreads();
 
-    // Online softmax update of the set this tile belongs to.
+    // Online softmax update of both sets: each logit joins the set its key's
+    // block belongs to for this row (causal mask already applied).
     {
-      const int set = sel ? 0 : 1;
-      float mt = kNegInf;
+      const unsigned long long cm = S.cm[sr] >> (sq * 16);
+      float mA = kNegInf, mD = kNegInf;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) mt = fmaxf(mt, S.p[sr][sq * 16 + c]);
-      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-      const float m_old = S.m[set][sr];
-      const float m_new = fmaxf(m_old, mt);
-      float sum = 0.f;
-      if (m_new != kNegInf) {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float x = S.p[sr][sq * 16 + c];
-          const float p = (x == kNegInf) ? 0.f : expf(x - m_new);
-          S.p[sr][sq * 16 + c] = p;
-          sum += p;
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) S.p[sr][sq * 16 + c] = 0.f;
+      for (int c = 0; c < 16; ++c) {
+        const float x = S.p[sr][sq * 16 + c];
+        if ((cm >> c) & 1ull) mA = fmaxf(mA, x);
+        else mD = fmaxf(mD, x);
       }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+      mD = fmaxf(mD, __shfl_xor_sync(0xffffffffu, mD, 1));
+      mD = fmaxf(mD, __shfl_xor_sync(0xffffffffu, mD, 2));
+      const float oldA = S.m[0][sr], oldD = S.m[1][sr];
+      const float newA = fmaxf(oldA, mA), newD = fmaxf(oldD, mD);
+      float sumA = 0.f, sumD = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float x = S.p[sr][sq * 16 + c];
+        float pA = 0.f, pD = 0.f;
+        if (x != kNegInf) {
+          if ((cm >> c) & 1ull) pA = expf(x - newA);
+          else pD = expf(x - newD);
+        }
+        S.p[sr][sq * 16 + c] = pA;
+        S.pd[sr][sq * 16 + c] = pD;
+        sumA += pA;
+        sumD += pD;
+      }
+      sumA += __shfl_xor_sync(0xffffffffu, sumA, 1);
+      sumA += __shfl_xor_sync(0xffffffffu, sumA, 2);
+      sumD += __shfl_xor_sync(0xffffffffu, sumD, 1);
+      sumD += __shfl_xor_sync(0xffffffffu, sumD, 2);
       if (sq == 0) {
-        const float corr = (m_old == kNegInf) ? 0.f : expf(m_old - m_new);
-        S.corr[sr] = corr;
-        S.l[set][sr] = S.l[set][sr] * corr + sum;
-        S.m[set][sr] = m_new;
+        const float cA = (oldA == kNegInf) ? 0.f : expf(oldA - newA);
+        const float cD = (oldD == kNegInf) ? 0.f : expf(oldD - newD);
+        S.corr[0][sr] = cA;
+        S.corr[1][sr] = cD;
+        S.l[0][sr] = S.l[0][sr] * cA + sumA;
+        S.l[1][sr] = S.l[1][sr] * cD + sumD;
+        S.m[0][sr] = newA;
+        S.m[1][sr] = newD;
       }
     }
     __syncthreads();
 
     if (WITH_V) {
+      // a set with no pair in this tile keeps its max (factor 1) and gains nothing
       float cr[4];
+      if (anyA) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) cr[r] = S.corr[pr * 4 + r];
-      if (sel) pv_update<D, CW>(oA, cr, S.p, S.v, pr, pc);
-      else pv_update<D, CW>(oD, cr, S.p, S.v, pr, pc);
+        for (int r = 0; r < 4; ++r) cr[r] = S.corr[0][pr * 4 + r];
+        pv_update<D, CW>(oA, cr, S.p, S.v, pr, pc);
+      }
+      if (anyD && !a.sparse_only) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) cr[r] = S.corr[1][pr * 4 + r];
+        pv_update<D, CW>(oD, cr, S.pd, S.v, pr, pc);
+      }
     }
   }
   __syncthreads();

@@ -28,9 +28,9 @@ ssa_status_t check_dims(const ssa_dims_t* in, Dims* out, bool* empty) {
   if (D.dtype != SSA_F32 && D.dtype != SSA_BF16) return SSA_ERR_INVALID_ARG;
   if (!(D.scale > 0.f) || D.scale == __builtin_huge_valf()) return SSA_ERR_INVALID_ARG;
   if (D.Hq % D.Hkv != 0) return SSA_ERR_INVALID_ARG;
-  if (D.s != 64 && D.s != 128) return SSA_ERR_UNSUPPORTED;
+  if (D.s != 16 && D.s != 32 && D.s != 64 && D.s != 128) return SSA_ERR_UNSUPPORTED;
   if (D.d != 64 && D.d != 128) return SSA_ERR_UNSUPPORTED;
-  if (D.N % D.s != 0) return SSA_ERR_UNSUPPORTED;
+  if (D.N % D.s != 0 || D.N % 64 != 0) return SSA_ERR_UNSUPPORTED;
   D.n = D.N / D.s;
   if (D.n > 2048) return SSA_ERR_UNSUPPORTED;
   D.k = D.topk < D.n ? D.topk : D.n;

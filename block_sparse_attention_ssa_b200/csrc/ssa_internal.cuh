@@ -68,6 +68,30 @@ template <> struct Vec16<__nv_bfloat16> {
 
 constexpr float kNegInf = -__builtin_huge_valf();
 
+// 64-key tiles at key u0 (CUDA-core kernels): bit c is set when key u0 + c
+// lies in a block whose bit is set in `blocks` (the selected-block set of a
+// row's query block); s is the block size.  Blocks of 64 or more keys cover
+// the whole tile; smaller blocks give one run of s bits per block.
+__device__ __forceinline__ unsigned long long tile_keep_mask(const uint32_t* blocks, int u0, int s) {
+  if (s >= 64) {
+    const int j = u0 / s;
+    return ((blocks[j >> 5] >> (j & 31)) & 1u) ? ~0ull : 0ull;
+  }
+  unsigned long long m = 0ull;
+  const unsigned long long run = (1ull << s) - 1ull;
+  for (int c0 = 0; c0 < 64; c0 += s) {
+    const int j = (u0 + c0) / s;
+    if ((blocks[j >> 5] >> (j & 31)) & 1u) m |= run << c0;
+  }
+  return m;
+}
+
+// Bit c is set when key u0 + c <= t (a causal pair of query t).
+__device__ __forceinline__ unsigned long long causal_mask(int t, int u0) {
+  const int lim = t - u0;
+  return lim >= 63 ? ~0ull : (lim < 0 ? 0ull : ((2ull << lim) - 1ull));
+}
+
 // Host-side count of kernels enqueued by this library (ssa_launch_count).
 void count_launches(int n);
 

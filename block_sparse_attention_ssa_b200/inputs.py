@@ -63,7 +63,8 @@ class Workload:
         return self.B * self.Hq * self.N * (self.N + 1) // 2
 
 
-# The five workloads of the benchmark suite.  Seeds are 1000 + the workload's
+# The benchmark workloads (the five synthetic suites and the pages' own model
+# shape).  Seeds are 1000 + the workload's
 # ordinal; the budget sweep reuses one tensor set for every budget.
 WORKLOADS = {
     "tiny_f32": Workload("tiny_f32", 1, 1, 1, 1024, 64, 64, 4, "f32", 1001, backward=False),
@@ -71,6 +72,10 @@ WORKLOADS = {
     "gqa_16k": Workload("gqa_16k", 2, 32, 8, 16384, 128, 64, 16, "bf16", 1003),
     "long_64k": Workload("long_64k", 1, 32, 8, 65536, 128, 128, 16, "bf16", 1004, plant="sparse5"),
     "sweep_32k": Workload("sweep_32k", 1, 32, 8, 32768, 128, 64, 16, "bf16", 1005),
+    # The attention layer of the pages' 1B model (32 query heads, 2 kv heads,
+    # hidden 2048 -> d = 64) with their 16 x 16 receptive field at the 8K
+    # training context.
+    "paper_b16_8k": Workload("paper_b16_8k", 1, 32, 2, 8192, 64, 16, 16, "bf16", 1006),
 }
 SWEEP_TOPK = (4, 8, 16, 32, 64)
 

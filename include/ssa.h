@@ -35,10 +35,14 @@
  *   H = Hq; K, V, dK, dV use H = Hkv.  Base pointers must be 16-byte aligned
  *   and every stride times the element size a multiple of 16 bytes.
  *   Plain arrays (scores, idx, lse_*, delta) are dense row-major as stated.
- * Shapes.  B, Hq, N >= 0 and Hkv >= 1 with Hq % Hkv == 0; block in {64, 128};
- *   N % block == 0; d in {64, 128}; topk >= 1 (a budget above n is clamped:
- *   k_eff = min(topk, n)); n <= 2048.  When B*Hq*N == 0 the call is a no-op
- *   and returns SSA_OK.
+ * Shapes.  B, Hq, N >= 0 and Hkv >= 1 with Hq % Hkv == 0; block in
+ *   {16, 32, 64, 128}; N a multiple of block and of 64; d in {64, 128};
+ *   topk >= 1 (a budget above n is clamped: k_eff = min(topk, n));
+ *   n <= 2048.  When B*Hq*N == 0 the call is a no-op and returns SSA_OK.
+ *   Blocks of 64 and 128 with bf16 and d = 128 run on the tensor-core
+ *   kernels; every other supported shape (fp32, d = 64, and the small
+ *   blocks 16 and 32 of the paper's models, [digest] "Model Architecture
+ *   Configuration") runs on the CUDA-core kernels.
  * Errors.  Arguments are checked on the host before anything is enqueued;
  *   a failed check returns SSA_ERR_INVALID_ARG (bad pointer, stride,
  *   alignment or value), SSA_ERR_UNSUPPORTED (a shape outside the list above,

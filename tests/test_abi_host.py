@@ -40,6 +40,8 @@ def test_workspace_bytes():
     assert api.ssa_workspace_bytes(api.make_dims(0, 32, 8, 16384, 128, 64, 16)) == 0
     assert api.ssa_workspace_bytes(api.make_dims(1, 4, 2, 1000, 128, 64, 16)) == 0  # N % block
     assert api.ssa_workspace_bytes(api.make_dims(1, 4, 3, 1024, 128, 64, 16)) == 0  # Hq % Hkv
+    assert api.ssa_workspace_bytes(api.make_dims(1, 4, 2, 1040, 64, 16, 16)) == 0   # N % 64 (block 16)
+    assert api.ssa_workspace_bytes(api.make_dims(1, 4, 2, 1024, 64, 16, 16)) > 0    # block 16
 
 
 def _tensor(ptr=16, sb=4096 * 128, sh=4096 * 128, sn=128):
@@ -47,7 +49,7 @@ def _tensor(ptr=16, sb=4096 * 128, sh=4096 * 128, sn=128):
 
 
 @pytest.mark.parametrize("field,value,code", [
-    ("block", 32, api.SSA_ERR_UNSUPPORTED),
+    ("block", 8, api.SSA_ERR_UNSUPPORTED),
     ("block", 96, api.SSA_ERR_UNSUPPORTED),
     ("d", 96, api.SSA_ERR_UNSUPPORTED),
     ("N", 1000, api.SSA_ERR_UNSUPPORTED),

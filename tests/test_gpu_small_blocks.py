@@ -1,0 +1,176 @@
+"""GPU parity at the pages' small block sizes (16 and 32 tokens; [digest]
+"Model Architecture Configuration": block size 16, 16 blocks), where a 64 x 64
+CUDA-core tile spans several query and key blocks and every element goes to
+the selected or the dropped set on its own.  Each entry point of the path is
+compared with the fp64 oracle: block scores and selection, the dual forward,
+the dropped mass (with and without the full log-sum-exp), the sparse stream
+alone forward and backward, the dual backward on both primaries, and the
+decode step.  Includes the pages' model shape (g = 16 query heads per kv
+head, d = 64).  Tolerances as elsewhere."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_ssa_b200 import api
+from block_sparse_attention_ssa_b200.inputs import make_upstream
+from oracle import ssa_oracle as O
+from tests.gpu_util import (TOL, case_inputs, compare_selection, custom_idx, ensure_library, f64, oracle_view,
+                            rel_l2, upload)
+
+pytestmark = pytest.mark.gpu
+
+# name: B, Hq, Hkv, N, d, s, k, dtype
+CASES = {
+    "f32_s16_d64": (1, 4, 2, 512, 64, 16, 16, "f32"),
+    "bf16_s16_g16_d64": (1, 16, 1, 768, 64, 16, 16, "bf16"),
+    "bf16_s32_d128": (2, 4, 2, 768, 128, 32, 6, "bf16"),
+    "f32_s16_d128_k4": (1, 2, 1, 640, 128, 16, 4, "f32"),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    return ensure_library()
+
+
+def _forward(name, seed=515):
+    B, Hq, Hkv, N, d, s, k, dt = CASES[name]
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, seed, dt)
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, dt)
+    ws = api.alloc_workspace(dims)
+    out = api.alloc_forward(dims)
+    api.ssa_block_scores(dims, dev["Q"], dev["K"], out["scores"], ws)
+    api.ssa_select_topk(dims, out["scores"], out["idx"])
+    scale = 1 / math.sqrt(d)
+    torch.cuda.synchronize()
+    ora_scores = O.block_scores(host["Q"], host["K"], s, scale)
+    ora_idx = O.select_blocks(ora_scores, k)
+    if compare_selection(out["idx"].cpu().numpy(), ora_idx, ora_scores):
+        out["idx"].copy_(torch.from_numpy(ora_idx))
+    api.ssa_fwd_dual(dims, dev["Q"], dev["K"], dev["V"], out["idx"], out["h_full"], out["h_sparse"],
+                     out["lse_full"], out["lse_sel"], out["delta"])
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    ora = O.forward_dual(host["Q"], host["K"], host["V"], ora_idx, s, scale)
+    return dict(dims=dims, dev=dev, host=host, out=out, ws=ws, ora=ora, ora_idx=ora_idx, scale=scale,
+                cfg=CASES[name])
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_forward_dual_small_blocks(name):
+    r = _forward(name)
+    tol = TOL[r["cfg"][7]]
+    for key in ("h_full", "h_sparse", "delta"):
+        err = np.abs(f64(r["out"][key]) - r["ora"][key]).max()
+        assert err <= tol["out"], (key, err)
+    for key in ("lse_full", "lse_sel"):
+        assert np.abs(f64(r["out"][key]) - r["ora"][key]).max() <= tol["lse"], key
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_dropped_mass_small_blocks(name):
+    r = _forward(name)
+    tol = TOL[r["cfg"][7]]["out"]
+    for lse in (r["out"]["lse_full"], None):
+        delta = torch.full_like(r["out"]["delta"], float("nan"))
+        api.ssa_dropped_mass(r["dims"], r["dev"]["Q"], r["dev"]["K"], r["out"]["idx"], lse, delta, r["ws"])
+        torch.cuda.synchronize()
+        assert np.abs(f64(delta) - r["ora"]["delta"]).max() <= tol
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_sparse_alone_small_blocks(name):
+    r = _forward(name)
+    B, Hq, Hkv, N, d, s, k, dt = r["cfg"]
+    dims, dev, host = r["dims"], r["dev"], r["host"]
+    hs = torch.full_like(r["out"]["h_sparse"], float("nan"))
+    lse = torch.full_like(r["out"]["lse_sel"], float("nan"))
+    api.ssa_fwd_sparse(dims, dev["Q"], dev["K"], dev["V"], r["out"]["idx"], hs, lse)
+    torch.cuda.synchronize()
+    ora = O.forward_sparse(host["Q"], host["K"], host["V"], r["ora_idx"], s, r["scale"])
+    assert np.abs(f64(hs) - ora["h_sparse"]).max() <= TOL[dt]["out"]
+    assert np.abs(f64(lse) - ora["lse_sel"]).max() <= TOL[dt]["lse"]
+    g = make_upstream((B, Hq, N, d), 47)
+    grads = api.alloc_backward(dims)
+    api.ssa_bwd_sparse(dims, dev["Q"], dev["K"], dev["V"], r["out"]["idx"], hs, lse, upload(g, dt), grads["dQ"],
+                       grads["dK"], grads["dV"], r["ws"])
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    dQ, dK, dV = O.backward_sparse(host["Q"], host["K"], host["V"], r["ora_idx"], s, r["scale"],
+                                   oracle_view(g, dt).astype(np.float64))
+    for key, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        assert rel_l2(f64(got), ref) < TOL[dt]["grad"], key
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("primary", ["sparse", "full"])
+def test_backward_dual_small_blocks(name, primary):
+    r = _forward(name)
+    B, Hq, Hkv, N, d, s, k, dt = r["cfg"]
+    g = make_upstream((B, Hq, N, d), 53)
+    gd = upload(g, dt)
+    gf, gs = (gd, None) if primary == "full" else (None, gd)
+    grads = api.alloc_backward(r["dims"])
+    api.backward(r["dims"], r["dev"]["Q"], r["dev"]["K"], r["dev"]["V"], r["out"], gf, gs, 10.0, grads, r["ws"])
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    go = oracle_view(g, dt).astype(np.float64)
+    ogf, ogs = (go, None) if primary == "full" else (None, go)
+    dQ, dK, dV, l_align, _ = O.ssa_backward(r["host"]["Q"], r["host"]["K"], r["host"]["V"], r["ora_idx"], s,
+                                            r["scale"], ogf, ogs, 10.0, fwd=r["ora"])
+    for key, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        assert rel_l2(f64(got), ref) < TOL[dt]["grad"], key
+    assert float(grads["align_loss"].item()) == pytest.approx(l_align, rel=5e-2 if dt == "bf16" else 1e-4)
+
+
+def test_given_selection_mixed_tiles():
+    """Random selections at block 16 (rows without their diagonal block,
+    duplicates, padding): most 64 x 64 tiles mix selected and dropped pairs
+    inside a row and between rows."""
+    B, Hq, Hkv, N, d, s, k = 1, 4, 2, 512, 64, 16, 6
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 616, "f32")
+    n = N // s
+    idx = custom_idx(B, Hq, n, k, seed=77, drop_diag_frac=0.3, pad_frac=0.2)
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "f32")
+    out = api.alloc_forward(dims)
+    ws = api.alloc_workspace(dims)
+    out["idx"] = torch.from_numpy(idx).cuda()
+    api.ssa_fwd_dual(dims, dev["Q"], dev["K"], dev["V"], out["idx"], out["h_full"], out["h_sparse"],
+                     out["lse_full"], out["lse_sel"], out["delta"])
+    gf, gs = make_upstream((B, Hq, N, d), 61), make_upstream((B, Hq, N, d), 62)
+    grads = api.alloc_backward(dims)
+    api.backward(dims, dev["Q"], dev["K"], dev["V"], out, upload(gf, "f32"), upload(gs, "f32"), 10.0, grads, ws)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    scale = 1 / math.sqrt(d)
+    dQ, dK, dV, _, ora = O.ssa_backward(host["Q"], host["K"], host["V"], idx, s, scale, gf.astype(np.float64),
+                                        gs.astype(np.float64), 10.0)
+    for key in ("h_full", "h_sparse", "delta"):
+        assert np.abs(f64(out[key]) - ora[key]).max() <= TOL["f32"]["out"], key
+    for key, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        assert rel_l2(f64(got), ref) < TOL["f32"]["grad"], key
+
+
+def test_decode_block16():
+    """Decode at block 16 across several block boundaries, against the oracle."""
+    B, Hq, Hkv, N, d, s, k = 1, 8, 2, 512, 64, 16, 16
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 717, "f32")
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "f32")
+    st = api.alloc_decode(dims)
+    ws = api.alloc_workspace(dims)
+    t0 = 16 * 17 + 5
+    api.ssa_decode_prefill(dims, dev["Q"], dev["K"], t0, st["qsum"], st["kbar"])
+    scale = 1 / math.sqrt(d)
+    for t in range(t0, t0 + 60):
+        i = t // s
+        api.ssa_decode_step(dims, dev["Q"][:, :, t:t + 1], dev["K"], dev["V"], t, st["qsum"], st["kbar"], st["h"],
+                            st["lse"], st["idx"], ws)
+        torch.cuda.synchronize()
+        gidx = st["idx"].cpu().numpy()
+        oidx = O.decode_select(host["Q"][:, :, i * s:t + 1], host["K"], t, s, k, scale, n_cache=N // s)
+        assert np.array_equal(gidx, oidx), t
+        h_ref, lse_ref = O.decode_attend(host["Q"][:, :, t], host["K"], host["V"], t, s, oidx, scale)
+        assert np.abs(f64(st["h"])[:, :, 0] - h_ref).max() <= TOL["f32"]["out"], t
+        assert np.abs(f64(st["lse"]) - lse_ref).max() <= TOL["f32"]["lse"], t
