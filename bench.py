@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="gqa_16k")
     ap.add_argument("--topk", type=int, default=None, help="override the workload's budget")
     ap.add_argument("--alpha", type=float, default=10.0)
+    ap.add_argument("--per-token", action="store_true",
+                    help="per-token selection (each query token ranks the blocks by its own query)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
@@ -169,7 +171,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU oracle sample
-def oracle_sample(w, host, budget_s: float, alpha: float):
+def oracle_sample(w, host, budget_s: float, alpha: float, per_token: bool = False):
     """Time the fp64 oracle (forward, backward, dropped mass) on sampled
     (batch, head, query block) units of the workload until `budget_s` of CPU
     time is used.  Returns (attended FLOPs done, seconds, description)."""
@@ -193,17 +195,21 @@ def oracle_sample(w, host, budget_s: float, alpha: float):
         Q = host["Q"][b:b + 1, h:h + 1, :N1].astype(np.float64)
         K = host["K"][b:b + 1, kv:kv + 1, :N1].astype(np.float64)
         V = host["V"][b:b + 1, kv:kv + 1, :N1].astype(np.float64)
-        idx = O.select_blocks(O.block_scores(Q, K, s, scale), w.topk)
+        if per_token:
+            idx = O.select_tokens(O.token_scores(Q, K, s, scale), w.topk, s)
+        else:
+            idx = O.select_blocks(O.block_scores(Q, K, s, scale), w.topk)
         g = np.ones((1, 1, N1, d))
-        O.ssa_backward(Q, K, V, idx, s, scale, None, g, alpha, qblocks=[i], M=M)
-        O.dropped_mass(Q[:, :, : N1], K, idx, s, scale)
+        O.ssa_backward(Q, K, V, idx, s, scale, None, g, alpha, qblocks=[i], M=M, per_token=per_token)
+        O.dropped_mass(Q[:, :, : N1], K, idx, s, scale, per_token=per_token)
         secs += time.perf_counter() - t0
         pairs = sum(t + 1 for t in range(i * s, (i + 1) * s))
         done += (4 + 10 + 2) * d * pairs
         units.append((b, h, i))
         if time.perf_counter() - t_start > 4 * budget_s:
             break
-    desc = (f"{len(units)} random (batch, head, query block) units of {w.name}: block scores + top-k "
+    sel = "per-token scores + top-k" if per_token else "block scores + top-k"
+    desc = (f"{len(units)} random (batch, head, query block) units of {w.name}: {sel} "
             f"over the unit's prefix, dual forward, backward (alpha={alpha}, sum(h_sparse)) and "
             f"dropped mass, fp64 numpy")
     return done, secs, desc
@@ -230,10 +236,10 @@ def run_reference(args, rank: int):
     host = make_workload_inputs(w)
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(w, host, per_step / 4, args.alpha)
+        oracle_sample(w, host, per_step / 4, args.alpha, args.per_token)
     tot_f, tot_s, desc = 0, 0.0, ""
     for _ in range(args.steps):
-        f, s_, desc = oracle_sample(w, host, per_step, args.alpha)
+        f, s_, desc = oracle_sample(w, host, per_step, args.alpha, args.per_token)
         tot_f += f
         tot_s += s_
     value = tot_f / tot_s / 1e12
@@ -255,6 +261,7 @@ def run_reference(args, rank: int):
 def config_dict(w, args):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "block": w.block,
             "topk": w.topk, "dtype": w.dtype, "alpha": args.alpha, "primary": "sparse",
+            "selection": "per token" if getattr(args, "per_token", False) else "per query block",
             "step": "block_scores+select_topk+fwd_dual+bwd_dual+dropped_mass",
             "l2": "no flush: inputs larger than L2 (Q alone exceeds 126 MB)" if w.N * w.Hq * w.B * w.d * 2 > 126e6
             else "inputs smaller than L2", "parallelism": f"dp{args.gpus} (independent replicas of the workload)"}
@@ -287,7 +294,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
 
     pinned = {k: to_pinned(k) for k in ("Q", "K", "V")}
     D = {k: v.to(dev, non_blocking=False) for k, v in pinned.items()}
-    dims = api.make_dims(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, w.topk, w.dtype)
+    dims = api.make_dims(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, w.topk, w.dtype, per_token=args.per_token)
     ws = api.alloc_workspace(dims, dev)
     out = api.alloc_forward(dims, dev)
     grads = api.alloc_backward(dims, dev)
@@ -298,10 +305,14 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     def step(evs=None, D=D):
         if evs is not None:
             evs[0].record(stream)
-        api.ssa_block_scores(dims, D["Q"], D["K"], out["scores"], ws, stream)
+        if args.per_token:  # one launch pair selects per token; the top-k row stays empty
+            api.ssa_select_tokens(dims, D["Q"], D["K"], out["idx"], ws, stream)
+        else:
+            api.ssa_block_scores(dims, D["Q"], D["K"], out["scores"], ws, stream)
         if evs is not None:
             evs[1].record(stream)
-        api.ssa_select_topk(dims, out["scores"], out["idx"], stream)
+        if not args.per_token:
+            api.ssa_select_topk(dims, out["scores"], out["idx"], stream)
         if evs is not None:
             evs[2].record(stream)
         api.ssa_fwd_dual(dims, D["Q"], D["K"], D["V"], out["idx"], out["h_full"], out["h_sparse"],
@@ -427,7 +438,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     row_flops = {"fwd_dual": F["fwd"], "bwd_dual": F["bwd"], "dropped_mass": F["dropped"]}
     # bf16 with d = 128 and blocks of 64 / 128 runs on the tensor-core kernels;
     # every other shape on the CUDA-core kernels (fp32 FMA bound)
-    tc_path = w.dtype == "bf16" and w.d == 128 and w.block in (64, 128)
+    tc_path = w.dtype == "bf16" and w.d == 128 and w.block in (64, 128) and not args.per_token
     if tc_path:
         scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_tc_kernel)",
                   "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_tc + finish + bwd_dkv_tc + bwd_dq_tc kernels",
@@ -600,7 +611,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, secs, desc = oracle_sample(w, host, args.cpu_seconds, args.alpha)
+        f, secs, desc = oracle_sample(w, host, args.cpu_seconds, args.alpha, args.per_token)
         cpu = {"value": f / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                "sample": desc, "seconds": secs}
 

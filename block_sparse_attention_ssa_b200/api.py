@@ -38,7 +38,8 @@ class SsaError(RuntimeError):
 class ssa_dims_t(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32),
-                ("topk", ctypes.c_int32), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
+                ("topk", ctypes.c_int32), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("per_token", ctypes.c_int32)]
 
     @property
     def n_blocks(self) -> int:
@@ -51,6 +52,11 @@ class ssa_dims_t(ctypes.Structure):
     @property
     def torch_dtype(self) -> torch.dtype:
         return _TORCH_DTYPES[self.dtype]
+
+    @property
+    def sel_rows(self) -> int:
+        """Rows of a selection per head: N (per-token selection) or n."""
+        return self.N if self.per_token else self.N // self.block
 
 
 class ssa_tensor_t(ctypes.Structure):
@@ -66,6 +72,8 @@ _SIGS = {
     "ssa_block_scores": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "ssa_select_topk": (ctypes.c_int, [_P(ssa_dims_t), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "ssa_select_tokens": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "ssa_fwd_dual": (ctypes.c_int, [_P(ssa_dims_t), _P(ssa_tensor_t), _P(ssa_tensor_t), _P(ssa_tensor_t),
                                      ctypes.c_void_p, _P(ssa_tensor_t), _P(ssa_tensor_t), ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
@@ -137,10 +145,10 @@ def _check(fn: str, code: int) -> None:
 
 
 def make_dims(B: int, Hq: int, Hkv: int, N: int, d: int, block: int, topk: int,
-              dtype: str = "bf16", scale: float | None = None) -> ssa_dims_t:
+              dtype: str = "bf16", scale: float | None = None, per_token: bool = False) -> ssa_dims_t:
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    return ssa_dims_t(B, Hq, Hkv, N, d, block, topk, float(scale), _DTYPES[dtype])
+    return ssa_dims_t(B, Hq, Hkv, N, d, block, topk, float(scale), _DTYPES[dtype], int(per_token))
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -181,6 +189,11 @@ def ssa_block_scores_noalloc(dims, Q, K, scores, stream=None) -> None:
 def ssa_select_topk(dims, scores, idx, stream=None) -> None:
     _check("ssa_select_topk", load_library().ssa_select_topk(
         ctypes.byref(dims), _p(scores), _p(idx), _stream(stream)))
+
+
+def ssa_select_tokens(dims, Q, K, idx, ws, stream=None) -> None:
+    _check("ssa_select_tokens", load_library().ssa_select_tokens(
+        ctypes.byref(dims), _t(Q), _t(K), _p(idx), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def ssa_fwd_dual(dims, Q, K, V, idx, h_full, h_sparse, lse_full, lse_sel, delta, stream=None) -> None:
@@ -259,7 +272,7 @@ def alloc_forward(dims: ssa_dims_t, device="cuda") -> dict[str, torch.Tensor]:
     dt = dims.torch_dtype
     return {
         "scores": torch.empty((B, Hq, n, n), dtype=torch.float32, device=device),
-        "idx": torch.empty((B, Hq, n, k), dtype=torch.int32, device=device),
+        "idx": torch.empty((B, Hq, dims.sel_rows, k), dtype=torch.int32, device=device),
         "h_full": torch.empty((B, Hq, N, d), dtype=dt, device=device),
         "h_sparse": torch.empty((B, Hq, N, d), dtype=dt, device=device),
         "lse_full": torch.empty((B, Hq, N), dtype=torch.float32, device=device),
@@ -291,9 +304,13 @@ def alloc_decode(dims: ssa_dims_t, device="cuda") -> dict[str, torch.Tensor]:
 
 
 def forward(dims, Q, K, V, out, ws, stream=None) -> dict[str, torch.Tensor]:
-    """The three forward steps in order: block scores, top-k, fused dual forward."""
-    ssa_block_scores(dims, Q, K, out["scores"], ws, stream)
-    ssa_select_topk(dims, out["scores"], out["idx"], stream)
+    """The forward steps in order: selection (block scores + top-k, or the
+    per-token selection), then the fused dual forward."""
+    if dims.per_token:
+        ssa_select_tokens(dims, Q, K, out["idx"], ws, stream)
+    else:
+        ssa_block_scores(dims, Q, K, out["scores"], ws, stream)
+        ssa_select_topk(dims, out["scores"], out["idx"], stream)
     ssa_fwd_dual(dims, Q, K, V, out["idx"], out["h_full"], out["h_sparse"], out["lse_full"],
                  out["lse_sel"], out["delta"], stream)
     return out

@@ -83,7 +83,6 @@ __global__ void __launch_bounds__(NT) bwd_pre_kernel(BwdArgs a, int Hq, int N, f
 // 64 rows; with smaller blocks each row's 64-bit mask of selected keys picks,
 // element by element, the combined (dO_c, D_c) or the full-stream
 // (dh_f, D_f) gradient.
-constexpr int QBMAX = 4;  // query blocks in a 64-row tile (block >= 16)
 
 template <int D>
 struct DqSmem {
@@ -95,7 +94,6 @@ struct DqSmem {
   float p[BT][BT + 1];
   float lse[BT], dc[BT], df[BT];
   unsigned long long cm[BT];  // per query row: keys of the tile in selected blocks
-  uint32_t sel[QBMAX][64];
 };
 
 // xs = Q K^T, dpc = dO_c V^T, dpf = dh_f V^T for a 4 x 4 patch (only the
@@ -128,20 +126,15 @@ __device__ __forceinline__ void dq_dots(const DqSmem<D>& S, int ty, int tx, floa
 
 template <typename T, int D>
 __global__ void __launch_bounds__(NT) bwd_dq_kernel(BwdArgs a, int Hq, int g, int N, int s, int n,
-                                                   float scale) {
+                                                   float scale, int per_token) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   DqSmem<D>& S = *reinterpret_cast<DqSmem<D>*>(smem_raw);
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z, kvh = h / g;
-  const int t0 = qt * BT, ib0 = t0 / s, tid = threadIdx.x;
-  const int nqb = s >= BT ? 1 : BT / s;
+  const int t0 = qt * BT, tid = threadIdx.x;
   const int64_t rbase = ((int64_t)b * Hq + h) * N + t0;
+  const int rph = per_token ? N : n;  // selection rows per head
   constexpr int VEC = Vec16<T>::kN;
 
-  const int words = (n + 31) / 32;
-  for (int w = tid; w < QBMAX * 64; w += NT) {
-    const int qb = w / 64, ww = w % 64;
-    S.sel[qb][ww] = (qb < nqb && ww < words) ? a.mask[(((int64_t)b * Hq + h) * n + ib0 + qb) * a.words + ww] : 0u;
-  }
   for (int e = tid; e < BT * D / VEC; e += NT) {
     const int r = e / (D / VEC), c = (e % (D / VEC)) * VEC;
     Vec16<T>::load(row_ptr<T>(a.q, b, h, t0 + r) + c, &S.q[r][c]);
@@ -171,8 +164,10 @@ __global__ void __launch_bounds__(NT) bwd_dq_kernel(BwdArgs a, int Hq, int g, in
     __syncthreads();
     bool myA = false, myD = false;
     if (tid < BT) {
-      const unsigned long long causal = causal_mask(t0 + tid, u0);
-      const unsigned long long cm = tile_keep_mask(S.sel[(t0 + tid) / s - ib0], u0, s) & causal;
+      const int t = t0 + tid;
+      const uint32_t* blocks = a.mask + (((int64_t)b * Hq + h) * rph + (per_token ? t : t / s)) * a.words;
+      const unsigned long long causal = causal_mask(t, u0);
+      const unsigned long long cm = tile_keep_mask(blocks, u0, s) & causal;
       S.cm[tid] = cm;
       myA = cm != 0ull;
       myD = (causal & ~cm) != 0ull;
@@ -288,7 +283,7 @@ __device__ __forceinline__ void dkv_dots(const DkvSmem<D>& S, int ty, int tx, fl
 
 template <typename T, int D>
 __global__ void __launch_bounds__(NT) bwd_dkv_kernel(BwdArgs a, int Hq, int g, int N, int s, int n,
-                                                    float scale) {
+                                                    float scale, int per_token) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   DkvSmem<D>& S = *reinterpret_cast<DkvSmem<D>*>(smem_raw);
   const int kt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -324,7 +319,8 @@ __global__ void __launch_bounds__(NT) bwd_dkv_kernel(BwdArgs a, int Hq, int g, i
       bool myA = false, myD = false;
       if (tid < BT) {
         const int t = t0 + tid;
-        const uint32_t* blocks = a.mask + (((int64_t)b * Hq + h) * n + t / s) * a.words;
+        const uint32_t* blocks =
+            a.mask + (((int64_t)b * Hq + h) * (per_token ? N : n) + (per_token ? t : t / s)) * a.words;
         const unsigned long long causal = causal_mask(t, u0);
         const unsigned long long cm = tile_keep_mask(blocks, u0, s) & causal;
         S.cm[tid] = cm;
@@ -473,12 +469,12 @@ cudaError_t bwd_t(const Dims& Dm, const BwdArgs& a, cudaStream_t st) {
   e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DkvSmem<D>));
   if (e != cudaSuccess) return e;
   kq<<<dim3(Dm.N / BT, Dm.Hq, Dm.B), NT, sizeof(DqSmem<D>), st>>>(a, Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n,
-                                                                 Dm.scale);
+                                                                 Dm.scale, Dm.per_token);
   count_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   kkv<<<dim3(Dm.N / BT, Dm.Hkv, Dm.B), NT, sizeof(DkvSmem<D>), st>>>(a, Dm.Hq, Dm.g, Dm.N, Dm.s,
-                                                                    Dm.n, Dm.scale);
+                                                                    Dm.n, Dm.scale, Dm.per_token);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -930,7 +930,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 bool bwd_tc_supported(const Dims& D) {
   const int NT = (D.N + TILE - 1) / TILE;
-  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048 &&
+  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048 && !D.per_token &&
          (int64_t)D.g * NT <= dkv::MAX_SPARSE && NT <= dq::MAX_KT && D.g <= 255;
 }
 

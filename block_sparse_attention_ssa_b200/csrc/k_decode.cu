@@ -8,7 +8,7 @@
 // Token t lies in block i = t / s.  The selection rule is the forward's, with
 // the query side read as the mean of the queries of block i seen so far
 // (positions i*s .. t; at the last token of a block this is the forward's
-// block mean exactly):
+// block mean exactly), or, with per-token selection, q_t itself:
 //   qbar   = (sum of q_u, u = i*s .. t) / (t - i*s + 1),
 //   score_j = scale * qbar . kbar_j for j < i (kbar_j = mean of key block j),
 //   Sel     = {i} + the k-1 largest scores (ties to the smaller j), or
@@ -43,6 +43,7 @@ constexpr int BPC = 2;   // selected blocks per attention CTA
 struct DecodeShape {
   int Hq, g, N, s, n, k, t, splits;
   float scale;
+  int per_token;  // the query side of the score is q_t itself (per-token selection)
 };
 
 // Per-call scratch in the caller's workspace.
@@ -113,9 +114,10 @@ __global__ void __launch_bounds__(NT) decode_select_kernel(TensorRef q, TensorRe
 
   if (tid < D) {
     float* qs = qsum + ((int64_t)b * sh.Hq + h) * D + tid;
-    const float acc = (t % s == 0 ? 0.f : *qs) + to_f32(row_ptr<T>(q, b, h, 0)[tid]);
+    const float x = to_f32(row_ptr<T>(q, b, h, 0)[tid]);
+    const float acc = (t % s == 0 ? 0.f : *qs) + x;
     *qs = acc;
-    sqbar[tid] = acc / (float)(t - i * s + 1);
+    sqbar[tid] = sh.per_token ? x : acc / (float)(t - i * s + 1);
   }
   if (tid < 64) sel[tid] = 0u;
   if (hh == 0 && tid == 0) ws.counter[bk] = 0u;
@@ -483,7 +485,7 @@ template <typename T, int D>
 cudaError_t decode_t(const Dims& Dm, const DecodeArgs& a, cudaStream_t st) {
   const int splits = decode_splits(Dm);
   const DecodeWs ws = decode_ws(a.ws, Dm);
-  DecodeShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, a.t, splits, Dm.scale};
+  DecodeShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, a.t, splits, Dm.scale, Dm.per_token};
   const size_t sm1 = SelectLayout(Dm.n, D).bytes, sm2 = AttendLayout(Dm.g, D).bytes;
   auto k1 = decode_select_kernel<T, D>;
   auto k2 = decode_attend_kernel<T, D>;

@@ -25,11 +25,11 @@ namespace {
 constexpr int BM = 64;   // query rows per CTA
 constexpr int BN = 64;   // keys per tile
 constexpr int NT = 256;  // threads
-constexpr int QBMAX = 4; // query blocks in a 64-row tile (block >= 16)
 
 struct SimtShape {
   int Hq, g, N, s, n, k;
   float scale;
+  int per_token;  // selection rows are tokens (1) or query blocks (0)
 };
 
 template <int D>
@@ -41,7 +41,7 @@ struct FwdSmem {
   float pd[BM][BN + 1];  // weights of set D
   float m[2][BM], l[2][BM], corr[2][BM];
   unsigned long long cm[BM];  // per row: keys of the tile in selected blocks (causal ones only)
-  uint32_t sel[QBMAX][64];    // selected-block bit sets of the tile's query blocks
+  uint32_t sel[BM][64];       // selected-block bit sets: per query block of the tile, or per row
 };
 
 // o = corr * o + P V for the 4 x CW patch this thread owns.
@@ -78,16 +78,17 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
   const int nqb = sh.s >= BM ? 1 : BM / sh.s;      // query blocks in the tile
   const int tid = threadIdx.x;
 
-  // Selected-block bits of the tile's query blocks.
-  for (int w = tid; w < QBMAX * 64; w += NT) (&S.sel[0][0])[w] = 0u;
+  // Selected-block bits of the tile's selection rows: its query blocks, or
+  // (per-token selection) its 64 tokens.
+  for (int w = tid; w < BM * 64; w += NT) (&S.sel[0][0])[w] = 0u;
   __syncthreads();
-  for (int qb = 0; qb < nqb; ++qb) {
-    const int iblk = ib0 + qb;
-    const int32_t* irow = a.idx + (((int64_t)b * sh.Hq + h) * sh.n + iblk) * sh.k;
-    for (int e = tid; e < sh.k; e += NT) {
-      const int j = irow[e];
-      if (j >= 0 && j <= iblk) atomicOr(&S.sel[qb][j >> 5], 1u << (j & 31));
-    }
+  const int nsel = sh.per_token ? BM : nqb;
+  for (int e = tid; e < nsel * sh.k; e += NT) {
+    const int r = e / sh.k;
+    const int64_t srow = sh.per_token ? (int64_t)t0 + r : (int64_t)ib0 + r;  // selection row within the head
+    const int iblk = sh.per_token ? (t0 + r) / sh.s : ib0 + r;               // its query block
+    const int j = a.idx[(((int64_t)b * sh.Hq + h) * (sh.per_token ? sh.N : sh.n) + srow) * sh.k + e % sh.k];
+    if (j >= 0 && j <= iblk) atomicOr(&S.sel[r][j >> 5], 1u << (j & 31));
   }
   // Q tile -> fp32 smem.
   constexpr int VEC = Vec16<T>::kN;
@@ -120,7 +121,8 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(FwdArgs a, SimtShape sh) {
     bool myA = false, myD = false;
     if (tid < BM) {
       const unsigned long long causal = causal_mask(t0 + tid, u0);
-      const unsigned long long cm = tile_keep_mask(S.sel[(t0 + tid) / sh.s - ib0], u0, sh.s) & causal;
+      const int r = sh.per_token ? tid : (t0 + tid) / sh.s - ib0;
+      const unsigned long long cm = tile_keep_mask(S.sel[r], u0, sh.s) & causal;
       S.cm[tid] = cm;
       myA = cm != 0ull;
       myD = (causal & ~cm) != 0ull;
@@ -279,7 +281,7 @@ cudaError_t launch_t(const Dims& Dm, const FwdArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(FwdSmem<D>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  SimtShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale};
+  SimtShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale, Dm.per_token};
   dim3 grid(Dm.N / BM, Dm.Hq, Dm.B);
   kern<<<grid, NT, smem, st>>>(a, sh);
   count_launches(1);

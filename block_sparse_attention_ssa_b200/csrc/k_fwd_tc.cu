@@ -622,7 +622,7 @@ bool make_tma_map_bf16(CUtensorMap* map, const TensorRef& t, int B, int H, int N
 }
 
 bool fwd_tc_supported(const Dims& D) {
-  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048;
+  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048 && !D.per_token;
 }
 
 cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st) {

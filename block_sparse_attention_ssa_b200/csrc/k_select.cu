@@ -96,29 +96,17 @@ __device__ __forceinline__ bool better(float a, int ja, float b, int jb) {
   return a > b || (a == b && ja < jb);
 }
 
+// Warp-wide top-k of one selection row whose query block is i: v[m] holds the
+// score of candidate j = lane + 32 m (j < i).  Writes Sel ascending to orow,
+// -1 padded.
 template <int CPL>
-__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ scores,
-                                                     int32_t* __restrict__ idx, int64_t rows,
-                                                     int n, int k) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const int i = (int)(row % n);
-  const float* srow = scores + row * n;
-  int32_t* orow = idx + row * k;
+__device__ __forceinline__ void select_row(float (&v)[CPL], int i, int n, int k, int lane, int32_t* orow) {
   uint64_t taken = 0;
   if (i + 1 <= k) {
 #pragma unroll
     for (int m = 0; m < CPL; ++m)
       if (lane + 32 * m <= i) taken |= 1ull << m;
   } else {
-    float v[CPL];
-#pragma unroll
-    for (int m = 0; m < CPL; ++m) {
-      const int j = lane + 32 * m;
-      float x = (j < i) ? srow[j] : kNegInf;
-      v[m] = (x != x) ? kNegInf : x;  // NaN ranks as -inf
-    }
     for (int round = 0; round < k - 1; ++round) {
       float bv = kNegInf;
       int bj = INT_MAX;
@@ -156,13 +144,82 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ s
   for (int p = base + lane; p < k; p += 32) orow[p] = -1;
 }
 
+template <int CPL>
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ scores,
+                                                     int32_t* __restrict__ idx, int64_t rows,
+                                                     int n, int k) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int i = (int)(row % n);
+  const float* srow = scores + row * n;
+  float v[CPL];
+#pragma unroll
+  for (int m = 0; m < CPL; ++m) {
+    const int j = lane + 32 * m;
+    float x = (j < i) ? srow[j] : kNegInf;
+    v[m] = (x != x) ? kNegInf : x;  // NaN ranks as -inf
+  }
+  select_row<CPL>(v, i, n, k, lane, idx + row * k);
+}
+
+// ------------------------------------------------------------------ per-token selection
+// One warp per (b, h, t) row: the token's own query scores the pooled keys of
+// the complete earlier blocks (score_j = scale q_t . kbar_j, j < i = t / s;
+// lanes split d, RPW pooled keys in flight), then the same top-k as above.
+template <typename T, int D, int CPL>
+__global__ void __launch_bounds__(256) token_select_kernel(TensorRef Q, const float* __restrict__ kbar,
+                                                           int32_t* __restrict__ idx, int64_t rows, int Hq, int g,
+                                                           int N, int s, int n, int k, float scale) {
+  constexpr int PER = D / 32, RPW = 4;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int t = (int)(row % N);
+  const int bh = (int)(row / N), b = bh / Hq, h = bh % Hq;
+  const int i = t / s;
+  float qv[PER];
+  const T* qrow = row_ptr<T>(Q, b, h, t);
+#pragma unroll
+  for (int c = 0; c < PER; ++c) qv[c] = to_f32(qrow[lane * PER + c]);
+  const float* kb = kbar + ((int64_t)b * (Hq / g) + h / g) * n * D;
+  float v[CPL];
+#pragma unroll
+  for (int m = 0; m < CPL; ++m) v[m] = kNegInf;
+  for (int j0 = 0; j0 < i; j0 += RPW) {
+    float kv[RPW][PER];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+#pragma unroll
+      for (int c = 0; c < PER; ++c) kv[r][c] = (j0 + r < i) ? kb[(int64_t)(j0 + r) * D + lane * PER + c] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      float p = 0.f;
+#pragma unroll
+      for (int c = 0; c < PER; ++c) p = fmaf(qv[c], kv[r][c], p);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+      const int j = j0 + r;
+      if (j < i && (j & 31) == lane) {
+        float x = scale * p;
+#pragma unroll
+        for (int m = 0; m < CPL; ++m)
+          if (m == (j >> 5)) v[m] = (x != x) ? kNegInf : x;
+      }
+    }
+  }
+  select_row<CPL>(v, i, n, k, lane, idx + row * k);
+}
+
 // ------------------------------------------------------------------ mask
-// grid = rows, 32 threads: words of the selected-block bit set of one row.
-__global__ void mask_kernel(const int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int n,
+// grid = rows, 32 threads: words of the selected-block bit set of one
+// selection row (a query block, or a token when div = s: i = (row % rph) / div).
+__global__ void mask_kernel(const int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int rph, int div,
                             int k, int words) {
   __shared__ uint32_t w[64];
   const int64_t row = blockIdx.x;
-  const int i = (int)(row % n);
+  const int i = (int)(row % rph) / div;
   for (int q = threadIdx.x; q < words; q += 32) w[q] = 0u;
   __syncwarp();
   for (int e = threadIdx.x; e < k; e += 32) {
@@ -215,10 +272,36 @@ cudaError_t launch_select(const Dims& D, const float* scores, int32_t* idx, cuda
 
 cudaError_t launch_build_mask(const Dims& D, const int32_t* idx, uint32_t* mask, int words,
                               cudaStream_t st) {
-  const int64_t rows = (int64_t)D.B * D.Hq * D.n;
-  mask_kernel<<<(unsigned)rows, 32, 0, st>>>(idx, mask, D.n, D.k, words);
+  const int64_t rows = (int64_t)D.B * D.Hq * D.rows_sel;
+  mask_kernel<<<(unsigned)rows, 32, 0, st>>>(idx, mask, D.rows_sel, D.per_token ? D.s : 1, D.k, words);
   count_launches(1);
   return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t token_select_t(const Dims& Dm, const TensorRef& Q, const float* kbar, int32_t* idx, cudaStream_t st) {
+  const int64_t rows = (int64_t)Dm.B * Dm.Hq * Dm.N;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  const int cpl = (Dm.n + 31) / 32;
+#define SSA_TOKSEL(C) token_select_kernel<T, D, C><<<grid, 256, 0, st>>>(Q, kbar, idx, rows, Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale)
+  if (cpl <= 1) SSA_TOKSEL(1);
+  else if (cpl <= 2) SSA_TOKSEL(2);
+  else if (cpl <= 4) SSA_TOKSEL(4);
+  else if (cpl <= 8) SSA_TOKSEL(8);
+  else if (cpl <= 16) SSA_TOKSEL(16);
+  else if (cpl <= 32) SSA_TOKSEL(32);
+  else SSA_TOKSEL(64);
+#undef SSA_TOKSEL
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_tokens(const Dims& D, const TensorRef& Q, const float* kbar, int32_t* idx,
+                                 cudaStream_t st) {
+  if (D.dtype == SSA_BF16)
+    return D.d == 128 ? token_select_t<__nv_bfloat16, 128>(D, Q, kbar, idx, st)
+                      : token_select_t<__nv_bfloat16, 64>(D, Q, kbar, idx, st);
+  return D.d == 128 ? token_select_t<float, 128>(D, Q, kbar, idx, st) : token_select_t<float, 64>(D, Q, kbar, idx, st);
 }
 
 }  // namespace ssa

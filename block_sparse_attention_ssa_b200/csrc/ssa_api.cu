@@ -26,6 +26,8 @@ ssa_status_t check_dims(const ssa_dims_t* in, Dims* out, bool* empty) {
   D.s = in->block; D.topk = in->topk; D.scale = in->scale; D.dtype = in->dtype;
   if (D.B < 0 || D.Hq < 0 || D.N < 0 || D.Hkv < 1 || D.topk < 1) return SSA_ERR_INVALID_ARG;
   if (D.dtype != SSA_F32 && D.dtype != SSA_BF16) return SSA_ERR_INVALID_ARG;
+  if (in->per_token != 0 && in->per_token != 1) return SSA_ERR_INVALID_ARG;
+  D.per_token = in->per_token;
   if (!(D.scale > 0.f) || D.scale == __builtin_huge_valf()) return SSA_ERR_INVALID_ARG;
   if (D.Hq % D.Hkv != 0) return SSA_ERR_INVALID_ARG;
   if (D.s != 16 && D.s != 32 && D.s != 64 && D.s != 128) return SSA_ERR_UNSUPPORTED;
@@ -35,6 +37,7 @@ ssa_status_t check_dims(const ssa_dims_t* in, Dims* out, bool* empty) {
   if (D.n > 2048) return SSA_ERR_UNSUPPORTED;
   D.k = D.topk < D.n ? D.topk : D.n;
   D.g = D.Hkv > 0 ? D.Hq / D.Hkv : 0;
+  D.rows_sel = D.per_token ? D.N : D.n;
   *empty = ((int64_t)D.B * D.Hq * D.N == 0);
   if (*empty) D.k = D.topk;
   *out = D;
@@ -96,7 +99,7 @@ Layout layout(const Dims& D) {
   L.doc = o; o = align_up(o + rows * D.d * 4);
   L.Df = o; o = align_up(o + rows * 4);
   L.Dc = o; o = align_up(o + rows * 4);
-  L.mask = o; o = align_up(o + (size_t)D.B * D.Hq * D.n * L.words * 4);
+  L.mask = o; o = align_up(o + (size_t)D.B * D.Hq * D.rows_sel * L.words * 4);
   L.partials = o; o = align_up(o + (size_t)L.n_partials * 4);
   L.bytes_bwd = o;
   L.lse = 0;
@@ -138,7 +141,7 @@ using namespace ssa;
 
 extern "C" {
 
-int ssa_version(void) { return 100; }
+int ssa_version(void) { return 110; }
 
 uint64_t ssa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -167,6 +170,7 @@ ssa_status_t ssa_block_scores(const ssa_dims_t* dims, const ssa_tensor_t* Q, con
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
   if (s != SSA_OK) return s;
+  if (D.per_token) return SSA_ERR_INVALID_ARG;  // per-token selection: ssa_select_tokens
   if (empty) return SSA_OK;
   TensorRef q, k;
   if ((s = check_tensor(D, Q, false, &q)) != SSA_OK) return s;
@@ -190,6 +194,7 @@ ssa_status_t ssa_select_topk(const ssa_dims_t* dims, const float* scores, int32_
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
   if (s != SSA_OK) return s;
+  if (D.per_token) return SSA_ERR_INVALID_ARG;  // per-token selection: ssa_select_tokens
   if (empty) return SSA_OK;
   if (scores == nullptr || idx == nullptr) return SSA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(scores) % 4 || reinterpret_cast<uintptr_t>(idx) % 4)
@@ -282,6 +287,28 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
   }
   e = launch_bwd_pre(D, a, st);
   if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
+  return from_cuda(e);
+}
+
+ssa_status_t ssa_select_tokens(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
+                               int32_t* idx, void* ws, size_t ws_bytes, ssa_stream_t stream) {
+  Dims D;
+  bool empty = false;
+  ssa_status_t s = check_dims(dims, &D, &empty);
+  if (s != SSA_OK) return s;
+  if (!D.per_token) return SSA_ERR_INVALID_ARG;  // per-block selection: ssa_block_scores + ssa_select_topk
+  if (empty) return SSA_OK;
+  TensorRef q, k;
+  if ((s = check_tensor(D, Q, false, &q)) != SSA_OK) return s;
+  if ((s = check_tensor(D, K, false, &k)) != SSA_OK) return s;
+  if (idx == nullptr || reinterpret_cast<uintptr_t>(idx) % 4) return SSA_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
+  if ((s = check_device()) != SSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(D);
+  float* kbar = at<float>(ws, L.kbar);
+  cudaError_t e = launch_pool(D, k, D.Hkv, kbar, st);
+  if (e == cudaSuccess) e = launch_select_tokens(D, q, kbar, idx, st);
   return from_cuda(e);
 }
 
@@ -532,6 +559,7 @@ extern "C" ssa_status_t ssa_block_scores_noalloc(const ssa_dims_t* dims, const s
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
   if (s != SSA_OK) return s;
+  if (D.per_token) return SSA_ERR_INVALID_ARG;  // block scores only
   if (empty) return SSA_OK;
   TensorRef q, k;
   if ((s = check_tensor(D, Q, false, &q)) != SSA_OK) return s;

@@ -16,6 +16,8 @@ struct Dims {
   int B, Hq, Hkv, N, d, s, topk, k, n, g;  // k = min(topk, n), g = Hq / Hkv
   float scale;
   int dtype;
+  int per_token;  // selection per query token (1) or per query block (0)
+  int rows_sel;   // rows of the selection per head: N (per token) or n
 };
 
 // A [B, H, N, d] tensor with a contiguous d dimension; strides in elements.
@@ -108,9 +110,14 @@ cudaError_t launch_scores(const Dims& D, const float* qbar, const float* kbar, f
 // Top-k block selection with the forced diagonal.
 cudaError_t launch_select(const Dims& D, const float* scores, int32_t* idx, cudaStream_t st);
 
-// Bit mask [B, Hq, n, words] of Sel(i) built from idx (entries outside [0,i] ignored).
+// Bit mask [B, Hq, rows_sel, words] of each selection row built from idx
+// (entries outside [0, i] ignored, i the row's query block).
 cudaError_t launch_build_mask(const Dims& D, const int32_t* idx, uint32_t* mask, int words,
                               cudaStream_t st);
+
+// Per-token selection: kbar [B,Hkv,n,d] fp32 (pooled keys) -> idx [B,Hq,N,k].
+cudaError_t launch_select_tokens(const Dims& D, const TensorRef& Q, const float* kbar, int32_t* idx,
+                                 cudaStream_t st);
 
 struct FwdArgs {
   TensorRef q, k, v, hf, hs;

@@ -87,7 +87,10 @@ typedef enum { SSA_F32 = 0, SSA_BF16 = 1 } ssa_dtype_t;
 typedef struct {
   int32_t B, Hq, Hkv, N, d, block, topk;
   float scale;
-  int32_t dtype; /* ssa_dtype_t */
+  int32_t dtype;     /* ssa_dtype_t */
+  int32_t per_token; /* 0: one selection per query block (idx rows = n);
+                        1: one selection per query token (idx rows = N),
+                        see ssa_select_tokens */
 } ssa_dims_t;
 
 typedef struct {
@@ -137,6 +140,22 @@ SSA_API ssa_status_t ssa_block_scores(const ssa_dims_t* dims, const ssa_tensor_t
 SSA_API ssa_status_t ssa_select_topk(const ssa_dims_t* dims, const float* scores,
                              int32_t* idx, ssa_stream_t stream);
 
+/* Step 1+2, per-token selection (dims->per_token = 1).
+ * The literal reading of [digest] "Practical Implementation of SSA" ("the
+ * query" is scored against every earlier block representation), as in
+ * MoBA: each query token t (block i = t/s) ranks the complete earlier
+ * blocks by its own query, score_j = scale * q_t . kbar_j (j < i, kbar_j the
+ * mean of key block j), and keeps Sel(t) = {i} plus the k_eff-1 best (ties to
+ * the smaller j; {0..i} when i + 1 <= k_eff).  Every other entry point takes
+ * the resulting per-token idx when dims->per_token = 1 (the CUDA-core kernels
+ * run; the tensor-core kernels and ssa_block_scores / ssa_select_topk are
+ * per-block only and return SSA_ERR_INVALID_ARG or fall back).
+ *   idx [B, Hq, N, k_eff] int32 (out): Sel(t) ascending, -1 padded.
+ *   ws: workspace of at least ssa_workspace_bytes(dims) bytes (pooled keys). */
+SSA_API ssa_status_t ssa_select_tokens(const ssa_dims_t* dims, const ssa_tensor_t* Q,
+                               const ssa_tensor_t* K, int32_t* idx, void* ws,
+                               size_t ws_bytes, ssa_stream_t stream);
+
 /* Step 3: fused dual-stream forward.
  * One pass over every causal K/V tile keeps two disjoint online softmaxes,
  * over A_t and over D_t, and merges them at the end:
@@ -149,7 +168,8 @@ SSA_API ssa_status_t ssa_select_topk(const ssa_dims_t* dims, const float* scores
  *     ([summary] "1. Probleemstelling"; [record] abstract); 0 when D_t is empty;
  *   lse_full[t], lse_sel[t] = natural-log normalisers of the two softmaxes.
  * x_tu = scale * q_t . k_u.
- *   idx [B, Hq, n, k_eff] int32 (in): as written by ssa_select_topk.  Any
+ *   idx [B, Hq, n, k_eff] int32 (in): as written by ssa_select_topk ([B, Hq,
+ *     N, k_eff] from ssa_select_tokens when dims->per_token = 1).  Any
  *     other selection may be passed: entries outside [0, i] are ignored and
  *     duplicates are harmless.  A row that omits its diagonal block attends
  *     only the listed blocks; a query whose A_t is empty gets h_sparse = 0,

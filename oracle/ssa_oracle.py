@@ -180,20 +180,72 @@ def _logsumexp(X: np.ndarray, mask: np.ndarray) -> np.ndarray:
 
 
 def _block_masks(idx_row: np.ndarray, i: int, s: int):
-    """For query block i: token-level (causal, selected) masks of shape [s, (i+1)s]."""
+    """For query block i: token-level (causal, selected) masks of shape [s, (i+1)s].
+
+    idx_row is the block's selection [k], or (per-token selection) one
+    selection per row of the block [s, k].
+    """
     cols = (i + 1) * s
     t = i * s + np.arange(s)[:, None]
     u = np.arange(cols)[None, :]
     causal = u <= t
-    sel_blocks = np.zeros(i + 1, dtype=bool)
-    for j in idx_row:
-        if 0 <= j <= i:
-            sel_blocks[j] = True
-    sel = np.repeat(sel_blocks, s)[None, :]
+    rows = np.asarray(idx_row).reshape(-1, np.asarray(idx_row).shape[-1])
+    sel = np.zeros((rows.shape[0], cols), dtype=bool)
+    for r, row in enumerate(rows):
+        for j in row:
+            if 0 <= j <= i:
+                sel[r, j * s:(j + 1) * s] = True
     return causal, causal & sel
 
 
-def forward_dual(Q, K, V, idx, s: int, scale: float, qblocks=None) -> dict[str, np.ndarray]:
+def _sel(idx, b: int, h: int, i: int, s: int, per_token: bool):
+    """Selection of query block i: idx[b, h, i] ([k]), or per token the
+    block's s rows idx[b, h, i*s:(i+1)*s] ([s, k])."""
+    return idx[b, h, i * s:(i + 1) * s] if per_token else idx[b, h, i]
+
+
+def token_scores(Q: np.ndarray, K: np.ndarray, s: int, scale: float) -> np.ndarray:
+    """Per-token block scores S[b, h, t, j] = scale * q_t . kbar_j for j < t // s.
+
+    The literal reading of [digest] "Practical Implementation of SSA": the
+    query (token t) is scored against every earlier block representation
+    (the mean of the block's keys); -inf for the current and later blocks.
+    """
+    Q, K = _f64(Q), _f64(K)
+    B, Hq, N, d = Q.shape
+    g = Hq // K.shape[1]
+    n = N // s
+    kbar = pool_blocks(K, s)[:, np.arange(Hq) // g]          # [B,Hq,n,d]
+    S = scale * np.einsum("bhtd,bhjd->bhtj", Q, kbar)
+    tb = (np.arange(N) // s)[:, None]
+    S[..., np.arange(n)[None, :] >= tb] = -np.inf
+    return S
+
+
+def select_tokens(scores: np.ndarray, k: int, s: int) -> np.ndarray:
+    """Per-token selection [B, H, N, min(k, n)] int32, ascending, -1 padded:
+    Sel(t) = {i} plus the k-1 highest-scoring blocks j < i = t // s, ties to
+    the smaller j; every block 0..i when i + 1 <= k (the block rule of
+    select_blocks applied to each token's own scores)."""
+    S = _f64(scores)
+    B, H, N, n = S.shape
+    kk = min(int(k), n)
+    idx = np.full((B, H, N, kk), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for t in range(N):
+                i = t // s
+                if i + 1 <= kk:
+                    chosen = np.arange(i + 1)
+                else:
+                    cand = S[b, h, t, :i]
+                    order = np.lexsort((np.arange(i), -cand))
+                    chosen = np.sort(np.append(order[: kk - 1], i))
+                idx[b, h, t, : chosen.size] = chosen
+    return idx
+
+
+def forward_dual(Q, K, V, idx, s: int, scale: float, qblocks=None, per_token: bool = False) -> dict[str, np.ndarray]:
     """Both attention streams, the dropped mass and the log-sum-exps.
 
     Returns float64 arrays:
@@ -208,6 +260,7 @@ def forward_dual(Q, K, V, idx, s: int, scale: float, qblocks=None) -> dict[str, 
       lse_full, lse_sel [B,Hq,N]  natural-log normalisers of the two softmaxes.
     qblocks: optional iterable of query-block indices to compute (rows of other
     blocks are left at zero); used to sample large problems.
+    per_token: idx holds one selection per token ([B, Hq, N, k]).
     """
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     B, Hq, N, d = Q.shape
@@ -226,7 +279,7 @@ def forward_dual(Q, K, V, idx, s: int, scale: float, qblocks=None) -> dict[str, 
                 rows = slice(i * s, (i + 1) * s)
                 cols = (i + 1) * s
                 X = _row_logits(Q[b, h, rows], K[b, kv, :cols], scale)
-                causal, A = _block_masks(idx[b, h, i], i, s)
+                causal, A = _block_masks(_sel(idx, b, h, i, s, per_token), i, s)
                 P_full = _masked_softmax(X, causal)
                 P_sel = _masked_softmax(X, A)
                 Vc = V[b, kv, :cols]
@@ -269,7 +322,8 @@ def align_grads(h_full, h_sparse, M: int | None = None) -> dict[str, np.ndarray]
             "cm_full": zero, "cm_sparse": 2.0 * (hs - hf) / M}
 
 
-def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse, qblocks=None):
+def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse, qblocks=None,
+                     per_token: bool = False):
     """Backpropagate upstream gradients of h_full and h_sparse to Q, K, V.
 
     The two streams are differentiated separately, each through its own
@@ -304,7 +358,7 @@ def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse, qbl
                 cols = (i + 1) * s
                 Kc, Vc = K[b, kv, :cols], V[b, kv, :cols]
                 X = _row_logits(Q[b, h, rows], Kc, scale)
-                causal, A = _block_masks(idx[b, h, i], i, s)
+                causal, A = _block_masks(_sel(idx, b, h, i, s, per_token), i, s)
                 P_full = _masked_softmax(X, causal)
                 P_sel = _masked_softmax(X, A)
                 dP_full = dhf[b, h, rows] @ Vc.T
@@ -319,7 +373,7 @@ def backward_streams(Q, K, V, idx, s: int, scale: float, dh_full, dh_sparse, qbl
 
 
 def ssa_backward(Q, K, V, idx, s: int, scale: float, g_full, g_sparse, alpha: float,
-                 fwd: dict | None = None, qblocks=None, M: int | None = None):
+                 fwd: dict | None = None, qblocks=None, M: int | None = None, per_token: bool = False):
     """Gradients of L = <g_full, h_full> + <g_sparse, h_sparse> + alpha * L_align.
 
     [summary] "Bidirectionele Uitlijning": the objective adds alpha times the
@@ -330,7 +384,7 @@ def ssa_backward(Q, K, V, idx, s: int, scale: float, g_full, g_sparse, alpha: fl
     Returns (dQ, dK, dV, L_align, fwd).
     """
     if fwd is None:
-        fwd = forward_dual(Q, K, V, idx, s, scale, qblocks=qblocks)
+        fwd = forward_dual(Q, K, V, idx, s, scale, qblocks=qblocks, per_token=per_token)
     hf, hs = fwd["h_full"], fwd["h_sparse"]
     gr = align_grads(hf, hs, M)
     dh_full = alpha * (gr["sp_full"] + gr["cm_full"])
@@ -339,12 +393,13 @@ def ssa_backward(Q, K, V, idx, s: int, scale: float, g_full, g_sparse, alpha: fl
         dh_full = dh_full + _f64(g_full)
     if g_sparse is not None:
         dh_sparse = dh_sparse + _f64(g_sparse)
-    dQ, dK, dV = backward_streams(Q, K, V, idx, s, scale, dh_full, dh_sparse, qblocks=qblocks)
+    dQ, dK, dV = backward_streams(Q, K, V, idx, s, scale, dh_full, dh_sparse, qblocks=qblocks,
+                                  per_token=per_token)
     l_sp, l_cm = align_losses(hf, hs)
     return dQ, dK, dV, l_sp + l_cm, fwd
 
 
-def dropped_mass(Q, K, idx, s: int, scale: float) -> np.ndarray:
+def dropped_mass(Q, K, idx, s: int, scale: float, per_token: bool = False) -> np.ndarray:
     """delta(t): the full causal softmax weight of row t summed over D_t.
 
     [summary] "1. Probleemstelling": the dropped attention mass is the
@@ -362,13 +417,13 @@ def dropped_mass(Q, K, idx, s: int, scale: float) -> np.ndarray:
                 rows = slice(i * s, (i + 1) * s)
                 cols = (i + 1) * s
                 X = _row_logits(Q[b, h, rows], K[b, h // g, :cols], scale)
-                causal, A = _block_masks(idx[b, h, i], i, s)
+                causal, A = _block_masks(_sel(idx, b, h, i, s, per_token), i, s)
                 P_full = _masked_softmax(X, causal)
                 delta[b, h, rows] = np.where(causal & ~A, P_full, 0.0).sum(-1)
     return delta
 
 
-def forward_sparse(Q, K, V, idx, s: int, scale: float, qblocks=None) -> dict[str, np.ndarray]:
+def forward_sparse(Q, K, V, idx, s: int, scale: float, qblocks=None, per_token: bool = False) -> dict[str, np.ndarray]:
     """The sparse stream alone: h_sparse and lse_sel, reading only selected blocks.
 
     [digest] "Practical Implementation of SSA": the selected blocks are
@@ -392,10 +447,11 @@ def forward_sparse(Q, K, V, idx, s: int, scale: float, qblocks=None) -> dict[str
         for h in range(Hq):
             kv = h // g
             for i in blocks:
-                sel = sorted(set(int(j) for j in idx[b, h, i] if 0 <= j <= i))
-                keys = np.concatenate([np.arange(j * s, (j + 1) * s) for j in sel]) if sel else np.zeros(0, int)
                 for r in range(s):
                     t = i * s + r
+                    row = idx[b, h, t] if per_token else idx[b, h, i]
+                    sel = sorted(set(int(j) for j in row if 0 <= j <= i))
+                    keys = np.concatenate([np.arange(j * s, (j + 1) * s) for j in sel]) if sel else np.zeros(0, int)
                     cols = keys[keys <= t]
                     if cols.size == 0:
                         lse_sel[b, h, t] = -np.inf
@@ -409,7 +465,7 @@ def forward_sparse(Q, K, V, idx, s: int, scale: float, qblocks=None) -> dict[str
     return {"h_sparse": h_sparse, "lse_sel": lse_sel}
 
 
-def backward_sparse(Q, K, V, idx, s: int, scale: float, g_sparse, qblocks=None):
+def backward_sparse(Q, K, V, idx, s: int, scale: float, g_sparse, qblocks=None, per_token: bool = False):
     """Gradients (dQ, dK, dV) of <g_sparse, h_sparse> for the sparse stream alone.
 
     The sparse stream's own softmax Jacobian over A_t, the selection held
@@ -417,7 +473,7 @@ def backward_sparse(Q, K, V, idx, s: int, scale: float, g_sparse, qblocks=None):
     Paradox": a purely sparse stream gives no gradient to the tokens it does
     not select).  It is backward_streams with no full-stream gradient.
     """
-    return backward_streams(Q, K, V, idx, s, scale, None, g_sparse, qblocks=qblocks)
+    return backward_streams(Q, K, V, idx, s, scale, None, g_sparse, qblocks=qblocks, per_token=per_token)
 
 
 def decode_select(q_prefix, K, t: int, s: int, k: int, scale: float, n_cache: int | None = None) -> np.ndarray:

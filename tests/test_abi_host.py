@@ -23,7 +23,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.ssa_version() == 100
+    assert lib.ssa_version() == 110
     for code, name in enumerate(["SSA_OK", "SSA_ERR_INVALID_ARG", "SSA_ERR_UNSUPPORTED", "SSA_ERR_CUDA",
                                  "SSA_ERR_TIMEOUT", "SSA_ERR_WORKSPACE"]):
         assert api.status_string(code) == name
@@ -59,6 +59,7 @@ def _tensor(ptr=16, sb=4096 * 128, sh=4096 * 128, sn=128):
     ("topk", 0, api.SSA_ERR_INVALID_ARG),
     ("B", -1, api.SSA_ERR_INVALID_ARG),
     ("dtype", 7, api.SSA_ERR_INVALID_ARG),
+    ("per_token", 2, api.SSA_ERR_INVALID_ARG),
     ("scale", float("nan"), api.SSA_ERR_INVALID_ARG),
     ("scale", 0.0, api.SSA_ERR_INVALID_ARG),
     ("scale", -0.125, api.SSA_ERR_INVALID_ARG),
@@ -114,3 +115,19 @@ def test_empty_shapes_are_noops(lib):
         setattr(d, field, 0)
         assert lib.ssa_fwd_dual(ctypes.byref(d), t, t, t, p, t, t, p, p, p, None) == api.SSA_OK
         assert lib.ssa_select_topk(ctypes.byref(d), p, p, None) == api.SSA_OK
+
+
+def test_selection_modes_are_exclusive(lib):
+    """Per-block scoring entry points refuse per-token dims and the per-token
+    selection refuses per-block dims, before anything is enqueued."""
+    t = _tensor()
+    dt = api.make_dims(1, 4, 2, 1024, 128, 64, 4, per_token=True)
+    db = api.make_dims(1, 4, 2, 1024, 128, 64, 4)
+    assert lib.ssa_block_scores(ctypes.byref(dt), t, t, ctypes.c_void_p(16), ctypes.c_void_p(256), 1 << 40,
+                                None) == api.SSA_ERR_INVALID_ARG
+    assert lib.ssa_select_topk(ctypes.byref(dt), ctypes.c_void_p(16), ctypes.c_void_p(16), None) == \
+        api.SSA_ERR_INVALID_ARG
+    assert lib.ssa_select_tokens(ctypes.byref(db), t, t, ctypes.c_void_p(16), ctypes.c_void_p(256), 1 << 40,
+                                 None) == api.SSA_ERR_INVALID_ARG
+    # the per-token selection mask is per token: the workspace grows accordingly
+    assert api.ssa_workspace_bytes(dt) >= api.ssa_workspace_bytes(db)

@@ -1,0 +1,152 @@
+"""GPU parity of per-token selection (dims.per_token = 1; each query token
+ranks the earlier blocks by its own query, the literal reading of "the
+query" in "Practical Implementation of SSA") against the fp64 oracle, through
+the C ABI: the selection itself (bit-exact, near ties logged and compared
+under the oracle's indices), the dual forward, the dropped mass, the sparse
+stream alone forward and backward, the dual backward and the decode step.
+Block sizes 64 and 16, bf16 and fp32, GQA.  Tolerances as elsewhere."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_ssa_b200 import api
+from block_sparse_attention_ssa_b200.inputs import make_upstream
+from oracle import ssa_oracle as O
+from tests.gpu_util import NEAR_TIE_REL, TOL, case_inputs, ensure_library, f64, oracle_view, rel_l2, upload
+
+pytestmark = pytest.mark.gpu
+
+# name: B, Hq, Hkv, N, d, s, k, dtype
+CASES = {
+    "f32_s64_d64": (1, 2, 1, 512, 64, 64, 3, "f32"),
+    "bf16_s64_d128_gqa": (1, 4, 2, 768, 128, 64, 4, "bf16"),
+    "bf16_s16_d64_g8": (1, 8, 1, 512, 64, 16, 8, "bf16"),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    return ensure_library()
+
+
+def _compare_token_selection(gpu_idx, ora_idx, ora_scores, s):
+    """Rows (b, h, t) where the selections differ must be near ties."""
+    diff = np.any(gpu_idx != ora_idx, axis=-1)
+    rows = list(zip(*np.nonzero(diff)))
+    for (b, h, t) in rows:
+        i = t // s
+        g = {int(j) for j in gpu_idx[b, h, t] if j >= 0}
+        o = {int(j) for j in ora_idx[b, h, t] if j >= 0}
+        assert len(g) == len(o) and i in g and i in o, (b, h, t, g, o)
+        thr = min(ora_scores[b, h, t, j] for j in o if j != i)
+        for j in g ^ o:
+            a = ora_scores[b, h, t, j]
+            assert abs(a - thr) <= NEAR_TIE_REL * max(abs(a), abs(thr)), (b, h, t, j, a, thr)
+    return rows
+
+
+def _run(name, seed=828):
+    B, Hq, Hkv, N, d, s, k, dt = CASES[name]
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, seed, dt)
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, dt, per_token=True)
+    ws = api.alloc_workspace(dims)
+    out = api.alloc_forward(dims)
+    scale = 1 / math.sqrt(d)
+    api.ssa_select_tokens(dims, dev["Q"], dev["K"], out["idx"], ws)
+    torch.cuda.synchronize()
+    ora_scores = O.token_scores(host["Q"], host["K"], s, scale)
+    ora_idx = O.select_tokens(ora_scores, k, s)
+    if _compare_token_selection(out["idx"].cpu().numpy(), ora_idx, ora_scores, s):
+        out["idx"].copy_(torch.from_numpy(ora_idx))
+    api.ssa_fwd_dual(dims, dev["Q"], dev["K"], dev["V"], out["idx"], out["h_full"], out["h_sparse"],
+                     out["lse_full"], out["lse_sel"], out["delta"])
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    ora = O.forward_dual(host["Q"], host["K"], host["V"], ora_idx, s, scale, per_token=True)
+    return dict(dims=dims, dev=dev, host=host, out=out, ws=ws, ora=ora, ora_idx=ora_idx, scale=scale,
+                cfg=CASES[name])
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_token_forward_dual(name):
+    r = _run(name)
+    dt = r["cfg"][7]
+    for key in ("h_full", "h_sparse", "delta"):
+        assert np.abs(f64(r["out"][key]) - r["ora"][key]).max() <= TOL[dt]["out"], key
+    for key in ("lse_full", "lse_sel"):
+        assert np.abs(f64(r["out"][key]) - r["ora"][key]).max() <= TOL[dt]["lse"], key
+    # selections really differ inside query blocks
+    idx = r["out"]["idx"].cpu().numpy()
+    s = r["cfg"][5]
+    assert any(len({tuple(idx[0, 0, t]) for t in range(i * s, i * s + s)}) > 1 for i in range(idx.shape[2] // s))
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_token_dropped_and_sparse_alone(name):
+    r = _run(name)
+    B, Hq, Hkv, N, d, s, k, dt = r["cfg"]
+    dims, dev, host = r["dims"], r["dev"], r["host"]
+    for lse in (r["out"]["lse_full"], None):
+        delta = torch.full_like(r["out"]["delta"], float("nan"))
+        api.ssa_dropped_mass(dims, dev["Q"], dev["K"], r["out"]["idx"], lse, delta, r["ws"])
+        torch.cuda.synchronize()
+        assert np.abs(f64(delta) - r["ora"]["delta"]).max() <= TOL[dt]["out"]
+    hs = torch.full_like(r["out"]["h_sparse"], float("nan"))
+    lse_s = torch.full_like(r["out"]["lse_sel"], float("nan"))
+    api.ssa_fwd_sparse(dims, dev["Q"], dev["K"], dev["V"], r["out"]["idx"], hs, lse_s)
+    torch.cuda.synchronize()
+    assert np.abs(f64(hs) - r["ora"]["h_sparse"]).max() <= TOL[dt]["out"]
+    g = make_upstream((B, Hq, N, d), 71)
+    grads = api.alloc_backward(dims)
+    api.ssa_bwd_sparse(dims, dev["Q"], dev["K"], dev["V"], r["out"]["idx"], hs, lse_s, upload(g, dt), grads["dQ"],
+                       grads["dK"], grads["dV"], r["ws"])
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    dQ, dK, dV = O.backward_sparse(host["Q"], host["K"], host["V"], r["ora_idx"], s, r["scale"],
+                                   oracle_view(g, dt).astype(np.float64), per_token=True)
+    for key, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        assert rel_l2(f64(got), ref) < TOL[dt]["grad"], key
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_token_backward_dual(name):
+    r = _run(name)
+    B, Hq, Hkv, N, d, s, k, dt = r["cfg"]
+    g = make_upstream((B, Hq, N, d), 72)
+    grads = api.alloc_backward(r["dims"])
+    api.backward(r["dims"], r["dev"]["Q"], r["dev"]["K"], r["dev"]["V"], r["out"], None, upload(g, dt), 10.0, grads,
+                 r["ws"])
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    dQ, dK, dV, _, _ = O.ssa_backward(r["host"]["Q"], r["host"]["K"], r["host"]["V"], r["ora_idx"], s, r["scale"],
+                                      None, oracle_view(g, dt).astype(np.float64), 10.0, fwd=r["ora"],
+                                      per_token=True)
+    for key, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        assert rel_l2(f64(got), ref) < TOL[dt]["grad"], key
+
+
+def test_token_decode():
+    """Per-token decode: the query side of the score is q_t itself."""
+    B, Hq, Hkv, N, d, s, k = 1, 4, 2, 512, 64, 16, 6
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 929, "f32")
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "f32", per_token=True)
+    st = api.alloc_decode(dims)
+    ws = api.alloc_workspace(dims)
+    t0 = 16 * 9 + 3
+    api.ssa_decode_prefill(dims, dev["Q"], dev["K"], t0, st["qsum"], st["kbar"])
+    scale = 1 / math.sqrt(d)
+    for t in range(t0, t0 + 40):
+        api.ssa_decode_step(dims, dev["Q"][:, :, t:t + 1], dev["K"], dev["V"], t, st["qsum"], st["kbar"], st["h"],
+                            st["lse"], st["idx"], ws)
+        torch.cuda.synchronize()
+        oidx = O.decode_select(host["Q"][:, :, t:t + 1], host["K"], t, s, k, scale, n_cache=N // s)
+        assert np.array_equal(st["idx"].cpu().numpy(), oidx), t
+        h_ref, lse_ref = O.decode_attend(host["Q"][:, :, t], host["K"], host["V"], t, s, oidx, scale)
+        assert np.abs(f64(st["h"])[:, :, 0] - h_ref).max() <= TOL["f32"]["out"], t
+        assert np.abs(f64(st["lse"]) - lse_ref).max() <= TOL["f32"]["lse"], t
+    # per-token decode agrees with the per-token forward on the last row
+    idx_f = O.select_tokens(O.token_scores(host["Q"], host["K"], s, scale), k, s)
+    t = t0 + 39
+    np.testing.assert_array_equal(idx_f[:, :, t], st["idx"].cpu().numpy())

@@ -509,6 +509,94 @@ def test_decode_full_budget_is_causal_attention():
         np.testing.assert_allclose(h, ref.numpy()[:, :, t], rtol=0, atol=1e-12)
 
 
+# ---------------------------------------------------------------- per-token selection
+
+def test_token_selection_brute_force():
+    """Per token, the kept set is the best (k-1)-subset of the earlier blocks,
+    found by enumeration from scores summed by explicit loops over q_t and the
+    block's keys; the token's own block is always kept."""
+    Q, K, _ = tiny(Hq=2, Hkv=1, N=40, d=3, s=8, seed=41)
+    s, k, scale = 8, 3, 0.6
+    idx = O.select_tokens(O.token_scores(Q, K, s, scale), k, s)
+    for h in range(2):
+        for t in range(40):
+            i = t // s
+            got = [int(j) for j in idx[0, h, t] if j >= 0]
+            if i + 1 <= k:
+                assert got == list(range(i + 1))
+                continue
+            sc = [scale * sum(Q[0, h, t, c] * sum(K[0, 0, u, c] for u in range(j * s, j * s + s)) / s
+                              for c in range(3)) for j in range(i)]
+            best = max(itertools.combinations(range(i), k - 1), key=lambda c: sum(sc[j] for j in c))
+            assert got == sorted(best) + [i]
+
+
+def test_token_mode_equals_block_mode_for_block_constant_queries():
+    """When every query of a block is the same vector, each token's score row
+    is its block's score row, so per-token selection equals per-block
+    selection and every output and gradient agrees."""
+    Q, K, V = tiny(Hq=4, Hkv=2, N=48, d=4, s=8, seed=42)
+    s, k, scale = 8, 2, 0.5
+    Qc = np.repeat(Q.reshape(1, 4, 6, 8, 4).mean(axis=3), 8, axis=2)     # block-constant queries
+    ib = O.select_blocks(O.block_scores(Qc, K, s, scale), k)
+    it = O.select_tokens(O.token_scores(Qc, K, s, scale), k, s)
+    np.testing.assert_array_equal(it, np.repeat(ib, 8, axis=2))
+    fb = O.forward_dual(Qc, K, V, ib, s, scale)
+    ft = O.forward_dual(Qc, K, V, it, s, scale, per_token=True)
+    for key in fb:
+        np.testing.assert_allclose(ft[key], fb[key], rtol=0, atol=1e-13)
+    g = make_upstream(Q.shape, 43).astype(np.float64)
+    gb = O.ssa_backward(Qc, K, V, ib, s, scale, None, g, 5.0)
+    gt = O.ssa_backward(Qc, K, V, it, s, scale, None, g, 5.0, per_token=True)
+    for a, b in zip(gt[:3], gb[:3]):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_token_mode_rows_by_explicit_loops():
+    """Rows of one block keep different sets; every row's sparse and full
+    softmax, dropped mass and the gathered sparse stream match loops over
+    that row's own kept keys."""
+    Q, K, V = tiny(Hq=2, Hkv=1, N=48, d=3, s=8, seed=44)
+    s, k, scale = 8, 2, 0.8
+    idx = O.select_tokens(O.token_scores(Q, K, s, scale), k, s)
+    assert any(len({tuple(idx[0, 0, t]) for t in range(i * s, i * s + s)}) > 1 for i in range(2, 6))
+    f = O.forward_dual(Q, K, V, idx, s, scale, per_token=True)
+    fs = O.forward_sparse(Q, K, V, idx, s, scale, per_token=True)
+    dm = O.dropped_mass(Q, K, idx, s, scale, per_token=True)
+    for h in range(2):
+        for t in range(48):
+            keep = {int(j) for j in idx[0, h, t] if j >= 0}
+            x = [scale * sum(Q[0, h, t, c] * K[0, 0, u, c] for c in range(3)) for u in range(t + 1)]
+            m = max(x)
+            w = [math.exp(v - m) for v in x]
+            A = [u for u in range(t + 1) if u // s in keep]
+            zA, z = sum(w[u] for u in A), sum(w)
+            hs = [sum(w[u] * V[0, 0, u, c] for u in A) / zA for c in range(3)]
+            hf = [sum(w[u] * V[0, 0, u, c] for u in range(t + 1)) / z for c in range(3)]
+            np.testing.assert_allclose(f["h_sparse"][0, h, t], hs, atol=1e-12)
+            np.testing.assert_allclose(fs["h_sparse"][0, h, t], hs, atol=1e-12)
+            np.testing.assert_allclose(f["h_full"][0, h, t], hf, atol=1e-12)
+            assert f["delta"][0, h, t] == pytest.approx(1 - zA / z, abs=1e-12)
+            assert dm[0, h, t] == pytest.approx(1 - zA / z, abs=1e-12)
+
+
+def test_token_mode_backward_matches_finite_differences():
+    """Central differences of <g, h_sparse> + alpha * mean((h_f - h_s)^2) with
+    per-token selections held fixed."""
+    Q, K, V = tiny(**FD_CFG, seed=45)
+    s, k, scale, alpha = 8, 2, 0.5, 10.0
+    idx = O.select_tokens(O.token_scores(Q, K, s, scale), k, s)
+    g = make_upstream(Q.shape, 46).astype(np.float64)
+
+    def loss():
+        f = O.forward_dual(Q, K, V, idx, s, scale, per_token=True)
+        return float((g * f["h_sparse"]).sum() + alpha * np.mean((f["h_full"] - f["h_sparse"]) ** 2))
+
+    dQ, dK, dV, _, _ = O.ssa_backward(Q, K, V, idx, s, scale, None, g, alpha, per_token=True)
+    fQ, fK, fV = _fd_grad(loss, [Q, K, V])
+    assert _rel(dQ, fQ) < 1e-6 and _rel(dK, fK) < 1e-6 and _rel(dV, fV) < 1e-6
+
+
 # ---------------------------------------------------------------- frozen regression fixture
 
 def test_golden_fixture_is_reproduced():
