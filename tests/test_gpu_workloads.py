@@ -145,3 +145,31 @@ def test_budget_sweep(k):
     _check_forward_samples(w, host, out, delta2, ora_idx, scale, rng)
     _check_backward_samples(w, host, grads, ora_idx, scale, rng)
     print(f"sweep_32k k={k}: mean delta {float(out['delta'].mean()):.4f}")
+
+
+def test_maximum_block_count():
+    """The largest supported selection: n = 2048 blocks (N = 131072 at block
+    64) with k = 64, through block scores, top-k (2047 candidates per row),
+    the dual forward, the dropped mass, the backward and the sparse stream
+    alone; checked on sampled query blocks, including the last one, and on
+    the last key block's gradients."""
+    from block_sparse_attention_ssa_b200.inputs import Workload
+    w = Workload("max_blocks", 1, 2, 1, 131072, 128, 64, 64, "bf16", 1007)
+    rng = np.random.Generator(np.random.PCG64(5))
+    host, out, grads, delta2, ora_idx, scale = _run(w, with_bwd=True)
+    _check_forward_samples(w, host, out, delta2, ora_idx, scale, rng)
+    _check_backward_samples(w, host, grads, ora_idx, scale, rng)
+    dims = api.make_dims(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, w.topk, w.dtype)
+    dev = _device(w, host)
+    hs = torch.empty_like(out["h_sparse"])
+    lse = torch.empty_like(out["lse_sel"])
+    api.ssa_fwd_sparse(dims, dev["Q"], dev["K"], dev["V"], out["idx"], hs, lse)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    for (b, h, i) in _samples(w, rng):
+        N1 = (i + 1) * w.block
+        f = O.forward_sparse(host["Q"][b:b + 1, h:h + 1, :N1], host["K"][b:b + 1, :, :N1],
+                             host["V"][b:b + 1, :, :N1], ora_idx[b:b + 1, h:h + 1, :i + 1], w.block, scale,
+                             qblocks=[i])
+        rows = slice(i * w.block, N1)
+        assert np.abs(f64(hs[b, h, rows]) - f["h_sparse"][0, 0, rows]).max() <= TOL["bf16"]["out"], (b, h, i)
