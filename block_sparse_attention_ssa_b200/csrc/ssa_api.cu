@@ -4,9 +4,21 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ssa_internal.cuh"
 
 namespace ssa {
+
+// One NVTX range per entry-point call, named after the call, so a profiler
+// timeline (nsys, ncu --nvtx) shows which call enqueued which kernels.
+// Header-only NVTX 3: without an attached tool the push / pop are no-ops.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -166,6 +178,7 @@ size_t ssa_workspace_bytes(const ssa_dims_t* dims) {
 
 ssa_status_t ssa_block_scores(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
                               float* scores, void* ws, size_t ws_bytes, ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_block_scores");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -190,6 +203,7 @@ ssa_status_t ssa_block_scores(const ssa_dims_t* dims, const ssa_tensor_t* Q, con
 
 ssa_status_t ssa_select_topk(const ssa_dims_t* dims, const float* scores, int32_t* idx,
                              ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_select_topk");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -207,6 +221,7 @@ ssa_status_t ssa_fwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
                           const ssa_tensor_t* V, const int32_t* idx, const ssa_tensor_t* h_full,
                           const ssa_tensor_t* h_sparse, float* lse_full, float* lse_sel,
                           float* delta, ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_fwd_dual");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -241,6 +256,7 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
                           const ssa_tensor_t* g_sparse, float alpha, float* align_loss,
                           const ssa_tensor_t* dQ, const ssa_tensor_t* dK, const ssa_tensor_t* dV,
                           void* ws, size_t ws_bytes, ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_bwd_dual");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -292,6 +308,7 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
 
 ssa_status_t ssa_select_tokens(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
                                int32_t* idx, void* ws, size_t ws_bytes, ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_select_tokens");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -315,6 +332,7 @@ ssa_status_t ssa_select_tokens(const ssa_dims_t* dims, const ssa_tensor_t* Q, co
 ssa_status_t ssa_fwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
                             const ssa_tensor_t* V, const int32_t* idx, const ssa_tensor_t* h_sparse,
                             float* lse_sel, ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_fwd_sparse");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -345,6 +363,7 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
                             const float* lse_sel, const ssa_tensor_t* g_sparse, const ssa_tensor_t* dQ,
                             const ssa_tensor_t* dK, const ssa_tensor_t* dV, void* ws, size_t ws_bytes,
                             ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_bwd_sparse");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -398,6 +417,7 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
 
 ssa_status_t ssa_decode_prefill(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
                                 int32_t t0, float* qsum, float* kbar, ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_decode_prefill");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -420,6 +440,7 @@ ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q, cons
                              const ssa_tensor_t* V, int32_t t, float* qsum, float* kbar,
                              const ssa_tensor_t* h, float* lse, int32_t* idx, void* ws, size_t ws_bytes,
                              ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_decode_step");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -450,6 +471,7 @@ ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q, cons
 ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,
                               const int32_t* idx, const float* lse_full, float* delta, void* ws,
                               size_t ws_bytes, ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_dropped_mass");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
@@ -476,6 +498,7 @@ ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, con
 ssa_status_t ssa_align_mse(const ssa_dims_t* dims, const ssa_tensor_t* h_full,
                            const ssa_tensor_t* h_sparse, float* loss, void* ws, size_t ws_bytes,
                            ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_align_mse");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);
