@@ -436,13 +436,20 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     # ---------------- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     row_flops = {"fwd_dual": F["fwd"], "bwd_dual": F["bwd"], "dropped_mass": F["dropped"]}
-    # bf16 with d = 128 and blocks of 64 / 128 runs on the tensor-core kernels;
-    # every other shape on the CUDA-core kernels (fp32 FMA bound)
+    # bf16 with d = 128 and blocks of 64 / 128 (per-block selection) runs on
+    # the tcgen05 kernels; other bf16 shapes on the warp-level mma.sync
+    # kernels; fp32 on the CUDA-core kernels (fp32 FMA bound)
     tc_path = w.dtype == "bf16" and w.d == 128 and w.block in (64, 128) and not args.per_token
+    mma_path = w.dtype == "bf16" and not tc_path
     if tc_path:
         scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_tc_kernel)",
                   "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_tc + finish + bwd_dkv_tc + bwd_dq_tc kernels",
                   "dropped_mass": "entry point ssa_dropped_mass = one kernel (dropped_tc_kernel)"}
+    elif mma_path:
+        scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_mma_kernel, mma.sync)",
+                  "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_mma + finish + bwd_dkv_mma + bwd_dq_mma "
+                              "(+ kvsum) kernels (mma.sync)",
+                  "dropped_mass": "entry point ssa_dropped_mass = one kernel (fwd_mma_kernel without V, mma.sync)"}
     else:
         scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_simt_kernel, CUDA cores)",
                   "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre + finish + bwd_dq + bwd_dkv kernels (CUDA cores)",
@@ -452,7 +459,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
 
     def roof(r):
         achieved = row_flops[r] / (row_ms[r] * 1e-3) / 1e12
-        if not tc_path:
+        if not (tc_path or mma_path):
             return {"bound": "alu", "kernel": r, "scope": scopes[r], "achieved": achieved, "peak": alu_peak,
                     "unit": "TFLOP/s", "frac": achieved / alu_peak, "traffic": None,
                     "peak_source": "fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz (attended FLOPs counted)"}
@@ -460,15 +467,16 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops_sustained"],
                 "frac_of_burst": achieved / peaks["bf16_tflops"],
-                "traffic": measured_traffic(r, w.name),
-                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); burst {peaks['bf16_tflops']}"}
+                "traffic": measured_traffic(r, w.name) if tc_path else None,
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); burst {peaks['bf16_tflops']}"
+                               + ("; warp-level mma.sync kernels (legacy tensor path)" if mma_path else "")}
 
     dom = max(row_flops, key=lambda r: row_ms[r])
     roofline = roof(dom)
     per_row = {r: {"ms": row_ms[r]} for r in rows}
     for r, f in row_flops.items():
         per_row[r]["attended_tflops"] = f / (row_ms[r] * 1e-3) / 1e12
-        if tc_path:
+        if tc_path or mma_path:
             per_row[r]["frac_of_sustained_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops_sustained"]
             per_row[r]["frac_of_burst_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops"]
         else:

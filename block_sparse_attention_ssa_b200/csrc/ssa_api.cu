@@ -91,7 +91,7 @@ ssa_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_E
 // ---------------------------------------------------------------- workspace
 struct Layout {
   size_t qbar, kbar;          // block scores
-  size_t dhf, doc, Df, Dc, mask, partials;  // backward
+  size_t dhf, doc, Df, Dc, mask, partials, kvpart;  // backward
   size_t lse;                 // dropped mass
   size_t bytes_scores, bytes_bwd, bytes_dropped, bytes_align, bytes_decode;
   int words, n_partials;
@@ -113,6 +113,8 @@ Layout layout(const Dims& D) {
   L.Dc = o; o = align_up(o + rows * 4);
   L.mask = o; o = align_up(o + (size_t)D.B * D.Hq * D.rows_sel * L.words * 4);
   L.partials = o; o = align_up(o + (size_t)L.n_partials * 4);
+  L.kvpart = o;
+  if (!bwd_tc_supported(D) && bwd_mma_supported(D)) o = align_up(o + bwd_mma_partial_bytes(D));
   L.bytes_bwd = o;
   L.lse = 0;
   L.bytes_dropped = align_up(rows * 4);
@@ -246,6 +248,7 @@ ssa_status_t ssa_fwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
     if (status == nullptr) return SSA_ERR_CUDA;
     return from_cuda(launch_fwd_tc(D, a, status, st));
   }
+  if (fwd_mma_supported(D)) return from_cuda(launch_fwd_mma(D, a, st));
   return from_cuda(launch_fwd_simt(D, a, st));
 }
 
@@ -301,6 +304,10 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
     if (status == nullptr) return SSA_ERR_CUDA;
     return from_cuda(launch_bwd_tc(D, a, status, st));
   }
+  if (bwd_mma_supported(D)) {
+    a.kvpart = at<float>(ws, L.kvpart);
+    return from_cuda(launch_bwd_mma(D, a, st));
+  }
   e = launch_bwd_pre(D, a, st);
   if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
   return from_cuda(e);
@@ -355,6 +362,7 @@ ssa_status_t ssa_fwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
     if (status == nullptr) return SSA_ERR_CUDA;
     return from_cuda(launch_fwd_tc(D, a, status, st));
   }
+  if (fwd_mma_supported(D)) return from_cuda(launch_fwd_mma(D, a, st));
   return from_cuda(launch_fwd_simt(D, a, st));
 }
 
@@ -409,6 +417,10 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
     int32_t* status = device_status_ptr();
     if (status == nullptr) return SSA_ERR_CUDA;
     return from_cuda(launch_bwd_tc(D, a, status, st));
+  }
+  if (bwd_mma_supported(D)) {
+    a.kvpart = at<float>(ws, L.kvpart);
+    return from_cuda(launch_bwd_mma(D, a, st));
   }
   e = launch_bwd_pre(D, a, st);
   if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
@@ -492,6 +504,7 @@ ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, con
     if (status == nullptr) return SSA_ERR_CUDA;
     return from_cuda(launch_dropped_tc(D, a, status, static_cast<cudaStream_t>(stream)));
   }
+  if (fwd_mma_supported(D)) return from_cuda(launch_dropped_mma(D, a, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_dropped_simt(D, a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -137,6 +137,12 @@ cudaError_t launch_dropped_simt(const Dims& D, const FwdArgs& a, cudaStream_t st
 // Tensor-core dropped mass (bf16, d = 128; same envelope as the forward).
 cudaError_t launch_dropped_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
 
+// Warp-level tensor-core (mma.sync) dual-stream forward and dropped mass:
+// bf16, d = 64 or 128, any block size and either selection mode.
+bool fwd_mma_supported(const Dims& D);
+cudaError_t launch_fwd_mma(const Dims& D, const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_dropped_mma(const Dims& D, const FwdArgs& a, cudaStream_t st);
+
 // Tensor-core (tcgen05 / TMEM / TMA) dual-stream forward, bf16, d = 128.
 // Returns cudaErrorNotSupported when the shape is outside its envelope.
 cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
@@ -166,6 +172,7 @@ struct BwdArgs {
   // gf = null and alpha = 0, so dh_f = 0 and r = 1; the kernels then skip
   // every (query block, key block) pair that is not selected.
   bool sparse_only;
+  float* kvpart;       // warp-level tensor-core backward: fp32 dK / dV partials (or null)
 };
 
 cudaError_t launch_bwd_pre(const Dims& D, const BwdArgs& a, cudaStream_t st);
@@ -173,6 +180,12 @@ cudaError_t launch_bwd_pre(const Dims& D, const BwdArgs& a, cudaStream_t st);
 bool bwd_tc_supported(const Dims& D);
 cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* dev_status, cudaStream_t st);
 cudaError_t launch_bwd_simt(const Dims& D, const BwdArgs& a, cudaStream_t st);
+// Warp-level tensor-core (mma.sync) backward: bf16, d = 64 or 128, any block
+// size and either selection mode (runs its own preprocess).
+bool bwd_mma_supported(const Dims& D);
+int bwd_mma_heads_per_cta(const Dims& D);
+size_t bwd_mma_partial_bytes(const Dims& D);  // workspace for a.kvpart (0: none needed)
+cudaError_t launch_bwd_mma(const Dims& D, const BwdArgs& a, cudaStream_t st);
 
 struct DecodeArgs {
   TensorRef q, k, v, h;  // q, h: [B,Hq,1,d] (prefill: q = the prompt's Q [B,Hq,N,d]); k, v: caches [B,Hkv,N,d]

@@ -125,15 +125,16 @@ def test_backward_dual_small_blocks(name, primary):
     assert float(grads["align_loss"].item()) == pytest.approx(l_align, rel=5e-2 if dt == "bf16" else 1e-4)
 
 
-def test_given_selection_mixed_tiles():
-    """Random selections at block 16 (rows without their diagonal block,
-    duplicates, padding): most 64 x 64 tiles mix selected and dropped pairs
-    inside a row and between rows."""
-    B, Hq, Hkv, N, d, s, k = 1, 4, 2, 512, 64, 16, 6
-    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 616, "f32")
+@pytest.mark.parametrize("s,d,dt", [(16, 64, "f32"), (16, 64, "bf16"), (32, 128, "bf16"), (16, 128, "bf16")])
+def test_given_selection_mixed_tiles(s, d, dt):
+    """Random selections at blocks of 16 and 32 (rows without their diagonal
+    block, duplicates, padding): most 64 x 64 tiles mix selected and dropped
+    pairs inside a row and between rows."""
+    B, Hq, Hkv, N, k = 1, 4, 2, 512, 6
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 616, dt)
     n = N // s
-    idx = custom_idx(B, Hq, n, k, seed=77, drop_diag_frac=0.3, pad_frac=0.2)
-    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "f32")
+    idx = custom_idx(B, Hq, n, k, seed=77 + s + d, drop_diag_frac=0.3, pad_frac=0.2)
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, dt)
     out = api.alloc_forward(dims)
     ws = api.alloc_workspace(dims)
     out["idx"] = torch.from_numpy(idx).cuda()
@@ -141,16 +142,50 @@ def test_given_selection_mixed_tiles():
                      out["lse_full"], out["lse_sel"], out["delta"])
     gf, gs = make_upstream((B, Hq, N, d), 61), make_upstream((B, Hq, N, d), 62)
     grads = api.alloc_backward(dims)
-    api.backward(dims, dev["Q"], dev["K"], dev["V"], out, upload(gf, "f32"), upload(gs, "f32"), 10.0, grads, ws)
+    api.backward(dims, dev["Q"], dev["K"], dev["V"], out, upload(gf, dt), upload(gs, dt), 10.0, grads, ws)
     torch.cuda.synchronize()
     assert api.ssa_device_status() == api.SSA_OK
     scale = 1 / math.sqrt(d)
-    dQ, dK, dV, _, ora = O.ssa_backward(host["Q"], host["K"], host["V"], idx, s, scale, gf.astype(np.float64),
-                                        gs.astype(np.float64), 10.0)
+    dQ, dK, dV, _, ora = O.ssa_backward(host["Q"], host["K"], host["V"], idx, s, scale,
+                                        oracle_view(gf, dt).astype(np.float64),
+                                        oracle_view(gs, dt).astype(np.float64), 10.0)
     for key in ("h_full", "h_sparse", "delta"):
-        assert np.abs(f64(out[key]) - ora[key]).max() <= TOL["f32"]["out"], key
+        assert np.abs(f64(out[key]) - ora[key]).max() <= TOL[dt]["out"], key
+    for key in ("lse_full", "lse_sel"):
+        fin = np.isfinite(ora[key])
+        got = f64(out[key])
+        assert np.array_equal(np.isfinite(got), fin), key
+        assert np.abs(got[fin] - ora[key][fin]).max() <= TOL[dt]["lse"], key
     for key, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
-        assert rel_l2(f64(got), ref) < TOL["f32"]["grad"], key
+        assert rel_l2(f64(got), ref) < TOL[dt]["grad"], key
+
+
+@pytest.mark.parametrize("s,d", [(16, 64), (32, 128)])
+def test_sparse_alone_never_reads_unselected_small_blocks(s, d):
+    """Blocks that no query selects hold NaN in K and V on the device while
+    their neighbours inside the same 64-key tile are selected: the sparse
+    stream alone must neither read nor weigh them."""
+    B, Hq, Hkv, N, k = 1, 4, 2, 1024, 5
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 929, "bf16")
+    n = N // s
+    idx = custom_idx(B, Hq, n, k, seed=5 + s)
+    poisoned = [1, 9, n // 2 + 1, n - 3]
+    for j in poisoned:
+        idx[idx == j] = -1
+        dev["K"][:, :, j * s:(j + 1) * s] = float("nan")
+        dev["V"][:, :, j * s:(j + 1) * s] = float("nan")
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
+    hs = torch.full((B, Hq, N, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device="cuda")
+    api.ssa_fwd_sparse(dims, dev["Q"], dev["K"], dev["V"], torch.from_numpy(idx).cuda(), hs, lse)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    assert torch.isfinite(hs.float()).all()
+    ora = O.forward_sparse(host["Q"], host["K"], host["V"], idx, s, 1 / math.sqrt(d))
+    assert np.abs(f64(hs) - ora["h_sparse"]).max() <= TOL["bf16"]["out"]
+    fin = np.isfinite(ora["lse_sel"])
+    assert np.array_equal(np.isfinite(f64(lse)), fin)
+    assert np.abs(f64(lse)[fin] - ora["lse_sel"][fin]).max() <= TOL["bf16"]["lse"]
 
 
 def test_decode_block16():
