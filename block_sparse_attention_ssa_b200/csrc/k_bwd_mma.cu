@@ -32,6 +32,8 @@
 // In the sparse-only mode (hf = hs, lse_full = lse_sel, no g_f, alpha = 0)
 // only selected pairs carry gradient, and both walks visit only the tiles
 // that hold one.
+#include <type_traits>
+
 #include "mma_sync.cuh"
 #include "ssa_internal.cuh"
 
@@ -259,27 +261,36 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
       cmr[i] = S.cm[rl[i]];
       dmr[i] = SPARSE ? 0ull : (causal & ~cmr[i]);
     }
-#pragma unroll
-    for (int ks = 0; ks < BN / NK; ++ks) {
+    const bool noneA = __all_sync(0xffffffffu, (cmr[0] | cmr[1]) == 0ull);
+    const bool allA = !diag && __all_sync(0xffffffffu, (cmr[0] & cmr[1]) == ~0ull);
+    // MODE 0: both sets in the sub-tile (element-wise routing); 1: every pair
+    // selected; 2: every pair dropped (both only off the diagonal).
+    auto step = [&](auto mode, int ks) {
+      constexpr int MODE = decltype(mode)::value;
+      if constexpr (SPARSE && MODE == 2) return;
       const int sh0 = ks * NK + 2 * q4;  // bit (n*8 + (e&1)) of the shifted masks: key of element (n, e)
-      unsigned long long inA[2], inD[2];
+      unsigned long long inA[2] = {0ull, 0ull}, inD[2] = {0ull, 0ull};
+      uint32_t fa = MODE == 1 ? (1u << NN) - 1u : 0u;  // bit n: the set has a pair in column group n
+      uint32_t fd = MODE == 2 ? (1u << NN) - 1u : 0u;
+      if constexpr (MODE == 0) {
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        inA[i] = cmr[i] >> sh0;
-        inD[i] = dmr[i] >> sh0;
-      }
-      uint32_t fa = 0, fd = 0;  // bit n: this thread has an element of the set in column group n
+        for (int i = 0; i < 2; ++i) {
+          inA[i] = cmr[i] >> sh0;
+          inD[i] = dmr[i] >> sh0;
+        }
 #pragma unroll
-      for (int n = 0; n < NN; ++n) {
-        if (((inA[0] | inA[1]) >> (n * 8)) & 3ull) fa |= 1u << n;
-        if (((inD[0] | inD[1]) >> (n * 8)) & 3ull) fd |= 1u << n;
+        for (int n = 0; n < NN; ++n) {
+          if (((inA[0] | inA[1]) >> (n * 8)) & 3ull) fa |= 1u << n;
+          if (((inD[0] | inD[1]) >> (n * 8)) & 3ull) fd |= 1u << n;
+        }
+        fa = warp_or(fa);
+        fd = warp_or(fd);
       }
-      fa = warp_or(fa);
-      fd = warp_or(fd);
       const uint32_t live = fa | fd;
-      if (live == 0u) continue;
+      if (live == 0u) return;
 
-      float sc[NN][4], dpc[NN][4], dpf[SPARSE ? 1 : NN][4];
+      float sc[NN][4], dpc[NN][4];
+      [[maybe_unused]] float dpf[SPARSE ? 1 : NN][4];
 #pragma unroll
       for (int n = 0; n < NN; ++n)
 #pragma unroll
@@ -292,7 +303,8 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t qa[4], oa[4], fa4[4];
+        uint32_t qa[4], oa[4];
+        [[maybe_unused]] uint32_t fa4[4];
         ldsm_x4(qa, &S.q[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
         if (fa) ldsm_x4(oa, &S.doc[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
         if constexpr (!SPARSE) {
@@ -325,8 +337,8 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = e >> 1, bit = n * 8 + (e & 1);
-          const bool isA = (inA[i] >> bit) & 1ull;
-          const bool isD = !SPARSE && ((inD[i] >> bit) & 1ull);
+          const bool isA = MODE == 1 || (MODE == 0 && ((inA[i] >> bit) & 1ull));
+          const bool isD = !SPARSE && (MODE == 2 || (MODE == 0 && ((inD[i] >> bit) & 1ull)));
           const float p = fast_ex2((isA || isD) ? fmaf(sc[n][e], sl2, -lse2[i]) : kNegInf);
           float dpd = 0.f;
           if constexpr (!SPARSE) dpd = dpf[n][e];
@@ -345,6 +357,14 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
           mma16816(dq[2 * j], da[kq], kb[0], kb[1]);
           mma16816(dq[2 * j + 1], da[kq], kb[2], kb[3]);
         }
+      }
+    };
+    if (!(SPARSE && noneA)) {
+#pragma unroll
+      for (int ks = 0; ks < BN / NK; ++ks) {
+        if (allA) step(std::integral_constant<int, 1>{}, ks);
+        else if (!SPARSE && noneA && !diag) step(std::integral_constant<int, 2>{}, ks);
+        else step(std::integral_constant<int, 0>{}, ks);
       }
     }
     __syncthreads();
@@ -433,19 +453,22 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
   // Steps are numbered hh * nq + (qt - kt).
   const int nsteps = sh.hpc * nq;
   auto next_step = [&](int from) -> int {
-    if constexpr (!SPARSE) return from < nsteps ? from : -1;
-    while (from < nsteps) {
-      const int hh = from / nq, x = from % nq;
-      uint32_t bits = S.tiles[hh * 128 + (x >> 5)] & (~0u << (x & 31));
-      if (bits) {
-        const int y = (x & ~31) + __ffs(bits) - 1;
-        if (y < nq) return hh * nq + y;
-        from = (hh + 1) * nq;
-      } else {
-        from = ((x | 31) + 1 < nq) ? hh * nq + (x | 31) + 1 : (hh + 1) * nq;
+    if constexpr (!SPARSE) {
+      return from < nsteps ? from : -1;
+    } else {
+      while (from < nsteps) {
+        const int hh = from / nq, x = from % nq;
+        uint32_t bits = S.tiles[hh * 128 + (x >> 5)] & (~0u << (x & 31));
+        if (bits) {
+          const int y = (x & ~31) + __ffs(bits) - 1;
+          if (y < nq) return hh * nq + y;
+          from = (hh + 1) * nq;
+        } else {
+          from = ((x | 31) + 1 < nq) ? hh * nq + (x | 31) + 1 : (hh + 1) * nq;
+        }
       }
+      return -1;
     }
-    return -1;
   };
   auto load_q = [&](int step, int buf) {
     const int hh = step / nq, qt = kt + step % nq;
@@ -477,7 +500,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
   const int g = lane >> 2, q4 = lane & 3;
   const int r0 = warp * 16;
   const int kl[2] = {r0 + g, r0 + g + 8};                        // this thread's keys in the tile
-  const int bpos[2] = {((u0 + kl[0]) / sh.s) & 31, ((u0 + kl[1]) / sh.s) & 31};
+  const int bp = ((u0 + r0) / sh.s) & 31;                         // their block's bit in a selection word
   const float sl2 = sh.scale * kLog2e;
   float dk[D / 8][4], dv[D / 8][4];
 #pragma unroll
@@ -495,38 +518,48 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
     __syncthreads();
     const bool diag = (step % nq) == 0;  // query tile == key tile
 
-#pragma unroll
-    for (int qs = 0; qs < BM / NQ; ++qs) {
+    // The warp's 16 keys lie in one key block (blocks have 16 keys or more):
+    // bit bp of a query row's selection word says whether that row selected it.
+    const bool sel0 = (S.word[buf][lane] >> bp) & 1u, sel1 = (S.word[buf][lane + 32] >> bp) & 1u;
+    const bool noneA = __all_sync(0xffffffffu, !sel0 && !sel1);
+    const bool allA = !diag && __all_sync(0xffffffffu, sel0 && sel1);
+    // MODE 0: both sets (element-wise routing); 1: every pair selected;
+    // 2: every pair dropped (both only off the diagonal).
+    auto step_q = [&](auto mode, int qs) {
+      constexpr int MODE = decltype(mode)::value;
+      if constexpr (SPARSE && MODE == 2) return;
       const int qb = qs * NQ;
       // Element (n, e): key kl[e >> 1], query qb + n*8 + 2*q4 + (e & 1).
       uint32_t mA = 0, mD = 0;  // bit n*4 + e
+      uint32_t fa = MODE == 1 ? (1u << NN) - 1u : 0u, fd = MODE == 2 ? (1u << NN) - 1u : 0u;
+      if constexpr (MODE == 0) {
 #pragma unroll
-      for (int n = 0; n < NN; ++n)
+        for (int n = 0; n < NN; ++n)
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          const int c = qb + n * 8 + 2 * q4 + c2;
-          const uint32_t wd = S.word[buf][c];
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int c = qb + n * 8 + 2 * q4 + c2;
+            const bool sel = (S.word[buf][c] >> bp) & 1u;
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const bool causal = !diag || kl[i] <= c;
-            const bool isA = causal && ((wd >> bpos[i]) & 1u);
-            const int e = 2 * i + c2;
-            if (isA) mA |= 1u << (n * 4 + e);
-            if (!SPARSE && causal && !isA) mD |= 1u << (n * 4 + e);
+            for (int i = 0; i < 2; ++i) {
+              const bool causal = !diag || kl[i] <= c;
+              const int e = 2 * i + c2;
+              if (causal && sel) mA |= 1u << (n * 4 + e);
+              if (!SPARSE && causal && !sel) mD |= 1u << (n * 4 + e);
+            }
           }
-        }
-      uint32_t fa = 0, fd = 0;
 #pragma unroll
-      for (int n = 0; n < NN; ++n) {
-        if ((mA >> (n * 4)) & 15u) fa |= 1u << n;
-        if ((mD >> (n * 4)) & 15u) fd |= 1u << n;
+        for (int n = 0; n < NN; ++n) {
+          if ((mA >> (n * 4)) & 15u) fa |= 1u << n;
+          if ((mD >> (n * 4)) & 15u) fd |= 1u << n;
+        }
+        fa = warp_or(fa);
+        fd = warp_or(fd);
       }
-      fa = warp_or(fa);
-      fd = warp_or(fd);
       const uint32_t live = fa | fd;
-      if (live == 0u) continue;
+      if (live == 0u) return;
 
-      float sc[NN][4], dpc[NN][4], dpf[SPARSE ? 1 : NN][4];
+      float sc[NN][4], dpc[NN][4];
+      [[maybe_unused]] float dpf[SPARSE ? 1 : NN][4];
 #pragma unroll
       for (int n = 0; n < NN; ++n)
 #pragma unroll
@@ -547,7 +580,8 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
           if (((live >> (2 * j)) & 3u) == 0u) continue;
           const int qrow = qb + j * 16 + (lane & 7) + ((lane >> 4) << 3);
           const int qcol = kk * 16 + ((lane >> 3) & 1) * 8;
-          uint32_t qf[4], of[4], ff[4];
+          uint32_t qf[4], of[4];
+          [[maybe_unused]] uint32_t ff[4];
           ldsm_x4(qf, &S.q[buf][qrow][qcol]);
           if ((fa >> (2 * j)) & 3u) ldsm_x4(of, &S.doc[buf][qrow][qcol]);
           if constexpr (!SPARSE) {
@@ -565,15 +599,16 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
         }
       }
       // P^T and dS^T in registers, packed as A operands over 16-query steps.
-      uint32_t pA[NN / 2][4], pD[SPARSE ? 1 : NN / 2][4], dS[NN / 2][4];
+      uint32_t pA[NN / 2][4], dS[NN / 2][4];
+      [[maybe_unused]] uint32_t pD[SPARSE ? 1 : NN / 2][4];
 #pragma unroll
       for (int n = 0; n < NN; ++n) {
         float wA[4], wD[4], ds[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c = qb + n * 8 + 2 * q4 + (e & 1);
-          const bool isA = (mA >> (n * 4 + e)) & 1u;
-          const bool isD = !SPARSE && ((mD >> (n * 4 + e)) & 1u);
+          const bool isA = MODE == 1 || (MODE == 0 && ((mA >> (n * 4 + e)) & 1u));
+          const bool isD = !SPARSE && (MODE == 2 || (MODE == 0 && ((mD >> (n * 4 + e)) & 1u)));
           const float p = fast_ex2((isA || isD) ? fmaf(sc[n][e], sl2, -S.lse[buf][c] * kLog2e) : kNegInf);
           float dpd = 0.f;
           if constexpr (!SPARSE) dpd = dpf[n][e];
@@ -596,7 +631,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
         const bool useL = (live >> (2 * kq)) & 3u;
         if (!useL) continue;
         const bool useA = (fa >> (2 * kq)) & 3u;
-        const bool useD = !SPARSE && ((fd >> (2 * kq)) & 3u);
+        [[maybe_unused]] const bool useD = !SPARSE && ((fd >> (2 * kq)) & 3u);
         const int qrow = qb + kq * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
         for (int j = 0; j < D / 16; ++j) {
@@ -620,6 +655,14 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
             }
           }
         }
+      }
+    };
+    if (!(SPARSE && noneA)) {
+#pragma unroll
+      for (int qs = 0; qs < BM / NQ; ++qs) {
+        if (allA) step_q(std::integral_constant<int, 1>{}, qs);
+        else if (!SPARSE && noneA && !diag) step_q(std::integral_constant<int, 2>{}, qs);
+        else step_q(std::integral_constant<int, 0>{}, qs);
       }
     }
     __syncthreads();

@@ -155,126 +155,190 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a,
     cp_async_wait<1>();
     __syncthreads();
 
-    float sc[8][4];
-#pragma unroll
-    for (int n = 0; n < 8; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sc[n][e] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t qa[4];
-      ldsm_x4(qa, &S.q[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t kb[4];
-        ldsm_x4(kb, &S.k[buf][j * 16 + (lane & 7) + ((lane >> 4) << 3)][kk * 16 + ((lane >> 3) & 1) * 8]);
-        mma16816(sc[2 * j], qa, kb[0], kb[1]);
-        mma16816(sc[2 * j + 1], qa, kb[2], kb[3]);
-      }
-    }
-
-    // Set membership of this thread's logits: bit nt*8 + (e & 1) of the
-    // row's masks shifted by 2*q4 is the key of sc[nt][e].
     const bool diag = (u0 == t0);
-    unsigned long long inA[2], inD[2];
+    const unsigned long long cm0 = S.cm[rl[0]], cm1 = S.cm[rl[1]];
+    // Warp-uniform shortcuts: none of the warp's pairs in this tile is
+    // selected, or (off the diagonal) all of them are.
+    const bool noneA = __all_sync(0xffffffffu, (cm0 | cm1) == 0ull);
+    const bool allA = !diag && __all_sync(0xffffffffu, (cm0 & cm1) == ~0ull);
+    // One set holds every logit of the warp: a plain online-softmax step.
+    auto uniform = [&](auto& o, float (&m)[2], float (&l)[2], const float (&sc)[8][4]) {
+      float mx[2] = {kNegInf, kNegInf}, c[2];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const unsigned long long causal = diag ? (2ull << rl[i]) - 1ull : ~0ull;  // rl <= 63
-      const unsigned long long cm = S.cm[rl[i]];
-      inA[i] = cm >> (2 * q4);
-      inD[i] = (causal & ~cm) >> (2 * q4);
-    }
-    float mxA[2] = {kNegInf, kNegInf}, mxD[2] = {kNegInf, kNegInf};
+      for (int n = 0; n < 8; ++n)
 #pragma unroll
-    for (int n = 0; n < 8; ++n)
+        for (int e = 0; e < 4; ++e) mx[e >> 1] = fmaxf(mx[e >> 1], sc[n][e]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = e >> 1, bit = n * 8 + (e & 1);
-        const float x = sc[n][e] * sl2;
-        sc[n][e] = x;
-        if ((inA[i] >> bit) & 1ull) mxA[i] = fmaxf(mxA[i], x);
-        if (!SPARSE && ((inD[i] >> bit) & 1ull)) mxD[i] = fmaxf(mxD[i], x);
+      for (int i = 0; i < 2; ++i) {
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+        const float nm = fmaxf(m[i], mx[i] * sl2);
+        c[i] = fast_ex2(m[i] - nm);
+        m[i] = nm;
+        l[i] *= c[i];
       }
-    float bA[2], bD[2], cA[2], cD[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      mxA[i] = fmaxf(mxA[i], __shfl_xor_sync(0xffffffffu, mxA[i], 1));
-      mxA[i] = fmaxf(mxA[i], __shfl_xor_sync(0xffffffffu, mxA[i], 2));
-      const float nA = fmaxf(mA[i], mxA[i]);
-      bA[i] = (nA == kNegInf) ? 0.f : nA;
-      cA[i] = fast_ex2(mA[i] - bA[i]);
-      mA[i] = nA;
-      lA[i] *= cA[i];
-      if (!SPARSE) {
-        mxD[i] = fmaxf(mxD[i], __shfl_xor_sync(0xffffffffu, mxD[i], 1));
-        mxD[i] = fmaxf(mxD[i], __shfl_xor_sync(0xffffffffu, mxD[i], 2));
-        const float nD = fmaxf(mD[i], mxD[i]);
-        bD[i] = (nD == kNegInf) ? 0.f : nD;
-        cD[i] = fast_ex2(mD[i] - bD[i]);
-        mD[i] = nD;
-        lD[i] *= cD[i];
-      }
-    }
-    if (WITH_V) {
-      if (__any_sync(0xffffffffu, cA[0] != 1.f || cA[1] != 1.f)) {
+      if (WITH_V && __any_sync(0xffffffffu, c[0] != 1.f || c[1] != 1.f)) {
 #pragma unroll
         for (int n = 0; n < D / 8; ++n) {
-          oA[n][0] *= cA[0]; oA[n][1] *= cA[0];
-          oA[n][2] *= cA[1]; oA[n][3] *= cA[1];
+          o[n][0] *= c[0]; o[n][1] *= c[0];
+          o[n][2] *= c[1]; o[n][3] *= c[1];
         }
       }
-      if constexpr (!SPARSE) {
-        if (__any_sync(0xffffffffu, cD[0] != 1.f || cD[1] != 1.f)) {
 #pragma unroll
-          for (int n = 0; n < ND; ++n) {
-            oD[n][0] *= cD[0]; oD[n][1] *= cD[0];
-            oD[n][2] *= cD[1]; oD[n][3] *= cD[1];
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t pa[4];
+#pragma unroll
+        for (int hn = 0; hn < 2; ++hn) {
+          float w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            w[e] = fast_ex2(fmaf(sc[2 * kk + hn][e], sl2, -m[e >> 1]));
+            l[e >> 1] += w[e];
+          }
+          pa[hn * 2] = pack2(w[0], w[1]);
+          pa[hn * 2 + 1] = pack2(w[2], w[3]);
+        }
+        if (WITH_V) {
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j) {
+            uint32_t vb[4];
+            ldsm_x4_t(vb, &S.v[buf][kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8][j * 16 + (lane >> 4) * 8]);
+            mma16816(o[2 * j], pa, vb[0], vb[1]);
+            mma16816(o[2 * j + 1], pa, vb[2], vb[3]);
           }
         }
       }
-    }
-    // Per 16-key step: the weights (one exponential per logit) packed as the
-    // A operand, then P V for each set that has a weight in the step.
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t pa[4], pd[4];
-#pragma unroll
-      for (int hn = 0; hn < 2; ++hn) {
-        const int n = 2 * kk + hn;
-        float wA[4], wD[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = e >> 1, bit = n * 8 + (e & 1);
-          const bool isA = (inA[i] >> bit) & 1ull;
-          const bool isD = !SPARSE && ((inD[i] >> bit) & 1ull);
-          const float p = fast_ex2(isA ? sc[n][e] - bA[i] : (isD ? sc[n][e] - bD[i] : kNegInf));
-          wA[e] = isA ? p : 0.f;
-          wD[e] = isA ? 0.f : p;
-          lA[i] += wA[e];
-          lD[i] += wD[e];
+    };
+
+    if (!(SPARSE && noneA)) {  // the sparse stream has nothing of this tile for the warp
+      float sc[8][4];
+  #pragma unroll
+      for (int n = 0; n < 8; ++n)
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) sc[n][e] = 0.f;
+  #pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t qa[4];
+        ldsm_x4(qa, &S.q[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+  #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t kb[4];
+          ldsm_x4(kb, &S.k[buf][j * 16 + (lane & 7) + ((lane >> 4) << 3)][kk * 16 + ((lane >> 3) & 1) * 8]);
+          mma16816(sc[2 * j], qa, kb[0], kb[1]);
+          mma16816(sc[2 * j + 1], qa, kb[2], kb[3]);
         }
-        pa[hn * 2] = pack2(wA[0], wA[1]);
-        pa[hn * 2 + 1] = pack2(wA[2], wA[3]);
-        pd[hn * 2] = pack2(wD[0], wD[1]);
-        pd[hn * 2 + 1] = pack2(wD[2], wD[3]);
       }
-      if (WITH_V) {
-        const unsigned long long stepbits = 0x303ull << (16 * kk);
-        const bool useA = __any_sync(0xffffffffu, ((inA[0] | inA[1]) & stepbits) != 0ull);
-        const bool useD = !SPARSE && __any_sync(0xffffffffu, ((inD[0] | inD[1]) & stepbits) != 0ull);
-        if (!useA && !useD) continue;
-#pragma unroll
-        for (int j = 0; j < D / 16; ++j) {
-          uint32_t vb[4];
-          ldsm_x4_t(vb, &S.v[buf][kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8][j * 16 + (lane >> 4) * 8]);
-          if (useA) {
-            mma16816(oA[2 * j], pa, vb[0], vb[1]);
-            mma16816(oA[2 * j + 1], pa, vb[2], vb[3]);
+
+      if (!diag && (allA || noneA)) {
+        if (allA) {
+          uniform(oA, mA, lA, sc);
+        } else {
+          if constexpr (!SPARSE) uniform(oD, mD, lD, sc);
+        }
+      } else {
+        // Set membership of this thread's logits: bit nt*8 + (e & 1) of the
+        // row's masks shifted by 2*q4 is the key of sc[nt][e].
+        unsigned long long inA[2], inD[2];
+    #pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const unsigned long long causal = diag ? (2ull << rl[i]) - 1ull : ~0ull;  // rl <= 63
+          const unsigned long long cm = i ? cm1 : cm0;
+          inA[i] = cm >> (2 * q4);
+          inD[i] = (causal & ~cm) >> (2 * q4);
+        }
+        float mxA[2] = {kNegInf, kNegInf}, mxD[2] = {kNegInf, kNegInf};
+    #pragma unroll
+        for (int n = 0; n < 8; ++n)
+    #pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = e >> 1, bit = n * 8 + (e & 1);
+            const float x = sc[n][e] * sl2;
+            sc[n][e] = x;
+            if ((inA[i] >> bit) & 1ull) mxA[i] = fmaxf(mxA[i], x);
+            if (!SPARSE && ((inD[i] >> bit) & 1ull)) mxD[i] = fmaxf(mxD[i], x);
+          }
+        float bA[2], bD[2], cA[2], cD[2];
+    #pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          mxA[i] = fmaxf(mxA[i], __shfl_xor_sync(0xffffffffu, mxA[i], 1));
+          mxA[i] = fmaxf(mxA[i], __shfl_xor_sync(0xffffffffu, mxA[i], 2));
+          const float nA = fmaxf(mA[i], mxA[i]);
+          bA[i] = (nA == kNegInf) ? 0.f : nA;
+          cA[i] = fast_ex2(mA[i] - bA[i]);
+          mA[i] = nA;
+          lA[i] *= cA[i];
+          if (!SPARSE) {
+            mxD[i] = fmaxf(mxD[i], __shfl_xor_sync(0xffffffffu, mxD[i], 1));
+            mxD[i] = fmaxf(mxD[i], __shfl_xor_sync(0xffffffffu, mxD[i], 2));
+            const float nD = fmaxf(mD[i], mxD[i]);
+            bD[i] = (nD == kNegInf) ? 0.f : nD;
+            cD[i] = fast_ex2(mD[i] - bD[i]);
+            mD[i] = nD;
+            lD[i] *= cD[i];
+          }
+        }
+        if (WITH_V) {
+          if (__any_sync(0xffffffffu, cA[0] != 1.f || cA[1] != 1.f)) {
+    #pragma unroll
+            for (int n = 0; n < D / 8; ++n) {
+              oA[n][0] *= cA[0]; oA[n][1] *= cA[0];
+              oA[n][2] *= cA[1]; oA[n][3] *= cA[1];
+            }
           }
           if constexpr (!SPARSE) {
-            if (useD) {
-              mma16816(oD[2 * j], pd, vb[0], vb[1]);
-              mma16816(oD[2 * j + 1], pd, vb[2], vb[3]);
+            if (__any_sync(0xffffffffu, cD[0] != 1.f || cD[1] != 1.f)) {
+    #pragma unroll
+              for (int n = 0; n < ND; ++n) {
+                oD[n][0] *= cD[0]; oD[n][1] *= cD[0];
+                oD[n][2] *= cD[1]; oD[n][3] *= cD[1];
+              }
+            }
+          }
+        }
+        // Per 16-key step: the weights (one exponential per logit) packed as the
+        // A operand, then P V for each set that has a weight in the step.
+    #pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t pa[4], pd[4];
+    #pragma unroll
+          for (int hn = 0; hn < 2; ++hn) {
+            const int n = 2 * kk + hn;
+            float wA[4], wD[4];
+    #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = e >> 1, bit = n * 8 + (e & 1);
+              const bool isA = (inA[i] >> bit) & 1ull;
+              const bool isD = !SPARSE && ((inD[i] >> bit) & 1ull);
+              const float p = fast_ex2(isA ? sc[n][e] - bA[i] : (isD ? sc[n][e] - bD[i] : kNegInf));
+              wA[e] = isA ? p : 0.f;
+              wD[e] = isA ? 0.f : p;
+              lA[i] += wA[e];
+              lD[i] += wD[e];
+            }
+            pa[hn * 2] = pack2(wA[0], wA[1]);
+            pa[hn * 2 + 1] = pack2(wA[2], wA[3]);
+            pd[hn * 2] = pack2(wD[0], wD[1]);
+            pd[hn * 2 + 1] = pack2(wD[2], wD[3]);
+          }
+          if (WITH_V) {
+            const unsigned long long stepbits = 0x303ull << (16 * kk);
+            const bool useA = __any_sync(0xffffffffu, ((inA[0] | inA[1]) & stepbits) != 0ull);
+            const bool useD = !SPARSE && __any_sync(0xffffffffu, ((inD[0] | inD[1]) & stepbits) != 0ull);
+            if (!useA && !useD) continue;
+    #pragma unroll
+            for (int j = 0; j < D / 16; ++j) {
+              uint32_t vb[4];
+              ldsm_x4_t(vb, &S.v[buf][kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8][j * 16 + (lane >> 4) * 8]);
+              if (useA) {
+                mma16816(oA[2 * j], pa, vb[0], vb[1]);
+                mma16816(oA[2 * j + 1], pa, vb[2], vb[3]);
+              }
+              if constexpr (!SPARSE) {
+                if (useD) {
+                  mma16816(oD[2 * j], pd, vb[0], vb[1]);
+                  mma16816(oD[2 * j + 1], pd, vb[2], vb[3]);
+                }
+              }
             }
           }
         }
