@@ -495,15 +495,20 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     # after the step; not part of `value`.  Attended FLOPs count the selected
     # causal pairs only: forward 4 d sum|A_t|, backward 10 d sum|A_t|.
     if not args.no_sparse:
-        idx_np = out["idx"].cpu().numpy()
-        n_ = w.n_blocks
-        i_ax = np.arange(n_).reshape(1, 1, n_, 1)
-        sel = np.zeros(idx_np.shape[:3] + (n_,), dtype=bool)
-        valid = (idx_np >= 0) & (idx_np <= i_ax)
-        bb, hh, ii, kk = np.nonzero(valid)
-        sel[bb, hh, ii, idx_np[bb, hh, ii, kk]] = True
-        diag = np.eye(n_, dtype=bool)[None, None]
-        pairs_sel = int((sel & ~diag).sum()) * w.block * w.block + int((sel & diag).sum()) * w.block * (w.block + 1) // 2
+        # distinct causal selected blocks per selection row (a query block, or
+        # a token with per-token selection), each counted with its causal keys
+        srt = np.sort(out["idx"].cpu().numpy().astype(np.int64), axis=-1)
+        dup = np.zeros(srt.shape, dtype=bool)
+        dup[..., 1:] = srt[..., 1:] == srt[..., :-1]
+        rows_ax = np.arange(srt.shape[2], dtype=np.int64).reshape(1, 1, -1, 1)
+        s_ = w.block
+        i_ax = rows_ax // s_ if args.per_token else rows_ax
+        valid = (srt >= 0) & (srt <= i_ax) & ~dup
+        if args.per_token:
+            cnt = np.where(srt < i_ax, s_, rows_ax - i_ax * s_ + 1)
+        else:
+            cnt = np.where(srt < i_ax, s_ * s_, s_ * (s_ + 1) // 2)
+        pairs_sel = int((cnt * valid).sum())
         hs2 = torch.empty_like(out["h_sparse"])
         lse2 = torch.empty_like(out["lse_sel"])
 

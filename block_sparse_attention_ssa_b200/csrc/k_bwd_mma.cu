@@ -53,6 +53,7 @@ struct MmaShape {
   int Hq, g, N, s, n, k;
   float scale;
   int per_token;
+  int ls;     // log2 of the block size
   int words;  // 32-bit words per selection row
   int hpc;    // query heads per dK/dV CTA
 };
@@ -143,19 +144,23 @@ struct DqSmem {
   bf16 dhf[SPARSE ? 1 : BM][LD];
   bf16 k[2][BN][LD];
   bf16 v[2][BN][LD];
-  uint32_t sel[BM][64];             // selection rows of the tile (per query block or per row)
   unsigned long long cm[BM];        // per row: selected causal keys of the current key tile
   uint32_t uni[64];
   uint32_t tiles[128];              // bit kt: key tile kt is visited
+  // followed by the tile's selection rows, 64 words each (one per query
+  // block of the tile, or per query row with per-token selection)
 };
 
+__host__ __device__ inline int sel_rows(int per_token, int s) { return per_token ? BM : (s >= BM ? 1 : BM / s); }
+
 template <int D, bool SPARSE>
-__global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
+__global__ void __launch_bounds__(NT, D == 64 ? 3 : 1)
     bwd_dq_mma_kernel(BwdArgs a, MmaShape sh, const bf16* __restrict__ dhf, const bf16* __restrict__ doc) {
-  constexpr int NK = D == 64 ? 64 : 32;  // keys per register sub-tile
+  constexpr int NK = 32;  // keys per register sub-tile
   constexpr int NN = NK / 8;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   DqSmem<D, SPARSE>& S = *reinterpret_cast<DqSmem<D, SPARSE>*>(smem_raw);
+  uint32_t (*sel)[64] = reinterpret_cast<uint32_t (*)[64]>(smem_raw + sizeof(DqSmem<D, SPARSE>));
   const int qt = gridDim.x - 1 - blockIdx.x;  // the longest rows first
   const int h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / sh.g;
@@ -173,7 +178,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
     cp_async16(&S.doc[r][c], doc + (rbase + r) * D + c, 16);
     if (!SPARSE) cp_async16(&S.dhf[r][c], dhf + (rbase + r) * D + c, 16);
   }
-  for (int w = tid; w < nsel * 64; w += NT) (&S.sel[0][0])[w] = 0u;
+  for (int w = tid; w < nsel * 64; w += NT) (&sel[0][0])[w] = 0u;
   if (tid < 64) S.uni[tid] = 0u;
   S.tiles[tid] = 0u;
   __syncthreads();
@@ -181,7 +186,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
     const int r = e / sh.words, wi = e % sh.words;
     const int64_t mrow = sh.per_token ? (int64_t)t0 + r : (int64_t)ib0 + r;
     const uint32_t v = a.mask[(((int64_t)b * sh.Hq + h) * rph + mrow) * sh.words + wi];
-    S.sel[r][wi] = v;
+    sel[r][wi] = v;
     if (SPARSE && v) atomicOr(&S.uni[wi], v);
   }
   __syncthreads();
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
       const int r = e / (D / 8), c = (e % (D / 8)) * 8;
       int bytes = 16;
       if (SPARSE && sh.s < BN) {
-        const int j = (u0 + r) / sh.s;
+        const int j = (u0 + r) >> sh.ls;
         bytes = ((S.uni[j >> 5] >> (j & 31)) & 1u) ? 16 : 0;
       }
       cp_async16(&S.k[buf][r][c], row_ptr<bf16>(a.k, b, kvh, u0 + r) + c, bytes);
@@ -247,8 +252,8 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
     cp_async_commit();
     const int u0 = kt * BN;
     if (tid < BM) {
-      const int rs = sh.per_token ? tid : (t0 + tid) / sh.s - ib0;
-      S.cm[tid] = tile_keep_mask(S.sel[rs], u0, sh.s) & causal_mask(t0 + tid, u0);
+      const int rs = sh.per_token ? tid : ((t0 + tid) >> sh.ls) - ib0;
+      S.cm[tid] = tile_keep_mask_p2(sel[rs], u0, sh.ls) & causal_mask(t0 + tid, u0);
     }
     cp_async_wait<1>();
     __syncthreads();
@@ -403,10 +408,10 @@ struct DkvSmem {
 };
 
 template <int D, bool SPARSE>
-__global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
+__global__ void __launch_bounds__(NT, D == 64 ? 3 : 1)
     bwd_dkv_mma_kernel(BwdArgs a, MmaShape sh, const bf16* __restrict__ dhf, const bf16* __restrict__ doc,
                        float* __restrict__ part) {
-  constexpr int NQ = D == 64 ? 64 : 32;  // queries per register sub-tile
+  constexpr int NQ = 32;  // queries per register sub-tile
   constexpr int NN = NQ / 8;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   DkvSmem<D, SPARSE>& S = *reinterpret_cast<DkvSmem<D, SPARSE>*>(smem_raw);
@@ -488,7 +493,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
       cp_async16(dst + c, src + rbase + c, 16);
     } else if (tid >= 64) {
       const int r = tid - 64;
-      const int64_t mrow = sh.per_token ? (int64_t)t0 + r : (int64_t)(t0 + r) / sh.s;
+      const int64_t mrow = sh.per_token ? (int64_t)t0 + r : (int64_t)((t0 + r) >> sh.ls);
       cp_async4(&S.word[buf][r], a.mask + (((int64_t)b * sh.Hq + h) * rph + mrow) * sh.words + wi);
     }
   };
@@ -729,11 +734,13 @@ __global__ void __launch_bounds__(256) kvsum_kernel(const float* __restrict__ pa
 
 template <int D, bool SPARSE>
 cudaError_t bwd_t(const Dims& Dm, const BwdArgs& a, const bf16* dhf, const bf16* doc, cudaStream_t st) {
-  MmaShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale, Dm.per_token, a.words, bwd_mma_heads_per_cta(Dm)};
+  MmaShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale, Dm.per_token, __builtin_ctz((unsigned)Dm.s),
+              a.words, bwd_mma_heads_per_cta(Dm)};
   const int chunks = Dm.g / sh.hpc;
   auto kdq = bwd_dq_mma_kernel<D, SPARSE>;
   auto kkv = bwd_dkv_mma_kernel<D, SPARSE>;
-  const size_t sq = sizeof(DqSmem<D, SPARSE>), skv = sizeof(DkvSmem<D, SPARSE>);
+  const size_t sq = sizeof(DqSmem<D, SPARSE>) + (size_t)sel_rows(Dm.per_token, Dm.s) * 64 * sizeof(uint32_t);
+  const size_t skv = sizeof(DkvSmem<D, SPARSE>);
   cudaError_t e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sq);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)skv);

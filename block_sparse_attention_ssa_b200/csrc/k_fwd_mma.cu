@@ -41,6 +41,7 @@ struct MmaShape {
   int Hq, g, N, s, n, k;
   float scale;
   int per_token;
+  int ls;  // log2 of the block size
 };
 
 template <int D>
@@ -49,16 +50,21 @@ struct Smem {
   bf16 q[BM][LD];                   // Q tile; each warp's 16 rows double as its output staging
   bf16 k[2][BN][LD];
   bf16 v[2][BN][LD];
-  uint32_t sel[BM][64];             // selected-block bit sets: per query block of the tile, or per row
   unsigned long long cm[BM];        // per row: kept keys of the current tile (selected and causal)
   uint32_t uni[64];                 // union of the tile's selection rows
   uint32_t tiles[128];              // bit kt set: key tile kt is visited
+  // followed by the selected-block bit sets, 64 words per selection row: one
+  // row per query block of the tile, or (per-token selection) per query row
 };
+
+// Selection rows a CTA holds.
+__host__ __device__ inline int sel_rows(int per_token, int s) { return per_token ? BM : (s >= BM ? 1 : BM / s); }
 
 template <int D, bool WITH_V, bool SPARSE>
 __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a, MmaShape sh) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Smem<D>& S = *reinterpret_cast<Smem<D>*>(smem_raw);
+  uint32_t (*sel)[64] = reinterpret_cast<uint32_t (*)[64]>(smem_raw + sizeof(Smem<D>));
   const int qt = gridDim.x - 1 - blockIdx.x;  // the longest rows first
   const int h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / sh.g;
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a,
     const int r = e / (D / 8), c = (e % (D / 8)) * 8;
     cp_async16(&S.q[r][c], row_ptr<bf16>(a.q, b, h, t0 + r) + c, 16);
   }
-  for (int w = tid; w < nsel * 64; w += NT) (&S.sel[0][0])[w] = 0u;
+  for (int w = tid; w < nsel * 64; w += NT) (&sel[0][0])[w] = 0u;
   if (tid < 64) S.uni[tid] = 0u;
   S.tiles[tid] = 0u;
   __syncthreads();
@@ -82,7 +88,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a,
     const int iblk = sh.per_token ? (t0 + r) / sh.s : ib0 + r;
     const int j = a.idx[(((int64_t)b * sh.Hq + h) * (sh.per_token ? sh.N : sh.n) + srow) * sh.k + e % sh.k];
     if (j >= 0 && j <= iblk) {
-      atomicOr(&S.sel[r][j >> 5], 1u << (j & 31));
+      atomicOr(&sel[r][j >> 5], 1u << (j & 31));
       if (SPARSE) atomicOr(&S.uni[j >> 5], 1u << (j & 31));
     }
   }
@@ -112,7 +118,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a,
       const int r = e / (D / 8), c = (e % (D / 8)) * 8;
       int bytes = 16;
       if (SPARSE && sh.s < BN) {
-        const int j = (u0 + r) / sh.s;
+        const int j = (u0 + r) >> sh.ls;
         bytes = ((S.uni[j >> 5] >> (j & 31)) & 1u) ? 16 : 0;
       }
       cp_async16(&S.k[buf][r][c], row_ptr<bf16>(a.k, b, kvh, u0 + r) + c, bytes);
@@ -149,8 +155,8 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a,
     cp_async_commit();
     const int u0 = kt * BN;
     if (tid < BM) {
-      const int rs = sh.per_token ? tid : (t0 + tid) / sh.s - ib0;
-      S.cm[tid] = tile_keep_mask(S.sel[rs], u0, sh.s) & causal_mask(t0 + tid, u0);
+      const int rs = sh.per_token ? tid : ((t0 + tid) >> sh.ls) - ib0;
+      S.cm[tid] = tile_keep_mask_p2(sel[rs], u0, sh.ls) & causal_mask(t0 + tid, u0);
     }
     cp_async_wait<1>();
     __syncthreads();
@@ -163,11 +169,22 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a,
     const bool allA = !diag && __all_sync(0xffffffffu, (cm0 & cm1) == ~0ull);
     // One set holds every logit of the warp: a plain online-softmax step.
     auto uniform = [&](auto& o, float (&m)[2], float (&l)[2], const float (&sc)[8][4]) {
-      float mx[2] = {kNegInf, kNegInf}, c[2];
+      // row maxima as balanced trees (short dependency chains)
+      float t0[8], t1[8], mx[2], c[2];
 #pragma unroll
-      for (int n = 0; n < 8; ++n)
+      for (int n = 0; n < 8; ++n) {
+        t0[n] = fmaxf(sc[n][0], sc[n][1]);
+        t1[n] = fmaxf(sc[n][2], sc[n][3]);
+      }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mx[e >> 1] = fmaxf(mx[e >> 1], sc[n][e]);
+      for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int n = 0; n < w; ++n) {
+          t0[n] = fmaxf(t0[n], t0[n + w]);
+          t1[n] = fmaxf(t1[n], t1[n + w]);
+        }
+      mx[0] = t0[0];
+      mx[1] = t1[0];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
@@ -187,17 +204,16 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a,
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         uint32_t pa[4];
+        float w[2][4];
 #pragma unroll
         for (int hn = 0; hn < 2; ++hn) {
-          float w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            w[e] = fast_ex2(fmaf(sc[2 * kk + hn][e], sl2, -m[e >> 1]));
-            l[e >> 1] += w[e];
-          }
-          pa[hn * 2] = pack2(w[0], w[1]);
-          pa[hn * 2 + 1] = pack2(w[2], w[3]);
+          for (int e = 0; e < 4; ++e) w[hn][e] = fast_ex2(fmaf(sc[2 * kk + hn][e], sl2, -m[e >> 1]));
+          pa[hn * 2] = pack2(w[hn][0], w[hn][1]);
+          pa[hn * 2 + 1] = pack2(w[hn][2], w[hn][3]);
         }
+        l[0] += (w[0][0] + w[0][1]) + (w[1][0] + w[1][1]);
+        l[1] += (w[0][2] + w[0][3]) + (w[1][2] + w[1][3]);
         if (WITH_V) {
 #pragma unroll
           for (int j = 0; j < D / 16; ++j) {
@@ -426,10 +442,10 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a,
 template <int D, bool WITH_V, bool SPARSE>
 cudaError_t launch_t(const Dims& Dm, const FwdArgs& a, cudaStream_t st) {
   auto kern = fwd_mma_kernel<D, WITH_V, SPARSE>;
-  const size_t smem = sizeof(Smem<D>);
+  const size_t smem = sizeof(Smem<D>) + (size_t)sel_rows(Dm.per_token, Dm.s) * 64 * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  MmaShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale, Dm.per_token};
+  MmaShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale, Dm.per_token, __builtin_ctz((unsigned)Dm.s)};
   dim3 grid(Dm.N / BM, Dm.Hq, Dm.B);
   kern<<<grid, NT, smem, st>>>(a, sh);
   count_launches(1);

@@ -88,6 +88,20 @@ __device__ __forceinline__ unsigned long long tile_keep_mask(const uint32_t* blo
   return m;
 }
 
+// The same mask for s = 1 << ls, s >= 16 (the supported block sizes are
+// powers of two): the tile's 64 / s blocks sit in one aligned 32-bit word.
+__device__ __forceinline__ unsigned long long tile_keep_mask_p2(const uint32_t* blocks, int u0, int ls) {
+  const int jb = u0 >> ls;
+  const uint32_t word = blocks[jb >> 5] >> (jb & 31);
+  if (ls >= 6) return (word & 1u) ? ~0ull : 0ull;
+  const int nb = 64 >> ls;
+  const unsigned long long run = (1ull << (1 << ls)) - 1ull;
+  unsigned long long m = 0ull;
+  for (int b = 0; b < nb; ++b)
+    if ((word >> b) & 1u) m |= run << (b << ls);
+  return m;
+}
+
 // Bit c is set when key u0 + c <= t (a causal pair of query t).
 __device__ __forceinline__ unsigned long long causal_mask(int t, int u0) {
   const int lim = t - u0;
