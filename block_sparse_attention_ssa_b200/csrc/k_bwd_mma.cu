@@ -408,7 +408,7 @@ struct DkvSmem {
 };
 
 template <int D, bool SPARSE>
-__global__ void __launch_bounds__(NT, D == 64 ? 3 : 1)
+__global__ void __launch_bounds__(NT, D == 64 ? 2 : 1)
     bwd_dkv_mma_kernel(BwdArgs a, MmaShape sh, const bf16* __restrict__ dhf, const bf16* __restrict__ doc,
                        float* __restrict__ part) {
   constexpr int NQ = 32;  // queries per register sub-tile
@@ -513,6 +513,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 1)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
 
+  uint32_t kfr[D / 16][4], vfr[D / 16][4];  // the warp's K and V rows as A fragments, loaded once
   int it = 0;
   while (step >= 0) {
     const int buf = it & 1;
@@ -522,6 +523,13 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 1)
     cp_async_wait<1>();
     __syncthreads();
     const bool diag = (step % nq) == 0;  // query tile == key tile
+    if (it == 0) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        ldsm_x4(kfr[kk], &S.k[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+        ldsm_x4(vfr[kk], &S.v[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+      }
+    }
 
     // The warp's 16 keys lie in one key block (blocks have 16 keys or more):
     // bit bp of a query row's selection word says whether that row selected it.
@@ -577,9 +585,8 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 1)
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t ka[4], va[4];
-        ldsm_x4(ka, &S.k[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
-        ldsm_x4(va, &S.v[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+        const uint32_t (&ka)[4] = kfr[kk];
+        const uint32_t (&va)[4] = vfr[kk];
 #pragma unroll
         for (int j = 0; j < NN / 2; ++j) {
           if (((live >> (2 * j)) & 3u) == 0u) continue;

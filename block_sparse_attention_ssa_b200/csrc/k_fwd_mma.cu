@@ -61,7 +61,7 @@ struct Smem {
 __host__ __device__ inline int sel_rows(int per_token, int s) { return per_token ? BM : (s >= BM ? 1 : BM / s); }
 
 template <int D, bool WITH_V, bool SPARSE>
-__global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_mma_kernel(FwdArgs a, MmaShape sh) {
+__global__ void __launch_bounds__(NT, D == 64 ? 4 : 2) fwd_mma_kernel(FwdArgs a, MmaShape sh) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Smem<D>& S = *reinterpret_cast<Smem<D>*>(smem_raw);
   uint32_t (*sel)[64] = reinterpret_cast<uint32_t (*)[64]>(smem_raw + sizeof(Smem<D>));
