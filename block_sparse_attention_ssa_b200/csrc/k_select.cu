@@ -8,7 +8,8 @@
 // the mean of the block's queries) and per query head; the diagonal block is
 // always kept and counts toward k.
 //
-// All three kernels are HBM- or latency-bound and run on CUDA cores.
+// The kernels are HBM-, latency- or (per-token scoring) FMA-bound and run on
+// CUDA cores.
 #include <climits>
 
 #include "ssa_internal.cuh"
@@ -107,15 +108,23 @@ __device__ __forceinline__ void select_row(float (&v)[CPL], int i, int n, int k,
     for (int m = 0; m < CPL; ++m)
       if (lane + 32 * m <= i) taken |= 1ull << m;
   } else {
+    // Candidates that cannot be chosen (j >= i, or already taken) hold NaN,
+    // which compares false with everything, so a round's lane-local scan is
+    // one ordered compare per slot (slots ascend in j: the first of equal
+    // scores is the smaller j; the first -inf counts when nothing better is
+    // left).
+    const float kOut = __int_as_float(0x7fffffff);
+#pragma unroll
+    for (int m = 0; m < CPL; ++m)
+      if (lane + 32 * m >= i) v[m] = kOut;
     for (int round = 0; round < k - 1; ++round) {
       float bv = kNegInf;
       int bj = INT_MAX;
 #pragma unroll
       for (int m = 0; m < CPL; ++m) {
-        const int j = lane + 32 * m;
-        if (j < i && !((taken >> m) & 1ull) && better(v[m], j, bv, bj)) {
+        if (v[m] > bv || (v[m] == bv && bj == INT_MAX)) {
           bv = v[m];
-          bj = j;
+          bj = lane + 32 * m;
         }
       }
 #pragma unroll
@@ -127,7 +136,12 @@ __device__ __forceinline__ void select_row(float (&v)[CPL], int i, int n, int k,
           bj = oj;
         }
       }
-      if (bj != INT_MAX && (bj & 31) == lane) taken |= 1ull << (bj >> 5);
+      if (bj != INT_MAX && (bj & 31) == lane) {
+        taken |= 1ull << (bj >> 5);
+#pragma unroll
+        for (int m = 0; m < CPL; ++m)
+          if (m == (bj >> 5)) v[m] = kOut;
+      }
     }
     if ((i & 31) == lane) taken |= 1ull << (i >> 5);
   }
@@ -212,6 +226,70 @@ __global__ void __launch_bounds__(256) token_select_kernel(TensorRef Q, const fl
   select_row<CPL>(v, i, n, k, lane, idx + row * k);
 }
 
+// Shared-memory form, used when the pooled keys of one kv head fit: a CTA of
+// TOK_WARPS warps takes TOK_PER_CTA consecutive tokens of one (b, h) and stages the
+// pooled keys its tokens can rank (blocks j < jmax) transposed, kT[c][j]
+// with a row pitch of n + 1 floats (the transposing stores fall in distinct
+// banks).  Lane l then forms whole dot products for its blocks j = l + 32 m
+// (the query broadcast from shared memory): no cross-lane reduction per
+// block, and each pooled key is read from global memory once per CTA
+// instead of once per token.
+constexpr int TOK_PER_CTA = 256;
+constexpr int TOK_WARPS = 16;  // 512 threads share one staged copy of the pooled keys
+
+template <typename T, int D, int CPL>
+__global__ void __launch_bounds__(TOK_WARPS * 32) token_select_smem_kernel(TensorRef Q, const float* __restrict__ kbar,
+                                                                int32_t* __restrict__ idx, int Hq, int g, int N,
+                                                                int s, int n, int k, float scale) {
+  extern __shared__ float kT[];  // [D][n + 1] (+ 32 floats of slack: lanes past i read, and discard, the tail)
+  __shared__ float qs[TOK_WARPS][D];  // each warp's current query row
+  const int t0 = blockIdx.x * TOK_PER_CTA, h = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tend = min(t0 + TOK_PER_CTA, N);
+  const int jmax = (tend - 1) / s;
+  const int pitch = n + 1;
+  const float* kb = kbar + ((int64_t)b * (Hq / g) + h / g) * n * D;
+  for (int e = threadIdx.x; e < jmax * D; e += TOK_WARPS * 32) {
+    const int j = e / D, c = e % D;
+    kT[c * pitch + j] = kb[(int64_t)j * D + c];
+  }
+  __syncthreads();
+  for (int t = t0 + warp; t < tend; t += TOK_WARPS) {
+    const int i = t / s;
+    const T* qrow = row_ptr<T>(Q, b, h, t);
+    for (int c = lane; c < D; c += 32) qs[warp][c] = to_f32(qrow[c]);
+    __syncwarp();
+    // One group of 32 blocks at a time; groups past the token's causal
+    // range are skipped as a whole (the guard is warp-uniform).
+    float acc[CPL];
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) {
+      acc[m] = 0.f;
+      if (32 * m < i) {
+        const float* col = kT + lane + 32 * m;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll 16
+        for (int c = 0; c < D; c += 2) {
+          a0 = fmaf(qs[warp][c], col[c * pitch], a0);
+          a1 = fmaf(qs[warp][c + 1], col[(c + 1) * pitch], a1);
+        }
+        acc[m] = a0 + a1;
+      }
+    }
+    __syncwarp();
+    float v[CPL];
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) {
+      const float x = scale * acc[m];
+      v[m] = (lane + 32 * m < i && x == x) ? x : kNegInf;  // NaN ranks as -inf
+    }
+    select_row<CPL>(v, i, n, k, lane, idx + (((int64_t)b * Hq + h) * N + t) * k);
+  }
+}
+
+size_t token_select_smem_bytes(int n, int d) { return ((size_t)d * (n + 1) + 32) * sizeof(float); }
+constexpr size_t kTokenSelectSmemMax = 200 * 1024;
+
 // ------------------------------------------------------------------ mask
 // grid = rows, 32 threads: words of the selected-block bit set of one
 // selection row (a query block, or a token when div = s: i = (row % rph) / div).
@@ -280,9 +358,34 @@ cudaError_t launch_build_mask(const Dims& D, const int32_t* idx, uint32_t* mask,
 
 template <typename T, int D>
 cudaError_t token_select_t(const Dims& Dm, const TensorRef& Q, const float* kbar, int32_t* idx, cudaStream_t st) {
+  const int cpl = (Dm.n + 31) / 32;
+  const size_t smem = token_select_smem_bytes(Dm.n, D);
+  if (smem <= kTokenSelectSmemMax) {
+    const dim3 grid((unsigned)((Dm.N + TOK_PER_CTA - 1) / TOK_PER_CTA), (unsigned)Dm.Hq, (unsigned)Dm.B);
+    cudaError_t e = cudaSuccess;
+#define SSA_TOKSEL_SMEM(C)                                                                                \
+  do {                                                                                                    \
+    auto kern = token_select_smem_kernel<T, D, C>;                                                        \
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);               \
+    if (e == cudaSuccess)                                                                                 \
+      kern<<<grid, TOK_WARPS * 32, smem, st>>>(Q, kbar, idx, Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale); \
+  } while (0)
+    if (cpl <= 1) SSA_TOKSEL_SMEM(1);
+    else if (cpl <= 2) SSA_TOKSEL_SMEM(2);
+    else if (cpl <= 4) SSA_TOKSEL_SMEM(4);
+    else if (cpl <= 8) SSA_TOKSEL_SMEM(8);
+    else if (cpl <= 16) SSA_TOKSEL_SMEM(16);
+    else {
+      if constexpr (D == 64) SSA_TOKSEL_SMEM(32);
+      else return cudaErrorInvalidConfiguration;  // unreachable: d = 128 fits at most 399 pooled keys
+    }
+#undef SSA_TOKSEL_SMEM
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+    return cudaGetLastError();
+  }
   const int64_t rows = (int64_t)Dm.B * Dm.Hq * Dm.N;
   const unsigned grid = (unsigned)((rows + 7) / 8);
-  const int cpl = (Dm.n + 31) / 32;
 #define SSA_TOKSEL(C) token_select_kernel<T, D, C><<<grid, 256, 0, st>>>(Q, kbar, idx, rows, Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, Dm.scale)
   if (cpl <= 1) SSA_TOKSEL(1);
   else if (cpl <= 2) SSA_TOKSEL(2);

@@ -150,3 +150,24 @@ def test_token_decode():
     idx_f = O.select_tokens(O.token_scores(host["Q"], host["K"], s, scale), k, s)
     t = t0 + 39
     np.testing.assert_array_equal(idx_f[:, :, t], st["idx"].cpu().numpy())
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_token_selection_many_blocks(d):
+    """512 blocks of 16 (the pages' block size at 8192 tokens): at d = 64 the
+    pooled keys of a kv head fit in shared memory and the staged kernel runs,
+    at d = 128 they do not and the per-token-warp kernel runs.  Both against
+    the oracle's per-token top-k, near ties logged."""
+    B, Hq, Hkv, N, s, k = 1, 2, 1, 8192, 16, 16
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 838 + d, "bf16")
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16", per_token=True)
+    ws = api.alloc_workspace(dims)
+    idx = torch.full((B, Hq, N, k), -7, dtype=torch.int32, device="cuda")
+    api.ssa_select_tokens(dims, dev["Q"], dev["K"], idx, ws)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    ora_scores = O.token_scores(host["Q"], host["K"], s, 1 / math.sqrt(d))
+    ora_idx = O.select_tokens(ora_scores, k, s)
+    near = _compare_token_selection(idx.cpu().numpy(), ora_idx, ora_scores, s)
+    if near:
+        print(f"d={d}: {len(near)} near-tie rows")
