@@ -604,10 +604,10 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 // 4-D map over a [B, H, N, d] bf16 tensor: dims (d, N, H, B), box (64, rows, 1, 1).
-bool make_tma_map_bf16(CUtensorMap* map, const TensorRef& t, int B, int H, int N, int rows) {
+bool make_tma_map_bf16(CUtensorMap* map, const TensorRef& t, int B, int H, int N, int rows, int d) {
   auto enc = get_encode();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+  if (enc == nullptr || (d != 64 && d != 128)) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)t.sn * 2, (cuuint64_t)t.sh * 2, (cuuint64_t)t.sb * 2};
   // A zero stride (a broadcast dimension of size 1) is not accepted; any
   // positive multiple of 16 describes the same single slice.

@@ -162,9 +162,15 @@ cudaError_t launch_dropped_mma(const Dims& D, const FwdArgs& a, cudaStream_t st)
 cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
 bool fwd_tc_supported(const Dims& D);
 
-// 4-D TMA map over a [B, H, N, 128] bf16 tensor: dims (d, N, H, B), box
-// (64 columns, `rows` rows), 128-byte swizzle, zero fill out of bounds.
-bool make_tma_map_bf16(CUtensorMap* map, const TensorRef& t, int B, int H, int N, int rows);
+// 4-D TMA map over a [B, H, N, d] bf16 tensor (d = 64 or 128): dims
+// (d, N, H, B), box (64 columns, `rows` rows), 128-byte swizzle, zero fill
+// out of bounds.
+bool make_tma_map_bf16(CUtensorMap* map, const TensorRef& t, int B, int H, int N, int rows, int d = 128);
+
+// Tensor-core dual-stream forward with per-row selection masks (bf16, d = 64
+// or 128, any block size, per-block or per-token selection; dual mode only).
+bool fwd_tcm_supported(const Dims& D);
+cudaError_t launch_fwd_tcm(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
 
 struct BwdArgs {
   TensorRef q, k, v, hf, hs, gf, gs, dq, dk, dv;  // gf / gs .p may be null
