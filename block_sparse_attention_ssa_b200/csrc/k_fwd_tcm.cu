@@ -317,16 +317,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int u0 = j * BN + q * SUB;  // first key of this warp's sub-block
       bool anyA, anyD;
       regions(u0, anyA, anyD);
-      // This row's keys of the sub-block: selected (A) and dropped (D).
-      const unsigned long long causal = valid ? causal_mask(t, u0) : 0ull;
-      const unsigned long long cm = causal & tile_keep_mask_p2(selw, u0, p.ls);
-      const unsigned long long dm = causal & ~cm;
-      const uint32_t a_lo = (uint32_t)cm, a_hi = (uint32_t)(cm >> 32);
-      const uint32_t d_lo = (uint32_t)dm, d_hi = (uint32_t)(dm >> 32);
+      // Blocks have 16 keys or more, so a row's selection is constant over
+      // each 16-key group of the sub-block: bit 16g of the row's kept-block
+      // mask says whether group g is selected.  Causality only cuts the
+      // diagonal sub-blocks; there the keys after t are set to -inf.
+      const unsigned long long km = tile_keep_mask_p2(selw, u0, p.ls);
+      bool gA[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) gA[g] = (km >> (16 * g)) & 1ull;
+      const int lim = valid ? t - u0 : -1;  // keys c <= lim are causal
       const uint32_t s_addr = lane_base + C::COL_S + (uint32_t)sb * BN;
       float x[SUB];  // raw S of this warp's sub-block; the scale is folded into the exponent
       float mxA = kNegInf, mxD = kNegInf;
-      if (__any_sync(0xffffffffu, causal != 0ull)) {
+      if (__any_sync(0xffffffffu, lim >= 0)) {
 #pragma unroll
         for (int c0 = 0; c0 < SUB; c0 += 32) {
           uint32_t r[32];
@@ -335,18 +338,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(r[c]);
         }
-        float a0 = kNegInf, a1 = kNegInf, d0 = kNegInf, d1 = kNegInf;
+        if (lim < SUB - 1) {
 #pragma unroll
-        for (int c = 0; c < SUB; c += 2) {
-          const uint32_t am = c < 32 ? a_lo : a_hi, dmw = c < 32 ? d_lo : d_hi;
-          const int bit = c & 31;
-          a0 = ((am >> bit) & 1u) ? fmaxf(a0, x[c]) : a0;
-          a1 = ((am >> (bit + 1)) & 1u) ? fmaxf(a1, x[c + 1]) : a1;
-          d0 = ((dmw >> bit) & 1u) ? fmaxf(d0, x[c]) : d0;
-          d1 = ((dmw >> (bit + 1)) & 1u) ? fmaxf(d1, x[c + 1]) : d1;
+          for (int c = 0; c < SUB; ++c) x[c] = (c <= lim) ? x[c] : kNegInf;
         }
-        mxA = fmaxf(a0, a1) * p.c;  // scale > 0
-        mxD = fmaxf(d0, d1) * p.c;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float a0 = x[16 * g], a1 = x[16 * g + 1], a2 = x[16 * g + 2], a3 = x[16 * g + 3];
+#pragma unroll
+          for (int c = 16 * g + 4; c < 16 * g + 16; c += 4) {
+            a0 = fmaxf(a0, x[c]);
+            a1 = fmaxf(a1, x[c + 1]);
+            a2 = fmaxf(a2, x[c + 2]);
+            a3 = fmaxf(a3, x[c + 3]);
+          }
+          const float gm = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+          mxA = gA[g] ? fmaxf(mxA, gm) : mxA;
+          mxD = gA[g] ? mxD : fmaxf(mxD, gm);
+        }
+        mxA *= p.c;  // scale > 0
+        mxD *= p.c;
+      } else {
+#pragma unroll
+        for (int c = 0; c < SUB; ++c) x[c] = kNegInf;
       }
       // Trade sub-block maxima with the partner warp; after this point both
       // warps have read their S columns, so P may overwrite them.
@@ -390,36 +404,36 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (m2[X] == kNegInf) m2[X] = mxs;
       }
       if (!ok) break;
-      // Weights: one exponential per key, routed to its set's region; two
-      // halves of 32 keys (16 packed columns each) keep fewer registers live.
+      // Weights: one exponential per key against its group's set max; each
+      // group's packed weights go to its set's region, zeros to the other.
       {
-        const float nA = -m2[0], nD = -m2[1];
-        float sA = 0.f, sD = 0.f;
+        const float nA = m2[0] == kNegInf ? 0.f : -m2[0];
+        const float nD = m2[1] == kNegInf ? 0.f : -m2[1];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t am = hh ? a_hi : a_lo, dmw = hh ? d_hi : d_lo;
           uint32_t pa[16], pd[16];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float wa[2], wd[2];
+          for (int gg = 0; gg < 2; ++gg) {
+            const int g = 2 * hh + gg;
+            const float ng = gA[g] ? nA : nD;
+            float sg0 = 0.f, sg1 = 0.f;
 #pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              const bool inA = (am >> (c + v)) & 1u, inD = (dmw >> (c + v)) & 1u;
-              const float xv = x[32 * hh + c + v];
-              const float e = ex2(inA ? fmaf(xv, p.c, nA) : (inD ? fmaf(xv, p.c, nD) : kNegInf));
-              wa[v] = inA ? e : 0.f;
-              wd[v] = inD ? e : 0.f;
+            for (int c = 0; c < 16; c += 2) {
+              const float e0 = ex2(fmaf(x[16 * g + c], p.c, ng));
+              const float e1 = ex2(fmaf(x[16 * g + c + 1], p.c, ng));
+              sg0 += e0;
+              sg1 += e1;
+              const uint32_t pk = pack_bf16(e0, e1);
+              pa[8 * gg + c / 2] = gA[g] ? pk : 0u;
+              pd[8 * gg + c / 2] = gA[g] ? 0u : pk;
             }
-            sA += wa[0] + wa[1];
-            sD += wd[0] + wd[1];
-            pa[c / 2] = pack_bf16(wa[0], wa[1]);
-            pd[c / 2] = pack_bf16(wd[0], wd[1]);
+            const float sg = sg0 + sg1;
+            l[0] += gA[g] ? sg : 0.f;
+            l[1] += gA[g] ? 0.f : sg;
           }
           if (anyA) tmem_st16(s_addr + 32 * q + 16 * hh, pa);
           if (anyD) tmem_st16(s_addr + 64 + 32 * q + 16 * hh, pd);
         }
-        l[0] += sA;
-        l[1] += sD;
       }
       tmem_wait_st();
       tc_fence_before();
