@@ -89,6 +89,7 @@ struct TcmParams {
   float* lse_full;
   float* lse_sel;
   float* delta;
+  const float* lse_in;  // dropped-mass mode: the given lse_full, or null
   int32_t* status;
   int Hq, g, N, n, k, ls, per_token;
   float c;  // scale * log2(e)
@@ -108,7 +109,9 @@ __device__ __forceinline__ bool pair_sync(uint64_t* bar, uint32_t& uses, int lan
   return ok;
 }
 
-template <int HD>
+// WITH_V = false is the dropped-mass probe: no V, no PV products, only the
+// two sets' running sums, and delta written (from lse_in when it is given).
+template <int HD, bool WITH_V>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_tcm_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, TcmParams p) {
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
+      if (WITH_V) prefetch_tensormap(&tmV);
       mbar_expect_tx(&M.q_full, C::Q_BYTES);
 #pragma unroll
       for (int hh = 0; hh < HD / 64; ++hh) tma_load_4d(sQ + hh * C::HALF_Q, &tmQ, &M.q_full, 64 * hh, q0, h, b);
@@ -217,6 +220,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (j >= NS && !mbar_wait(&M.k_empty[st], (use - 1) & 1u, abort)) break;
         load_tile(sK + st * C::KV_BYTES, &tmK, &M.k_full[st]);
         k_issued = j + 1;
+        if (!WITH_V) continue;
         if (j >= NS && !mbar_wait(&M.v_empty[st], (use - 1) & 1u, abort)) break;
         load_tile(sV + st * C::KV_BYTES, &tmV, &M.v_full[st]);
         v_issued = j + 1;
@@ -242,6 +246,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       auto issue_pv = [&](int jj) -> bool {
         const int sb = jj & 1;
         if (!mbar_wait(&M.p_full[sb], (uint32_t)(jj >> 1) & 1u, abort)) return false;
+        if (!WITH_V) return true;  // the S buffer is free again; nothing to multiply
         const int st = jj % NS;
         if (!mbar_wait(&M.v_full[st], (uint32_t)(jj / NS) & 1u, abort)) return false;
         tc_fence_after();
@@ -305,6 +310,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     float m2[2] = {kNegInf, kNegInf};  // running max (scaled, base 2), [0]=A [1]=D
     float l[2] = {0.f, 0.f};           // this warp's partial sums
+    const bool direct = !WITH_V && p.lse_in != nullptr;  // uniform over the CTA
+    const float lse2_in = (direct && valid) ? p.lse_in[((int64_t)b * p.Hq + h) * p.N + t] * 1.4426950408889634f : 0.f;
     uint32_t pair_uses = 0;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
@@ -327,6 +334,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int g = 0; g < 4; ++g) gA[g] = (km >> (16 * g)) & 1ull;
       const int lim = valid ? t - u0 : -1;  // keys c <= lim are causal
       const uint32_t s_addr = lane_base + C::COL_S + (uint32_t)sb * BN;
+      if (direct) {
+        // Dropped mass with lse_full given: sum 2^(S*c - lse2) over the
+        // dropped keys directly; no running max, nothing traded.
+        if (__any_sync(0xffffffffu, lim >= 0)) {
+#pragma unroll
+          for (int c0 = 0; c0 < SUB; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(s_addr + q * SUB + c0, r);
+            tmem_wait_ld();
+            float sD = 0.f;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const bool use = !gA[(c0 + c) >> 4] && (c0 + c <= lim);
+              sD += use ? ex2(fmaf(__uint_as_float(r[c]), p.c, -lse2_in)) : 0.f;
+            }
+            l[1] += sD;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&M.p_full[sb]);
+        continue;
+      }
       float x[SUB];  // raw S of this warp's sub-block; the scale is folded into the exponent
       float mxA = kNegInf, mxD = kNegInf;
       if (__any_sync(0xffffffffu, lim >= 0)) {
@@ -375,7 +405,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float mxs = fmaxf(X == 0 ? mxA : mxD, M.xmax[sb][q ^ 1][X][row]);
         const float m_old = m2[X];
         const bool need = (m_old != kNegInf) && (mxs > m_old + kRescaleThreshold);
-        if (__any_sync(0xffffffffu, need)) {
+        if (!WITH_V) {
+          if (need) {
+            l[X] *= ex2(m_old - mxs);
+            m2[X] = mxs;
+          }
+        } else if (__any_sync(0xffffffffu, need)) {
           // O_X must hold every earlier PV before it is rescaled; this warp
           // rescales its half of the columns.
           if (j >= 1 && !mbar_wait(&M.o_done, (uint32_t)(j - 1) & 1u, abort)) ok = false;
@@ -431,8 +466,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             l[0] += gA[g] ? sg : 0.f;
             l[1] += gA[g] ? 0.f : sg;
           }
-          if (anyA) tmem_st16(s_addr + 32 * q + 16 * hh, pa);
-          if (anyD) tmem_st16(s_addr + 64 + 32 * q + 16 * hh, pd);
+          if (WITH_V && anyA) tmem_st16(s_addr + 32 * q + 16 * hh, pa);
+          if (WITH_V && anyD) tmem_st16(s_addr + 64 + 32 * q + 16 * hh, pd);
         }
       }
       tmem_wait_st();
@@ -446,7 +481,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     M.lsum[q][0][row] = l[0];
     M.lsum[q][1][row] = l[1];
     if (ok && !pair_sync(&M.pair[quarter], pair_uses, lane, abort)) ok = false;
-    if (ok && mbar_wait(&M.o_final, 0, abort)) {
+    if (ok && !WITH_V && q == 0 && valid) {
+      const float lA = l[0] + M.lsum[1][0][row], lD = l[1] + M.lsum[1][1][row];
+      const int64_t o = ((int64_t)b * p.Hq + h) * p.N + t;
+      if (direct) {
+        p.delta[o] = lD;
+      } else {
+        const float lse2_a = (lA > 0.f) ? m2[0] + log2f(lA) : kNegInf;
+        const float lse2_d = (lD > 0.f) ? m2[1] + log2f(lD) : kNegInf;
+        const float hi = fmaxf(lse2_a, lse2_d), lo = fminf(lse2_a, lse2_d);
+        const float lse2_f = (lo == kNegInf) ? hi : hi + log2f(1.0f + ex2(lo - hi));
+        p.delta[o] = (lD > 0.f) ? ex2(lse2_d - lse2_f) : 0.f;
+      }
+    }
+    if (WITH_V && ok && mbar_wait(&M.o_final, 0, abort)) {
       tc_fence_after();
       const float lA = l[0] + M.lsum[q ^ 1][0][row], lD = l[1] + M.lsum[q ^ 1][1][row];
       const float mA = m2[0], mD = m2[1];
@@ -508,7 +556,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <int HD>
+template <int HD, bool WITH_V>
 cudaError_t launch_hd(const Dims& D, const FwdArgs& a, int32_t* status, cudaStream_t st) {
   using C = Cfg<HD>;
   CUtensorMap mq, mk, mv;
@@ -522,6 +570,7 @@ cudaError_t launch_hd(const Dims& D, const FwdArgs& a, int32_t* status, cudaStre
   p.lse_full = a.lse_full;
   p.lse_sel = a.lse_sel;
   p.delta = a.delta;
+  p.lse_in = WITH_V ? nullptr : a.lse_in;
   p.status = status;
   p.Hq = D.Hq;
   p.g = D.g;
@@ -532,7 +581,7 @@ cudaError_t launch_hd(const Dims& D, const FwdArgs& a, int32_t* status, cudaStre
   p.per_token = D.per_token;
   p.c = D.scale * 1.4426950408889634f;
   const int smem = C::OFF_MISC + (int)sizeof(Misc<C::NS>) + tcm_sel_rows(D.per_token, p.ls) * 64 * 4 + 1024;
-  auto kern = fwd_tcm_kernel<HD>;
+  auto kern = fwd_tcm_kernel<HD, WITH_V>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((D.N + BM - 1) / BM, D.Hq, D.B);
@@ -549,7 +598,12 @@ bool fwd_tcm_supported(const Dims& D) {
 
 cudaError_t launch_fwd_tcm(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st) {
   if (!fwd_tcm_supported(D) || a.sparse_only) return cudaErrorNotSupported;
-  return D.d == 128 ? launch_hd<128>(D, a, dev_status, st) : launch_hd<64>(D, a, dev_status, st);
+  return D.d == 128 ? launch_hd<128, true>(D, a, dev_status, st) : launch_hd<64, true>(D, a, dev_status, st);
+}
+
+cudaError_t launch_dropped_tcm(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st) {
+  if (!fwd_tcm_supported(D)) return cudaErrorNotSupported;
+  return D.d == 128 ? launch_hd<128, false>(D, a, dev_status, st) : launch_hd<64, false>(D, a, dev_status, st);
 }
 
 }  // namespace ssa

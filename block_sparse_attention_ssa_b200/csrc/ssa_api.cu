@@ -499,10 +499,11 @@ ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, con
   a.idx = idx;
   a.delta = delta;
   a.lse_in = lse_full;
-  if (fwd_tc_supported(D)) {
+  if (fwd_tc_supported(D) || fwd_tcm_supported(D)) {
     int32_t* status = device_status_ptr();
     if (status == nullptr) return SSA_ERR_CUDA;
-    return from_cuda(launch_dropped_tc(D, a, status, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return from_cuda(fwd_tc_supported(D) ? launch_dropped_tc(D, a, status, st) : launch_dropped_tcm(D, a, status, st));
   }
   if (fwd_mma_supported(D)) return from_cuda(launch_dropped_mma(D, a, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_dropped_simt(D, a, static_cast<cudaStream_t>(stream)));

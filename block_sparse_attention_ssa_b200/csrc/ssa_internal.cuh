@@ -171,6 +171,8 @@ bool make_tma_map_bf16(CUtensorMap* map, const TensorRef& t, int B, int H, int N
 // or 128, any block size, per-block or per-token selection; dual mode only).
 bool fwd_tcm_supported(const Dims& D);
 cudaError_t launch_fwd_tcm(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
+// Its dropped-mass mode (QK^T only; delta from a.lse_in when given).
+cudaError_t launch_dropped_tcm(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
 
 struct BwdArgs {
   TensorRef q, k, v, hf, hs, gf, gs, dq, dk, dv;  // gf / gs .p may be null
