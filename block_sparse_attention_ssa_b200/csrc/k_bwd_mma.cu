@@ -787,7 +787,16 @@ size_t bwd_mma_partial_bytes(const Dims& D) {
   return (size_t)chunks * 2 * D.B * D.Hkv * D.N * D.d * sizeof(float);
 }
 
-cudaError_t launch_bwd_mma(const Dims& D, const BwdArgs& a, cudaStream_t st) {
+cudaError_t launch_kvsum(const Dims& D, const BwdArgs& a, const float* part, int chunks, cudaStream_t st) {
+  const int64_t plane = (int64_t)D.B * D.Hkv * D.N * D.d;
+  const unsigned blocks = (unsigned)((plane / 4 + 255) / 256);
+  if (D.d == 128) kvsum_kernel<128><<<blocks, 256, 0, st>>>(part, chunks, D.Hkv, D.N, D.scale, a.dk, a.dv, plane);
+  else kvsum_kernel<64><<<blocks, 256, 0, st>>>(part, chunks, D.Hkv, D.N, D.scale, a.dk, a.dv, plane);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_mma(const Dims& D, const BwdArgs& a, int32_t* status, cudaStream_t st) {
   // The fp32 dh_f / dO_c workspace regions hold the bf16 operands in their
   // lower halves.
   bf16* dhf = reinterpret_cast<bf16*>(a.dhf);
@@ -804,6 +813,9 @@ cudaError_t launch_bwd_mma(const Dims& D, const BwdArgs& a, cudaStream_t st) {
     e = launch_finish_mean(a.partials, a.n_partials, M, 2.0f, a.align_loss, 1, st);
     if (e != cudaSuccess) return e;
   }
+  // Dual backward at d = 64: the tcgen05 kernels with per-row masks.
+  if (!a.sparse_only && status != nullptr && bwd_tcm_supported(D))
+    return launch_bwd_tcm(D, a, dhf, doc, bwd_mma_heads_per_cta(D), status, st);
   if (D.d == 128)
     return a.sparse_only ? bwd_t<128, true>(D, a, dhf, doc, st) : bwd_t<128, false>(D, a, dhf, doc, st);
   return a.sparse_only ? bwd_t<64, true>(D, a, dhf, doc, st) : bwd_t<64, false>(D, a, dhf, doc, st);

@@ -1,0 +1,719 @@
+// Tensor-core backward with per-row selection masks (sm_100a, bf16, d = 64):
+// blocks of 16 to 128 keys, selection per query block or per query token.
+//
+// Objective ("Technische Samenvatting: SSA", "Bidirectionele Uitlijning";
+// "SSA: Achieving Sparser Attention ...", "Bidirectional Attention
+// Alignment"): L = <g_f, h_full> + <g_s, h_sparse> + alpha (L_sp + L_cm).
+// As in the warp-level kernels the two streams collapse into one softmax
+// backward over the full stream's weights P = exp(x - lse_full):
+//   selected pair (u in A_t): dX = P (dO_c . v_u - D_c),  dV_u += P dO_c,
+//   dropped pair  (u in D_t): dX = P (dh_f . v_u - D_f),  dV_u += P dh_f,
+// dQ_t = scale sum_u dX K_u, dK_u = scale sum_t dX Q_t (the preprocess of the
+// warp-level backward supplies dO_c and dh_f in bf16, D_c and D_f).
+//
+// Two kernels, 320 threads each: warps 0-7 compute (warps w and w+4 share
+// TMEM lanes 32(w%4).., warp w takes the 64 columns w/4), warp 8 loads by
+// TMA, warp 9 owns TMEM and issues the MMAs.  All tiles are 128 x 64 bf16
+// (one 128-byte swizzle span per row).
+//
+//   dq   one 128-row query tile per CTA, walking its causal key tiles.  TMEM:
+//        dQ [0,64), S [64,192), dP_c [192,320), dP_f [320,448).  Per tile:
+//        S = Q K^T, dP_c = dO_c V^T, dP_f = dh_f V^T (each only when a row of
+//        the tile can use it), dS = P (dP_x - D_x) routed per 16-key group by
+//        the row's selection, written as bf16 over the warp's own S columns,
+//        then dQ += dS K.
+//   dkv  one 128-key tile per CTA, walking a chunk of at most 4 query heads
+//        of its kv group and their causal query tiles.  TMEM: dK [0,64),
+//        dV [64,128), S^T [128,256), dP_c^T [256,384), dP_f^T [384,512).  Per
+//        step: S^T = K Q^T, dP_c^T = V dO_c^T, dP_f^T = V dh_f^T, then P_A^T
+//        over S^T, P_D^T over dP_f^T and dS^T over dP_c^T (each warp packs into
+//        columns it has already read), dV += P_A^T dO_c + P_D^T dh_f and
+//        dK += dS^T Q.  A query's selection word decides, per key block, the
+//        set of each element.  With more than one chunk per group the chunks
+//        write fp32 partials that the warp-level backward's sum adds in order.
+// No atomics: every output element is written by one CTA in a fixed order.
+#include "ssa_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace ssa {
+namespace {
+
+using namespace sm100;
+using bf16 = __nv_bfloat16;
+
+constexpr int HD = 64;
+constexpr int TILE = 128;
+constexpr int TB = TILE * HD * 2;  // 16 KB: one 128 x 64 bf16 tile
+constexpr int NTHREADS = 320;
+constexpr int WARP_TMA = 8, WARP_MMA = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, TILE, false, false);  // both K-major
+constexpr uint32_t IDESC_ACC = idesc_bf16_f32(TILE, HD, false, true);   // B MN-major (rows = reduction)
+
+struct TcmBwdParams {
+  TensorRef dq, dk, dv;
+  const float* lse;  // lse_full [B,Hq,N]
+  const float* Dc;   // [B,Hq,N]
+  const float* Df;
+  const uint32_t* mask;  // [B,Hq,rows,words] selected-block bit sets
+  int words;
+  float* part;  // fp32 dK / dV partials, or null
+  int32_t* status;
+  int Hq, g, N, n, ls, per_token, hpc, NT;
+  float c;  // scale * log2(e)
+  float scale;
+};
+
+// D (128 x 128) = A (128 x 64) B^T with both operands K-major smem tiles.
+__device__ __forceinline__ void mma_ss_d64(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk)
+    mma_ss(d_tmem, smem_desc_sw128(a_smem + kk * 32, 16, 1024), smem_desc_sw128(b_smem + kk * 32, 16, 1024),
+           IDESC_S, kk > 0 ? 1u : 0u);
+}
+
+// D (128 x 64) (+)= A (TMEM, 128 rows x 128 reduction as bf16 pairs: indices
+// 0-63 at columns a..a+31, 64-127 at a+64..a+95) x B (smem 128 x 64 tile,
+// rows = reduction index).
+__device__ __forceinline__ void mma_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < TILE / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), smem_desc_sw128(b_smem + kk * 2048, TB, 1024), IDESC_ACC,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__host__ __device__ inline int sel_rows_tile(int per_token, int ls) {
+  return per_token ? TILE : (ls >= 7 ? 1 : (TILE >> ls));
+}
+
+// ================================================================ dQ
+namespace dqm {
+constexpr int NS = 3;
+constexpr int OFF_Q = 0, OFF_OC = TB, OFF_F = 2 * TB, OFF_K = 3 * TB, OFF_V = OFF_K + NS * TB;
+constexpr int OFF_MISC = OFF_V + NS * TB;
+constexpr uint32_t COL_DQ = 0, COL_S = 64, COL_DPC = 192, COL_DPF = 320;
+struct Misc {
+  uint64_t q_full;
+  uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
+  uint64_t s_full, ds_full, done, drain;
+  uint32_t tmem_base;
+  int abort;
+  uint32_t uni[64], inter[64];  // OR / AND of the tile's selection rows
+  // followed by the selection rows (64 words each)
+};
+}  // namespace dqm
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    bwd_dq_tcm_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOc,
+                      const __grid_constant__ CUtensorMap tmF, TcmBwdParams p) {
+  using namespace dqm;
+  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  Misc& M = *reinterpret_cast<Misc*>(smem + OFF_MISC);
+  uint32_t (*sel)[64] = reinterpret_cast<uint32_t (*)[64]>(smem + OFF_MISC + sizeof(Misc));
+  volatile int* abort = &M.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = (int)(gridDim.x - 1 - blockIdx.x);  // the longest rows first
+  const int h = blockIdx.y, b = blockIdx.z, kvh = h / p.g;
+  const int q0 = qt * TILE;
+  const int ib0 = q0 >> p.ls;
+  const int nsel = sel_rows_tile(p.per_token, p.ls);
+  const int rph = p.per_token ? p.N : p.n;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&M.q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&M.k_full[s], 1);
+      mbar_init(&M.k_empty[s], 1);
+      mbar_init(&M.v_full[s], 1);
+      mbar_init(&M.v_empty[s], 1);
+    }
+    mbar_init(&M.s_full, 1);
+    mbar_init(&M.ds_full, 8);
+    mbar_init(&M.done, 1);
+    mbar_init(&M.drain, 1);
+    M.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(&M.tmem_base, 512);
+    tmem_relinquish();
+  }
+  const int nvalid = p.per_token ? min(TILE, p.N - q0) : min(nsel, p.n - ib0);
+  for (int e = threadIdx.x; e < nsel * 64; e += NTHREADS) {
+    const int r = e >> 6, w = e & 63;
+    uint32_t v = 0u;
+    if (r < nvalid && w < p.words) {
+      const int64_t mrow = p.per_token ? (int64_t)q0 + r : (int64_t)ib0 + r;
+      v = p.mask[(((int64_t)b * p.Hq + h) * rph + mrow) * p.words + w];
+    }
+    sel[r][w] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    uint32_t o = 0u, a = ~0u;
+    for (int r = 0; r < nvalid; ++r) {
+      o |= sel[r][threadIdx.x];
+      a &= sel[r][threadIdx.x];
+    }
+    M.uni[threadIdx.x] = o;
+    M.inter[threadIdx.x] = a;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // Whether some row of the tile can have a selected / dropped key in key tile j.
+  auto flags = [&](int j, bool& anyA, bool& anyD) {
+    anyA = anyD = false;
+#pragma unroll
+    for (int sub = 0; sub < 2; ++sub) {
+      const int u = j * TILE + 64 * sub;
+      const int jb = u >> p.ls;
+      const int nb = p.ls >= 6 ? 1 : (64 >> p.ls);
+      const uint32_t m = ((1u << nb) - 1u) << (jb & 31);
+      anyA |= (M.uni[jb >> 5] & m) != 0u;
+      anyD |= (M.inter[jb >> 5] & m) != m;
+    }
+  };
+
+  const int T = qt + 1;  // causal key tiles
+  const uint32_t tmem = M.tmem_base;
+  uint8_t* sQ = smem + OFF_Q;
+  uint8_t* sOc = smem + OFF_OC;
+  uint8_t* sF = smem + OFF_F;
+  uint8_t* sK = smem + OFF_K;
+  uint8_t* sV = smem + OFF_V;
+
+  if (warp == WARP_TMA) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      mbar_expect_tx(&M.q_full, 3 * TB);
+      tma_load_4d(sQ, &tmQ, &M.q_full, 0, q0, h, b);
+      tma_load_4d(sOc, &tmOc, &M.q_full, 0, q0, h, b);
+      tma_load_4d(sF, &tmF, &M.q_full, 0, q0, h, b);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < T; ++j) {
+        const int st = j % NS;
+        const uint32_t use = (uint32_t)(j / NS);
+        if (j >= NS && !mbar_wait(&M.k_empty[st], (use - 1) & 1u, abort)) break;
+        mbar_expect_tx(&M.k_full[st], TB);
+        tma_load_4d(sK + st * TB, &tmK, &M.k_full[st], 0, j * TILE, kvh, b);
+        k_issued = j + 1;
+        if (j >= NS && !mbar_wait(&M.v_empty[st], (use - 1) & 1u, abort)) break;
+        mbar_expect_tx(&M.v_full[st], TB);
+        tma_load_4d(sV + st * TB, &tmV, &M.v_full[st], 0, j * TILE, kvh, b);
+        v_issued = j + 1;
+      }
+      int dummy = 0;
+      mbar_wait(&M.q_full, 0, &dummy);
+      for (int j = (k_issued > NS ? k_issued - NS : 0); j < k_issued; ++j) {
+        dummy = 0;
+        mbar_wait(&M.k_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
+      }
+      for (int j = (v_issued > NS ? v_issued - NS : 0); j < v_issued; ++j) {
+        dummy = 0;
+        mbar_wait(&M.v_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      const uint32_t aq = smem_u32(sQ), aoc = smem_u32(sOc), af = smem_u32(sF);
+      bool ok = mbar_wait(&M.q_full, 0, abort);
+      for (int j = 0; ok && j < T; ++j) {
+        const int st = j % NS;
+        const uint32_t ph = (uint32_t)(j / NS) & 1u;
+        bool anyA, anyD;
+        flags(j, anyA, anyD);
+        const uint32_t ak = smem_u32(sK + st * TB), av = smem_u32(sV + st * TB);
+        if (!mbar_wait(&M.k_full[st], ph, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_ss_d64(tmem + COL_S, aq, ak);
+        if (!mbar_wait(&M.v_full[st], ph, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (anyA) mma_ss_d64(tmem + COL_DPC, aoc, av);
+        if (anyD) mma_ss_d64(tmem + COL_DPF, af, av);
+        tc_commit(&M.s_full);
+        tc_commit(&M.v_empty[st]);
+        if (!mbar_wait(&M.ds_full, (uint32_t)j & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_ts_acc(tmem + COL_DQ, tmem + COL_S, ak, j > 0);
+        tc_commit(&M.k_empty[st]);
+      }
+      tc_commit(&M.done);
+      tc_commit(&M.drain);
+      int dummy = 0;
+      mbar_wait(&M.drain, 0, &dummy);
+    }
+  } else {
+    const int quarter = warp & 3, ch = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const int t = q0 + row;
+    const bool valid = t < p.N;
+    const uint32_t* selw = sel[p.per_token ? row : min((t >> p.ls) - ib0, nsel - 1)];
+    const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + t;
+    const float lse2 = valid ? p.lse[ro] * kLog2e : 0.f;
+    const float Dc = valid ? p.Dc[ro] : 0.f, Df = valid ? p.Df[ro] : 0.f;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      if (!mbar_wait(&M.s_full, (uint32_t)j & 1u, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      bool anyA, anyD;
+      flags(j, anyA, anyD);
+      const int u0 = j * TILE + 64 * ch;  // first key of this warp's columns
+      const unsigned long long km = tile_keep_mask_p2(selw, u0, p.ls);
+      const int lim = valid ? t - u0 : -1;  // keys c <= lim are causal
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t col = 64 * ch + 32 * hh;
+        uint32_t s[32], pc[32], pf[32];
+        tmem_ld32(lane_base + COL_S + col, s);
+        if (anyA) tmem_ld32(lane_base + COL_DPC + col, pc);
+        if (anyD) tmem_ld32(lane_base + COL_DPF + col, pf);
+        tmem_wait_ld();
+        uint32_t ds[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float v[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kc = 32 * hh + c + e;  // key within the warp's 64
+            const bool inA = (km >> (kc & ~15)) & 1ull;
+            const bool live = kc <= lim;
+            const float pv = ex2(fmaf(__uint_as_float(s[c + e]), p.c, -lse2));
+            const float dpx = inA ? __uint_as_float(pc[c + e]) - Dc : __uint_as_float(pf[c + e]) - Df;
+            v[e] = live ? pv * dpx : 0.f;
+          }
+          ds[c / 2] = pack_bf16(v[0], v[1]);
+        }
+        tmem_st16(lane_base + COL_S + 64 * ch + 16 * hh, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.ds_full);
+    }
+    if (ok && mbar_wait(&M.done, 0, abort)) {
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld32(lane_base + COL_DQ + 32 * ch, r);
+      tmem_wait_ld();
+      if (valid) {
+        uint32_t o[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          o[c] = pack_bf16(__uint_as_float(r[2 * c]) * p.scale, __uint_as_float(r[2 * c + 1]) * p.scale);
+        uint4* d4 = reinterpret_cast<uint4*>(row_ptr_w<bf16>(p.dq, b, h, t) + 32 * ch);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) d4[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (M.abort && threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_TIMEOUT);
+  if (warp == WARP_MMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ================================================================ dK, dV
+namespace dkvm {
+constexpr int NS = 2;
+// A stage: the step's Q, dO_c and dh_f tiles, then lse, D_c, D_f (128 floats
+// each) and the 128 query rows' selection words that cover this key tile.
+constexpr int SC = TILE * 4;
+constexpr int STAGE = 3 * TB + 4 * SC;
+constexpr int OFF_K = 0, OFF_V = TB, OFF_STAGE = 2 * TB;
+constexpr int OFF_MISC = OFF_STAGE + NS * STAGE;
+constexpr uint32_t COL_DK = 0, COL_DV = 64, COL_S = 128, COL_DPC = 256, COL_DPF = 384;
+struct Misc {
+  uint64_t kv_full;
+  uint64_t q_full[NS], q_empty[NS];
+  uint64_t s_full, p_full, done, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
+}  // namespace dkvm
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    bwd_dkv_tcm_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOc,
+                       const __grid_constant__ CUtensorMap tmF, TcmBwdParams p) {
+  using namespace dkvm;
+  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  Misc& M = *reinterpret_cast<Misc*>(smem + OFF_MISC);
+  volatile int* abort = &M.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = (int)blockIdx.x;  // the most query tiles first
+  const int chunks = p.g / p.hpc;
+  const int kvh = blockIdx.y / chunks, chunk = blockIdx.y % chunks;
+  const int b = blockIdx.z;
+  const int Hkv = p.Hq / p.g;
+  const int u0 = kt * TILE;
+  const int nq = p.NT - kt;  // causal query tiles per head
+  const int T = p.hpc * nq;  // steps: hh * nq + (qt - kt)
+  const int rph = p.per_token ? p.N : p.n;
+  const int wi = (u0 >> p.ls) >> 5;  // the selection word holding this key tile's blocks
+  const int nbt = p.ls >= 7 ? 1 : (TILE >> p.ls);
+  const uint32_t tbm = ((nbt >= 32 ? 0u : (1u << nbt)) - 1u) << ((u0 >> p.ls) & 31);
+  auto stage_ptr = [&](int st) { return smem + OFF_STAGE + st * STAGE; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(&M.kv_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&M.q_full[s], 1);
+      mbar_init(&M.q_empty[s], 1);
+    }
+    mbar_init(&M.s_full, 1);
+    mbar_init(&M.p_full, 8);
+    mbar_init(&M.done, 1);
+    mbar_init(&M.drain, 1);
+    M.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(&M.tmem_base, 512);
+    tmem_relinquish();
+  }
+  // Scalar slots of ragged query tiles stay finite (their columns are masked).
+  for (int i = threadIdx.x; i < NS * 4 * TILE; i += NTHREADS)
+    reinterpret_cast<float*>(stage_ptr(i / (4 * TILE)) + 3 * TB)[i % (4 * TILE)] = 0.f;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = M.tmem_base;
+  uint8_t* sK = smem + OFF_K;
+  uint8_t* sV = smem + OFF_V;
+  auto decode = [&](int j, int& h, int& qt) {
+    h = (kvh * chunks + chunk) * p.hpc + j / nq;
+    qt = kt + j % nq;
+  };
+  // Whether some query of the step selected / dropped some key block of the tile.
+  auto step_flags = [&](const uint32_t* words, bool& anyA, bool& anyD) {
+    bool a = false, d = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w = words[lane + 32 * i] & tbm;
+      a |= w != 0u;
+      d |= w != tbm;
+    }
+    anyA = __any_sync(0xffffffffu, a);
+    anyD = __any_sync(0xffffffffu, d);
+  };
+
+  if (warp == WARP_TMA) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmOc);
+      prefetch_tensormap(&tmF);
+      mbar_expect_tx(&M.kv_full, 2 * TB);
+      tma_load_4d(sK, &tmK, &M.kv_full, 0, u0, kvh, b);
+      tma_load_4d(sV, &tmV, &M.kv_full, 0, u0, kvh, b);
+    }
+    int issued = 0;
+    for (int j = 0; j < T; ++j) {
+      const int st = j % NS;
+      bool okw = true;
+      if (lane == 0 && j >= NS) okw = mbar_wait(&M.q_empty[st], (uint32_t)(j / NS - 1) & 1u, abort);
+      if (!__shfl_sync(0xffffffffu, okw ? 1 : 0, 0)) break;
+      int h, qt;
+      decode(j, h, qt);
+      const int t0 = qt * TILE;
+      const int valid = min(TILE, p.N - t0);  // a multiple of 64
+      uint8_t* sp_ = stage_ptr(st);
+      // selection words of the step's query rows (0 past the end)
+      uint32_t* words = reinterpret_cast<uint32_t*>(sp_ + 3 * TB + 3 * SC);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane + 32 * i;
+        uint32_t w = 0u;
+        if (r < valid) {
+          const int64_t mrow = p.per_token ? (int64_t)t0 + r : (int64_t)((t0 + r) >> p.ls);
+          w = p.mask[(((int64_t)b * p.Hq + h) * rph + mrow) * p.words + wi];
+        }
+        words[r] = w;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const int64_t ro = ((int64_t)b * p.Hq + h) * p.N + t0;
+        mbar_expect_tx(&M.q_full[st], 3 * TB + 3 * (uint32_t)valid * 4);
+        tma_load_4d(sp_, &tmQ, &M.q_full[st], 0, t0, h, b);
+        tma_load_4d(sp_ + TB, &tmOc, &M.q_full[st], 0, t0, h, b);
+        tma_load_4d(sp_ + 2 * TB, &tmF, &M.q_full[st], 0, t0, h, b);
+        bulk_load(sp_ + 3 * TB, p.lse + ro, (uint32_t)valid * 4, &M.q_full[st]);
+        bulk_load(sp_ + 3 * TB + SC, p.Dc + ro, (uint32_t)valid * 4, &M.q_full[st]);
+        bulk_load(sp_ + 3 * TB + 2 * SC, p.Df + ro, (uint32_t)valid * 4, &M.q_full[st]);
+      }
+      issued = j + 1;
+    }
+    if (lane == 0) {
+      int dummy = 0;
+      mbar_wait(&M.kv_full, 0, &dummy);
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) {
+        dummy = 0;
+        mbar_wait(&M.q_full[j % NS], (uint32_t)(j / NS) & 1u, &dummy);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    const uint32_t ak = smem_u32(sK), av = smem_u32(sV);
+    bool ok = true;
+    if (lane == 0) ok = T == 0 || mbar_wait(&M.kv_full, 0, abort);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    bool started_dv = false, started_dk = false;
+    for (int j = 0; ok && j < T; ++j) {
+      const int st = j % NS;
+      // every lane reads the step's selection words: every lane acquires the stage
+      ok = mbar_wait(&M.q_full[st], (uint32_t)(j / NS) & 1u, abort);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint8_t* sp_ = stage_ptr(st);
+      bool anyA, anyD;
+      step_flags(reinterpret_cast<const uint32_t*>(sp_ + 3 * TB + 3 * SC), anyA, anyD);
+      const uint32_t aq = smem_u32(sp_), aoc = smem_u32(sp_ + TB), af = smem_u32(sp_ + 2 * TB);
+      if (lane == 0) {
+        mma_ss_d64(tmem + COL_S, ak, aq);
+        if (anyA) mma_ss_d64(tmem + COL_DPC, av, aoc);
+        if (anyD) mma_ss_d64(tmem + COL_DPF, av, af);
+        tc_commit(&M.s_full);
+        ok = mbar_wait(&M.p_full, (uint32_t)j & 1u, abort);
+        if (ok) {
+          tc_fence_after();
+          if (anyA) {
+            mma_ts_acc(tmem + COL_DV, tmem + COL_S, aoc, started_dv);
+            started_dv = true;
+          }
+          if (anyD) {
+            mma_ts_acc(tmem + COL_DV, tmem + COL_DPF, af, started_dv);
+            started_dv = true;
+          }
+          mma_ts_acc(tmem + COL_DK, tmem + COL_DPC, aq, started_dk);
+          started_dk = true;
+          tc_commit(&M.q_empty[st]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0) {
+      tc_commit(&M.done);
+      tc_commit(&M.drain);
+      int dummy = 0;
+      mbar_wait(&M.drain, 0, &dummy);
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3, ch = warp >> 2;  // key lanes 32*quarter.., query columns 64*ch..
+    const int r = quarter * 32 + lane;              // key row within the tile
+    const int bp = ((u0 + r) >> p.ls) & 31;        // its block's bit in a selection word
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int st = j % NS;
+      if (!mbar_wait(&M.q_full[st], (uint32_t)(j / NS) & 1u, abort) ||
+          !mbar_wait(&M.s_full, (uint32_t)j & 1u, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      int h, qt;
+      decode(j, h, qt);
+      const bool diag = qt == kt;
+      const int lim = p.N - qt * TILE;  // columns c < lim are queries of the sequence
+      const uint8_t* sp_ = stage_ptr(st);
+      const float* L = reinterpret_cast<const float*>(sp_ + 3 * TB);
+      const float* DcS = reinterpret_cast<const float*>(sp_ + 3 * TB + SC);
+      const float* DfS = reinterpret_cast<const float*>(sp_ + 3 * TB + 2 * SC);
+      const uint32_t* words = reinterpret_cast<const uint32_t*>(sp_ + 3 * TB + 3 * SC);
+      bool anyA, anyD;
+      step_flags(words, anyA, anyD);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c0 = 64 * ch + 32 * hh;
+        uint32_t s[32], pc[32], pf[32];
+        tmem_ld32(lane_base + COL_S + c0, s);
+        if (anyA) tmem_ld32(lane_base + COL_DPC + c0, pc);
+        if (anyD) tmem_ld32(lane_base + COL_DPF + c0, pf);
+        tmem_wait_ld();
+        uint32_t pa[16], pd[16], ds[16];
+#pragma unroll
+        for (int k8 = 0; k8 < 32; k8 += 8) {
+          // the eight columns' scalars and selection words as 16-byte loads
+          float lv[8], dcv[8], dfv[8];
+          uint32_t wv[8];
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const float4 l4 = *reinterpret_cast<const float4*>(L + c0 + k8 + 4 * v);
+            const float4 c4 = *reinterpret_cast<const float4*>(DcS + c0 + k8 + 4 * v);
+            const float4 f4 = *reinterpret_cast<const float4*>(DfS + c0 + k8 + 4 * v);
+            const uint4 w4 = *reinterpret_cast<const uint4*>(words + c0 + k8 + 4 * v);
+            lv[4 * v] = l4.x; lv[4 * v + 1] = l4.y; lv[4 * v + 2] = l4.z; lv[4 * v + 3] = l4.w;
+            dcv[4 * v] = c4.x; dcv[4 * v + 1] = c4.y; dcv[4 * v + 2] = c4.z; dcv[4 * v + 3] = c4.w;
+            dfv[4 * v] = f4.x; dfv[4 * v + 1] = f4.y; dfv[4 * v + 2] = f4.z; dfv[4 * v + 3] = f4.w;
+            wv[4 * v] = w4.x; wv[4 * v + 1] = w4.y; wv[4 * v + 2] = w4.z; wv[4 * v + 3] = w4.w;
+          }
+#pragma unroll
+          for (int c = 0; c < 8; c += 2) {
+            float va[2], vd[2], vs[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int i = k8 + c + e;  // column within the 32
+              const int col = c0 + i;
+              const bool live = col < lim && (!diag || r <= col);
+              const bool inA = (wv[c + e] >> bp) & 1u;
+              const float pv = ex2(fmaf(__uint_as_float(s[i]), p.c, -lv[c + e] * kLog2e));
+              const float dpx = inA ? __uint_as_float(pc[i]) - dcv[c + e] : __uint_as_float(pf[i]) - dfv[c + e];
+              va[e] = (live && inA) ? pv : 0.f;
+              vd[e] = (live && !inA) ? pv : 0.f;
+              vs[e] = live ? pv * dpx : 0.f;
+            }
+            pa[(k8 + c) / 2] = pack_bf16(va[0], va[1]);
+            pd[(k8 + c) / 2] = pack_bf16(vd[0], vd[1]);
+            ds[(k8 + c) / 2] = pack_bf16(vs[0], vs[1]);
+          }
+        }
+        tmem_st16(lane_base + COL_S + 64 * ch + 16 * hh, pa);
+        if (anyD) tmem_st16(lane_base + COL_DPF + 64 * ch + 16 * hh, pd);
+        tmem_st16(lane_base + COL_DPC + 64 * ch + 16 * hh, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.p_full);
+    }
+    if (ok && (T == 0 || mbar_wait(&M.done, 0, abort))) {
+      tc_fence_after();
+      const int u = u0 + r;
+      uint32_t rk[32], rv[32];
+      tmem_ld32(lane_base + COL_DK + 32 * ch, rk);
+      tmem_ld32(lane_base + COL_DV + 32 * ch, rv);
+      tmem_wait_ld();
+      if (T == 0) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) rk[c] = rv[c] = 0u;
+      }
+      if (u < p.N) {
+        if (p.part == nullptr) {
+          uint32_t ok_[16], ov_[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            ok_[c] = pack_bf16(__uint_as_float(rk[2 * c]) * p.scale, __uint_as_float(rk[2 * c + 1]) * p.scale);
+            ov_[c] = pack_bf16(__uint_as_float(rv[2 * c]), __uint_as_float(rv[2 * c + 1]));
+          }
+          uint4* dk4 = reinterpret_cast<uint4*>(row_ptr_w<bf16>(p.dk, b, kvh, u) + 32 * ch);
+          uint4* dv4 = reinterpret_cast<uint4*>(row_ptr_w<bf16>(p.dv, b, kvh, u) + 32 * ch);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            dk4[q] = make_uint4(ok_[4 * q], ok_[4 * q + 1], ok_[4 * q + 2], ok_[4 * q + 3]);
+            dv4[q] = make_uint4(ov_[4 * q], ov_[4 * q + 1], ov_[4 * q + 2], ov_[4 * q + 3]);
+          }
+        } else {
+          // fp32 partials [chunk][2][B][Hkv][N][64] (dK unscaled, dV)
+          const int64_t plane = (int64_t)gridDim.z * Hkv * p.N * HD;
+          float* pk = p.part + (int64_t)chunk * 2 * plane + (((int64_t)b * Hkv + kvh) * p.N + u) * HD + 32 * ch;
+          float* pv = pk + plane;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            reinterpret_cast<float4*>(pk)[q] = make_float4(__uint_as_float(rk[4 * q]), __uint_as_float(rk[4 * q + 1]),
+                                                           __uint_as_float(rk[4 * q + 2]), __uint_as_float(rk[4 * q + 3]));
+            reinterpret_cast<float4*>(pv)[q] = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
+                                                           __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (M.abort && threadIdx.x == 0) atomicCAS(p.status, 0, (int)SSA_ERR_TIMEOUT);
+  if (warp == WARP_MMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool bwd_tcm_supported(const Dims& D) { return D.dtype == SSA_BF16 && D.d == 64 && D.n <= 2048; }
+
+cudaError_t launch_bwd_tcm(const Dims& D, const BwdArgs& a, const void* dhf_bf16, const void* doc_bf16, int hpc,
+                           int32_t* status, cudaStream_t st) {
+  if (!bwd_tcm_supported(D) || a.sparse_only) return cudaErrorNotSupported;
+  const int64_t rs = (int64_t)D.N * HD;
+  const TensorRef rdhf{dhf_bf16, (int64_t)D.Hq * rs, rs, HD};
+  const TensorRef rdoc{doc_bf16, (int64_t)D.Hq * rs, rs, HD};
+  CUtensorMap mq, mk, mv, moc, mf;
+  if (!make_tma_map_bf16(&mq, a.q, D.B, D.Hq, D.N, TILE, HD) || !make_tma_map_bf16(&mk, a.k, D.B, D.Hkv, D.N, TILE, HD) ||
+      !make_tma_map_bf16(&mv, a.v, D.B, D.Hkv, D.N, TILE, HD) || !make_tma_map_bf16(&moc, rdoc, D.B, D.Hq, D.N, TILE, HD) ||
+      !make_tma_map_bf16(&mf, rdhf, D.B, D.Hq, D.N, TILE, HD))
+    return cudaErrorInvalidValue;
+  TcmBwdParams p;
+  p.dq = a.dq;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.lse = a.lse_full;
+  p.Dc = a.Dc;
+  p.Df = a.Df;
+  p.mask = a.mask;
+  p.words = a.words;
+  p.status = status;
+  p.Hq = D.Hq;
+  p.g = D.g;
+  p.N = D.N;
+  p.n = D.n;
+  p.ls = __builtin_ctz((unsigned)D.s);
+  p.per_token = D.per_token;
+  p.hpc = hpc;
+  p.NT = (D.N + TILE - 1) / TILE;
+  p.c = D.scale * kLog2e;
+  p.scale = D.scale;
+  const int chunks = D.g / hpc;
+  p.part = chunks > 1 ? a.kvpart : nullptr;
+  const int smem_dkv = dkvm::OFF_MISC + (int)sizeof(dkvm::Misc) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkv_tcm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv);
+  if (e != cudaSuccess) return e;
+  bwd_dkv_tcm_kernel<<<dim3(p.NT, D.Hkv * chunks, D.B), NTHREADS, smem_dkv, st>>>(mq, mk, mv, moc, mf, p);
+  count_launches(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int smem_dq =
+      dqm::OFF_MISC + (int)sizeof(dqm::Misc) + sel_rows_tile(D.per_token, p.ls) * 64 * (int)sizeof(uint32_t) + 1024;
+  e = cudaFuncSetAttribute(bwd_dq_tcm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq);
+  if (e != cudaSuccess) return e;
+  bwd_dq_tcm_kernel<<<dim3(p.NT, D.Hq, D.B), NTHREADS, smem_dq, st>>>(mq, mk, mv, moc, mf, p);
+  count_launches(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (chunks > 1) e = launch_kvsum(D, a, a.kvpart, chunks, st);
+  return e;
+}
+
+}  // namespace ssa

@@ -306,7 +306,7 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
   }
   if (bwd_mma_supported(D)) {
     a.kvpart = at<float>(ws, L.kvpart);
-    return from_cuda(launch_bwd_mma(D, a, st));
+    return from_cuda(launch_bwd_mma(D, a, device_status_ptr(), st));
   }
   e = launch_bwd_pre(D, a, st);
   if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
@@ -420,7 +420,7 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
   }
   if (bwd_mma_supported(D)) {
     a.kvpart = at<float>(ws, L.kvpart);
-    return from_cuda(launch_bwd_mma(D, a, st));
+    return from_cuda(launch_bwd_mma(D, a, device_status_ptr(), st));
   }
   e = launch_bwd_pre(D, a, st);
   if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);

@@ -207,7 +207,14 @@ cudaError_t launch_bwd_simt(const Dims& D, const BwdArgs& a, cudaStream_t st);
 bool bwd_mma_supported(const Dims& D);
 int bwd_mma_heads_per_cta(const Dims& D);
 size_t bwd_mma_partial_bytes(const Dims& D);  // workspace for a.kvpart (0: none needed)
-cudaError_t launch_bwd_mma(const Dims& D, const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_mma(const Dims& D, const BwdArgs& a, int32_t* status, cudaStream_t st);
+// Ordered sum of fp32 dK / dV partials (chunks of a kv group) into a.dk, a.dv.
+cudaError_t launch_kvsum(const Dims& D, const BwdArgs& a, const float* part, int chunks, cudaStream_t st);
+// Tensor-core (tcgen05) dual backward with per-row selection masks, bf16,
+// d = 64; takes the bf16 dh_f / dO_c written by the warp-level preprocess.
+bool bwd_tcm_supported(const Dims& D);
+cudaError_t launch_bwd_tcm(const Dims& D, const BwdArgs& a, const void* dhf_bf16, const void* doc_bf16, int hpc,
+                           int32_t* status, cudaStream_t st);
 
 struct DecodeArgs {
   TensorRef q, k, v, h;  // q, h: [B,Hq,1,d] (prefill: q = the prompt's Q [B,Hq,N,d]); k, v: caches [B,Hkv,N,d]
