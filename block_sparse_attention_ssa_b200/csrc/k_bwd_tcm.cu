@@ -23,10 +23,12 @@
 //        the row's selection, written as bf16 over the warp's own S columns,
 //        then dQ += dS K.
 //   dkv  one 128-key tile per CTA, walking a chunk of at most 4 query heads
-//        of its kv group and their causal query tiles.  TMEM: dK [0,64),
-//        dV [64,128), S^T [128,256), dP_c^T [256,384), dP_f^T [384,512).  Per
-//        step: S^T = K Q^T, dP_c^T = V dO_c^T, dP_f^T = V dh_f^T, then P_A^T
-//        over S^T, P_D^T over dP_f^T and dS^T over dP_c^T (each warp packs into
+//        of its kv group and their causal query tiles, 64 queries (a half
+//        step) at a time.  TMEM: dK [0,64), dV [64,128), then two buffers of
+//        S^T, dP_c^T, dP_f^T (64 columns each), so that the products of the
+//        next half step run while this one is computed.  Per half step:
+//        S^T = K Q^T, dP_c^T = V dO_c^T, dP_f^T = V dh_f^T, then P_A^T over
+//        S^T, P_D^T over dP_f^T and dS^T over dP_c^T (each warp packs into
 //        columns it has already read), dV += P_A^T dO_c + P_D^T dh_f and
 //        dK += dS^T Q.  A query's selection word decides, per key block, the
 //        set of each element.  With more than one chunk per group the chunks
@@ -79,6 +81,27 @@ __device__ __forceinline__ void mma_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uin
 #pragma unroll
   for (int kk = 0; kk < TILE / 16; ++kk)
     mma_ts(d_tmem, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), smem_desc_sw128(b_smem + kk * 2048, TB, 1024), IDESC_ACC,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// Half steps of 64 along the MMA's N / reduction dimension.
+constexpr uint32_t IDESC_S64 = idesc_bf16_f32(TILE, 64, false, false);  // both K-major, N = 64
+
+// D (128 x 64) = A (128 x 64) B^T, B = 64 rows of a K-major smem tile.
+__device__ __forceinline__ void mma_ss_n64(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk)
+    mma_ss(d_tmem, smem_desc_sw128(a_smem + kk * 32, 16, 1024), smem_desc_sw128(b_smem + kk * 32, 16, 1024),
+           IDESC_S64, kk > 0 ? 1u : 0u);
+}
+
+// D (128 x 64) (+)= A (TMEM, 128 rows x 64 reduction as bf16 pairs: indices
+// 0-31 at columns a..a+15, 32-63 at a+32..a+47) x B (64 rows of a smem tile,
+// rows = reduction index).
+__device__ __forceinline__ void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    mma_ts(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1), smem_desc_sw128(b_smem + kk * 2048, TB, 1024), IDESC_ACC,
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -349,11 +372,13 @@ constexpr int SC = TILE * 4;
 constexpr int STAGE = 3 * TB + 4 * SC;
 constexpr int OFF_K = 0, OFF_V = TB, OFF_STAGE = 2 * TB;
 constexpr int OFF_MISC = OFF_STAGE + NS * STAGE;
-constexpr uint32_t COL_DK = 0, COL_DV = 64, COL_S = 128, COL_DPC = 256, COL_DPF = 384;
+// TMEM: dK, dV, then two buffers of one 64-query half step each: S^T, dP_c^T,
+// dP_f^T (64 columns apiece) at COL_BUF + 192 b.
+constexpr uint32_t COL_DK = 0, COL_DV = 64, COL_BUF = 128;
 struct Misc {
   uint64_t kv_full;
   uint64_t q_full[NS], q_empty[NS];
-  uint64_t s_full, p_full, done, drain;
+  uint64_t s_full[2], p_full[2], done, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -391,8 +416,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&M.q_full[s], 1);
       mbar_init(&M.q_empty[s], 1);
     }
-    mbar_init(&M.s_full, 1);
-    mbar_init(&M.p_full, 8);
+    for (int bb = 0; bb < 2; ++bb) {
+      mbar_init(&M.s_full[bb], 1);
+      mbar_init(&M.p_full[bb], 8);
+    }
     mbar_init(&M.done, 1);
     mbar_init(&M.drain, 1);
     M.abort = 0;
@@ -416,11 +443,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     h = (kvh * chunks + chunk) * p.hpc + j / nq;
     qt = kt + j % nq;
   };
-  // Whether some query of the step selected / dropped some key block of the tile.
-  auto step_flags = [&](const uint32_t* words, bool& anyA, bool& anyD) {
+  // Whether some of the 64 queries of a half step selected / dropped some key
+  // block of the tile (words: the half's 64 selection words).
+  auto half_flags = [&](const uint32_t* words, bool& anyA, bool& anyD) {
     bool a = false, d = false;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       const uint32_t w = words[lane + 32 * i] & tbm;
       a |= w != 0u;
       d |= w != tbm;
@@ -483,46 +511,77 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (warp == WARP_MMA) {
+    // Half step hs = 2 j + x covers queries 64x.. of step j and uses TMEM
+    // buffer hs & 1: its S^T / dP^T products are issued before the dV / dK
+    // products of half step hs - 1, so they overlap that half step's compute.
     const uint32_t ak = smem_u32(sK), av = smem_u32(sV);
     bool ok = true;
     if (lane == 0) ok = T == 0 || mbar_wait(&M.kv_full, 0, abort);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     bool started_dv = false, started_dk = false;
-    for (int j = 0; ok && j < T; ++j) {
-      const int st = j % NS;
+    bool fA0 = false, fD0 = false, fA1 = false, fD1 = false;  // flags of the half steps in buffers 0 / 1
+    const int H = 2 * T;
+    auto front = [&](int hs) -> bool {
+      const int j = hs >> 1, x = hs & 1, st = j % NS, bsel = hs & 1;
       // every lane reads the step's selection words: every lane acquires the stage
-      ok = mbar_wait(&M.q_full[st], (uint32_t)(j / NS) & 1u, abort);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
+      const bool okf = mbar_wait(&M.q_full[st], (uint32_t)(j / NS) & 1u, abort);
+      if (!__all_sync(0xffffffffu, okf)) return false;
       tc_fence_after();
       uint8_t* sp_ = stage_ptr(st);
       bool anyA, anyD;
-      step_flags(reinterpret_cast<const uint32_t*>(sp_ + 3 * TB + 3 * SC), anyA, anyD);
-      const uint32_t aq = smem_u32(sp_), aoc = smem_u32(sp_ + TB), af = smem_u32(sp_ + 2 * TB);
+      half_flags(reinterpret_cast<const uint32_t*>(sp_ + 3 * TB + 3 * SC) + 64 * x, anyA, anyD);
+      if (bsel) {
+        fA1 = anyA;
+        fD1 = anyD;
+      } else {
+        fA0 = anyA;
+        fD0 = anyD;
+      }
       if (lane == 0) {
-        mma_ss_d64(tmem + COL_S, ak, aq);
-        if (anyA) mma_ss_d64(tmem + COL_DPC, av, aoc);
-        if (anyD) mma_ss_d64(tmem + COL_DPF, av, af);
-        tc_commit(&M.s_full);
-        ok = mbar_wait(&M.p_full, (uint32_t)j & 1u, abort);
-        if (ok) {
+        const uint32_t base = tmem + COL_BUF + 192 * bsel, off = 8192u * x;
+        mma_ss_n64(base, ak, smem_u32(sp_) + off);
+        if (anyA) mma_ss_n64(base + 64, av, smem_u32(sp_ + TB) + off);
+        if (anyD) mma_ss_n64(base + 128, av, smem_u32(sp_ + 2 * TB) + off);
+        tc_commit(&M.s_full[bsel]);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto back = [&](int hs) -> bool {
+      const int j = hs >> 1, x = hs & 1, st = j % NS, bsel = hs & 1;
+      const bool anyA = bsel ? fA1 : fA0, anyD = bsel ? fD1 : fD0;
+      bool okb = true;
+      if (lane == 0) {
+        okb = mbar_wait(&M.p_full[bsel], (uint32_t)(hs >> 1) & 1u, abort);
+        if (okb) {
           tc_fence_after();
+          uint8_t* sp_ = stage_ptr(st);
+          const uint32_t base = tmem + COL_BUF + 192 * bsel, off = 8192u * x;
           if (anyA) {
-            mma_ts_acc(tmem + COL_DV, tmem + COL_S, aoc, started_dv);
+            mma_ts_k64(tmem + COL_DV, base, smem_u32(sp_ + TB) + off, started_dv);
             started_dv = true;
           }
           if (anyD) {
-            mma_ts_acc(tmem + COL_DV, tmem + COL_DPF, af, started_dv);
+            mma_ts_k64(tmem + COL_DV, base + 128, smem_u32(sp_ + 2 * TB) + off, started_dv);
             started_dv = true;
           }
-          mma_ts_acc(tmem + COL_DK, tmem + COL_DPC, aq, started_dk);
+          mma_ts_k64(tmem + COL_DK, base + 64, smem_u32(sp_) + off, started_dk);
           started_dk = true;
-          tc_commit(&M.q_empty[st]);
+          if (x == 1) tc_commit(&M.q_empty[st]);
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      return __shfl_sync(0xffffffffu, okb ? 1 : 0, 0) != 0;
+    };
+    if (ok && H > 0) ok = front(0);
+    for (int hs = 0; ok && hs < H; ++hs) {
+      if (hs + 1 < H && !front(hs + 1)) {
+        ok = false;
+        break;
+      }
+      if (!back(hs)) {
+        ok = false;
+        break;
+      }
     }
     if (lane == 0) {
       tc_commit(&M.done);
@@ -532,15 +591,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     __syncwarp();
   } else {
-    const int quarter = warp & 3, ch = warp >> 2;  // key lanes 32*quarter.., query columns 64*ch..
+    const int quarter = warp & 3, ch = warp >> 2;  // key lanes 32*quarter.., query columns 32*ch.. of a half
     const int r = quarter * 32 + lane;              // key row within the tile
     const int bp = ((u0 + r) >> p.ls) & 31;        // its block's bit in a selection word
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int st = j % NS;
+    for (int hs = 0; hs < 2 * T; ++hs) {
+      const int j = hs >> 1, x = hs & 1, st = j % NS, bsel = hs & 1;
       if (!mbar_wait(&M.q_full[st], (uint32_t)(j / NS) & 1u, abort) ||
-          !mbar_wait(&M.s_full, (uint32_t)j & 1u, abort)) {
+          !mbar_wait(&M.s_full[bsel], (uint32_t)(hs >> 1) & 1u, abort)) {
         ok = false;
         break;
       }
@@ -555,60 +614,59 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float* DfS = reinterpret_cast<const float*>(sp_ + 3 * TB + 2 * SC);
       const uint32_t* words = reinterpret_cast<const uint32_t*>(sp_ + 3 * TB + 3 * SC);
       bool anyA, anyD;
-      step_flags(words, anyA, anyD);
+      half_flags(words + 64 * x, anyA, anyD);
+      const uint32_t base = lane_base + COL_BUF + 192 * bsel;
+      const int c0 = 64 * x + 32 * ch;  // first query column (within the tile) of this warp
+      uint32_t s[32], pc[32], pf[32];
+      tmem_ld32(base + 32 * ch, s);
+      if (anyA) tmem_ld32(base + 64 + 32 * ch, pc);
+      if (anyD) tmem_ld32(base + 128 + 32 * ch, pf);
+      tmem_wait_ld();
+      uint32_t pa[16], pd[16], ds[16];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int c0 = 64 * ch + 32 * hh;
-        uint32_t s[32], pc[32], pf[32];
-        tmem_ld32(lane_base + COL_S + c0, s);
-        if (anyA) tmem_ld32(lane_base + COL_DPC + c0, pc);
-        if (anyD) tmem_ld32(lane_base + COL_DPF + c0, pf);
-        tmem_wait_ld();
-        uint32_t pa[16], pd[16], ds[16];
+      for (int k8 = 0; k8 < 32; k8 += 8) {
+        // the eight columns' scalars and selection words as 16-byte loads
+        float lv[8], dcv[8], dfv[8];
+        uint32_t wv[8];
 #pragma unroll
-        for (int k8 = 0; k8 < 32; k8 += 8) {
-          // the eight columns' scalars and selection words as 16-byte loads
-          float lv[8], dcv[8], dfv[8];
-          uint32_t wv[8];
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const float4 l4 = *reinterpret_cast<const float4*>(L + c0 + k8 + 4 * v);
-            const float4 c4 = *reinterpret_cast<const float4*>(DcS + c0 + k8 + 4 * v);
-            const float4 f4 = *reinterpret_cast<const float4*>(DfS + c0 + k8 + 4 * v);
-            const uint4 w4 = *reinterpret_cast<const uint4*>(words + c0 + k8 + 4 * v);
-            lv[4 * v] = l4.x; lv[4 * v + 1] = l4.y; lv[4 * v + 2] = l4.z; lv[4 * v + 3] = l4.w;
-            dcv[4 * v] = c4.x; dcv[4 * v + 1] = c4.y; dcv[4 * v + 2] = c4.z; dcv[4 * v + 3] = c4.w;
-            dfv[4 * v] = f4.x; dfv[4 * v + 1] = f4.y; dfv[4 * v + 2] = f4.z; dfv[4 * v + 3] = f4.w;
-            wv[4 * v] = w4.x; wv[4 * v + 1] = w4.y; wv[4 * v + 2] = w4.z; wv[4 * v + 3] = w4.w;
-          }
-#pragma unroll
-          for (int c = 0; c < 8; c += 2) {
-            float va[2], vd[2], vs[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int i = k8 + c + e;  // column within the 32
-              const int col = c0 + i;
-              const bool live = col < lim && (!diag || r <= col);
-              const bool inA = (wv[c + e] >> bp) & 1u;
-              const float pv = ex2(fmaf(__uint_as_float(s[i]), p.c, -lv[c + e] * kLog2e));
-              const float dpx = inA ? __uint_as_float(pc[i]) - dcv[c + e] : __uint_as_float(pf[i]) - dfv[c + e];
-              va[e] = (live && inA) ? pv : 0.f;
-              vd[e] = (live && !inA) ? pv : 0.f;
-              vs[e] = live ? pv * dpx : 0.f;
-            }
-            pa[(k8 + c) / 2] = pack_bf16(va[0], va[1]);
-            pd[(k8 + c) / 2] = pack_bf16(vd[0], vd[1]);
-            ds[(k8 + c) / 2] = pack_bf16(vs[0], vs[1]);
-          }
+        for (int v = 0; v < 2; ++v) {
+          const float4 l4 = *reinterpret_cast<const float4*>(L + c0 + k8 + 4 * v);
+          const float4 c4 = *reinterpret_cast<const float4*>(DcS + c0 + k8 + 4 * v);
+          const float4 f4 = *reinterpret_cast<const float4*>(DfS + c0 + k8 + 4 * v);
+          const uint4 w4 = *reinterpret_cast<const uint4*>(words + c0 + k8 + 4 * v);
+          lv[4 * v] = l4.x; lv[4 * v + 1] = l4.y; lv[4 * v + 2] = l4.z; lv[4 * v + 3] = l4.w;
+          dcv[4 * v] = c4.x; dcv[4 * v + 1] = c4.y; dcv[4 * v + 2] = c4.z; dcv[4 * v + 3] = c4.w;
+          dfv[4 * v] = f4.x; dfv[4 * v + 1] = f4.y; dfv[4 * v + 2] = f4.z; dfv[4 * v + 3] = f4.w;
+          wv[4 * v] = w4.x; wv[4 * v + 1] = w4.y; wv[4 * v + 2] = w4.z; wv[4 * v + 3] = w4.w;
         }
-        tmem_st16(lane_base + COL_S + 64 * ch + 16 * hh, pa);
-        if (anyD) tmem_st16(lane_base + COL_DPF + 64 * ch + 16 * hh, pd);
-        tmem_st16(lane_base + COL_DPC + 64 * ch + 16 * hh, ds);
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+          float va[2], vd[2], vs[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int i = k8 + c + e;  // column within the warp's 32
+            const int col = c0 + i;
+            const bool live = col < lim && (!diag || r <= col);
+            const bool inA = (wv[c + e] >> bp) & 1u;
+            const float pv = ex2(fmaf(__uint_as_float(s[i]), p.c, -lv[c + e] * kLog2e));
+            const float dpx = inA ? __uint_as_float(pc[i]) - dcv[c + e] : __uint_as_float(pf[i]) - dfv[c + e];
+            va[e] = (live && inA) ? pv : 0.f;
+            vd[e] = (live && !inA) ? pv : 0.f;
+            vs[e] = live ? pv * dpx : 0.f;
+          }
+          pa[(k8 + c) / 2] = pack_bf16(va[0], va[1]);
+          pd[(k8 + c) / 2] = pack_bf16(vd[0], vd[1]);
+          ds[(k8 + c) / 2] = pack_bf16(vs[0], vs[1]);
+        }
       }
+      // packed into the first 16 of the warp's own 32 columns of each product
+      tmem_st16(base + 32 * ch, pa);
+      if (anyD) tmem_st16(base + 128 + 32 * ch, pd);
+      tmem_st16(base + 64 + 32 * ch, ds);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&M.p_full);
+      if (lane == 0) mbar_arrive(&M.p_full[bsel]);
     }
     if (ok && (T == 0 || mbar_wait(&M.done, 0, abort))) {
       tc_fence_after();
