@@ -437,8 +437,9 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     peaks, peak_src = load_peaks()
     row_flops = {"fwd_dual": F["fwd"], "bwd_dual": F["bwd"], "dropped_mass": F["dropped"]}
     # bf16 with d = 128 and blocks of 64 / 128 (per-block selection) runs on
-    # the tcgen05 kernels; other bf16 shapes on the warp-level mma.sync
-    # kernels; fp32 on the CUDA-core kernels (fp32 FMA bound)
+    # the first tcgen05 kernels; other bf16 shapes on the tcgen05 kernels with
+    # per-row masks (mma.sync for the d = 128 backward); fp32 on the CUDA-core
+    # kernels (fp32 FMA bound)
     tc_path = w.dtype == "bf16" and w.d == 128 and w.block in (64, 128) and not args.per_token
     mma_path = w.dtype == "bf16" and not tc_path
     if tc_path:
@@ -446,10 +447,11 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
                   "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_tc + finish + bwd_dkv_tc + bwd_dq_tc kernels",
                   "dropped_mass": "entry point ssa_dropped_mass = one kernel (dropped_tc_kernel)"}
     elif mma_path:
-        scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_mma_kernel, mma.sync)",
-                  "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_mma + finish + bwd_dkv_mma + bwd_dq_mma "
-                              "(+ kvsum) kernels (mma.sync)",
-                  "dropped_mass": "entry point ssa_dropped_mass = one kernel (fwd_mma_kernel without V, mma.sync)"}
+        bwd_kernels = ("bwd_dkv_tcm + bwd_dq_tcm (+ kvsum) kernels (tcgen05, per-row masks)" if w.d == 64 else
+                       "bwd_dkv_mma + bwd_dq_mma (+ kvsum) kernels (mma.sync)")
+        scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_tcm_kernel: tcgen05, per-row masks)",
+                  "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_mma + finish + " + bwd_kernels,
+                  "dropped_mass": "entry point ssa_dropped_mass = one kernel (fwd_tcm_kernel without V: tcgen05)"}
     else:
         scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_simt_kernel, CUDA cores)",
                   "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre + finish + bwd_dq + bwd_dkv kernels (CUDA cores)",
@@ -468,8 +470,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
                 "frac": achieved / peaks["bf16_tflops_sustained"],
                 "frac_of_burst": achieved / peaks["bf16_tflops"],
                 "traffic": measured_traffic(r, w.name) if tc_path else None,
-                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); burst {peaks['bf16_tflops']}"
-                               + ("; warp-level mma.sync kernels (legacy tensor path)" if mma_path else "")}
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); burst {peaks['bf16_tflops']}"}
 
     dom = max(row_flops, key=lambda r: row_ms[r])
     roofline = roof(dom)

@@ -39,11 +39,13 @@
  *   {16, 32, 64, 128}; N a multiple of block and of 64; d in {64, 128};
  *   topk >= 1 (a budget above n is clamped: k_eff = min(topk, n));
  *   n <= 2048.  When B*Hq*N == 0 the call is a no-op and returns SSA_OK.
- *   Blocks of 64 and 128 with bf16 and d = 128 (per-block selection) run on
- *   the tcgen05 tensor-core kernels; the other bf16 shapes (d = 64, the
- *   small blocks 16 and 32 of the paper's models, [digest] "Model
- *   Architecture Configuration", and per-token selection) on warp-level
- *   mma.sync tensor-core kernels; fp32 on the CUDA-core kernels.
+ *   bf16 runs on tensor cores: blocks of 64 and 128 with d = 128 and
+ *   per-block selection on the tcgen05 kernels; the other bf16 shapes (d =
+ *   64, the small blocks 16 and 32 of the paper's models, [digest] "Model
+ *   Architecture Configuration", and per-token selection) on tcgen05
+ *   kernels with per-row selection masks (dual forward, dropped mass, d = 64
+ *   backward) and warp-level mma.sync kernels (sparse stream alone, d = 128
+ *   backward); fp32 on the CUDA-core kernels.
  * Errors.  Arguments are checked on the host before anything is enqueued;
  *   a failed check returns SSA_ERR_INVALID_ARG (bad pointer, stride,
  *   alignment or value), SSA_ERR_UNSUPPORTED (a shape outside the list above,
@@ -148,10 +150,10 @@ SSA_API ssa_status_t ssa_select_topk(const ssa_dims_t* dims, const float* scores
  * blocks by its own query, score_j = scale * q_t . kbar_j (j < i, kbar_j the
  * mean of key block j), and keeps Sel(t) = {i} plus the k_eff-1 best (ties to
  * the smaller j; {0..i} when i + 1 <= k_eff).  Every other entry point takes
- * the resulting per-token idx when dims->per_token = 1 (the mma.sync kernels
- * run for bf16, the CUDA-core kernels for fp32; the tcgen05 kernels and
- * ssa_block_scores / ssa_select_topk are per-block only: the former are
- * not used, the latter return SSA_ERR_INVALID_ARG).
+ * the resulting per-token idx when dims->per_token = 1 (the per-row-mask
+ * tensor-core kernels run for bf16, the CUDA-core kernels for fp32;
+ * ssa_block_scores / ssa_select_topk are per-block only and return
+ * SSA_ERR_INVALID_ARG).
  *   idx [B, Hq, N, k_eff] int32 (out): Sel(t) ascending, -1 padded.
  *   ws: workspace of at least ssa_workspace_bytes(dims) bytes (pooled keys). */
 SSA_API ssa_status_t ssa_select_tokens(const ssa_dims_t* dims, const ssa_tensor_t* Q,
