@@ -27,6 +27,9 @@ CASES = {
     "bf16_s16_g16_d64": (1, 16, 1, 768, 64, 16, 16, "bf16"),
     "bf16_s32_d128": (2, 4, 2, 768, 128, 32, 6, "bf16"),
     "f32_s16_d128_k4": (1, 2, 1, 640, 128, 16, 4, "f32"),
+    # a ragged last 128-row tile (576 = 4.5 x 128) with g = 8 (two head chunks)
+    "bf16_s16_ragged_g8_d64": (1, 8, 1, 576, 64, 16, 8, "bf16"),
+    "bf16_s32_ragged_d128": (1, 2, 1, 704, 128, 32, 5, "bf16"),
 }
 
 

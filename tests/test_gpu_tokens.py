@@ -23,6 +23,7 @@ CASES = {
     "f32_s64_d64": (1, 2, 1, 512, 64, 64, 3, "f32"),
     "bf16_s64_d128_gqa": (1, 4, 2, 768, 128, 64, 4, "bf16"),
     "bf16_s16_d64_g8": (1, 8, 1, 512, 64, 16, 8, "bf16"),
+    "bf16_s32_d64_ragged": (1, 4, 2, 704, 64, 32, 5, "bf16"),
 }
 
 
