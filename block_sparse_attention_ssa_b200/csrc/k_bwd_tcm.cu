@@ -16,12 +16,14 @@
 // TMA, warp 9 owns TMEM and issues the MMAs.  All tiles are 128 x 64 bf16
 // (one 128-byte swizzle span per row).
 //
-//   dq   one 128-row query tile per CTA, walking its causal key tiles.  TMEM:
-//        dQ [0,64), S [64,192), dP_c [192,320), dP_f [320,448).  Per tile:
-//        S = Q K^T, dP_c = dO_c V^T, dP_f = dh_f V^T (each only when a row of
-//        the tile can use it), dS = P (dP_x - D_x) routed per 16-key group by
-//        the row's selection, written as bf16 over the warp's own S columns,
-//        then dQ += dS K.
+//   dq   one 128-row query tile per CTA, walking its causal key tiles 64 keys
+//        (a half step) at a time.  TMEM: dQ [0,64), then two buffers of S,
+//        dP_c, dP_f (64 columns each), so that the products of the next half
+//        step run while this one is computed.  Per half step: S = Q K^T,
+//        dP_c = dO_c V^T, dP_f = dh_f V^T (each only when a row of the tile
+//        can use it), dS = P (dP_x - D_x) routed per 16-key group by the row's
+//        selection, written as bf16 over the warp's own S columns, then
+//        dQ += dS K.
 //   dkv  one 128-key tile per CTA, walking a chunk of at most 4 query heads
 //        of its kv group and their causal query tiles, 64 queries (a half
 //        step) at a time.  TMEM: dK [0,64), dV [64,128), then two buffers of
@@ -49,7 +51,6 @@ constexpr int TB = TILE * HD * 2;  // 16 KB: one 128 x 64 bf16 tile
 constexpr int NTHREADS = 320;
 constexpr int WARP_TMA = 8, WARP_MMA = 9;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, TILE, false, false);  // both K-major
 constexpr uint32_t IDESC_ACC = idesc_bf16_f32(TILE, HD, false, true);   // B MN-major (rows = reduction)
 
 struct TcmBwdParams {
@@ -65,24 +66,6 @@ struct TcmBwdParams {
   float c;  // scale * log2(e)
   float scale;
 };
-
-// D (128 x 128) = A (128 x 64) B^T with both operands K-major smem tiles.
-__device__ __forceinline__ void mma_ss_d64(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
-#pragma unroll
-  for (int kk = 0; kk < HD / 16; ++kk)
-    mma_ss(d_tmem, smem_desc_sw128(a_smem + kk * 32, 16, 1024), smem_desc_sw128(b_smem + kk * 32, 16, 1024),
-           IDESC_S, kk > 0 ? 1u : 0u);
-}
-
-// D (128 x 64) (+)= A (TMEM, 128 rows x 128 reduction as bf16 pairs: indices
-// 0-63 at columns a..a+31, 64-127 at a+64..a+95) x B (smem 128 x 64 tile,
-// rows = reduction index).
-__device__ __forceinline__ void mma_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < TILE / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), smem_desc_sw128(b_smem + kk * 2048, TB, 1024), IDESC_ACC,
-           (accumulate || kk > 0) ? 1u : 0u);
-}
 
 // Half steps of 64 along the MMA's N / reduction dimension.
 constexpr uint32_t IDESC_S64 = idesc_bf16_f32(TILE, 64, false, false);  // both K-major, N = 64
@@ -118,11 +101,13 @@ namespace dqm {
 constexpr int NS = 3;
 constexpr int OFF_Q = 0, OFF_OC = TB, OFF_F = 2 * TB, OFF_K = 3 * TB, OFF_V = OFF_K + NS * TB;
 constexpr int OFF_MISC = OFF_V + NS * TB;
-constexpr uint32_t COL_DQ = 0, COL_S = 64, COL_DPC = 192, COL_DPF = 320;
+// TMEM: dQ, then two buffers of one 64-key half step each: S, dP_c, dP_f
+// (64 columns apiece) at COL_BUF + 192 b.
+constexpr uint32_t COL_DQ = 0, COL_BUF = 64;
 struct Misc {
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
-  uint64_t s_full, ds_full, done, drain;
+  uint64_t s_full[2], ds_full[2], done, drain;
   uint32_t tmem_base;
   int abort;
   uint32_t uni[64], inter[64];  // OR / AND of the tile's selection rows
@@ -157,8 +142,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&M.v_full[s], 1);
       mbar_init(&M.v_empty[s], 1);
     }
-    mbar_init(&M.s_full, 1);
-    mbar_init(&M.ds_full, 8);
+    for (int bb = 0; bb < 2; ++bb) {
+      mbar_init(&M.s_full[bb], 1);
+      mbar_init(&M.ds_full[bb], 8);
+    }
     mbar_init(&M.done, 1);
     mbar_init(&M.drain, 1);
     M.abort = 0;
@@ -192,18 +179,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
 
-  // Whether some row of the tile can have a selected / dropped key in key tile j.
-  auto flags = [&](int j, bool& anyA, bool& anyD) {
-    anyA = anyD = false;
-#pragma unroll
-    for (int sub = 0; sub < 2; ++sub) {
-      const int u = j * TILE + 64 * sub;
-      const int jb = u >> p.ls;
-      const int nb = p.ls >= 6 ? 1 : (64 >> p.ls);
-      const uint32_t m = ((1u << nb) - 1u) << (jb & 31);
-      anyA |= (M.uni[jb >> 5] & m) != 0u;
-      anyD |= (M.inter[jb >> 5] & m) != m;
-    }
+  // Whether some row of the tile can have a selected / dropped key in the
+  // 64 keys starting at u.
+  auto flags = [&](int u, bool& anyA, bool& anyD) {
+    const int jb = u >> p.ls;
+    const int nb = p.ls >= 6 ? 1 : (64 >> p.ls);
+    const uint32_t m = ((1u << nb) - 1u) << (jb & 31);
+    anyA = (M.uni[jb >> 5] & m) != 0u;
+    anyD = (M.inter[jb >> 5] & m) != m;
   };
 
   const int T = qt + 1;  // causal key tiles
@@ -248,37 +231,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else if (warp == WARP_MMA) {
+    // Half step hs = 2 j + y covers keys 64y.. of key tile j and uses TMEM
+    // buffer hs & 1: its S / dP products are issued before the dQ product of
+    // half step hs - 1, so they overlap that half step's compute.
     if (lane == 0) {
       const uint32_t aq = smem_u32(sQ), aoc = smem_u32(sOc), af = smem_u32(sF);
       bool ok = mbar_wait(&M.q_full, 0, abort);
-      for (int j = 0; ok && j < T; ++j) {
-        const int st = j % NS;
+      const int H = 2 * T;
+      auto front = [&](int hs) -> bool {
+        const int j = hs >> 1, y = hs & 1, st = j % NS, bsel = hs & 1;
         const uint32_t ph = (uint32_t)(j / NS) & 1u;
         bool anyA, anyD;
-        flags(j, anyA, anyD);
-        const uint32_t ak = smem_u32(sK + st * TB), av = smem_u32(sV + st * TB);
-        if (!mbar_wait(&M.k_full[st], ph, abort)) {
+        flags(j * TILE + 64 * y, anyA, anyD);
+        const uint32_t ak = smem_u32(sK + st * TB) + 8192u * y, av = smem_u32(sV + st * TB) + 8192u * y;
+        const uint32_t base = tmem + COL_BUF + 192 * bsel;
+        if (!mbar_wait(&M.k_full[st], ph, abort)) return false;
+        tc_fence_after();
+        mma_ss_n64(base, aq, ak);
+        if (!mbar_wait(&M.v_full[st], ph, abort)) return false;
+        tc_fence_after();
+        if (anyA) mma_ss_n64(base + 64, aoc, av);
+        if (anyD) mma_ss_n64(base + 128, af, av);
+        tc_commit(&M.s_full[bsel]);
+        if (y == 1) tc_commit(&M.v_empty[st]);
+        return true;
+      };
+      auto back = [&](int hs) -> bool {
+        const int j = hs >> 1, y = hs & 1, st = j % NS, bsel = hs & 1;
+        if (!mbar_wait(&M.ds_full[bsel], (uint32_t)(hs >> 1) & 1u, abort)) return false;
+        tc_fence_after();
+        mma_ts_k64(tmem + COL_DQ, tmem + COL_BUF + 192 * bsel, smem_u32(sK + st * TB) + 8192u * y, hs > 0);
+        if (y == 1) tc_commit(&M.k_empty[st]);
+        return true;
+      };
+      if (ok && H > 0) ok = front(0);
+      for (int hs = 0; ok && hs < H; ++hs) {
+        if (hs + 1 < H && !front(hs + 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        mma_ss_d64(tmem + COL_S, aq, ak);
-        if (!mbar_wait(&M.v_full[st], ph, abort)) {
+        if (!back(hs)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (anyA) mma_ss_d64(tmem + COL_DPC, aoc, av);
-        if (anyD) mma_ss_d64(tmem + COL_DPF, af, av);
-        tc_commit(&M.s_full);
-        tc_commit(&M.v_empty[st]);
-        if (!mbar_wait(&M.ds_full, (uint32_t)j & 1u, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        mma_ts_acc(tmem + COL_DQ, tmem + COL_S, ak, j > 0);
-        tc_commit(&M.k_empty[st]);
       }
       tc_commit(&M.done);
       tc_commit(&M.drain);
@@ -286,7 +281,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_wait(&M.drain, 0, &dummy);
     }
   } else {
-    const int quarter = warp & 3, ch = warp >> 2;
+    const int quarter = warp & 3, ch = warp >> 2;  // rows 32*quarter.., keys 32*ch.. of a half step
     const int row = quarter * 32 + lane;
     const int t = q0 + row;
     const bool valid = t < p.N;
@@ -296,46 +291,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const float Dc = valid ? p.Dc[ro] : 0.f, Df = valid ? p.Df[ro] : 0.f;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      if (!mbar_wait(&M.s_full, (uint32_t)j & 1u, abort)) {
+    for (int hs = 0; hs < 2 * T; ++hs) {
+      const int j = hs >> 1, y = hs & 1, bsel = hs & 1;
+      if (!mbar_wait(&M.s_full[bsel], (uint32_t)(hs >> 1) & 1u, abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
       bool anyA, anyD;
-      flags(j, anyA, anyD);
-      const int u0 = j * TILE + 64 * ch;  // first key of this warp's columns
-      const unsigned long long km = tile_keep_mask_p2(selw, u0, p.ls);
-      const int lim = valid ? t - u0 : -1;  // keys c <= lim are causal
+      const int uh = j * TILE + 64 * y;  // first key of the half step
+      flags(uh, anyA, anyD);
+      // bit 16g of km: key group g of this warp's 32 keys
+      const unsigned long long km = tile_keep_mask_p2(selw, uh, p.ls) >> (32 * ch);
+      const int lim = valid ? t - (uh + 32 * ch) : -1;  // keys c <= lim are causal
+      const uint32_t base = lane_base + COL_BUF + 192 * bsel + 32 * ch;
+      uint32_t s[32], pc[32], pf[32];
+      tmem_ld32(base, s);
+      if (anyA) tmem_ld32(base + 64, pc);
+      if (anyD) tmem_ld32(base + 128, pf);
+      tmem_wait_ld();
+      uint32_t ds[16];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t col = 64 * ch + 32 * hh;
-        uint32_t s[32], pc[32], pf[32];
-        tmem_ld32(lane_base + COL_S + col, s);
-        if (anyA) tmem_ld32(lane_base + COL_DPC + col, pc);
-        if (anyD) tmem_ld32(lane_base + COL_DPF + col, pf);
-        tmem_wait_ld();
-        uint32_t ds[16];
+      for (int c = 0; c < 32; c += 2) {
+        float v[2];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float v[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int kc = 32 * hh + c + e;  // key within the warp's 64
-            const bool inA = (km >> (kc & ~15)) & 1ull;
-            const bool live = kc <= lim;
-            const float pv = ex2(fmaf(__uint_as_float(s[c + e]), p.c, -lse2));
-            const float dpx = inA ? __uint_as_float(pc[c + e]) - Dc : __uint_as_float(pf[c + e]) - Df;
-            v[e] = live ? pv * dpx : 0.f;
-          }
-          ds[c / 2] = pack_bf16(v[0], v[1]);
+        for (int e = 0; e < 2; ++e) {
+          const int kc = c + e;  // key within the warp's 32
+          const bool inA = (km >> (kc & ~15)) & 1ull;
+          const bool live = kc <= lim;
+          const float pv = ex2(fmaf(__uint_as_float(s[kc]), p.c, -lse2));
+          const float dpx = inA ? __uint_as_float(pc[kc]) - Dc : __uint_as_float(pf[kc]) - Df;
+          v[e] = live ? pv * dpx : 0.f;
         }
-        tmem_st16(lane_base + COL_S + 64 * ch + 16 * hh, ds);
+        ds[c / 2] = pack_bf16(v[0], v[1]);
       }
+      tmem_st16(base, ds);  // packed into the first 16 of the warp's own 32 S columns
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&M.ds_full);
+      if (lane == 0) mbar_arrive(&M.ds_full[bsel]);
     }
     if (ok && mbar_wait(&M.done, 0, abort)) {
       tc_fence_after();
