@@ -63,29 +63,24 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-KERNEL_SOURCES = {
-    "fwd_dual": "block_sparse_attention_ssa_b200/csrc/k_fwd_tc.cu",
-    "bwd_dual": "block_sparse_attention_ssa_b200/csrc/k_bwd_tc.cu",
-    "dropped_mass": "block_sparse_attention_ssa_b200/csrc/k_dropped_tc.cu",
-}
-
-
 def measured_traffic(row: str, workload: str):
-    """DRAM bytes per launch of an entry point's kernels, from the ncu capture
-    recorded in profiles/traffic.json -- only while the kernel source still has
-    the hash it had when the counters were taken (else None)."""
+    """DRAM bytes per launch of an entry point's kernels on a workload, from
+    the ncu capture recorded in profiles/traffic.json (keyed "row@workload")
+    -- only while the recorded kernel sources still have the hashes they had
+    when the counters were taken (else None)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = KERNEL_SOURCES.get(row)
-    if src is None or not os.path.exists(path):
+    if not os.path.exists(path):
         return None
     with open(path) as fh:
-        rec = json.load(fh).get(row)
-    if not rec or rec.get("workload") != workload:
+        rec = json.load(fh).get(f"{row}@{workload}")
+    if not rec:
         return None
-    with open(os.path.join(ROOT, src), "rb") as fh:
-        sha = hashlib.sha256(fh.read()).hexdigest()
-    return rec["dram_bytes_per_launch"] if rec.get("source_sha256") == sha else None
+    for src, sha in rec["source_sha256"].items():
+        with open(os.path.join(ROOT, src), "rb") as fh:
+            if hashlib.sha256(fh.read()).hexdigest() != sha:
+                return None
+    return rec["dram_bytes_per_launch"]
 
 
 def load_peaks():
@@ -469,7 +464,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops_sustained"],
                 "frac_of_burst": achieved / peaks["bf16_tflops"],
-                "traffic": measured_traffic(r, w.name) if tc_path else None,
+                "traffic": measured_traffic(r, w.name),
                 "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); burst {peaks['bf16_tflops']}"}
 
     dom = max(row_flops, key=lambda r: row_ms[r])
