@@ -19,17 +19,17 @@
 // current block's queries) and kbar [B,Hkv,n,d] (means of complete blocks);
 // the call folds q_t into qsum and, when t closes block i, writes kbar_i.
 //
-// Two launches per token (CUDA cores, fp32 arithmetic; a token moves a few MB):
-//   select: one CTA per (query head, batch) scores the pooled blocks and
-//     keeps its top-k (block-wide arg-max rounds), leaving the kept-block
-//     bits in the workspace;
-//   attend: the union of the g query heads' kept blocks is split BPC blocks
-//     per CTA (flash-decoding style); each CTA reads its K/V rows once for
-//     all g heads, leaves a partial (o, max, sum) per head, and the last CTA
-//     of a (kv head, batch) to finish -- an atomic counter, no waiting --
-//     merges the partials.
+// One launch per token (CUDA cores, fp32 arithmetic; a token moves a few
+// MB): a thread-block cluster of CL CTAs per (batch, kv head) selects the
+// blocks of the g query heads, attends the union of their kept blocks split
+// CL ways (each K/V row read once for all g heads) and merges the partials,
+// exchanging the selections and the partials through distributed shared
+// memory between cluster barriers (no workspace, no atomics, no waiting on
+// flags).
 #include <algorithm>
 #include <climits>
+
+#include <cooperative_groups.h>
 
 #include "ssa_internal.cuh"
 
@@ -38,180 +38,175 @@ namespace {
 
 constexpr int NT = 256;
 constexpr int CH = 64;   // keys per chunk
-constexpr int BPC = 2;   // selected blocks per attention CTA
+constexpr int CL = 8;    // CTAs per cluster: one cluster per (batch, kv head)
 
 struct DecodeShape {
-  int Hq, g, N, s, n, k, t, splits;
+  int Hq, g, N, s, n, k, t;
   float scale;
   int per_token;  // the query side of the score is q_t itself (per-token selection)
 };
 
-// Per-call scratch in the caller's workspace.
-struct DecodeWs {
-  unsigned* counter;  // [B*Hkv]         attention CTAs finished (reset by the select kernel)
-  uint32_t* sel;      // [B*Hkv][g][64]  selected-block bits per query head
-  float* part;        // [B*Hq][splits][D+2] partial (o, m, l) per attention CTA
-};
-
-__host__ __device__ inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
-
-inline DecodeWs decode_ws(void* ws, const Dims& Dm) {
-  char* p = static_cast<char*>(ws);
-  const size_t bk = (size_t)Dm.B * Dm.Hkv;
-  DecodeWs w;
-  size_t o = 0;
-  w.counter = reinterpret_cast<unsigned*>(p + o); o += align256(bk * 4);
-  w.sel = reinterpret_cast<uint32_t*>(p + o); o += align256(bk * Dm.g * 64 * 4);
-  w.part = reinterpret_cast<float*>(p + o);
-  return w;
-}
-
-int decode_splits(const Dims& Dm) {
-  const int most = std::min(Dm.g * Dm.k, Dm.n);  // blocks in a union
-  return (most + BPC - 1) / BPC;
-}
-
-// Byte offsets of the select kernel's shared memory.
-struct SelectLayout {
-  size_t qbar, sc, sel, red, bytes;
-  __host__ __device__ SelectLayout(int n, int D) {
+// Byte offsets of the decode kernel's shared memory.
+struct DecodeLayout {
+  size_t qbar, sc, selh, red, q, o, mx, sum, x, k, v, lst, usel, bytes;
+  __host__ __device__ DecodeLayout(int n, int g, int k_eff, int D) {
     size_t at = 0;
     auto take = [&](size_t nbytes) {
       const size_t r = at;
       at = (at + nbytes + 15) / 16 * 16;
       return r;
     };
-    qbar = take((size_t)D * 4);   // [D] block-prefix query mean
-    sc = take((size_t)n * 4);     // [n] block scores
-    sel = take(64 * 4);           // [64] selected-block bits
-    red = take((size_t)NT * 8);   // per-warp arg-max candidates / key-sum staging
+    const int gl = (g + CL - 1) / CL;                       // heads this CTA selects
+    const int most = (std::min(g * k_eff, n) + CL - 1) / CL;  // union blocks this CTA attends
+    qbar = take((size_t)D * 4);           // [D] query side of the block scores
+    sc = take((size_t)n * 4);             // [n] block scores
+    selh = take((size_t)gl * 64 * 4);     // [gl][64] selected-block bits of this CTA's heads
+    red = take((size_t)NT * 8);           // arg-max candidates / key-sum staging
+    q = take((size_t)g * D * 4);          // [g][D] q_t
+    o = take((size_t)g * D * 4);          // [g][D] partial output
+    mx = take((size_t)g * 4);             // [g] running max
+    sum = take((size_t)g * 4);            // [g] running sum
+    x = take((size_t)g * CH * 4);         // [g][CH] logits / weights of a chunk
+    k = take((size_t)CH * (D + 1) * 4);   // [CH][D+1] K chunk
+    v = take((size_t)CH * D * 4);         // [CH][D] V chunk
+    lst = take((size_t)(1 + most) * 4);   // this CTA's blocks of the union
+    usel = take((size_t)g * 64 * 4);      // [g][64] every head's selected-block bits
     bytes = at;
   }
 };
 
-// ---- step 1: query-block mean, block scores and top-k of one query head.
-// grid (Hq, B).  Also folds q_t into qsum; the first head of each kv head
-// resets the attention counter and, when t closes block i, writes the
-// block's key mean into kbar.
-template <typename T, int D>
-__global__ void __launch_bounds__(NT) decode_select_kernel(TensorRef q, TensorRef K, int32_t* idx, float* qsum,
-                                                           float* kbar, DecodeWs ws, DecodeShape sh) {
-  const int h = blockIdx.x, b = blockIdx.y;
+// grid (CL, Hkv, B), one cluster of CL CTAs per (batch, kv head).
+//   1. selection: CTA r scores the pooled blocks for the query heads
+//      r, r + CL, .. of the group (folding q_t into qsum) and keeps each
+//      head's top-k in its shared memory; CTA 0 writes the key mean of a
+//      block the token closes;
+//   2. after a cluster barrier every CTA reads all heads' selections from
+//      the selecting CTAs (distributed shared memory), forms their union and
+//      attends its share of the union's blocks (CL-way split, ascending),
+//      reading each K/V row once for all g heads and keeping a partial
+//      (o, max, sum) per head;
+//   3. after a second barrier CTA r merges the partials of heads r, r + CL,
+//      .. from the CL CTAs and writes h and lse; a last barrier keeps every
+//      CTA's shared memory alive until the merges have read it.
+// CPL: top-k candidate slots per lane (32 * CPL >= n).
+template <typename T, int D, int CPL>
+__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT)
+    decode_kernel(TensorRef q, TensorRef K, TensorRef V, TensorRef hout, float* lse, int32_t* idx, float* qsum,
+                  float* kbar, DecodeShape sh) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int kvh = blockIdx.y, b = blockIdx.z;
   const int G = sh.g, n = sh.n, s = sh.s, t = sh.t;
-  const int kvh = h / G, hh = h % G;
   const int i = t / s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hkv = sh.Hq / G;
   const int bk = b * Hkv + kvh;
 
   extern __shared__ __align__(16) uint8_t smem[];
-  const SelectLayout L(n, D);
+  const DecodeLayout L(n, G, sh.k, D);
   float* sqbar = reinterpret_cast<float*>(smem + L.qbar);
   float* ssc = reinterpret_cast<float*>(smem + L.sc);
-  uint32_t* sel = reinterpret_cast<uint32_t*>(smem + L.sel);
+  uint32_t* selh = reinterpret_cast<uint32_t*>(smem + L.selh);
   float* rv = reinterpret_cast<float*>(smem + L.red);
-  int* rj = reinterpret_cast<int*>(rv + NT);
+  float* sq = reinterpret_cast<float*>(smem + L.q);
+  float* so = reinterpret_cast<float*>(smem + L.o);
+  float* smax = reinterpret_cast<float*>(smem + L.mx);
+  float* ssum = reinterpret_cast<float*>(smem + L.sum);
+  float* sx = reinterpret_cast<float*>(smem + L.x);
+  float* sk = reinterpret_cast<float*>(smem + L.k);
+  float* sv = reinterpret_cast<float*>(smem + L.v);
+  int* slst = reinterpret_cast<int*>(smem + L.lst);
+  uint32_t* usel = reinterpret_cast<uint32_t*>(smem + L.usel);
 
-  if (tid < D) {
-    float* qs = qsum + ((int64_t)b * sh.Hq + h) * D + tid;
-    const float x = to_f32(row_ptr<T>(q, b, h, 0)[tid]);
-    const float acc = (t % s == 0 ? 0.f : *qs) + x;
-    *qs = acc;
-    sqbar[tid] = sh.per_token ? x : acc / (float)(t - i * s + 1);
-  }
-  if (tid < 64) sel[tid] = 0u;
-  if (hh == 0 && tid == 0) ws.counter[bk] = 0u;
-  __syncthreads();
-
-  // scores of the complete blocks j < i: a warp takes RPW pooled keys at a
-  // time (a lane holds PER consecutive dims of each), so RPW coalesced row
-  // loads are in flight before the dot products and lane reductions
-  constexpr int PER = D / 32, RPW = 4;
-  const float* kb = kbar + (int64_t)bk * n * D;
-  float qv[PER];
-#pragma unroll
-  for (int c = 0; c < PER; ++c) qv[c] = sqbar[lane * PER + c];
-  for (int j0 = warp * RPW; j0 < i; j0 += (NT / 32) * RPW) {
-    float kv[RPW][PER];
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-#pragma unroll
-      for (int c = 0; c < PER; ++c) kv[r][c] = (j0 + r < i) ? kb[(int64_t)(j0 + r) * D + lane * PER + c] : 0.f;
+  // ================================================================ 1. selection
+  for (int hl = 0; rank + CL * hl < G; ++hl) {
+    const int hh = rank + CL * hl, h = kvh * G + hh;
+    uint32_t* sel = selh + hl * 64;
+    if (tid < D) {
+      float* qs = qsum + ((int64_t)b * sh.Hq + h) * D + tid;
+      const float xq = to_f32(row_ptr<T>(q, b, h, 0)[tid]);
+      const float acc = (t % s == 0 ? 0.f : *qs) + xq;
+      *qs = acc;
+      sqbar[tid] = sh.per_token ? xq : acc / (float)(t - i * s + 1);
     }
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      float p = 0.f;
-#pragma unroll
-      for (int c = 0; c < PER; ++c) p = fmaf(qv[c], kv[r][c], p);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-      if (lane == 0 && j0 + r < i) ssc[j0 + r] = sh.scale * p;
-    }
-  }
-  __syncthreads();
+    if (tid < 64) sel[tid] = 0u;
+    __syncthreads();
 
-  // top-(k-1) of the scores plus the diagonal block; each round is a
-  // block-wide arg-max (score descending, index ascending)
-  if (i + 1 <= sh.k) {
-    for (int j = tid; j <= i; j += NT) atomicOr(&sel[j >> 5], 1u << (j & 31));
-  } else {
-    if (tid == 0) sel[i >> 5] |= 1u << (i & 31);
-    for (int r = 0; r < sh.k - 1; ++r) {
-      __syncthreads();
-      float best = kNegInf;
-      int bj = INT_MAX;
-      for (int j = tid; j < i; j += NT) {
-        if ((sel[j >> 5] >> (j & 31)) & 1u) continue;
-        float v = ssc[j];
-        if (v != v) v = kNegInf;  // NaN ranks last
-        if (v > best || (v == best && j < bj)) {
-          best = v;
-          bj = j;
-        }
+    // scores of the complete blocks j < i: a thread per pooled key, its row
+    // read as 16-byte vectors against the query side in shared memory
+    const float* kb = kbar + (int64_t)bk * n * D;
+    for (int j = tid; j < i; j += NT) {
+      const float4* row = reinterpret_cast<const float4*>(kb + (int64_t)j * D);
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 kv = row[c4];
+        const float4 qv = *reinterpret_cast<const float4*>(sqbar + 4 * c4);
+        a0 = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, a0));
+        a1 = fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, a1));
       }
+      const float x = sh.scale * (a0 + a1);
+      ssc[j] = (x != x) ? kNegInf : x;  // NaN ranks last
+    }
+    __syncthreads();
+
+    // top-(k-1) of the scores plus the diagonal block (score descending,
+    // index ascending): one warp, candidate j in lane j % 32, slot j / 32;
+    // slots that may not be chosen (j >= i, or taken) hold NaN, which
+    // compares false with everything
+    if (i + 1 <= sh.k) {
+      for (int j = tid; j <= i; j += NT) atomicOr(&sel[j >> 5], 1u << (j & 31));
+    } else if (warp == 0) {
+      const float kOut = __int_as_float(0x7fffffff);
+      float v[CPL];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, best, off);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-        if (ov > best || (ov == best && oj < bj)) {
-          best = ov;
-          bj = oj;
-        }
-      }
-      if (lane == 0) {
-        rv[warp] = best;
-        rj[warp] = bj;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        best = lane < NT / 32 ? rv[lane] : kNegInf;
-        bj = lane < NT / 32 ? rj[lane] : INT_MAX;
+      for (int m = 0; m < CPL; ++m) v[m] = (lane + 32 * m < i) ? ssc[lane + 32 * m] : kOut;
+      uint64_t taken = 0;
+      for (int round = 0; round < sh.k - 1; ++round) {
+        float bv = kNegInf;
+        int bj = INT_MAX;
+#pragma unroll
+        for (int m = 0; m < CPL; ++m)
+          if (v[m] > bv || (v[m] == bv && bj == INT_MAX)) {
+            bv = v[m];
+            bj = lane + 32 * m;
+          }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
           const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-          if (ov > best || (ov == best && oj < bj)) {
-            best = ov;
+          if (ov > bv || (ov == bv && oj < bj)) {
+            bv = ov;
             bj = oj;
           }
         }
-        if (lane == 0 && bj < i) sel[bj >> 5] |= 1u << (bj & 31);
+        if (bj != INT_MAX && (bj & 31) == lane) {
+          taken |= 1ull << (bj >> 5);
+#pragma unroll
+          for (int m = 0; m < CPL; ++m)
+            if (m == (bj >> 5)) v[m] = kOut;
+        }
       }
+#pragma unroll
+      for (int m = 0; m < CPL; ++m)
+        if ((taken >> m) & 1ull) atomicOr(&sel[(lane + 32 * m) >> 5], 1u << ((lane + 32 * m) & 31));
+      if (lane == 0) atomicOr(&sel[i >> 5], 1u << (i & 31));
     }
-  }
-  __syncthreads();
-  if (tid < 64) ws.sel[((size_t)bk * G + hh) * 64 + tid] = sel[tid];
-  if (tid == 0) {  // Sel ascending, -1 padded
-    int32_t* out = idx + ((int64_t)b * sh.Hq + h) * sh.k;
-    int c = 0;
-    for (int w = 0; w <= (i >> 5); ++w)
-      for (uint32_t x = sel[w]; x && c < sh.k; x &= x - 1) out[c++] = 32 * w + __ffs(x) - 1;
-    for (; c < sh.k; ++c) out[c] = -1;
+    __syncthreads();
+    if (tid == 0) {  // Sel ascending, -1 padded
+      int32_t* out = idx + ((int64_t)b * sh.Hq + h) * sh.k;
+      int c = 0;
+      for (int w = 0; w <= (i >> 5); ++w)
+        for (uint32_t xw = sel[w]; xw && c < sh.k; xw &= xw - 1) out[c++] = 32 * w + __ffs(xw) - 1;
+      for (; c < sh.k; ++c) out[c] = -1;
+    }
+    __syncthreads();
   }
 
   // the token closes block i: its key mean joins the pooled cache (no
-  // reader of this call uses kbar[i]); the kv head's first query head does it
-  if (t % s == s - 1 && hh == 0) {
+  // reader of this call uses kbar[i])
+  if (rank == 0 && t % s == s - 1) {
     // NT / D row groups sum interleaved rows (8 loads in flight each), then fold
     constexpr int RG = NT / D;
     const int c = tid % D, rg = tid / D;
@@ -231,81 +226,13 @@ __global__ void __launch_bounds__(NT) decode_select_kernel(TensorRef q, TensorRe
       kbar[((int64_t)bk * n + i) * D + tid] = sum / (float)s;
     }
   }
-}
+  cluster.sync();  // every head's selection is visible to the cluster
 
-// Byte offsets of the attention kernel's shared memory.
-struct AttendLayout {
-  size_t q, o, mx, sum, x, k, v, lst, bytes;
-  __host__ __device__ AttendLayout(int g, int D) {
-    size_t at = 0;
-    auto take = [&](size_t nbytes) {
-      const size_t r = at;
-      at = (at + nbytes + 15) / 16 * 16;
-      return r;
-    };
-    q = take((size_t)g * D * 4);         // [g][D] q_t
-    o = take((size_t)g * D * 4);         // [g][D] partial output
-    mx = take((size_t)g * 4);            // [g] running max
-    sum = take((size_t)g * 4);           // [g] running sum
-    x = take((size_t)g * CH * 4);        // [g][CH] logits / weights of a chunk
-    k = take((size_t)CH * (D + 1) * 4);  // [CH][D+1] K chunk
-    v = take((size_t)CH * D * 4);        // [CH][D] V chunk
-    lst = take(16 + 4 * BPC);            // this CTA's blocks of the union, flag
-    bytes = at;
-  }
-};
-
-// ---- step 2: attention over the union of the g heads' selected blocks,
-// BPC blocks per CTA.  The next chunk's K/V rows are loaded into registers
-// while the current chunk is processed.  Each CTA leaves a partial
-// (o, m, l) per query head and the last CTA of a (batch, kv head) to finish
-// merges them.  grid (splits, Hkv, B).
-template <typename T, int D>
-__global__ void __launch_bounds__(NT) decode_attend_kernel(TensorRef q, TensorRef K, TensorRef V, TensorRef hout,
-                                                           float* lse, DecodeWs ws, DecodeShape sh) {
-  constexpr int VEC = Vec16<T>::kN;
-  constexpr int ITERS = CH * (D / VEC) / NT;  // 16-byte loads per thread per chunk and tensor
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int G = sh.g, s = sh.s, t = sh.t;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Hkv = sh.Hq / G;
-  const int bk = b * Hkv + kvh;
-
-  extern __shared__ __align__(16) uint8_t smem[];
-  const AttendLayout L(G, D);
-  float* sq = reinterpret_cast<float*>(smem + L.q);
-  float* so = reinterpret_cast<float*>(smem + L.o);
-  float* smax = reinterpret_cast<float*>(smem + L.mx);
-  float* ssum = reinterpret_cast<float*>(smem + L.sum);
-  float* sx = reinterpret_cast<float*>(smem + L.x);
-  float* sk = reinterpret_cast<float*>(smem + L.k);
-  float* sv = reinterpret_cast<float*>(smem + L.v);
-  int* slst = reinterpret_cast<int*>(smem + L.lst);  // [0] count, [1..] blocks, [1 + BPC] last flag
-
-  const uint32_t* selw = ws.sel + (size_t)bk * G * 64;
-  // this CTA's entries [split*BPC, split*BPC + BPC) of the ascending union
-  if (warp == 0) {
-    uint32_t w0 = 0, w1 = 0;
-#pragma unroll 4
-    for (int hh = 0; hh < G; ++hh) {
-      const uint2 wv = *reinterpret_cast<const uint2*>(selw + hh * 64 + 2 * lane);
-      w0 |= wv.x;
-      w1 |= wv.y;
-    }
-    const int c = __popc(w0) + __popc(w1);
-    int incl = c;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    const int e0 = split * BPC;
-    int pos = incl - c;
-    for (uint32_t x = w0; x; x &= x - 1, ++pos)
-      if (pos >= e0 && pos < e0 + BPC) slst[1 + pos - e0] = 64 * lane + __ffs(x) - 1;
-    for (uint32_t x = w1; x; x &= x - 1, ++pos)
-      if (pos >= e0 && pos < e0 + BPC) slst[1 + pos - e0] = 64 * lane + 32 + __ffs(x) - 1;
-    if (lane == 31) slst[0] = max(0, min(BPC, incl - e0));
+  // ================================================================ 2. attention
+  for (int e = tid; e < G * 64; e += NT) {
+    const int hh = e >> 6, w = e & 63;
+    const uint32_t* peer = cluster.map_shared_rank(selh, hh % CL);
+    usel[e] = peer[(hh / CL) * 64 + w];
   }
   for (int e = tid; e < G * D; e += NT) {
     sq[e] = to_f32(row_ptr<T>(q, b, kvh * G + e / D, 0)[e % D]);
@@ -316,147 +243,143 @@ __global__ void __launch_bounds__(NT) decode_attend_kernel(TensorRef q, TensorRe
     ssum[tid] = 0.f;
   }
   __syncthreads();
-  const int nb = slst[0];
-  const int cpb = (s + CH - 1) / CH;  // chunks per block
-  const int nch = nb * cpb;
-  auto chunk_rows = [&](int ch, int& j, int& c0) {
-    j = slst[1 + ch / cpb];
-    c0 = j * s + (ch % cpb) * CH;
-    return max(0, min(CH, min(j * s + s, t + 1) - c0));
-  };
-
-  float tk[ITERS][VEC], tv[ITERS][VEC];
-  auto load_chunk = [&](int ch) {
-    int j, c0;
-    const int rows = chunk_rows(ch, j, c0);
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int x = tid + it * NT, r = x / (D / VEC), c = (x % (D / VEC)) * VEC;
-      if (r < rows) {
-        Vec16<T>::load(row_ptr<T>(K, b, kvh, (int64_t)c0 + r) + c, tk[it]);
-        Vec16<T>::load(row_ptr<T>(V, b, kvh, (int64_t)c0 + r) + c, tv[it]);
-      }
+  // this CTA's entries [cnt*rank/CL, cnt*(rank+1)/CL) of the ascending union
+  if (warp == 0) {
+    uint32_t w0 = 0, w1 = 0;
+    for (int hh = 0; hh < G; ++hh) {
+      w0 |= usel[hh * 64 + 2 * lane];
+      w1 |= usel[hh * 64 + 2 * lane + 1];
     }
-  };
-  if (nch > 0) load_chunk(0);
-  for (int ch = 0; ch < nch; ++ch) {
-    int j, c0;
-    const int rows = chunk_rows(ch, j, c0);
+    const int c = __popc(w0) + __popc(w1);
+    int incl = c;
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int x = tid + it * NT, r = x / (D / VEC), c = (x % (D / VEC)) * VEC;
-      if (r < rows) {
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+    const int lo = cnt * rank / CL, hi = cnt * (rank + 1) / CL;
+    int pos = incl - c;
+    for (uint32_t xw = w0; xw; xw &= xw - 1, ++pos)
+      if (pos >= lo && pos < hi) slst[1 + pos - lo] = 64 * lane + __ffs(xw) - 1;
+    for (uint32_t xw = w1; xw; xw &= xw - 1, ++pos)
+      if (pos >= lo && pos < hi) slst[1 + pos - lo] = 64 * lane + 32 + __ffs(xw) - 1;
+    if (lane == 0) slst[0] = hi - lo;
+  }
+  __syncthreads();
+  {
+    constexpr int VEC = Vec16<T>::kN;
+    constexpr int ITERS = CH * (D / VEC) / NT;  // 16-byte loads per thread per chunk and tensor
+    const int nb = slst[0];
+    const int cpb = (s + CH - 1) / CH;  // chunks per block
+    const int nch = nb * cpb;
+    auto chunk_rows = [&](int chk, int& j, int& c0) {
+      j = slst[1 + chk / cpb];
+      c0 = j * s + (chk % cpb) * CH;
+      return max(0, min(CH, min(j * s + s, t + 1) - c0));
+    };
+    float tk[ITERS][VEC], tv[ITERS][VEC];
+    auto load_chunk = [&](int chk) {
+      int j, c0;
+      const int rows = chunk_rows(chk, j, c0);
 #pragma unroll
-        for (int y = 0; y < VEC; ++y) {
-          sk[r * (D + 1) + c + y] = tk[it][y];
-          sv[r * D + c + y] = tv[it][y];
+      for (int it = 0; it < ITERS; ++it) {
+        const int xx = tid + it * NT, r = xx / (D / VEC), c = (xx % (D / VEC)) * VEC;
+        if (r < rows) {
+          Vec16<T>::load(row_ptr<T>(K, b, kvh, (int64_t)c0 + r) + c, tk[it]);
+          Vec16<T>::load(row_ptr<T>(V, b, kvh, (int64_t)c0 + r) + c, tv[it]);
         }
       }
-    }
-    if (ch + 1 < nch) load_chunk(ch + 1);  // in flight while this chunk is used
-    __syncthreads();
-    for (int x = tid; x < G * CH; x += NT) {
-      const int hh = x / CH, uu = x % CH;
-      float v = kNegInf;
-      if (uu < rows && ((selw[hh * 64 + (j >> 5)] >> (j & 31)) & 1u)) {
-        const float* qv = sq + hh * D;
-        const float* kv = sk + uu * (D + 1);
-        float acc = 0.f;
+    };
+    if (nch > 0) load_chunk(0);
+    for (int chk = 0; chk < nch; ++chk) {
+      int j, c0;
+      const int rows = chunk_rows(chk, j, c0);
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it) {
+        const int xx = tid + it * NT, r = xx / (D / VEC), c = (xx % (D / VEC)) * VEC;
+        if (r < rows) {
+#pragma unroll
+          for (int y = 0; y < VEC; ++y) {
+            sk[r * (D + 1) + c + y] = tk[it][y];
+            sv[r * D + c + y] = tv[it][y];
+          }
+        }
+      }
+      if (chk + 1 < nch) load_chunk(chk + 1);  // in flight while this chunk is used
+      __syncthreads();
+      for (int xx = tid; xx < G * CH; xx += NT) {
+        const int hh = xx / CH, uu = xx % CH;
+        float v = kNegInf;
+        if (uu < rows && ((usel[hh * 64 + (j >> 5)] >> (j & 31)) & 1u)) {
+          const float* qvv = sq + hh * D;
+          const float* kvv = sk + uu * (D + 1);
+          float acc = 0.f;
 #pragma unroll 8
-        for (int c = 0; c < D; ++c) acc = fmaf(qv[c], kv[c], acc);
-        v = sh.scale * acc;
+          for (int c = 0; c < D; ++c) acc = fmaf(qvv[c], kvv[c], acc);
+          v = sh.scale * acc;
+        }
+        sx[xx] = v;
       }
-      sx[x] = v;
+      __syncthreads();
+      for (int hh = warp; hh < G; hh += NT / 32) {
+        if (!((usel[hh * 64 + (j >> 5)] >> (j & 31)) & 1u)) continue;
+        float* xs = sx + hh * CH;
+        float mt = fmaxf(xs[lane], xs[lane + 32]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        const float m_old = smax[hh];
+        const float m_new = fmaxf(m_old, mt);
+        const float p0 = (xs[lane] == kNegInf) ? 0.f : __expf(xs[lane] - m_new);
+        const float p1 = (xs[lane + 32] == kNegInf) ? 0.f : __expf(xs[lane + 32] - m_new);
+        float ps = p0 + p1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        const float corr = (m_old == kNegInf) ? 0.f : __expf(m_old - m_new);
+        __syncwarp();
+        xs[lane] = p0;
+        xs[lane + 32] = p1;
+        __syncwarp();
+        float* o = so + hh * D;
+#pragma unroll
+        for (int r = 0; r < D / 32; ++r) {
+          const int c = lane + 32 * r;
+          float acc = o[c] * corr;
+          for (int uu = 0; uu < rows; ++uu) acc = fmaf(xs[uu], sv[uu * D + c], acc);
+          o[c] = acc;
+        }
+        if (lane == 0) {
+          smax[hh] = m_new;
+          ssum[hh] = ssum[hh] * corr + ps;
+        }
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    for (int hh = warp; hh < G; hh += NT / 32) {
-      if (!((selw[hh * 64 + (j >> 5)] >> (j & 31)) & 1u)) continue;
-      float* xs = sx + hh * CH;
-      float mt = fmaxf(xs[lane], xs[lane + 32]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-      const float m_old = smax[hh];
-      const float m_new = fmaxf(m_old, mt);
-      const float p0 = (xs[lane] == kNegInf) ? 0.f : __expf(xs[lane] - m_new);
-      const float p1 = (xs[lane + 32] == kNegInf) ? 0.f : __expf(xs[lane + 32] - m_new);
-      float ps = p0 + p1;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-      const float corr = (m_old == kNegInf) ? 0.f : __expf(m_old - m_new);
-      __syncwarp();
-      xs[lane] = p0;
-      xs[lane + 32] = p1;
-      __syncwarp();
-      float* o = so + hh * D;
-#pragma unroll
-      for (int r = 0; r < D / 32; ++r) {
-        const int c = lane + 32 * r;
-        float acc = o[c] * corr;
-        for (int uu = 0; uu < rows; ++uu) acc = fmaf(xs[uu], sv[uu * D + c], acc);
-        o[c] = acc;
-      }
-      if (lane == 0) {
-        smax[hh] = m_new;
-        ssum[hh] = ssum[hh] * corr + ps;
-      }
-    }
-    __syncthreads();
   }
+  cluster.sync();  // every CTA's partial (o, max, sum) is visible to the cluster
 
-  // partial (o, m, l) of this CTA for each of the g heads
-  for (int e = tid; e < G * (D + 2); e += NT) {
-    const int hh = e / (D + 2), c = e % (D + 2);
-    const float v = c < D ? so[hh * D + c] : (c == D ? smax[hh] : ssum[hh]);
-    ws.part[(((size_t)b * sh.Hq + kvh * G + hh) * sh.splits + split) * (D + 2) + c] = v;
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) slst[1 + BPC] = (atomicAdd(&ws.counter[bk], 1u) == (unsigned)sh.splits - 1) ? 1 : 0;
-  __syncthreads();
-  if (!slst[1 + BPC]) return;
-  __threadfence();
-
-  // last CTA: merge the splits; warp hh merges head hh (lanes over splits for
-  // the statistics, over dims for the output, four splits' rows in flight)
-  constexpr int PER = D / 32;
-  for (int hh = warp; hh < G; hh += NT / 32) {
-    const float* p = ws.part + ((size_t)b * sh.Hq + kvh * G + hh) * sh.splits * (D + 2);
+  // ================================================================ 3. merge
+  for (int hh = rank; hh < G; hh += CL) {
     float M = kNegInf;
-    for (int x = lane; x < sh.splits; x += 32) M = fmaxf(M, __ldcg(p + (size_t)x * (D + 2) + D));
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float Lsum = 0.f;
-    for (int x = lane; x < sh.splits; x += 32) {
-      const float m = __ldcg(p + (size_t)x * (D + 2) + D);
-      if (m != kNegInf) Lsum += __ldcg(p + (size_t)x * (D + 2) + D + 1) * __expf(m - M);
+    for (int r = 0; r < CL; ++r) M = fmaxf(M, *cluster.map_shared_rank(smax + hh, r));
+    float Lsum = 0.f, wgt[CL];
+#pragma unroll
+    for (int r = 0; r < CL; ++r) {
+      const float m = *cluster.map_shared_rank(smax + hh, r);
+      wgt[r] = (m == kNegInf) ? 0.f : __expf(m - M);
+      Lsum += *cluster.map_shared_rank(ssum + hh, r) * wgt[r];
     }
+    for (int c = tid; c < D; c += NT) {
+      float acc = 0.f;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
-    float acc[PER];
-#pragma unroll
-    for (int c = 0; c < PER; ++c) acc[c] = 0.f;
-    for (int x0 = 0; x0 < sh.splits; x0 += 4) {
-      float m[4], o[4][PER];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int x = x0 + r;
-        m[r] = x < sh.splits ? __ldcg(p + (size_t)x * (D + 2) + D) : kNegInf;
-#pragma unroll
-        for (int c = 0; c < PER; ++c) o[r][c] = x < sh.splits ? __ldcg(p + (size_t)x * (D + 2) + lane * PER + c) : 0.f;
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        if (m[r] == kNegInf) continue;
-        const float wgt = __expf(m[r] - M);
-#pragma unroll
-        for (int c = 0; c < PER; ++c) acc[c] = fmaf(o[r][c], wgt, acc[c]);
-      }
+      for (int r = 0; r < CL; ++r)
+        if (wgt[r] != 0.f) acc = fmaf(*cluster.map_shared_rank(so + hh * D + c, r), wgt[r], acc);
+      row_ptr_w<T>(hout, b, kvh * G + hh, 0)[c] = from_f32<T>(Lsum > 0.f ? acc / Lsum : 0.f);
     }
-    T* dst = row_ptr_w<T>(hout, b, kvh * G + hh, 0) + lane * PER;
-#pragma unroll
-    for (int c = 0; c < PER; ++c) dst[c] = from_f32<T>(Lsum > 0.f ? acc[c] / Lsum : 0.f);
-    if (lane == 0) lse[(int64_t)b * sh.Hq + kvh * G + hh] = Lsum > 0.f ? M + logf(Lsum) : kNegInf;
+    if (tid == 0) lse[(int64_t)b * sh.Hq + kvh * G + hh] = Lsum > 0.f ? M + logf(Lsum) : kNegInf;
   }
+  cluster.sync();  // peers' shared memory stays alive until every merge has read it
 }
 
 // Prefill of the decode state from a prompt of t0 tokens: kbar of the
@@ -483,22 +406,21 @@ __global__ void __launch_bounds__(128) decode_prefill_kernel(TensorRef Q, Tensor
 
 template <typename T, int D>
 cudaError_t decode_t(const Dims& Dm, const DecodeArgs& a, cudaStream_t st) {
-  const int splits = decode_splits(Dm);
-  const DecodeWs ws = decode_ws(a.ws, Dm);
-  DecodeShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, a.t, splits, Dm.scale, Dm.per_token};
-  const size_t sm1 = SelectLayout(Dm.n, D).bytes, sm2 = AttendLayout(Dm.g, D).bytes;
-  auto k1 = decode_select_kernel<T, D>;
-  auto k2 = decode_attend_kernel<T, D>;
-  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-  if (e != cudaSuccess) return e;
-  k1<<<dim3(Dm.Hq, Dm.B), NT, sm1, st>>>(a.q, a.k, a.idx, a.qsum, a.kbar, ws, sh);
-  count_launches(1);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  k2<<<dim3(splits, Dm.Hkv, Dm.B), NT, sm2, st>>>(a.q, a.k, a.v, a.h, a.lse, ws, sh);
-  count_launches(1);
-  return cudaGetLastError();
+  DecodeShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, a.t, Dm.scale, Dm.per_token};
+  const size_t smem = DecodeLayout(Dm.n, Dm.g, Dm.k, D).bytes;
+  auto run = [&](auto kern) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(CL, Dm.Hkv, Dm.B), NT, smem, st>>>(a.q, a.k, a.v, a.h, a.lse, a.idx, a.qsum, a.kbar, sh);
+    count_launches(1);
+    return cudaGetLastError();
+  };
+  const int cpl = (Dm.n + 31) / 32;
+  if (cpl <= 2) return run(decode_kernel<T, D, 2>);
+  if (cpl <= 8) return run(decode_kernel<T, D, 8>);
+  if (cpl <= 16) return run(decode_kernel<T, D, 16>);
+  if (cpl <= 32) return run(decode_kernel<T, D, 32>);
+  return run(decode_kernel<T, D, 64>);
 }
 
 template <typename T, int D>
@@ -511,15 +433,11 @@ cudaError_t prefill_t(const Dims& Dm, const DecodeArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-size_t decode_smem_bytes(const Dims& D) {
-  const size_t a = SelectLayout(D.n, D.d).bytes, b = AttendLayout(D.g, D.d).bytes;
-  return a > b ? a : b;
-}
+size_t decode_smem_bytes(const Dims& D) { return DecodeLayout(D.n, D.g, D.k, D.d).bytes; }
 
 size_t decode_ws_bytes(const Dims& D) {
-  const size_t bk = (size_t)D.B * D.Hkv;
-  return align256(bk * 4) + align256(bk * D.g * 64 * 4) +
-         align256((size_t)D.B * D.Hq * decode_splits(D) * (D.d + 2) * 4);
+  (void)D;
+  return 0;  // the decode step keeps its scratch in the cluster's shared memory
 }
 
 cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, cudaStream_t st) {

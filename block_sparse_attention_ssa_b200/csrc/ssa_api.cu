@@ -465,7 +465,7 @@ ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q, cons
   if ((s = check_tensor(D, h, false, &a.h)) != SSA_OK) return s;
   if (t < 0 || t >= D.N) return SSA_ERR_INVALID_ARG;
   if (!qsum || !kbar || !lse || !idx) return SSA_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(qsum) % 4 || reinterpret_cast<uintptr_t>(kbar) % 4 ||
+  if (reinterpret_cast<uintptr_t>(qsum) % 4 || reinterpret_cast<uintptr_t>(kbar) % 16 ||
       reinterpret_cast<uintptr_t>(lse) % 4 || reinterpret_cast<uintptr_t>(idx) % 4)
     return SSA_ERR_INVALID_ARG;
   if (decode_smem_bytes(D) > 232448) return SSA_ERR_UNSUPPORTED;

@@ -223,7 +223,7 @@ struct DecodeArgs {
   float* qsum;           // [B,Hq,d] running sum of the current block's queries
   float* kbar;           // [B,Hkv,n,d] means of the complete key blocks
   int t;                 // position of the new token (prefill: prompt length)
-  void* ws;              // decode step: caller workspace (decode_ws_bytes)
+  void* ws;              // decode step: caller workspace (unused: scratch lives in shared memory)
 };
 
 // Sparse-stream decode of the token at position a.t (CUDA cores).

@@ -263,10 +263,12 @@ SSA_API ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* 
  *   when i + 1 <= k_eff;  h = softmax over A_t of scale q_t . k_u, times V.
  * Two state buffers carry the pooling between calls:
  *   qsum [B, Hq, d] fp32: sum of the queries of the current block so far;
- *   kbar [B, Hkv, n, d] fp32: means of the complete key blocks.
+ *   kbar [B, Hkv, n, d] fp32: means of the complete key blocks (16-byte
+ *     aligned for the decode step).
  * dims->N is the capacity of the K/V caches [B, Hkv, N, d] (a multiple of
- * block); Hq/Hkv * n * 4 bytes of scores must fit the decode kernel's shared
- * memory (SSA_ERR_UNSUPPORTED otherwise; every workload here fits). */
+ * block); the decode kernel's shared memory (n scores, the g heads' queries,
+ * partial outputs and selections, a 64-key K/V chunk) must fit a CTA
+ * (SSA_ERR_UNSUPPORTED otherwise; every workload here fits). */
 
 /* Builds the decode state from a prompt of t0 tokens (0 <= t0 <= N): kbar of
  * the complete blocks 0 .. t0/s - 1 and qsum of the queries of the partial
@@ -287,9 +289,9 @@ SSA_API ssa_status_t ssa_decode_prefill(const ssa_dims_t* dims, const ssa_tensor
  *   h [B, Hq, 1, d] (out), lse [B, Hq] fp32 (out, natural log of the
  *     softmax normaliser), idx [B, Hq, k_eff] int32 (out, Sel ascending,
  *     -1 padded).
- *   ws: workspace of at least ssa_workspace_bytes(dims) bytes (holds the
- *     union of the kept blocks and the partial softmax states of the split
- *     attention).
+ *   ws: workspace of at least ssa_workspace_bytes(dims) bytes (checked; the
+ *     step keeps its scratch in the shared memory of one thread-block cluster
+ *     per (batch, kv head) and does not write it).
  * Calls for consecutive tokens must be ordered (same stream). */
 SSA_API ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q,
                              const ssa_tensor_t* K, const ssa_tensor_t* V, int32_t t,
