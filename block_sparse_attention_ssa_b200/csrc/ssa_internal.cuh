@@ -155,6 +155,10 @@ cudaError_t launch_dropped_tc(const Dims& D, const FwdArgs& a, int32_t* dev_stat
 // bf16, d = 64 or 128, any block size and either selection mode.
 bool fwd_mma_supported(const Dims& D);
 cudaError_t launch_fwd_mma(const Dims& D, const FwdArgs& a, cudaStream_t st);
+// Sparse stream alone, blocks of 16 or 32, per-block selection (bf16, mma.sync):
+// each query block walks its own selected key blocks.
+bool fwd_walk_supported(const Dims& D);
+cudaError_t launch_fwd_walk(const Dims& D, const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_dropped_mma(const Dims& D, const FwdArgs& a, cudaStream_t st);
 
 // Tensor-core (tcgen05 / TMEM / TMA) dual-stream forward, bf16, d = 128.

@@ -191,6 +191,44 @@ def test_sparse_alone_never_reads_unselected_small_blocks(s, d):
     assert np.abs(f64(lse)[fin] - ora["lse_sel"][fin]).max() <= TOL["bf16"]["lse"]
 
 
+@pytest.mark.parametrize("s,d,g", [(16, 64, 4), (32, 64, 1), (16, 128, 2), (32, 128, 2)])
+def test_sparse_alone_small_blocks_given_selection(s, d, g):
+    """Given selections at blocks of 16 and 32: rows without their diagonal
+    block, duplicate entries, -1 padding, and one query block that attends
+    nothing (its h_sparse is zero and its lse_sel is -inf)."""
+    B, Hkv, N, k = 1, 2, 1088, 7
+    Hq = g * Hkv
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 939 + s + d, "bf16")
+    n = N // s
+    idx = custom_idx(B, Hq, n, k, seed=17 + s + d, drop_diag_frac=0.3, pad_frac=0.3)
+    idx[0, 1, n // 2] = -1
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
+    hs = torch.full((B, Hq, N, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device="cuda")
+    api.ssa_fwd_sparse(dims, dev["Q"], dev["K"], dev["V"], torch.from_numpy(idx).cuda(), hs, lse)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    ora = O.forward_sparse(host["Q"], host["K"], host["V"], idx, s, 1 / math.sqrt(d))
+    assert np.abs(f64(hs) - ora["h_sparse"]).max() <= TOL["bf16"]["out"]
+    fin = np.isfinite(ora["lse_sel"])
+    assert not fin[0, 1, (n // 2) * s:(n // 2 + 1) * s].any()
+    assert np.array_equal(np.isfinite(f64(lse)), fin)
+    assert np.all(f64(lse)[~fin] == -np.inf)
+    assert np.abs(f64(lse)[fin] - ora["lse_sel"][fin]).max() <= TOL["bf16"]["lse"]
+    assert torch.all(hs[0, 1, (n // 2) * s:(n // 2 + 1) * s].float() == 0)
+    g_up = make_upstream((B, Hq, N, d), 53)
+    grads = api.alloc_backward(dims)
+    ws = api.alloc_workspace(dims)
+    api.ssa_bwd_sparse(dims, dev["Q"], dev["K"], dev["V"], torch.from_numpy(idx).cuda(), hs, lse,
+                       upload(g_up, "bf16"), grads["dQ"], grads["dK"], grads["dV"], ws)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    dQ, dK, dV = O.backward_sparse(host["Q"], host["K"], host["V"], idx, s, 1 / math.sqrt(d),
+                                   oracle_view(g_up, "bf16").astype(np.float64))
+    for key, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        assert rel_l2(f64(got), ref) < TOL["bf16"]["grad"], key
+
+
 def test_decode_block16():
     """Decode at block 16 across several block boundaries, against the oracle."""
     B, Hq, Hkv, N, d, s, k = 1, 8, 2, 512, 64, 16, 16
