@@ -414,6 +414,7 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_build_mask(D, idx, a.mask, L.words, st);
   if (e != cudaSuccess) return from_cuda(e);
+  if (bwd_walk_supported(D)) return from_cuda(launch_bwd_walk(D, a, st));
   if (bwd_tc_supported(D)) {
     int32_t* status = device_status_ptr();
     if (status == nullptr) return SSA_ERR_CUDA;
