@@ -57,15 +57,14 @@ struct DqCfg {
   static constexpr int G = 4 / W;
   static constexpr int NS = D == 64 ? 3 : 2;
   static constexpr int LD = D + 8;
-  static constexpr int Q_BYTES = 16 * LD * 2;  // per warp: output staging
-  static constexpr int STAGE = S * LD * 2;
+  static constexpr int STAGE = S * LD * 2;  // stage 0 later stages the output
   static constexpr int GRP_BYTES = NS * 2 * STAGE;
-  static constexpr int SEL_OFF = 4 * Q_BYTES + G * GRP_BYTES;
+  static constexpr int SEL_OFF = G * GRP_BYTES;
   static constexpr int SMEM = SEL_OFF + G * 64 * 4;
 };
 
 template <int D, int S>
-__global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) bwd_dq_walk_kernel(BwdArgs a, WalkShape sh) {
+__global__ void __launch_bounds__(NT, D == 64 ? 4 : 2) bwd_dq_walk_kernel(BwdArgs a, WalkShape sh) {
   using C = DqCfg<D, S>;
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -77,8 +76,7 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) bwd_dq_walk_kernel(BwdArg
   const int r0 = t0 + warp * 16;
   const int64_t rowbase = ((int64_t)b * sh.Hq + h) * sh.N;
 
-  bf16 (*qs)[C::LD] = reinterpret_cast<bf16 (*)[C::LD]>(smem + warp * C::Q_BYTES);
-  unsigned char* gbase = smem + 4 * C::Q_BYTES + grp * C::GRP_BYTES;
+  unsigned char* gbase = smem + grp * C::GRP_BYTES;
   uint32_t* sel = reinterpret_cast<uint32_t*>(smem + C::SEL_OFF) + grp * 64;
   auto kbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(gbase + (2 * st) * C::STAGE); };
   auto vbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(gbase + (2 * st + 1) * C::STAGE); };
@@ -235,7 +233,8 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) bwd_dq_walk_kernel(BwdArg
     cur = next_blk(cur + 1);
   }
   cp_async_wait<0>();
-
+  group_sync<C::W>(grp);  // every warp of the group is done with the stages
+  bf16 (*qs)[C::LD] = kbuf(0) + (warp % C::W) * 16;  // this warp's 16 output rows
 #pragma unroll
   for (int n = 0; n < D / 8; ++n)
 #pragma unroll
@@ -250,6 +249,27 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) bwd_dq_walk_kernel(BwdArg
 }
 
 // ------------------------------------------------------------- dK, dV -----
+
+// maskT[b,h,j] = the set of query blocks i whose selection holds key block j:
+// the selection bit matrix of every head transposed in 32 x 32 tiles, one warp
+// per (32 query blocks, head) with ballots.
+__global__ void __launch_bounds__(32) mask_transpose_kernel(const uint32_t* __restrict__ mask,
+                                                            uint32_t* __restrict__ maskT, int n, int words) {
+  const int it = blockIdx.x, lane = threadIdx.x;
+  const int64_t base = (int64_t)blockIdx.y * n * words;
+  const int i = it * 32 + lane;
+  for (int jt = 0; jt < words; ++jt) {
+    const uint32_t w = (i < n && jt <= it) ? mask[base + (int64_t)i * words + jt] : 0u;  // j <= i only
+    uint32_t mine = 0u;
+#pragma unroll
+    for (int bit = 0; bit < 32; ++bit) {
+      const uint32_t col = __ballot_sync(0xffffffffu, (w >> bit) & 1u);
+      if (lane == bit) mine = col;
+    }
+    const int j = jt * 32 + lane;
+    if (j < n) maskT[base + (int64_t)j * words + it] = mine;
+  }
+}
 
 template <int D, int S>
 struct KvCfg {
@@ -284,23 +304,27 @@ __global__ void __launch_bounds__(NT) bwd_dkv_walk_kernel(BwdArgs a, WalkShape s
   }
   cp_async_commit();
 
-  // Query blocks i >= j whose selection holds j, ascending.
-  const uint32_t* mcol = a.mask + (rowbase / sh.N * sh.n) * sh.words + (j >> 5);
-  int total = 0;
-  for (int base = j; base < sh.n; base += NT) {
-    const int i = base + tid;
-    const bool hit = i < sh.n && ((mcol[(int64_t)i * sh.words] >> (j & 31)) & 1u);
-    const unsigned bal = __ballot_sync(0xffffffffu, hit);
-    if (lane == 0) wcnt[warp] = __popc(bal);
-    __syncthreads();
-    int off = total;
-    for (int w = 0; w < warp; ++w) off += wcnt[w];
-    if (hit) list[off + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)i;
-    total += wcnt[0] + wcnt[1] + wcnt[2] + wcnt[3];
-    __syncthreads();
+  // Query blocks whose selection holds j, ascending: lane l of warp 0 takes
+  // words 2l and 2l+1 of the transposed mask row, a warp scan places them.
+  if (warp == 0) {
+    const uint32_t* trow = a.maskT + (rowbase / sh.N * sh.n + j) * sh.words;
+    const uint32_t w0 = 2 * lane < sh.words ? trow[2 * lane] : 0u;
+    const uint32_t w1 = 2 * lane + 1 < sh.words ? trow[2 * lane + 1] : 0u;
+    const int c = __popc(w0) + __popc(w1);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int pos = incl - c;
+    for (uint32_t bits = w0; bits; bits &= bits - 1u) list[pos++] = (uint16_t)(64 * lane + __ffs(bits) - 1);
+    for (uint32_t bits = w1; bits; bits &= bits - 1u) list[pos++] = (uint16_t)(64 * lane + 32 + __ffs(bits) - 1);
+    if (lane == 31) wcnt[0] = incl;
   }
   cp_async_wait<0>();
-  __syncthreads();  // the K / V slice, copied by every thread, has landed
+  __syncthreads();  // the list and the K / V slice (copied by every thread) are in place
+  const int total = wcnt[0];
 
   unsigned char* ring = smem + warp * C::NS * C::STAGE;
   auto qbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(ring + st * C::STAGE); };
@@ -447,6 +471,12 @@ cudaError_t launch_t(const Dims& Dm, const BwdArgs& a, cudaStream_t st) {
     kern<<<dim3(Dm.N / BM, Dm.Hq, Dm.B), NT, C::SMEM, st>>>(a, sh);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    mask_transpose_kernel<<<dim3((Dm.n + 31) / 32, Dm.B * Dm.Hq), 32, 0, st>>>(a.mask, a.maskT, Dm.n, a.words);
+    count_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
   float* part = a.dhf;  // the dh_f and dO_c regions, unused by the sparse stream alone, hold g partials
   {

@@ -43,10 +43,9 @@ struct WalkCfg {
   static constexpr int G = 4 / W;                  // query blocks per CTA
   static constexpr int NS = D == 64 ? 3 : 2;       // K/V stages per query block
   static constexpr int LD = D + 8;                 // row pitch (conflict-free ldmatrix)
-  static constexpr int Q_BYTES = 16 * LD * 2;      // per warp: its Q rows, later its output staging
-  static constexpr int STAGE = S * LD * 2;         // one key (or value) block
+  static constexpr int STAGE = S * LD * 2;         // one key (or value) block; stage 0 stages the output
   static constexpr int GRP_BYTES = NS * 2 * STAGE;
-  static constexpr int SEL_OFF = 4 * Q_BYTES + G * GRP_BYTES;
+  static constexpr int SEL_OFF = G * GRP_BYTES;
   static constexpr int SMEM = SEL_OFF + G * 64 * 4;  // + one 2048-bit selection set per query block
 };
 
@@ -61,7 +60,7 @@ __device__ __forceinline__ void group_sync(int grp) {
 }
 
 template <int D, int S>
-__global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_walk_kernel(FwdArgs a, WalkShape sh) {
+__global__ void __launch_bounds__(NT, D == 64 ? 4 : 2) fwd_walk_kernel(FwdArgs a, WalkShape sh) {
   using C = WalkCfg<D, S>;
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -72,17 +71,10 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_walk_kernel(FwdArgs a
   const int i = t0 / S + grp;      // this group's query block
   const int r0 = t0 + warp * 16;   // this warp's first row
 
-  bf16 (*qs)[C::LD] = reinterpret_cast<bf16 (*)[C::LD]>(smem + warp * C::Q_BYTES);
-  unsigned char* gbase = smem + 4 * C::Q_BYTES + grp * C::GRP_BYTES;
+  unsigned char* gbase = smem + grp * C::GRP_BYTES;
   uint32_t* sel = reinterpret_cast<uint32_t*>(smem + C::SEL_OFF) + grp * 64;
   auto kbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(gbase + (2 * st) * C::STAGE); };
   auto vbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(gbase + (2 * st + 1) * C::STAGE); };
-
-  for (int e = lane; e < 16 * D / 8; e += 32) {
-    const int r = e / (D / 8), c = (e % (D / 8)) * 8;
-    cp_async16(&qs[r][c], row_ptr<bf16>(a.q, b, h, r0 + r) + c, 16);
-  }
-  cp_async_commit();
 
   for (int w = gt; w < 64; w += 32 * C::W) sel[w] = 0u;
   group_sync<C::W>(grp);
@@ -131,16 +123,24 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_walk_kernel(FwdArgs a
   for (int n = 0; n < D / 8; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
-  uint32_t qa[D / 16][4];
+  uint32_t qa[D / 16][4];  // the warp's Q rows as A fragments, straight from global memory
+  {
+    const bf16* q0p = row_ptr<bf16>(a.q, b, h, r0 + g8);
+    const bf16* q1p = row_ptr<bf16>(a.q, b, h, r0 + g8 + 8);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int c = kk * 16 + 2 * q4;
+      qa[kk][0] = *reinterpret_cast<const uint32_t*>(q0p + c);
+      qa[kk][1] = *reinterpret_cast<const uint32_t*>(q1p + c);
+      qa[kk][2] = *reinterpret_cast<const uint32_t*>(q0p + c + 8);
+      qa[kk][3] = *reinterpret_cast<const uint32_t*>(q1p + c + 8);
+    }
+  }
 
   int cur = next_blk(0);
   for (int it = 0; cur >= 0; ++it) {
     cp_async_wait<C::NS - 2>();
     group_sync<C::W>(grp);  // block `it` has landed for the group; stage (it - 1) is free
-    if (it == 0) {
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) ldsm_x4(qa[kk], &qs[lane & 15][kk * 16 + (lane >> 4) * 8]);
-    }
     {
       const int j = next_blk(issued + 1);
       if (j >= 0) {
@@ -219,7 +219,8 @@ __global__ void __launch_bounds__(NT, D == 64 ? 3 : 2) fwd_walk_kernel(FwdArgs a
     cur = next_blk(cur + 1);
   }
   cp_async_wait<0>();
-  __syncwarp();
+  group_sync<C::W>(grp);  // every warp of the group is done with the stages
+  bf16 (*qs)[C::LD] = kbuf(0) + (warp % C::W) * 16;  // this warp's 16 output rows
 
   float inv[2];
 #pragma unroll

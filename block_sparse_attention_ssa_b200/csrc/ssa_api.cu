@@ -91,7 +91,7 @@ ssa_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_E
 // ---------------------------------------------------------------- workspace
 struct Layout {
   size_t qbar, kbar;          // block scores
-  size_t dhf, doc, Df, Dc, mask, partials, kvpart;  // backward
+  size_t dhf, doc, Df, Dc, mask, partials, kvpart, maskT;  // backward
   size_t lse;                 // dropped mass
   size_t bytes_scores, bytes_bwd, bytes_dropped, bytes_align, bytes_decode;
   int words, n_partials;
@@ -115,6 +115,8 @@ Layout layout(const Dims& D) {
   L.partials = o; o = align_up(o + (size_t)L.n_partials * 4);
   L.kvpart = o;
   if (!bwd_tc_supported(D) && bwd_mma_supported(D)) o = align_up(o + bwd_mma_partial_bytes(D));
+  L.maskT = o;
+  if (bwd_walk_supported(D)) o = align_up(o + (size_t)D.B * D.Hq * D.n * L.words * 4);
   L.bytes_bwd = o;
   L.lse = 0;
   L.bytes_dropped = align_up(rows * 4);
@@ -414,7 +416,10 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_build_mask(D, idx, a.mask, L.words, st);
   if (e != cudaSuccess) return from_cuda(e);
-  if (bwd_walk_supported(D)) return from_cuda(launch_bwd_walk(D, a, st));
+  if (bwd_walk_supported(D)) {
+    a.maskT = at<uint32_t>(ws, L.maskT);
+    return from_cuda(launch_bwd_walk(D, a, st));
+  }
   if (bwd_tc_supported(D)) {
     int32_t* status = device_status_ptr();
     if (status == nullptr) return SSA_ERR_CUDA;

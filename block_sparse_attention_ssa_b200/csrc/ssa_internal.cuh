@@ -199,6 +199,8 @@ struct BwdArgs {
   // every (query block, key block) pair that is not selected.
   bool sparse_only;
   float* kvpart;       // warp-level tensor-core backward: fp32 dK / dV partials (or null)
+  uint32_t* maskT;     // sparse stream alone at blocks of 16 / 32: [B,Hq,n,words], bit i of row j set
+                       // when query block i selected key block j (or null)
 };
 
 cudaError_t launch_bwd_pre(const Dims& D, const BwdArgs& a, cudaStream_t st);
