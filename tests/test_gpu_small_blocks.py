@@ -229,6 +229,100 @@ def test_sparse_alone_small_blocks_given_selection(s, d, g):
         assert rel_l2(f64(got), ref) < TOL["bf16"]["grad"], key
 
 
+def _skewed_idx(B, H, n, k, seed):
+    """Every query block keeps key blocks 0 and 1 (with its diagonal and
+    random others): the dK/dV lists of those two key blocks hold every query
+    block, many pairs per warp."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    idx = np.full((B, H, n, k), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(n):
+                if i + 1 <= k:
+                    row = list(range(i + 1))
+                else:
+                    rest = rng.choice(np.arange(2, i), size=k - 3, replace=False).tolist()
+                    row = sorted([0, 1, i] + rest)
+                idx[b, h, i, :len(row)] = row
+    return idx
+
+
+@pytest.mark.parametrize("s,d", [(16, 64), (32, 128)])
+def test_sparse_alone_skewed_selection(s, d):
+    """The sparse stream alone when a few key blocks are chosen by every query
+    block, whole-problem parity of h_sparse, lse_sel, dQ, dK, dV."""
+    B, Hq, Hkv, N, k = 1, 4, 2, 2048, 5
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 951 + s, "bf16")
+    n = N // s
+    idx = _skewed_idx(B, Hq, n, k, 61 + s)
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
+    idx_d = torch.from_numpy(idx).cuda()
+    hs = torch.full((B, Hq, N, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device="cuda")
+    api.ssa_fwd_sparse(dims, dev["Q"], dev["K"], dev["V"], idx_d, hs, lse)
+    g_up = make_upstream((B, Hq, N, d), 59)
+    grads = api.alloc_backward(dims)
+    ws = api.alloc_workspace(dims)
+    api.ssa_bwd_sparse(dims, dev["Q"], dev["K"], dev["V"], idx_d, hs, lse, upload(g_up, "bf16"), grads["dQ"],
+                       grads["dK"], grads["dV"], ws)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    scale = 1 / math.sqrt(d)
+    ora = O.forward_sparse(host["Q"], host["K"], host["V"], idx, s, scale)
+    assert np.abs(f64(hs) - ora["h_sparse"]).max() <= TOL["bf16"]["out"]
+    assert np.abs(f64(lse) - ora["lse_sel"]).max() <= TOL["bf16"]["lse"]
+    dQ, dK, dV = O.backward_sparse(host["Q"], host["K"], host["V"], idx, s, scale,
+                                   oracle_view(g_up, "bf16").astype(np.float64))
+    for key, got, ref in (("dQ", grads["dQ"], dQ), ("dK", grads["dK"], dK), ("dV", grads["dV"], dV)):
+        assert rel_l2(f64(got), ref) < TOL["bf16"]["grad"], key
+    for j in (0, 1):  # the two key blocks every query block chose
+        rows = slice(j * s, (j + 1) * s)
+        assert rel_l2(f64(grads["dK"][:, :, rows]), dK[:, :, rows]) < TOL["bf16"]["grad"], ("dK", j)
+        assert rel_l2(f64(grads["dV"][:, :, rows]), dV[:, :, rows]) < TOL["bf16"]["grad"], ("dV", j)
+
+
+def test_sparse_alone_max_blocks_block16():
+    """The largest block count at block 16 (n = 2048, N = 32768): the
+    selection bit sets and dK/dV lists at full width; sampled query blocks of
+    h_sparse, lse_sel and dQ, and the last key block's dK, dV (only the last
+    query block can select it)."""
+    B, Hq, Hkv, N, d, s, k = 1, 2, 1, 32768, 64, 16, 16
+    host, dev = case_inputs(B, Hq, Hkv, N, d, s, 961, "bf16")
+    n = N // s
+    idx = custom_idx(B, Hq, n, k, seed=67, drop_diag_frac=0.1, pad_frac=0.1)
+    dims = api.make_dims(B, Hq, Hkv, N, d, s, k, "bf16")
+    idx_d = torch.from_numpy(idx).cuda()
+    hs = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    api.ssa_fwd_sparse(dims, dev["Q"], dev["K"], dev["V"], idx_d, hs, lse)
+    g_up = make_upstream((B, Hq, N, d), 71)
+    grads = api.alloc_backward(dims)
+    ws = api.alloc_workspace(dims)
+    api.ssa_bwd_sparse(dims, dev["Q"], dev["K"], dev["V"], idx_d, hs, lse, upload(g_up, "bf16"), grads["dQ"],
+                       grads["dK"], grads["dV"], ws)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    scale = 1 / math.sqrt(d)
+    g64 = oracle_view(g_up, "bf16").astype(np.float64)
+    for h, i in ((0, 0), (1, 5), (0, 777), (1, 1500), (0, n - 1), (1, n - 1)):
+        N1 = (i + 1) * s
+        sl = (slice(0, 1), slice(h, h + 1))
+        f = O.forward_sparse(host["Q"][sl + (slice(0, N1),)], host["K"][:, :, :N1], host["V"][:, :, :N1],
+                             idx[sl + (slice(0, i + 1),)], s, scale, qblocks=[i])
+        rows = slice(i * s, N1)
+        assert np.abs(f64(hs[0, h, rows]) - f["h_sparse"][0, 0, rows]).max() <= TOL["bf16"]["out"], (h, i)
+        if np.isfinite(f["lse_sel"][0, 0, rows]).all():
+            assert np.abs(f64(lse[0, h, rows]) - f["lse_sel"][0, 0, rows]).max() <= TOL["bf16"]["lse"], (h, i)
+        dQ, _, _ = O.backward_sparse(host["Q"][sl + (slice(0, N1),)], host["K"][:, :, :N1], host["V"][:, :, :N1],
+                                     idx[sl + (slice(0, i + 1),)], s, scale, g64[sl + (slice(0, N1),)],
+                                     qblocks=[i])
+        assert rel_l2(f64(grads["dQ"][0, h, rows]), dQ[0, 0, rows]) < TOL["bf16"]["grad"], (h, i)
+    _, dK, dV = O.backward_sparse(host["Q"], host["K"], host["V"], idx, s, scale, g64, qblocks=[n - 1])
+    rows = slice((n - 1) * s, N)
+    assert rel_l2(f64(grads["dK"][0, 0, rows]), dK[0, 0, rows]) < TOL["bf16"]["grad"]
+    assert rel_l2(f64(grads["dV"][0, 0, rows]), dV[0, 0, rows]) < TOL["bf16"]["grad"]
+
+
 def test_decode_block16():
     """Decode at block 16 across several block boundaries, against the oracle."""
     B, Hq, Hkv, N, d, s, k = 1, 8, 2, 512, 64, 16, 16
