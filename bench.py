@@ -532,8 +532,18 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
             raise RuntimeError(f"device status after the sparse rows: {api.status_string(status)}")
         f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
         b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+        if tc_path:
+            sparse_kernels = "fwd_tc (sparse mode); bwd_pre_tc + bwd_dkv_tc + bwd_dq_tc (tcgen05)"
+        elif w.dtype == "bf16" and w.block in (16, 32) and not args.per_token:
+            sparse_kernels = ("fwd_walk; mask + bwd_dq_walk + mask_transpose + bwd_dkv_walk + kvsum "
+                              "(mma.sync block walks: each query block visits only its own selected blocks)")
+        elif w.dtype == "bf16":
+            sparse_kernels = "fwd_mma (sparse mode); mask + bwd_dq_mma + bwd_dkv_mma (+ kvsum) (mma.sync)"
+        else:
+            sparse_kernels = "CUDA-core kernels (fp32)"
         extra["sparse_only"] = {
             "entry_points": "ssa_fwd_sparse, ssa_bwd_sparse (timed separately, not in value)",
+            "kernels": sparse_kernels,
             "sparse_pairs": pairs_sel, "share_of_causal_pairs": pairs_sel / w.causal_pairs(),
             "fwd_ms": f_ms, "bwd_ms": b_ms,
             "fwd_attended_tflops": 4 * w.d * pairs_sel / (f_ms * 1e-3) / 1e12,
