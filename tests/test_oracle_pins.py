@@ -609,3 +609,52 @@ def test_golden_fixture_is_reproduced():
     assert now["idx"] == gold["idx"]
     for key in ("delta", "lse_full", "lse_sel", "h_full_row0", "h_sparse_row0", "dQ_sum", "dK_sum", "dV_sum", "l_align"):
         np.testing.assert_allclose(np.array(now[key]), np.array(gold[key]), rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- sampled query blocks
+
+def test_query_block_sampling_matches_the_whole_problem():
+    """The full-size GPU checks compare sampled query blocks against the oracle
+    run on a prefix with qblocks=[i].  Causality fixes what that must give: rows
+    of block i see only keys u <= t, so the prefix of rows 0 .. (i+1)s - 1 with
+    only block i computed yields exactly the whole problem's rows of block i
+    (outputs, log-sum-exps, dropped mass, dQ, with the alignment term scaled by
+    the whole problem's element count M); and key block n-1 is reachable only
+    from query block n-1, so its dK, dV from qblocks=[n-1] alone are the whole
+    problem's."""
+    Q, K, V = tiny(Hq=4, Hkv=2, N=48, d=4, s=8, seed=11)
+    s, scale, k, alpha = 8, 0.41, 3, 10.0
+    N = Q.shape[2]
+    n = N // s
+    idx = O.select_blocks(O.block_scores(Q, K, s, scale), k)
+    g = make_upstream(Q.shape, 5)
+    M = Q.size
+    fs = O.forward_sparse(Q, K, V, idx, s, scale)
+    fd = O.forward_dual(Q, K, V, idx, s, scale)
+    dQs, dKs, dVs = O.backward_sparse(Q, K, V, idx, s, scale, g)
+    dQd, dKd, dVd, _, _ = O.ssa_backward(Q, K, V, idx, s, scale, None, g, alpha)
+    close = dict(rtol=1e-10, atol=1e-12)
+    for i in range(n):
+        N1, rows = (i + 1) * s, slice(i * s, (i + 1) * s)
+        pre = (Q[:, :, :N1], K[:, :, :N1], V[:, :, :N1], idx[:, :, :i + 1])
+        f = O.forward_sparse(*pre, s, scale, qblocks=[i])
+        np.testing.assert_allclose(f["h_sparse"][:, :, rows], fs["h_sparse"][:, :, rows], **close)
+        np.testing.assert_allclose(f["lse_sel"][:, :, rows], fs["lse_sel"][:, :, rows], **close)
+        f = O.forward_dual(*pre, s, scale, qblocks=[i])
+        for key in ("h_full", "h_sparse", "delta", "lse_full", "lse_sel"):
+            np.testing.assert_allclose(f[key][:, :, rows], fd[key][:, :, rows], **close, err_msg=key)
+        dq, _, _ = O.backward_sparse(*pre, s, scale, g[:, :, :N1], qblocks=[i])
+        np.testing.assert_allclose(dq[:, :, rows], dQs[:, :, rows], **close)
+        dq, _, _, _, _ = O.ssa_backward(*pre, s, scale, None, g[:, :, :N1], alpha, qblocks=[i], M=M)
+        np.testing.assert_allclose(dq[:, :, rows], dQd[:, :, rows], **close)
+    last = slice((n - 1) * s, N)
+    _, dk, dv = O.backward_sparse(Q, K, V, idx, s, scale, g, qblocks=[n - 1])
+    np.testing.assert_allclose(dk[:, :, last], dKs[:, :, last], **close)
+    np.testing.assert_allclose(dv[:, :, last], dVs[:, :, last], **close)
+    # the sample restricts: key block 0 takes gradient from query blocks other
+    # than the sampled one, so there the sample and the whole problem differ
+    assert not np.allclose(dk[:, :, :s], dKs[:, :, :s], rtol=1e-3, atol=1e-6)
+    _, dk, dv, _, _ = O.ssa_backward(Q, K, V, idx, s, scale, None, g, alpha, qblocks=[n - 1], M=M)
+    np.testing.assert_allclose(dk[:, :, last], dKd[:, :, last], **close)
+    np.testing.assert_allclose(dv[:, :, last], dVd[:, :, last], **close)
+    assert not np.allclose(dk[:, :, :s], dKd[:, :, :s], rtol=1e-3, atol=1e-6)
