@@ -417,6 +417,9 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
   cudaError_t e = launch_build_mask(D, idx, a.mask, L.words, st);
   if (e != cudaSuccess) return from_cuda(e);
   if (bwd_walk_supported(D)) {
+    // The walk's g per-head fp32 dK / dV partials fill the adjacent dh_f and
+    // dO_c regions (2 x B*Hq*N*d floats), which the sparse stream leaves unused.
+    if (L.Df - L.dhf < 2 * (size_t)D.B * D.Hq * D.N * D.d * sizeof(float)) return SSA_ERR_WORKSPACE;
     a.maskT = at<uint32_t>(ws, L.maskT);
     return from_cuda(launch_bwd_walk(D, a, st));
   }
