@@ -83,6 +83,28 @@ def measured_traffic(row: str, workload: str):
     return rec["dram_bytes_per_launch"]
 
 
+def selected_pairs(idx: np.ndarray, s: int, per_token: bool) -> int:
+    """Sum over query tokens t of |A_t|: the causal (t, u) pairs whose key block
+    is selected for t.  idx is [B, H, rows, k] (a row per query block, or per
+    token with per-token selection); entries < 0 or after the row's own block
+    are ignored and a block listed twice counts once.  A selected block j < i
+    gives each of the row's tokens s keys; the row's own block i gives token t
+    the t - i*s + 1 keys up to itself."""
+    import numpy as np
+
+    srt = np.sort(np.asarray(idx).astype(np.int64), axis=-1)
+    dup = np.zeros(srt.shape, dtype=bool)
+    dup[..., 1:] = srt[..., 1:] == srt[..., :-1]
+    rows_ax = np.arange(srt.shape[2], dtype=np.int64).reshape(1, 1, -1, 1)
+    i_ax = rows_ax // s if per_token else rows_ax
+    valid = (srt >= 0) & (srt <= i_ax) & ~dup
+    if per_token:
+        cnt = np.where(srt < i_ax, s, rows_ax - i_ax * s + 1)
+    else:
+        cnt = np.where(srt < i_ax, s * s, s * (s + 1) // 2)
+    return int((cnt * valid).sum())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -491,20 +513,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     # after the step; not part of `value`.  Attended FLOPs count the selected
     # causal pairs only: forward 4 d sum|A_t|, backward 10 d sum|A_t|.
     if not args.no_sparse:
-        # distinct causal selected blocks per selection row (a query block, or
-        # a token with per-token selection), each counted with its causal keys
-        srt = np.sort(out["idx"].cpu().numpy().astype(np.int64), axis=-1)
-        dup = np.zeros(srt.shape, dtype=bool)
-        dup[..., 1:] = srt[..., 1:] == srt[..., :-1]
-        rows_ax = np.arange(srt.shape[2], dtype=np.int64).reshape(1, 1, -1, 1)
-        s_ = w.block
-        i_ax = rows_ax // s_ if args.per_token else rows_ax
-        valid = (srt >= 0) & (srt <= i_ax) & ~dup
-        if args.per_token:
-            cnt = np.where(srt < i_ax, s_, rows_ax - i_ax * s_ + 1)
-        else:
-            cnt = np.where(srt < i_ax, s_ * s_, s_ * (s_ + 1) // 2)
-        pairs_sel = int((cnt * valid).sum())
+        pairs_sel = selected_pairs(out["idx"].cpu().numpy(), w.block, args.per_token)
         hs2 = torch.empty_like(out["h_sparse"])
         lse2 = torch.empty_like(out["lse_sel"])
 
