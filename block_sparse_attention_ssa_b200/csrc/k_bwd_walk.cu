@@ -281,7 +281,7 @@ struct KvCfg {
   static constexpr int RED = 2 * 4 * 16 * D * 4;              // four warps' dK, dV (fp32)
   static constexpr int KV_OFF = RING > RED ? RING : RED;
   static constexpr int LIST_OFF = KV_OFF + 2 * 16 * LD * 2;   // K and V slice staging
-  static constexpr int SMEM = LIST_OFF + 2048 * 2 + 16;       // query-block list + warp counts
+  static constexpr int SMEM = LIST_OFF + 2048 * 2 + 16;       // query-block list (n <= 2048) + its length
 };
 
 template <int D, int S>
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(NT) bwd_dkv_walk_kernel(BwdArgs a, WalkShape s
   const int64_t rowbase = ((int64_t)b * sh.Hq + h) * sh.N;
   bf16 (*kvs)[C::LD] = reinterpret_cast<bf16 (*)[C::LD]>(smem + C::KV_OFF);  // rows 0-15 K, 16-31 V
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::LIST_OFF);
-  int* wcnt = reinterpret_cast<int*>(smem + C::LIST_OFF + 2048 * 2);
+  int* list_len = reinterpret_cast<int*>(smem + C::LIST_OFF + 2048 * 2);
 
   for (int e = tid; e < 2 * 16 * D / 8; e += NT) {
     const int r = e / (D / 8), c = (e % (D / 8)) * 8;
@@ -320,11 +320,11 @@ __global__ void __launch_bounds__(NT) bwd_dkv_walk_kernel(BwdArgs a, WalkShape s
     int pos = incl - c;
     for (uint32_t bits = w0; bits; bits &= bits - 1u) list[pos++] = (uint16_t)(64 * lane + __ffs(bits) - 1);
     for (uint32_t bits = w1; bits; bits &= bits - 1u) list[pos++] = (uint16_t)(64 * lane + 32 + __ffs(bits) - 1);
-    if (lane == 31) wcnt[0] = incl;
+    if (lane == 31) *list_len = incl;
   }
   cp_async_wait<0>();
   __syncthreads();  // the list and the K / V slice (copied by every thread) are in place
-  const int total = wcnt[0];
+  const int total = *list_len;
 
   unsigned char* ring = smem + warp * C::NS * C::STAGE;
   auto qbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(ring + st * C::STAGE); };
