@@ -38,7 +38,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
 PAGES_DROPPED_MASS = 0.47  # share of attention mass dropped by sparse attention in full-attention models
 
 
@@ -110,7 +111,7 @@ def load_peaks():
     if os.path.exists(p):
         with open(p) as fh:
             d = json.load(fh)
-        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+        return {k: float(d.get(k, v)) for k, v in FALLBACK_PEAKS.items()}, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
 
 
@@ -482,12 +483,23 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
             return {"bound": "alu", "kernel": r, "scope": scopes[r], "achieved": achieved, "peak": alu_peak,
                     "unit": "TFLOP/s", "frac": achieved / alu_peak, "traffic": None,
                     "peak_source": "fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz (attended FLOPs counted)"}
+        # The burst peak is the denominator: the step is tens of milliseconds
+        # (the timed region well under a second), the regime of a GEMM timed
+        # alone, not the seconds-long power-capped loop behind the sustained
+        # figure.  The clock-normalised figure scales the achieved rate to the
+        # maximum SM clock by the median clock sampled during the timed region,
+        # so fractions taken at different clocks compare.
+        med = clocks.get("sm_mhz") if clocks else None
+        mx = (clocks.get("sm_max_mhz") if clocks else None) or peaks.get("sm_max_mhz")
+        at_max = achieved * mx / med if (med and mx) else None
         return {"bound": "tensor", "kernel": r, "scope": scopes[r], "achieved": achieved,
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops_sustained"],
-                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "sm_mhz_median": med, "achieved_at_sm_max_mhz": at_max,
                 "traffic": measured_traffic(r, w.name),
-                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); burst {peaks['bf16_tflops']}"}
+                "peak_source": (f"{peak_src} bf16 burst (cuBLAS 8192^3 GEMM, best of 10); "
+                                f"sustained {peaks['bf16_tflops_sustained']} reported beside it")}
 
     dom = max(row_flops, key=lambda r: row_ms[r])
     roofline = roof(dom)
@@ -495,8 +507,8 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     for r, f in row_flops.items():
         per_row[r]["attended_tflops"] = f / (row_ms[r] * 1e-3) / 1e12
         if tc_path or mma_path:
-            per_row[r]["frac_of_sustained_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops_sustained"]
             per_row[r]["frac_of_burst_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops"]
+            per_row[r]["frac_of_sustained_peak"] = per_row[r]["attended_tflops"] / peaks["bf16_tflops_sustained"]
         else:
             per_row[r]["frac_of_fp32_fma_peak"] = per_row[r]["attended_tflops"] / alu_peak
     fwd_ms = row_ms["block_scores"] + row_ms["select_topk"] + row_ms["fwd_dual"]

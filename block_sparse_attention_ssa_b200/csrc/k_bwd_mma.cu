@@ -814,7 +814,7 @@ cudaError_t launch_bwd_mma(const Dims& D, const BwdArgs& a, int32_t* status, cud
     if (e != cudaSuccess) return e;
   }
   // Dual backward at d = 64: the tcgen05 kernels with per-row masks.
-  if (!a.sparse_only && status != nullptr && bwd_tcm_supported(D))
+  if (!a.sparse_only && bwd_tcm_supported(D))
     return launch_bwd_tcm(D, a, dhf, doc, bwd_mma_heads_per_cta(D), status, st);
   if (D.d == 128)
     return a.sparse_only ? bwd_t<128, true>(D, a, dhf, doc, st) : bwd_t<128, false>(D, a, dhf, doc, st);

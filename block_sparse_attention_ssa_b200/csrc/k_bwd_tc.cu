@@ -322,7 +322,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDhf,
                       const __grid_constant__ CUtensorMap tmDhs, BwdTcParams p) {
   using namespace dkv;
-  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
   // Used directly (no pointer arithmetic on the address) so that accesses
   // through it stay shared-memory loads; TMA tiles with 128-byte swizzle need
   // the 1024-byte alignment, which is checked rather than assumed.
@@ -668,7 +667,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      TensorRef Qr, TensorRef dhf_r, TensorRef dhs_r, BwdTcParams p) {
   using namespace dq;
-  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   if (smem_u32(smem) & 1023u) {

@@ -120,7 +120,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOc,
                       const __grid_constant__ CUtensorMap tmF, TcmBwdParams p) {
   using namespace dqm;
-  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   Misc& M = *reinterpret_cast<Misc*>(smem + OFF_MISC);
@@ -384,7 +383,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOc,
                        const __grid_constant__ CUtensorMap tmF, TcmBwdParams p) {
   using namespace dkvm;
-  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   Misc& M = *reinterpret_cast<Misc*>(smem + OFF_MISC);

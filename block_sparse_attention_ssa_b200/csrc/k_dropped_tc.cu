@@ -70,7 +70,6 @@ template <int S_BLK, bool GIVEN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     dropped_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, DParams p) {
   using C = DCfg;
-  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
   // Used directly (no pointer arithmetic on the address) so that accesses
   // through it stay shared-memory loads; TMA tiles with 128-byte swizzle need
   // the 1024-byte alignment, which is checked rather than assumed.

@@ -117,7 +117,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tmV, TcmParams p) {
   using C = Cfg<HD>;
   constexpr int NS = C::NS;
-  if (*reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Misc<NS>& M = *reinterpret_cast<Misc<NS>*>(smem + C::OFF_MISC);

@@ -4,6 +4,7 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
 #include <nvtx3/nvToolsExt.h>
 
 #include "ssa_internal.cuh"
@@ -308,7 +309,9 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
   }
   if (bwd_mma_supported(D)) {
     a.kvpart = at<float>(ws, L.kvpart);
-    return from_cuda(launch_bwd_mma(D, a, device_status_ptr(), st));
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_bwd_mma(D, a, status, st));
   }
   e = launch_bwd_pre(D, a, st);
   if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
@@ -430,7 +433,9 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
   }
   if (bwd_mma_supported(D)) {
     a.kvpart = at<float>(ws, L.kvpart);
-    return from_cuda(launch_bwd_mma(D, a, device_status_ptr(), st));
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_bwd_mma(D, a, status, st));
   }
   e = launch_bwd_pre(D, a, st);
   if (e == cudaSuccess) e = launch_bwd_simt(D, a, st);
@@ -579,18 +584,49 @@ namespace {
 
 constexpr int kMaxDevices = 128;
 float* g_noalloc_ptr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};  // context the cached address belongs to
 std::mutex g_noalloc_mu;
 
-// Device address of g_noalloc_scratch on the current device, looked up once.
+// Unique id of the calling thread's current CUDA context (0 if unavailable).
+// cudaDeviceReset destroys a device's primary context; the next runtime call
+// creates a new one with a new id, in which the library's module -- and with
+// it the scratch array -- is loaded again, possibly at another address.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur == nullptr || get_id == nullptr || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch on the current device: looked up once
+// per device, and again whenever the device's context has been replaced since.
 ssa_status_t noalloc_scratch(float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SSA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_noalloc_ptr[dev] == nullptr || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return SSA_ERR_CUDA;
     g_noalloc_ptr[dev] = static_cast<float*>(p);
+    // cudaGetSymbolAddress made the primary context current if it was not.
+    g_noalloc_ctx[dev] = ctx != 0 ? ctx : current_context_id();
   }
   *out = g_noalloc_ptr[dev];
   return SSA_OK;
@@ -602,6 +638,7 @@ ssa_status_t noalloc_scratch(float** out) {
 extern "C" ssa_status_t ssa_block_scores_noalloc(const ssa_dims_t* dims, const ssa_tensor_t* Q,
                                                  const ssa_tensor_t* K, float* scores,
                                                  ssa_stream_t stream) {
+  const NvtxRange nvtx_range("ssa_block_scores_noalloc");
   Dims D;
   bool empty = false;
   ssa_status_t s = check_dims(dims, &D, &empty);

@@ -52,10 +52,12 @@
  *   or a device that is not sm_100) or SSA_ERR_WORKSPACE (ws_bytes below
  *   ssa_workspace_bytes) and enqueues nothing.  A failed launch returns
  *   SSA_ERR_CUDA.  Kernels that wait on hardware barriers bound every wait;
- *   a wait that runs out records SSA_ERR_TIMEOUT in a device status word
- *   (read it with ssa_device_status) and the kernel returns.  While that word
- *   holds an error, the tensor-core kernels skip their work (their outputs
- *   are then undefined) until ssa_device_status clears it.  No kernel traps.
+ *   a wait that runs out records SSA_ERR_TIMEOUT in a per-device status
+ *   report (read and clear it with ssa_device_status) and the kernel returns;
+ *   the outputs of that call are then undefined.  The report changes nothing
+ *   for later calls: every call does its full work whatever the report
+ *   holds, so a timed-out call on one stream leaves calls on other streams
+ *   correct.  No kernel traps.
  * Precision.  dtype SSA_BF16: inputs/outputs bf16, products on tensor cores
  *   with fp32 accumulation and fp32 softmax statistics.  SSA_F32: fp32 inputs
  *   and outputs, fp32 arithmetic throughout (CUDA cores).
@@ -343,7 +345,9 @@ SSA_API ssa_status_t ssa_align_mse(const ssa_dims_t* dims, const ssa_tensor_t* h
  *     B * (Hq + Hkv) * n * d > SSA_NOALLOC_SCRATCH_FLOATS.
  * The first call on a device looks up the array's device address once (with
  * that device current) and caches it; make that first call before any
- * stream capture.  All calls share the one array and it keeps the last
+ * stream capture.  After cudaDeviceReset the next call looks the address up
+ * again in the device's new context (so that call, too, belongs before any
+ * capture).  All calls share the one array and it keeps the last
  * call's contents; nothing in it needs to start at zero, because every value
  * the scoring kernel reads was written by the same call.  Calls whose work
  * overlaps on the GPU (different streams, or different host threads without
@@ -359,15 +363,17 @@ SSA_API uint64_t ssa_launch_count(void);
 /* Failure-detection self-test.  Enqueues a one-CTA kernel that waits on a
  * barrier nothing will ever complete, using the same bounded wait as every
  * tensor-core kernel; after about 10 ms the wait gives up, the kernel records
- * SSA_ERR_TIMEOUT in the device status word and returns.  Nothing faults or
- * hangs; the status word then behaves as after a real timeout (read and clear
- * it with ssa_device_status).  Returns SSA_ERR_UNSUPPORTED off sm_100. */
+ * SSA_ERR_TIMEOUT in the device status report and returns.  Nothing faults
+ * or hangs; the report then reads as after a real timeout (read and clear it
+ * with ssa_device_status).  Returns SSA_ERR_UNSUPPORTED off sm_100. */
 SSA_API ssa_status_t ssa_selftest_timeout(ssa_stream_t stream);
 
-/* Synchronises `stream`, copies the device status word of the current device
- * to *status (SSA_OK, or the first SSA_ERR_TIMEOUT a kernel recorded) and,
- * if clear != 0, resets it.  Returns SSA_ERR_CUDA if the synchronisation or
- * the copy fails. */
+/* Synchronises `stream`, copies the status report of the current device to
+ * *status (SSA_OK, or SSA_ERR_TIMEOUT once any kernel of this library on the
+ * device -- any stream, any host thread -- gave up on a wait since the last
+ * clear) and, if clear != 0, resets it.  The report is only read here: no
+ * kernel consults it.  Returns SSA_ERR_CUDA if the synchronisation or the
+ * copy fails. */
 SSA_API ssa_status_t ssa_device_status(int32_t* status, int clear, ssa_stream_t stream);
 
 #ifdef __cplusplus

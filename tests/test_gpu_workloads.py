@@ -8,6 +8,9 @@ configuration bench.py times (same entry points, same buffers, one stream).
   that the oracle computes one by one from the prefix they depend on:
   forward rows, dropped mass, dQ rows of the sampled query blocks, and dK / dV
   of the last key block of a kv head (which only its own query block reaches).
+* dK / dV of one whole (batch, kv head) group are checked at full size on
+  gqa_16k and on sweep_32k with k = 64, with the oracle's backward over every
+  query block of the group (the early key blocks collect from all of them).
 """
 import math
 
@@ -116,6 +119,74 @@ def _check_backward_samples(w, host, grads, ora_idx, scale, rng):
     rows = slice((n - 1) * s, w.N)
     assert rel_l2(f64(grads["dK"][b, kv, rows]), dK[0, 0, rows]) < tol
     assert rel_l2(f64(grads["dV"][b, kv, rows]), dV[0, 0, rows]) < tol
+
+
+def _compare_group(w, got_k, got_v, dK, dV, rng, what):
+    tol = TOL[w.dtype]["grad"]
+    s, n = w.block, w.n_blocks
+    assert rel_l2(got_k, dK) < tol, (w.name, what, "dK")
+    assert rel_l2(got_v, dV) < tol, (w.name, what, "dV")
+    for j in sorted({0, n // 2, int(rng.integers(n))}):
+        rows = slice(j * s, (j + 1) * s)
+        ek, ev = rel_l2(got_k[rows], dK[rows]), rel_l2(got_v[rows], dV[rows])
+        assert ek < tol and ev < tol, (w.name, what, "key block", j, ek, ev)
+
+
+def test_full_size_group_backward_gqa16k():
+    """dK, dV of one whole (batch, kv head) group of gqa_16k in the bench's
+    configuration (sum(h_sparse), alpha = 10): the oracle runs the backward
+    over every query block of the group's g heads, so every key block
+    receives all its contributions -- key block 0 from all n query blocks of
+    each head, the longest walks of the dK/dV kernel.  Compared on the whole
+    group and on key blocks 0, n/2 and a random one."""
+    w = WORKLOADS["gqa_16k"]
+    rng = np.random.Generator(np.random.PCG64(4242))
+    host, _, grads, _, ora_idx, scale = _run(w, with_bwd=True)
+    M = w.B * w.Hq * w.N * w.d
+    b, kv = int(rng.integers(w.B)), int(rng.integers(w.Hkv))
+    heads = slice(kv * w.group, (kv + 1) * w.group)
+    g = np.ones((1, w.group, w.N, w.d))
+    _, dK, dV, _, _ = O.ssa_backward(host["Q"][b:b + 1, heads], host["K"][b:b + 1, kv:kv + 1],
+                                     host["V"][b:b + 1, kv:kv + 1], ora_idx[b:b + 1, heads], w.block, scale, None, g,
+                                     10.0, M=M)
+    _compare_group(w, f64(grads["dK"][b, kv]), f64(grads["dV"][b, kv]), dK[0, 0], dV[0, 0], rng, (b, kv))
+
+
+def test_full_size_group_backward_sweep32k_k64():
+    """The same at sweep_32k with k = 64 (n = 512 key blocks, 64 selected per
+    query block), with the upstream gradient on the full stream of one query
+    head of the group (zero elsewhere, alpha = 0) so that the oracle needs one
+    head: the kernel still walks all g heads and every causal query tile for
+    each key tile, 512 of them for key block 0, adding the other heads' exact
+    zeros."""
+    w = WORKLOADS["sweep_32k"].with_topk(64)
+    rng = np.random.Generator(np.random.PCG64(4343))
+    host = make_workload_inputs(w)
+    dev = _device(w, host)
+    dims = api.make_dims(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, w.topk, w.dtype)
+    ws = api.alloc_workspace(dims)
+    out = api.alloc_forward(dims)
+    api.forward(dims, dev["Q"], dev["K"], dev["V"], out, ws)
+    torch.cuda.synchronize()
+    scale = 1.0 / math.sqrt(w.d)
+    ora_scores = O.block_scores(host["Q"], host["K"], w.block, scale)
+    ora_idx = O.select_blocks(ora_scores, w.topk)
+    if compare_selection(out["idx"].cpu().numpy(), ora_idx, ora_scores):
+        out["idx"].copy_(torch.from_numpy(ora_idx))
+        api.ssa_fwd_dual(dims, dev["Q"], dev["K"], dev["V"], out["idx"], out["h_full"], out["h_sparse"],
+                         out["lse_full"], out["lse_sel"], out["delta"])
+    b, kv = 0, int(rng.integers(w.Hkv))
+    h = kv * w.group + int(rng.integers(w.group))
+    g_full = torch.zeros((w.B, w.Hq, w.N, w.d), dtype=dims.torch_dtype, device="cuda")
+    g_full[b, h] = 1.0
+    grads = api.alloc_backward(dims)
+    api.backward(dims, dev["Q"], dev["K"], dev["V"], out, g_full, None, 0.0, grads, ws)
+    torch.cuda.synchronize()
+    assert api.ssa_device_status() == api.SSA_OK
+    _, dK, dV = O.backward_streams(host["Q"][b:b + 1, h:h + 1], host["K"][b:b + 1, kv:kv + 1],
+                                   host["V"][b:b + 1, kv:kv + 1], ora_idx[b:b + 1, h:h + 1], w.block, scale,
+                                   np.ones((1, 1, w.N, w.d)), None)
+    _compare_group(w, f64(grads["dK"][b, kv]), f64(grads["dV"][b, kv]), dK[0, 0], dV[0, 0], rng, (b, h))
 
 
 def test_tiny_f32_whole_problem():
