@@ -548,12 +548,8 @@ cudaError_t launch_ord(const Dims& D, const FwdArgs& a, int32_t* status, cudaStr
 
 }  // namespace
 
-bool fwd_ord_supported(const Dims& D) {
-  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048 && !D.per_token;
-}
-
 cudaError_t launch_fwd_ord(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st) {
-  if (!fwd_ord_supported(D)) return cudaErrorNotSupported;
+  if (!fwd_tc_supported(D)) return cudaErrorNotSupported;
   if (a.sparse_only)
     return D.s == 64 ? launch_ord<64, true>(D, a, dev_status, st) : launch_ord<128, true>(D, a, dev_status, st);
   return D.s == 64 ? launch_ord<64, false>(D, a, dev_status, st) : launch_ord<128, false>(D, a, dev_status, st);

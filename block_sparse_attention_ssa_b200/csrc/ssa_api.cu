@@ -249,7 +249,7 @@ ssa_status_t ssa_fwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
   if (fwd_tc_supported(D) || fwd_tcm_supported(D)) {
     int32_t* status = device_status_ptr();
     if (status == nullptr) return SSA_ERR_CUDA;
-    return from_cuda(fwd_ord_supported(D) ? launch_fwd_ord(D, a, status, st) : launch_fwd_tcm(D, a, status, st));
+    return from_cuda(fwd_tc_supported(D) ? launch_fwd_ord(D, a, status, st) : launch_fwd_tcm(D, a, status, st));
   }
   if (fwd_mma_supported(D)) return from_cuda(launch_fwd_mma(D, a, st));
   return from_cuda(launch_fwd_simt(D, a, st));
@@ -362,7 +362,7 @@ ssa_status_t ssa_fwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
   a.lse_sel = lse_sel;
   a.sparse_only = true;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (fwd_ord_supported(D)) {
+  if (fwd_tc_supported(D)) {
     int32_t* status = device_status_ptr();
     if (status == nullptr) return SSA_ERR_CUDA;
     return from_cuda(launch_fwd_ord(D, a, status, st));

@@ -161,14 +161,14 @@ bool fwd_walk_supported(const Dims& D);
 cudaError_t launch_fwd_walk(const Dims& D, const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_dropped_mma(const Dims& D, const FwdArgs& a, cudaStream_t st);
 
-// Tensor-core (tcgen05 / TMEM / TMA) dual-stream forward, bf16, d = 128.
-// Returns cudaErrorNotSupported when the shape is outside its envelope.
-cudaError_t launch_fwd_tc(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
+// Envelope of the first tensor-core kernels: bf16, d = 128, blocks of 64 or
+// 128, per-block selection (n <= 2048).
 bool fwd_tc_supported(const Dims& D);
-// The same envelope, selected blocks first: one softmax and one accumulator
-// per query tile, h_sparse read off after the selected blocks, two CTAs per SM.
+// Tensor-core (tcgen05 / TMEM / TMA) dual-stream forward and sparse stream
+// alone in that envelope, selected blocks first: one softmax and one
+// accumulator per query tile, h_sparse read off after the selected blocks, two
+// CTAs per SM.  Returns cudaErrorNotSupported outside the envelope.
 cudaError_t launch_fwd_ord(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
-bool fwd_ord_supported(const Dims& D);
 
 // 4-D TMA map over a [B, H, N, d] bf16 tensor (d = 64 or 128): dims
 // (d, N, H, B), box (64 columns, `rows` rows), 128-byte swizzle, zero fill
