@@ -78,7 +78,10 @@ def measured_traffic(row: str, workload: str):
     if not rec:
         return None
     for src, sha in rec["source_sha256"].items():
-        with open(os.path.join(ROOT, src), "rb") as fh:
+        path_src = os.path.join(ROOT, src)
+        if not os.path.exists(path_src):
+            return None
+        with open(path_src, "rb") as fh:
             if hashlib.sha256(fh.read()).hexdigest() != sha:
                 return None
     return rec["dram_bytes_per_launch"]
@@ -461,7 +464,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
     tc_path = w.dtype == "bf16" and w.d == 128 and w.block in (64, 128) and not args.per_token
     mma_path = w.dtype == "bf16" and not tc_path
     if tc_path:
-        scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_tc_kernel)",
+        scopes = {"fwd_dual": "entry point ssa_fwd_dual = one kernel (fwd_ord_kernel: selected blocks first, two CTAs per SM)",
                   "bwd_dual": "entry point ssa_bwd_dual = mask + bwd_pre_tc + finish + bwd_dkv_tc + bwd_dq_tc kernels",
                   "dropped_mass": "entry point ssa_dropped_mass = one kernel (dropped_tc_kernel)"}
     elif mma_path:
@@ -554,7 +557,7 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
         f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
         b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
         if tc_path:
-            sparse_kernels = "fwd_tc (sparse mode); bwd_pre_tc + bwd_dkv_tc + bwd_dq_tc (tcgen05)"
+            sparse_kernels = "fwd_ord (phase A only); bwd_pre_tc + bwd_dkv_tc + bwd_dq_tc (tcgen05)"
         elif w.dtype == "bf16" and w.block in (16, 32) and not args.per_token:
             sparse_kernels = ("fwd_walk; mask + bwd_dq_walk + mask_transpose + bwd_dkv_walk + kvsum "
                               "(mma.sync block walks: each query block visits only its own selected blocks)")
