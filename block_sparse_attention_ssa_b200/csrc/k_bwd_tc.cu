@@ -125,17 +125,77 @@ struct BwdTcParams {
   TensorRef dq, dk, dv;     // outputs (bf16, strided)
   const float* lse2[2];     // [B,Hq,N] per stream (0 = full, 1 = sparse), base 2
   const float* D[2];        // [B,Hq,N] per stream
-  const uint32_t* mask;     // [B,Hq,n,words]
-  int words;
+  const uint32_t* mask;     // [B,Hq,rows,words]: a row per query block (or per token)
+  int words, rows;
   int32_t* status;
-  int Hq, g, N, n, s, NT;   // NT = number of 128-row tiles
+  int Hq, g, N, n, s, ls, NT;  // ls = log2(s); NT = number of 128-row tiles
   int full;                 // 0: sparse stream alone (no stream-f steps)
+  // Element masks for the sparse stream: blocks of 16 / 32, or a selection
+  // per token, make the selected set vary inside a 64 x 64 quarter of a step.
+  int fine, per_token;
+  // dK / dV kernel: a CTA walks hpc of the g query heads of its kv head; with
+  // more than one chunk per group it writes fp32 partials [chunk][2][B][Hkv][N][d]
+  // (dK unscaled, dV) that a second kernel adds in chunk order.
+  int hpc;
+  float* part;
   float c;                  // scale * log2(e)
   float scale;
 };
 
+// Word j / 32 of selection row i (a query block, or a token when per_token).
 __device__ __forceinline__ uint32_t mask_word(const BwdTcParams& p, int b, int h, int i, int j) {
-  return __ldg(p.mask + (((int64_t)b * p.Hq + h) * p.n + i) * p.words + (j >> 5));
+  return __ldg(p.mask + (((int64_t)b * p.Hq + h) * p.rows + i) * p.words + (j >> 5));
+}
+
+// Selection bits of key blocks kb0 .. kb0 + nb - 1 (nb | 32, kb0 a multiple of
+// nb, so they share a word) for selection row i, in the low nb bits.
+__device__ __forceinline__ uint32_t row_key_bits(const BwdTcParams& p, int b, int h, int i, int kb0, int nb) {
+  const uint32_t w = mask_word(p, b, h, i, kb0) >> (kb0 & 31);
+  return nb >= 32 ? w : (w & ((1u << nb) - 1u));
+}
+
+// Fine selections: bit c of the result is set when query t0 + c (c < 64,
+// queries past N excluded) selected the key block of key u (lane-cooperative:
+// every lane of the warp passes the same t0; u may differ per lane).
+__device__ __forceinline__ unsigned long long query_sel_mask64(const BwdTcParams& p, int b, int h, int t0, int u,
+                                                               int lane) {
+  const int kb = u >> p.ls, sh = kb & 31;
+  if (!p.per_token) {
+    // the 64 queries span 64 / s query blocks (or lie inside one block)
+    unsigned long long m = 0ull;
+    const int qb0 = t0 >> p.ls, nq = p.s >= 64 ? 1 : 64 >> p.ls;
+    for (int e = 0; e < nq; ++e) {
+      const int qb = qb0 + e;
+      if (qb >= p.n) break;
+      if ((mask_word(p, b, h, qb, kb) >> sh) & 1u)
+        m |= (p.s >= 64 ? ~0ull : ((1ull << p.s) - 1ull) << (e * p.s));
+    }
+    return m;
+  }
+  const int ta = t0 + lane, tb = t0 + 32 + lane;
+  const uint32_t wa = ta < p.N ? mask_word(p, b, h, ta, kb) : 0u;  // word index is lane-uniform per key tile
+  const uint32_t wb = tb < p.N ? mask_word(p, b, h, tb, kb) : 0u;
+  unsigned long long m = 0ull;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const uint32_t xa = __shfl_sync(0xffffffffu, wa, c), xb = __shfl_sync(0xffffffffu, wb, c);
+    m |= (unsigned long long)((xa >> sh) & 1u) << c;
+    m |= (unsigned long long)((xb >> sh) & 1u) << (32 + c);
+  }
+  return m;
+}
+
+// Fine selections: bit c set when key u0 + c (c < 64) lies in a block that
+// selection row i selected.
+__device__ __forceinline__ unsigned long long key_sel_mask64(const BwdTcParams& p, int b, int h, int i, int u0) {
+  if (p.s >= 64) return ((mask_word(p, b, h, i, u0 >> p.ls) >> ((u0 >> p.ls) & 31)) & 1u) ? ~0ull : 0ull;
+  const int nb = 64 >> p.ls;
+  const uint32_t bits = row_key_bits(p, b, h, i, u0 >> p.ls, nb);
+  unsigned long long m = 0ull;
+  const unsigned long long run = (1ull << p.s) - 1ull;
+  for (int e = 0; e < nb; ++e)
+    if ((bits >> e) & 1u) m |= run << (e * p.s);
+  return m;
 }
 
 // Which (query block, key block) pairs of the 128 x 128 tile (qt, kt) of query
@@ -143,6 +203,21 @@ __device__ __forceinline__ uint32_t mask_word(const BwdTcParams& p, int b, int h
 // 64), all four bits for block 128.  Blocks past the end and key blocks after
 // the query block are never set.
 __device__ __forceinline__ uint32_t tile_bits(const BwdTcParams& p, int b, int h, int qt, int kt) {
+  if (p.fine) {
+    // any selected (query, key) pair in the step: the 128 keys are 128 / s
+    // blocks of one word; element masks then pick the pairs
+    if (kt > qt) return 0u;
+    const int nb = 128 >> p.ls, kb0 = (kt * TILE) >> p.ls;
+    uint32_t any = 0u;
+    if (p.per_token) {
+      const int t1 = min(qt * TILE + TILE, p.N);
+      for (int t = qt * TILE; t < t1 && !any; ++t) any |= row_key_bits(p, b, h, t, kb0, nb);
+    } else {
+      const int i1 = min(((qt + 1) * TILE) >> p.ls, p.n);
+      for (int i = (qt * TILE) >> p.ls; i < i1 && !any; ++i) any |= row_key_bits(p, b, h, i, kb0, nb);
+    }
+    return any ? 0xFu : 0u;
+  }
   if (p.s == 128) {
     if (kt > qt || qt >= p.n) return 0u;
     return ((mask_word(p, b, h, qt, kt) >> (kt & 31)) & 1u) ? 0xFu : 0u;
@@ -317,6 +392,7 @@ static_assert(SMEM <= kMaxSmem, "dkv shared-memory budget");
 static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
 }  // namespace dkv
 
+template <bool FINE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDhf,
@@ -335,10 +411,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   volatile int* abort = &M.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = (int)blockIdx.x;  // low key tiles have the most query tiles and launch first
-  const int kvh = blockIdx.y, b = blockIdx.z;
+  const int chunks = p.g / p.hpc;
+  const int kvh = blockIdx.y / chunks, chunk = blockIdx.y % chunks, b = blockIdx.z;
+  const int h0 = kvh * p.g + chunk * p.hpc;  // first query head of this CTA
   const int u0 = kt * TILE;
   const int nqt = p.NT - kt;       // causal query tiles per head
-  const int n_cand = p.g * nqt;    // (head, query tile) pairs of the causal range
+  const int n_cand = p.hpc * nqt;  // (head, query tile) pairs of the causal range
   const int n_full = p.full ? n_cand : 0;
   auto stage_ptr = [&](int st) { return smem + OFF_STAGE + st * STAGE; };
 
@@ -372,7 +450,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   for (int base = 0; base < n_cand; base += NTHREADS) {
     const int it = base + (int)threadIdx.x;
     uint32_t bits = 0;
-    if (it < n_cand) bits = tile_bits(p, b, kvh * p.g + it / nqt, kt + it % nqt, kt);
+    if (it < n_cand) bits = tile_bits(p, b, h0 + it / nqt, kt + it % nqt, kt);
     compact_append(bits != 0, ((uint32_t)it << 4) | bits, M.list, MAX_SPARSE, M.wsum, n_sparse);
   }
   n_sparse = min(n_sparse, MAX_SPARSE);
@@ -419,7 +497,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int hh, qt, sp;
         uint32_t bits;
         decode(j, hh, qt, sp, bits);
-        const int h = kvh * p.g + hh, t0 = qt * TILE;
+        const int h = h0 + hh, t0 = qt * TILE;
         uint8_t* sp_ = stage_ptr(st);
         // dh first: its slot frees after dV, before the Q slot frees after dK
         if (j >= NS && !mbar_wait(&M.dh_empty[st], ph, abort)) break;
@@ -532,17 +610,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       const float* L2 = reinterpret_cast<const float*>(stage_ptr(st) + 2 * TILE_B) + 64 * ch;
       const float* Dq = reinterpret_cast<const float*>(stage_ptr(st) + 2 * TILE_B + SCAL) + 64 * ch;
-      const bool sel = (bits >> (2 * ch + (r >> 6))) & 1u;
+      bool sel = (bits >> (2 * ch + (r >> 6))) & 1u;
       const int tq = qt * TILE + 64 * ch;  // first query of this warp's columns
       const bool diag = qt == kt;
       const bool ragged = tq + 64 > p.N;
+      // Sparse-stream step with fine selections: the pairs this key row holds
+      // among the warp's 64 queries (the warp skips the step when none does).
+      unsigned long long fm = ~0ull;
+      if (FINE && sp) {
+        fm = query_sel_mask64(p, b, h0 + hh, tq, u0 + r, lane);
+        sel = __any_sync(0xffffffffu, fm != 0ull);
+      }
       uint32_t pk[32];
       if (sel) {
         uint32_t x0[32], x1[32];
         tmem_ld32(cS, x0);
         tmem_ld32(cS + 32, x1);
         tmem_wait_ld();
-        if (diag || ragged) {
+        if (FINE && sp) {
+          const int lim = p.N - tq;
+          auto keep0 = [&](int col) { return ((fm >> col) & 1ull) && (!diag || r <= 64 * ch + col) && col < lim; };
+          auto keep1 = [&](int col) {
+            return ((fm >> (32 + col)) & 1ull) && (!diag || r <= 64 * ch + 32 + col) && 32 + col < lim;
+          };
+          p_block<true>(x0, L2, p.c, keep0, pk);
+          p_block<true>(x1, L2 + 32, p.c, keep1, pk + 16);
+        } else if (diag || ragged) {
           // key u0 + r may attend query tq + col only if r <= 64 ch + col, and the query must exist
           const int lim = p.N - tq;
           auto keep0 = [&](int col) { return (!diag || r <= 64 * ch + col) && col < lim; };
@@ -602,9 +695,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) rk[c] = rv[c] = 0u;
         }
-        if (store) {
+        if (store && p.part == nullptr) {
           store_row_bf16(okp + c0, rk, p.scale);
           store_row_bf16(ovp + c0, rv, 1.f);
+        } else if (store) {
+          const int64_t plane = (int64_t)gridDim.z * (gridDim.y / chunks) * p.N * HD;
+          float* pk = p.part + (int64_t)chunk * 2 * plane + (((int64_t)b * (gridDim.y / chunks) + kvh) * p.N + u) * HD + c0;
+          float* pv = pk + plane;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            reinterpret_cast<float4*>(pk)[q] = make_float4(__uint_as_float(rk[4 * q]), __uint_as_float(rk[4 * q + 1]),
+                                                           __uint_as_float(rk[4 * q + 2]), __uint_as_float(rk[4 * q + 3]));
+            reinterpret_cast<float4*>(pv)[q] = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
+                                                           __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
+          }
         }
       }
     }
@@ -663,6 +767,7 @@ __device__ __forceinline__ void row_to_tmem(const TensorRef& X, int b, int h, in
   tmem_st32(taddr, v);
 }
 
+template <bool FINE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      TensorRef Qr, TensorRef dhf_r, TensorRef dhs_r, BwdTcParams p) {
@@ -845,7 +950,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
-      const bool sel = (bits >> (2 * (r >> 6) + ch)) & 1u;
+      bool sel = (bits >> (2 * (r >> 6) + ch)) & 1u;
+      // Sparse-stream step with fine selections: the keys of the warp's 64
+      // columns this query row selected (the warp skips when no row does).
+      unsigned long long fm = ~0ull;
+      if (FINE && sp) {
+        fm = in_range ? key_sel_mask64(p, b, h, p.per_token ? t : (t >> p.ls), kt * TILE + 64 * ch) : 0ull;
+        sel = __any_sync(0xffffffffu, fm != 0ull);
+      }
       uint32_t x0[32], x1[32];
       if (sel) {
         tmem_ld32(cS, x0);
@@ -858,7 +970,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t pk[32];
       if (sel) {
         const float lv = sp ? l2[1] : l2[0];
-        if (kt == qt) {
+        if (FINE && sp) {
+          const bool dg = kt == qt;
+          auto keep0 = [&](int col) { return ((fm >> col) & 1ull) && (!dg || 64 * ch + col <= r); };
+          auto keep1 = [&](int col) { return ((fm >> (32 + col)) & 1ull) && (!dg || 64 * ch + 32 + col <= r); };
+          p_block_row<true>(x0, lv, p.c, keep0, pk);
+          p_block_row<true>(x1, lv, p.c, keep1, pk + 16);
+        } else if (kt == qt) {
           // query q0 + r attends key 128 kt + 64 ch + col only if 64 ch + col <= r
           auto keep0 = [&](int col) { return 64 * ch + col <= r; };
           auto keep1 = [&](int col) { return 64 * ch + 32 + col <= r; };
@@ -928,8 +1046,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 bool bwd_tc_supported(const Dims& D) {
   const int NT = (D.N + TILE - 1) / TILE;
-  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 64 || D.s == 128) && D.n <= 2048 && !D.per_token &&
-         (int64_t)D.g * NT <= dkv::MAX_SPARSE && NT <= dq::MAX_KT && D.g <= 255;
+  return D.dtype == SSA_BF16 && D.d == 128 && (D.s == 16 || D.s == 32 || D.s == 64 || D.s == 128) && D.n <= 2048 &&
+         (int64_t)bwd_mma_heads_per_cta(D) * NT <= dkv::MAX_SPARSE && NT <= dq::MAX_KT && D.g <= 255;
 }
 
 cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cudaStream_t st) {
@@ -972,6 +1090,13 @@ cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cuda
   p.D[1] = a.Dc;
   p.mask = a.mask;
   p.words = a.words;
+  p.rows = D.rows_sel;
+  p.ls = D.s == 16 ? 4 : D.s == 32 ? 5 : D.s == 64 ? 6 : 7;
+  p.per_token = D.per_token;
+  p.fine = (D.s < 64 || D.per_token) ? 1 : 0;
+  p.hpc = bwd_mma_heads_per_cta(D);
+  const int chunks = D.g / p.hpc;
+  p.part = chunks > 1 ? a.kvpart : nullptr;
   p.status = status;
   p.Hq = D.Hq;
   p.g = D.g;
@@ -982,15 +1107,18 @@ cudaError_t launch_bwd_tc(const Dims& D, const BwdArgs& a, int32_t* status, cuda
   p.c = D.scale * kLog2e;
   p.scale = D.scale;
   p.full = a.sparse_only ? 0 : 1;
-  e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::SMEM);
+  auto kdq = p.fine ? bwd_dq_tc_kernel<true> : bwd_dq_tc_kernel<false>;
+  auto kdkv = p.fine ? bwd_dkv_tc_kernel<true> : bwd_dkv_tc_kernel<false>;
+  e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM);
+  e = cudaFuncSetAttribute(kdkv, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM);
   if (e != cudaSuccess) return e;
-  bwd_dkv_tc_kernel<<<dim3(p.NT, D.Hkv, D.B), NTHREADS, dkv::SMEM, st>>>(mq, mk, mv, mf, ms, p);
+  kdkv<<<dim3(p.NT, D.Hkv * chunks, D.B), NTHREADS, dkv::SMEM, st>>>(mq, mk, mv, mf, ms, p);
   count_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq_tc_kernel<<<dim3(p.NT, D.Hq, D.B), NTHREADS, dq::SMEM, st>>>(mk, mv, a.q, rdhf, rdhs, p);
+  if (chunks > 1 && (e = launch_kvsum(D, a, a.kvpart, chunks, st)) != cudaSuccess) return e;
+  kdq<<<dim3(p.NT, D.Hq, D.B), NTHREADS, dq::SMEM, st>>>(mk, mv, a.q, rdhf, rdhs, p);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -115,7 +115,7 @@ Layout layout(const Dims& D) {
   L.mask = o; o = align_up(o + (size_t)D.B * D.Hq * D.rows_sel * L.words * 4);
   L.partials = o; o = align_up(o + (size_t)L.n_partials * 4);
   L.kvpart = o;
-  if (!bwd_tc_supported(D) && bwd_mma_supported(D)) o = align_up(o + bwd_mma_partial_bytes(D));
+  if (bwd_tc_supported(D) || bwd_mma_supported(D)) o = align_up(o + bwd_mma_partial_bytes(D));
   L.maskT = o;
   if (bwd_walk_supported(D)) o = align_up(o + (size_t)D.B * D.Hq * D.n * L.words * 4);
   L.bytes_bwd = o;
@@ -305,6 +305,7 @@ ssa_status_t ssa_bwd_dual(const ssa_dims_t* dims, const ssa_tensor_t* Q, const s
   if (bwd_tc_supported(D)) {
     int32_t* status = device_status_ptr();
     if (status == nullptr) return SSA_ERR_CUDA;
+    a.kvpart = at<float>(ws, L.kvpart);
     return from_cuda(launch_bwd_tc(D, a, status, st));
   }
   if (bwd_mma_supported(D)) {
@@ -429,6 +430,7 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
   if (bwd_tc_supported(D)) {
     int32_t* status = device_status_ptr();
     if (status == nullptr) return SSA_ERR_CUDA;
+    a.kvpart = at<float>(ws, L.kvpart);
     return from_cuda(launch_bwd_tc(D, a, status, st));
   }
   if (bwd_mma_supported(D)) {

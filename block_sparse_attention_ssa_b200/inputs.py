@@ -76,6 +76,9 @@ WORKLOADS = {
     # hidden 2048 -> d = 64) with their 16 x 16 receptive field at the 8K
     # training context.
     "paper_b16_8k": Workload("paper_b16_8k", 1, 32, 2, 8192, 64, 16, 16, "bf16", 1006),
+    # The same selection (block 16, 16 blocks) at head dimension 128, the
+    # head size of the five suites above.
+    "paper_b16_8k_d128": Workload("paper_b16_8k_d128", 1, 32, 2, 8192, 128, 16, 16, "bf16", 1008),
 }
 SWEEP_TOPK = (4, 8, 16, 32, 64)
 

@@ -30,6 +30,8 @@ CASES = {
     # a ragged last 128-row tile (576 = 4.5 x 128) with g = 8 (two head chunks)
     "bf16_s16_ragged_g8_d64": (1, 8, 1, 576, 64, 16, 8, "bf16"),
     "bf16_s32_ragged_d128": (1, 2, 1, 704, 128, 32, 5, "bf16"),
+    # block 16 at d = 128 with g = 4 and a ragged last 128-row tile
+    "bf16_s16_d128_g4": (1, 8, 2, 960, 128, 16, 16, "bf16"),
 }
 
 

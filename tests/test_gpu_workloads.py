@@ -198,7 +198,7 @@ def test_tiny_f32_whole_problem():
     assert np.abs(f64(delta2) - f["delta"]).max() <= 1e-4
 
 
-@pytest.mark.parametrize("name", ["mha_8k", "gqa_16k", "long_64k", "paper_b16_8k"])
+@pytest.mark.parametrize("name", ["mha_8k", "gqa_16k", "long_64k", "paper_b16_8k", "paper_b16_8k_d128"])
 def test_full_size_sampled(name):
     w = WORKLOADS[name]
     rng = np.random.Generator(np.random.PCG64(77))
