@@ -21,11 +21,13 @@
 //
 // One launch per token (CUDA cores, fp32 arithmetic; a token moves a few
 // MB): a thread-block cluster of CL CTAs per (batch, kv head) selects the
-// blocks of the g query heads, attends the union of their kept blocks split
-// CL ways (each K/V row read once for all g heads) and merges the partials,
-// exchanging the selections and the partials through distributed shared
-// memory between cluster barriers (no workspace, no atomics, no waiting on
-// flags).
+// blocks of the g query heads (every CTA scores a slice of the pooled blocks
+// for every head and keeps each head's best k-1 of its slice; the head's
+// owner merges the CL lists), attends the union of their kept blocks split CL
+// ways (each K/V row read once for all g heads) and merges the partials,
+// exchanging the candidate lists, the selections and the partials through
+// distributed shared memory between cluster barriers (no workspace, no
+// atomics, no waiting on flags).
 #include <algorithm>
 #include <climits>
 
@@ -48,7 +50,7 @@ struct DecodeShape {
 
 // Byte offsets of the decode kernel's shared memory.
 struct DecodeLayout {
-  size_t qbar, sc, selh, red, q, o, mx, sum, x, k, v, lst, usel, bytes;
+  size_t qbar, sc, cand, selh, red, q, o, mx, sum, x, k, v, lst, usel, corr, bytes;
   __host__ __device__ DecodeLayout(int n, int g, int k_eff, int D) {
     size_t at = 0;
     auto take = [&](size_t nbytes) {
@@ -58,8 +60,10 @@ struct DecodeLayout {
     };
     const int gl = (g + CL - 1) / CL;                       // heads this CTA selects
     const int most = (std::min(g * k_eff, n) + CL - 1) / CL;  // union blocks this CTA attends
-    qbar = take((size_t)D * 4);           // [D] query side of the block scores
-    sc = take((size_t)n * 4);             // [n] block scores
+    const int slice = (n + CL - 1) / CL;                    // pooled blocks this CTA scores
+    qbar = take((size_t)g * D * 4);       // [g][D] query side of the block scores
+    sc = take((size_t)g * slice * 4);     // [g][slice] block scores of this CTA's slice
+    cand = take((size_t)g * 64 * 8);      // [g][64] best k-1 (score, block) of the slice
     selh = take((size_t)gl * 64 * 4);     // [gl][64] selected-block bits of this CTA's heads
     red = take((size_t)NT * 8);           // arg-max candidates / key-sum staging
     q = take((size_t)g * D * 4);          // [g][D] q_t
@@ -71,6 +75,7 @@ struct DecodeLayout {
     v = take((size_t)CH * D * 4);         // [CH][D] V chunk
     lst = take((size_t)(1 + most) * 4);   // this CTA's blocks of the union
     usel = take((size_t)g * 64 * 4);      // [g][64] every head's selected-block bits
+    corr = take((size_t)g * 4);           // [g] rescale factor of a chunk
     bytes = at;
   }
 };
@@ -88,9 +93,11 @@ struct DecodeLayout {
 //   3. after a second barrier CTA r merges the partials of heads r, r + CL,
 //      .. from the CL CTAs and writes h and lse; a last barrier keeps every
 //      CTA's shared memory alive until the merges have read it.
-// CPL: top-k candidate slots per lane (32 * CPL >= n).
-template <typename T, int D, int CPL>
-__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT)
+// k_eff <= 64 (each slice keeps at most 63 candidates per head).
+// Two CTAs fit an SM (registers and shared memory), so that the clusters
+// of every (batch, kv head) are resident at once.
+template <typename T, int D>
+__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
     decode_kernel(TensorRef q, TensorRef K, TensorRef V, TensorRef hout, float* lse, int32_t* idx, float* qsum,
                   float* kbar, DecodeShape sh) {
   namespace cg = cooperative_groups;
@@ -107,6 +114,8 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT)
   const DecodeLayout L(n, G, sh.k, D);
   float* sqbar = reinterpret_cast<float*>(smem + L.qbar);
   float* ssc = reinterpret_cast<float*>(smem + L.sc);
+  float2* scand = reinterpret_cast<float2*>(smem + L.cand);  // (score, block index bits)
+  float* scorr = reinterpret_cast<float*>(smem + L.corr);
   uint32_t* selh = reinterpret_cast<uint32_t*>(smem + L.selh);
   float* rv = reinterpret_cast<float*>(smem + L.red);
   float* sq = reinterpret_cast<float*>(smem + L.q);
@@ -120,78 +129,140 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT)
   uint32_t* usel = reinterpret_cast<uint32_t*>(smem + L.usel);
 
   // ================================================================ 1. selection
+  // (a) the query side of every head (q_t folded into the block's query sum;
+  //     the head's owner, rank hh % CL, writes the sum back after the first
+  //     cluster barrier, when every CTA has read the old value)
+  const int slice = (n + CL - 1) / CL;
+  const int j0 = min(i, i * rank / CL), j1 = min(i, i * (rank + 1) / CL);  // this CTA's blocks of [0, i)
+  // (loads of four elements per thread issued before their use; q_t is
+  //  kept in the partial-output buffer until the attention phase)
+  for (int base = 0; base < G * D; base += 4 * NT) {
+    float xq[4], old[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = base + u * NT + tid;
+      xq[u] = old[u] = 0.f;
+      if (e < G * D) {
+        const int hh = e / D, c = e % D, h = kvh * G + hh;
+        xq[u] = to_f32(row_ptr<T>(q, b, h, 0)[c]);
+        if (t % s != 0) old[u] = qsum[((int64_t)b * sh.Hq + h) * D + c];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = base + u * NT + tid;
+      if (e < G * D) {
+        const float acc = old[u] + xq[u];
+        sqbar[e] = sh.per_token ? xq[u] : acc / (float)(t - i * s + 1);
+        sq[e] = acc;  // the new sum, written back by the owner below
+        so[e] = xq[u];
+      }
+    }
+  }
+  for (int e = tid; e < ((G + CL - 1) / CL) * 64; e += NT) selh[e] = 0u;
+  __syncthreads();
+  // (b) scores of this CTA's slice for every head: a thread per (head,
+  //     block), the whole pooled key row loaded at once as 16-byte vectors
+  //     (the slice's rows stay in L1 across the heads)
+  const float* kb = kbar + (int64_t)bk * n * D;
+  const int ns = j1 - j0;  // <= slice <= NT
+  // a thread per (block, head group): the block's row is loaded once and
+  // dotted with the queries of heads hg, hg + HG, ..
+  const int HG = ns > 0 ? min(G, max(1, NT / ns)) : 1;
+  if (tid < ns * HG) {
+    const int jj = tid % ns, hg = tid / ns;
+    const float4* row = reinterpret_cast<const float4*>(kb + (int64_t)(j0 + jj) * D);
+    // the row in pieces of 64 floats (registers); partial dots per head in
+    // the score slots
+    constexpr int P4 = 16;
+#pragma unroll 1
+    for (int p0 = 0; p0 < D / 4; p0 += P4) {
+      float4 kv[P4];
+#pragma unroll
+      for (int c4 = 0; c4 < P4; ++c4) kv[c4] = row[p0 + c4];
+      for (int hh = hg; hh < G; hh += HG) {
+        const float* qv = sqbar + hh * D + 4 * p0;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < P4; ++c4) {
+          const float4 qq = *reinterpret_cast<const float4*>(qv + 4 * c4);
+          a0 = fmaf(qq.x, kv[c4].x, fmaf(qq.y, kv[c4].y, a0));
+          a1 = fmaf(qq.z, kv[c4].z, fmaf(qq.w, kv[c4].w, a1));
+        }
+        float* slot = ssc + hh * slice + jj;
+        *slot = (p0 == 0 ? 0.f : *slot) + (a0 + a1);
+      }
+    }
+    for (int hh = hg; hh < G; hh += HG) {
+      const float x = sh.scale * ssc[hh * slice + jj];
+      ssc[hh * slice + jj] = (x != x) ? kNegInf : x;  // NaN ranks last
+    }
+  }
+  __syncthreads();
+  // (c) per head, the best k-1 of the slice, sorted: each candidate's rank
+  //     is the number of slice entries that beat it (score descending, block
+  //     ascending); ranks below k-1 are kept, at their rank.  Unfilled list
+  //     entries are NaN (compares false with everything).
+  const float kOut = __int_as_float(0x7fffffff);
+  const int km1 = sh.k - 1;
+  if (i + 1 > sh.k) {
+    for (int e = tid; e < G * km1; e += NT) scand[(e / km1) * 64 + e % km1] = make_float2(kOut, __int_as_float(INT_MAX));
+    __syncthreads();
+    for (int e = tid; e < G * ns; e += NT) {
+      const int hh = e / ns, jj = e % ns;
+      const float* sc = ssc + hh * slice;
+      const float v = sc[jj];
+      int rk = 0;
+      for (int o = 0; o < ns; ++o) {
+        const float w = sc[o];
+        rk += (w > v || (w == v && o < jj)) ? 1 : 0;
+      }
+      if (rk < km1) scand[hh * 64 + rk] = make_float2(v, __int_as_float(j0 + jj));
+    }
+  }
+  cluster.sync();  // every CTA's candidate lists are visible to the cluster
+  // (d) the owner of head hh merges the CL sorted lists: every entry's rank
+  //     in the union is its rank in its own list plus, for each other list,
+  //     the number of entries that beat it (a binary search, after the lists
+  //     are copied to this CTA); the k-1 best are kept with the diagonal
+  //     block, and the head's query sum, selection bits and idx row written
+  float2* mlist = reinterpret_cast<float2*>(sk);  // [CL][64] copy of one head's lists (the K chunk is free here)
   for (int hl = 0; rank + CL * hl < G; ++hl) {
     const int hh = rank + CL * hl, h = kvh * G + hh;
     uint32_t* sel = selh + hl * 64;
-    if (tid < D) {
-      float* qs = qsum + ((int64_t)b * sh.Hq + h) * D + tid;
-      const float xq = to_f32(row_ptr<T>(q, b, h, 0)[tid]);
-      const float acc = (t % s == 0 ? 0.f : *qs) + xq;
-      *qs = acc;
-      sqbar[tid] = sh.per_token ? xq : acc / (float)(t - i * s + 1);
-    }
-    if (tid < 64) sel[tid] = 0u;
-    __syncthreads();
-
-    // scores of the complete blocks j < i: a thread per pooled key, its row
-    // read as 16-byte vectors against the query side in shared memory
-    const float* kb = kbar + (int64_t)bk * n * D;
-    for (int j = tid; j < i; j += NT) {
-      const float4* row = reinterpret_cast<const float4*>(kb + (int64_t)j * D);
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll 8
-      for (int c4 = 0; c4 < D / 4; ++c4) {
-        const float4 kv = row[c4];
-        const float4 qv = *reinterpret_cast<const float4*>(sqbar + 4 * c4);
-        a0 = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, a0));
-        a1 = fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, a1));
-      }
-      const float x = sh.scale * (a0 + a1);
-      ssc[j] = (x != x) ? kNegInf : x;  // NaN ranks last
-    }
-    __syncthreads();
-
-    // top-(k-1) of the scores plus the diagonal block (score descending,
-    // index ascending): one warp, candidate j in lane j % 32, slot j / 32;
-    // slots that may not be chosen (j >= i, or taken) hold NaN, which
-    // compares false with everything
+    for (int c = tid; c < D; c += NT) qsum[((int64_t)b * sh.Hq + h) * D + c] = sq[hh * D + c];
     if (i + 1 <= sh.k) {
       for (int j = tid; j <= i; j += NT) atomicOr(&sel[j >> 5], 1u << (j & 31));
-    } else if (warp == 0) {
-      const float kOut = __int_as_float(0x7fffffff);
-      float v[CPL];
-#pragma unroll
-      for (int m = 0; m < CPL; ++m) v[m] = (lane + 32 * m < i) ? ssc[lane + 32 * m] : kOut;
-      uint64_t taken = 0;
-      for (int round = 0; round < sh.k - 1; ++round) {
-        float bv = kNegInf;
-        int bj = INT_MAX;
-#pragma unroll
-        for (int m = 0; m < CPL; ++m)
-          if (v[m] > bv || (v[m] == bv && bj == INT_MAX)) {
-            bv = v[m];
-            bj = lane + 32 * m;
-          }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-          if (ov > bv || (ov == bv && oj < bj)) {
-            bv = ov;
-            bj = oj;
-          }
-        }
-        if (bj != INT_MAX && (bj & 31) == lane) {
-          taken |= 1ull << (bj >> 5);
-#pragma unroll
-          for (int m = 0; m < CPL; ++m)
-            if (m == (bj >> 5)) v[m] = kOut;
-        }
+    } else {
+      for (int e = tid; e < CL * km1; e += NT) {
+        const int r = e / km1, c = e % km1;
+        mlist[r * 64 + c] = cluster.map_shared_rank(scand, r)[hh * 64 + c];
       }
-#pragma unroll
-      for (int m = 0; m < CPL; ++m)
-        if ((taken >> m) & 1ull) atomicOr(&sel[(lane + 32 * m) >> 5], 1u << ((lane + 32 * m) & 31));
-      if (lane == 0) atomicOr(&sel[i >> 5], 1u << (i & 31));
+      __syncthreads();
+      for (int e = tid; e < CL * km1; e += NT) {
+        const int r = e / km1, c = e % km1;
+        const float2 x = mlist[r * 64 + c];
+        const float v = x.x;
+        const int jx = __float_as_int(x.y);
+        if (jx == INT_MAX) continue;  // an unfilled entry
+        int rk = c;
+        for (int r2 = 0; r2 < CL; ++r2) {
+          if (r2 == r) continue;
+          // entries of list r2 that beat (v, jx): a prefix of the sorted list
+          int lo = 0, hi = km1;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            const float2 y = mlist[r2 * 64 + mid];
+            const int jy = __float_as_int(y.y);
+            const bool beats = jy != INT_MAX && (y.x > v || (y.x == v && jy < jx));
+            if (beats) lo = mid + 1;
+            else hi = mid;
+          }
+          rk += lo;
+        }
+        if (rk < km1) atomicOr(&sel[jx >> 5], 1u << (jx & 31));
+      }
+      if (tid == 0) atomicOr(&sel[i >> 5], 1u << (i & 31));
     }
     __syncthreads();
     if (tid == 0) {  // Sel ascending, -1 padded
@@ -201,9 +272,10 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT)
         for (uint32_t xw = sel[w]; xw && c < sh.k; xw &= xw - 1) out[c++] = 32 * w + __ffs(xw) - 1;
       for (; c < sh.k; ++c) out[c] = -1;
     }
+    // the head's selection into every CTA's copy of all heads' selections
+    for (int e = tid; e < CL * 64; e += NT) cluster.map_shared_rank(usel, e >> 6)[hh * 64 + (e & 63)] = sel[e & 63];
     __syncthreads();
   }
-
   // the token closes block i: its key mean joins the pooled cache (no
   // reader of this call uses kbar[i])
   if (rank == 0 && t % s == s - 1) {
@@ -229,13 +301,9 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT)
   cluster.sync();  // every head's selection is visible to the cluster
 
   // ================================================================ 2. attention
-  for (int e = tid; e < G * 64; e += NT) {
-    const int hh = e >> 6, w = e & 63;
-    const uint32_t* peer = cluster.map_shared_rank(selh, hh % CL);
-    usel[e] = peer[(hh / CL) * 64 + w];
-  }
+  // (every head's selection was pushed into usel by its owner; q_t waits in so)
   for (int e = tid; e < G * D; e += NT) {
-    sq[e] = to_f32(row_ptr<T>(q, b, kvh * G + e / D, 0)[e % D]);
+    sq[e] = so[e];
     so[e] = 0.f;
   }
   if (tid < G) {
@@ -322,6 +390,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT)
         sx[xx] = v;
       }
       __syncthreads();
+      // softmax statistics: a warp per head; the weights go back over the logits
       for (int hh = warp; hh < G; hh += NT / 32) {
         if (!((usel[hh * 64 + (j >> 5)] >> (j & 31)) & 1u)) continue;
         float* xs = sx + hh * CH;
@@ -339,19 +408,21 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT)
         __syncwarp();
         xs[lane] = p0;
         xs[lane + 32] = p1;
-        __syncwarp();
-        float* o = so + hh * D;
-#pragma unroll
-        for (int r = 0; r < D / 32; ++r) {
-          const int c = lane + 32 * r;
-          float acc = o[c] * corr;
-          for (int uu = 0; uu < rows; ++uu) acc = fmaf(xs[uu], sv[uu * D + c], acc);
-          o[c] = acc;
-        }
         if (lane == 0) {
           smax[hh] = m_new;
           ssum[hh] = ssum[hh] * corr + ps;
+          scorr[hh] = corr;
         }
+      }
+      __syncthreads();
+      // o += P V: a thread per (head, column), every warp busy
+      for (int xx = tid; xx < G * D; xx += NT) {
+        const int hh = xx / D, c = xx % D;
+        if (!((usel[hh * 64 + (j >> 5)] >> (j & 31)) & 1u)) continue;
+        const float* xs = sx + hh * CH;
+        float acc = so[xx] * scorr[hh];
+        for (int uu = 0; uu < rows; ++uu) acc = fmaf(xs[uu], sv[uu * D + c], acc);
+        so[xx] = acc;
       }
       __syncthreads();
     }
@@ -415,12 +486,7 @@ cudaError_t decode_t(const Dims& Dm, const DecodeArgs& a, cudaStream_t st) {
     count_launches(1);
     return cudaGetLastError();
   };
-  const int cpl = (Dm.n + 31) / 32;
-  if (cpl <= 2) return run(decode_kernel<T, D, 2>);
-  if (cpl <= 8) return run(decode_kernel<T, D, 8>);
-  if (cpl <= 16) return run(decode_kernel<T, D, 16>);
-  if (cpl <= 32) return run(decode_kernel<T, D, 32>);
-  return run(decode_kernel<T, D, 64>);
+  return run(decode_kernel<T, D>);
 }
 
 template <typename T, int D>
@@ -434,6 +500,8 @@ cudaError_t prefill_t(const Dims& Dm, const DecodeArgs& a, cudaStream_t st) {
 }  // namespace
 
 size_t decode_smem_bytes(const Dims& D) { return DecodeLayout(D.n, D.g, D.k, D.d).bytes; }
+
+bool decode_supported(const Dims& D) { return D.k <= 64 && decode_smem_bytes(D) <= 232448; }
 
 size_t decode_ws_bytes(const Dims& D) {
   (void)D;

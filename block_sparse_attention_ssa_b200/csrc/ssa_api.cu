@@ -485,7 +485,7 @@ ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q, cons
   if (reinterpret_cast<uintptr_t>(qsum) % 4 || reinterpret_cast<uintptr_t>(kbar) % 16 ||
       reinterpret_cast<uintptr_t>(lse) % 4 || reinterpret_cast<uintptr_t>(idx) % 4)
     return SSA_ERR_INVALID_ARG;
-  if (decode_smem_bytes(D) > 232448) return SSA_ERR_UNSUPPORTED;
+  if (!decode_supported(D)) return SSA_ERR_UNSUPPORTED;
   if ((s = check_ws(D, ws, ws_bytes)) != SSA_OK) return s;
   if ((s = check_device()) != SSA_OK) return s;
   a.ws = ws;

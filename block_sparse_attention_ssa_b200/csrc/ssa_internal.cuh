@@ -246,6 +246,8 @@ cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_decode_prefill(const Dims& D, const DecodeArgs& a, cudaStream_t st);
 // Dynamic shared memory the decode kernels need for these dims.
 size_t decode_smem_bytes(const Dims& D);
+// The decode step's envelope: k_eff <= 64 and its shared memory fits a CTA.
+bool decode_supported(const Dims& D);
 // Workspace bytes of one decode step.
 size_t decode_ws_bytes(const Dims& D);
 

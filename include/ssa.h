@@ -268,8 +268,9 @@ SSA_API ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* 
  *   kbar [B, Hkv, n, d] fp32: means of the complete key blocks (16-byte
  *     aligned for the decode step).
  * dims->N is the capacity of the K/V caches [B, Hkv, N, d] (a multiple of
- * block); the decode kernel's shared memory (n scores, the g heads' queries,
- * partial outputs and selections, a 64-key K/V chunk) must fit a CTA
+ * block); the decode step needs k_eff <= 64 and its shared memory (the g
+ * heads' scores of one eighth of the pooled blocks and their candidate lists,
+ * queries, partial outputs and selections, a 64-key K/V chunk) must fit a CTA
  * (SSA_ERR_UNSUPPORTED otherwise; every workload here fits). */
 
 /* Builds the decode state from a prompt of t0 tokens (0 <= t0 <= N): kbar of

@@ -27,6 +27,9 @@ CASES = {
     "f32_d64": (1, 4, 4, 512, 64, 64, 3, "f32", 64 + 40, 100),
     "bf16_full_budget": (1, 4, 2, 512, 128, 64, 16, "bf16", 30, 60),
     "f32_from_empty_prompt": (1, 2, 1, 256, 128, 64, 2, "f32", 0, 140),
+    # 16 heads per kv head (two per selecting CTA) and k = 40: each CTA's
+    # slice keeps 39 candidates per head, merged from eight lists
+    "bf16_g16_k40_s16": (1, 16, 1, 4096, 64, 16, 40, "bf16", 2600, 120),
 }
 
 
