@@ -368,7 +368,11 @@ ssa_status_t ssa_fwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
     if (status == nullptr) return SSA_ERR_CUDA;
     return from_cuda(launch_fwd_ord(D, a, status, st));
   }
-  if (fwd_walk_supported(D)) return from_cuda(launch_fwd_walk(D, a, st));
+  if (fwd_walk_supported(D)) {
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_fwd_walk(D, a, status, st));
+  }
   if (fwd_mma_supported(D)) return from_cuda(launch_fwd_mma(D, a, st));
   return from_cuda(launch_fwd_simt(D, a, st));
 }

@@ -158,7 +158,7 @@ cudaError_t launch_fwd_mma(const Dims& D, const FwdArgs& a, cudaStream_t st);
 // Sparse stream alone, blocks of 16 or 32, per-block selection (bf16, mma.sync):
 // each query block walks its own selected key blocks.
 bool fwd_walk_supported(const Dims& D);
-cudaError_t launch_fwd_walk(const Dims& D, const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_fwd_walk(const Dims& D, const FwdArgs& a, int32_t* dev_status, cudaStream_t st);
 cudaError_t launch_dropped_mma(const Dims& D, const FwdArgs& a, cudaStream_t st);
 
 // Envelope of the first tensor-core kernels: bf16, d = 128, blocks of 64 or
