@@ -23,12 +23,14 @@
 // fixed order and writes one fp32 partial per query head; the GQA group's
 // partials are then added in head order.  No atomics: bit-reproducible.
 #include "mma_sync.cuh"
+#include "sm100_ptx.cuh"
 #include "ssa_internal.cuh"
 
 namespace ssa {
 namespace {
 
 using namespace warp_mma;
+using namespace sm100;
 using bf16 = __nv_bfloat16;
 
 constexpr int BM = 64;   // query rows per dQ CTA
@@ -38,6 +40,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct WalkShape {
   int Hq, g, N, n, words;
   float scale;
+  int32_t* status;
 };
 
 template <int W>
@@ -271,39 +274,70 @@ __global__ void __launch_bounds__(32) mask_transpose_kernel(const uint32_t* __re
   }
 }
 
+// Shared memory of a dK / dV CTA: per warp a ring of NS query blocks (Q,
+// then g_s, each as 64-column halves of S rows x 128 B in the TMA 128-byte
+// swizzle: the 16-byte chunk c of row r sits at chunk c ^ (r & 7), so ldmatrix
+// reads are conflict-free without padding), the 16-key K and V slice in the
+// same layout, and the ascending list of query blocks that chose the key
+// block.  The rings become the reduction buffer at the end.
 template <int D, int S>
 struct KvCfg {
-  static constexpr int NS = (D == 64 && S == 16) ? 3 : 2;
-  static constexpr int LD = D + 8;
-  static constexpr int ROWS = S * LD * 2;                     // S query rows
-  static constexpr int STAGE = 2 * ROWS + 2 * S * 4;          // Q, g_s, lse, D
-  static constexpr int RING = 4 * NS * STAGE;
-  static constexpr int RED = 2 * 4 * 16 * D * 4;              // four warps' dK, dV (fp32)
-  static constexpr int KV_OFF = RING > RED ? RING : RED;
-  static constexpr int LIST_OFF = KV_OFF + 2 * 16 * LD * 2;   // K and V slice staging
-  static constexpr int SMEM = LIST_OFF + 2048 * 2 + 16;       // query-block list (n <= 2048) + its length
+  static constexpr int NW = 4;                  // warps, dealt the list in turn
+  static constexpr int NS = D == 64 ? 3 : 2;    // query blocks in a warp's ring
+  static constexpr int HALF = S * 128;          // 64 columns of S query rows
+  static constexpr int QT = (D / 64) * HALF;    // one Q (or g_s) block
+  static constexpr int SLOT = 2 * QT;           // Q, then g_s
+  static constexpr int RING = NS * SLOT;
+  static constexpr int KHALF = 16 * 128;        // 64 columns of the 16-key slice
+  static constexpr int KT = (D / 64) * KHALF;   // the K (or V) slice
+  static constexpr int RED = NW * 2 * 16 * D * 4;  // the warps' dK, dV (fp32)
+  static constexpr int KV_OFF = NW * RING > RED ? NW * RING : RED;
+  static constexpr int LIST_OFF = KV_OFF + 2 * KT;
+  static constexpr int BAR_OFF = LIST_OFF + 2048 * 2 + 16;   // query-block list (n <= 2048) + its length
+  static constexpr int FLAG_OFF = BAR_OFF + (NW * NS + 1) * 8;  // NW rings' barriers, the slice barrier
+  static constexpr int SMEM = FLAG_OFF + 16 + 1024;              // abort flag, alignment slack
+  static constexpr int MINB = (D == 64 && S == 16) ? 3 : (D == 128 && S == 32) ? 1 : 2;  // resident CTAs per SM the registers are sized for
 };
 
+// Byte offset of the 16-byte chunk `ch` (0..7) of row r in a swizzled half.
+__device__ __forceinline__ uint32_t swz(int r, int ch) { return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4)); }
+
+// One CTA per (query head, 16-key slice u0 .. u0 + 15 of key block j), heads
+// innermost so that every head's early key blocks (the ones most query
+// blocks choose) start first.  The ascending list of query blocks whose
+// selection holds j is dealt to the four warps in turn; per query block:
+// S^T = K Q^T and dP^T = V g_s^T (16 keys x S rows), P^T from lse_sel,
+// dS^T = P^T (dP^T - D), then dV += P^T g_s and dK += dS^T Q.  A warp issues
+// the products of its next query block before the gradients of the current
+// one, so the tensor core has independent work while the exponentials run.
+// The four warps' sums are added in a fixed order into one fp32 partial per
+// query head (dK unscaled, dV); the GQA group's partials are added in head
+// order afterwards.
 template <int D, int S>
-__global__ void __launch_bounds__(NT) bwd_dkv_walk_kernel(BwdArgs a, WalkShape sh, float* part) {
+__global__ void __launch_bounds__(NT, KvCfg<D, S>::MINB)
+    bwd_dkv_walk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
+                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        BwdArgs a, WalkShape sh, float* part) {
   using C = KvCfg<D, S>;
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int j = blockIdx.x / (S / 16), half = blockIdx.x % (S / 16);
-  const int h = blockIdx.y, b = blockIdx.z, kvh = h / sh.g;
-  const int u0 = j * S + half * 16;  // first key of the slice
+  const int h = blockIdx.x, j = blockIdx.y / (S / 16), b = blockIdx.z, kvh = h / sh.g;
+  const int u0 = j * S + (blockIdx.y % (S / 16)) * 16;  // first key of the slice
   const int64_t rowbase = ((int64_t)b * sh.Hq + h) * sh.N;
-  bf16 (*kvs)[C::LD] = reinterpret_cast<bf16 (*)[C::LD]>(smem + C::KV_OFF);  // rows 0-15 K, 16-31 V
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::LIST_OFF);
   int* list_len = reinterpret_cast<int*>(smem + C::LIST_OFF + 2048 * 2);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + warp * C::NS;  // this warp's ring
+  uint64_t* kvbar = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + C::NW * C::NS;
+  int* abort_flag = reinterpret_cast<int*>(smem + C::FLAG_OFF);
+  unsigned char* ring = smem + warp * C::RING;
 
-  for (int e = tid; e < 2 * 16 * D / 8; e += NT) {
-    const int r = e / (D / 8), c = (e % (D / 8)) * 8;
-    const TensorRef& t = r < 16 ? a.k : a.v;
-    cp_async16(&kvs[r][c], row_ptr<bf16>(t, b, kvh, u0 + (r & 15)) + c, 16);
+  if (tid == 0) {
+    for (int s = 0; s <= C::NW * C::NS; ++s) mbar_init(reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + s, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  cp_async_commit();
-
   // Query blocks whose selection holds j, ascending: lane l of warp 0 takes
   // words 2l and 2l+1 of the transposed mask row, a warp scan places them.
   if (warp == 0) {
@@ -322,89 +356,100 @@ __global__ void __launch_bounds__(NT) bwd_dkv_walk_kernel(BwdArgs a, WalkShape s
     for (uint32_t bits = w1; bits; bits &= bits - 1u) list[pos++] = (uint16_t)(64 * lane + 32 + __ffs(bits) - 1);
     if (lane == 31) *list_len = incl;
   }
-  cp_async_wait<0>();
-  __syncthreads();  // the list and the K / V slice (copied by every thread) are in place
-  const int total = *list_len;
-
-  unsigned char* ring = smem + warp * C::NS * C::STAGE;
-  auto qbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(ring + st * C::STAGE); };
-  auto gbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(ring + st * C::STAGE + C::ROWS); };
-  auto lbuf = [&](int st) { return reinterpret_cast<float*>(ring + st * C::STAGE + 2 * C::ROWS); };
-  auto dbuf = [&](int st) { return reinterpret_cast<float*>(ring + st * C::STAGE + 2 * C::ROWS + S * 4); };
-  auto load_pair = [&](int i, int st) {
-    bf16 (*qs)[C::LD] = qbuf(st);
-    bf16 (*gs)[C::LD] = gbuf(st);
-    for (int e = lane; e < S * D / 8; e += 32) {
-      const int r = e / (D / 8), c = (e % (D / 8)) * 8;
-      cp_async16(&qs[r][c], row_ptr<bf16>(a.q, b, h, (int64_t)i * S + r) + c, 16);
-      cp_async16(&gs[r][c], row_ptr<bf16>(a.gs, b, h, (int64_t)i * S + r) + c, 16);
-    }
-    if (lane < S / 4) {
-      cp_async16(lbuf(st) + 4 * lane, a.lse_sel + rowbase + (int64_t)i * S + 4 * lane, 16);
-      cp_async16(dbuf(st) + 4 * lane, a.Dc + rowbase + (int64_t)i * S + 4 * lane, 16);
-    }
-  };
-  // this warp's pairs: list[warp], list[warp + 4], ...
-  const int mine = total > warp ? (total - warp + 3) / 4 : 0;
+  __syncthreads();  // the list and the barriers are in place
+  if (tid == 0) {  // the slice's K and V rows
+    mbar_expect_tx(kvbar, 2 * C::KT);
 #pragma unroll
-  for (int p = 0; p < C::NS - 1; ++p) {
-    if (p < mine) load_pair(list[warp + 4 * p], p);
-    cp_async_commit();
+    for (int hh = 0; hh < D / 64; ++hh) {
+      unsigned char* dst = smem + C::KV_OFF + hh * C::KHALF;
+      tma_load_4d(dst, &tmK, kvbar, hh * 64, u0, kvh, b);
+      tma_load_4d(dst + C::KT, &tmV, kvbar, hh * 64, u0, kvh, b);
+    }
+  }
+  const int total = *list_len;
+  const int mine = total > warp ? (total - warp + C::NW - 1) / C::NW : 0;  // list[warp + NW p], p < mine
+
+  // Lane 0 of each warp issues its own ring's loads.
+  int issued = 0;
+  auto issue_next = [&](int slot) {
+    const int i = list[warp + C::NW * issued];
+    unsigned char* dst = ring + slot * C::SLOT;
+    mbar_expect_tx(&full[slot], C::SLOT);
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh) {
+      tma_load_4d(dst + hh * C::HALF, &tmQ, &full[slot], hh * 64, i * S, h, b);
+      tma_load_4d(dst + C::QT + hh * C::HALF, &tmG, &full[slot], hh * 64, i * S, h, b);
+    }
+    ++issued;
+  };
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < C::NS - 1; ++s)
+      if (issued < mine) issue_next(s);
   }
 
   const int g8 = lane >> 2, q4 = lane & 3;
   const float sl2 = sh.scale * kLog2e;
-  float dk[D / 8][4], dv[D / 8][4];
+  // lse_sel (log2 units) and D of the query rows n*8 + 2*q4 + {0, 1}.
+  auto load_rows = [&](int i, float2 (&ls)[S / 8], float2 (&dd)[S / 8]) {
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
+    for (int n = 0; n < S / 8; ++n) {
+      const int64_t o = rowbase + (int64_t)i * S + n * 8 + 2 * q4;
+      const float2 l = *reinterpret_cast<const float2*>(a.lse_sel + o);
+      ls[n] = make_float2(l.x * kLog2e, l.y * kLog2e);
+      dd[n] = *reinterpret_cast<const float2*>(a.Dc + o);
+    }
+  };
 
-  for (int p = 0; p < mine; ++p) {
-    cp_async_wait<C::NS - 2>();
-    __syncwarp();
-    if (p + C::NS - 1 < mine) load_pair(list[warp + 4 * (p + C::NS - 1)], (p + C::NS - 1) % C::NS);
-    cp_async_commit();
-    const int st = p % C::NS;
-    const int i = list[warp + 4 * p];
-    bf16 (*qs)[C::LD] = qbuf(st);
-    bf16 (*gs)[C::LD] = gbuf(st);
-    const float* ls = lbuf(st);
-    const float* ds = dbuf(st);
-
-    // S^T (16 keys x S rows) and dP^T
-    float sT[S / 8][4], pT[S / 8][4];
+  bool ok = true;
+  auto wait_bar = [&](uint64_t* bar, uint32_t ph) {
+    ok = __all_sync(0xffffffffu, mbar_wait(bar, ph, abort_flag)) && ok;
+  };
+  const uint32_t kt = smem_u32(smem + C::KV_OFF), vt = kt + C::KT;
+  auto products = [&](float (&sT)[S / 8][4], float (&pT)[S / 8][4], int slot) {
+    const uint32_t qt = smem_u32(ring + slot * C::SLOT), gq = qt + C::QT;
 #pragma unroll
     for (int n = 0; n < S / 8; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sT[n][e] = pT[n][e] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t ka[4], va[4];  // the key slice's K and V rows as A fragments
-      ldsm_x4(ka, &kvs[lane & 15][kk * 16 + (lane >> 4) * 8]);
-      ldsm_x4(va, &kvs[16 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+      uint32_t ka[4], va[4];  // the slice's K and V rows as A fragments
+      const uint32_t aoff = (kk / 4) * C::KHALF + swz(lane & 15, (kk % 4) * 2 + (lane >> 4));
+      ldsm_x4_addr(ka, kt + aoff);
+      ldsm_x4_addr(va, vt + aoff);
 #pragma unroll
       for (int jn = 0; jn < S / 16; ++jn) {
         uint32_t qb[4], gb[4];
-        const int rr = jn * 16 + (lane & 7) + ((lane >> 4) << 3), cc = kk * 16 + ((lane >> 3) & 1) * 8;
-        ldsm_x4(qb, &qs[rr][cc]);
-        ldsm_x4(gb, &gs[rr][cc]);
+        const int r = jn * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const uint32_t boff = (kk / 4) * C::HALF + swz(r, (kk % 4) * 2 + ((lane >> 3) & 1));
+        ldsm_x4_addr(qb, qt + boff);
+        ldsm_x4_addr(gb, gq + boff);
         mma16816(sT[2 * jn], ka, qb[0], qb[1]);
         mma16816(sT[2 * jn + 1], ka, qb[2], qb[3]);
         mma16816(pT[2 * jn], va, gb[0], gb[1]);
         mma16816(pT[2 * jn + 1], va, gb[2], gb[3]);
       }
     }
-    const bool diag = (i == j);
+  };
+  float dk[D / 8][4], dv[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
+  auto grads = [&](float (&sT)[S / 8][4], float (&pT)[S / 8][4], int slot, const float2 (&ls)[S / 8],
+                   const float2 (&dd)[S / 8], int i) {
+    const uint32_t qt = smem_u32(ring + slot * C::SLOT), gq = qt + C::QT;
+    const bool diag = i == j;
 #pragma unroll
     for (int n = 0; n < S / 8; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int c = n * 8 + 2 * q4 + (e & 1);  // query row within the block
-        float p_ = fast_ex2(fmaf(sT[n][e], sl2, -ls[c] * kLog2e));
+        float p_ = fast_ex2(fmaf(sT[n][e], sl2, -((e & 1) ? ls[n].y : ls[n].x)));
         if (diag && u0 + g8 + 8 * (e >> 1) > i * S + c) p_ = 0.f;
         sT[n][e] = p_;
-        pT[n][e] = p_ * (pT[n][e] - ds[c]);  // dS^T
+        pT[n][e] = p_ * (pT[n][e] - ((e & 1) ? dd[n].y : dd[n].x));  // dS^T
       }
 #pragma unroll
     for (int kk = 0; kk < S / 16; ++kk) {
@@ -417,21 +462,62 @@ __global__ void __launch_bounds__(NT) bwd_dkv_walk_kernel(BwdArgs a, WalkShape s
       da[1] = pack2(pT[2 * kk][2], pT[2 * kk][3]);
       da[2] = pack2(pT[2 * kk + 1][0], pT[2 * kk + 1][1]);
       da[3] = pack2(pT[2 * kk + 1][2], pT[2 * kk + 1][3]);
+      const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int jd = 0; jd < D / 16; ++jd) {
         uint32_t gb[4], qb[4];
-        const int rr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, cc = jd * 16 + (lane >> 4) * 8;
-        ldsm_x4_t(gb, &gs[rr][cc]);
-        ldsm_x4_t(qb, &qs[rr][cc]);
+        const uint32_t off = (jd / 4) * C::HALF + swz(r, (jd % 4) * 2 + (lane >> 4));
+        ldsm_x4_t_addr(gb, gq + off);
+        ldsm_x4_t_addr(qb, qt + off);
         mma16816(dv[2 * jd], pa, gb[0], gb[1]);
         mma16816(dv[2 * jd + 1], pa, gb[2], gb[3]);
         mma16816(dk[2 * jd], da, qb[0], qb[1]);
         mma16816(dk[2 * jd + 1], da, qb[2], qb[3]);
       }
     }
-    __syncwarp();  // the stage is read before a later load_pair refills it
+  };
+
+  float sc[S / 8][4], pc[S / 8][4];  // products of the current query block
+  float2 lc[S / 8], dc[S / 8];
+  int ic = 0;
+  int st = 0;
+  uint32_t ph = 0;
+  wait_bar(kvbar, 0);
+  if (mine > 0) {
+    ic = list[warp];
+    load_rows(ic, lc, dc);
+    wait_bar(&full[0], 0);
+    products(sc, pc, 0);
   }
-  cp_async_wait<0>();
+  for (int p = 0; p < mine; ++p) {
+    const int st1 = st + 1 == C::NS ? 0 : st + 1;
+    const uint32_t ph1 = st1 == 0 ? ph ^ 1u : ph;
+    __syncwarp();  // the warp is done with query block p - 1's slot
+    if (lane == 0 && issued < mine) issue_next(st == 0 ? C::NS - 1 : st - 1);
+    float sn[S / 8][4], pn[S / 8][4];
+    float2 ln[S / 8], dn[S / 8];
+    int in = 0;
+    if (p + 1 < mine) {
+      in = list[warp + C::NW * (p + 1)];
+      load_rows(in, ln, dn);
+      wait_bar(&full[st1], ph1);
+      products(sn, pn, st1);
+    }
+    grads(sc, pc, st, lc, dc, ic);
+#pragma unroll
+    for (int n = 0; n < S / 8; ++n) {
+      lc[n] = ln[n];
+      dc[n] = dn[n];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        sc[n][e] = sn[n][e];
+        pc[n][e] = pn[n][e];
+      }
+    }
+    ic = in;
+    st = st1;
+    ph = ph1;
+  }
   __syncthreads();  // every warp is done with its ring: it becomes the reduction buffer
 
   float* red = reinterpret_cast<float*>(smem);  // [warp][2][16][D]
@@ -452,17 +538,18 @@ __global__ void __launch_bounds__(NT) bwd_dkv_walk_kernel(BwdArgs a, WalkShape s
     const int which = e / (16 * D), off = e % (16 * D);
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < C::NW; ++w) {
       const float4 x = *reinterpret_cast<const float4*>(red + (w * 2 + which) * 16 * D + off);
       s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
     }
     *reinterpret_cast<float4*>(pk + which * plane + off) = s;
   }
+  if (!ok && lane == 0) atomicCAS(sh.status, 0, (int)SSA_ERR_TIMEOUT);
 }
 
 template <int D, int S>
-cudaError_t launch_t(const Dims& Dm, const BwdArgs& a, cudaStream_t st) {
-  WalkShape sh{Dm.Hq, Dm.g, Dm.N, Dm.n, a.words, Dm.scale};
+cudaError_t launch_t(const Dims& Dm, const BwdArgs& a, int32_t* status, cudaStream_t st) {
+  WalkShape sh{Dm.Hq, Dm.g, Dm.N, Dm.n, a.words, Dm.scale, status};
   {
     using C = DqCfg<D, S>;
     auto kern = bwd_dq_walk_kernel<D, S>;
@@ -481,10 +568,15 @@ cudaError_t launch_t(const Dims& Dm, const BwdArgs& a, cudaStream_t st) {
   float* part = a.dhf;  // the dh_f and dO_c regions, unused by the sparse stream alone, hold g partials
   {
     using C = KvCfg<D, S>;
+    CUtensorMap mq, mg, mk, mv;
+    if (!make_tma_map_bf16(&mq, a.q, Dm.B, Dm.Hq, Dm.N, S, D) || !make_tma_map_bf16(&mg, a.gs, Dm.B, Dm.Hq, Dm.N, S, D) ||
+        !make_tma_map_bf16(&mk, a.k, Dm.B, Dm.Hkv, Dm.N, 16, D) || !make_tma_map_bf16(&mv, a.v, Dm.B, Dm.Hkv, Dm.N, 16, D))
+      return cudaErrorInvalidValue;
     auto kern = bwd_dkv_walk_kernel<D, S>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(Dm.n * (S / 16), Dm.Hq, Dm.B), NT, C::SMEM, st>>>(a, sh, part);
+    kern<<<dim3(Dm.Hq, Dm.n * (S / 16), Dm.B), NT, C::SMEM, st>>>(mq, mg, mk, mv, a, sh, part);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -497,9 +589,9 @@ bool bwd_walk_supported(const Dims& D) {
   return D.dtype == SSA_BF16 && !D.per_token && (D.s == 16 || D.s == 32) && (D.d == 64 || D.d == 128);
 }
 
-cudaError_t launch_bwd_walk(const Dims& D, const BwdArgs& a, cudaStream_t st) {
-  if (D.d == 64) return D.s == 16 ? launch_t<64, 16>(D, a, st) : launch_t<64, 32>(D, a, st);
-  return D.s == 16 ? launch_t<128, 16>(D, a, st) : launch_t<128, 32>(D, a, st);
+cudaError_t launch_bwd_walk(const Dims& D, const BwdArgs& a, int32_t* dev_status, cudaStream_t st) {
+  if (D.d == 64) return D.s == 16 ? launch_t<64, 16>(D, a, dev_status, st) : launch_t<64, 32>(D, a, dev_status, st);
+  return D.s == 16 ? launch_t<128, 16>(D, a, dev_status, st) : launch_t<128, 32>(D, a, dev_status, st);
 }
 
 }  // namespace ssa

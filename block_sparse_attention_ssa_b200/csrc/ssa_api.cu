@@ -429,7 +429,9 @@ ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* Q, const
     // dO_c regions (2 x B*Hq*N*d floats), which the sparse stream leaves unused.
     if (L.Df - L.dhf < 2 * (size_t)D.B * D.Hq * D.N * D.d * sizeof(float)) return SSA_ERR_WORKSPACE;
     a.maskT = at<uint32_t>(ws, L.maskT);
-    return from_cuda(launch_bwd_walk(D, a, st));
+    int32_t* status = device_status_ptr();
+    if (status == nullptr) return SSA_ERR_CUDA;
+    return from_cuda(launch_bwd_walk(D, a, status, st));
   }
   if (bwd_tc_supported(D)) {
     int32_t* status = device_status_ptr();

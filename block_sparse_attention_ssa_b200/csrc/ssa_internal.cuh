@@ -223,7 +223,7 @@ cudaError_t launch_kvsum(const Dims& D, const BwdArgs& a, const float* part, int
 // Sparse stream alone at blocks of 16 or 32, backward: dQ walk (also writes D_t to a.Dc), dK / dV per (query head,
 // key slice) into fp32 partials in the a.dhf / a.doc regions, then kvsum.
 bool bwd_walk_supported(const Dims& D);
-cudaError_t launch_bwd_walk(const Dims& D, const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_walk(const Dims& D, const BwdArgs& a, int32_t* dev_status, cudaStream_t st);
 // Tensor-core (tcgen05) dual backward with per-row selection masks, bf16,
 // d = 64; takes the bf16 dh_f / dO_c written by the warp-level preprocess.
 bool bwd_tcm_supported(const Dims& D);
