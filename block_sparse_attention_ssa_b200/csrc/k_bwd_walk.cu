@@ -54,24 +54,38 @@ __device__ __forceinline__ void group_sync(int grp) {
 
 // ---------------------------------------------------------------- dQ -----
 
+// Shared memory of a dQ CTA, per query block (group of W warps): NS slots,
+// each the K block then the V block of one selected key block, stored as
+// 64-column halves of S rows x 128 B in the TMA 128-byte swizzle (the 16-byte
+// chunk c of row r sits at chunk c ^ (r & 7)).
 template <int D, int S>
 struct DqCfg {
   static constexpr int W = S / 16;
   static constexpr int G = 4 / W;
-  static constexpr int NS = D == 64 ? 3 : 2;
-  static constexpr int LD = D + 8;
-  static constexpr int STAGE = S * LD * 2;  // stage 0 later stages the output
-  static constexpr int GRP_BYTES = NS * 2 * STAGE;
-  static constexpr int SEL_OFF = G * GRP_BYTES;
-  static constexpr int SMEM = SEL_OFF + G * 64 * 4;
+  static constexpr int NS = 3;             // block it (dS K), block it + 1 (its products), one load ahead
+  static constexpr int HALF = S * 128;     // 64 columns of one block
+  static constexpr int TILE = (D / 64) * HALF;
+  static constexpr int SLOT = 2 * TILE;    // K, then V
+  static constexpr int GRP_BYTES = NS * SLOT;
+  static constexpr int BAR_OFF = G * GRP_BYTES;          // NS mbarriers per query block
+  static constexpr int FLAG_OFF = BAR_OFF + G * NS * 8;  // one abort flag per query block
+  static constexpr int SEL_OFF = FLAG_OFF + G * 4;       // one 2048-bit selection set per query block
+  static constexpr int SMEM = SEL_OFF + G * 64 * 4 + 1024;  // + alignment slack
 };
 
+// Byte offset of the 16-byte chunk `ch` (0..7) of row r in a swizzled half.
+__device__ __forceinline__ uint32_t swz(int r, int ch) { return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4)); }
+
 template <int D, int S>
-__global__ void __launch_bounds__(NT, D == 64 ? 4 : 2) bwd_dq_walk_kernel(BwdArgs a, WalkShape sh) {
+__global__ void __launch_bounds__(NT, D == 64 ? (S == 16 ? 4 : 3) : 2)
+    bwd_dq_walk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, BwdArgs a,
+                       WalkShape sh) {
   using C = DqCfg<D, S>;
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int grp = warp / C::W, gt = (warp % C::W) * 32 + lane;
+  const int grp = warp / C::W, wig = warp % C::W, gt = wig * 32 + lane;
   const int qt = gridDim.x - 1 - blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z, kvh = h / sh.g;
   const int t0 = qt * BM;
@@ -80,41 +94,49 @@ __global__ void __launch_bounds__(NT, D == 64 ? 4 : 2) bwd_dq_walk_kernel(BwdArg
   const int64_t rowbase = ((int64_t)b * sh.Hq + h) * sh.N;
 
   unsigned char* gbase = smem + grp * C::GRP_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + grp * C::NS;
+  int* abort_flag = reinterpret_cast<int*>(smem + C::FLAG_OFF) + grp;
   uint32_t* sel = reinterpret_cast<uint32_t*>(smem + C::SEL_OFF) + grp * 64;
-  auto kbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(gbase + (2 * st) * C::STAGE); };
-  auto vbuf = [&](int st) { return reinterpret_cast<bf16 (*)[C::LD]>(gbase + (2 * st + 1) * C::STAGE); };
 
   const uint32_t* mrow = a.mask + (rowbase / sh.N * sh.n + i) * sh.words;
   for (int w = gt; w < 64; w += 32 * C::W) sel[w] = w < sh.words ? mrow[w] : 0u;
+  if (gt == 0) {
+#pragma unroll
+    for (int s = 0; s < C::NS; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
   group_sync<C::W>(grp);
 
+  // Number of selected blocks, and whether the diagonal one (always the last
+  // in ascending order) is among them.
   const int nw = i / 32 + 1;
-  auto next_blk = [&](int from) -> int {
-    for (int w = from >> 5; w < nw; ++w) {
-      uint32_t bits = sel[w];
-      if (w == (from >> 5)) bits &= ~0u << (from & 31);
-      if (bits) return w * 32 + __ffs(bits) - 1;
-    }
-    return -1;
-  };
-  auto load_blk = [&](int j, int st) {
-    bf16 (*ks)[C::LD] = kbuf(st);
-    bf16 (*vs)[C::LD] = vbuf(st);
-    for (int e = gt; e < S * D / 8; e += 32 * C::W) {
-      const int r = e / (D / 8), c = (e % (D / 8)) * 8;
-      cp_async16(&ks[r][c], row_ptr<bf16>(a.k, b, kvh, (int64_t)j * S + r) + c, 16);
-      cp_async16(&vs[r][c], row_ptr<bf16>(a.v, b, kvh, (int64_t)j * S + r) + c, 16);
-    }
-  };
-  int issued = -1;
+  int cnt = 0;
+  for (int w = lane; w < nw; w += 32) cnt += __popc(sel[w]);
 #pragma unroll
-  for (int p = 0; p < C::NS - 1; ++p) {
-    const int j = next_blk(issued + 1);
-    if (j >= 0) {
-      load_blk(j, p);
-      issued = j;
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  const bool diag_sel = (sel[i >> 5] >> (i & 31)) & 1u;
+
+  // Thread gt == 0 issues the loads, in ascending block order.
+  int iw = 0, issued = 0;
+  uint32_t ibits = sel[0];
+  auto issue_next = [&](int slot) {
+    while (ibits == 0u) ibits = sel[++iw];  // bounded: fewer than cnt blocks issued
+    const int j = iw * 32 + __ffs(ibits) - 1;
+    ibits &= ibits - 1u;
+    unsigned char* dst = gbase + slot * C::SLOT;
+    mbar_expect_tx(&full[slot], C::SLOT);
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh) {
+      tma_load_4d(dst + hh * C::HALF, &tmK, &full[slot], hh * 64, j * S, kvh, b);
+      tma_load_4d(dst + C::TILE + hh * C::HALF, &tmV, &full[slot], hh * 64, j * S, kvh, b);
     }
-    cp_async_commit();
+    ++issued;
+  };
+  if (gt == 0) {
+#pragma unroll
+    for (int s = 0; s < C::NS - 1; ++s)
+      if (issued < cnt) issue_next(s);
   }
 
   // D_t = g_s[t] . h_s[t]: two lanes per row, then to the fragment rows.
@@ -167,30 +189,13 @@ __global__ void __launch_bounds__(NT, D == 64 ? 4 : 2) bwd_dq_walk_kernel(BwdArg
     }
   }
 
-  const float sl2 = sh.scale * kLog2e;
-  float dq[D / 8][4];
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dq[n][e] = 0.f;
-
-  int cur = next_blk(0);
-  for (int it = 0; cur >= 0; ++it) {
-    cp_async_wait<C::NS - 2>();
-    group_sync<C::W>(grp);
-    {
-      const int j = next_blk(issued + 1);
-      if (j >= 0) {
-        load_blk(j, (it + C::NS - 1) % C::NS);
-        issued = j;
-      }
-      cp_async_commit();
-    }
-    const int st = it % C::NS;
-    bf16 (*ks)[C::LD] = kbuf(st);
-    bf16 (*vs)[C::LD] = vbuf(st);
-
-    float sc[S / 8][4], dp[S / 8][4];
+  bool ok = true;
+  auto wait_slot = [&](int slot, uint32_t ph) {
+    ok = __all_sync(0xffffffffu, mbar_wait(&full[slot], ph, abort_flag)) && ok;
+  };
+  // S = Q K^T and dP = g_s V^T of one key block (16 rows x S keys).
+  auto products = [&](float (&sc)[S / 8][4], float (&dp)[S / 8][4], int slot) {
+    const uint32_t kt = smem_u32(gbase + slot * C::SLOT), vt = kt + C::TILE;
 #pragma unroll
     for (int n = 0; n < S / 8; ++n)
 #pragma unroll
@@ -200,23 +205,33 @@ __global__ void __launch_bounds__(NT, D == 64 ? 4 : 2) bwd_dq_walk_kernel(BwdArg
 #pragma unroll
       for (int jn = 0; jn < S / 16; ++jn) {
         uint32_t kb[4], vb[4];
-        const int rr = jn * 16 + (lane & 7) + ((lane >> 4) << 3), cc = kk * 16 + ((lane >> 3) & 1) * 8;
-        ldsm_x4(kb, &ks[rr][cc]);
-        ldsm_x4(vb, &vs[rr][cc]);
+        const int r = jn * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const uint32_t off = (kk / 4) * C::HALF + swz(r, (kk % 4) * 2 + ((lane >> 3) & 1));
+        ldsm_x4_addr(kb, kt + off);
+        ldsm_x4_addr(vb, vt + off);
         mma16816(sc[2 * jn], qa[kk], kb[0], kb[1]);
         mma16816(sc[2 * jn + 1], qa[kk], kb[2], kb[3]);
         mma16816(dp[2 * jn], ga[kk], vb[0], vb[1]);
         mma16816(dp[2 * jn + 1], ga[kk], vb[2], vb[3]);
       }
-    const bool diag = (cur == i);
+  };
+  const float sl2 = sh.scale * kLog2e;
+  float dq[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dq[n][e] = 0.f;
+  // dS = P (dP - D), then dQ += dS K.
+  auto grads = [&](float (&sc)[S / 8][4], const float (&dp)[S / 8][4], int slot, bool diag) {
+    const uint32_t kt = smem_u32(gbase + slot * C::SLOT);
 #pragma unroll
     for (int n = 0; n < S / 8; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = e >> 1;
         float p = fast_ex2(fmaf(sc[n][e], sl2, -lse2[r]));
-        if (diag && cur * S + n * 8 + 2 * q4 + (e & 1) > r0 + g8 + 8 * r) p = 0.f;
-        sc[n][e] = p * (dp[n][e] - Dt[r]);  // dS
+        if (diag && i * S + n * 8 + 2 * q4 + (e & 1) > r0 + g8 + 8 * r) p = 0.f;
+        sc[n][e] = p * (dp[n][e] - Dt[r]);
       }
 #pragma unroll
     for (int kk = 0; kk < S / 16; ++kk) {
@@ -225,30 +240,66 @@ __global__ void __launch_bounds__(NT, D == 64 ? 4 : 2) bwd_dq_walk_kernel(BwdArg
       da[1] = pack2(sc[2 * kk][2], sc[2 * kk][3]);
       da[2] = pack2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
       da[3] = pack2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+      const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int jd = 0; jd < D / 16; ++jd) {
         uint32_t kb[4];
-        ldsm_x4_t(kb, &ks[kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8][jd * 16 + (lane >> 4) * 8]);
+        ldsm_x4_t_addr(kb, kt + (jd / 4) * C::HALF + swz(r, (jd % 4) * 2 + (lane >> 4)));
         mma16816(dq[2 * jd], da, kb[0], kb[1]);
         mma16816(dq[2 * jd + 1], da, kb[2], kb[3]);
       }
     }
-    cur = next_blk(cur + 1);
+  };
+
+  // Software pipeline: the products of block it + 1 are issued before the
+  // gradients of block it.
+  float sc[S / 8][4], dp[S / 8][4];
+  int st = 0;
+  uint32_t ph = 0;
+  if (cnt > 0) {
+    wait_slot(0, 0);
+    products(sc, dp, 0);
   }
-  cp_async_wait<0>();
-  group_sync<C::W>(grp);  // every warp of the group is done with the stages
-  bf16 (*qs)[C::LD] = kbuf(0) + (warp % C::W) * 16;  // this warp's 16 output rows
+  for (int it = 0; it < cnt; ++it) {
+    const int st1 = st + 1 == C::NS ? 0 : st + 1;
+    const uint32_t ph1 = st1 == 0 ? ph ^ 1u : ph;
+    group_sync<C::W>(grp);  // every warp of the group is done with block it - 1's slot
+    if (gt == 0 && issued < cnt) issue_next(st == 0 ? C::NS - 1 : st - 1);
+    float sn[S / 8][4], dn[S / 8][4];
+    if (it + 1 < cnt) {
+      wait_slot(st1, ph1);
+      products(sn, dn, st1);
+    }
+    grads(sc, dp, st, diag_sel && it == cnt - 1);
+#pragma unroll
+    for (int n = 0; n < S / 8; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        sc[n][e] = sn[n][e];
+        dp[n][e] = dn[n][e];
+      }
+    st = st1;
+    ph = ph1;
+  }
+  group_sync<C::W>(grp);  // every warp of the group is done with the slots
+
+  // Epilogue: scale * dQ through a swizzled staging tile in slot 0, 16-byte stores.
+  unsigned char* stage = gbase;
 #pragma unroll
   for (int n = 0; n < D / 8; ++n)
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
-      *reinterpret_cast<uint32_t*>(&qs[g8 + 8 * r][n * 8 + 2 * q4]) =
+    for (int r = 0; r < 2; ++r) {
+      const int rr = wig * 16 + g8 + 8 * r;
+      *reinterpret_cast<uint32_t*>(stage + (n / 8) * C::HALF + swz(rr, n % 8) + q4 * 4) =
           pack2(sh.scale * dq[n][2 * r], sh.scale * dq[n][2 * r + 1]);
+    }
   __syncwarp();
   for (int e = lane; e < 16 * D / 8; e += 32) {
-    const int r = e / (D / 8), col = (e % (D / 8)) * 8;
-    *reinterpret_cast<uint4*>(row_ptr_w<bf16>(a.dq, b, h, r0 + r) + col) = *reinterpret_cast<const uint4*>(&qs[r][col]);
+    const int r = e / (D / 8), c = e % (D / 8);
+    *reinterpret_cast<uint4*>(row_ptr_w<bf16>(a.dq, b, h, r0 + r) + c * 8) =
+        *reinterpret_cast<const uint4*>(stage + (c / 8) * C::HALF + swz(wig * 16 + r, c % 8));
   }
+  if (!ok && lane == 0) atomicCAS(sh.status, 0, (int)SSA_ERR_TIMEOUT);
 }
 
 // ------------------------------------------------------------- dK, dV -----
@@ -298,9 +349,6 @@ struct KvCfg {
   static constexpr int SMEM = FLAG_OFF + 16 + 1024;              // abort flag, alignment slack
   static constexpr int MINB = (D == 64 && S == 16) ? 3 : (D == 128 && S == 32) ? 1 : 2;  // resident CTAs per SM the registers are sized for
 };
-
-// Byte offset of the 16-byte chunk `ch` (0..7) of row r in a swizzled half.
-__device__ __forceinline__ uint32_t swz(int r, int ch) { return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4)); }
 
 // One CTA per (query head, 16-key slice u0 .. u0 + 15 of key block j), heads
 // innermost so that every head's early key blocks (the ones most query
@@ -552,10 +600,14 @@ cudaError_t launch_t(const Dims& Dm, const BwdArgs& a, int32_t* status, cudaStre
   WalkShape sh{Dm.Hq, Dm.g, Dm.N, Dm.n, a.words, Dm.scale, status};
   {
     using C = DqCfg<D, S>;
+    CUtensorMap mk, mv;
+    if (!make_tma_map_bf16(&mk, a.k, Dm.B, Dm.Hkv, Dm.N, S, D) || !make_tma_map_bf16(&mv, a.v, Dm.B, Dm.Hkv, Dm.N, S, D))
+      return cudaErrorInvalidValue;
     auto kern = bwd_dq_walk_kernel<D, S>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(Dm.N / BM, Dm.Hq, Dm.B), NT, C::SMEM, st>>>(a, sh);
+    kern<<<dim3(Dm.N / BM, Dm.Hq, Dm.B), NT, C::SMEM, st>>>(mk, mv, a, sh);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
