@@ -560,7 +560,8 @@ def run_ours(args, rank: int, world: int, dist_on: bool):
             sparse_kernels = "fwd_ord (phase A only); bwd_pre_tc + bwd_dkv_tc + bwd_dq_tc (tcgen05)"
         elif w.dtype == "bf16" and w.block in (16, 32) and not args.per_token:
             sparse_kernels = ("fwd_walk; mask + bwd_dq_walk + mask_transpose + bwd_dkv_walk + kvsum "
-                              "(mma.sync block walks: each query block visits only its own selected blocks)")
+                              "(mma.sync block walks fed by TMA: each query block visits only its own selected blocks, "
+                              "each key slice only the query blocks that chose it)")
         elif w.dtype == "bf16":
             sparse_kernels = "fwd_mma (sparse mode); mask + bwd_dq_mma + bwd_dkv_mma (+ kvsum) (mma.sync)"
         else:
