@@ -30,9 +30,12 @@
 // atomics, no waiting on flags).
 #include <algorithm>
 #include <climits>
+#include <type_traits>
 
 #include <cooperative_groups.h>
 
+#include "mma_sync.cuh"
+#include "sm100_ptx.cuh"
 #include "ssa_internal.cuh"
 
 namespace ssa {
@@ -45,12 +48,24 @@ constexpr int CL = 8;    // CTAs per cluster: one cluster per (batch, kv head)
 struct DecodeShape {
   int Hq, g, N, s, n, k, t;
   float scale;
-  int per_token;  // the query side of the score is q_t itself (per-token selection)
+  int per_token;   // the query side of the score is q_t itself (per-token selection)
+  int mma;         // attention on mma.sync with TMA-loaded bf16 K / V chunks (bf16, g <= 16)
+  int chr;         // rows of a chunk on that path: min(CH, s)
+  int32_t* status; // per-device status report (a bounded wait that ran out)
 };
+
+// The bf16 attention phase stages a chunk's K and V as 64-column halves of
+// CH rows x 128 B in the TMA 128-byte swizzle (the 16-byte piece c of row r
+// sits at piece c ^ (r & 7): the 8 rows of an ldmatrix hit different banks),
+// two chunks in flight; the ring needs 1024-byte alignment.
+template <int D>
+constexpr int kTileBytes = (D / 64) * CH * 128;  // one tensor of one chunk
+template <int D>
+constexpr int kRingBytes = 2 * 2 * kTileBytes<D>;
 
 // Byte offsets of the decode kernel's shared memory.
 struct DecodeLayout {
-  size_t qbar, sc, cand, selh, red, q, o, mx, sum, x, k, v, lst, usel, corr, bytes;
+  size_t qbar, sc, cand, selh, red, q, o, mx, sum, x, k, v, lst, usel, corr, bar, bytes;
   __host__ __device__ DecodeLayout(int n, int g, int k_eff, int D) {
     size_t at = 0;
     auto take = [&](size_t nbytes) {
@@ -71,14 +86,160 @@ struct DecodeLayout {
     mx = take((size_t)g * 4);             // [g] running max
     sum = take((size_t)g * 4);            // [g] running sum
     x = take((size_t)g * CH * 4);         // [g][CH] logits / weights of a chunk
-    k = take((size_t)CH * (D + 1) * 4);   // [CH][D+1] K chunk
-    v = take((size_t)CH * D * 4);         // [CH][D] V chunk
+    // [CH][D+1] K chunk and [CH][D] V chunk (fp32), or, contiguous with it,
+    // the bf16 ring of two chunks (K rows, then V rows, kRowPitch bytes each)
+    const size_t kv32 = (size_t)CH * (D + 1) * 4 + (size_t)CH * D * 4;
+    const size_t ring = (size_t)2 * 2 * (D / 64) * CH * 128 + 1024;
+    k = take(std::max((size_t)CH * (D + 1) * 4, (ring > kv32 ? ring - kv32 : 0) + (size_t)CH * (D + 1) * 4));
+    v = take((size_t)CH * D * 4);
     lst = take((size_t)(1 + most) * 4);   // this CTA's blocks of the union
     usel = take((size_t)g * 64 * 4);      // [g][64] every head's selected-block bits
     corr = take((size_t)g * 4);           // [g] rescale factor of a chunk
+    bar = take(32);                       // the ring's two mbarriers and an abort flag
     bytes = at;
   }
 };
+
+// Attention phase of the bf16 decode step on mma.sync: the g <= 16 query heads
+// of the kv head are the 16 rows of one A fragment, so a 64-key chunk is read
+// from shared memory once for every head.  Warp w forms the logits of keys
+// 8w .. 8w + 7 (S = q_t K^T, fp32 accumulation of exact bf16 products), a warp
+// per head updates the online softmax, and warp w adds P V for the columns
+// 16w .. 16w + 15 (P rounded to bf16 for the product, as in the other
+// tensor-core kernels).  The chunk's K / V rows arrive by bulk copies into a
+// two-slot ring (one mbarrier per slot, bounded waits); the partial (o, max,
+// sum) lands where the merge phase reads it.
+template <int D, typename RowsF, typename IssueF>
+__device__ __forceinline__ void decode_attend_mma(const DecodeShape& sh, int G, int rank, int t, int tid, int lane,
+                                                  int warp, const int* slst, const uint32_t* usel, const float* sq,
+                                                  float* so, float* smax, float* ssum, float* scorr, float* sx,
+                                                  uint8_t* ring, uint64_t* cbar, int* cabort, RowsF chunk_rows,
+                                                  IssueF issue_chunk, int cpb) {
+  using namespace warp_mma;
+  (void)rank;
+  (void)t;
+  const int g8 = lane >> 2, q4 = lane & 3;
+  // byte offset of the 16-byte piece `pc` (0..7) of row r in the 64-column half hh
+  auto swz = [](int hh, int r, int pc) { return hh * CH * 128 + r * 128 + ((pc ^ (r & 7)) << 4); };
+  const bool r0ok = g8 < G, r1ok = g8 + 8 < G;  // fragment rows g8, g8 + 8 are heads
+  const int nch = slst[0] * cpb;
+  auto frag = [&](const float* base, int pitch, int c, uint32_t (&a)[4]) {  // rows g8 / g8 + 8, columns c.., c + 8..
+    const float2 z = make_float2(0.f, 0.f);
+    const float2 x0 = r0ok ? *reinterpret_cast<const float2*>(base + g8 * pitch + c) : z;
+    const float2 x1 = r1ok ? *reinterpret_cast<const float2*>(base + (g8 + 8) * pitch + c) : z;
+    const float2 x2 = r0ok ? *reinterpret_cast<const float2*>(base + g8 * pitch + c + 8) : z;
+    const float2 x3 = r1ok ? *reinterpret_cast<const float2*>(base + (g8 + 8) * pitch + c + 8) : z;
+    a[0] = pack2(x0.x, x0.y);
+    a[1] = pack2(x1.x, x1.y);
+    a[2] = pack2(x2.x, x2.y);
+    a[3] = pack2(x3.x, x3.y);
+  };
+  float o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  bool ok = true;
+  for (int chk = 0; chk < nch; ++chk) {
+    const int slot = chk & 1;
+    ok = sm100::mbar_wait(&cbar[slot], (uint32_t)(chk >> 1) & 1u, cabort) && ok;
+    int j, c0;
+    const int rows = chunk_rows(chk, j, c0);
+    const uint8_t* kb = ring + slot * 2 * kTileBytes<D>;
+    uint8_t* vb = ring + slot * 2 * kTileBytes<D> + kTileBytes<D>;
+    if (rows < CH) {  // V rows past the chunk's end (a later block, or beyond t) become zeros
+      for (int e = tid; e < (CH - rows) * (D / 8); e += NT) {
+        const int r = rows + e / (D / 8), c = e % (D / 8);
+        *reinterpret_cast<uint4*>(vb + swz(c / 8, r, c % 8)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      sm100::fence_proxy_async_smem();  // before a later TMA load into the same bytes
+    }
+    {  // logits of keys 8w .. 8w + 7 for every head
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (8 * warp < rows) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; kk += 2) {
+          uint32_t kf[4], qa[4], qb[4];
+          ldsm_x4_addr(kf, saddr(kb + swz(kk / 4, 8 * warp + (lane & 7), (kk % 4) * 2 + (lane >> 3))));
+          frag(sq, D, kk * 16 + 2 * q4, qa);
+          frag(sq, D, (kk + 1) * 16 + 2 * q4, qb);
+          mma16816(a0, qa, kf[0], kf[1]);
+          mma16816(a1, qb, kf[2], kf[3]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int hh = g8 + 8 * (e >> 1), key = 8 * warp + 2 * q4 + (e & 1);
+        if (hh < G) {
+          const bool selh = (usel[hh * 64 + (j >> 5)] >> (j & 31)) & 1u;
+          sx[hh * CH + key] = (selh && key < rows) ? sh.scale * (a0[e] + a1[e]) : kNegInf;
+        }
+      }
+    }
+    __syncthreads();
+    // softmax statistics: a warp per head; the weights go back over the logits
+    for (int hh = warp; hh < G; hh += NT / 32) {
+      float* xs = sx + hh * CH;
+      if (!((usel[hh * 64 + (j >> 5)] >> (j & 31)) & 1u)) {  // the head skips this block
+        xs[lane] = 0.f;
+        xs[lane + 32] = 0.f;
+        if (lane == 0) scorr[hh] = 1.f;
+        continue;
+      }
+      float mt = fmaxf(xs[lane], xs[lane + 32]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+      const float m_old = smax[hh];
+      const float m_new = fmaxf(m_old, mt);
+      const float p0 = (xs[lane] == kNegInf) ? 0.f : __expf(xs[lane] - m_new);
+      const float p1 = (xs[lane + 32] == kNegInf) ? 0.f : __expf(xs[lane + 32] - m_new);
+      float ps = p0 + p1;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      const float corr = (m_old == kNegInf) ? 0.f : __expf(m_old - m_new);
+      __syncwarp();
+      xs[lane] = p0;
+      xs[lane + 32] = p1;
+      if (lane == 0) {
+        smax[hh] = m_new;
+        ssum[hh] = ssum[hh] * corr + ps;
+        scorr[hh] = corr;
+      }
+    }
+    __syncthreads();
+    // o = o * corr + P V for the columns 16w .. 16w + 15
+    if (16 * warp < D) {
+      const float f0 = r0ok ? scorr[g8] : 1.f, f1 = r1ok ? scorr[g8 + 8] : 1.f;
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        o[n][0] *= f0;
+        o[n][1] *= f0;
+        o[n][2] *= f1;
+        o[n][3] *= f1;
+      }
+      const int nks = (rows + 15) / 16;
+      for (int ks = 0; ks < nks; ++ks) {
+        uint32_t pa[4], vf[4];
+        frag(sx, CH, ks * 16 + 2 * q4, pa);
+        ldsm_x4_t_addr(vf, saddr(vb + swz(warp / 4, ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, (warp % 4) * 2 + (lane >> 4))));
+        mma16816(o[0], pa, vf[0], vf[1]);
+        mma16816(o[1], pa, vf[2], vf[3]);
+      }
+    }
+    __syncthreads();  // every warp is done with the slot and the weights
+    if (tid == 0 && chk + 2 < nch) issue_chunk(chk + 2, slot);
+  }
+  if (16 * warp < D) {
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int hh = g8 + 8 * r;
+        if (hh < G) {
+          const int c = 16 * warp + 8 * n + 2 * q4;
+          so[hh * D + c] = o[n][2 * r];
+          so[hh * D + c + 1] = o[n][2 * r + 1];
+        }
+      }
+  }
+  if (!ok) atomicCAS(sh.status, 0, (int)SSA_ERR_TIMEOUT);
+}
 
 // grid (CL, Hkv, B), one cluster of CL CTAs per (batch, kv head).
 //   1. selection: CTA r scores the pooled blocks for the query heads
@@ -98,8 +259,9 @@ struct DecodeLayout {
 // of every (batch, kv head) are resident at once.
 template <typename T, int D>
 __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
-    decode_kernel(TensorRef q, TensorRef K, TensorRef V, TensorRef hout, float* lse, int32_t* idx, float* qsum,
-                  float* kbar, DecodeShape sh) {
+    decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, TensorRef q,
+                  TensorRef K, TensorRef V, TensorRef hout, float* lse, int32_t* idx, float* qsum, float* kbar,
+                  DecodeShape sh) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
@@ -310,6 +472,41 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
     smax[tid] = kNegInf;
     ssum[tid] = 0.f;
   }
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + L.bar);  // the bf16 ring's two slots
+  int* cabort = reinterpret_cast<int*>(smem + L.bar + 16);
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem + L.k) + 1023) & ~uintptr_t(1023));
+  if (sh.mma) {
+    if (tid == 0) {
+      sm100::mbar_init(&cbar[0], 1);
+      sm100::mbar_init(&cbar[1], 1);
+      *cabort = 0;
+      sm100::fence_mbar_init();
+    }
+  }
+  // chunks of the CTA's union blocks: CH rows (chr rows of a block of s < CH
+  // on the bf16 path), the last one cut at t
+  const int crows = sh.mma ? sh.chr : CH;
+  const int cpb = (s + crows - 1) / crows;  // chunks per block
+  auto chunk_rows = [&](int chk, int& j, int& c0) {
+    j = slst[1 + chk / cpb];
+    c0 = j * s + (chk % cpb) * crows;
+    return max(0, min(crows, min(j * s + s, t + 1) - c0));
+  };
+  // bf16 path: one thread loads a chunk's K and V halves into ring slot
+  // `slot` by TMA (the slot's barrier counts the bytes; rows past N read zeros)
+  auto issue_chunk = [&](int chk, int slot) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      int j, c0;
+      chunk_rows(chk, j, c0);
+      uint8_t* base = ring + slot * 2 * kTileBytes<D>;
+      sm100::mbar_expect_tx(&cbar[slot], (uint32_t)(2 * (D / 64) * sh.chr * 128));
+#pragma unroll
+      for (int hh = 0; hh < D / 64; ++hh) {
+        sm100::tma_load_4d(base + hh * CH * 128, &tmK, &cbar[slot], hh * 64, c0, kvh, b);
+        sm100::tma_load_4d(base + kTileBytes<D> + hh * CH * 128, &tmV, &cbar[slot], hh * 64, c0, kvh, b);
+      }
+    }
+  };
   __syncthreads();
   // this CTA's entries [cnt*rank/CL, cnt*(rank+1)/CL) of the ascending union
   if (warp == 0) {
@@ -333,19 +530,23 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
     for (uint32_t xw = w1; xw; xw &= xw - 1, ++pos)
       if (pos >= lo && pos < hi) slst[1 + pos - lo] = 64 * lane + 32 + __ffs(xw) - 1;
     if (lane == 0) slst[0] = hi - lo;
+    if (sh.mma) {  // the first two chunks start at once
+      __syncwarp();
+      const int nch0 = slst[0] * cpb;
+      if (lane == 0)
+        for (int c2 = 0; c2 < 2 && c2 < nch0; ++c2) issue_chunk(c2, c2);
+    }
   }
   __syncthreads();
-  {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (sh.mma) decode_attend_mma<D>(sh, G, rank, t, tid, lane, warp, slst, usel, sq, so, smax, ssum, scorr, sx,
+                                     ring, cbar, cabort, chunk_rows, issue_chunk, cpb);
+  }
+  if (!sh.mma) {
     constexpr int VEC = Vec16<T>::kN;
     constexpr int ITERS = CH * (D / VEC) / NT;  // 16-byte loads per thread per chunk and tensor
     const int nb = slst[0];
-    const int cpb = (s + CH - 1) / CH;  // chunks per block
     const int nch = nb * cpb;
-    auto chunk_rows = [&](int chk, int& j, int& c0) {
-      j = slst[1 + chk / cpb];
-      c0 = j * s + (chk % cpb) * CH;
-      return max(0, min(CH, min(j * s + s, t + 1) - c0));
-    };
     float tk[ITERS][VEC], tv[ITERS][VEC];
     auto load_chunk = [&](int chk) {
       int j, c0;
@@ -476,13 +677,20 @@ __global__ void __launch_bounds__(128) decode_prefill_kernel(TensorRef Q, Tensor
 }
 
 template <typename T, int D>
-cudaError_t decode_t(const Dims& Dm, const DecodeArgs& a, cudaStream_t st) {
-  DecodeShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, a.t, Dm.scale, Dm.per_token};
+cudaError_t decode_t(const Dims& Dm, const DecodeArgs& a, int32_t* status, cudaStream_t st) {
+  // the bf16 path reads chunks of min(CH, s) rows through TMA maps (which
+  // need 16-byte aligned rows and strides; otherwise the CUDA-core path runs)
+  const int chr = std::min(CH, Dm.s);
+  CUtensorMap mk{}, mv{};
+  const int mma = std::is_same<T, __nv_bfloat16>::value && Dm.g <= 16 &&
+                  make_tma_map_bf16(&mk, a.k, Dm.B, Dm.Hkv, Dm.N, chr, D) &&
+                  make_tma_map_bf16(&mv, a.v, Dm.B, Dm.Hkv, Dm.N, chr, D);
+  DecodeShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, a.t, Dm.scale, Dm.per_token, mma, chr, status};
   const size_t smem = DecodeLayout(Dm.n, Dm.g, Dm.k, D).bytes;
   auto run = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(CL, Dm.Hkv, Dm.B), NT, smem, st>>>(a.q, a.k, a.v, a.h, a.lse, a.idx, a.qsum, a.kbar, sh);
+    kern<<<dim3(CL, Dm.Hkv, Dm.B), NT, smem, st>>>(mk, mv, a.q, a.k, a.v, a.h, a.lse, a.idx, a.qsum, a.kbar, sh);
     count_launches(1);
     return cudaGetLastError();
   };
@@ -508,10 +716,11 @@ size_t decode_ws_bytes(const Dims& D) {
   return 0;  // the decode step keeps its scratch in the cluster's shared memory
 }
 
-cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, int32_t* dev_status, cudaStream_t st) {
   if (D.dtype == SSA_BF16)
-    return D.d == 128 ? decode_t<__nv_bfloat16, 128>(D, a, st) : decode_t<__nv_bfloat16, 64>(D, a, st);
-  return D.d == 128 ? decode_t<float, 128>(D, a, st) : decode_t<float, 64>(D, a, st);
+    return D.d == 128 ? decode_t<__nv_bfloat16, 128>(D, a, dev_status, st)
+                      : decode_t<__nv_bfloat16, 64>(D, a, dev_status, st);
+  return D.d == 128 ? decode_t<float, 128>(D, a, dev_status, st) : decode_t<float, 64>(D, a, dev_status, st);
 }
 
 cudaError_t launch_decode_prefill(const Dims& D, const DecodeArgs& a, cudaStream_t st) {

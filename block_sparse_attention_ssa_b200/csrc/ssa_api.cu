@@ -500,7 +500,9 @@ ssa_status_t ssa_decode_step(const ssa_dims_t* dims, const ssa_tensor_t* q, cons
   a.qsum = qsum;
   a.kbar = kbar;
   a.t = t;
-  return from_cuda(launch_decode(D, a, static_cast<cudaStream_t>(stream)));
+  int32_t* status = device_status_ptr();
+  if (status == nullptr) return SSA_ERR_CUDA;
+  return from_cuda(launch_decode(D, a, status, static_cast<cudaStream_t>(stream)));
 }
 
 ssa_status_t ssa_dropped_mass(const ssa_dims_t* dims, const ssa_tensor_t* Q, const ssa_tensor_t* K,

@@ -241,7 +241,7 @@ struct DecodeArgs {
 };
 
 // Sparse-stream decode of the token at position a.t (CUDA cores).
-cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, int32_t* dev_status, cudaStream_t st);
 // Decode state from a prompt of a.t tokens: kbar of its complete blocks, qsum of the partial block.
 cudaError_t launch_decode_prefill(const Dims& D, const DecodeArgs& a, cudaStream_t st);
 // Dynamic shared memory the decode kernels need for these dims.
