@@ -51,6 +51,7 @@ struct DecodeShape {
   int per_token;   // the query side of the score is q_t itself (per-token selection)
   int mma;         // attention on mma.sync with TMA-loaded bf16 K / V chunks (bf16, g <= 16)
   int chr;         // rows of a chunk on that path: min(CH, s)
+  int kbs;         // this CTA's slice of the pooled keys comes into shared memory by one bulk copy
   int32_t* status; // per-device status report (a bounded wait that ran out)
 };
 
@@ -95,7 +96,7 @@ struct DecodeLayout {
     lst = take((size_t)(1 + most) * 4);   // this CTA's blocks of the union
     usel = take((size_t)g * 64 * 4);      // [g][64] every head's selected-block bits
     corr = take((size_t)g * 4);           // [g] rescale factor of a chunk
-    bar = take(32);                       // the ring's two mbarriers and an abort flag
+    bar = take(32);                       // the ring's two mbarriers, the pooled-key slice's, an abort flag
     bytes = at;
   }
 };
@@ -296,6 +297,22 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
   //     cluster barrier, when every CTA has read the old value)
   const int slice = (n + CL - 1) / CL;
   const int j0 = min(i, i * rank / CL), j1 = min(i, i * (rank + 1) / CL);  // this CTA's blocks of [0, i)
+  // The slice's pooled keys (j1 - j0 rows of D floats, contiguous) start
+  // towards the idle attention ring at once, in flight during (a).
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + L.bar);  // [0], [1]: the attention ring; [2]: the slice
+  int* cabort = reinterpret_cast<int*>(smem + L.bar + 24);
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem + L.k) + 1023) & ~uintptr_t(1023));
+  const bool kb_copy = sh.kbs && j1 > j0;
+  if (tid == 0) {
+    *cabort = 0;
+    if (kb_copy) {
+      sm100::mbar_init(&cbar[2], 1);
+      sm100::fence_mbar_init();
+      const uint32_t bytes = (uint32_t)((j1 - j0) * D * 4);
+      sm100::mbar_expect_tx(&cbar[2], bytes);
+      sm100::bulk_load(ring, kbar + ((int64_t)bk * n + j0) * D, bytes, &cbar[2]);
+    }
+  }
   // (loads of four elements per thread issued before their use; q_t is
   //  kept in the partial-output buffer until the attention phase)
   for (int base = 0; base < G * D; base += 4 * NT) {
@@ -328,26 +345,34 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
   //     (the slice's rows stay in L1 across the heads)
   const float* kb = kbar + (int64_t)bk * n * D;
   const int ns = j1 - j0;  // <= slice <= NT
+  const float* kslice = kb + (int64_t)j0 * D;  // the slice's rows: in shared memory, or read from global
+  bool ok_slice = true;
+  if (kb_copy) {
+    ok_slice = sm100::mbar_wait(&cbar[2], 0, cabort);
+    if (!ok_slice) atomicCAS(sh.status, 0, (int)SSA_ERR_TIMEOUT);
+    kslice = reinterpret_cast<const float*>(ring);
+  }
   // a thread per (block, head group): the block's row is loaded once and
   // dotted with the queries of heads hg, hg + HG, ..
   const int HG = ns > 0 ? min(G, max(1, NT / ns)) : 1;
   if (tid < ns * HG) {
     const int jj = tid % ns, hg = tid / ns;
-    const float4* row = reinterpret_cast<const float4*>(kb + (int64_t)(j0 + jj) * D);
-    // the row in pieces of 64 floats (registers); partial dots per head in
-    // the score slots
-    constexpr int P4 = 16;
+    const float4* row = reinterpret_cast<const float4*>(kslice + (int64_t)jj * D);
+    // the row in pieces of 32 floats (registers); partial dots per head in
+    // the score slots.  Row jj starts at its own 16-byte piece, so that the
+    // rows of a warp read different shared-memory banks.
+    constexpr int P4 = 8;
 #pragma unroll 1
     for (int p0 = 0; p0 < D / 4; p0 += P4) {
       float4 kv[P4];
 #pragma unroll
-      for (int c4 = 0; c4 < P4; ++c4) kv[c4] = row[p0 + c4];
+      for (int c4 = 0; c4 < P4; ++c4) kv[c4] = row[(p0 + c4 + jj) & (D / 4 - 1)];
       for (int hh = hg; hh < G; hh += HG) {
-        const float* qv = sqbar + hh * D + 4 * p0;
+        const float4* qv = reinterpret_cast<const float4*>(sqbar + hh * D);
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int c4 = 0; c4 < P4; ++c4) {
-          const float4 qq = *reinterpret_cast<const float4*>(qv + 4 * c4);
+          const float4 qq = qv[(p0 + c4 + jj) & (D / 4 - 1)];
           a0 = fmaf(qq.x, kv[c4].x, fmaf(qq.y, kv[c4].y, a0));
           a1 = fmaf(qq.z, kv[c4].z, fmaf(qq.w, kv[c4].w, a1));
         }
@@ -374,70 +399,102 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
       const int hh = e / ns, jj = e % ns;
       const float* sc = ssc + hh * slice;
       const float v = sc[jj];
-      int rk = 0;
-      for (int o = 0; o < ns; ++o) {
-        const float w = sc[o];
-        rk += (w > v || (w == v && o < jj)) ? 1 : 0;
+      int rk0 = 0, rk1 = 0, o = 0;
+      for (; o + 8 <= ns; o += 8) {  // eight loads in flight, two counters
+#pragma unroll
+        for (int u = 0; u < 8; u += 2) {
+          const float w0 = sc[o + u], w1 = sc[o + u + 1];
+          rk0 += (w0 > v || (w0 == v && o + u < jj)) ? 1 : 0;
+          rk1 += (w1 > v || (w1 == v && o + u + 1 < jj)) ? 1 : 0;
+        }
       }
+      for (; o < ns; ++o) {
+        const float w = sc[o];
+        rk0 += (w > v || (w == v && o < jj)) ? 1 : 0;
+      }
+      const int rk = rk0 + rk1;
       if (rk < km1) scand[hh * 64 + rk] = make_float2(v, __int_as_float(j0 + jj));
     }
   }
   cluster.sync();  // every CTA's candidate lists are visible to the cluster
-  // (d) the owner of head hh merges the CL sorted lists: every entry's rank
-  //     in the union is its rank in its own list plus, for each other list,
-  //     the number of entries that beat it (a binary search, after the lists
-  //     are copied to this CTA); the k-1 best are kept with the diagonal
-  //     block, and the head's query sum, selection bits and idx row written
-  float2* mlist = reinterpret_cast<float2*>(sk);  // [CL][64] copy of one head's lists (the K chunk is free here)
-  for (int hl = 0; rank + CL * hl < G; ++hl) {
-    const int hh = rank + CL * hl, h = kvh * G + hh;
-    uint32_t* sel = selh + hl * 64;
-    for (int c = tid; c < D; c += NT) qsum[((int64_t)b * sh.Hq + h) * D + c] = sq[hh * D + c];
-    if (i + 1 <= sh.k) {
-      for (int j = tid; j <= i; j += NT) atomicOr(&sel[j >> 5], 1u << (j & 31));
-    } else {
-      for (int e = tid; e < CL * km1; e += NT) {
-        const int r = e / km1, c = e % km1;
-        mlist[r * 64 + c] = cluster.map_shared_rank(scand, r)[hh * 64 + c];
-      }
-      __syncthreads();
-      for (int e = tid; e < CL * km1; e += NT) {
-        const int r = e / km1, c = e % km1;
-        const float2 x = mlist[r * 64 + c];
-        const float v = x.x;
-        const int jx = __float_as_int(x.y);
-        if (jx == INT_MAX) continue;  // an unfilled entry
-        int rk = c;
-        for (int r2 = 0; r2 < CL; ++r2) {
-          if (r2 == r) continue;
-          // entries of list r2 that beat (v, jx): a prefix of the sorted list
-          int lo = 0, hi = km1;
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            const float2 y = mlist[r2 * 64 + mid];
-            const int jy = __float_as_int(y.y);
-            const bool beats = jy != INT_MAX && (y.x > v || (y.x == v && jy < jx));
-            if (beats) lo = mid + 1;
-            else hi = mid;
-          }
-          rk += lo;
-        }
-        if (rk < km1) atomicOr(&sel[jx >> 5], 1u << (jx & 31));
-      }
-      if (tid == 0) atomicOr(&sel[i >> 5], 1u << (i & 31));
-    }
-    __syncthreads();
-    if (tid == 0) {  // Sel ascending, -1 padded
-      int32_t* out = idx + ((int64_t)b * sh.Hq + h) * sh.k;
-      int c = 0;
-      for (int w = 0; w <= (i >> 5); ++w)
-        for (uint32_t xw = sel[w]; xw && c < sh.k; xw &= xw - 1) out[c++] = 32 * w + __ffs(xw) - 1;
-      for (; c < sh.k; ++c) out[c] = -1;
-    }
-    // the head's selection into every CTA's copy of all heads' selections
-    for (int e = tid; e < CL * 64; e += NT) cluster.map_shared_rank(usel, e >> 6)[hh * 64 + (e & 63)] = sel[e & 63];
-    __syncthreads();
+  // (d) the owner of head hh (CTA hh mod CL) merges the CL sorted lists:
+  //     every entry's rank in the union is its rank in its own list plus, for
+  //     each other list, the number of entries that beat it (a binary search,
+  //     after the lists are copied to this CTA); the k-1 best are kept with
+  //     the diagonal block, and the head's query sum, selection bits and idx
+  //     row written.  A CTA owning several heads merges them in one pass.
+  const int nown = rank < G ? (G - 1 - rank) / CL + 1 : 0;  // heads rank, rank + CL, ..
+  float2* mlist = reinterpret_cast<float2*>(sk);  // [nown][CL][64] copies of the lists (the K chunk is free here)
+  for (int e = tid; e < nown * D; e += NT) {
+    const int hh = rank + CL * (e / D), c = e % D;
+    qsum[((int64_t)b * sh.Hq + kvh * G + hh) * D + c] = sq[hh * D + c];
   }
+  if (i + 1 <= sh.k) {
+    for (int e = tid; e < nown * (i + 1); e += NT) {
+      const int hl = e / (i + 1), j = e % (i + 1);
+      atomicOr(&selh[hl * 64 + (j >> 5)], 1u << (j & 31));
+    }
+  } else {
+    const int per = CL * km1;  // entries of one head's lists
+    for (int e = tid; e < nown * per; e += NT) {
+      const int hl = e / per, r = (e % per) / km1, c = e % km1;
+      mlist[(hl * CL + r) * 64 + c] = cluster.map_shared_rank(scand, r)[(rank + CL * hl) * 64 + c];
+    }
+    __syncthreads();
+    for (int e = tid; e < nown * per; e += NT) {
+      const int hl = e / per, r = (e % per) / km1, c = e % km1;
+      const float2* ml = mlist + hl * CL * 64;
+      const float2 x = ml[r * 64 + c];
+      const float v = x.x;
+      const int jx = __float_as_int(x.y);
+      if (jx == INT_MAX) continue;  // an unfilled entry
+      int rk = c;
+      for (int r2 = 0; r2 < CL; ++r2) {
+        if (r2 == r) continue;
+        // entries of list r2 that beat (v, jx): a prefix of the sorted list
+        int lo = 0, hi = km1;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          const float2 y = ml[r2 * 64 + mid];
+          const int jy = __float_as_int(y.y);
+          const bool beats = jy != INT_MAX && (y.x > v || (y.x == v && jy < jx));
+          if (beats) lo = mid + 1;
+          else hi = mid;
+        }
+        rk += lo;
+      }
+      if (rk < km1) atomicOr(&selh[hl * 64 + (jx >> 5)], 1u << (jx & 31));
+    }
+    if (tid < nown) atomicOr(&selh[tid * 64 + (i >> 5)], 1u << (i & 31));
+  }
+  __syncthreads();
+  // idx rows, ascending and -1 padded: warp hl writes head rank + CL*hl's
+  // (lane l places the blocks of words 2l and 2l + 1 after a prefix count)
+  if (warp < nown) {
+    const uint32_t* sel = selh + warp * 64;
+    int32_t* out = idx + ((int64_t)b * sh.Hq + kvh * G + rank + CL * warp) * sh.k;
+    const uint32_t w0 = sel[2 * lane], w1 = sel[2 * lane + 1];
+    const int c = __popc(w0) + __popc(w1);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+    int pos = incl - c;
+    for (uint32_t xw = w0; xw; xw &= xw - 1, ++pos)
+      if (pos < sh.k) out[pos] = 64 * lane + __ffs(xw) - 1;
+    for (uint32_t xw = w1; xw; xw &= xw - 1, ++pos)
+      if (pos < sh.k) out[pos] = 64 * lane + 32 + __ffs(xw) - 1;
+    for (int q = cnt + lane; q < sh.k; q += 32) out[q] = -1;
+  }
+  // the heads' selections into every CTA's copy of all heads' selections
+  for (int e = tid; e < nown * CL * 64; e += NT) {
+    const int hl = e / (CL * 64), x = e % (CL * 64);
+    cluster.map_shared_rank(usel, x >> 6)[(rank + CL * hl) * 64 + (x & 63)] = selh[hl * 64 + (x & 63)];
+  }
+  __syncthreads();
   // the token closes block i: its key mean joins the pooled cache (no
   // reader of this call uses kbar[i])
   if (rank == 0 && t % s == s - 1) {
@@ -472,14 +529,13 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
     smax[tid] = kNegInf;
     ssum[tid] = 0.f;
   }
-  uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + L.bar);  // the bf16 ring's two slots
-  int* cabort = reinterpret_cast<int*>(smem + L.bar + 16);
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem + L.k) + 1023) & ~uintptr_t(1023));
   if (sh.mma) {
+    // the ring held the pooled-key slice and the merge's list copies (generic
+    // accesses) before the TMA loads write it
+    sm100::fence_proxy_async_smem();
     if (tid == 0) {
       sm100::mbar_init(&cbar[0], 1);
       sm100::mbar_init(&cbar[1], 1);
-      *cabort = 0;
       sm100::fence_mbar_init();
     }
   }
@@ -685,7 +741,10 @@ cudaError_t decode_t(const Dims& Dm, const DecodeArgs& a, int32_t* status, cudaS
   const int mma = std::is_same<T, __nv_bfloat16>::value && Dm.g <= 16 &&
                   make_tma_map_bf16(&mk, a.k, Dm.B, Dm.Hkv, Dm.N, chr, D) &&
                   make_tma_map_bf16(&mv, a.v, Dm.B, Dm.Hkv, Dm.N, chr, D);
-  DecodeShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, a.t, Dm.scale, Dm.per_token, mma, chr, status};
+  // the pooled-key slice of a CTA fits the ring and starts 16-byte aligned
+  const int kbs = reinterpret_cast<uintptr_t>(a.kbar) % 16 == 0 &&
+                  (size_t)((Dm.n + CL - 1) / CL) * D * 4 <= (size_t)kRingBytes<D>;
+  DecodeShape sh{Dm.Hq, Dm.g, Dm.N, Dm.s, Dm.n, Dm.k, a.t, Dm.scale, Dm.per_token, mma, chr, kbs, status};
   const size_t smem = DecodeLayout(Dm.n, Dm.g, Dm.k, D).bytes;
   auto run = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
