@@ -19,15 +19,17 @@
 // current block's queries) and kbar [B,Hkv,n,d] (means of complete blocks);
 // the call folds q_t into qsum and, when t closes block i, writes kbar_i.
 //
-// One launch per token (CUDA cores, fp32 arithmetic; a token moves a few
-// MB): a thread-block cluster of CL CTAs per (batch, kv head) selects the
-// blocks of the g query heads (every CTA scores a slice of the pooled blocks
-// for every head and keeps each head's best k-1 of its slice; the head's
-// owner merges the CL lists), attends the union of their kept blocks split CL
-// ways (each K/V row read once for all g heads) and merges the partials,
-// exchanging the candidate lists, the selections and the partials through
-// distributed shared memory between cluster barriers (no workspace, no
-// atomics, no waiting on flags).
+// One launch per token (a token moves a few MB): a thread-block cluster of CL
+// CTAs per (batch, kv head) selects the blocks of the g query heads (every CTA
+// scores a slice of the pooled blocks for every head, fp32 on CUDA cores, and
+// keeps each head's best k-1 of its slice; the head's owner merges the CL
+// lists), attends the union of their kept blocks split CL ways (each K/V row
+// read once for all g heads; bf16 on mma.sync with the heads as the rows of
+// one fragment, fp32 on CUDA cores) and merges the partials, exchanging the
+// candidate lists, the selections and the partials through distributed shared
+// memory between cluster barriers (no workspace, no atomics, no waiting on
+// flags; the only waits are the bounded ones on the copies into shared
+// memory).
 #include <algorithm>
 #include <climits>
 #include <type_traits>

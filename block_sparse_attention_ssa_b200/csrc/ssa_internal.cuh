@@ -240,7 +240,8 @@ struct DecodeArgs {
   void* ws;              // decode step: caller workspace (unused: scratch lives in shared memory)
 };
 
-// Sparse-stream decode of the token at position a.t (CUDA cores).
+// Sparse-stream decode of the token at position a.t (one cluster launch; the
+// bf16 attention products on mma.sync).
 cudaError_t launch_decode(const Dims& D, const DecodeArgs& a, int32_t* dev_status, cudaStream_t st);
 // Decode state from a prompt of a.t tokens: kbar of its complete blocks, qsum of the partial block.
 cudaError_t launch_decode_prefill(const Dims& D, const DecodeArgs& a, cudaStream_t st);

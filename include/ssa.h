@@ -270,8 +270,10 @@ SSA_API ssa_status_t ssa_bwd_sparse(const ssa_dims_t* dims, const ssa_tensor_t* 
  * dims->N is the capacity of the K/V caches [B, Hkv, N, d] (a multiple of
  * block); the decode step needs k_eff <= 64 and its shared memory (the g
  * heads' scores of one eighth of the pooled blocks and their candidate lists,
- * queries, partial outputs and selections, a 64-key K/V chunk) must fit a CTA
- * (SSA_ERR_UNSUPPORTED otherwise; every workload here fits). */
+ * queries, partial outputs and selections, two 64-key K/V chunks) must fit a
+ * CTA (SSA_ERR_UNSUPPORTED otherwise; every workload here fits).  Its copies
+ * into shared memory are waited on with a bound: a wait that runs out records
+ * SSA_ERR_TIMEOUT in the per-device report that ssa_device_status reads. */
 
 /* Builds the decode state from a prompt of t0 tokens (0 <= t0 <= N): kbar of
  * the complete blocks 0 .. t0/s - 1 and qsum of the queries of the partial
