@@ -394,7 +394,62 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
   //     entries are NaN (compares false with everything).
   const float kOut = __int_as_float(0x7fffffff);
   const int km1 = sh.k - 1;
-  if (i + 1 > sh.k) {
+  if (i + 1 > sh.k && ns <= 64) {
+    // A warp per head sorts the slice's (score, block) pairs with a bitonic
+    // network, score descending and block ascending (the rank rule's order),
+    // two pairs per lane (elements 2 lane and 2 lane + 1; missing ones rank
+    // last), and keeps the first k-1.
+    for (int hh = warp; hh < G; hh += NT / 32) {
+      const float* sc = ssc + hh * slice;
+      float v[2];
+      int jb[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int e = 2 * lane + q;
+        v[q] = e < ns ? sc[e] : kNegInf;
+        jb[q] = e < ns ? j0 + e : INT_MAX;
+      }
+      auto better = [](float va, int ja, float vb, int jbb) { return va > vb || (va == vb && ja < jbb); };
+#pragma unroll
+      for (int sz = 2; sz <= 64; sz <<= 1) {
+#pragma unroll
+        for (int d = sz >> 1; d > 0; d >>= 1) {
+          if (d == 1) {  // both elements in this lane
+            const bool desc = ((2 * lane) & sz) == 0;
+            if (better(v[1], jb[1], v[0], jb[0]) == desc) {
+              const float tv = v[0];
+              v[0] = v[1];
+              v[1] = tv;
+              const int tj = jb[0];
+              jb[0] = jb[1];
+              jb[1] = tj;
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int e = 2 * lane + q;
+              const float ov = __shfl_xor_sync(0xffffffffu, v[q], d >> 1);
+              const int oj = __shfl_xor_sync(0xffffffffu, jb[q], d >> 1);
+              const bool low = (e & d) == 0;       // the lower index of the pair
+              const bool desc = (e & sz) == 0;     // this run sorts descending
+              // the lower index keeps the better pair in a descending run, the worse in an ascending one
+              const bool take = better(ov, oj, v[q], jb[q]) == (low == desc);
+              if (take) {
+                v[q] = ov;
+                jb[q] = oj;
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int e = 2 * lane + q;
+        if (e < km1) scand[hh * 64 + e] = e < ns ? make_float2(v[q], __int_as_float(jb[q]))
+                                                 : make_float2(kOut, __int_as_float(INT_MAX));
+      }
+    }
+  } else if (i + 1 > sh.k) {
     for (int e = tid; e < G * km1; e += NT) scand[(e / km1) * 64 + e % km1] = make_float2(kOut, __int_as_float(INT_MAX));
     __syncthreads();
     for (int e = tid; e < G * ns; e += NT) {
