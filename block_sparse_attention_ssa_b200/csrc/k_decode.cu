@@ -68,7 +68,7 @@ constexpr int kRingBytes = 2 * 2 * kTileBytes<D>;
 
 // Byte offsets of the decode kernel's shared memory.
 struct DecodeLayout {
-  size_t qbar, sc, cand, selh, red, q, o, mx, sum, x, k, v, lst, usel, corr, bar, bytes;
+  size_t qbar, sc, cand, red, q, o, mx, sum, x, k, v, lst, usel, corr, bar, bytes;
   __host__ __device__ DecodeLayout(int n, int g, int k_eff, int D) {
     size_t at = 0;
     auto take = [&](size_t nbytes) {
@@ -76,13 +76,11 @@ struct DecodeLayout {
       at = (at + nbytes + 15) / 16 * 16;
       return r;
     };
-    const int gl = (g + CL - 1) / CL;                       // heads this CTA selects
     const int most = (std::min(g * k_eff, n) + CL - 1) / CL;  // union blocks this CTA attends
     const int slice = (n + CL - 1) / CL;                    // pooled blocks this CTA scores
     qbar = take((size_t)g * D * 4);       // [g][D] query side of the block scores
     sc = take((size_t)g * slice * 4);     // [g][slice] block scores of this CTA's slice
     cand = take((size_t)g * 64 * 8);      // [g][64] best k-1 (score, block) of the slice
-    selh = take((size_t)gl * 64 * 4);     // [gl][64] selected-block bits of this CTA's heads
     red = take((size_t)NT * 8);           // arg-max candidates / key-sum staging
     q = take((size_t)g * D * 4);          // [g][D] q_t
     o = take((size_t)g * D * 4);          // [g][D] partial output
@@ -281,7 +279,6 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
   float* ssc = reinterpret_cast<float*>(smem + L.sc);
   float2* scand = reinterpret_cast<float2*>(smem + L.cand);  // (score, block index bits)
   float* scorr = reinterpret_cast<float*>(smem + L.corr);
-  uint32_t* selh = reinterpret_cast<uint32_t*>(smem + L.selh);
   float* rv = reinterpret_cast<float*>(smem + L.red);
   float* sq = reinterpret_cast<float*>(smem + L.q);
   float* so = reinterpret_cast<float*>(smem + L.o);
@@ -340,7 +337,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
       }
     }
   }
-  for (int e = tid; e < ((G + CL - 1) / CL) * 64; e += NT) selh[e] = 0u;
+  for (int e = tid; e < G * 64; e += NT) usel[e] = 0u;
   __syncthreads();
   // (b) scores of this CTA's slice for every head: a thread per (head,
   //     block), the whole pooled key row loaded at once as 16-byte vectors
@@ -474,61 +471,124 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
     }
   }
   cluster.sync();  // every CTA's candidate lists are visible to the cluster
-  // (d) the owner of head hh (CTA hh mod CL) merges the CL sorted lists:
-  //     every entry's rank in the union is its rank in its own list plus, for
-  //     each other list, the number of entries that beat it (a binary search,
-  //     after the lists are copied to this CTA); the k-1 best are kept with
-  //     the diagonal block, and the head's query sum, selection bits and idx
-  //     row written.  A CTA owning several heads merges them in one pass.
+  // (d) every CTA merges every head's CL sorted lists, read straight from the
+  //     peers' shared memory: a warp per head sorts the CL lists' candidates
+  //     (score descending, block ascending) with a bitonic network and keeps
+  //     the k-1 best with the diagonal block in this CTA's copy of every
+  //     head's selection bits (k <= 16: four pairs per lane in registers;
+  //     larger k: the warp's share of the idle attention ring).  No selection
+  //     has to cross the cluster afterwards.  The head's owner (CTA hh mod CL)
+  //     writes its query sum and idx row.
+  auto better = [](float va, int ja, float vb, int jb) { return va > vb || (va == vb && ja < jb); };
+  auto merge_heads = [&]() {
+    constexpr int E = 4;
+    constexpr int PER_LIST = 32 * E / CL;  // 16 candidate slots per list (>= k - 1)
+    for (int hh = warp; hh < G; hh += NT / 32) {
+      // Each list is sorted already: odd lists are read in reverse, so every
+      // pair of lists is a bitonic sequence and the network starts at the
+      // merges of 32.
+      float v[E];
+      int jb[E];
+#pragma unroll
+      for (int q = 0; q < E; ++q) {
+        const int e = E * lane + q, r = e / PER_LIST, c0 = e % PER_LIST;
+        const int c = (r & 1) ? PER_LIST - 1 - c0 : c0;
+        float2 x = make_float2(kNegInf, __int_as_float(INT_MAX));
+        if (c < km1) x = cluster.map_shared_rank(scand, r)[hh * 64 + c];
+        jb[q] = __float_as_int(x.y);
+        v[q] = jb[q] == INT_MAX ? kNegInf : x.x;  // unfilled entries rank last
+      }
+#pragma unroll
+      for (int sz = 2 * PER_LIST; sz <= 32 * E; sz <<= 1) {
+#pragma unroll
+        for (int d = sz >> 1; d > 0; d >>= 1) {
+          if (d < E) {  // both elements of a pair in this lane
+#pragma unroll
+            for (int q = 0; q < E; ++q) {
+              if (q & d) continue;
+              const int hi = q | d;
+              const bool desc = ((E * lane + q) & sz) == 0;
+              if (better(v[hi], jb[hi], v[q], jb[q]) == desc) {
+                const float tv = v[q];
+                v[q] = v[hi];
+                v[hi] = tv;
+                const int tj = jb[q];
+                jb[q] = jb[hi];
+                jb[hi] = tj;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < E; ++q) {
+              const int e = E * lane + q;
+              const float ov = __shfl_xor_sync(0xffffffffu, v[q], d / E);
+              const int oj = __shfl_xor_sync(0xffffffffu, jb[q], d / E);
+              const bool low = (e & d) == 0, desc = (e & sz) == 0;
+              // the lower index keeps the better pair in a descending run, the worse in an ascending one
+              if (better(ov, oj, v[q], jb[q]) == (low == desc)) {
+                v[q] = ov;
+                jb[q] = oj;
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < E; ++q)
+        if (E * lane + q < km1 && jb[q] != INT_MAX) atomicOr(&usel[hh * 64 + (jb[q] >> 5)], 1u << (jb[q] & 31));
+      if (lane == 0) atomicOr(&usel[hh * 64 + (i >> 5)], 1u << (i & 31));
+    }
+  };
+  if (i + 1 <= sh.k) {
+    for (int e = tid; e < G * (i + 1); e += NT) {
+      const int hh = e / (i + 1), j = e % (i + 1);
+      atomicOr(&usel[hh * 64 + (j >> 5)], 1u << (j & 31));
+    }
+  } else if (km1 <= 15) {
+    merge_heads();
+  } else {
+    const int per_list = km1 <= 31 ? 32 : 64, n2 = CL * per_list;  // 256 or 512 candidates
+    float2* buf = reinterpret_cast<float2*>(ring) + warp * 512;   // the ring is idle until phase 2
+    for (int hh = warp; hh < G; hh += NT / 32) {
+      for (int e = lane; e < n2; e += 32) {
+        const int r = e / per_list, c = e % per_list;
+        float2 x = make_float2(kNegInf, __int_as_float(INT_MAX));
+        if (c < km1) x = cluster.map_shared_rank(scand, r)[hh * 64 + c];
+        if (__float_as_int(x.y) == INT_MAX) x.x = kNegInf;  // unfilled entries rank last
+        buf[e] = x;
+      }
+      __syncwarp();
+      for (int sz = 2; sz <= n2; sz <<= 1)
+        for (int d = sz >> 1; d > 0; d >>= 1) {
+          for (int pr = lane; pr < n2 / 2; pr += 32) {
+            const int lo = 2 * d * (pr / d) + pr % d, hi = lo + d;  // the pr-th pair at stride d
+            const bool desc = (lo & sz) == 0;
+            const float2 xa = buf[lo], xb = buf[hi];
+            if (better(xb.x, __float_as_int(xb.y), xa.x, __float_as_int(xa.y)) == desc) {
+              buf[lo] = xb;
+              buf[hi] = xa;
+            }
+          }
+          __syncwarp();
+        }
+      for (int e = lane; e < km1; e += 32) {
+        const int jx = __float_as_int(buf[e].y);
+        if (jx != INT_MAX) atomicOr(&usel[hh * 64 + (jx >> 5)], 1u << (jx & 31));
+      }
+      if (lane == 0) atomicOr(&usel[hh * 64 + (i >> 5)], 1u << (i & 31));
+      __syncwarp();  // the buffer is read before the next head refills it
+    }
+  }
+  __syncthreads();
   const int nown = rank < G ? (G - 1 - rank) / CL + 1 : 0;  // heads rank, rank + CL, ..
-  float2* mlist = reinterpret_cast<float2*>(sk);  // [nown][CL][64] copies of the lists (the K chunk is free here)
   for (int e = tid; e < nown * D; e += NT) {
     const int hh = rank + CL * (e / D), c = e % D;
     qsum[((int64_t)b * sh.Hq + kvh * G + hh) * D + c] = sq[hh * D + c];
   }
-  if (i + 1 <= sh.k) {
-    for (int e = tid; e < nown * (i + 1); e += NT) {
-      const int hl = e / (i + 1), j = e % (i + 1);
-      atomicOr(&selh[hl * 64 + (j >> 5)], 1u << (j & 31));
-    }
-  } else {
-    const int per = CL * km1;  // entries of one head's lists
-    for (int e = tid; e < nown * per; e += NT) {
-      const int hl = e / per, r = (e % per) / km1, c = e % km1;
-      mlist[(hl * CL + r) * 64 + c] = cluster.map_shared_rank(scand, r)[(rank + CL * hl) * 64 + c];
-    }
-    __syncthreads();
-    for (int e = tid; e < nown * per; e += NT) {
-      const int hl = e / per, r = (e % per) / km1, c = e % km1;
-      const float2* ml = mlist + hl * CL * 64;
-      const float2 x = ml[r * 64 + c];
-      const float v = x.x;
-      const int jx = __float_as_int(x.y);
-      if (jx == INT_MAX) continue;  // an unfilled entry
-      int rk = c;
-      for (int r2 = 0; r2 < CL; ++r2) {
-        if (r2 == r) continue;
-        // entries of list r2 that beat (v, jx): a prefix of the sorted list
-        int lo = 0, hi = km1;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          const float2 y = ml[r2 * 64 + mid];
-          const int jy = __float_as_int(y.y);
-          const bool beats = jy != INT_MAX && (y.x > v || (y.x == v && jy < jx));
-          if (beats) lo = mid + 1;
-          else hi = mid;
-        }
-        rk += lo;
-      }
-      if (rk < km1) atomicOr(&selh[hl * 64 + (jx >> 5)], 1u << (jx & 31));
-    }
-    if (tid < nown) atomicOr(&selh[tid * 64 + (i >> 5)], 1u << (i & 31));
-  }
-  __syncthreads();
   // idx rows, ascending and -1 padded: warp hl writes head rank + CL*hl's
   // (lane l places the blocks of words 2l and 2l + 1 after a prefix count)
   if (warp < nown) {
-    const uint32_t* sel = selh + warp * 64;
+    const uint32_t* sel = usel + (rank + CL * warp) * 64;
     int32_t* out = idx + ((int64_t)b * sh.Hq + kvh * G + rank + CL * warp) * sh.k;
     const uint32_t w0 = sel[2 * lane], w1 = sel[2 * lane + 1];
     const int c = __popc(w0) + __popc(w1);
@@ -546,12 +606,6 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
       if (pos < sh.k) out[pos] = 64 * lane + 32 + __ffs(xw) - 1;
     for (int q = cnt + lane; q < sh.k; q += 32) out[q] = -1;
   }
-  // the heads' selections into every CTA's copy of all heads' selections
-  for (int e = tid; e < nown * CL * 64; e += NT) {
-    const int hl = e / (CL * 64), x = e % (CL * 64);
-    cluster.map_shared_rank(usel, x >> 6)[(rank + CL * hl) * 64 + (x & 63)] = selh[hl * 64 + (x & 63)];
-  }
-  __syncthreads();
   // the token closes block i: its key mean joins the pooled cache (no
   // reader of this call uses kbar[i])
   if (rank == 0 && t % s == s - 1) {
@@ -574,7 +628,8 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NT, 2)
       kbar[((int64_t)bk * n + i) * D + tid] = sum / (float)s;
     }
   }
-  cluster.sync();  // every head's selection is visible to the cluster
+  // (no cluster barrier here: every CTA holds every head's selection, and the
+  //  peers' candidate lists stay untouched until the last barrier)
 
   // ================================================================ 2. attention
   // (every head's selection was pushed into usel by its owner; q_t waits in so)
