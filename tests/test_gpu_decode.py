@@ -27,9 +27,12 @@ CASES = {
     "f32_d64": (1, 4, 4, 512, 64, 64, 3, "f32", 64 + 40, 100),
     "bf16_full_budget": (1, 4, 2, 512, 128, 64, 16, "bf16", 30, 60),
     "f32_from_empty_prompt": (1, 2, 1, 256, 128, 64, 2, "f32", 0, 140),
-    # 16 heads per kv head (two per selecting CTA) and k = 40: each CTA's
-    # slice keeps 39 candidates per head, merged from eight lists
+    # 16 heads per kv head and k = 40: each CTA's slice keeps 39 candidates
+    # per head, merged from eight lists in shared memory (k > 16)
     "bf16_g16_k40_s16": (1, 16, 1, 4096, 64, 16, 40, "bf16", 2600, 120),
+    # 32 heads per kv head: more than one 16-row fragment, so the attention
+    # phase runs on CUDA cores with bf16 inputs
+    "bf16_g32_cuda_cores": (1, 32, 1, 1024, 64, 64, 6, "bf16", 500, 60),
 }
 
 
