@@ -120,7 +120,7 @@ def test_decode_rejects_bad_positions():
         api.ssa_decode_prefill(dims, dev["Q"], dev["K"], N + 1, st["qsum"], st["kbar"])
 
 
-@pytest.mark.parametrize("wname", ["gqa_16k", "long_64k"])
+@pytest.mark.parametrize("wname", ["gqa_16k", "long_64k", "paper_b16_8k"])
 def test_decode_last_token_full_size(wname):
     """Prefill N-1 tokens of a full-size workload and decode the last token
     (it closes the last block, so the selection is the forward's)."""
