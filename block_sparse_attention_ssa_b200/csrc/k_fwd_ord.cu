@@ -24,21 +24,24 @@
 // With block 64 a 128-row query tile holds two query blocks whose selections
 // differ: phase A walks the union of the two selections and phase D the blocks
 // that either half dropped; a 64-key unit that belongs to the other phase for
-// one half is masked for that half's rows (P = 0).  Steps pair two 64-key units
-// (in ascending order, not necessarily adjacent), loaded by 64-row TMA boxes;
-// with block 128 a step is one block.
+// one half is masked for that half's rows (P = 0).  A step is one 64-key unit
+// (a block of 64, or half of a block of 128), loaded by 64-row TMA boxes into
+// two-slot K and V rings.
 //
 // CTA = one 128-row query tile of one (batch, query head), 192 threads:
 //   warps 0-3  softmax, rescale, snapshot and epilogue: warp w owns TMEM lanes
 //              32w..32w+31 = query rows 32w.. of the tile, one row per thread,
-//              all 128 key columns of a step;
-//   warp 4     TMA producer (Q once, then K and V of each step, one buffer each);
+//              the 64 key columns of a step;
+//   warp 4     TMA producer (Q once, then K and V of each step, two slots each);
 //   warp 5     TMEM allocator and single-thread tcgen05.mma issuer.
-// TMEM (256 columns): O [0,128), S [128,256); P (bf16, two per column)
-// overwrites the first 64 columns of S and feeds the PV product from TMEM.
-// The tensor core runs one CTA's products in issue order, so S of the next
-// step may be issued right after PV of this one (which reads P from the same
-// columns), and its completion implies that PV has completed.
+// TMEM (256 columns): O [0,128), two S buffers [128,192) and [192,256); step
+// j uses buffer j & 1.  P (bf16, two per column) overwrites the first 32
+// columns of its S buffer and feeds the PV product from TMEM.  The products
+// of step j + 2 are issued right after PV of step j, so the tensor core forms
+// the next step's logits while the softmax warps work on this one's.  The
+// tensor core runs one CTA's products in issue order: S of step j + 2 reuses
+// the columns PV of step j read.  O is touched by the softmax warps only for a
+// rescale or a snapshot, after the preceding PV has completed.
 //
 // Softmax in base 2 with the scale folded in: p = 2^(S*c - m), c = scale*log2(e).
 // A row's running max m is raised only when a step's max exceeds it by more
@@ -52,8 +55,7 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128;    // query rows per CTA
-constexpr int BN = 128;    // keys per step
-constexpr int UNIT = 64;   // keys per unit (a TMA box of 64 rows)
+constexpr int UNIT = 64;   // keys per step (a TMA box of 64 rows)
 constexpr int HD = 128;
 constexpr int NTHREADS = 192;
 constexpr int WARP_TMA = 4, WARP_MMA = 5;
@@ -61,18 +63,19 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int MAX_LIST = 4096;  // phase-A plus phase-D entries (<= 2 n, n <= 2048)
 
 constexpr int Q_BYTES = BM * HD * 2;
-constexpr int KV_BYTES = BN * HD * 2;  // one K or V tile
-constexpr int UNIT_BYTES = UNIT * 128; // one 64-row box of 64 columns
+constexpr int KV_BYTES = UNIT * HD * 2;  // one K or V tile of a step
+constexpr int KV_HALF = UNIT * 128;      // its 64-column half (64 rows x 128 B)
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = Q_BYTES;
-constexpr int OFF_V = OFF_K + KV_BYTES;
-constexpr int OFF_MISC = OFF_V + KV_BYTES;
-constexpr uint32_t COL_O = 0, COL_S = 128;
-constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
+constexpr int OFF_K = Q_BYTES;               // two K slots
+constexpr int OFF_V = OFF_K + 2 * KV_BYTES;  // two V slots
+constexpr int OFF_MISC = OFF_V + 2 * KV_BYTES;
+constexpr uint32_t COL_O = 0, COL_S = 128;  // S buffers at COL_S and COL_S + 64
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, UNIT, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
 
 struct Misc {
-  uint64_t q_full, k_full, k_empty, v_full, v_empty, s_full, p_full, o_final, drain;
+  // one barrier per S buffer where the waiter could otherwise fall two phases behind
+  uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], pv_done, o_final, drain;
   uint32_t tmem_base;
   int abort;
   int nA, nD;             // entries of the two phases in list[]
@@ -114,12 +117,15 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   // ---- set-up
   if (threadIdx.x == 0) {
     mbar_init(&M.q_full, 1);
-    mbar_init(&M.k_full, 1);
-    mbar_init(&M.k_empty, 1);
-    mbar_init(&M.v_full, 1);
-    mbar_init(&M.v_empty, 1);
-    mbar_init(&M.s_full, 1);
-    mbar_init(&M.p_full, 4);
+    for (int s2 = 0; s2 < 2; ++s2) {
+      mbar_init(&M.k_full[s2], 1);
+      mbar_init(&M.k_empty[s2], 1);
+      mbar_init(&M.v_full[s2], 1);
+      mbar_init(&M.v_empty[s2], 1);
+      mbar_init(&M.s_full[s2], 1);
+      mbar_init(&M.p_full[s2], 4);
+    }
+    mbar_init(&M.pv_done, 1);
     mbar_init(&M.o_final, 1);
     mbar_init(&M.drain, 1);
     M.abort = 0;
@@ -199,28 +205,17 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   __syncthreads();
   tc_fence_after();
   const int nA = M.nA, nD = M.nD;
-  // Steps: with block 128 one list entry per step; with block 64 two.
-  const int TA = S_BLK == 128 ? nA : (nA + 1) / 2;
-  const int TD = S_BLK == 128 ? nD : (nD + 1) / 2;
+  // Steps: one 64-key unit each (a list entry at block 64, half of one at 128).
+  constexpr int UPB = S_BLK / UNIT;  // units per block
+  const int TA = UPB * nA, TD = UPB * nD;
   const int T = TA + TD;
   const uint32_t tmem = M.tmem_base;
 
-  // Unit q of step j: first key, block, and whether it is a real entry (an odd
-  // last entry of a phase at block 64 is paired with a copy of itself, masked).
-  auto unit_of = [&](int j, int q, int& u0, int& blk, bool& real) {
-    if (S_BLK == 128) {
-      const int e = j < TA ? j : nA + (j - TA);
-      blk = M.list[e];
-      u0 = blk * 128 + q * UNIT;
-      real = true;
-    } else {
-      const int base = j < TA ? 0 : nA, cnt = j < TA ? nA : nD, jj = j < TA ? j : j - TA;
-      int e = 2 * jj + q;
-      real = e < cnt;
-      if (!real) e = cnt - 1;
-      blk = M.list[base + e];
-      u0 = blk * 64;
-    }
+  // The unit of step j: its first key and its block.
+  auto unit_of = [&](int j, int& u0, int& blk) {
+    const int jj = j < TA ? j : j - TA;
+    blk = M.list[(j < TA ? 0 : nA) + jj / UPB];
+    u0 = blk * S_BLK + (jj % UPB) * UNIT;
   };
 
   uint8_t* sQ = smem + OFF_Q;
@@ -238,37 +233,31 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       tma_load_4d(sQ + Q_BYTES / 2, &tmQ, &M.q_full, 64, q0, h, b);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < T; ++j) {
-        int ua, ub, blk;
-        bool real;
-        unit_of(j, 0, ua, blk, real);
-        unit_of(j, 1, ub, blk, real);
-        // one 64-row box per unit and column half, placed at the unit's rows
-        // (the 128-byte swizzle repeats every 8 rows, so the layout equals
-        // that of a 128-row box)
-        auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar) {
-          mbar_expect_tx(bar, KV_BYTES);
-          tma_load_4d(dst, map, bar, 0, ua, kvh, b);
-          tma_load_4d(dst + KV_BYTES / 2, map, bar, 64, ua, kvh, b);
-          tma_load_4d(dst + UNIT_BYTES, map, bar, 0, ub, kvh, b);
-          tma_load_4d(dst + KV_BYTES / 2 + UNIT_BYTES, map, bar, 64, ub, kvh, b);
-        };
-        if (j >= 1 && !mbar_wait(&M.k_empty, (uint32_t)(j - 1) & 1u, abort)) break;
-        load_tile(sK, &tmK, &M.k_full);
+        const int sl = j & 1;
+        int u0, blk;
+        unit_of(j, u0, blk);
+        // the slot's previous tile (step j - 2) must have been consumed
+        if (j >= 2 && !mbar_wait(&M.k_empty[sl], (uint32_t)((j - 2) >> 1) & 1u, abort)) break;
+        mbar_expect_tx(&M.k_full[sl], KV_BYTES);
+        tma_load_4d(sK + sl * KV_BYTES, &tmK, &M.k_full[sl], 0, u0, kvh, b);
+        tma_load_4d(sK + sl * KV_BYTES + KV_HALF, &tmK, &M.k_full[sl], 64, u0, kvh, b);
         k_issued = j + 1;
-        if (j >= 1 && !mbar_wait(&M.v_empty, (uint32_t)(j - 1) & 1u, abort)) break;
-        load_tile(sV, &tmV, &M.v_full);
+        if (j >= 2 && !mbar_wait(&M.v_empty[sl], (uint32_t)((j - 2) >> 1) & 1u, abort)) break;
+        mbar_expect_tx(&M.v_full[sl], KV_BYTES);
+        tma_load_4d(sV + sl * KV_BYTES, &tmV, &M.v_full[sl], 0, u0, kvh, b);
+        tma_load_4d(sV + sl * KV_BYTES + KV_HALF, &tmV, &M.v_full[sl], 64, u0, kvh, b);
         v_issued = j + 1;
       }
       // Drain: every copy this thread issued must have landed before the CTA exits.
       int dummy = 0;
       mbar_wait(&M.q_full, 0, &dummy);
-      if (k_issued > 0) {
+      for (int j = k_issued > 2 ? k_issued - 2 : 0; j < k_issued; ++j) {
         dummy = 0;
-        mbar_wait(&M.k_full, (uint32_t)(k_issued - 1) & 1u, &dummy);
+        mbar_wait(&M.k_full[j & 1], (uint32_t)(j >> 1) & 1u, &dummy);
       }
-      if (v_issued > 0) {
+      for (int j = v_issued > 2 ? v_issued - 2 : 0; j < v_issued; ++j) {
         dummy = 0;
-        mbar_wait(&M.v_full, (uint32_t)(v_issued - 1) & 1u, &dummy);
+        mbar_wait(&M.v_full[j & 1], (uint32_t)(j >> 1) & 1u, &dummy);
       }
     }
   } else if (warp == WARP_MMA) {
@@ -276,33 +265,44 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     if (lane == 0) {
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       bool ok = mbar_wait(&M.q_full, 0, abort);
-      for (int j = 0; ok && j < T; ++j) {
-        const uint32_t ph = (uint32_t)j & 1u;
-        if (!mbar_wait(&M.k_full, ph, abort)) {
-          ok = false;
-          break;
-        }
+      // S of step j into buffer j & 1
+      auto issue_s = [&](int j) {
+        const int sl = j & 1;
+        if (!mbar_wait(&M.k_full[sl], (uint32_t)(j >> 1) & 1u, abort)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off_q = (kk >> 2) * (Q_BYTES / 2) + (kk & 3) * 32;
-          const uint32_t off_k = (kk >> 2) * (KV_BYTES / 2) + (kk & 3) * 32;
-          mma_ss(tmem + COL_S, smem_desc_sw128(q_addr + off_q, 16, 1024), smem_desc_sw128(k_addr + off_k, 16, 1024),
-                 IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off_k = sl * KV_BYTES + (kk >> 2) * KV_HALF + (kk & 3) * 32;
+          mma_ss(tmem + COL_S + 64 * sl, smem_desc_sw128(q_addr + off_q, 16, 1024),
+                 smem_desc_sw128(k_addr + off_k, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&M.s_full);
-        tc_commit(&M.k_empty);
-        if (!mbar_wait(&M.p_full, ph, abort) || !mbar_wait(&M.v_full, ph, abort)) {
+        tc_commit(&M.s_full[sl]);
+        tc_commit(&M.k_empty[sl]);
+        return true;
+      };
+      if (ok && T > 0) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < T; ++j) {
+        const int sl = j & 1;
+        if (!mbar_wait(&M.p_full[sl], (uint32_t)(j >> 1) & 1u, abort) ||
+            !mbar_wait(&M.v_full[sl], (uint32_t)(j >> 1) & 1u, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, KV_BYTES / 2, 1024);
-          mma_ts(tmem + COL_O, tmem + COL_S + 8 * kk, bdesc, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < UNIT / 16; ++kk) {
+          const uint64_t bdesc = smem_desc_sw128(v_addr + sl * KV_BYTES + kk * 16 * 128, KV_HALF, 1024);
+          mma_ts(tmem + COL_O, tmem + COL_S + 64 * sl + 8 * kk, bdesc, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&M.v_empty);
+        tc_commit(&M.v_empty[sl]);
+        tc_commit(&M.pv_done);
+        // S of step j + 2 reuses the buffer this PV read (in issue order)
+        if (j + 2 < T && !issue_s(j + 2)) {
+          ok = false;
+          break;
+        }
       }
       tc_commit(&M.o_final);
       tc_commit(&M.drain);
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const bool hvalid = half ? valid1 : true;
     const uint32_t* selw = (half && two) ? M.sel[1] : M.sel[0];
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t s_addr = lane_base + COL_S, o_addr = lane_base + COL_O;
+    const uint32_t s_base = lane_base + COL_S, o_addr = lane_base + COL_O;
     const bool store = t < p.N;
     constexpr float kLn2 = 0.6931471805599453f;
     float m = kNegInf;   // running max (scaled, base 2)
@@ -355,42 +355,45 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       snapped = true;
     };
 
+    // O is quiescent once PV of step j - 1 has completed (the only product
+    // that may still be running while the softmax of step j starts).
+    auto wait_prev_pv = [&](int j) {
+      if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(&M.pv_done, (uint32_t)(j - 1) & 1u, abort))) ok = false;
+      tc_fence_after();
+    };
     for (int j = 0; j < T; ++j) {
       const bool phaseA = j < TA;
+      const int sb = j & 1;
+      const uint32_t s_addr = s_base + 64 * sb;
       // all lanes leave together (the TMEM accesses below are warp-wide)
-      if (!__all_sync(0xffffffffu, mbar_wait(&M.s_full, (uint32_t)j & 1u, abort))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&M.s_full[sb], (uint32_t)(j >> 1) & 1u, abort))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // First phase-D step: every phase-A product has completed (S of this
-      // step was issued after them).
-      if (!phaseA && !snapped) snapshot();
-      // Which of the step's two units this row keeps: in phase A the blocks of
-      // its own selection, in phase D the others; causal only.
-      bool keep[2];
-      int u0s[2];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        int blk;
-        bool real;
-        unit_of(j, q, u0s[q], blk, real);
-        const bool causal = hvalid && blk <= ib;
-        const bool insel = (selw[blk >> 5] >> (blk & 31)) & 1u;
-        keep[q] = real && causal && (phaseA ? insel : !insel);
+      // First phase-D step: O holds every phase-A product once the last
+      // phase-A PV has completed.
+      if (!phaseA && !snapped) {
+        wait_prev_pv(j);
+        snapshot();
       }
-      // Row max over the kept keys, then P.  Both passes read a unit's 64 raw
-      // logits from TMEM with one wait (keys after t are masked only in a
-      // unit that reaches past t), so at most 64 of them are live at a time.
+      // Whether this row keeps the step's unit: in phase A the blocks of its
+      // own selection, in phase D the others; causal only.
+      int u0, blk;
+      unit_of(j, u0, blk);
+      const bool causal = hvalid && blk <= ib;
+      const bool insel = (selw[blk >> 5] >> (blk & 31)) & 1u;
+      const bool keep = causal && (phaseA ? insel : !insel);
+      // The unit's 64 raw logits stay in registers from the row max to the
+      // exponentials (keys after t are masked only in a unit that reaches
+      // past t).
+      float xq[UNIT];
       float mx = kNegInf;
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        if (!keep[q]) continue;
-        float xq[UNIT];
-        tmem_ld32(s_addr + q * UNIT, *reinterpret_cast<uint32_t(*)[32]>(&xq[0]));
-        tmem_ld32(s_addr + q * UNIT + 32, *reinterpret_cast<uint32_t(*)[32]>(&xq[32]));
+      if (keep) {
+        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&xq[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&xq[32]));
         tmem_wait_ld();
-        const int lim = t - u0s[q];  // keys u0 + c with c > lim are after t
+        const int lim = t - u0;  // keys u0 + c with c > lim are after t
         if (lim < UNIT - 1) {
 #pragma unroll
           for (int c = 0; c < UNIT; ++c)
@@ -404,14 +407,15 @@ __global__ void __launch_bounds__(NTHREADS, 2)
           a2 = fmaxf(a2, xq[c + 2]);
           a3 = fmaxf(a3, xq[c + 3]);
         }
-        mx = fmaxf(mx, fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)));
+        mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
       }
       mx *= p.c;  // scale > 0
       // Raise the running max when the step's max exceeds it by more than the
-      // threshold; O (quiescent: the previous PV completed before this step's
-      // S) and the row sums are rescaled in place.
+      // threshold; O (after the previous PV) and the row sums are rescaled in
+      // place.
       const bool need = (m != kNegInf) && (mx > m + kRescaleThreshold);
       if (__any_sync(0xffffffffu, need)) {
+        wait_prev_pv(j);
         const float f = need ? ex2(m - mx) : 1.0f;
 #pragma unroll 1
         for (int c0 = 0; c0 < HD; c0 += 32) {
@@ -431,46 +435,31 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       if (m == kNegInf) m = mx;
       const float nm = -m;
-      // P over the first 64 columns of S: unit 0 at [0, 32), unit 1 at [32, 64).
-      // Unit q's raw values sit at [64q, 64q + 64) and are read again before
-      // the store of unit q's P, which overwrites only columns below 64q + 32.
+      // P (bf16 pairs) over the first 32 columns of the step's S buffer.
+      uint32_t pk[32];
       float sum = 0.f;
+      if (keep) {
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t pk[32];
-        if (keep[q]) {
-          float xq[UNIT];
-          tmem_ld32(s_addr + q * UNIT, *reinterpret_cast<uint32_t(*)[32]>(&xq[0]));
-          tmem_ld32(s_addr + q * UNIT + 32, *reinterpret_cast<uint32_t(*)[32]>(&xq[32]));
-          tmem_wait_ld();
-          const int lim = t - u0s[q];
-          if (lim < UNIT - 1) {
-#pragma unroll
-            for (int c = 0; c < UNIT; ++c)
-              if (c > lim) xq[c] = kNegInf;
-          }
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int c = 0; c < UNIT; c += 2) {
-            const float e0 = ex2(fmaf(xq[c], p.c, nm));
-            const float e1 = ex2(fmaf(xq[c + 1], p.c, nm));
-            s0 += e0;
-            s1 += e1;
-            pk[c / 2] = pack_bf16(e0, e1);
-          }
-          sum += s0 + s1;
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        for (int c = 0; c < UNIT; c += 2) {
+          const float e0 = ex2(fmaf(xq[c], p.c, nm));
+          const float e1 = ex2(fmaf(xq[c + 1], p.c, nm));
+          s0 += e0;
+          s1 += e1;
+          pk[c / 2] = pack_bf16(e0, e1);
         }
-        tmem_st32(s_addr + 32 * q, pk);
+        sum = s0 + s1;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
+      tmem_st32(s_addr, pk);
       l += sum;
       if (!phaseA) lD += sum;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&M.p_full);
+      if (lane == 0) mbar_arrive(&M.p_full[sb]);
     }
 
     // ================================================================ epilogue
