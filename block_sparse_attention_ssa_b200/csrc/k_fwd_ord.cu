@@ -16,10 +16,10 @@
 // the same softmax over the rest of the causal keys, which ends as the full
 // stream.  delta is the phase-D share of the final row sum (kept separately,
 // so small masses keep their relative precision).  Every causal K/V tile is
-// still multiplied once, as in one causal attention, and the TMEM a query tile
-// needs halves (O 128 + S 128 columns), so two CTAs share an SM: while one
-// CTA's softmax warps work on its tile, the tensor core runs the other CTA's
-// products.
+// still multiplied once, as in one causal attention, and a query tile needs
+// only 256 TMEM columns (O 128 + two 64-column S buffers), so two CTAs share
+// an SM: while one CTA's softmax warps work, the tensor core runs its own next
+// logits and the other CTA's products.
 //
 // With block 64 a 128-row query tile holds two query blocks whose selections
 // differ: phase A walks the union of the two selections and phase D the blocks
