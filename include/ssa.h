@@ -43,9 +43,11 @@
  *   per-block selection on the tcgen05 kernels; the other bf16 shapes (d =
  *   64, the small blocks 16 and 32 of the paper's models, [digest] "Model
  *   Architecture Configuration", and per-token selection) on tcgen05
- *   kernels with per-row selection masks (dual forward, dropped mass, d = 64
- *   backward) and warp-level mma.sync kernels (sparse stream alone, d = 128
- *   backward); fp32 on the CUDA-core kernels.
+ *   kernels with per-row selection masks (dual forward, dropped mass,
+ *   backward; at d = 128 the backward masks single elements) and on
+ *   warp-level mma.sync kernels for the sparse stream alone (block walks fed
+ *   by TMA at blocks of 16 and 32, per-token selection); the decode step's
+ *   attention products on mma.sync; fp32 on the CUDA-core kernels.
  * Errors.  Arguments are checked on the host before anything is enqueued;
  *   a failed check returns SSA_ERR_INVALID_ARG (bad pointer, stride,
  *   alignment or value), SSA_ERR_UNSUPPORTED (a shape outside the list above,
