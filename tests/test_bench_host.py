@@ -39,3 +39,25 @@ def test_selected_pairs_full_budget_is_every_causal_pair():
     idx = np.tile(np.arange(n, dtype=np.int32), (B, H, n, 1))
     N = n * s
     assert bench.selected_pairs(idx, s, False) == B * H * N * (N + 1) // 2
+
+
+def test_measured_traffic_only_while_sources_match(tmp_path, monkeypatch):
+    """A recorded DRAM-traffic figure is reported only while every kernel source
+    it was taken from still has the recorded hash; a changed or missing source,
+    or an unknown key, gives None."""
+    import hashlib
+    import json
+
+    src = tmp_path / "k.cu"
+    src.write_text("// kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    rec = {"fwd_dual@w": {"dram_bytes_per_launch": 1234,
+                          "source_sha256": {"k.cu": hashlib.sha256(src.read_bytes()).hexdigest()}}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("fwd_dual", "w") == 1234
+    assert bench.measured_traffic("bwd_dual", "w") is None
+    src.write_text("// kernel v2\n")
+    assert bench.measured_traffic("fwd_dual", "w") is None
+    src.unlink()
+    assert bench.measured_traffic("fwd_dual", "w") is None
